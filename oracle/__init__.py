@@ -1,0 +1,142 @@
+"""Oracle for the paged KV-cache decode path: plain, slow, obviously correct.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product package imports this; only
+the tests, the smoke check of ``__graft_entry__`` and the CPU-baseline leg of
+``bench.py`` may call it.  It shares no code with the CUDA library.
+
+Parts:
+  * ``pa_oracle.c`` (loaded here through ctypes): fp64 attention over the
+    paged cache, the new-token append and the copy-on-write block copy;
+  * ``allocator.py``: the block manager (allocate on demand, share by
+    reference count, copy on write, reclaim);
+  * ``kv_size.py``: the KV-cache size formula of "1. KV 캐시란" (hjr-study-book
+    Day 3).
+
+Every function cites the passage of the three vLLM / PagedAttention pages it
+follows; the module headers list the readings taken where the pages are silent.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+F32, F16, BF16 = 0, 1, 2
+_NP_STORAGE = {F32: np.float32, F16: np.uint16, BF16: np.uint16}
+
+_lib = None
+
+
+def lib():
+    """Load (building first if needed) the C oracle."""
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        p, i64, i32, dbl = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double
+        L.or_decode.argtypes = [p, p, i32, i64]
+        L.or_decode.restype = None
+        L.or_f16_to_f64.argtypes = [ctypes.c_uint16]
+        L.or_f16_to_f64.restype = dbl
+        L.or_bf16_to_f64.argtypes = [ctypes.c_uint16]
+        L.or_bf16_to_f64.restype = dbl
+        L.or_paged_attention.argtypes = [p, p, i64, p, p, p, i32, p, i32, p,
+                                         i32, i32, i32, i32, i32, i32, dbl, i32]
+        L.or_paged_attention.restype = i32
+        L.or_reshape_and_cache.argtypes = [p, p, p, p, p, i64, i32, i32, i32, i64, i32]
+        L.or_reshape_and_cache.restype = i32
+        L.or_copy_blocks.argtypes = [p, p, p, i64, i32, i32, i32, i64, i32]
+        L.or_copy_blocks.restype = i32
+        L.or_max_threads.argtypes = []
+        L.or_max_threads.restype = i32
+        _lib = L
+    return _lib
+
+
+def max_threads() -> int:
+    return int(lib().or_max_threads())
+
+
+def _ptr(a):
+    return ctypes.c_void_p(a.ctypes.data) if a is not None else None
+
+
+def _c(a, dtype=None):
+    a = np.ascontiguousarray(a if dtype is None else a.astype(dtype, copy=False))
+    return a
+
+
+def decode(storage: np.ndarray, dtype: int) -> np.ndarray:
+    """Exact fp64 values of stored fp32 / fp16 / bf16 bit patterns."""
+    storage = np.ascontiguousarray(storage)
+    out = np.empty(storage.size, dtype=np.float64)
+    lib().or_decode(_ptr(out), _ptr(storage), dtype, storage.size)
+    return out.reshape(storage.shape)
+
+
+def paged_attention(q, k_cache, v_cache, dtype, block_tables, context_lens, scale,
+                    rows=None, nthreads=None):
+    """Decode attention over the paged cache, fp64, for every (b, h) or for ``rows``.
+
+    q: [B, Hq, D] storage array (float32, or uint16 bit patterns for fp16/bf16);
+    k_cache, v_cache: [num_blocks, Hkv, block_size, D] storage arrays;
+    block_tables: [B, max_blocks] int32; context_lens: [B] int32;
+    rows: optional [n, 2] int64 array of (b, h).  Returns [B, Hq, D] or [n, D] float64.
+
+    Follows "자기회귀 생성과 KV 캐시" (scores q.k/sqrt(d_k), softmax over valid
+    past positions, weighted sum of V) and "PagedAttention의 설계" (gather
+    through the block table in logical order, one normaliser over all tokens)
+    of the supersilo.blog vLLM summary.
+    """
+    q, k_cache, v_cache = _c(q), _c(k_cache), _c(v_cache)
+    block_tables, context_lens = _c(block_tables, np.int32), _c(context_lens, np.int32)
+    B, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_cache.shape
+    assert D2 == D and v_cache.shape == k_cache.shape and block_tables.shape[0] == B
+    if rows is not None:
+        rows = _c(rows, np.int64).reshape(-1, 2)
+        out = np.zeros((rows.shape[0], D), dtype=np.float64)
+        n = rows.shape[0]
+    else:
+        out = np.zeros((B, Hq, D), dtype=np.float64)
+        n = B * Hq
+    nt = max_threads() if nthreads is None else int(nthreads)
+    rc = lib().or_paged_attention(_ptr(out), _ptr(rows), n, _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                  dtype, _ptr(block_tables), block_tables.shape[1],
+                                  _ptr(context_lens), B, Hq, Hkv, D, bs, NB, float(scale), nt)
+    if rc != 0:
+        raise ValueError("oracle: input out of range")
+    return out
+
+
+def reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, dtype):
+    """Store the new tokens' K and V at their slots, in place (raw bytes).
+
+    key, value: [N, Hkv, D] storage arrays; caches [num_blocks, Hkv, block_size, D]
+    (modified in place, must be C-contiguous); slot_mapping: [N] int64, < 0 skips.
+    Follows "1. KV 캐시란" (hjr-study-book Day 3) and its block-table example.
+    """
+    key, value = _c(key), _c(value)
+    slot_mapping = _c(slot_mapping, np.int64)
+    assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
+    NB, Hkv, bs, D = k_cache.shape
+    rc = lib().or_reshape_and_cache(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
+                                    _ptr(slot_mapping), slot_mapping.size, Hkv, D, bs, NB, dtype)
+    if rc != 0:
+        raise ValueError("oracle: slot out of range")
+
+
+def copy_blocks(k_cache, v_cache, pairs, dtype):
+    """Copy-on-write: block pairs[p,1] := block pairs[p,0] in both caches, in order.
+
+    Follows "블록 공유" (supersilo.blog) and the copy-on-write bullet of
+    "3. vLLM: KV cache를 블록 단위로 관리하기" (blog.aqudi.me).
+    """
+    pairs = _c(pairs, np.int64).reshape(-1, 2)
+    assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
+    NB, Hkv, bs, D = k_cache.shape
+    rc = lib().or_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(pairs), pairs.shape[0],
+                              Hkv, D, bs, NB, dtype)
+    if rc != 0:
+        raise ValueError("oracle: block id out of range")

@@ -1,0 +1,164 @@
+"""Oracle block manager: the bookkeeping behind the block tables, in plain Python.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring).  An independent model of
+the host allocator exported by the CUDA library; the tests require the two to
+agree bit for bit on block tables, context lengths, slots, copy-on-write pairs,
+reference counts and the free list.
+
+What the pages fix:
+  * "PagedAttention의 설계" (supersilo.blog vLLM summary): the cache is cut into
+    fixed-size blocks; a block table links each request's logical blocks to
+    physical blocks; the block manager allocates the blocks a request needs as
+    it grows and reclaims them.
+  * "3. vLLM: KV cache를 블록 단위로 관리하기" (blog.aqudi.me): physical blocks
+    need not be contiguous; a new block is taken only when the tokens fill the
+    current one; requests with a common prompt point at the same physical
+    blocks, copied only when one side has to modify one (copy-on-write).
+  * "블록 공유" (supersilo.blog): parallel samples / beams start from one prompt
+    and share its blocks.
+  * "4.2 PagedAttention의 접근" (hjr-study-book Day 3): worked example, 16-token
+    blocks, a 37-token request mapped to physical blocks 7, 2, 9 with 5 tokens
+    in the last one.
+
+Readings where the pages are silent (a chosen convention, stated so two
+implementations can agree exactly):
+  * free blocks form a LIFO stack; the caller may give its initial order (the
+    last entry is handed out first), else it is [num_blocks-1, ..., 1, 0] so
+    block 0 comes first;
+  * freeing a sequence drops one reference from each of its blocks in logical
+    order; a block whose count reaches zero is pushed onto the stack;
+  * an append that writes into a partially filled last block whose reference
+    count is above one first takes a fresh block dst, records the pair
+    (old, dst), drops one reference from old and puts dst in the table (the
+    copy-on-write); the copy is taken before any new blocks, which follow in
+    logical order;
+  * an append or fork that cannot get all its blocks changes nothing and fails
+    with OOM.
+"""
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional, Sequence, Tuple
+
+
+class OOM(Exception):
+    pass
+
+
+class Invalid(Exception):
+    pass
+
+
+@dataclass
+class _Seq:
+    blocks: List[int] = field(default_factory=list)
+    num_tokens: int = 0
+
+
+class BlockManager:
+    def __init__(self, num_blocks: int, block_size: int,
+                 initial_free_order: Optional[Sequence[int]] = None):
+        if num_blocks <= 0 or block_size <= 0:
+            raise Invalid("num_blocks and block_size must be positive")
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+        if initial_free_order is None:
+            self.free = list(range(num_blocks - 1, -1, -1))
+        else:
+            order = [int(x) for x in initial_free_order]
+            if sorted(order) != list(range(num_blocks)):
+                raise Invalid("initial_free_order must be a permutation of 0..num_blocks-1")
+            self.free = order
+        self.refcount = [0] * num_blocks
+        self.seqs: Dict[int, _Seq] = {}
+
+    # -- queries --
+    def num_free(self) -> int:
+        return len(self.free)
+
+    def free_stack(self) -> List[int]:
+        """The free stack bottom to top (the last entry is handed out next)."""
+        return list(self.free)
+
+    def blocks_of(self, seq_id: int) -> List[int]:
+        return list(self.seqs[seq_id].blocks)
+
+    def num_tokens(self, seq_id: int) -> int:
+        return self.seqs[seq_id].num_tokens
+
+    # -- operations --
+    def add(self, seq_id: int) -> None:
+        if seq_id in self.seqs:
+            raise Invalid("sequence exists")
+        self.seqs[seq_id] = _Seq()
+
+    def fork(self, parent: int, child: int) -> None:
+        """The child shares every block of the parent ("블록 공유")."""
+        if parent not in self.seqs or child in self.seqs:
+            raise Invalid("missing parent or existing child")
+        p = self.seqs[parent]
+        for blk in p.blocks:
+            self.refcount[blk] += 1
+        self.seqs[child] = _Seq(list(p.blocks), p.num_tokens)
+
+    def append(self, seq_id: int, n_tokens: int) -> Tuple[List[int], List[Tuple[int, int]]]:
+        """Reserve slots for n_tokens new tokens; returns (slots, cow_pairs).
+
+        slot = physical_block * block_size + offset_in_block, as in the
+        37-token example of "4.2 PagedAttention의 접근".
+        """
+        if seq_id not in self.seqs:
+            raise Invalid("unknown sequence")
+        if n_tokens < 0:
+            raise Invalid("negative token count")
+        s = self.seqs[seq_id]
+        bs = self.block_size
+        T = s.num_tokens
+        if n_tokens == 0:
+            return [], []
+        # Copy-on-write is needed when the first new token lands inside an
+        # existing, shared last block.
+        cow = (T % bs != 0) and self.refcount[s.blocks[-1]] > 1
+        blocks_after = -(-(T + n_tokens) // bs)
+        new_blocks = blocks_after - len(s.blocks)
+        need = new_blocks + (1 if cow else 0)
+        if need > len(self.free):
+            raise OOM("not enough free blocks")
+        pairs: List[Tuple[int, int]] = []
+        if cow:
+            old = s.blocks[-1]
+            dst = self.free.pop()
+            self.refcount[dst] = 1
+            self.refcount[old] -= 1
+            s.blocks[-1] = dst
+            pairs.append((old, dst))
+        for _ in range(new_blocks):
+            blk = self.free.pop()
+            self.refcount[blk] = 1
+            s.blocks.append(blk)
+        slots = [s.blocks[t // bs] * bs + t % bs for t in range(T, T + n_tokens)]
+        s.num_tokens = T + n_tokens
+        return slots, pairs
+
+    def release(self, seq_id: int) -> None:
+        """Drop the sequence; blocks nobody references go back to the stack."""
+        if seq_id not in self.seqs:
+            raise Invalid("unknown sequence")
+        for blk in self.seqs.pop(seq_id).blocks:
+            self.refcount[blk] -= 1
+            if self.refcount[blk] == 0:
+                self.free.append(blk)
+
+    def build_tables(self, seq_ids: Sequence[int], max_blocks: int):
+        """Block tables [B][max_blocks] (padding -1) and context lengths [B]."""
+        import numpy as np
+        B = len(seq_ids)
+        tables = np.full((B, max_blocks), -1, dtype=np.int32)
+        lens = np.zeros(B, dtype=np.int32)
+        for i, sid in enumerate(seq_ids):
+            if sid not in self.seqs:
+                raise Invalid("unknown sequence")
+            s = self.seqs[sid]
+            if len(s.blocks) > max_blocks:
+                raise Invalid("table row too short")
+            tables[i, :len(s.blocks)] = s.blocks
+            lens[i] = s.num_tokens
+        return tables, lens

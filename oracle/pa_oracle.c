@@ -1,0 +1,275 @@
+/*
+ * pa_oracle.c -- plain, slow, fp64 CPU oracle for the paged KV-cache decode path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the checker, not the product: only the
+ * test suite, the smoke check and the CPU-baseline leg of the benchmark may load
+ * it.  It shares no code, header, table or helper with the CUDA library under
+ * paged_kv_cache_443_b200/; neither side includes or links the other.
+ *
+ * What it follows (sources are the three pages on vLLM / PagedAttention):
+ *   - "자기회귀 생성과 KV 캐시" (supersilo.blog vLLM summary): the query of the
+ *     current position attends to the keys of all valid past positions with
+ *     scores q.k_j / sqrt(d_k), softmax-normalised over those positions, and the
+ *     result is the score-weighted sum of the values.
+ *   - "PagedAttention의 설계" (same page): K/V live in fixed-size blocks; a block
+ *     table maps a sequence's logical blocks to physical blocks; the kernel reads
+ *     K/V through that table in logical order and normalises the softmax over
+ *     all valid tokens jointly (not per-block softmaxes added up).  The last
+ *     block may hold unused slots, which carry no token.
+ *   - "블록 공유" (same page) and "3. vLLM: KV cache를 블록 단위로 관리하기"
+ *     (blog.aqudi.me): sequences may point at the same physical blocks; a block is
+ *     copied only when one side must modify it (copy-on-write).
+ *   - "1. KV 캐시란" (hjr-study-book Day 3): every decode step appends the new
+ *     token's K and V to the cache.
+ *
+ * Nothing here is blocked, fused or reordered: attention rebuilds each
+ * sequence's K and V contiguously from the block table, then evaluates the
+ * softmax definition in two plain passes, in double precision.  Inputs are read
+ * from their stored bit patterns (fp32 / fp16 / bf16) by the decoders below,
+ * which do exponent/mantissa arithmetic, so the oracle sees exactly the values
+ * the GPU sees.  OpenMP only spreads independent (sequence, head) rows over
+ * threads; it does not change any row's arithmetic.
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *   - grouped-query heads: query head h reads kv head floor(h / G), G = Hq / Hkv
+ *     (contiguous groups);
+ *   - cache layout [num_blocks][Hkv][block_size][D]; token j of a sequence sits in
+ *     physical block block_tables[b][j / block_size] at offset j % block_size;
+ *   - a sequence with context length 0 produces an all-zero output row;
+ *   - copy-on-write pairs are applied in the given order.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { OR_F32 = 0, OR_F16 = 1, OR_BF16 = 2 };
+
+/* ---- element decoders (IEEE 754 binary16 and bfloat16 by field arithmetic) ---- */
+
+/* binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
+double or_f16_to_f64(uint16_t bits) {
+  int sign = (bits >> 15) & 1;
+  int e = (bits >> 10) & 0x1f;
+  int f = bits & 0x3ff;
+  double v;
+  if (e == 0) {
+    v = ldexp((double)f, -24); /* subnormal: f * 2^(1-15-10) */
+  } else if (e == 31) {
+    v = f ? NAN : INFINITY;
+  } else {
+    v = ldexp((double)(f + 1024), e - 25); /* (1 + f/2^10) * 2^(e-15) */
+  }
+  return sign ? -v : v;
+}
+
+/* bfloat16: 1 sign bit, 8 exponent bits (bias 127), 7 fraction bits. */
+double or_bf16_to_f64(uint16_t bits) {
+  int sign = (bits >> 15) & 1;
+  int e = (bits >> 7) & 0xff;
+  int f = bits & 0x7f;
+  double v;
+  if (e == 0) {
+    v = ldexp((double)f, -133); /* subnormal: f * 2^(1-127-7) */
+  } else if (e == 255) {
+    v = f ? NAN : INFINITY;
+  } else {
+    v = ldexp((double)(f + 128), e - 134); /* (1 + f/2^7) * 2^(e-127) */
+  }
+  return sign ? -v : v;
+}
+
+int or_elem_size(int dtype) {
+  switch (dtype) {
+    case OR_F32: return 4;
+    case OR_F16: return 2;
+    case OR_BF16: return 2;
+    default: return 0;
+  }
+}
+
+/* Value of element idx of an array of the given storage type. */
+static double load_elem(const void* base, int dtype, size_t idx) {
+  if (dtype == OR_F32) {
+    float x;
+    memcpy(&x, (const char*)base + 4 * idx, 4);
+    return (double)x;
+  }
+  uint16_t bits;
+  memcpy(&bits, (const char*)base + 2 * idx, 2);
+  return dtype == OR_F16 ? or_f16_to_f64(bits) : or_bf16_to_f64(bits);
+}
+
+/* Decode n elements (test helper: lets the tests pin the decoders directly). */
+void or_decode(double* out, const void* src, int dtype, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = load_elem(src, dtype, (size_t)i);
+}
+
+/* ---- attention over the paged cache ----
+ * Follows the score and softmax definition of "자기회귀 생성과 KV 캐시" and the
+ * block-table gather with one joint normaliser of "PagedAttention의 설계"
+ * (supersilo.blog vLLM summary). */
+
+/*
+ * out[r][d] for each requested row r = (b, h) in rows[2r], rows[2r+1]; rows may
+ * be NULL, meaning every (b, h) in order b-major (r = b * Hq + h).
+ *
+ * q:        [B][Hq][D]                     (dtype)
+ * k_cache:  [num_blocks][Hkv][block_size][D] (dtype), v_cache the same
+ * block_tables: [B][max_blocks] int32, context_lens: [B] int32
+ *
+ * Returns 0, or -1 if an input is out of range (a table entry outside
+ * [0, num_blocks), a context length < 0 or beyond max_blocks * block_size, a
+ * head count that does not divide, a row outside [0,B) x [0,Hq)).
+ */
+int or_paged_attention(double* out, const int64_t* rows, int64_t nrows, const void* q,
+                       const void* k_cache, const void* v_cache, int dtype,
+                       const int32_t* block_tables, int max_blocks, const int32_t* context_lens,
+                       int B, int Hq, int Hkv, int D, int block_size, int num_blocks,
+                       double scale, int nthreads) {
+  if (Hkv <= 0 || Hq % Hkv != 0 || or_elem_size(dtype) == 0 || block_size <= 0 || D <= 0)
+    return -1;
+  const int G = Hq / Hkv;
+  if (rows == NULL) nrows = (int64_t)B * Hq;
+  int bad = 0;
+  if (nthreads < 1) nthreads = 1;
+
+#pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t r = 0; r < nrows; ++r) {
+    const int64_t b = rows ? rows[2 * r] : r / Hq;
+    const int64_t h = rows ? rows[2 * r + 1] : r % Hq;
+    double* o = out + r * D;
+    if (b < 0 || b >= B || h < 0 || h >= Hq) {
+      bad = 1;
+      continue;
+    }
+    const int64_t g = h / G; /* kv head of this query head */
+    const int64_t L = context_lens[b];
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    if (L < 0 || L > (int64_t)max_blocks * block_size) {
+      bad = 1;
+      continue;
+    }
+    if (L == 0) continue;
+
+    /* 1. Rebuild this sequence's K and V contiguously, in logical order. */
+    double* K = (double*)malloc(sizeof(double) * (size_t)L * D);
+    double* V = (double*)malloc(sizeof(double) * (size_t)L * D);
+    double* s = (double*)malloc(sizeof(double) * (size_t)L);
+    int row_bad = 0;
+    for (int64_t j = 0; j < L && !row_bad; ++j) {
+      const int64_t phys = block_tables[b * max_blocks + j / block_size];
+      const int64_t off = j % block_size;
+      if (phys < 0 || phys >= num_blocks) {
+        row_bad = 1;
+        break;
+      }
+      const size_t base = (size_t)(((phys * Hkv + g) * block_size + off) * D);
+      for (int d = 0; d < D; ++d) {
+        K[j * D + d] = load_elem(k_cache, dtype, base + d);
+        V[j * D + d] = load_elem(v_cache, dtype, base + d);
+      }
+    }
+    if (!row_bad) {
+      /* 2. Scores s_j = scale * q . K_j over the valid positions j < L. */
+      const size_t qbase = (size_t)((b * Hq + h) * D);
+      for (int64_t j = 0; j < L; ++j) {
+        double acc = 0.0;
+        for (int d = 0; d < D; ++d) acc += load_elem(q, dtype, qbase + d) * K[j * D + d];
+        s[j] = scale * acc;
+      }
+      /* 3. Softmax over all L positions at once (one normaliser for the whole
+       *    sequence), then the weighted sum of V. */
+      double mx = s[0];
+      for (int64_t j = 1; j < L; ++j)
+        if (s[j] > mx) mx = s[j];
+      double Z = 0.0;
+      for (int64_t j = 0; j < L; ++j) {
+        s[j] = exp(s[j] - mx);
+        Z += s[j];
+      }
+      for (int64_t j = 0; j < L; ++j) {
+        const double w = s[j] / Z;
+        for (int d = 0; d < D; ++d) o[d] += w * V[j * D + d];
+      }
+    } else {
+      bad = 1;
+    }
+    free(K);
+    free(V);
+    free(s);
+  }
+  return bad ? -1 : 0;
+}
+
+/* ---- appending the new tokens' K and V ----
+ * Follows "1. KV 캐시란" (hjr-study-book Day 3: each step stores the new K, V
+ * pair) and the slot arithmetic of the block-table example in "4.2
+ * PagedAttention의 접근" (16-token blocks, logical block -> physical block). */
+
+/*
+ * For every t < N with slot = slot_mapping[t] >= 0:
+ *   k_cache[slot / block_size][h][slot % block_size][:] = key[t][h][:]   (all h)
+ *   v_cache[...]                                        = value[t][h][:]
+ * A negative slot means "no token to store" and is skipped.  Elements are moved
+ * as raw bytes.  Returns -1 (after writing nothing further) on a slot beyond the
+ * cache.
+ */
+int or_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
+                         const int64_t* slot_mapping, int64_t N, int Hkv, int D, int block_size,
+                         int64_t num_blocks, int dtype) {
+  const size_t es = (size_t)or_elem_size(dtype);
+  if (es == 0) return -1;
+  for (int64_t t = 0; t < N; ++t) {
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0) continue;
+    if (slot >= num_blocks * block_size) return -1;
+    const int64_t blk = slot / block_size;
+    const int64_t off = slot % block_size;
+    for (int64_t h = 0; h < Hkv; ++h) {
+      const size_t dst = (size_t)(((blk * Hkv + h) * block_size + off) * D) * es;
+      const size_t src = (size_t)((t * Hkv + h) * D) * es;
+      memcpy((char*)k_cache + dst, (const char*)key + src, (size_t)D * es);
+      memcpy((char*)v_cache + dst, (const char*)value + src, (size_t)D * es);
+    }
+  }
+  return 0;
+}
+
+/* ---- copy-on-write block copies ----
+ * Follows "블록 공유" (supersilo.blog) and the copy-on-write bullet of "3. vLLM:
+ * KV cache를 블록 단위로 관리하기" (blog.aqudi.me): a shared block is duplicated
+ * before one of its sharers modifies it. */
+
+/*
+ * For each pair p in order: physical block pairs[2p+1] of both caches becomes a
+ * copy of physical block pairs[2p] (all kv heads, all slots).  Returns -1 on an
+ * id outside [0, num_blocks).
+ */
+int or_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int64_t P, int Hkv, int D,
+                   int block_size, int64_t num_blocks, int dtype) {
+  const size_t es = (size_t)or_elem_size(dtype);
+  if (es == 0) return -1;
+  const size_t block_bytes = (size_t)Hkv * block_size * D * es;
+  for (int64_t p = 0; p < P; ++p) {
+    const int64_t src = pairs[2 * p], dst = pairs[2 * p + 1];
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) return -1;
+    for (size_t i = 0; i < block_bytes; ++i) {
+      ((char*)k_cache)[dst * block_bytes + i] = ((const char*)k_cache)[src * block_bytes + i];
+      ((char*)v_cache)[dst * block_bytes + i] = ((const char*)v_cache)[src * block_bytes + i];
+    }
+  }
+  return 0;
+}
+
+int or_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}

@@ -1,0 +1,288 @@
+"""Seeded synthetic decode workloads shaped like the vLLM / PagedAttention pages.
+
+This module is shared by the tests, the benchmark and the oracle checks, and
+holds none of the method's arithmetic: it only draws context lengths, free-list
+orders and random K/V/q contents, and writes down the block-manager operations
+(add / fork / append / release) that build each batch.  Each side (CUDA library
+or oracle) replays those operations on its own allocator, writes the K/V with
+its own append routine and computes attention on its own cache.
+
+Workloads (stand-ins for the ShareGPT / Alpaca-shaped OPT and LLaMA serving
+workloads of "구현과 실험 환경" on the supersilo.blog vLLM summary, which are
+not available here; shapes follow the public model configurations):
+
+  tiny         8 seqs, context ~ U[1,64], Hq=Hkv=4, D=64, block 16, 64 blocks in
+               a permuted pool, fp32 N(0,1), scale 1/8
+  opt13b       64 seqs, Hq=Hkv=40, D=128, block 16, fp16 N(0,1), context
+               lognormal(median 600, sigma 0.5) clipped to [16,2048], pool 20,000
+  llama13b_ps  16 prompts x 6 samples, Hq=Hkv=40, D=128, bf16, prompt ~ U[512,1024]
+               shared through forked (refcounted) blocks, 1..256 divergent tokens
+  gqa70b       256 seqs, Hq=64, Hkv=8, D=128, bf16, block 16, context ~ U[256,4096]
+  long_prefix  128 requests forked from one 4096-token prefix (same physical
+               blocks) plus a unique suffix ~ U[1,28672]; Hq=32, Hkv=8, D=128,
+               bf16, block 8/16/32, split-K partitions of 512 tokens
+
+Choices the workload descriptions leave open (stated here and in the design
+notes): the lognormal sigma 0.5; integer-uniform prompt, divergent and suffix
+lengths; pool sizes of 1.25x the blocks needed (rounded up) where no pool is
+given; q drawn like K/V, in the cache dtype; sample 0 of each prompt is the
+prompt sequence itself and samples 1..5 are forks of it.
+
+The "step" of a workload is the last group of appends: one new token per
+sequence for tiny / opt13b / gqa70b / long_prefix, and every sample's divergent
+tokens (with their copy-on-write of the shared prompt tail) for llama13b_ps.
+Context lengths include the tokens the step appends.
+"""
+from dataclasses import dataclass, field, replace
+from typing import List, Optional, Tuple
+
+import numpy as np
+
+DTYPE_CODES = {"f32": 0, "f16": 1, "bf16": 2}
+DTYPE_BYTES = {"f32": 4, "f16": 2, "bf16": 2}
+
+
+@dataclass(frozen=True)
+class Spec:
+    name: str
+    dtype: str
+    Hq: int
+    Hkv: int
+    D: int
+    block_size: int
+    kind: str                       # 'independent' | 'parallel_sampling' | 'shared_prefix'
+    num_seqs: int                   # decode batch size B
+    seed: int
+    num_blocks: Optional[int] = None  # pool size; None = 1.25x what the script needs
+    scale: Optional[float] = None     # None = 1/sqrt(D)
+    partition_size: int = 512
+    # independent
+    ctx_dist: str = "uniform"       # 'uniform' | 'lognormal'
+    ctx_lo: int = 1
+    ctx_hi: int = 64
+    ctx_median: float = 600.0
+    ctx_sigma: float = 0.5
+    # parallel sampling
+    num_prompts: int = 0
+    samples_per_prompt: int = 0
+    prompt_lo: int = 0
+    prompt_hi: int = 0
+    div_lo: int = 0
+    div_hi: int = 0
+    # shared prefix
+    prefix_len: int = 0
+    suffix_lo: int = 0
+    suffix_hi: int = 0
+
+    @property
+    def dtype_code(self) -> int:
+        return DTYPE_CODES[self.dtype]
+
+    @property
+    def esize(self) -> int:
+        return DTYPE_BYTES[self.dtype]
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def softmax_scale(self) -> float:
+        s = self.scale if self.scale is not None else 1.0 / np.sqrt(self.D)
+        return float(np.float32(s))
+
+
+TINY = Spec("tiny", "f32", 4, 4, 64, 16, "independent", 8, seed=443, num_blocks=64,
+            scale=1.0 / 8, ctx_dist="uniform", ctx_lo=1, ctx_hi=64)
+OPT13B = Spec("opt13b", "f16", 40, 40, 128, 16, "independent", 64, seed=444,
+              num_blocks=20000, ctx_dist="lognormal", ctx_median=600.0, ctx_sigma=0.5,
+              ctx_lo=16, ctx_hi=2048)
+LLAMA13B_PS = Spec("llama13b_ps", "bf16", 40, 40, 128, 16, "parallel_sampling", 96, seed=445,
+                   num_prompts=16, samples_per_prompt=6, prompt_lo=512, prompt_hi=1024,
+                   div_lo=1, div_hi=256)
+GQA70B = Spec("gqa70b", "bf16", 64, 8, 128, 16, "independent", 256, seed=446,
+              ctx_dist="uniform", ctx_lo=256, ctx_hi=4096)
+LONG_PREFIX = Spec("long_prefix", "bf16", 32, 8, 128, 16, "shared_prefix", 128, seed=447,
+                   prefix_len=4096, suffix_lo=1, suffix_hi=28672, partition_size=512)
+
+FULL = {s.name: s for s in (TINY, OPT13B, LLAMA13B_PS, GQA70B, LONG_PREFIX)}
+
+
+def long_prefix(block_size: int) -> Spec:
+    return replace(LONG_PREFIX, name=f"long_prefix_bs{block_size}", block_size=block_size)
+
+
+def small(name: str) -> Spec:
+    """Scaled-down versions the oracle finishes in seconds; each still spans
+    several tiles, several split-K partitions and a ragged last block."""
+    if name == "tiny":
+        return TINY
+    if name == "opt13b":
+        return replace(OPT13B, name="opt13b_small", num_seqs=12, Hq=6, Hkv=6, num_blocks=2000,
+                       ctx_median=600.0, seed=1444)
+    if name == "llama13b_ps":
+        return replace(LLAMA13B_PS, name="llama13b_ps_small", num_prompts=3, samples_per_prompt=6,
+                       num_seqs=18, Hq=4, Hkv=4, seed=1445)
+    if name == "gqa70b":
+        return replace(GQA70B, name="gqa70b_small", num_seqs=10, Hq=16, Hkv=2, ctx_lo=1,
+                       ctx_hi=1500, seed=1446)
+    if name == "long_prefix":
+        return replace(LONG_PREFIX, name="long_prefix_small", num_seqs=6, Hq=8, Hkv=2,
+                       prefix_len=1024, suffix_lo=1, suffix_hi=1800, seed=1447)
+    raise KeyError(name)
+
+
+@dataclass
+class Op:
+    kind: str          # 'add' | 'fork' | 'append' | 'release'
+    seq: int
+    arg: int = 0       # fork: child id; append: token count
+    kv_id: int = -1    # append: which K/V content draw
+
+
+@dataclass
+class Scenario:
+    spec: Spec
+    num_blocks: int
+    free_order: np.ndarray          # int32 permutation; the last entry is used first
+    setup_ops: List[Op]
+    step_ops: List[Op]
+    batch: List[int]                # decode order of sequence ids
+    context_lens: np.ndarray        # int32 [B], expected after the step (for sizing only)
+    max_blocks: int                 # block-table row length
+    max_context_len: int
+
+    @property
+    def B(self) -> int:
+        return len(self.batch)
+
+
+def _ctx_lengths(spec: Spec, rng) -> np.ndarray:
+    B = spec.num_seqs
+    if spec.ctx_dist == "uniform":
+        return rng.integers(spec.ctx_lo, spec.ctx_hi + 1, size=B)
+    if spec.ctx_dist == "lognormal":
+        x = rng.lognormal(mean=np.log(spec.ctx_median), sigma=spec.ctx_sigma, size=B)
+        return np.clip(np.rint(x), spec.ctx_lo, spec.ctx_hi).astype(np.int64)
+    raise ValueError(spec.ctx_dist)
+
+
+def scenario(spec: Spec) -> Scenario:
+    """The block-manager script and sizes of one workload (seeded)."""
+    rng = np.random.default_rng(spec.seed)
+    bs = spec.block_size
+    setup: List[Op] = []
+    step: List[Op] = []
+    kv = 0
+
+    def app(lst, sid, n):
+        nonlocal kv
+        if n > 0:
+            lst.append(Op("append", sid, int(n), kv))
+            kv += 1
+
+    if spec.kind == "independent":
+        lens = _ctx_lengths(spec, rng)
+        batch = list(range(spec.num_seqs))
+        for sid, L in zip(batch, lens):
+            setup.append(Op("add", sid))
+            app(setup, sid, L - 1)
+        for sid in batch:
+            app(step, sid, 1)
+        blocks_needed = int(sum(-(-int(L) // bs) for L in lens))
+    elif spec.kind == "parallel_sampling":
+        P, S = spec.num_prompts, spec.samples_per_prompt
+        prompts = rng.integers(spec.prompt_lo, spec.prompt_hi + 1, size=P)
+        divs = rng.integers(spec.div_lo, spec.div_hi + 1, size=(P, S))
+        batch, lens = [], []
+        for p in range(P):
+            root = p * S
+            setup.append(Op("add", root))
+            app(setup, root, prompts[p])
+            for s in range(1, S):
+                setup.append(Op("fork", root, root + s))
+        for p in range(P):
+            for s in range(S):
+                sid = p * S + s
+                batch.append(sid)
+                app(step, sid, divs[p, s])
+                lens.append(int(prompts[p] + divs[p, s]))
+        lens = np.array(lens)
+        blocks_needed = int(sum(-(-int(x) // bs) for x in prompts)) + \
+            int(sum(-(-int(prompts[p] + divs[p, s]) // bs) - int(prompts[p]) // bs
+                    for p in range(P) for s in range(S)))
+    elif spec.kind == "shared_prefix":
+        root = 1_000_000
+        setup.append(Op("add", root))
+        app(setup, root, spec.prefix_len)
+        suffix = rng.integers(spec.suffix_lo, spec.suffix_hi + 1, size=spec.num_seqs)
+        batch = list(range(spec.num_seqs))
+        for sid in batch:
+            setup.append(Op("fork", root, sid))
+        setup.append(Op("release", root))
+        for sid, sfx in zip(batch, suffix):
+            app(setup, sid, sfx - 1)
+        for sid in batch:
+            app(step, sid, 1)
+        lens = spec.prefix_len + suffix
+        blocks_needed = -(-spec.prefix_len // bs) + int(sum(-(-int(x) // bs) for x in suffix))
+    else:
+        raise ValueError(spec.kind)
+
+    nb = spec.num_blocks if spec.num_blocks is not None else int(np.ceil(1.25 * blocks_needed))
+    free_order = rng.permutation(nb).astype(np.int32)
+    lens = np.asarray(lens, dtype=np.int32)
+    max_ctx = int(lens.max()) if lens.size else 0
+    max_blocks = max(1, -(-max_ctx // bs))
+    return Scenario(spec, nb, free_order, setup, step, batch, lens, max_blocks, max_ctx)
+
+
+# ---------------------------------------------------------------------------
+# Random contents.  Drawn with torch so large pools can be filled on the GPU;
+# a draw is reproducible for a given (seed, id, device type).
+
+
+def _gen(device, seed: int):
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) & 0x7FFFFFFFFFFFFFFF)
+    return g
+
+
+def torch_dtype(spec: Spec):
+    import torch
+    return {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[spec.dtype]
+
+
+def kv_content(spec: Spec, kv_id: int, n: int, device="cpu"):
+    """K and V of n appended tokens, [n, Hkv, D] each, N(0,1) in the cache dtype."""
+    import torch
+    g = _gen(device, spec.seed * 1_000_003 + 7919 * kv_id + 17)
+    shape = (n, spec.Hkv, spec.D)
+    k = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    v = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    return k.to(torch_dtype(spec)), v.to(torch_dtype(spec))
+
+
+def q_content(spec: Spec, B: int, device="cpu"):
+    """Decode queries [B, Hq, D], N(0,1) in the cache dtype."""
+    import torch
+    g = _gen(device, spec.seed * 1_000_003 + 5)
+    q = torch.randn((B, spec.Hq, spec.D), generator=g, device=device, dtype=torch.float32)
+    return q.to(torch_dtype(spec))
+
+
+def poison_value(spec: Spec):
+    """Fill for every cache slot no token was written to (NaN): a kernel that
+    reads an unused tail slot into its result turns the output into NaN."""
+    return float("nan")
+
+
+def storage_view(t):
+    """A CPU tensor as the numpy array of its stored bits (float32 stays
+    float32; fp16 / bf16 become uint16 bit patterns)."""
+    import torch
+    t = t.detach().contiguous().cpu()
+    if t.dtype == torch.float32:
+        return t.numpy()
+    return t.view(torch.int16).numpy().view(np.uint16)

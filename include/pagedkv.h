@@ -1,0 +1,275 @@
+/*
+ * pagedkv.h -- C ABI of libpagedkv.so: the decode hot path of PagedAttention
+ * (attention over a KV cache kept in fixed-size physical blocks) for NVIDIA
+ * B200 (sm_100a), plus the host-side block manager that produces its block
+ * tables.
+ *
+ * Sources (three web pages on vLLM / PagedAttention):
+ *   [P1] supersilo.blog, "vLLM" summary of the PagedAttention paper:
+ *        "자기회귀 생성과 KV 캐시" (attention scores q.k_j / sqrt(d_k),
+ *        softmax over valid past positions, weighted sum of V);
+ *        "PagedAttention의 설계" (fixed-size blocks, block table from logical to
+ *        physical blocks, kernel gathers K/V through the table in logical
+ *        order with one softmax over all valid tokens, unused slots in the last
+ *        block, block manager allocating and reclaiming blocks);
+ *        "블록 공유" (parallel samples / beams share prompt blocks, copy when
+ *        modified).
+ *   [P2] blog.aqudi.me, "3. vLLM: KV cache를 블록 단위로 관리하기" (a new block
+ *        when the current one fills; copy-on-write of shared prompt blocks).
+ *   [P3] hjr-study-book Day 3, "1. KV 캐시란" (each decode step stores the new
+ *        token's K and V) and "4.2 PagedAttention의 접근" (block-table example).
+ *
+ * Conventions for every call below:
+ *   - Shapes use B = num_seqs, Hq = num_heads (query heads), Hkv = num_kv_heads,
+ *     D = head_size, bs = block_size, NB = num_blocks.  All arrays are dense,
+ *     row-major (C order), with the element type given by `dtype`.
+ *   - KV cache layout: k_cache and v_cache are each [NB][Hkv][bs][D]; token j of
+ *     a sequence b lives in physical block block_tables[b][j / bs] at slot
+ *     offset j % bs.  A slot index is physical_block * bs + offset.
+ *   - Grouped-query attention: query head h reads kv head h / (Hq / Hkv).
+ *   - Device pointers are owned by the caller; the library allocates no device
+ *     memory on any of these paths (scratch space is passed in).  Device calls
+ *     are asynchronous on `stream` (a cudaStream_t passed as void*, NULL = the
+ *     legacy default stream) on the current CUDA device, and never synchronise
+ *     the host.
+ *   - Every shape, dtype, alignment and size check runs on the host before any
+ *     launch; a failed check returns PA_ERR_INVALID (or PA_ERR_UNSUPPORTED for a
+ *     shape the kernels do not implement) with no side effect, and
+ *     pa_last_error() describes it.  A failed launch returns PA_ERR_CUDA.
+ *   - Checks that need device data (block ids in block_tables, context lengths,
+ *     slots, copy pairs) run inside the kernels: an out-of-range value is never
+ *     dereferenced; the kernel skips that access and sets a bit in a per-device
+ *     status word read by pa_device_status().  The output of that call is then
+ *     unspecified.  No kernel traps or asserts.
+ *   - Supported: dtype f32 / f16 / bf16; D in {64, 128}; bs in {8, 16, 32};
+ *     Hq / Hkv in {1, 2, 4, 8}.
+ */
+#ifndef PAGEDKV_H_
+#define PAGEDKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID = 1,     /* bad argument; nothing was done */
+  PA_ERR_OOM = 2,         /* block manager: not enough free blocks; nothing was done */
+  PA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  PA_ERR_UNSUPPORTED = 4  /* valid request outside the implemented shapes */
+} pa_status;
+
+typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
+
+/* Bits of the per-device status word (see pa_device_status). */
+#define PA_DEVERR_TABLE 0x1u    /* a block-table entry outside [0, NB) was met */
+#define PA_DEVERR_CONTEXT 0x2u  /* a context length < 0, beyond the table, or beyond max_context_len */
+#define PA_DEVERR_SLOT 0x4u     /* a slot_mapping entry >= NB * bs */
+#define PA_DEVERR_PAIR 0x8u     /* a copy pair with an id outside [0, NB) */
+#define PA_DEVERR_TIMEOUT 0x10u /* an internal pipeline wait gave up (about one second) */
+
+/* Message for the last non-OK status returned on this host thread. */
+const char* pa_last_error(void);
+
+/* Library version string. */
+const char* pa_version(void);
+
+/* Number of kernels this library has launched in this process (all devices). */
+uint64_t pa_launch_count(void);
+
+/*
+ * Reads the status word of the current device into *flags_out (PA_DEVERR_*
+ * bits; 0 = no device-side problem seen) and clears it if `clear` is non-zero.
+ * Synchronises the current device.
+ */
+pa_status pa_device_status(unsigned int* flags_out, int clear);
+
+/* ------------------------------------------------------------------------ */
+/* Decode attention ([P1] "자기회귀 생성과 KV 캐시", "PagedAttention의 설계")  */
+
+/*
+ * The split-K partition length used when partition_size = 0 is passed
+ * (tokens; a multiple of 32).
+ */
+int pa_decode_default_partition_size(void);
+
+/*
+ * Number of split-K partitions per sequence for a batch whose longest context
+ * is max_context_len: ceil(max_context_len / P), P = the partition size (0 =
+ * default).  Returns -1 for an invalid partition size.
+ */
+int pa_decode_num_partitions(int max_context_len, int partition_size);
+
+/*
+ * Bytes of scratch `workspace` pa_decode needs: 0 when every sequence fits one
+ * partition, else B * Hq * num_partitions * (D + 2) * 4 rounded up to 256.
+ */
+size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_size, int max_context_len,
+                                 int partition_size);
+
+/*
+ * Single-query attention for every sequence b < B and query head h < Hq:
+ *
+ *   out[b][h][:] = sum_j w_j V_b[j][:],  w = softmax_j(scale * q[b][h] . K_b[j]),
+ *
+ * over the valid positions j < context_lens[b] only, where K_b[j] / V_b[j] is
+ * row j % bs of kv head h / G in physical block block_tables[b][j / bs] of
+ * k_cache / v_cache.  The softmax is normalised jointly over all of a
+ * sequence's tokens (a running max and sum carried across blocks and
+ * partitions), never as per-block softmaxes added up; unused slots of the last
+ * block are never read into the result, whatever they hold.  The plain reading
+ * of [P1] gives scale = 1 / sqrt(D).
+ *
+ *   out           [B][Hq][D] dtype, written (16-byte aligned)
+ *   q             [B][Hq][D] dtype (16-byte aligned)
+ *   k_cache, v_cache  [NB][Hkv][bs][D] dtype (16-byte aligned)
+ *   block_tables  [B][max_blocks_per_seq] int32; entries past a sequence's
+ *                 last block are never read (any value, e.g. -1)
+ *   context_lens  [B] int32, each in [0, max_context_len] and
+ *                 <= max_blocks_per_seq * bs; a length of 0 gives a zero row
+ *   partition_size  0 = default, else a multiple of 32 tokens: contexts longer
+ *                 than this are split into partitions reduced by a second kernel
+ *   max_context_len  an upper bound of context_lens (sizes the launch grid and
+ *                 the workspace)
+ *   workspace     device scratch of at least pa_decode_workspace_bytes(...)
+ *                 bytes, 16-byte aligned; may be NULL when that is 0.  Its
+ *                 contents need no initialisation and are clobbered.
+ *
+ * Precision: products and sums in fp32; the result is rounded to dtype once.
+ * Exactly pa_decode_partitions followed (when the workspace size is not 0) by
+ * pa_decode_reduce on the same stream.
+ */
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int max_blocks_per_seq,
+                    const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads,
+                    int head_size, int block_size, int num_blocks, float scale, pa_dtype dtype,
+                    int partition_size, int max_context_len, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/*
+ * First phase of pa_decode (same arguments): one CTA per (sequence, kv head,
+ * partition).  Sequences that fit one partition get their final `out` rows;
+ * the others leave per-partition (max, sum, unnormalised output) partials in
+ * the workspace.
+ */
+pa_status pa_decode_partitions(void* out, const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* block_tables, int max_blocks_per_seq,
+                               const int32_t* context_lens, int num_seqs, int num_heads,
+                               int num_kv_heads, int head_size, int block_size, int num_blocks,
+                               float scale, pa_dtype dtype, int partition_size,
+                               int max_context_len, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/*
+ * Second phase of pa_decode: merges the partials of every multi-partition
+ * sequence into `out` with one global max and normaliser ([P1] "PagedAttention의
+ * 설계": one softmax over all valid tokens).  A no-op returning PA_OK when the
+ * workspace size for these arguments is 0.
+ */
+pa_status pa_decode_reduce(void* out, const int32_t* context_lens, int num_seqs, int num_heads,
+                           int head_size, pa_dtype dtype, int partition_size, int max_context_len,
+                           const void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Cache updates                                                           */
+
+/*
+ * Append ([P3] "1. KV 캐시란": each decode step stores the new token's K and
+ * V): for every t < num_tokens with s = slot_mapping[t] >= 0,
+ *   k_cache[s / bs][h][s % bs][:] = key[t][h][:]  and the same for value, all h.
+ * A negative slot is skipped (padding).  Bytes are copied exactly.
+ *
+ *   key, value    [num_tokens][Hkv][D] dtype (16-byte aligned)
+ *   k_cache, v_cache  [NB][Hkv][bs][D] dtype (16-byte aligned), updated in place
+ *   slot_mapping  [num_tokens] int64 (device)
+ * Two tokens given the same slot race (one of them wins).
+ */
+pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
+                               const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                               int head_size, int block_size, int num_blocks, pa_dtype dtype,
+                               void* stream);
+
+/*
+ * Copy-on-write ([P1] "블록 공유", [P2] copy-on-write bullet): for each pair p,
+ * physical block block_pairs[p][1] of both caches becomes a byte copy of block
+ * block_pairs[p][0] (all kv heads, all slots).
+ *
+ *   block_pairs  [num_pairs][2] int64 (device): (src, dst)
+ * The destinations must be distinct and must not appear as a source of the
+ * same call (true of the pairs the block manager emits); otherwise the result
+ * is unspecified.
+ */
+pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_pairs, int num_pairs,
+                         int num_kv_heads, int head_size, int block_size, int num_blocks,
+                         pa_dtype dtype, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Block manager (host memory; [P1] "PagedAttention의 설계", "블록 공유";     */
+/* [P2] section 3; [P3] "4.2 PagedAttention의 접근").  Not thread-safe: use one */
+/* handle per thread or lock around calls.                                 */
+
+typedef struct pa_allocator pa_allocator;
+
+/*
+ * Creates a manager of num_blocks blocks of block_size tokens.  Free blocks are
+ * a LIFO stack: initial_free_order (num_blocks distinct ids; the LAST entry is
+ * handed out first) or, if NULL, [num_blocks-1, ..., 1, 0].  *out receives the
+ * handle (free with pa_alloc_destroy).
+ */
+pa_status pa_alloc_create(int num_blocks, int block_size, const int32_t* initial_free_order,
+                          pa_allocator** out);
+void pa_alloc_destroy(pa_allocator* a);
+
+/* Free blocks left; -1 for a NULL handle. */
+int pa_alloc_num_free(const pa_allocator* a);
+
+/* Reference count of a block (number of sequences using it); -1 if out of range. */
+int pa_alloc_refcount(const pa_allocator* a, int32_t block);
+
+/* Copies the free stack, bottom to top, into out[0..capacity); *n_out = its size. */
+pa_status pa_alloc_free_stack(const pa_allocator* a, int32_t* out, int capacity, int* n_out);
+
+/* New empty sequence; PA_ERR_INVALID if the id exists. */
+pa_status pa_seq_add(pa_allocator* a, int64_t seq_id);
+
+/* The child shares all of the parent's blocks (each block's count + 1). */
+pa_status pa_seq_fork(pa_allocator* a, int64_t parent, int64_t child);
+
+/*
+ * Reserves slots for n_tokens new tokens of the sequence and writes them to
+ * slots_out[0..n_tokens).  A new block is taken only when the current last
+ * block is full.  If the first new token lands in a partly filled last block
+ * that other sequences share, that block is replaced by a fresh one and the
+ * pair (old, new) is written to cow_pair_out[0..2) with *n_cow = 1: the caller
+ * must run pa_copy_blocks on it before writing the new tokens; otherwise
+ * *n_cow = 0.  The copy block is taken first, then new blocks in logical order.
+ * PA_ERR_OOM (nothing changed) when the free stack is too short.
+ */
+pa_status pa_seq_append(pa_allocator* a, int64_t seq_id, int n_tokens, int64_t* slots_out,
+                        int64_t* cow_pair_out, int* n_cow);
+
+/* Drops the sequence; its blocks lose one reference each, in logical order, and
+ * blocks reaching zero are pushed on the free stack. */
+pa_status pa_seq_free(pa_allocator* a, int64_t seq_id);
+
+/* Tokens held by the sequence. */
+pa_status pa_seq_num_tokens(const pa_allocator* a, int64_t seq_id, int* out);
+
+/*
+ * Host block tables for a decode batch: row b of block_tables_out
+ * [num_seqs][max_blocks_per_seq] holds the physical blocks of seq_ids[b] in
+ * logical order, padded with -1; context_lens_out[b] its token count.
+ * PA_ERR_INVALID if a sequence is unknown or has more blocks than a row holds.
+ */
+pa_status pa_build_tables(const pa_allocator* a, const int64_t* seq_ids, int num_seqs,
+                          int max_blocks_per_seq, int32_t* block_tables_out,
+                          int32_t* context_lens_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H_ */

@@ -1,0 +1,113 @@
+"""PagedKVCache: one layer's paged K/V cache with its block manager.
+
+Orchestration of the C-ABI calls a decode step makes, in the order the
+vLLM / PagedAttention pages describe: the block manager reserves slots for new
+tokens, taking a fresh block only when the current one is full and copying a
+shared block before it is modified ("PagedAttention의 설계", "블록 공유" on the
+supersilo.blog summary; section 3 of the blog.aqudi.me write-up); the new
+tokens' K/V are stored at their slots ("1. KV 캐시란", hjr-study-book Day 3);
+attention then reads every sequence's K/V through its block table.  No
+arithmetic happens here: slots and copy pairs come from the C++ block manager,
+every device operation is a libpagedkv.so kernel.
+"""
+from typing import List, Optional, Sequence, Tuple
+
+import torch
+
+from . import (BlockAllocator, pa_copy_blocks, pa_decode, pa_decode_num_partitions,
+               pa_decode_workspace_bytes, pa_reshape_and_cache)
+
+
+class PagedKVCache:
+    def __init__(self, num_blocks: int, block_size: int, num_kv_heads: int, head_size: int,
+                 dtype: torch.dtype, device="cuda", initial_free_order: Optional[Sequence[int]] = None,
+                 fill: Optional[float] = None):
+        self.num_blocks, self.block_size = num_blocks, block_size
+        self.num_kv_heads, self.head_size = num_kv_heads, head_size
+        self.dtype, self.device = dtype, torch.device(device)
+        shape = (num_blocks, num_kv_heads, block_size, head_size)
+        if fill is None:
+            self.k_cache = torch.empty(shape, dtype=dtype, device=self.device)
+            self.v_cache = torch.empty(shape, dtype=dtype, device=self.device)
+        else:
+            self.k_cache = torch.full(shape, fill, dtype=dtype, device=self.device)
+            self.v_cache = torch.full(shape, fill, dtype=dtype, device=self.device)
+        self.alloc = BlockAllocator(num_blocks, block_size, initial_free_order)
+
+    # ---- block manager ----
+    def add(self, seq_id: int) -> None:
+        self.alloc.add(seq_id)
+
+    def fork(self, parent: int, child: int) -> None:
+        self.alloc.fork(parent, child)
+
+    def release(self, seq_id: int) -> None:
+        self.alloc.release(seq_id)
+
+    def reserve(self, seq_ids: Sequence[int], counts: Sequence[int]
+                ) -> Tuple[List[int], List[Tuple[int, int]]]:
+        """Host only: slots for counts[i] new tokens of seq_ids[i] (concatenated in
+        that order) and the copy-on-write pairs to run before writing them."""
+        slots: List[int] = []
+        pairs: List[Tuple[int, int]] = []
+        for sid, n in zip(seq_ids, counts):
+            s, p = self.alloc.append(sid, int(n))
+            slots += s
+            pairs += p
+        return slots, pairs
+
+    # ---- device steps ----
+    def copy_on_write(self, pairs, stream=None) -> None:
+        if isinstance(pairs, torch.Tensor):
+            t = pairs
+        else:
+            if not pairs:
+                return
+            t = torch.tensor(pairs, dtype=torch.int64, device=self.device)
+        if t.numel():
+            pa_copy_blocks(self.k_cache, self.v_cache, t, stream=stream)
+
+    def store(self, key: torch.Tensor, value: torch.Tensor, slot_mapping, stream=None) -> None:
+        if not isinstance(slot_mapping, torch.Tensor):
+            slot_mapping = torch.tensor(slot_mapping, dtype=torch.int64, device=self.device)
+        if slot_mapping.numel():
+            pa_reshape_and_cache(key, value, self.k_cache, self.v_cache, slot_mapping, stream=stream)
+
+    def append(self, seq_ids: Sequence[int], counts: Sequence[int], key: torch.Tensor,
+               value: torch.Tensor, stream=None) -> Tuple[List[int], List[Tuple[int, int]]]:
+        """Reserve, copy shared blocks, then store key/value ([sum(counts), Hkv, D])."""
+        slots, pairs = self.reserve(seq_ids, counts)
+        self.copy_on_write(pairs, stream=stream)
+        self.store(key, value, slots, stream=stream)
+        return slots, pairs
+
+    def tables(self, seq_ids: Sequence[int], max_blocks: Optional[int] = None):
+        """Device block tables [B, max_blocks] int32 and context lengths [B] int32,
+        plus the longest context (host int)."""
+        if max_blocks is None:
+            n = [self.alloc.num_tokens(s) for s in seq_ids]
+            max_blocks = max(1, -(-max(n, default=1) // self.block_size))
+        t, l = self.alloc.build_tables(list(seq_ids), max_blocks)
+        return (torch.from_numpy(t).to(self.device), torch.from_numpy(l).to(self.device),
+                int(l.max()) if l.size else 0)
+
+    def workspace(self, num_seqs: int, num_heads: int, max_context_len: int,
+                  partition_size: int = 0) -> Optional[torch.Tensor]:
+        n = pa_decode_workspace_bytes(num_seqs, num_heads, self.head_size, max_context_len,
+                                      partition_size)
+        if n == 0:
+            return None
+        return torch.empty(n // 4, dtype=torch.float32, device=self.device)
+
+    def decode(self, q: torch.Tensor, block_tables: torch.Tensor, context_lens: torch.Tensor,
+               max_context_len: int, scale: float, out: Optional[torch.Tensor] = None,
+               partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+        if out is None:
+            out = torch.empty_like(q)
+        if workspace is None:
+            workspace = self.workspace(q.shape[0], q.shape[1], max_context_len, partition_size)
+        pa_decode(out, q, self.k_cache, self.v_cache, block_tables, context_lens, scale,
+                  max_context_len, partition_size=partition_size, workspace=workspace,
+                  stream=stream)
+        return out

@@ -1,0 +1,286 @@
+// api.cpp -- the C ABI of libpagedkv.so for the device calls: argument checks
+// (all before any launch, so a rejected call has no side effect), workspace
+// sizing and dispatch to the kernel launchers.  See include/pagedkv.h for the
+// contract of every entry point.
+#include <cmath>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "pa_internal.h"
+#include "pagedkv.h"
+
+namespace {
+
+constexpr const char* kVersion = "pagedkv-b200 0.1.0 (sm_100a)";
+
+bool supported_head(int d) { return d == 64 || d == 128; }
+bool supported_block(int bs) { return bs == 8 || bs == 16 || bs == 32; }
+bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
+
+int resolve_partition(int partition_size) {
+  if (partition_size == 0) return pa::kDefaultPartition;
+  if (partition_size < 0 || partition_size % pa::kStageTokens != 0) return -1;
+  return partition_size;
+}
+
+int64_t num_partitions(int max_context_len, int P) {
+  if (max_context_len <= 0) return 1;
+  return (static_cast<int64_t>(max_context_len) + P - 1) / P;
+}
+
+size_t workspace_bytes(int64_t B, int64_t Hq, int64_t D, int64_t NP) {
+  if (NP <= 1 || B <= 0) return 0;
+  const size_t raw = static_cast<size_t>(B * Hq * NP * (D + 2) * 4);
+  return (raw + 255) / 256 * 256;
+}
+
+// Shared checks of pa_decode / pa_decode_partitions / pa_decode_reduce.
+pa_status check_decode(const char* fn, int num_seqs, int num_heads, int num_kv_heads,
+                       int head_size, pa_dtype dtype, int partition_size, int max_context_len,
+                       int* P_out, int64_t* NP_out) {
+  if (pa::elem_size(dtype) == 0) return pa::fail(PA_ERR_INVALID, "%s: unknown dtype %d", fn, dtype);
+  if (num_seqs < 0) return pa::fail(PA_ERR_INVALID, "%s: num_seqs < 0", fn);
+  if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0)
+    return pa::fail(PA_ERR_INVALID, "%s: num_heads (%d) must be a positive multiple of num_kv_heads (%d)",
+                    fn, num_heads, num_kv_heads);
+  if (num_kv_heads > 65535) return pa::fail(PA_ERR_UNSUPPORTED, "%s: num_kv_heads > 65535", fn);
+  if (!supported_group(num_heads / num_kv_heads))
+    return pa::fail(PA_ERR_UNSUPPORTED, "%s: query heads per kv head must be 1, 2, 4 or 8 (got %d)",
+                    fn, num_heads / num_kv_heads);
+  if (head_size <= 0) return pa::fail(PA_ERR_INVALID, "%s: head_size <= 0", fn);
+  if (!supported_head(head_size))
+    return pa::fail(PA_ERR_UNSUPPORTED, "%s: head_size must be 64 or 128 (got %d)", fn, head_size);
+  const int P = resolve_partition(partition_size);
+  if (P < 0)
+    return pa::fail(PA_ERR_INVALID, "%s: partition_size must be 0 or a positive multiple of %d",
+                    fn, pa::kStageTokens);
+  if (max_context_len < 0) return pa::fail(PA_ERR_INVALID, "%s: max_context_len < 0", fn);
+  const int64_t NP = num_partitions(max_context_len, P);
+  if (NP > 65535) return pa::fail(PA_ERR_UNSUPPORTED, "%s: more than 65535 partitions", fn);
+  *P_out = P;
+  *NP_out = NP;
+  return PA_OK;
+}
+
+pa_status check_decode_full(const char* fn, void* out, const void* q, const void* k_cache,
+                            const void* v_cache, const int32_t* block_tables,
+                            int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                            int num_heads, int num_kv_heads, int head_size, int block_size,
+                            int num_blocks, float scale, pa_dtype dtype, int partition_size,
+                            int max_context_len, void* workspace, size_t workspace_bytes_in,
+                            pa::DecodeArgs* a) {
+  int P = 0;
+  int64_t NP = 0;
+  pa_status st = check_decode(fn, num_seqs, num_heads, num_kv_heads, head_size, dtype,
+                              partition_size, max_context_len, &P, &NP);
+  if (st != PA_OK) return st;
+  if (block_size <= 0) return pa::fail(PA_ERR_INVALID, "%s: block_size <= 0", fn);
+  if (!supported_block(block_size))
+    return pa::fail(PA_ERR_UNSUPPORTED, "%s: block_size must be 8, 16 or 32 (got %d)", fn, block_size);
+  if (num_blocks <= 0) return pa::fail(PA_ERR_INVALID, "%s: num_blocks <= 0", fn);
+  if (max_blocks_per_seq <= 0) return pa::fail(PA_ERR_INVALID, "%s: max_blocks_per_seq <= 0", fn);
+  if (static_cast<int64_t>(max_context_len) > static_cast<int64_t>(max_blocks_per_seq) * block_size)
+    return pa::fail(PA_ERR_INVALID, "%s: max_context_len %d exceeds max_blocks_per_seq * block_size",
+                    fn, max_context_len);
+  if (!std::isfinite(scale)) return pa::fail(PA_ERR_INVALID, "%s: scale is not finite", fn);
+  if (num_seqs > 0) {
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+      return pa::fail(PA_ERR_INVALID, "%s: NULL device pointer", fn);
+    if (!pa::aligned16(out) || !pa::aligned16(q) || !pa::aligned16(k_cache) ||
+        !pa::aligned16(v_cache))
+      return pa::fail(PA_ERR_INVALID, "%s: out, q and the caches must be 16-byte aligned", fn);
+    if ((reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+        (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+      return pa::fail(PA_ERR_INVALID, "%s: block_tables / context_lens must be 4-byte aligned", fn);
+  }
+  const size_t need = workspace_bytes(num_seqs, num_heads, head_size, NP);
+  if (need > 0) {
+    if (!workspace || workspace_bytes_in < need)
+      return pa::fail(PA_ERR_INVALID, "%s: workspace of %zu bytes needed (got %zu%s)", fn, need,
+                      workspace_bytes_in, workspace ? "" : ", NULL");
+    if (!pa::aligned16(workspace))
+      return pa::fail(PA_ERR_INVALID, "%s: workspace must be 16-byte aligned", fn);
+  }
+  a->out = out;
+  a->q = q;
+  a->k_cache = k_cache;
+  a->v_cache = v_cache;
+  a->block_tables = block_tables;
+  a->context_lens = context_lens;
+  a->workspace = need > 0 ? static_cast<float*>(workspace) : nullptr;
+  a->max_blocks = max_blocks_per_seq;
+  a->num_seqs = num_seqs;
+  a->Hq = num_heads;
+  a->Hkv = num_kv_heads;
+  a->D = head_size;
+  a->block_size = block_size;
+  a->num_blocks = num_blocks;
+  a->partition_size = P;
+  a->num_partitions = static_cast<int>(NP);
+  a->scale = scale;
+  a->dtype = dtype;
+  return PA_OK;
+}
+
+pa_status launch_status(const char* fn, int err, int n_launched) {
+  if (err != cudaSuccess)
+    return pa::fail(PA_ERR_CUDA, "%s: launch failed: %s", fn,
+                    cudaGetErrorString(static_cast<cudaError_t>(err)));
+  pa::count_launch(n_launched);
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" const char* pa_version(void) { return kVersion; }
+
+extern "C" int pa_decode_default_partition_size(void) { return pa::kDefaultPartition; }
+
+extern "C" int pa_decode_num_partitions(int max_context_len, int partition_size) {
+  const int P = resolve_partition(partition_size);
+  if (P < 0) return -1;
+  const int64_t np = num_partitions(max_context_len, P);
+  return np > 0x7fffffff ? -1 : static_cast<int>(np);
+}
+
+extern "C" size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_size,
+                                            int max_context_len, int partition_size) {
+  const int P = resolve_partition(partition_size);
+  if (P < 0 || num_seqs < 0 || num_heads < 0 || head_size < 0) return 0;
+  return workspace_bytes(num_seqs, num_heads, head_size, num_partitions(max_context_len, P));
+}
+
+extern "C" pa_status pa_decode_partitions(void* out, const void* q, const void* k_cache,
+                                          const void* v_cache, const int32_t* block_tables,
+                                          int max_blocks_per_seq, const int32_t* context_lens,
+                                          int num_seqs, int num_heads, int num_kv_heads,
+                                          int head_size, int block_size, int num_blocks,
+                                          float scale, pa_dtype dtype, int partition_size,
+                                          int max_context_len, void* workspace,
+                                          size_t workspace_bytes_in, void* stream) {
+  pa::DecodeArgs a;
+  pa_status st = check_decode_full("pa_decode_partitions", out, q, k_cache, v_cache, block_tables,
+                                   max_blocks_per_seq, context_lens, num_seqs, num_heads,
+                                   num_kv_heads, head_size, block_size, num_blocks, scale, dtype,
+                                   partition_size, max_context_len, workspace, workspace_bytes_in,
+                                   &a);
+  if (st != PA_OK || num_seqs == 0) return st;
+  unsigned int* status = pa::device_status_word();
+  if (!status) return PA_ERR_CUDA;
+  return launch_status("pa_decode_partitions", pa::launch_decode_partitions(a, status, stream), 1);
+}
+
+extern "C" pa_status pa_decode_reduce(void* out, const int32_t* context_lens, int num_seqs,
+                                      int num_heads, int head_size, pa_dtype dtype,
+                                      int partition_size, int max_context_len,
+                                      const void* workspace, size_t workspace_bytes_in,
+                                      void* stream) {
+  int P = 0;
+  int64_t NP = 0;
+  // the kv-head count does not matter here; pass num_heads for both
+  pa_status st = check_decode("pa_decode_reduce", num_seqs, num_heads, num_heads, head_size, dtype,
+                              partition_size, max_context_len, &P, &NP);
+  if (st != PA_OK) return st;
+  const size_t need = workspace_bytes(num_seqs, num_heads, head_size, NP);
+  if (need == 0 || num_seqs == 0) return PA_OK;
+  if (!out || !context_lens || !workspace)
+    return pa::fail(PA_ERR_INVALID, "pa_decode_reduce: NULL device pointer");
+  if (workspace_bytes_in < need)
+    return pa::fail(PA_ERR_INVALID, "pa_decode_reduce: workspace of %zu bytes needed (got %zu)",
+                    need, workspace_bytes_in);
+  if (!pa::aligned16(out) || !pa::aligned16(workspace))
+    return pa::fail(PA_ERR_INVALID, "pa_decode_reduce: out and workspace must be 16-byte aligned");
+  pa::DecodeArgs a{};
+  a.out = out;
+  a.context_lens = context_lens;
+  a.workspace = const_cast<float*>(static_cast<const float*>(workspace));
+  a.num_seqs = num_seqs;
+  a.Hq = num_heads;
+  a.Hkv = num_heads;
+  a.D = head_size;
+  a.partition_size = P;
+  a.num_partitions = static_cast<int>(NP);
+  a.dtype = dtype;
+  return launch_status("pa_decode_reduce", pa::launch_decode_reduce(a, nullptr, stream), 1);
+}
+
+extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* block_tables, int max_blocks_per_seq,
+                               const int32_t* context_lens, int num_seqs, int num_heads,
+                               int num_kv_heads, int head_size, int block_size, int num_blocks,
+                               float scale, pa_dtype dtype, int partition_size,
+                               int max_context_len, void* workspace, size_t workspace_bytes_in,
+                               void* stream) {
+  pa::DecodeArgs a;
+  pa_status st = check_decode_full("pa_decode", out, q, k_cache, v_cache, block_tables,
+                                   max_blocks_per_seq, context_lens, num_seqs, num_heads,
+                                   num_kv_heads, head_size, block_size, num_blocks, scale, dtype,
+                                   partition_size, max_context_len, workspace, workspace_bytes_in,
+                                   &a);
+  if (st != PA_OK || num_seqs == 0) return st;
+  unsigned int* status = pa::device_status_word();
+  if (!status) return PA_ERR_CUDA;
+  st = launch_status("pa_decode", pa::launch_decode_partitions(a, status, stream), 1);
+  if (st != PA_OK || a.num_partitions <= 1) return st;
+  return launch_status("pa_decode", pa::launch_decode_reduce(a, status, stream), 1);
+}
+
+extern "C" pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache,
+                                          void* v_cache, const int64_t* slot_mapping,
+                                          int num_tokens, int num_kv_heads, int head_size,
+                                          int block_size, int num_blocks, pa_dtype dtype,
+                                          void* stream) {
+  const char* fn = "pa_reshape_and_cache";
+  const int es = pa::elem_size(dtype);
+  if (es == 0) return pa::fail(PA_ERR_INVALID, "%s: unknown dtype %d", fn, dtype);
+  if (num_tokens < 0) return pa::fail(PA_ERR_INVALID, "%s: num_tokens < 0", fn);
+  if (num_kv_heads <= 0 || head_size <= 0 || block_size <= 0 || num_blocks <= 0)
+    return pa::fail(PA_ERR_INVALID, "%s: sizes must be positive", fn);
+  if (!supported_head(head_size))
+    return pa::fail(PA_ERR_UNSUPPORTED, "%s: head_size must be 64 or 128", fn);
+  if (!supported_block(block_size))
+    return pa::fail(PA_ERR_UNSUPPORTED, "%s: block_size must be 8, 16 or 32", fn);
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !k_cache || !v_cache || !slot_mapping)
+    return pa::fail(PA_ERR_INVALID, "%s: NULL device pointer", fn);
+  if (!pa::aligned16(key) || !pa::aligned16(value) || !pa::aligned16(k_cache) ||
+      !pa::aligned16(v_cache) || (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+    return pa::fail(PA_ERR_INVALID, "%s: key/value/caches must be 16-byte aligned, slots 8", fn);
+  unsigned int* status = pa::device_status_word();
+  if (!status) return PA_ERR_CUDA;
+  return launch_status(fn,
+                       pa::launch_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping,
+                                                    num_tokens, num_kv_heads, head_size,
+                                                    block_size, num_blocks, es, status, stream),
+                       1);
+}
+
+extern "C" pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_pairs,
+                                    int num_pairs, int num_kv_heads, int head_size,
+                                    int block_size, int num_blocks, pa_dtype dtype,
+                                    void* stream) {
+  const char* fn = "pa_copy_blocks";
+  const int es = pa::elem_size(dtype);
+  if (es == 0) return pa::fail(PA_ERR_INVALID, "%s: unknown dtype %d", fn, dtype);
+  if (num_pairs < 0) return pa::fail(PA_ERR_INVALID, "%s: num_pairs < 0", fn);
+  if (num_kv_heads <= 0 || head_size <= 0 || block_size <= 0 || num_blocks <= 0)
+    return pa::fail(PA_ERR_INVALID, "%s: sizes must be positive", fn);
+  if (!supported_head(head_size))
+    return pa::fail(PA_ERR_UNSUPPORTED, "%s: head_size must be 64 or 128", fn);
+  if (!supported_block(block_size))
+    return pa::fail(PA_ERR_UNSUPPORTED, "%s: block_size must be 8, 16 or 32", fn);
+  if (num_pairs == 0) return PA_OK;
+  if (!k_cache || !v_cache || !block_pairs)
+    return pa::fail(PA_ERR_INVALID, "%s: NULL device pointer", fn);
+  if (!pa::aligned16(k_cache) || !pa::aligned16(v_cache) ||
+      (reinterpret_cast<uintptr_t>(block_pairs) & 7u))
+    return pa::fail(PA_ERR_INVALID, "%s: caches must be 16-byte aligned, pairs 8", fn);
+  unsigned int* status = pa::device_status_word();
+  if (!status) return PA_ERR_CUDA;
+  return launch_status(fn,
+                       pa::launch_copy_blocks(k_cache, v_cache, block_pairs, num_pairs,
+                                              num_kv_heads, head_size, block_size, num_blocks, es,
+                                              status, stream),
+                       1);
+}

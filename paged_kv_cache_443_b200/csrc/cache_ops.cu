@@ -1,0 +1,133 @@
+// cache_ops.cu -- KV-cache updates: the append of new tokens' K/V at their
+// slots and the copy-on-write block copy.
+//
+// Append: "1. KV 캐시란" (hjr-study-book Day 3) -- every decode step stores the
+// new token's K and V; the slot arithmetic (physical block * block_size +
+// offset) is that of the block-table example of "4.2 PagedAttention의 접근".
+// Copy-on-write: "블록 공유" (supersilo.blog) and section 3 of the blog.aqudi.me
+// write-up -- a block shared by several sequences is copied before one writes.
+//
+// Both are pure data movement in 16-byte chunks: loads are coalesced along
+// the source, stores along a D-element cache row (append) or a whole
+// contiguous [Hkv][bs][D] block (copy).  Out-of-range slots or block ids are
+// skipped and flagged in the status word, never dereferenced.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+namespace {
+
+// One thread per 16-byte chunk of key/value [N][Hkv][D].
+__global__ void __launch_bounds__(256)
+    reshape_and_cache_kernel(const uint4* __restrict__ key, const uint4* __restrict__ value,
+                             uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                             const int64_t* __restrict__ slot_mapping, int64_t total_chunks,
+                             int Hkv, int chunks_per_row, int log2_bs, int64_t num_slots,
+                             unsigned int* status) {
+  const int64_t per_token = static_cast<int64_t>(Hkv) * chunks_per_row;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total_chunks;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = i / per_token;
+    const int64_t rem = i - t * per_token;  // h * chunks_per_row + chunk
+    const int64_t slot = __ldg(slot_mapping + t);
+    if (slot < 0) continue;
+    if (slot >= num_slots) {
+      atomicOr(status, PA_DEVERR_SLOT);
+      continue;
+    }
+    const int64_t blk = slot >> log2_bs;
+    const int64_t off = slot & ((1 << log2_bs) - 1);
+    const int64_t h = rem / chunks_per_row;
+    const int64_t chunk = rem - h * chunks_per_row;
+    const int64_t dst = (((blk * Hkv + h) << log2_bs) + off) * chunks_per_row + chunk;
+    k_cache[dst] = __ldg(key + i);
+    v_cache[dst] = __ldg(value + i);
+  }
+}
+
+// grid.y strides over pairs; grid.x * blockDim.x threads stride over one block.
+__global__ void __launch_bounds__(256)
+    copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                       const int64_t* __restrict__ pairs, int num_pairs, int64_t chunks_per_block,
+                       int64_t num_blocks, unsigned int* status) {
+  for (int pr = blockIdx.y; pr < num_pairs; pr += gridDim.y) {
+    const int64_t src = __ldg(pairs + 2 * pr);
+    const int64_t dst = __ldg(pairs + 2 * pr + 1);
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+      if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(status, PA_DEVERR_PAIR);
+      continue;
+    }
+    const uint4* ks = k_cache + src * chunks_per_block;
+    const uint4* vs = v_cache + src * chunks_per_block;
+    uint4* kd = k_cache + dst * chunks_per_block;
+    uint4* vd = v_cache + dst * chunks_per_block;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < chunks_per_block;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+      kd[i] = ks[i];
+      vd[i] = vs[i];
+    }
+  }
+}
+
+int ilog2(int x) {
+  int r = 0;
+  while ((1 << r) < x) ++r;
+  return r;
+}
+
+int num_sms() {
+  static thread_local int cached_dev = -1, cached_sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev != cached_dev) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+      cached_sms = n;
+    cached_dev = dev;
+  }
+  return cached_sms;
+}
+
+}  // namespace
+
+int launch_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
+                             const int64_t* slot_mapping, int num_tokens, int Hkv, int D,
+                             int block_size, int num_blocks, int esize, unsigned int* status,
+                             void* stream) {
+  const int chunks_per_row = D * esize / 16;
+  const int64_t total = static_cast<int64_t>(num_tokens) * Hkv * chunks_per_row;
+  const int threads = 256;
+  int64_t blocks = (total + threads - 1) / threads;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  reshape_and_cache_kernel<<<static_cast<unsigned>(blocks), threads, 0,
+                             static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(key), static_cast<const uint4*>(value),
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), slot_mapping, total, Hkv,
+      chunks_per_row, ilog2(block_size), static_cast<int64_t>(num_blocks) * block_size, status);
+  return cudaGetLastError();
+}
+
+int launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_pairs, int Hkv,
+                       int D, int block_size, int num_blocks, int esize, unsigned int* status,
+                       void* stream) {
+  const int64_t chunks = static_cast<int64_t>(Hkv) * block_size * D * esize / 16;
+  const int threads = 256;
+  int64_t gx = (chunks + threads * 4 - 1) / (threads * 4);  // ~4 chunks per thread per cache
+  if (gx < 1) gx = 1;
+  if (gx > 1024) gx = 1024;
+  const int gy = num_pairs < 65535 ? num_pairs : 65535;
+  dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
+  copy_blocks_kernel<<<grid, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), pairs, num_pairs, chunks,
+      num_blocks, status);
+  return cudaGetLastError();
+}
+
+}  // namespace pa

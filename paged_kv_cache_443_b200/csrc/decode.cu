@@ -1,0 +1,566 @@
+// decode.cu -- paged decode attention for sm_100a: the split-K partition kernel
+// and the partition-reduce kernel.
+//
+// What is computed ("자기회귀 생성과 KV 캐시" and "PagedAttention의 설계" of the
+// supersilo.blog vLLM summary): for sequence b and query head h,
+//   out[b][h] = sum_j softmax_j(scale * q[b][h] . K_b[j]) V_b[j],  j < context_lens[b],
+// where K_b[j] / V_b[j] are fetched through the block table in logical order and
+// one softmax spans all of the sequence's tokens: a running max m and sum l are
+// carried across blocks inside a partition, and across partitions by the
+// reduce kernel (never per-block softmaxes summed).  Unused slots of a last
+// block are masked out and never reach the result.
+//
+// Design (B200):
+//   * one CTA per (sequence, kv head, partition of P tokens); all G = Hq/Hkv
+//     query heads of the kv head are served by the same CTA, so every K/V byte
+//     is read from HBM once;
+//   * warp 0 is the producer: it reads the block table (32 entries per
+//     coalesced load) and moves each physical (block, kv head) K and V tile --
+//     a contiguous bs*D run -- into shared memory with 1-D bulk copies on the
+//     TMA engine, into a ring of S stages of 32 tokens (about 64 KB in flight per
+//     CTA) tracked by mbarriers with transaction counts;
+//   * NCW consumer warps each own 8 tokens of a stage: q (pre-scaled by
+//     scale*log2 e) sits in registers, a lane owns one 16-byte chunk of a K/V row,
+//     dot products are finished with a butterfly reduce-scatter across the lanes
+//     of a row, softmax runs in base 2 on the warp's scores in shared memory,
+//     and P.V accumulates in fp32 registers;
+//   * at the end the consumer warps merge their (m, l, o) states; a sequence that
+//     fits one partition gets its normalised output directly, otherwise the
+//     partial (m, l, o) goes to the workspace for the reduce kernel.
+//   Every mbarrier wait is bounded (pa_device.cuh); a block id outside the pool
+//   is never dereferenced (the copy is skipped and PA_DEVERR_TABLE set).
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+namespace {
+
+constexpr unsigned FULL_MASK = 0xffffffffu;
+
+constexpr int cmax(int a, int b) { return a > b ? a : b; }
+constexpr int cmin(int a, int b) { return a < b ? a : b; }
+constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+template <typename T, int D, int G, int NCW>
+struct Cfg {
+  static constexpr int ES = sizeof(T);
+  static constexpr int EPL = 16 / ES;          // elements per 16-byte chunk
+  static constexpr int LPR = D / EPL;          // lanes per K/V row
+  static constexpr int RPW = 32 / LPR;         // rows a warp covers per iteration
+  static constexpr int TOK = kStageTokens;     // tokens per stage
+  static constexpr int TPW = TOK / NCW;        // tokens per consumer warp per stage
+  static constexpr int ITERS = TPW / RPW;
+  static constexpr int ROW_BYTES = D * ES;
+  static constexpr int TILE_BYTES = TOK * ROW_BYTES;  // K (or V) part of a stage
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  static constexpr int S = cmin(8, cmax(2, 65536 / STAGE_BYTES));
+  static constexpr int NV = G * ITERS;         // partial dots per lane per stage
+  static constexpr int NSM = G * TPW;          // scores per warp per stage
+  static constexpr int NPASS = (NSM + 31) / 32;
+  static constexpr int SC_BYTES = round_up(NCW * NSM * 4, 128);
+  static constexpr int HDR_BYTES = 128 + SC_BYTES;
+  static constexpr int SMEM = HDR_BYTES + S * STAGE_BYTES;
+  static constexpr int THREADS = 32 * (NCW + 1);
+  static constexpr int CB_STRIDE = D + 2;      // combine buffer row: o[D], m, l
+  static_assert(LPR >= 1 && LPR <= 32 && (32 % LPR) == 0, "row must map onto a warp");
+  static_assert(TPW % RPW == 0 && ITERS >= 1, "warp tokens must be whole iterations");
+  static_assert(TPW <= 32 && (TPW & (TPW - 1)) == 0, "score segment must fit a warp");
+  static_assert(NCW * G * CB_STRIDE * 4 <= S * STAGE_BYTES, "combine buffer must fit the stages");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+// Butterfly reduce-scatter of N values over the lanes of a row (lane bits
+// below LPR): each halving step keeps one half of the values and adds the
+// partner's copy of it; once one value is left the remaining steps all-reduce.
+template <int N, int OFF>
+__device__ __forceinline__ void reduce_scatter(float* v, int lane) {
+  if constexpr (OFF >= 1) {
+    if constexpr (N >= 2) {
+      constexpr int H = N / 2;
+      const bool upper = (lane & OFF) != 0;
+#pragma unroll
+      for (int i = 0; i < H; ++i) {
+        const float send = upper ? v[i] : v[i + H];
+        const float keep = upper ? v[i + H] : v[i];
+        v[i] = keep + __shfl_xor_sync(FULL_MASK, send, OFF);
+      }
+      reduce_scatter<H, OFF / 2>(v, lane);
+    } else {
+      v[0] += __shfl_xor_sync(FULL_MASK, v[0], OFF);
+      reduce_scatter<1, OFF / 2>(v, lane);
+    }
+  }
+}
+
+// Index (in the original array) of v[0] after reduce_scatter<N, OFF>.
+template <int N, int OFF>
+__device__ __forceinline__ int reduce_scatter_base(int lane) {
+  if constexpr (OFF >= 1 && N >= 2) {
+    return ((lane & OFF) ? N / 2 : 0) + reduce_scatter_base<N / 2, OFF / 2>(lane);
+  } else {
+    return 0;
+  }
+}
+
+struct PartitionParams {
+  void* out;
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  float* ws_o;  // [B][Hq][NP][D]
+  float* ws_m;  // [B][Hq][NP]
+  float* ws_l;  // [B][Hq][NP]
+  unsigned int* status;
+  int64_t max_blocks;
+  int Hq, Hkv, num_blocks, block_size, partition_size, num_partitions;
+  float scale_log2;  // scale * log2(e)
+};
+
+template <typename T, int D, int G, int NCW>
+__global__ void __launch_bounds__(Cfg<T, D, G, NCW>::THREADS)
+    decode_partition_kernel(const PartitionParams p) {
+  using C = Cfg<T, D, G, NCW>;
+  using E = Elem<T>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + C::S;
+  float* scores = reinterpret_cast<float*>(smem + 128);
+  uint8_t* stages = smem + C::HDR_BYTES;
+
+  const int b = blockIdx.x;
+  const int g = blockIdx.y;
+  const int part = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- this partition's token range (validated) ----
+  int L = p.context_lens[b];
+  const int P = p.partition_size;
+  // longest context this launch can serve: the table row and the partition grid
+  int64_t cap = p.max_blocks * p.block_size;
+  const int64_t grid_cap = static_cast<int64_t>(p.num_partitions) * P;
+  cap = cap < grid_cap ? cap : grid_cap;
+  if (L < 0 || L > cap) {
+    if (threadIdx.x == 0 && part == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
+    L = L < 0 ? 0 : static_cast<int>(cap);
+  }
+  const int start = part * P;
+  if (L == 0) {
+    if (part == 0) {
+      T* o = static_cast<T*>(p.out) + (static_cast<int64_t>(b) * p.Hq + g * G) * D;
+      for (int i = threadIdx.x; i < G * D; i += C::THREADS) o[i] = E::from_float(0.f);
+    }
+    return;
+  }
+  if (start >= L) return;
+  const int end = min(L, start + P);
+  const int n_tiles = (end - start + C::TOK - 1) / C::TOK;
+  const bool single = (L <= P);
+
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int s = 0; s < C::S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], NCW);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    // ================= producer =================
+    const int bs = p.block_size;
+    const int bpt = C::TOK / bs;                      // blocks per stage
+    const int first_blk = start / bs;
+    const int last_blk = (end + bs - 1) / bs;         // exclusive
+    const uint32_t blk_bytes = static_cast<uint32_t>(bs) * C::ROW_BYTES;
+    const int64_t head_off = static_cast<int64_t>(g) * blk_bytes;
+    const int64_t blk_stride = static_cast<int64_t>(p.Hkv) * blk_bytes;
+    const int32_t* trow = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
+    const char* kbase = static_cast<const char*>(p.k_cache) + head_off;
+    const char* vbase = static_cast<const char*>(p.v_cache) + head_off;
+    int cached = -1;
+    int issued = 0;
+    bool ok = true;
+    for (int t = 0; t < n_tiles; ++t) {
+      const int s = t % C::S;
+      if (t >= C::S && !mbar_wait(&empty[s], ((t / C::S) - 1) & 1, p.status)) {
+        ok = false;
+        break;
+      }
+      const int rel = t * bpt;                        // block index within the partition
+      if ((rel & 31) == 0) {
+        const int lb = first_blk + rel + lane;
+        cached = lb < last_blk ? __ldg(trow + lb) : -1;
+      }
+      const int nb = min(bpt, last_blk - (first_blk + rel));
+      const int src_lane = (rel & 31) + (lane < nb ? lane : 0);
+      const int pb = __shfl_sync(FULL_MASK, cached, src_lane);
+      const bool mine = lane < nb;
+      const bool valid = mine && pb >= 0 && pb < p.num_blocks;
+      if (mine && !valid) atomicOr(p.status, PA_DEVERR_TABLE);
+      const unsigned vmask = __ballot_sync(FULL_MASK, valid);
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], __popc(vmask) * 2u * blk_bytes);
+      __syncwarp();
+      if (valid) {
+        uint8_t* kdst = stages + s * C::STAGE_BYTES + lane * blk_bytes;
+        uint8_t* vdst = kdst + C::TILE_BYTES;
+        const int64_t off = static_cast<int64_t>(pb) * blk_stride;
+        bulk_load(kdst, kbase + off, blk_bytes, &full[s]);
+        bulk_load(vdst, vbase + off, blk_bytes, &full[s]);
+      }
+      issued = t + 1;
+    }
+    if (!ok) {
+      // a consumer stopped: wait (bounded) for our own copies still in flight
+      for (int t = issued - C::S < 0 ? 0 : issued - C::S; t < issued; ++t)
+        mbar_wait(&full[t % C::S], (t / C::S) & 1, p.status);
+    }
+    return;
+  }
+
+  // ================= consumers =================
+  const int w = warp - 1;
+  const int r = lane / C::LPR;      // row group within the warp
+  const int c = lane % C::LPR;      // 16-byte chunk of the row this lane owns
+  float* sc = scores + w * C::NSM;  // [G][TPW]
+
+  float qf[G][C::EPL];
+  {
+    const T* qrow = static_cast<const T*>(p.q) + (static_cast<int64_t>(b) * p.Hq + g * G) * D;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(qrow + h * D + c * C::EPL));
+      E::unpack(u, qf[h]);
+#pragma unroll
+      for (int e = 0; e < C::EPL; ++e) qf[h][e] *= p.scale_log2;
+    }
+  }
+  float m[G], l[G], o[G][C::EPL];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    m[h] = -INFINITY;
+    l[h] = 0.f;
+#pragma unroll
+    for (int e = 0; e < C::EPL; ++e) o[h][e] = 0.f;
+  }
+
+  bool ok = true;
+  for (int t = 0; t < n_tiles; ++t) {
+    const int s = t % C::S;
+    if (!mbar_wait(&full[s], (t / C::S) & 1, p.status)) {
+      ok = false;
+      break;
+    }
+    const T* Ks = reinterpret_cast<const T*>(stages + s * C::STAGE_BYTES);
+    const T* Vs = reinterpret_cast<const T*>(stages + s * C::STAGE_BYTES + C::TILE_BYTES);
+    const int n_valid = min(C::TOK, end - (start + t * C::TOK));
+
+    // ---- scores: partial dots over this lane's chunk, then across the row ----
+    float part_dot[C::NV];
+#pragma unroll
+    for (int it = 0; it < C::ITERS; ++it) {
+      const int row = w * C::TPW + it * C::RPW + r;
+      const uint4 u = *reinterpret_cast<const uint4*>(Ks + row * D + c * C::EPL);
+      float kf[C::EPL];
+      E::unpack(u, kf);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float acc = 0.f;
+#pragma unroll
+        for (int e = 0; e < C::EPL; ++e) acc = fmaf(qf[h][e], kf[e], acc);
+        part_dot[h * C::ITERS + it] = acc;
+      }
+    }
+    reduce_scatter<C::NV, C::LPR / 2>(part_dot, lane);
+    {
+      constexpr int NF = C::NV >= C::LPR ? C::NV / C::LPR : 1;
+      constexpr int REP = C::NV >= C::LPR ? 1 : C::LPR / C::NV;
+      const int base = reduce_scatter_base<C::NV, C::LPR / 2>(lane);
+      if ((c % REP) == 0) {
+#pragma unroll
+        for (int i = 0; i < NF; ++i) {
+          const int idx = base + i;
+          const int h = idx / C::ITERS;
+          const int it = idx % C::ITERS;
+          const int row_local = it * C::RPW + r;
+          const bool valid = (w * C::TPW + row_local) < n_valid;
+          sc[h * C::TPW + row_local] = valid ? part_dot[i] : -INFINITY;
+        }
+      }
+    }
+    __syncwarp();
+
+    // ---- online softmax (base 2) over the warp's tokens, per head ----
+    float sv[C::NPASS], seg[C::NPASS];
+#pragma unroll
+    for (int ps = 0; ps < C::NPASS; ++ps) {
+      const int idx = ps * 32 + lane;
+      sv[ps] = idx < C::NSM ? sc[idx] : -INFINITY;
+      float x = sv[ps];
+#pragma unroll
+      for (int off = C::TPW / 2; off >= 1; off >>= 1) x = fmaxf(x, __shfl_xor_sync(FULL_MASK, x, off));
+      seg[ps] = x;
+    }
+    float mnew[G], alpha[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float tmax = __shfl_sync(FULL_MASK, seg[(h * C::TPW) / 32], (h * C::TPW) % 32);
+      mnew[h] = fmaxf(m[h], tmax);
+      alpha[h] = (mnew[h] == -INFINITY) ? 1.f : exp2f(m[h] - mnew[h]);
+    }
+#pragma unroll
+    for (int ps = 0; ps < C::NPASS; ++ps) {
+      const int idx = ps * 32 + lane;
+      const int hh = idx / C::TPW;
+      float mh = -INFINITY;
+#pragma unroll
+      for (int h = 0; h < G; ++h) mh = (h == hh) ? mnew[h] : mh;
+      const float pr = (sv[ps] == -INFINITY) ? 0.f : exp2f(sv[ps] - mh);
+      if (idx < C::NSM) sc[idx] = pr;
+      float x = pr;
+#pragma unroll
+      for (int off = C::TPW / 2; off >= 1; off >>= 1) x += __shfl_xor_sync(FULL_MASK, x, off);
+      seg[ps] = x;
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float tsum = __shfl_sync(FULL_MASK, seg[(h * C::TPW) / 32], (h * C::TPW) % 32);
+      l[h] = l[h] * alpha[h] + tsum;
+      m[h] = mnew[h];
+#pragma unroll
+      for (int e = 0; e < C::EPL; ++e) o[h][e] *= alpha[h];
+    }
+    __syncwarp();
+
+    // ---- P.V over the warp's valid rows ----
+#pragma unroll
+    for (int it = 0; it < C::ITERS; ++it) {
+      const int row_local = it * C::RPW + r;
+      const int row = w * C::TPW + row_local;
+      if (row < n_valid) {
+        const uint4 u = *reinterpret_cast<const uint4*>(Vs + row * D + c * C::EPL);
+        float vf[C::EPL];
+        E::unpack(u, vf);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float pr = sc[h * C::TPW + row_local];
+#pragma unroll
+          for (int e = 0; e < C::EPL; ++e) o[h][e] = fmaf(pr, vf[e], o[h][e]);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+
+  // ---- merge row groups of the warp, then the consumer warps ----
+#pragma unroll
+  for (int off = C::LPR; off < 32; off <<= 1) {
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int e = 0; e < C::EPL; ++e) o[h][e] += __shfl_xor_sync(FULL_MASK, o[h][e], off);
+  }
+  named_sync(1, NCW * 32);  // every consumer is done with the stages
+  float* cb = reinterpret_cast<float*>(stages);
+  if (r == 0) {
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int e = 0; e < C::EPL; ++e) cb[(w * G + h) * C::CB_STRIDE + c * C::EPL + e] = o[h][e];
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      cb[(w * G + h) * C::CB_STRIDE + D] = m[h];
+      cb[(w * G + h) * C::CB_STRIDE + D + 1] = l[h];
+    }
+  }
+  named_sync(1, NCW * 32);
+  if (!ok) return;  // status already records the failure
+
+  const int tid = threadIdx.x - 32;
+  for (int idx = tid; idx < G * D; idx += NCW * 32) {
+    const int h = idx / D;
+    const int d = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int ww = 0; ww < NCW; ++ww) M = fmaxf(M, cb[(ww * G + h) * C::CB_STRIDE + D]);
+    float Ls = 0.f, O = 0.f;
+#pragma unroll
+    for (int ww = 0; ww < NCW; ++ww) {
+      const float mw = cb[(ww * G + h) * C::CB_STRIDE + D];
+      const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+      Ls = fmaf(cb[(ww * G + h) * C::CB_STRIDE + D + 1], f, Ls);
+      O = fmaf(cb[(ww * G + h) * C::CB_STRIDE + d], f, O);
+    }
+    const int64_t hq = static_cast<int64_t>(b) * p.Hq + g * G + h;
+    if (single) {
+      static_cast<T*>(p.out)[hq * D + d] = E::from_float(O / Ls);
+    } else {
+      const int64_t slot = hq * p.num_partitions + part;
+      p.ws_o[slot * D + d] = O;
+      if (d == 0) {
+        p.ws_m[slot] = M;
+        p.ws_l[slot] = Ls;
+      }
+    }
+  }
+}
+
+struct ReduceParams {
+  void* out;
+  const int32_t* context_lens;
+  const float* ws_o;
+  const float* ws_m;
+  const float* ws_l;
+  int num_seqs, Hq, partition_size, num_partitions;
+};
+
+// One warp per (sequence, query head) with more than one partition:
+// out = sum_p o_p 2^(m_p - M) / sum_p l_p 2^(m_p - M),  M = max_p m_p.
+template <typename T, int D>
+__global__ void __launch_bounds__(128) decode_reduce_kernel(const ReduceParams p) {
+  using E = Elem<T>;
+  constexpr int DPL = D / 32;  // dims per lane
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= static_cast<int64_t>(p.num_seqs) * p.Hq) return;
+  const int b = static_cast<int>(row / p.Hq);
+  int L = p.context_lens[b];
+  L = L < 0 ? 0 : L;
+  const int64_t grid_cap = static_cast<int64_t>(p.num_partitions) * p.partition_size;
+  if (L > grid_cap) L = static_cast<int>(grid_cap);  // flagged by the partition kernel
+  const int np = (L + p.partition_size - 1) / p.partition_size;
+  if (np <= 1) return;  // written directly by the partition kernel
+  const int64_t base = row * p.num_partitions;
+  float M = -INFINITY;
+  for (int i = lane; i < np; i += 32) M = fmaxf(M, p.ws_m[base + i]);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, off));
+  float Ls = 0.f;
+  for (int i = lane; i < np; i += 32) Ls += p.ws_l[base + i] * exp2f(p.ws_m[base + i] - M);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) Ls += __shfl_xor_sync(FULL_MASK, Ls, off);
+  float acc[DPL];
+#pragma unroll
+  for (int k = 0; k < DPL; ++k) acc[k] = 0.f;
+  for (int i = 0; i < np; ++i) {
+    const float f = exp2f(p.ws_m[base + i] - M);
+    const float* src = p.ws_o + (base + i) * D + lane * DPL;
+#pragma unroll
+    for (int k = 0; k < DPL; ++k) acc[k] = fmaf(f, src[k], acc[k]);
+  }
+  T* dst = static_cast<T*>(p.out) + row * D + lane * DPL;
+  const float inv = 1.f / Ls;
+#pragma unroll
+  for (int k = 0; k < DPL; ++k) dst[k] = E::from_float(acc[k] * inv);
+}
+
+constexpr int kConsumerWarps = 4;
+
+template <typename T, int D, int G>
+cudaError_t launch_partition_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
+  using C = Cfg<T, D, G, kConsumerWarps>;
+  auto kern = decode_partition_kernel<T, D, G, kConsumerWarps>;
+  // opt in to > 48 KB of dynamic shared memory (idempotent, cheap)
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  PartitionParams p;
+  p.out = a.out;
+  p.q = a.q;
+  p.k_cache = a.k_cache;
+  p.v_cache = a.v_cache;
+  p.block_tables = a.block_tables;
+  p.context_lens = a.context_lens;
+  const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.Hq * a.num_partitions;
+  p.ws_o = a.workspace;
+  p.ws_m = a.workspace ? a.workspace + rows * D : nullptr;
+  p.ws_l = a.workspace ? a.workspace + rows * (D + 1) : nullptr;
+  p.status = status;
+  p.max_blocks = a.max_blocks;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.num_blocks = a.num_blocks;
+  p.block_size = a.block_size;
+  p.partition_size = a.partition_size;
+  p.num_partitions = a.num_partitions;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  dim3 grid(a.num_seqs, a.Hkv, a.num_partitions);
+  kern<<<grid, C::THREADS, C::SMEM, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_partition_g(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
+  switch (a.Hq / a.Hkv) {
+    case 1: return launch_partition_t<T, D, 1>(a, status, stream);
+    case 2: return launch_partition_t<T, D, 2>(a, status, stream);
+    case 4: return launch_partition_t<T, D, 4>(a, status, stream);
+    case 8: return launch_partition_t<T, D, 8>(a, status, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <typename T>
+cudaError_t launch_partition_d(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
+  switch (a.D) {
+    case 64: return launch_partition_g<T, 64>(a, status, stream);
+    case 128: return launch_partition_g<T, 128>(a, status, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <typename T>
+cudaError_t launch_reduce_t(const DecodeArgs& a, cudaStream_t stream) {
+  ReduceParams p;
+  p.out = a.out;
+  p.context_lens = a.context_lens;
+  const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.Hq * a.num_partitions;
+  p.ws_o = a.workspace;
+  p.ws_m = a.workspace + rows * a.D;
+  p.ws_l = a.workspace + rows * (a.D + 1);
+  p.num_seqs = a.num_seqs;
+  p.Hq = a.Hq;
+  p.partition_size = a.partition_size;
+  p.num_partitions = a.num_partitions;
+  const int64_t warps = static_cast<int64_t>(a.num_seqs) * a.Hq;
+  const unsigned grid = static_cast<unsigned>((warps + 3) / 4);
+  if (a.D == 64)
+    decode_reduce_kernel<T, 64><<<grid, 128, 0, stream>>>(p);
+  else
+    decode_reduce_kernel<T, 128><<<grid, 128, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int launch_decode_partitions(const DecodeArgs& a, unsigned int* status, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (a.dtype) {
+    case PA_F32: return launch_partition_d<float>(a, status, st);
+    case PA_F16: return launch_partition_d<__half>(a, status, st);
+    case PA_BF16: return launch_partition_d<__nv_bfloat16>(a, status, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+int launch_decode_reduce(const DecodeArgs& a, unsigned int* /*status*/, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (a.dtype) {
+    case PA_F32: return launch_reduce_t<float>(a, st);
+    case PA_F16: return launch_reduce_t<__half>(a, st);
+    case PA_BF16: return launch_reduce_t<__nv_bfloat16>(a, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace pa

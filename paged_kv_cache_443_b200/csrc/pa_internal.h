@@ -1,0 +1,68 @@
+// pa_internal.h -- declarations shared by the library's translation units
+// (host side only; nothing here is part of the public ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "pagedkv.h"
+
+namespace pa {
+
+// Records a message for pa_last_error() and returns `st`.
+pa_status fail(pa_status st, const char* fmt, ...)
+#if defined(__GNUC__)
+    __attribute__((format(printf, 2, 3)))
+#endif
+    ;
+
+// Counts successful kernel launches (pa_launch_count).
+void count_launch(uint64_t n = 1);
+
+// Device address of the current device's status word (cached per device).
+// Returns nullptr (and records a message) if CUDA fails.
+unsigned int* device_status_word();
+
+// Element size of a dtype, 0 if invalid.
+inline int elem_size(pa_dtype dt) {
+  switch (dt) {
+    case PA_F32: return 4;
+    case PA_F16: return 2;
+    case PA_BF16: return 2;
+    default: return 0;
+  }
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kDefaultPartition = 512;  // tokens per split-K partition
+constexpr int kStageTokens = 32;        // tokens per pipeline stage of the decode kernel
+
+// ---- decode launch description (validated on the host) ----
+struct DecodeArgs {
+  void* out;
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  float* workspace;  // may be null when num_partitions == 1
+  int64_t max_blocks;
+  int num_seqs, Hq, Hkv, D, block_size, num_blocks;
+  int partition_size, num_partitions;
+  float scale;
+  pa_dtype dtype;
+};
+
+// Kernel launchers (kernels.cu).  They return cudaError_t as int.
+int launch_decode_partitions(const DecodeArgs& a, unsigned int* status, void* stream);
+int launch_decode_reduce(const DecodeArgs& a, unsigned int* status, void* stream);
+int launch_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
+                             const int64_t* slot_mapping, int num_tokens, int Hkv, int D,
+                             int block_size, int num_blocks, int esize, unsigned int* status,
+                             void* stream);
+int launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_pairs, int Hkv,
+                       int D, int block_size, int num_blocks, int esize, unsigned int* status,
+                       void* stream);
+
+}  // namespace pa

@@ -1,0 +1,156 @@
+"""Lockstep builder of a workload on the CUDA library and on the oracle.
+
+Both sides replay the same block-manager script (from the workloads module)
+on their own allocator, copy shared blocks and store the same seeded K/V with
+their own routines, and build their own block tables.  The oracle receives
+only generator output (host copies of the seeded draws) -- never a value
+produced by the CUDA path.  Comparisons: tables / slots / pairs / cache bytes
+bit-exact, attention within the stated tolerance.
+"""
+from dataclasses import dataclass
+from typing import List, Optional, Tuple
+
+import numpy as np
+import torch
+
+import oracle
+import workloads as W
+from oracle.allocator import BlockManager
+from paged_kv_cache_443_b200.cache import PagedKVCache
+
+# tolerances: fp32 accumulation; max abs error on outputs (fp16 / bf16 / fp32)
+TOL = {"f32": 1e-5, "f16": 2e-2, "bf16": 2e-2}
+
+
+def poison_bits(spec: W.Spec):
+    """Bit pattern torch stores for NaN in the cache dtype (the fill of every
+    slot no token was written to)."""
+    t = torch.full((1,), float("nan"), dtype=W.torch_dtype(spec))
+    return W.storage_view(t)[0]
+
+
+@dataclass
+class Product:
+    cache: PagedKVCache
+    step_slots: torch.Tensor
+    step_pairs: torch.Tensor
+    step_key: torch.Tensor
+    step_value: torch.Tensor
+    tables: torch.Tensor
+    lens: torch.Tensor
+    max_ctx: int
+    q: torch.Tensor
+    slots_host: List[int]
+    pairs_host: List[Tuple[int, int]]
+
+
+@dataclass
+class Oracle:
+    bm: BlockManager
+    k: np.ndarray
+    v: np.ndarray
+    tables: np.ndarray
+    lens: np.ndarray
+    q: np.ndarray
+    slots: List[int]
+    pairs: List[Tuple[int, int]]
+
+
+def build(sc: W.Scenario, device="cuda", with_oracle=True, poison=True):
+    spec = sc.spec
+    shape = (sc.num_blocks, spec.Hkv, spec.block_size, spec.D)
+    cache = PagedKVCache(sc.num_blocks, spec.block_size, spec.Hkv, spec.D, W.torch_dtype(spec),
+                         device, sc.free_order.tolist(),
+                         fill=float("nan") if poison else 0.0)
+    orc = None
+    if with_oracle:
+        bm = BlockManager(sc.num_blocks, spec.block_size, sc.free_order.tolist())
+        fill = poison_bits(spec) if poison else W.storage_view(torch.zeros(1, dtype=W.torch_dtype(spec)))[0]
+        st = np.float32 if spec.dtype == "f32" else np.uint16
+        ok = np.full(shape, fill, dtype=st)
+        ov = np.full(shape, fill, dtype=st)
+    for op in sc.setup_ops:
+        if op.kind == "add":
+            cache.add(op.seq)
+            with_oracle and bm.add(op.seq)
+        elif op.kind == "fork":
+            cache.fork(op.seq, op.arg)
+            with_oracle and bm.fork(op.seq, op.arg)
+        elif op.kind == "release":
+            cache.release(op.seq)
+            with_oracle and bm.release(op.seq)
+        else:
+            k, v = W.kv_content(spec, op.kv_id, op.arg, device)
+            cache.append([op.seq], [op.arg], k, v)
+            if with_oracle:
+                slots, pairs = bm.append(op.seq, op.arg)
+                if pairs:
+                    oracle.copy_blocks(ok, ov, np.array(pairs), spec.dtype_code)
+                oracle.reshape_and_cache(W.storage_view(k), W.storage_view(v), ok, ov,
+                                         np.array(slots), spec.dtype_code)
+            del k, v
+    # the step's appends: reserved now, executed by run_step
+    seqs = [op.seq for op in sc.step_ops]
+    counts = [op.arg for op in sc.step_ops]
+    draws = [W.kv_content(spec, op.kv_id, op.arg, device) for op in sc.step_ops]
+    key = torch.cat([d[0] for d in draws]) if draws else torch.empty((0, spec.Hkv, spec.D), dtype=W.torch_dtype(spec), device=device)
+    value = torch.cat([d[1] for d in draws]) if draws else torch.empty_like(key)
+    del draws
+    slots, pairs = cache.reserve(seqs, counts)
+    tables, lens, max_ctx = cache.tables(sc.batch, sc.max_blocks)
+    q = W.q_content(spec, len(sc.batch), device)
+    prod = Product(cache, torch.tensor(slots, dtype=torch.int64, device=device),
+                   torch.tensor(pairs, dtype=torch.int64, device=device).reshape(-1, 2),
+                   key.contiguous(), value.contiguous(), tables, lens, max_ctx, q, slots, pairs)
+    if with_oracle:
+        oslots, opairs = [], []
+        for sid, n in zip(seqs, counts):
+            s, p = bm.append(sid, n)
+            oslots += s
+            opairs += p
+        if opairs:
+            oracle.copy_blocks(ok, ov, np.array(opairs), spec.dtype_code)
+        oracle.reshape_and_cache(W.storage_view(key), W.storage_view(value), ok, ov,
+                                 np.array(oslots, dtype=np.int64), spec.dtype_code)
+        ot, ol = bm.build_tables(sc.batch, sc.max_blocks)
+        orc = Oracle(bm, ok, ov, ot, ol, W.storage_view(q), oslots, opairs)
+    return prod, orc
+
+
+def run_step(p: Product, spec: W.Spec, partition_size: Optional[int] = None, out=None,
+             workspace=None, stream=None):
+    """One pass of the hot path: copy-on-write, append, decode."""
+    P = spec.partition_size if partition_size is None else partition_size
+    p.cache.copy_on_write(p.step_pairs, stream=stream)
+    p.cache.store(p.step_key, p.step_value, p.step_slots, stream=stream)
+    return p.cache.decode(p.q, p.tables, p.lens, p.max_ctx, spec.softmax_scale, out=out,
+                          partition_size=P, workspace=workspace, stream=stream)
+
+
+def as_f64(t: torch.Tensor, spec: W.Spec) -> np.ndarray:
+    return oracle.decode(W.storage_view(t), spec.dtype_code)
+
+
+def oracle_attention(o: Oracle, spec: W.Spec, rows=None):
+    return oracle.paged_attention(o.q, o.k, o.v, spec.dtype_code, o.tables, o.lens,
+                                  spec.softmax_scale, rows=rows)
+
+
+def check_bookkeeping(p: Product, o: Oracle):
+    assert p.slots_host == o.slots
+    assert [tuple(x) for x in p.pairs_host] == [tuple(x) for x in o.pairs]
+    assert np.array_equal(p.tables.cpu().numpy(), o.tables)
+    assert np.array_equal(p.lens.cpu().numpy(), o.lens)
+
+
+def check_caches(p: Product, o: Oracle, blocks=None):
+    """Byte equality of the caches (all blocks, or the given block ids)."""
+    for dev, host in ((p.cache.k_cache, o.k), (p.cache.v_cache, o.v)):
+        if blocks is None:
+            got = W.storage_view(dev)
+            want = host
+        else:
+            idx = torch.as_tensor(np.asarray(blocks, dtype=np.int64), device=dev.device)
+            got = W.storage_view(dev.index_select(0, idx))
+            want = host[np.asarray(blocks)]
+        assert got.tobytes() == want.tobytes()

@@ -1,0 +1,121 @@
+"""The C-ABI library loads, exports every declared symbol and rejects bad
+arguments on the host before any launch (CPU only: no device call is made)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import paged_kv_cache_443_b200 as pk
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pagedkv.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from paged_kv_cache_443_b200 import build
+    build.build()
+    return pk.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 20
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(pk.EXPORTS) == names
+
+
+def test_version_and_counters(L):
+    assert "sm_100a" in pk.pa_version()
+    assert pk.pa_launch_count() >= 0
+    assert pk.pa_decode_default_partition_size() % 32 == 0
+
+
+def test_partition_and_workspace_sizes(L):
+    P = pk.pa_decode_default_partition_size()
+    assert pk.pa_decode_num_partitions(0) == 1
+    assert pk.pa_decode_num_partitions(P) == 1
+    assert pk.pa_decode_num_partitions(P + 1) == 2
+    assert pk.pa_decode_num_partitions(1000, 64) == 16
+    assert pk.pa_decode_num_partitions(10, 48) == -1
+    assert pk.pa_decode_workspace_bytes(64, 40, 128, P) == 0
+    n = pk.pa_decode_workspace_bytes(3, 5, 64, 1000, 256)
+    assert n >= 3 * 5 * 4 * 66 * 4 and n % 256 == 0
+
+
+FAKE = 1 << 20   # a 16-byte aligned non-null address; never dereferenced on these paths
+
+
+def decode_call(L, **kw):
+    a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, tables=FAKE, maxb=8, lens=FAKE, B=2, Hq=8, Hkv=2,
+             D=128, bs=16, NB=100, scale=0.1, dtype=pk.PA_BF16, P=0, maxctx=100, ws=None,
+             wsb=0, stream=None)
+    a.update(kw)
+    st = L.pa_decode(a["out"], a["q"], a["k"], a["v"], a["tables"], a["maxb"], a["lens"], a["B"],
+                     a["Hq"], a["Hkv"], a["D"], a["bs"], a["NB"], a["scale"], a["dtype"], a["P"],
+                     a["maxctx"], a["ws"], a["wsb"], a["stream"])
+    return st
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(dtype=7), pk.PA_ERR_INVALID),
+    (dict(B=-1), pk.PA_ERR_INVALID),
+    (dict(Hq=6, Hkv=4), pk.PA_ERR_INVALID),
+    (dict(Hq=6, Hkv=2), pk.PA_ERR_UNSUPPORTED),
+    (dict(Hq=32, Hkv=2), pk.PA_ERR_UNSUPPORTED),
+    (dict(D=96), pk.PA_ERR_UNSUPPORTED),
+    (dict(D=0), pk.PA_ERR_INVALID),
+    (dict(bs=64), pk.PA_ERR_UNSUPPORTED),
+    (dict(bs=0), pk.PA_ERR_INVALID),
+    (dict(NB=0), pk.PA_ERR_INVALID),
+    (dict(maxb=0), pk.PA_ERR_INVALID),
+    (dict(P=100), pk.PA_ERR_INVALID),
+    (dict(maxctx=-1), pk.PA_ERR_INVALID),
+    (dict(maxctx=8 * 16 + 1), pk.PA_ERR_INVALID),
+    (dict(scale=float("nan")), pk.PA_ERR_INVALID),
+    (dict(q=None), pk.PA_ERR_INVALID),
+    (dict(out=FAKE + 8), pk.PA_ERR_INVALID),
+    (dict(tables=FAKE + 2), pk.PA_ERR_INVALID),
+    (dict(maxctx=100, P=32), pk.PA_ERR_INVALID),            # workspace needed, none given
+    (dict(maxctx=100, P=32, ws=FAKE, wsb=64), pk.PA_ERR_INVALID),
+])
+def test_decode_rejects_bad_arguments(L, kw, want):
+    before = pk.pa_launch_count()
+    assert decode_call(L, **kw) == want
+    assert pk.pa_last_error()
+    assert pk.pa_launch_count() == before
+
+
+def test_decode_with_no_sequences_is_a_no_op(L):
+    assert decode_call(L, B=0) == pk.PA_OK
+
+
+def test_reshape_and_copy_reject_bad_arguments(L):
+    r = lambda **kw: L.pa_reshape_and_cache(kw.get("key", FAKE), FAKE, FAKE, FAKE,
+                                            kw.get("slots", FAKE), kw.get("N", 4), 2,
+                                            kw.get("D", 128), kw.get("bs", 16), 10,
+                                            kw.get("dtype", pk.PA_F16), None)
+    assert r(dtype=5) == pk.PA_ERR_INVALID
+    assert r(N=-1) == pk.PA_ERR_INVALID
+    assert r(D=80) == pk.PA_ERR_UNSUPPORTED
+    assert r(bs=12) == pk.PA_ERR_UNSUPPORTED
+    assert r(key=None) == pk.PA_ERR_INVALID
+    assert r(key=FAKE + 4) == pk.PA_ERR_INVALID
+    assert r(slots=FAKE + 4) == pk.PA_ERR_INVALID
+    assert r(N=0) == pk.PA_OK
+    c = lambda **kw: L.pa_copy_blocks(FAKE, kw.get("v", FAKE), kw.get("pairs", FAKE),
+                                      kw.get("P", 3), 2, 128, 16, 10, kw.get("dtype", pk.PA_BF16),
+                                      None)
+    assert c(P=-1) == pk.PA_ERR_INVALID
+    assert c(v=None) == pk.PA_ERR_INVALID
+    assert c(pairs=FAKE + 4) == pk.PA_ERR_INVALID
+    assert c(dtype=9) == pk.PA_ERR_INVALID
+    assert c(P=0) == pk.PA_OK

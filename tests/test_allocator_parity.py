@@ -1,0 +1,124 @@
+"""The C++ block manager of libpagedkv.so agrees bit for bit with the oracle's
+(block tables, context lengths, slots, copy-on-write pairs, reference counts,
+free stack, OOM behaviour) on the worked example, the workloads and long
+random operation sequences.  CPU only."""
+import numpy as np
+import pytest
+
+import paged_kv_cache_443_b200 as pk
+import workloads as W
+from oracle.allocator import OOM, BlockManager, Invalid
+from pa_testlib import read_golden
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from paged_kv_cache_443_b200 import build
+    build.build()
+
+
+def same_state(a: pk.BlockAllocator, o: BlockManager, live):
+    assert a.num_free() == o.num_free()
+    assert a.free_stack() == o.free_stack()
+    for b in range(o.num_blocks):
+        assert a.refcount(b) == o.refcount[b]
+    if live:
+        mb = max(1, max(len(o.blocks_of(s)) for s in live))
+        ta, la = a.build_tables(live, mb)
+        to, lo = o.build_tables(live, mb)
+        assert np.array_equal(ta, to) and np.array_equal(la, lo)
+
+
+def test_worked_example():
+    g = read_golden("block_table_example.txt")
+    bs, L, table = g["block_size"][0], g["seq_len"][0], g["table"]
+    order = [b for b in range(12) if b not in table] + list(reversed(table))
+    a = pk.BlockAllocator(12, bs, order)
+    a.add(5)
+    slots, pairs = a.append(5, L)
+    t, lens = a.build_tables([5], 3)
+    assert t.tolist() == [table] and lens.tolist() == [L] and pairs == []
+    assert slots[36] == 148
+
+
+def test_errors_map_to_statuses():
+    a = pk.BlockAllocator(4, 4)
+    a.add(0)
+    with pytest.raises(pk.PagedKVError):
+        a.add(0)
+    with pytest.raises(pk.PagedKVError):
+        a.fork(3, 4)
+    with pytest.raises(pk.PagedKVError):
+        a.append(9, 1)
+    with pytest.raises(pk.PagedKVError):
+        a.release(9)
+    a.append(0, 6)
+    a.fork(0, 1)
+    before = (a.free_stack(), a.num_tokens(1))
+    with pytest.raises(pk.OutOfBlocks):
+        a.append(1, 11)
+    assert before == (a.free_stack(), a.num_tokens(1))
+    with pytest.raises(pk.PagedKVError):
+        pk.BlockAllocator(3, 4, [0, 1, 1])
+    with pytest.raises(pk.PagedKVError):
+        a.build_tables([0], 1)
+    assert a.refcount(-1) == -1 and a.refcount(4) == -1
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_operation_sequences_match_oracle(seed):
+    rng = np.random.default_rng(1000 + seed)
+    for trial in range(8):
+        NB, bs = int(rng.integers(3, 48)), int(rng.choice([1, 2, 8, 16, 32]))
+        order = rng.permutation(NB).tolist() if rng.random() < 0.7 else None
+        a = pk.BlockAllocator(NB, bs, order)
+        o = BlockManager(NB, bs, order)
+        next_id = 0
+        for _ in range(150):
+            live = sorted(o.seqs)
+            r = rng.random()
+            if r < 0.18 or not live:
+                a.add(next_id)
+                o.add(next_id)
+                next_id += 1
+            elif r < 0.33:
+                p = int(rng.choice(live))
+                a.fork(p, next_id)
+                o.fork(p, next_id)
+                next_id += 1
+            elif r < 0.85:
+                sid = int(rng.choice(live))
+                n = int(rng.integers(0, 3 * bs + 3))
+                try:
+                    want = o.append(sid, n)
+                except OOM:
+                    with pytest.raises(pk.OutOfBlocks):
+                        a.append(sid, n)
+                else:
+                    got = a.append(sid, n)
+                    assert got[0] == want[0] and [tuple(x) for x in got[1]] == want[1]
+            else:
+                sid = int(rng.choice(live))
+                a.release(sid)
+                o.release(sid)
+            same_state(a, o, sorted(o.seqs))
+
+
+@pytest.mark.parametrize("name", ["tiny", "opt13b", "llama13b_ps", "gqa70b", "long_prefix"])
+def test_workload_scripts_match_oracle(name):
+    sc = W.scenario(W.small(name) if name != "tiny" else W.TINY)
+    a = pk.BlockAllocator(sc.num_blocks, sc.spec.block_size, sc.free_order.tolist())
+    o = BlockManager(sc.num_blocks, sc.spec.block_size, sc.free_order.tolist())
+    for op in sc.setup_ops + sc.step_ops:
+        if op.kind == "add":
+            a.add(op.seq); o.add(op.seq)
+        elif op.kind == "fork":
+            a.fork(op.seq, op.arg); o.fork(op.seq, op.arg)
+        elif op.kind == "release":
+            a.release(op.seq); o.release(op.seq)
+        else:
+            ga, wo = a.append(op.seq, op.arg), o.append(op.seq, op.arg)
+            assert ga[0] == wo[0] and [tuple(x) for x in ga[1]] == wo[1]
+    ta, la = a.build_tables(sc.batch, sc.max_blocks)
+    to, lo = o.build_tables(sc.batch, sc.max_blocks)
+    assert np.array_equal(ta, to) and np.array_equal(la, lo)

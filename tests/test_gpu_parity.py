@@ -1,0 +1,192 @@
+"""GPU parity: the CUDA library against the oracle, on the same seeded inputs.
+
+Bit-exact: block tables, context lengths, slots, copy-on-write pairs (block
+manager) and cache bytes after copy_blocks + reshape_and_cache.  Within the
+stated tolerance (max abs error of the output, 2e-2 for fp16/bf16, 1e-5 for
+fp32, fp32 accumulation): decode attention.  Every cache slot no token was
+written to holds NaN, so reading an unused tail slot into a result shows up.
+"""
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_443_b200 as pk
+import workloads as W
+from pa_harness import (TOL, as_f64, build, check_bookkeeping, check_caches, oracle_attention,
+                        run_step)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def clean_status():
+    pk.pa_device_status(clear=True)
+    yield
+
+
+def full_check(spec, partition_size=None):
+    sc = W.scenario(spec)
+    p, o = build(sc)
+    out = run_step(p, spec, partition_size)
+    torch.cuda.synchronize()
+    assert pk.pa_device_status() == 0
+    check_bookkeeping(p, o)
+    check_caches(p, o)
+    got = as_f64(out, spec)
+    want = oracle_attention(o, spec)
+    assert np.isfinite(got).all()
+    err = np.abs(got - want).max()
+    assert err <= TOL[spec.dtype], (spec.name, err)
+    return got, want
+
+
+@pytest.mark.parametrize("name", ["tiny", "opt13b", "llama13b_ps", "gqa70b", "long_prefix"])
+def test_small_workloads(name):
+    full_check(W.small(name))
+
+
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_long_prefix_block_sizes(bs):
+    full_check(replace(W.small("long_prefix"), block_size=bs, name=f"lp_small_bs{bs}"))
+
+
+@pytest.mark.parametrize("P", [32, 64, 96, 256, 512, 4096])
+def test_partition_sizes(P):
+    full_check(W.small("opt13b"), partition_size=P)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_dtype_head_group_matrix(dtype, D, G):
+    spec = W.Spec(f"m_{dtype}_{D}_{G}", dtype, 2 * G, 2, D, 16, "independent", 5, seed=77 + G + D,
+                  ctx_dist="explicit", ctx_list=(1, 77, 300, 513, 1100), partition_size=256)
+    full_check(spec)
+
+
+def test_edge_context_lengths():
+    lens = (0, 1, 15, 16, 17, 31, 32, 33, 511, 512, 513, 1024, 1025, 2047)
+    spec = W.Spec("edges", "bf16", 8, 2, 128, 16, "independent", len(lens), seed=5,
+                  ctx_dist="explicit", ctx_list=lens, partition_size=512)
+    got, _ = full_check(spec)
+    assert np.all(got[0] == 0.0)            # context 0 -> zero row
+    spec32 = replace(spec, block_size=32, name="edges32", partition_size=64)
+    full_check(spec32)
+
+
+def test_physical_placement_gives_bit_identical_output():
+    spec = W.small("gqa70b")
+    sc1 = W.scenario(spec)
+    sc2 = W.scenario(spec)
+    sc2.free_order = np.random.default_rng(99).permutation(sc2.num_blocks).astype(np.int32)
+    p1, _ = build(sc1, with_oracle=False)
+    p2, _ = build(sc2, with_oracle=False)
+    assert not torch.equal(p1.tables, p2.tables)
+    o1 = run_step(p1, spec)
+    o2 = run_step(p2, spec)
+    torch.cuda.synchronize()
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+
+
+def test_two_phase_equals_one_call():
+    spec = W.small("opt13b")
+    p, _ = build(W.scenario(spec), with_oracle=False)
+    run_step(p, spec)
+    ws = p.cache.workspace(p.q.shape[0], p.q.shape[1], p.max_ctx, 64)
+    a = torch.empty_like(p.q)
+    b = torch.empty_like(p.q)
+    pk.pa_decode(a, p.q, p.cache.k_cache, p.cache.v_cache, p.tables, p.lens, spec.softmax_scale,
+                 p.max_ctx, partition_size=64, workspace=ws)
+    pk.pa_decode_partitions(b, p.q, p.cache.k_cache, p.cache.v_cache, p.tables, p.lens,
+                            spec.softmax_scale, p.max_ctx, partition_size=64, workspace=ws)
+    pk.pa_decode_reduce(b, p.lens, p.max_ctx, partition_size=64, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_repeated_steps_are_idempotent():
+    spec = W.small("llama13b_ps")
+    p, o = build(W.scenario(spec))
+    first = run_step(p, spec).clone()
+    for _ in range(3):
+        again = run_step(p, spec)
+    torch.cuda.synchronize()
+    assert torch.equal(first.view(torch.int16), again.view(torch.int16))
+    check_caches(p, o)
+
+
+def test_device_checks_flag_bad_values_without_faulting():
+    spec = W.small("opt13b")
+    p, _ = build(W.scenario(spec), with_oracle=False)
+    cache = p.cache
+    # block-table entry outside the pool
+    bad = p.tables.clone()
+    bad[0, 0] = cache.num_blocks + 5
+    out = cache.decode(p.q, bad, p.lens, p.max_ctx, spec.softmax_scale)
+    assert pk.pa_device_status() & pk.PA_DEVERR_TABLE
+    # context longer than the table row / the declared maximum
+    lens = p.lens.clone()
+    lens[1] = p.tables.shape[1] * spec.block_size + 100
+    cache.decode(p.q, p.tables, lens, p.max_ctx, spec.softmax_scale)
+    assert pk.pa_device_status() & pk.PA_DEVERR_CONTEXT
+    # slot beyond the cache
+    slots = p.step_slots.clone()
+    slots[0] = cache.num_blocks * spec.block_size
+    cache.store(p.step_key, p.step_value, slots)
+    assert pk.pa_device_status() & pk.PA_DEVERR_SLOT
+    # copy pair outside the pool
+    cache.copy_on_write(torch.tensor([[0, cache.num_blocks]], dtype=torch.int64, device="cuda"))
+    assert pk.pa_device_status() & pk.PA_DEVERR_PAIR
+    # the context is still healthy
+    run_step(p, spec)
+    torch.cuda.synchronize()
+    assert pk.pa_device_status() == 0
+
+
+def test_launch_counter_counts_kernels():
+    spec = W.small("opt13b")
+    p, _ = build(W.scenario(spec), with_oracle=False)
+    n0 = pk.pa_launch_count()
+    run_step(p, spec, partition_size=512)
+    np_ = pk.pa_decode_num_partitions(p.max_ctx, 512)
+    expect = (1 if p.step_pairs.numel() else 0) + 1 + 1 + (1 if np_ > 1 else 0)
+    assert pk.pa_launch_count() - n0 == expect
+
+
+# ---------------------------------------------------------------------------
+# full sizes of the five workloads, in the launch configuration the benchmark
+# times (default partition size), checked on sampled rows
+
+
+def sampled_rows(o, spec, n=96, seed=0):
+    rng = np.random.default_rng(seed)
+    B = len(o.lens)
+    rows = {(int(b), int(h)) for b, h in zip(rng.integers(0, B, n), rng.integers(0, spec.Hq, n))}
+    for b in (int(np.argmax(o.lens)), int(np.argmin(o.lens))):
+        rows |= {(b, 0), (b, spec.Hq - 1)}
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+@pytest.mark.parametrize("name", ["tiny", "opt13b", "llama13b_ps", "gqa70b", "long_prefix_bs8",
+                                  "long_prefix_bs16", "long_prefix_bs32"])
+def test_full_size_workloads_sampled(name):
+    spec = W.long_prefix(int(name[-2:].lstrip("s"))) if name.startswith("long_prefix") else W.FULL[name]
+    sc = W.scenario(spec)
+    p, o = build(sc)
+    out = run_step(p, spec)
+    torch.cuda.synchronize()
+    assert pk.pa_device_status() == 0
+    check_bookkeeping(p, o)
+    touched = sorted({s // spec.block_size for s in o.slots} | {d for _, d in o.pairs})
+    rng = np.random.default_rng(1)
+    extra = rng.choice(sc.num_blocks, size=min(256, sc.num_blocks), replace=False).tolist()
+    check_caches(p, o, blocks=sorted(set(touched) | set(extra)))
+    rows = sampled_rows(o, spec)
+    want = oracle_attention(o, spec, rows=rows)
+    got_all = as_f64(out, spec)
+    got = got_all[rows[:, 0], rows[:, 1]]
+    assert np.isfinite(got_all).all()
+    assert np.abs(got - want).max() <= TOL[spec.dtype]

@@ -57,7 +57,8 @@ class Spec:
     scale: Optional[float] = None     # None = 1/sqrt(D)
     partition_size: int = 512
     # independent
-    ctx_dist: str = "uniform"       # 'uniform' | 'lognormal'
+    ctx_dist: str = "uniform"       # 'uniform' | 'lognormal' | 'explicit'
+    ctx_list: Tuple[int, ...] = ()  # explicit context lengths (num_seqs of them)
     ctx_lo: int = 1
     ctx_hi: int = 64
     ctx_median: float = 600.0
@@ -164,6 +165,9 @@ def _ctx_lengths(spec: Spec, rng) -> np.ndarray:
     if spec.ctx_dist == "lognormal":
         x = rng.lognormal(mean=np.log(spec.ctx_median), sigma=spec.ctx_sigma, size=B)
         return np.clip(np.rint(x), spec.ctx_lo, spec.ctx_hi).astype(np.int64)
+    if spec.ctx_dist == "explicit":
+        assert len(spec.ctx_list) == B
+        return np.asarray(spec.ctx_list, dtype=np.int64)
     raise ValueError(spec.ctx_dist)
 
 
@@ -187,9 +191,10 @@ def scenario(spec: Spec) -> Scenario:
         for sid, L in zip(batch, lens):
             setup.append(Op("add", sid))
             app(setup, sid, L - 1)
-        for sid in batch:
-            app(step, sid, 1)
-        blocks_needed = int(sum(-(-int(L) // bs) for L in lens))
+        for sid, L in zip(batch, lens):
+            if L > 0:                   # an empty sequence appends nothing
+                app(step, sid, 1)
+        blocks_needed = max(1, int(sum(-(-int(L) // bs) for L in lens)))
     elif spec.kind == "parallel_sampling":
         P, S = spec.num_prompts, spec.samples_per_prompt
         prompts = rng.integers(spec.prompt_lo, spec.prompt_hi + 1, size=P)

@@ -154,3 +154,19 @@ def check_caches(p: Product, o: Oracle, blocks=None):
             got = W.storage_view(dev.index_select(0, idx))
             want = host[np.asarray(blocks)]
         assert got.tobytes() == want.tobytes()
+
+
+def check_token_slots(p: Product, o: Oracle):
+    """Byte equality of every cache slot that holds a token of the batch (unused
+    tail slots excluded)."""
+    bs = p.cache.block_size
+    blk, off = [], []
+    for b in range(len(o.lens)):
+        j = np.arange(int(o.lens[b]))
+        blk.append(o.tables[b, j // bs])
+        off.append(j % bs)
+    blk = np.concatenate(blk).astype(np.int64)
+    off = np.concatenate(off).astype(np.int64)
+    for dev, host in ((p.cache.k_cache, o.k), (p.cache.v_cache, o.v)):
+        got = W.storage_view(dev)[blk, :, off, :]
+        assert got.tobytes() == host[blk, :, off, :].tobytes()

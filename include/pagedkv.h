@@ -173,6 +173,36 @@ pa_status pa_decode_reduce(void* out, const int32_t* context_lens, int num_seqs,
                            int head_size, pa_dtype dtype, int partition_size, int max_context_len,
                            const void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * pa_decode for callers that cannot allocate device memory.  The pages have no
+ * counterpart: this is an interface convenience, not part of the method.
+ *
+ * Same arguments and result as pa_decode, without the workspace: the split-K
+ * scratch comes from a fixed 32 MiB array compiled into the library, which
+ * every GPU that loads the library holds until the process exits.  No call
+ * allocates (no cudaMalloc / cudaFree or allocating library routine).  Meant
+ * for callers whose device memory is all committed to a KV-cache pool, plain C
+ * hosts without a device allocator, and loops that cannot take cudaMalloc's
+ * implicit device synchronisation.
+ *
+ *   - A batch whose pa_decode_workspace_bytes(...) exceeds 32 MiB is rejected
+ *     with PA_ERR_UNSUPPORTED (and a message) before any launch.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array, which keeps the last call's
+ *     contents.  Nothing in it needs to start at zero (each call writes every
+ *     partial it reads), but calls that overlap on the GPU -- on different
+ *     streams, or from different host threads -- race on it and give wrong
+ *     results; order them on one stream.
+ */
+pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, int max_blocks_per_seq,
+                            const int32_t* context_lens, int num_seqs, int num_heads,
+                            int num_kv_heads, int head_size, int block_size, int num_blocks,
+                            float scale, pa_dtype dtype, int partition_size, int max_context_len,
+                            void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Cache updates                                                           */
 

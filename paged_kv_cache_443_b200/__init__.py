@@ -28,7 +28,8 @@ PA_DEVERR_TABLE, PA_DEVERR_CONTEXT, PA_DEVERR_SLOT, PA_DEVERR_PAIR, PA_DEVERR_TI
 EXPORTS = (
     "pa_last_error", "pa_version", "pa_launch_count", "pa_device_status",
     "pa_decode_default_partition_size", "pa_decode_num_partitions", "pa_decode_workspace_bytes",
-    "pa_decode", "pa_decode_partitions", "pa_decode_reduce", "pa_reshape_and_cache",
+    "pa_decode", "pa_decode_partitions", "pa_decode_reduce", "pa_decode_noalloc",
+    "pa_reshape_and_cache",
     "pa_copy_blocks", "pa_alloc_create", "pa_alloc_destroy", "pa_alloc_num_free",
     "pa_alloc_refcount", "pa_alloc_free_stack", "pa_seq_add", "pa_seq_fork", "pa_seq_append",
     "pa_seq_free", "pa_seq_num_tokens", "pa_build_tables",
@@ -76,6 +77,8 @@ def lib():
         "pa_decode_partitions": ([vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, f32,
                                   i32, i32, i32, vp, sz, vp], i32),
         "pa_decode_reduce": ([vp, vp, i32, i32, i32, i32, i32, i32, vp, sz, vp], i32),
+        "pa_decode_noalloc": ([vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, f32,
+                               i32, i32, i32, vp], i32),
         "pa_reshape_and_cache": ([vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp], i32),
         "pa_copy_blocks": ([vp, vp, vp, i32, i32, i32, i32, i32, i32, vp], i32),
         "pa_alloc_create": ([i32, i32, pi32, ctypes.POINTER(vp)], i32),
@@ -216,6 +219,17 @@ def pa_decode_reduce(out, context_lens, max_context_len, partition_size=0, works
     _check(lib().pa_decode_reduce(_ptr(out), _ptr(context_lens), B, Hq, D, _dtype_code(out),
                                   int(partition_size), int(max_context_len), _ptr(workspace),
                                   ws_bytes, _stream(stream)))
+
+
+def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                      max_context_len, partition_size=0, stream=None) -> None:
+    """pa_decode without a workspace argument, for callers that cannot allocate
+    device memory: the split-K scratch is a fixed 32 MiB array inside the
+    library (shared by all calls on a device; calls that overlap on the GPU
+    race).  Batches needing more scratch raise PagedKVError (unsupported)."""
+    a = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, partition_size,
+                     max_context_len, None, stream)
+    _check(lib().pa_decode_noalloc(*a[:17], a[19]))
 
 
 def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None) -> None:

@@ -47,6 +47,11 @@ FALLBACK_HBM_GBS = 6650.0
 
 
 def workload_spec(name):
+    if name == "opt13b_compact":
+        # the opt13b launch with a pool of 1.25x the blocks it needs (about 1 GB
+        # on the device instead of 6.6): the profiling case
+        from dataclasses import replace
+        return replace(W.FULL["opt13b"], name="opt13b_compact", num_blocks=None)
     if name.startswith("long_prefix_bs"):
         return W.long_prefix(int(name[len("long_prefix_bs"):]))
     if name == "long_prefix":
@@ -64,6 +69,8 @@ WORKLOAD_TEXT = {
 
 
 def workload_text(name):
+    if name == "opt13b_compact":
+        return WORKLOAD_TEXT["opt13b"].replace("20,000-block pool", "pool of 1.25x the blocks needed")
     base = name.split("_bs")[0] if name.startswith("long_prefix") else name
     txt = WORKLOAD_TEXT[base]
     if base == "long_prefix":
@@ -383,7 +390,7 @@ def run_ours(args):
 
     unique, logical, other = step_bytes(spec, tables.cpu().numpy(), lens.cpu().numpy())
     flush = unique < 8 * L2_BYTES
-    scratch = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device) if flush else None
+    scratch = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=device) if flush else None
 
     def step(ev=None):
         if ev is not None:
@@ -408,9 +415,10 @@ def run_ours(args):
         step()
     torch.cuda.synchronize(device)
     assert pk.pa_device_status() == 0, "device-side check failed during warm-up"
-    # clock soak: keep the GPU under this load for ~0.5 s before timing
+    # clock soak: keep the GPU under this load for a while before timing, so the
+    # clock samples describe the timed region's state
     soak_t0 = time.time()
-    while time.time() - soak_t0 < 0.5:
+    while time.time() - soak_t0 < args.soak_seconds:
         for _ in range(20):
             step()
         torch.cuda.synchronize(device)
@@ -420,9 +428,12 @@ def run_ours(args):
     launches0 = pk.pa_launch_count()
     barrier(world, device)
     torch.cuda.synchronize(device)
+    sink = torch.empty((), dtype=torch.float32, device=device)
     for i in range(K):
         if flush:
-            scratch.fill_(float(i))           # evicts the previous step's lines from L2
+            # evict the previous step's lines from L2 by streaming a 2x-L2 buffer;
+            # a read leaves no dirty lines for the timed kernels to write back
+            torch.amax(scratch, dim=0, out=sink)
         step(evs[i])
     torch.cuda.synchronize(device)
     barrier(world, device)
@@ -515,7 +526,7 @@ def run_ours(args):
                 "max_context_len": max_ctx, "partition_size": P, "num_partitions": n_part,
                 "kv_bytes_unique": unique, "kv_bytes_logical": logical,
                 "new_tokens_per_step": int(key.shape[0]), "cow_pairs_per_step": int(pairs.shape[0]),
-                "l2": ("L2 flushed between timed steps (256 MB write, excluded from the step time)"
+                "l2": ("L2 flushed between timed steps (252 MB streamed read, excluded from the step time)"
                        if flush else f"inputs larger than L2: {unique / 1e9:.2f} GB of KV per step"),
                 "parallelism": "replicas" if world == 1 else f"replicas x{world} (no collective)",
             },
@@ -549,8 +560,10 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    choices=["tiny", "opt13b", "llama13b_ps", "gqa70b", "long_prefix_bs8",
-                             "long_prefix_bs16", "long_prefix_bs32"])
+                    choices=["tiny", "opt13b", "opt13b_compact", "llama13b_ps", "gqa70b",
+                             "long_prefix_bs8", "long_prefix_bs16", "long_prefix_bs32"])
+    ap.add_argument("--soak-seconds", type=float, default=0.5,
+                    help="untimed load before the timed steps (clock samples)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

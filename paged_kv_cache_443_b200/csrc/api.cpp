@@ -123,6 +123,11 @@ pa_status check_decode_full(const char* fn, void* out, const void* q, const void
   return PA_OK;
 }
 
+int launch_partitions(const pa::DecodeArgs& a, unsigned int* status, void* stream) {
+  return pa::decode_tc_supported(a) ? pa::launch_decode_partitions_tc(a, status, stream)
+                                    : pa::launch_decode_partitions(a, status, stream);
+}
+
 pa_status launch_status(const char* fn, int err, int n_launched) {
   if (err != cudaSuccess)
     return pa::fail(PA_ERR_CUDA, "%s: launch failed: %s", fn,
@@ -168,7 +173,7 @@ extern "C" pa_status pa_decode_partitions(void* out, const void* q, const void* 
   if (st != PA_OK || num_seqs == 0) return st;
   unsigned int* status = pa::device_status_word();
   if (!status) return PA_ERR_CUDA;
-  return launch_status("pa_decode_partitions", pa::launch_decode_partitions(a, status, stream), 1);
+  return launch_status("pa_decode_partitions", launch_partitions(a, status, stream), 1);
 }
 
 extern "C" pa_status pa_decode_reduce(void* out, const int32_t* context_lens, int num_seqs,
@@ -221,7 +226,7 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   if (st != PA_OK || num_seqs == 0) return st;
   unsigned int* status = pa::device_status_word();
   if (!status) return PA_ERR_CUDA;
-  st = launch_status("pa_decode", pa::launch_decode_partitions(a, status, stream), 1);
+  st = launch_status("pa_decode", launch_partitions(a, status, stream), 1);
   if (st != PA_OK || a.num_partitions <= 1) return st;
   return launch_status("pa_decode", pa::launch_decode_reduce(a, status, stream), 1);
 }

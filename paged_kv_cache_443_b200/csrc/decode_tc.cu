@@ -1,0 +1,605 @@
+// decode_tc.cu -- paged decode attention on the 5th-generation tensor cores
+// (tcgen05 + TMEM) for grouped-query heads (G = Hq/Hkv in {4, 8}), fp16/bf16,
+// head size 128.
+//
+// Same contract and split-K partials as decode.cu ("자기회귀 생성과 KV 캐시" and
+// "PagedAttention의 설계", supersilo.blog vLLM summary: scores q.k/sqrt(d_k),
+// softmax over all valid tokens with one running max/sum across blocks and
+// partitions, unused tail slots masked).  When G query heads share a kv head the
+// per-token work is a real dense contraction, so the two products run on the
+// tensor cores with tokens as the MMA's M dimension:
+//
+//   S^T [128 tokens x 16] = K [128 x 128] . Q^T [128 x 16]     (heads padded to 16)
+//   O^T [128 dims   x 16] += V^T [128 x 128] . P^T [128 x 16]
+//
+// Roles in a CTA of 6 warps, one CTA per (sequence, kv head, partition):
+//   warp 0   producer: block-table lookups, 2-D TMA loads (128-byte swizzle) of
+//            every physical block's K and V rows into a ring of three 32 KB slots
+//            holding K_0, V_0, K_1, V_1, ... (two boxes of 64 columns per block);
+//   warp 1   TMEM owner and MMA issuer (one thread): S = K Q^T into one of two
+//            TMEM score buffers, O += V^T P^T into the TMEM output buffer;
+//   warps 2-5  softmax: each thread owns one token row of S (its TMEM lane),
+//            masks invalid tokens, keeps a running max that is raised only when
+//            a score exceeds it by 2^8 (then O and the partial sums are
+//            rescaled), writes P (cache dtype) into shared memory for the
+//            second MMA, zeroes the V rows of invalid tokens of a final tile, and
+//            at the end reads its row of O from TMEM and writes the output or the
+//            split-K partial.
+// About 110 KB of shared memory, so two CTAs share an SM and hide each other's
+// pipeline fill.  Every mbarrier wait is bounded; block ids outside the pool are
+// skipped and flagged.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <mutex>
+#include <type_traits>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+namespace {
+
+constexpr unsigned FULL = 0xffffffffu;
+constexpr int TOK = 128;                     // tokens per tile (M of the first MMA)
+constexpr int NPAD = 16;                     // N of both MMAs (heads padded)
+constexpr int DH = 128;                      // head size
+constexpr int SLOTS = 3;                     // ring slots (K or V of one tile each)
+constexpr int HALF_BYTES = TOK * 128;        // 128 rows x 64 elements x 2 B
+constexpr int SLOT_BYTES = 2 * HALF_BYTES;   // 32 KB
+constexpr int OPB_BYTES = 2 * NPAD * 128;    // a 16-row operand in two 64-column blocks: 4 KB
+constexpr int OFF_RING = 0;
+constexpr int OFF_Q = OFF_RING + SLOTS * SLOT_BYTES;
+constexpr int OFF_P = OFF_Q + OPB_BYTES;     // two P buffers
+constexpr int OFF_BAR = OFF_P + 2 * OPB_BYTES;
+constexpr int NBARS = 2 * SLOTS + 8;         // ring full/empty, s_full/s_free, p_full/p_free
+constexpr int OFF_TMEM = OFF_BAR + NBARS * 8;
+constexpr int OFF_RED = OFF_TMEM + 16;       // 4 warps x 16 floats
+constexpr int SMEM_USED = OFF_RED + 4 * NPAD * 4;
+constexpr int SMEM_BYTES = SMEM_USED + 1024; // slack to align the base to 1024 B
+constexpr int THREADS = 192;
+constexpr int TMEM_COLS = 64;                // S0 [0,16), S1 [16,32), O [32,48)
+constexpr float RESCALE_THRESHOLD = 8.0f;    // log2 units: raise the max past 2^8 growth
+
+static_assert(SMEM_BYTES * 2 + 2048 <= 228 * 1024, "two CTAs per SM");
+
+struct TcParams {
+  void* out;
+  const void* q;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  float* ws_o;
+  float* ws_m;
+  float* ws_l;
+  unsigned int* status;
+  int64_t max_blocks;
+  int Hq, Hkv, num_blocks, block_size, partition_size, num_partitions;
+  float scale_log2;
+};
+
+// ---- tcgen05 / TMA helpers ----
+
+// Byte offset of element (row, col) of a [rows x 64] 16-bit operand block stored
+// with the 128-byte swizzle (16-byte chunk index XOR row % 8).
+__device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t col) {
+  return row * 128u + ((((col >> 3) ^ (row & 7u)) & 7u) << 4) + (col & 7u) * 2u;
+}
+
+// Shared-memory matrix descriptor (sm_100): start, leading / stride byte
+// offsets (16-byte units), version 1, 128-byte swizzle.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor of kind::f16 with fp32 accumulation, M = 128, N = 16.
+template <typename T>
+__device__ __forceinline__ constexpr uint32_t instr_desc(bool a_mn_major) {
+  constexpr uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+         ((uint32_t)(NPAD >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_addr(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, "
+      "[%16];\n\ttcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15]))
+      : "memory");
+}
+
+// 2-D TMA tile load (this GPU's memory, no multicast) completing on `bar`.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4}], [%2];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// OR of `pred` over the `n` threads reaching named barrier `id`.
+__device__ __forceinline__ bool bar_or(int id, int n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+template <typename T>
+__device__ __forceinline__ uint16_t to_bits(float x) {
+  T h = Elem<T>::from_float(x);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
+
+template <typename T, int G>
+__global__ void __launch_bounds__(THREADS, 2)
+    decode_partition_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmap_k,
+                               const __grid_constant__ CUtensorMap tmap_v) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* ring = smem + OFF_RING;
+  uint8_t* qop = smem + OFF_Q;
+  uint8_t* pop = smem + OFF_P;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* ring_full = bars;
+  uint64_t* ring_empty = bars + SLOTS;
+  uint64_t* s_full = bars + 2 * SLOTS;      // [2]
+  uint64_t* s_free = s_full + 2;            // [2]
+  uint64_t* p_full = s_free + 2;            // [2]
+  uint64_t* p_free = p_full + 2;            // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
+  float* red = reinterpret_cast<float*>(smem + OFF_RED);
+
+  const int b = blockIdx.x, g = blockIdx.y, part = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  int L = p.context_lens[b];
+  const int P = p.partition_size;
+  int64_t cap = p.max_blocks * p.block_size;
+  const int64_t grid_cap = static_cast<int64_t>(p.num_partitions) * P;
+  cap = cap < grid_cap ? cap : grid_cap;
+  if (L < 0 || L > cap) {
+    if (threadIdx.x == 0 && part == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
+    L = L < 0 ? 0 : static_cast<int>(cap);
+  }
+  const int start = part * P;
+  if (L == 0) {
+    if (part == 0) {
+      T* o = static_cast<T*>(p.out) + (static_cast<int64_t>(b) * p.Hq + g * G) * DH;
+      for (int i = threadIdx.x; i < G * DH; i += THREADS) o[i] = Elem<T>::from_float(0.f);
+    }
+    return;
+  }
+  if (start >= L) return;
+  const int end = min(L, start + P);
+  const int n_tiles = (end - start + TOK - 1) / TOK;
+  const bool single = (L <= P);
+
+  // ---- set-up ----
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < SLOTS; ++s) {
+      mbar_init(&ring_full[s], 1);
+      mbar_init(&ring_empty[s], 1);
+    }
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(&s_full[j], 1);
+      mbar_init(&s_free[j], 4);
+      mbar_init(&p_full[j], 4);
+      mbar_init(&p_free[j], 1);
+    }
+    fence_mbar_init();
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (warp >= 2) {
+    // Q^T operand (16 rows = heads, 128 columns = dims, two swizzled 64-column
+    // blocks), rows >= G zero; both P buffers zeroed (their rows >= G stay 0).
+    const int t = threadIdx.x - 64;
+    const T* qrow = static_cast<const T*>(p.q) + (static_cast<int64_t>(b) * p.Hq + g * G) * DH;
+    for (int i = t; i < NPAD * (DH / 8); i += 128) {   // one 16-byte chunk each
+      const int h = i / (DH / 8);
+      const int c = i % (DH / 8);                      // chunk of 8 dims
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (h < G) v = __ldg(reinterpret_cast<const uint4*>(qrow + h * DH + c * 8));
+      const uint32_t off = (c / 8) * (NPAD * 128) + sw128(h, (c % 8) * 8);
+      *reinterpret_cast<uint4*>(qop + off) = v;
+    }
+    for (int i = t; i < 2 * OPB_BYTES / 16; i += 128)
+      reinterpret_cast<uint4*>(pop)[i] = make_uint4(0, 0, 0, 0);
+    fence_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ================= producer =================
+    const int bs = p.block_size;
+    const int bpt = TOK / bs;                            // blocks per tile: 4, 8 or 16
+    const int first_blk = start / bs;
+    const int last_blk = (end + bs - 1) / bs;
+    const int32_t* trow = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
+    const int row_stride = p.Hkv * bs;                   // rows of one physical block
+    bool ok = true;
+    int issued = 0;
+    for (int i = 0; i < n_tiles && ok; ++i) {
+      const int b0 = first_blk + i * bpt;
+      const int nb = min(bpt, last_blk - b0);
+      int pb = -1;
+      if (lane < nb) pb = __ldg(trow + b0 + lane);
+      const bool mine = lane < nb;
+      const bool valid = mine && pb >= 0 && pb < p.num_blocks;
+      if (mine && !valid) atomicOr(p.status, PA_DEVERR_TABLE);
+      const unsigned vmask = __ballot_sync(FULL, valid);
+      const uint32_t bytes = __popc(vmask) * 2u * static_cast<uint32_t>(bs) * 128u;
+      const int y = valid ? pb * row_stride + g * bs : 0;
+      for (int kv = 0; kv < 2; ++kv) {                   // 0: K, 1: V
+        const int u = 2 * i + kv;
+        const int s = u % SLOTS;
+        if (u >= SLOTS && !mbar_wait(&ring_empty[s], ((u / SLOTS) - 1) & 1, p.status)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) mbar_arrive_expect_tx(&ring_full[s], bytes);
+        __syncwarp();
+        if (valid) {
+          uint8_t* dst = ring + s * SLOT_BYTES + lane * bs * 128;
+          const CUtensorMap* map = kv == 0 ? &tmap_k : &tmap_v;
+          tma_load_2d(dst, map, 0, y, &ring_full[s]);
+          tma_load_2d(dst + HALF_BYTES, map, 64, y, &ring_full[s]);
+        }
+        issued = u + 1;
+      }
+    }
+    if (!ok) {
+      for (int u = issued - SLOTS < 0 ? 0 : issued - SLOTS; u < issued; ++u)
+        mbar_wait(&ring_full[u % SLOTS], (u / SLOTS) & 1, p.status);
+    }
+    return;
+  }
+
+  if (warp == 1) {
+    // ================= MMA issuer =================
+    if (lane == 0) {
+      const uint32_t id_qk = instr_desc<T>(false);
+      const uint32_t id_pv = instr_desc<T>(true);
+      const uint32_t ring_a = smem_addr(ring), q_a = smem_addr(qop), p_a = smem_addr(pop);
+      bool ok = true;
+      auto issue_qk = [&](int i) -> bool {
+        const int u = 2 * i, s = u % SLOTS;
+        if (!mbar_wait(&ring_full[s], (u / SLOTS) & 1, p.status)) return false;
+        if (i >= 2 && !mbar_wait(&s_free[i & 1], ((i >> 1) - 1) & 1, p.status)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + (i & 1) * NPAD;
+#pragma unroll
+        for (int k = 0; k < DH / 16; ++k) {
+          const uint32_t koff = (k >> 2) * HALF_BYTES + (k & 3) * 32;
+          const uint64_t a = smem_desc(ring_a + s * SLOT_BYTES + koff, 16, 1024);
+          const uint64_t bq = smem_desc(q_a + (k >> 2) * (NPAD * 128) + (k & 3) * 32, 16, 1024);
+          mma_f16(d, a, bq, id_qk, k > 0);
+        }
+        mma_commit(&s_full[i & 1]);
+        mma_commit(&ring_empty[s]);
+        return true;
+      };
+      auto issue_pv = [&](int i) -> bool {
+        const int u = 2 * i + 1, s = u % SLOTS;
+        if (!mbar_wait(&ring_full[s], (u / SLOTS) & 1, p.status)) return false;
+        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, p.status)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + 2 * NPAD;
+#pragma unroll
+        for (int k = 0; k < TOK / 16; ++k) {
+          const uint64_t a = smem_desc(ring_a + s * SLOT_BYTES + k * 2048, HALF_BYTES, 1024);
+          const uint64_t bp =
+              smem_desc(p_a + (i & 1) * OPB_BYTES + (k >> 2) * (NPAD * 128) + (k & 3) * 32, 16, 1024);
+          mma_f16(d, a, bp, id_pv, (i > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(&ring_empty[s]);
+        mma_commit(&p_free[i & 1]);
+        return true;
+      };
+      ok = issue_qk(0);
+      for (int i = 0; i < n_tiles && ok; ++i) {
+        if (i + 1 < n_tiles) ok = issue_qk(i + 1);
+        if (ok) ok = issue_pv(i);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ================= softmax warps =================
+    const int quad = warp & 3;                 // TMEM lane quadrant of this warp
+    const int r = quad * 32 + lane;            // token row of the tile / dim row of O
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    float m_run[G], l_part[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      m_run[h] = -INFINITY;
+      l_part[h] = 0.f;
+    }
+    // A failed (timed-out) wait makes `ok` false for the whole warp; later waits
+    // are then skipped, but every named barrier is still joined so the four
+    // softmax warps never wait on each other forever.
+    bool ok = true;
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+      if (ok) ok = mbar_wait(bar, parity, p.status);
+      ok = __all_sync(FULL, ok);
+      return ok;
+    };
+    for (int i = 0; i < n_tiles; ++i) {
+      const int n_valid = min(TOK, end - (start + i * TOK));
+      const bool valid = r < n_valid;
+      float sv[16];
+      if (wait(&s_full[i & 1], (i >> 1) & 1)) {
+        tc_fence_after();
+        tmem_ld16(tmem + lane_base + (i & 1) * NPAD, sv);
+      } else {
+#pragma unroll
+        for (int h = 0; h < 16; ++h) sv[h] = 0.f;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[i & 1]);
+      float s[G];
+      bool need = false;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        s[h] = valid ? sv[h] * p.scale_log2 : -INFINITY;
+        need |= s[h] > m_run[h] + RESCALE_THRESHOLD;
+      }
+      if (bar_or(1, 128, need)) {
+        // raise the running max to this tile's max (all 128 threads agree)
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float x = s[h];
+#pragma unroll
+          for (int off = 16; off >= 1; off >>= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, off));
+          if (lane == 0) red[quad * NPAD + h] = x;
+        }
+        named_sync(1, 128);
+        float alpha[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float tmax =
+              fmaxf(fmaxf(red[h], red[NPAD + h]), fmaxf(red[2 * NPAD + h], red[3 * NPAD + h]));
+          const float mnew = fmaxf(m_run[h], tmax);
+          alpha[h] = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - mnew);
+          m_run[h] = mnew;
+          l_part[h] *= alpha[h];
+        }
+        named_sync(1, 128);
+        // O must hold every earlier tile before it is rescaled
+        if (i > 0 && wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
+          tc_fence_after();
+          float o[16];
+          tmem_ld16(tmem + lane_base + 2 * NPAD, o);
+#pragma unroll
+          for (int h = 0; h < G; ++h) o[h] *= alpha[h];
+          tmem_st16(tmem + lane_base + 2 * NPAD, o);
+        }
+      }
+      float pr[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        pr[h] = valid ? exp2f(s[h] - m_run[h]) : 0.f;
+        l_part[h] += pr[h];
+      }
+      if (i >= 2) wait(&p_free[i & 1], ((i >> 1) - 1) & 1);
+      uint8_t* pb = pop + (i & 1) * OPB_BYTES + (r >> 6) * (NPAD * 128);
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+        *reinterpret_cast<uint16_t*>(pb + sw128(h, r & 63)) = to_bits<T>(pr[h]);
+      if (n_valid < TOK) {
+        // the last tile: zero the V rows of tokens past the end, so that
+        // whatever they hold (unused slots, stale data) adds 0 * 0 to O
+        const int u = 2 * i + 1, s_ = u % SLOTS;
+        if (wait(&ring_full[s_], (u / SLOTS) & 1) && !valid) {
+          uint8_t* row = ring + s_ * SLOT_BYTES + r * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            *reinterpret_cast<uint4*>(row + c * 16) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(row + HALF_BYTES + c * 16) = make_uint4(0, 0, 0, 0);
+          }
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[i & 1]);
+    }
+    // ---- epilogue: row r of O^T (dim r, all heads) and the sums ----
+    wait(&p_free[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1);
+    tc_fence_after();
+    float o[16];
+    tmem_ld16(tmem + lane_base + 2 * NPAD, o);
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float x = l_part[h];
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(FULL, x, off);
+      l_part[h] = x;
+    }
+    named_sync(1, 128);
+    if (lane == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) red[quad * NPAD + h] = l_part[h];
+    }
+    named_sync(1, 128);
+    if (ok) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float Ls = red[h] + red[NPAD + h] + red[2 * NPAD + h] + red[3 * NPAD + h];
+        const int64_t hq = static_cast<int64_t>(b) * p.Hq + g * G + h;
+        if (single) {
+          static_cast<T*>(p.out)[hq * DH + r] = Elem<T>::from_float(o[h] / Ls);
+        } else {
+          const int64_t slot = hq * p.num_partitions + part;
+          p.ws_o[slot * DH + r] = o[h];
+          if (r == 0) {
+            p.ws_m[slot] = m_run[h];
+            p.ws_l[slot] = Ls;
+          }
+        }
+      }
+    }
+  }
+
+  // ---- teardown: warps 1-5 meet, warp 1 frees TMEM ----
+  tc_fence_before();
+  named_sync(2, 160);
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---- host side ----
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// The cache [NB][Hkv][bs][128] seen as a 2-D tensor of NB*Hkv*bs rows of 128
+// elements; a box is bs rows x 64 elements, stored with the 128-byte swizzle.
+bool make_cache_map(CUtensorMap* map, const void* base, int64_t rows, int bs, pa_dtype dt) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(DH), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(DH * 2)};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(bs)};
+  cuuint32_t estr[2] = {1u, 1u};
+  const CUtensorMapDataType t =
+      dt == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  return fn(map, t, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T, int G>
+cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
+  auto kern = decode_partition_tc_kernel<T, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  CUtensorMap mk, mv;
+  const int64_t rows = static_cast<int64_t>(a.num_blocks) * a.Hkv * a.block_size;
+  if (!make_cache_map(&mk, a.k_cache, rows, a.block_size, a.dtype) ||
+      !make_cache_map(&mv, a.v_cache, rows, a.block_size, a.dtype))
+    return cudaErrorInvalidValue;
+  TcParams p;
+  p.out = a.out;
+  p.q = a.q;
+  p.block_tables = a.block_tables;
+  p.context_lens = a.context_lens;
+  const int64_t nrows = static_cast<int64_t>(a.num_seqs) * a.Hq * a.num_partitions;
+  p.ws_o = a.workspace;
+  p.ws_m = a.workspace ? a.workspace + nrows * DH : nullptr;
+  p.ws_l = a.workspace ? a.workspace + nrows * (DH + 1) : nullptr;
+  p.status = status;
+  p.max_blocks = a.max_blocks;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.num_blocks = a.num_blocks;
+  p.block_size = a.block_size;
+  p.partition_size = a.partition_size;
+  p.num_partitions = a.num_partitions;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  dim3 grid(a.num_seqs, a.Hkv, a.num_partitions);
+  kern<<<grid, THREADS, SMEM_BYTES, stream>>>(p, mk, mv);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool decode_tc_supported(const DecodeArgs& a) {
+  const int G = a.Hq / a.Hkv;
+  return (a.dtype == PA_F16 || a.dtype == PA_BF16) && a.D == DH && (G == 4 || G == 8) &&
+         a.partition_size % TOK == 0 &&
+         static_cast<int64_t>(a.num_blocks) * a.Hkv * a.block_size < (int64_t(1) << 31) &&
+         encode_fn() != nullptr;
+}
+
+int launch_decode_partitions_tc(const DecodeArgs& a, unsigned int* status, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int G = a.Hq / a.Hkv;
+  if (a.dtype == PA_BF16) {
+    return G == 8 ? launch_tc_t<__nv_bfloat16, 8>(a, status, st)
+                  : launch_tc_t<__nv_bfloat16, 4>(a, status, st);
+  }
+  return G == 8 ? launch_tc_t<__half, 8>(a, status, st) : launch_tc_t<__half, 4>(a, status, st);
+}
+
+}  // namespace pa

@@ -57,6 +57,10 @@ struct DecodeArgs {
 // Kernel launchers (kernels.cu).  They return cudaError_t as int.
 int launch_decode_partitions(const DecodeArgs& a, unsigned int* status, void* stream);
 int launch_decode_reduce(const DecodeArgs& a, unsigned int* status, void* stream);
+// Tensor-core partition kernel (decode_tc.cu): fp16/bf16, head size 128, 4 or 8
+// query heads per kv head, partition length a multiple of 128.
+bool decode_tc_supported(const DecodeArgs& a);
+int launch_decode_partitions_tc(const DecodeArgs& a, unsigned int* status, void* stream);
 int launch_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
                              const int64_t* slot_mapping, int num_tokens, int Hkv, int D,
                              int block_size, int num_blocks, int esize, unsigned int* status,

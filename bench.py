@@ -47,6 +47,12 @@ FALLBACK_HBM_GBS = 6650.0
 
 
 def workload_spec(name):
+    if name.endswith("_quarter"):
+        # a quarter of the sequences of a workload (same kernel, same per-sequence
+        # shapes): the profiling case for captures that must stay small
+        from dataclasses import replace
+        base = workload_spec(name[: -len("_quarter")])
+        return replace(base, name=name, num_seqs=max(1, base.num_seqs // 4))
     if name == "opt13b_compact":
         # the opt13b launch with a pool of 1.25x the blocks it needs (about 1 GB
         # on the device instead of 6.6): the profiling case
@@ -69,6 +75,8 @@ WORKLOAD_TEXT = {
 
 
 def workload_text(name):
+    if name.endswith("_quarter"):
+        return workload_text(name[: -len("_quarter")]) + " (a quarter of the sequences)"
     if name == "opt13b_compact":
         return WORKLOAD_TEXT["opt13b"].replace("20,000-block pool", "pool of 1.25x the blocks needed")
     base = name.split("_bs")[0] if name.startswith("long_prefix") else name
@@ -381,7 +389,7 @@ def run_ours(args):
     tables, lens, max_ctx = cache.tables(sc.batch, sc.max_blocks)
     q = W.q_content(spec, len(sc.batch), device)
     out = torch.empty_like(q)
-    P = spec.partition_size
+    P = args.partition_size if args.partition_size else spec.partition_size
     ws = cache.workspace(q.shape[0], q.shape[1], max_ctx, P)
     scale = spec.softmax_scale
     n_part = pk.pa_decode_num_partitions(max_ctx, P)
@@ -561,7 +569,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=["tiny", "opt13b", "opt13b_compact", "llama13b_ps", "gqa70b",
-                             "long_prefix_bs8", "long_prefix_bs16", "long_prefix_bs32"])
+                             "long_prefix_bs8", "long_prefix_bs16", "long_prefix_bs32",
+                             "gqa70b_quarter", "long_prefix_bs8_quarter",
+                             "long_prefix_bs16_quarter"])
+    ap.add_argument("--partition-size", type=int, default=0,
+                    help="split-K partition length (0: the workload's own, 512)")
     ap.add_argument("--soak-seconds", type=float, default=0.5,
                     help="untimed load before the timed steps (clock samples)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

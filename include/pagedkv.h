@@ -105,7 +105,8 @@ int pa_decode_num_partitions(int max_context_len, int partition_size);
 
 /*
  * Bytes of scratch `workspace` pa_decode needs: 0 when every sequence fits one
- * partition, else B * Hq * num_partitions * (D + 2) * 4 rounded up to 256.
+ * partition, else B * Hq * num_partitions * (D + 2) * 4 rounded up to 256 (the
+ * split-K partials).
  */
 size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_size, int max_context_len,
                                  int partition_size);
@@ -136,9 +137,13 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_size, int
  *                 the workspace)
  *   workspace     device scratch of at least pa_decode_workspace_bytes(...)
  *                 bytes, 16-byte aligned; may be NULL when that is 0.  Its
- *                 contents need no initialisation and are clobbered.
+ *                 contents need no initialisation and are clobbered; calls
+ *                 that share a workspace must not overlap on the GPU.
  *
  * Precision: products and sums in fp32; the result is rounded to dtype once.
+ * With 4 or 8 query heads per kv head in fp16/bf16 (head size 128, partition a
+ * multiple of 128) the products run on the tensor cores, whose operands share
+ * one type: the probabilities are rounded to dtype before they weight V.
  * Exactly pa_decode_partitions followed (when the workspace size is not 0) by
  * pa_decode_reduce on the same stream.
  */

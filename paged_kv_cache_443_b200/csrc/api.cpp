@@ -124,8 +124,8 @@ pa_status check_decode_full(const char* fn, void* out, const void* q, const void
 }
 
 int launch_partitions(const pa::DecodeArgs& a, unsigned int* status, void* stream) {
-  return pa::decode_tc_supported(a) ? pa::launch_decode_partitions_tc(a, status, stream)
-                                    : pa::launch_decode_partitions(a, status, stream);
+  if (pa::decode_tc_supported(a)) return pa::launch_decode_partitions_tc(a, status, stream);
+  return pa::launch_decode_partitions(a, status, stream);
 }
 
 pa_status launch_status(const char* fn, int err, int n_launched) {

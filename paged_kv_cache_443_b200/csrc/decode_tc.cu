@@ -38,10 +38,13 @@
 
 #include "pa_device.cuh"
 #include "pa_internal.h"
+#include "tc_common.cuh"
 
 namespace pa {
 
 namespace {
+
+using namespace tc;
 
 constexpr unsigned FULL = 0xffffffffu;
 constexpr int TOK = 128;                     // tokens per tile (M of the first MMA)
@@ -55,7 +58,7 @@ constexpr int OFF_RING = 0;
 constexpr int OFF_Q = OFF_RING + SLOTS * SLOT_BYTES;
 constexpr int OFF_P = OFF_Q + OPB_BYTES;     // two P buffers
 constexpr int OFF_BAR = OFF_P + 2 * OPB_BYTES;
-constexpr int NBARS = 2 * SLOTS + 8;         // ring full/empty, s_full/s_free, p_full/p_free
+constexpr int NBARS = 2 * SLOTS + 9;         // ring full/empty, s/p full/free, q_ready
 constexpr int OFF_TMEM = OFF_BAR + NBARS * 8;
 constexpr int OFF_RED = OFF_TMEM + 16;       // 4 warps x 16 floats
 constexpr int SMEM_USED = OFF_RED + 4 * NPAD * 4;
@@ -80,110 +83,6 @@ struct TcParams {
   float scale_log2;
 };
 
-// ---- tcgen05 / TMA helpers ----
-
-// Byte offset of element (row, col) of a [rows x 64] 16-bit operand block stored
-// with the 128-byte swizzle (16-byte chunk index XOR row % 8).
-__device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t col) {
-  return row * 128u + ((((col >> 3) ^ (row & 7u)) & 7u) << 4) + (col & 7u) * 2u;
-}
-
-// Shared-memory matrix descriptor (sm_100): start, leading / stride byte
-// offsets (16-byte units), version 1, 128-byte swizzle.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-// Instruction descriptor of kind::f16 with fp32 accumulation, M = 128, N = 16.
-template <typename T>
-__device__ __forceinline__ constexpr uint32_t instr_desc(bool a_mn_major) {
-  constexpr uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
-  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((a_mn_major ? 1u : 0u) << 15) |
-         ((uint32_t)(NPAD >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_addr(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, "
-      "[%16];\n\ttcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
-      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-      "r"(__float_as_uint(v[15]))
-      : "memory");
-}
-
-// 2-D TMA tile load (this GPU's memory, no multicast) completing on `bar`.
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
-      "%4}], [%2];" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y)
-      : "memory");
-}
-
-// OR of `pred` over the `n` threads reaching named barrier `id`.
-__device__ __forceinline__ bool bar_or(int id, int n, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id), "r"(n)
-      : "memory");
-  return r != 0;
-}
-
-template <typename T>
-__device__ __forceinline__ uint16_t to_bits(float x) {
-  T h = Elem<T>::from_float(x);
-  return *reinterpret_cast<uint16_t*>(&h);
-}
-
 template <typename T, int G>
 __global__ void __launch_bounds__(THREADS, 2)
     decode_partition_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmap_k,
@@ -201,6 +100,7 @@ __global__ void __launch_bounds__(THREADS, 2)
   uint64_t* s_free = s_full + 2;            // [2]
   uint64_t* p_full = s_free + 2;            // [2]
   uint64_t* p_free = p_full + 2;            // [2]
+  uint64_t* q_ready = p_free + 2;           // Q^T operand staged
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
   float* red = reinterpret_cast<float*>(smem + OFF_RED);
 
@@ -229,21 +129,32 @@ __global__ void __launch_bounds__(THREADS, 2)
   const int n_tiles = (end - start + TOK - 1) / TOK;
   const bool single = (L <= P);
 
-  // ---- set-up ----
-  if (warp == 0 && lane == 0) {
-    for (int s = 0; s < SLOTS; ++s) {
-      mbar_init(&ring_full[s], 1);
-      mbar_init(&ring_empty[s], 1);
+  // ---- set-up: the producer starts streaming right after the barrier, while
+  // the softmax warps stage Q^T and the MMA issuer waits for it ----
+  const int bs = p.block_size;
+  const int bpt = TOK / bs;                              // blocks per tile: 4, 8 or 16
+  const int first_blk = start / bs;
+  const int last_blk = (end + bs - 1) / bs;
+  const int32_t* trow = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
+  int pb_first = -1;                                     // tile 0's table entries, read early
+  if (warp == 0) {
+    if (lane < min(bpt, last_blk - first_blk)) pb_first = __ldg(trow + first_blk + lane);
+    if (lane == 0) {
+      for (int s = 0; s < SLOTS; ++s) {
+        mbar_init(&ring_full[s], 1);
+        mbar_init(&ring_empty[s], 1);
+      }
+      for (int j = 0; j < 2; ++j) {
+        mbar_init(&s_full[j], 1);
+        mbar_init(&s_free[j], 4);
+        mbar_init(&p_full[j], 4);
+        mbar_init(&p_free[j], 1);
+      }
+      mbar_init(q_ready, 4);
+      fence_mbar_init();
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
     }
-    for (int j = 0; j < 2; ++j) {
-      mbar_init(&s_full[j], 1);
-      mbar_init(&s_free[j], 4);
-      mbar_init(&p_full[j], 4);
-      mbar_init(&p_free[j], 1);
-    }
-    fence_mbar_init();
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -252,6 +163,10 @@ __global__ void __launch_bounds__(THREADS, 2)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
   if (warp >= 2) {
     // Q^T operand (16 rows = heads, 128 columns = dims, two swizzled 64-column
     // blocks), rows >= G zero; both P buffers zeroed (their rows >= G stay 0).
@@ -268,27 +183,20 @@ __global__ void __launch_bounds__(THREADS, 2)
     for (int i = t; i < 2 * OPB_BYTES / 16; i += 128)
       reinterpret_cast<uint4*>(pop)[i] = make_uint4(0, 0, 0, 0);
     fence_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(q_ready);
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
     // ================= producer =================
-    const int bs = p.block_size;
-    const int bpt = TOK / bs;                            // blocks per tile: 4, 8 or 16
-    const int first_blk = start / bs;
-    const int last_blk = (end + bs - 1) / bs;
-    const int32_t* trow = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
     const int row_stride = p.Hkv * bs;                   // rows of one physical block
     bool ok = true;
     int issued = 0;
     for (int i = 0; i < n_tiles && ok; ++i) {
       const int b0 = first_blk + i * bpt;
       const int nb = min(bpt, last_blk - b0);
-      int pb = -1;
-      if (lane < nb) pb = __ldg(trow + b0 + lane);
+      int pb = pb_first;
+      if (i > 0) pb = lane < nb ? __ldg(trow + b0 + lane) : -1;
       const bool mine = lane < nb;
       const bool valid = mine && pb >= 0 && pb < p.num_blocks;
       if (mine && !valid) atomicOr(p.status, PA_DEVERR_TABLE);
@@ -361,7 +269,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         mma_commit(&p_free[i & 1]);
         return true;
       };
-      ok = issue_qk(0);
+      ok = mbar_wait(q_ready, 0, p.status) && issue_qk(0);
       for (int i = 0; i < n_tiles && ok; ++i) {
         if (i + 1 < n_tiles) ok = issue_qk(i + 1);
         if (ok) ok = issue_pv(i);
@@ -519,45 +427,17 @@ __global__ void __launch_bounds__(THREADS, 2)
 
 // ---- host side ----
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  });
-  return fn;
-}
-
-// The cache [NB][Hkv][bs][128] seen as a 2-D tensor of NB*Hkv*bs rows of 128
-// elements; a box is bs rows x 64 elements, stored with the 128-byte swizzle.
-bool make_cache_map(CUtensorMap* map, const void* base, int64_t rows, int bs, pa_dtype dt) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(DH), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(DH * 2)};
-  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(bs)};
-  cuuint32_t estr[2] = {1u, 1u};
-  const CUtensorMapDataType t =
-      dt == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  return fn(map, t, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <typename T, int G>
 cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
   auto kern = decode_partition_tc_kernel<T, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
+  // the cache [NB][Hkv][bs][128] as a 2-D tensor of NB*Hkv*bs rows of 128
+  // elements; a box is bs rows x 64 elements, stored with the 128-byte swizzle
   CUtensorMap mk, mv;
   const int64_t rows = static_cast<int64_t>(a.num_blocks) * a.Hkv * a.block_size;
-  if (!make_cache_map(&mk, a.k_cache, rows, a.block_size, a.dtype) ||
-      !make_cache_map(&mv, a.v_cache, rows, a.block_size, a.dtype))
+  if (!make_tmap_2d(&mk, a.k_cache, DH, rows, DH * 2, 64, a.block_size, a.dtype) ||
+      !make_tmap_2d(&mv, a.v_cache, DH, rows, DH * 2, 64, a.block_size, a.dtype))
     return cudaErrorInvalidValue;
   TcParams p;
   p.out = a.out;
@@ -583,6 +463,37 @@ cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t 
 }
 
 }  // namespace
+
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+}  // namespace
+
+bool make_tmap_2d(void* map, const void* base, int64_t inner, int64_t rows, int64_t row_stride_bytes,
+                  int box_inner, int box_rows, pa_dtype dt) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride_bytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  const CUtensorMapDataType t =
+      dt == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  return fn(static_cast<CUtensorMap*>(map), t, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 bool decode_tc_supported(const DecodeArgs& a) {
   const int G = a.Hq / a.Hkv;

@@ -1,0 +1,85 @@
+"""Host logic of bench.py on CPU: the multi-rank plumbing (world size 2, gloo)
+and the algorithmic byte accounting of a step."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+import workloads as W
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    r, w, lr = bench.dist_env()
+    dist = bench.dist_init(w, "gloo")
+    # each rank a replica of the workload with its own seed (weak scaling)
+    spec = bench.rank_spec(W.small("opt13b"), r)
+    sc = W.scenario(spec)
+    t_ms = 1.0 + r                     # per-rank step time
+    units = float(sc.context_lens.sum())
+    bench.barrier(w)
+    tmax = bench.reduce_max(t_ms, w)
+    usum = bench.reduce_sum(units, w)
+    q.put((r, spec.seed, tmax, usum, units))
+    dist.destroy_process_group()
+
+
+def test_two_rank_replicas_reduce_max_time_and_sum_units():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    seeds = {r[1] for r in res}
+    assert len(seeds) == world                 # replicas draw different batches
+    for r in res:
+        assert r[2] == 2.0                     # max over ranks of 1.0, 2.0
+        assert r[3] == pytest.approx(res[0][4] + res[1][4])
+
+
+def test_single_rank_helpers_are_identity():
+    assert bench.reduce_max(3.5, 1) == 3.5
+    assert bench.reduce_sum(2.0, 1) == 2.0
+    assert bench.rank_spec(W.TINY, 0) is W.TINY
+
+
+def test_step_bytes_unique_and_logical():
+    spec = W.Spec("t", "bf16", 8, 2, 128, 16, "independent", 3, seed=1)
+    # two sequences share their first block (id 5); the third is separate
+    tables = np.array([[5, 6], [5, 7], [9, -1]], dtype=np.int32)
+    lens = np.array([20, 18, 16], dtype=np.int32)
+    unique, logical, other = bench.step_bytes(spec, tables, lens)
+    row = 2 * 2 * 128 * 2                      # K and V, 2 kv heads, D 128, bf16
+    assert logical == (20 + 18 + 16) * row
+    assert unique == (16 + 4 + 2 + 16) * row   # block 5 once, 6: 4 tokens, 7: 2, 9: 16
+    assert other == 2 * 3 * 8 * 128 * 2 + (2 + 2 + 1) * 4 + 3 * 4
+
+
+def test_profile_digest_gates_traffic(tmp_path, monkeypatch):
+    d = bench.source_digest()
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "decode_partition_x.md").write_text(f"traffic_bytes_per_launch: 123\nsource_digest: {d}\n")
+    (prof / "decode_partition_y.md").write_text("traffic_bytes_per_launch: 123\nsource_digest: 0000\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    # the digest is computed from the sources under ROOT; point it back at the repo
+    monkeypatch.setattr(bench, "source_digest", lambda: d)
+    assert bench.profiled_traffic("x") == 123.0
+    assert bench.profiled_traffic("y") is None
+    assert bench.profiled_traffic("z") is None

@@ -13,9 +13,13 @@
 //   O^T [128 dims   x 16] += V^T [128 x 128] . P^T [128 x 16]
 //
 // Roles in a CTA of 6 warps, one CTA per (sequence, kv head, partition):
-//   warp 0   producer: block-table lookups, 2-D TMA loads (128-byte swizzle) of
-//            every physical block's K and V rows into a ring of three 32 KB slots
-//            holding K_0, V_0, K_1, V_1, ... (two boxes of 64 columns per block);
+//   warp 0   producer: block-table lookups, one TMA load per physical block of
+//            its K (or V) rows into a ring of three 32 KB slots holding K_0, V_0,
+//            K_1, V_1, ...  The cache is viewed as a 4-D tensor (64 columns, 8
+//            rows, 2 column halves, 8-row groups), so a block lands as
+//            [8-row group][half][8 rows x 128 B] with the 128-byte swizzle: the
+//            canonical K-major layout of K and MN-major layout of V^T, with
+//            8-row groups 2 KB apart and halves 1 KB apart;
 //   warp 1   TMEM owner and MMA issuer (one thread): S = K Q^T into one of two
 //            TMEM score buffers, O += V^T P^T into the TMEM output buffer;
 //   warps 2-5  softmax: each thread owns one token row of S (its TMEM lane),
@@ -51,8 +55,9 @@ constexpr int TOK = 128;                     // tokens per tile (M of the first 
 constexpr int NPAD = 16;                     // N of both MMAs (heads padded)
 constexpr int DH = 128;                      // head size
 constexpr int SLOTS = 3;                     // ring slots (K or V of one tile each)
-constexpr int HALF_BYTES = TOK * 128;        // 128 rows x 64 elements x 2 B
-constexpr int SLOT_BYTES = 2 * HALF_BYTES;   // 32 KB
+constexpr int SLOT_BYTES = TOK * 256;        // one tile of K (or V): 32 KB
+constexpr int GROUP_BYTES = 2048;            // 8 token rows, both 64-column halves
+constexpr int HALF_OFF = 1024;               // second 64-column half of a group
 constexpr int OPB_BYTES = 2 * NPAD * 128;    // a 16-row operand in two 64-column blocks: 4 KB
 constexpr int OFF_RING = 0;
 constexpr int OFF_Q = OFF_RING + SLOTS * SLOT_BYTES;
@@ -202,7 +207,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       if (mine && !valid) atomicOr(p.status, PA_DEVERR_TABLE);
       const unsigned vmask = __ballot_sync(FULL, valid);
       const uint32_t bytes = __popc(vmask) * 2u * static_cast<uint32_t>(bs) * 128u;
-      const int y = valid ? pb * row_stride + g * bs : 0;
+      const int grp = valid ? (pb * row_stride + g * bs) / 8 : 0;   // first 8-row group
       for (int kv = 0; kv < 2; ++kv) {                   // 0: K, 1: V
         const int u = 2 * i + kv;
         const int s = u % SLOTS;
@@ -213,10 +218,9 @@ __global__ void __launch_bounds__(THREADS, 2)
         if (lane == 0) mbar_arrive_expect_tx(&ring_full[s], bytes);
         __syncwarp();
         if (valid) {
-          uint8_t* dst = ring + s * SLOT_BYTES + lane * bs * 128;
+          uint8_t* dst = ring + s * SLOT_BYTES + lane * bs * 256;
           const CUtensorMap* map = kv == 0 ? &tmap_k : &tmap_v;
-          tma_load_2d(dst, map, 0, y, &ring_full[s]);
-          tma_load_2d(dst + HALF_BYTES, map, 64, y, &ring_full[s]);
+          tma_load_4d(dst, map, 0, 0, 0, grp, &ring_full[s]);
         }
         issued = u + 1;
       }
@@ -243,8 +247,8 @@ __global__ void __launch_bounds__(THREADS, 2)
         const uint32_t d = tmem + (i & 1) * NPAD;
 #pragma unroll
         for (int k = 0; k < DH / 16; ++k) {
-          const uint32_t koff = (k >> 2) * HALF_BYTES + (k & 3) * 32;
-          const uint64_t a = smem_desc(ring_a + s * SLOT_BYTES + koff, 16, 1024);
+          const uint32_t koff = (k >> 2) * HALF_OFF + (k & 3) * 32;
+          const uint64_t a = smem_desc(ring_a + s * SLOT_BYTES + koff, 16, GROUP_BYTES);
           const uint64_t bq = smem_desc(q_a + (k >> 2) * (NPAD * 128) + (k & 3) * 32, 16, 1024);
           mma_f16(d, a, bq, id_qk, k > 0);
         }
@@ -260,7 +264,8 @@ __global__ void __launch_bounds__(THREADS, 2)
         const uint32_t d = tmem + 2 * NPAD;
 #pragma unroll
         for (int k = 0; k < TOK / 16; ++k) {
-          const uint64_t a = smem_desc(ring_a + s * SLOT_BYTES + k * 2048, HALF_BYTES, 1024);
+          const uint64_t a =
+              smem_desc(ring_a + s * SLOT_BYTES + k * 2 * GROUP_BYTES, HALF_OFF, GROUP_BYTES);
           const uint64_t bp =
               smem_desc(p_a + (i & 1) * OPB_BYTES + (k >> 2) * (NPAD * 128) + (k & 3) * 32, 16, 1024);
           mma_f16(d, a, bp, id_pv, (i > 0 || k > 0) ? 1u : 0u);
@@ -364,11 +369,11 @@ __global__ void __launch_bounds__(THREADS, 2)
         // whatever they hold (unused slots, stale data) adds 0 * 0 to O
         const int u = 2 * i + 1, s_ = u % SLOTS;
         if (wait(&ring_full[s_], (u / SLOTS) & 1) && !valid) {
-          uint8_t* row = ring + s_ * SLOT_BYTES + r * 128;
+          uint8_t* row = ring + s_ * SLOT_BYTES + (r >> 3) * GROUP_BYTES + (r & 7) * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             *reinterpret_cast<uint4*>(row + c * 16) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(row + HALF_BYTES + c * 16) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(row + HALF_OFF + c * 16) = make_uint4(0, 0, 0, 0);
           }
         }
       }
@@ -432,12 +437,16 @@ cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t 
   auto kern = decode_partition_tc_kernel<T, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  // the cache [NB][Hkv][bs][128] as a 2-D tensor of NB*Hkv*bs rows of 128
-  // elements; a box is bs rows x 64 elements, stored with the 128-byte swizzle
+  // the cache [NB][Hkv][bs][128] as a 4-D tensor: 64 columns (stride 2 B),
+  // 8 rows (256 B), 2 column halves (128 B), NB*Hkv*bs/8 row groups (2 KB); a
+  // box is one physical block: 64 x 8 x 2 x bs/8, stored with the 128-byte swizzle
   CUtensorMap mk, mv;
-  const int64_t rows = static_cast<int64_t>(a.num_blocks) * a.Hkv * a.block_size;
-  if (!make_tmap_2d(&mk, a.k_cache, DH, rows, DH * 2, 64, a.block_size, a.dtype) ||
-      !make_tmap_2d(&mv, a.v_cache, DH, rows, DH * 2, 64, a.block_size, a.dtype))
+  const int64_t groups = static_cast<int64_t>(a.num_blocks) * a.Hkv * a.block_size / 8;
+  const int64_t dims[4] = {64, 8, 2, groups};
+  const int64_t strides[3] = {DH * 2, 128, 8 * DH * 2};
+  const int box[4] = {64, 8, 2, a.block_size / 8};
+  if (!make_tmap(&mk, a.k_cache, 4, dims, strides, box, a.dtype) ||
+      !make_tmap(&mv, a.v_cache, 4, dims, strides, box, a.dtype))
     return cudaErrorInvalidValue;
   TcParams p;
   p.out = a.out;
@@ -480,19 +489,24 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 }  // namespace
 
-bool make_tmap_2d(void* map, const void* base, int64_t inner, int64_t rows, int64_t row_stride_bytes,
-                  int box_inner, int box_rows, pa_dtype dt) {
+bool make_tmap(void* map, const void* base, int rank, const int64_t* dims,
+               const int64_t* strides_bytes, const int* box, pa_dtype dt) {
   auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride_bytes)};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows)};
-  cuuint32_t estr[2] = {1u, 1u};
+  if (!fn || rank < 1 || rank > 5) return false;
+  cuuint64_t gdim[5], gstride[4];
+  cuuint32_t bdim[5], estr[5];
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = static_cast<cuuint64_t>(dims[i]);
+    bdim[i] = static_cast<cuuint32_t>(box[i]);
+    estr[i] = 1u;
+    if (i + 1 < rank) gstride[i] = static_cast<cuuint64_t>(strides_bytes[i]);
+  }
   const CUtensorMapDataType t =
       dt == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  return fn(static_cast<CUtensorMap*>(map), t, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(static_cast<CUtensorMap*>(map), t, static_cast<cuuint32_t>(rank),
+            const_cast<void*>(base), gdim, gstride, bdim, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool decode_tc_supported(const DecodeArgs& a) {

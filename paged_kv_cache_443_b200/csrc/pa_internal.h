@@ -61,10 +61,11 @@ int launch_decode_reduce(const DecodeArgs& a, unsigned int* status, void* stream
 // query heads per kv head, partition length a multiple of 128.
 bool decode_tc_supported(const DecodeArgs& a);
 int launch_decode_partitions_tc(const DecodeArgs& a, unsigned int* status, void* stream);
-// A 2-D TMA tensor map (128-byte swizzle, 16-bit elements) over `rows` rows of
-// `inner` elements; `map` points at a CUtensorMap.  False if encoding fails.
-bool make_tmap_2d(void* map, const void* base, int64_t inner, int64_t rows, int64_t row_stride_bytes,
-                  int box_inner, int box_rows, pa_dtype dt);
+// A TMA tensor map of 16-bit elements with the 128-byte swizzle: `rank` dims
+// (innermost first), byte strides of dims 1..rank-1, a box; `map` points at a
+// CUtensorMap.  False if encoding fails.
+bool make_tmap(void* map, const void* base, int rank, const int64_t* dims,
+               const int64_t* strides_bytes, const int* box, pa_dtype dt);
 
 int launch_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
                              const int64_t* slot_mapping, int num_tokens, int Hkv, int D,

@@ -235,24 +235,40 @@ def rank_spec(spec, rank):
 # profile summaries committed under profiles/ (dram traffic of the dominant kernel)
 
 
-def source_digest():
+KERNEL_SOURCES = {
+    "decode_partition_kernel": ("decode.cu", "pa_device.cuh", "pa_internal.h"),
+    "decode_partition_tc_kernel": ("decode_tc.cu", "tc_common.cuh", "pa_device.cuh", "pa_internal.h"),
+}
+
+
+def partition_kernel(spec, P):
+    """The decode-partition kernel the library picks for this launch: the
+    tensor-core one for 4 or 8 query heads per kv head in fp16/bf16, head size
+    128 and a partition length that is a multiple of 128; else CUDA cores."""
+    G = spec.Hq // spec.Hkv
+    if spec.dtype in ("f16", "bf16") and spec.D == 128 and G in (4, 8) and P % 128 == 0:
+        return "decode_partition_tc_kernel"
+    return "decode_partition_kernel"
+
+
+def source_digest(files=KERNEL_SOURCES["decode_partition_kernel"]):
     h = hashlib.sha256()
-    for f in ("decode.cu", "pa_device.cuh", "pa_internal.h"):
+    for f in files:
         with open(os.path.join(ROOT, "paged_kv_cache_443_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload):
+def profiled_traffic(workload, kernel="decode_partition_kernel"):
     """dram bytes per launch of the decode-partition kernel from the committed
-    ncu summary, if it was taken on the current kernel source; else None."""
+    ncu summary, if it was taken on the current source of that kernel; else None."""
     path = os.path.join(ROOT, "profiles", f"decode_partition_{workload}.md")
     if not os.path.exists(path):
         return None
     txt = open(path).read()
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.e+]+)", txt)
     s = re.search(r"source_digest:\s*([0-9a-f]+)", txt)
-    if not m or not s or s.group(1) != source_digest():
+    if not m or not s or s.group(1) != source_digest(KERNEL_SOURCES[kernel]):
         return None
     return float(m.group(1))
 
@@ -507,7 +523,8 @@ def run_ours(args):
     peak, peak_kind = measured_peak_hbm()
     alg = unique + other
     achieved = alg / (part_avg * 1e-3) / 1e9
-    traffic = profiled_traffic(args.workload)
+    kname = partition_kernel(spec, P)
+    traffic = profiled_traffic(args.workload, kname)
 
     result = None
     if rank == 0:
@@ -544,7 +561,7 @@ def run_ours(args):
                 "decode_reduce": round(float(np.mean(red_ms)) * 1e3, 3),
             },
             "roofline": {
-                "kernel": "decode_partition_kernel",
+                "kernel": kname,
                 "bound": "hbm",
                 "achieved": round(achieved, 1),
                 "peak": peak,

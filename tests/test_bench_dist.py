@@ -79,7 +79,15 @@ def test_profile_digest_gates_traffic(tmp_path, monkeypatch):
     (prof / "decode_partition_y.md").write_text("traffic_bytes_per_launch: 123\nsource_digest: 0000\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     # the digest is computed from the sources under ROOT; point it back at the repo
-    monkeypatch.setattr(bench, "source_digest", lambda: d)
+    monkeypatch.setattr(bench, "source_digest", lambda files=None: d)
     assert bench.profiled_traffic("x") == 123.0
     assert bench.profiled_traffic("y") is None
     assert bench.profiled_traffic("z") is None
+
+
+def test_partition_kernel_choice():
+    assert bench.partition_kernel(W.GQA70B, 512) == "decode_partition_tc_kernel"
+    assert bench.partition_kernel(W.LONG_PREFIX, 512) == "decode_partition_tc_kernel"
+    assert bench.partition_kernel(W.OPT13B, 512) == "decode_partition_kernel"
+    assert bench.partition_kernel(W.GQA70B, 96) == "decode_partition_kernel"
+    assert bench.partition_kernel(W.TINY, 512) == "decode_partition_kernel"

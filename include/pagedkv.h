@@ -97,6 +97,18 @@ pa_status pa_device_status(unsigned int* flags_out, int clear);
 int pa_decode_default_partition_size(void);
 
 /*
+ * The partition length pa_decode uses when it is given partition_size = 0
+ * (tokens; 512, 1024 or 2048).  With 4 or 8 query heads per kv head in
+ * fp16/bf16 and head size 128 (the tensor-core kernel) it is the longest of
+ * 2048 / 1024 that still gives num_seqs * num_kv_heads * ceil(max_context_len /
+ * P) >= 8 * (number of SMs) CTAs; otherwise the default.  Pass it explicitly to
+ * pa_decode_partitions / pa_decode_reduce to reproduce pa_decode's automatic
+ * choice.  Returns -1 for invalid arguments.
+ */
+int pa_decode_auto_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_size,
+                                  pa_dtype dtype, int max_context_len);
+
+/*
  * Number of split-K partitions per sequence for a batch whose longest context
  * is max_context_len: ceil(max_context_len / P), P = the partition size (0 =
  * default).  Returns -1 for an invalid partition size.
@@ -131,8 +143,9 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_size, int
  *                 last block are never read (any value, e.g. -1)
  *   context_lens  [B] int32, each in [0, max_context_len] and
  *                 <= max_blocks_per_seq * bs; a length of 0 gives a zero row
- *   partition_size  0 = default, else a multiple of 32 tokens: contexts longer
- *                 than this are split into partitions reduced by a second kernel
+ *   partition_size  0 = automatic (pa_decode_auto_partition_size), else a
+ *                 multiple of 32 tokens: contexts longer than this are split
+ *                 into partitions reduced by a second kernel
  *   max_context_len  an upper bound of context_lens (sizes the launch grid and
  *                 the workspace)
  *   workspace     device scratch of at least pa_decode_workspace_bytes(...)
@@ -140,12 +153,16 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_size, int
  *                 contents need no initialisation and are clobbered; calls
  *                 that share a workspace must not overlap on the GPU.
  *
+ * pa_decode_workspace_bytes(..., partition_size = 0, ...) bytes always suffice
+ * for the automatic length.
+ *
  * Precision: products and sums in fp32; the result is rounded to dtype once.
  * With 4 or 8 query heads per kv head in fp16/bf16 (head size 128, partition a
  * multiple of 128) the products run on the tensor cores, whose operands share
  * one type: the probabilities are rounded to dtype before they weight V.
  * Exactly pa_decode_partitions followed (when the workspace size is not 0) by
- * pa_decode_reduce on the same stream.
+ * pa_decode_reduce on the same stream, with the same partition length (for
+ * partition_size = 0: pa_decode_auto_partition_size(...), passed to both).
  */
 pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* block_tables, int max_blocks_per_seq,
@@ -155,8 +172,8 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                     size_t workspace_bytes, void* stream);
 
 /*
- * First phase of pa_decode (same arguments): one CTA per (sequence, kv head,
- * partition).  Sequences that fit one partition get their final `out` rows;
+ * First phase of pa_decode (same arguments; partition_size = 0 means the
+ * default 512 here): one CTA per (sequence, kv head, partition).  Sequences that fit one partition get their final `out` rows;
  * the others leave per-partition (max, sum, unnormalised output) partials in
  * the workspace.
  */

@@ -27,7 +27,8 @@ PA_DEVERR_TABLE, PA_DEVERR_CONTEXT, PA_DEVERR_SLOT, PA_DEVERR_PAIR, PA_DEVERR_TI
 # every symbol include/pagedkv.h declares
 EXPORTS = (
     "pa_last_error", "pa_version", "pa_launch_count", "pa_device_status",
-    "pa_decode_default_partition_size", "pa_decode_num_partitions", "pa_decode_workspace_bytes",
+    "pa_decode_default_partition_size", "pa_decode_auto_partition_size",
+    "pa_decode_num_partitions", "pa_decode_workspace_bytes",
     "pa_decode", "pa_decode_partitions", "pa_decode_reduce", "pa_decode_noalloc",
     "pa_reshape_and_cache",
     "pa_copy_blocks", "pa_alloc_create", "pa_alloc_destroy", "pa_alloc_num_free",
@@ -70,6 +71,7 @@ def lib():
         "pa_launch_count": ([], ctypes.c_uint64),
         "pa_device_status": ([ctypes.POINTER(ctypes.c_uint), i32], i32),
         "pa_decode_default_partition_size": ([], i32),
+        "pa_decode_auto_partition_size": ([i32, i32, i32, i32, i32, i32], i32),
         "pa_decode_num_partitions": ([i32, i32], i32),
         "pa_decode_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
         "pa_decode": ([vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, f32, i32, i32,
@@ -156,6 +158,13 @@ def pa_device_status(clear: bool = True) -> int:
 
 def pa_decode_default_partition_size() -> int:
     return int(lib().pa_decode_default_partition_size())
+
+
+def pa_decode_auto_partition_size(num_seqs: int, num_heads: int, num_kv_heads: int,
+                                  head_size: int, dtype: int, max_context_len: int) -> int:
+    """The partition length pa_decode picks for partition_size = 0 (dtype: PA_*)."""
+    return int(lib().pa_decode_auto_partition_size(num_seqs, num_heads, num_kv_heads, head_size,
+                                                   dtype, max_context_len))
 
 
 def pa_decode_num_partitions(max_context_len: int, partition_size: int = 0) -> int:

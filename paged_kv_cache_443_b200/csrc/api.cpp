@@ -29,6 +29,32 @@ int64_t num_partitions(int max_context_len, int P) {
   return (static_cast<int64_t>(max_context_len) + P - 1) / P;
 }
 
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+// Partition length pa_decode uses for partition_size = 0.  The tensor-core
+// kernel (fp16/bf16, head size 128, 4 or 8 query heads per kv head) pays a
+// fixed set-up and drain per CTA, so it takes the longest of 2048 / 1024 tokens
+// that still gives at least ~4 waves of CTAs (2 per SM) at the longest context;
+// everything else keeps the default.
+int auto_partition(int num_seqs, int num_heads, int num_kv_heads, int head_size, pa_dtype dtype,
+                   int max_context_len) {
+  const int G = num_kv_heads > 0 ? num_heads / num_kv_heads : 0;
+  const bool tc = (dtype == PA_F16 || dtype == PA_BF16) && head_size == 128 && (G == 4 || G == 8);
+  if (!tc) return pa::kDefaultPartition;
+  const int64_t want = 8ll * num_sms();
+  for (int P : {2048, 1024}) {
+    const int64_t ctas = static_cast<int64_t>(num_seqs) * num_kv_heads * num_partitions(max_context_len, P);
+    if (ctas >= want) return P;
+  }
+  return pa::kDefaultPartition;
+}
+
 size_t workspace_bytes(int64_t B, int64_t Hq, int64_t D, int64_t NP) {
   if (NP <= 1 || B <= 0) return 0;
   const size_t raw = static_cast<size_t>(B * Hq * NP * (D + 2) * 4);
@@ -210,6 +236,14 @@ extern "C" pa_status pa_decode_reduce(void* out, const int32_t* context_lens, in
   return launch_status("pa_decode_reduce", pa::launch_decode_reduce(a, nullptr, stream), 1);
 }
 
+extern "C" int pa_decode_auto_partition_size(int num_seqs, int num_heads, int num_kv_heads,
+                                             int head_size, pa_dtype dtype, int max_context_len) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 ||
+      head_size <= 0 || pa::elem_size(dtype) == 0 || max_context_len < 0)
+    return -1;
+  return auto_partition(num_seqs, num_heads, num_kv_heads, head_size, dtype, max_context_len);
+}
+
 extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
                                const int32_t* block_tables, int max_blocks_per_seq,
                                const int32_t* context_lens, int num_seqs, int num_heads,
@@ -217,6 +251,12 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
                                float scale, pa_dtype dtype, int partition_size,
                                int max_context_len, void* workspace, size_t workspace_bytes_in,
                                void* stream) {
+  // 0 = the automatic length; it never needs more workspace than the default
+  // (a longer partition means fewer partials), which is what
+  // pa_decode_workspace_bytes(..., 0) sized
+  if (partition_size == 0 && num_heads > 0 && num_kv_heads > 0)
+    partition_size =
+        auto_partition(num_seqs, num_heads, num_kv_heads, head_size, dtype, max_context_len);
   pa::DecodeArgs a;
   pa_status st = check_decode_full("pa_decode", out, q, k_cache, v_cache, block_tables,
                                    max_blocks_per_seq, context_lens, num_seqs, num_heads,

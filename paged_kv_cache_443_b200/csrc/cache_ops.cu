@@ -29,6 +29,7 @@ __global__ void __launch_bounds__(256)
                              const int64_t* __restrict__ slot_mapping, int64_t total_chunks,
                              int Hkv, int chunks_per_row, int log2_bs, int64_t num_slots,
                              unsigned int* status) {
+  allow_dependents();   // the decode kernels may start launching (they wait for us)
   const int64_t per_token = static_cast<int64_t>(Hkv) * chunks_per_row;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total_chunks;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -55,6 +56,7 @@ __global__ void __launch_bounds__(256)
     copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                        const int64_t* __restrict__ pairs, int num_pairs, int64_t chunks_per_block,
                        int64_t num_blocks, unsigned int* status) {
+  allow_dependents();
   for (int pr = blockIdx.y; pr < num_pairs; pr += gridDim.y) {
     const int64_t src = __ldg(pairs + 2 * pr);
     const int64_t dst = __ldg(pairs + 2 * pr + 1);

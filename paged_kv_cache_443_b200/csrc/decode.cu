@@ -140,6 +140,8 @@ __global__ void __launch_bounds__(Cfg<T, D, G, NCW>::THREADS)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  grid_dependency_wait();   // the appended tokens of the previous kernel are in the cache
+  allow_dependents();       // the reduce kernel may start launching
   // ---- this partition's token range (validated) ----
   int L = p.context_lens[b];
   const int P = p.partition_size;
@@ -431,6 +433,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(128) decode_reduce_kernel(const ReduceParams p) {
   using E = Elem<T>;
   constexpr int DPL = D / 32;  // dims per lane
+  grid_dependency_wait();   // every partial of the partition kernel is written
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= static_cast<int64_t>(p.num_seqs) * p.Hq) return;
@@ -495,8 +498,7 @@ cudaError_t launch_partition_t(const DecodeArgs& a, unsigned int* status, cudaSt
   p.num_partitions = a.num_partitions;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   dim3 grid(a.num_seqs, a.Hkv, a.num_partitions);
-  kern<<<grid, C::THREADS, C::SMEM, stream>>>(p);
-  return cudaGetLastError();
+  return launch_overlapped(kern, grid, dim3(C::THREADS), C::SMEM, stream, p);
 }
 
 template <typename T, int D>
@@ -534,11 +536,8 @@ cudaError_t launch_reduce_t(const DecodeArgs& a, cudaStream_t stream) {
   p.num_partitions = a.num_partitions;
   const int64_t warps = static_cast<int64_t>(a.num_seqs) * a.Hq;
   const unsigned grid = static_cast<unsigned>((warps + 3) / 4);
-  if (a.D == 64)
-    decode_reduce_kernel<T, 64><<<grid, 128, 0, stream>>>(p);
-  else
-    decode_reduce_kernel<T, 128><<<grid, 128, 0, stream>>>(p);
-  return cudaGetLastError();
+  if (a.D == 64) return launch_overlapped(decode_reduce_kernel<T, 64>, dim3(grid), dim3(128), 0, stream, p);
+  return launch_overlapped(decode_reduce_kernel<T, 128>, dim3(grid), dim3(128), 0, stream, p);
 }
 
 }  // namespace

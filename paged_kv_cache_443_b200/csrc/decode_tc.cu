@@ -112,6 +112,8 @@ __global__ void __launch_bounds__(THREADS, 2)
   const int b = blockIdx.x, g = blockIdx.y, part = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  grid_dependency_wait();   // the appended tokens of the previous kernel are in the cache
+  allow_dependents();       // the reduce kernel may start launching
   int L = p.context_lens[b];
   const int P = p.partition_size;
   int64_t cap = p.max_blocks * p.block_size;
@@ -467,8 +469,7 @@ cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t 
   p.num_partitions = a.num_partitions;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   dim3 grid(a.num_seqs, a.Hkv, a.num_partitions);
-  kern<<<grid, THREADS, SMEM_BYTES, stream>>>(p, mk, mv);
-  return cudaGetLastError();
+  return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
 }
 
 }  // namespace

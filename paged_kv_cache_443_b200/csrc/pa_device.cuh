@@ -104,6 +104,18 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
   return p;
 }
 
+// Programmatic dependent launch: a kernel launched right after another on the
+// same stream (with programmatic stream serialisation) may start before that
+// one finishes; grid_dependency_wait() blocks until it has completed and its
+// memory is visible (a no-op when there is no such dependency), and
+// allow_dependents() lets the next kernel of the stream begin launching.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Named barrier over `nthreads` threads (a multiple of 32) with id `id` (1..15).
 __device__ __forceinline__ void named_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

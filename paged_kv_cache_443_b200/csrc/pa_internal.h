@@ -4,6 +4,9 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <utility>
+
+#include <cuda_runtime.h>
 
 #include "pagedkv.h"
 
@@ -74,5 +77,24 @@ int launch_reshape_and_cache(const void* key, const void* value, void* k_cache, 
 int launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_pairs, int Hkv,
                        int D, int block_size, int num_blocks, int esize, unsigned int* status,
                        void* stream);
+
+// Launches `kernel` on `stream` allowing it to overlap the tail of the previous
+// kernel on the stream (programmatic stream serialisation); the kernel must
+// call grid_dependency_wait() before it reads anything an earlier launch wrote.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_overlapped(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                     cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 }  // namespace pa

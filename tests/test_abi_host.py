@@ -119,3 +119,21 @@ def test_reshape_and_copy_reject_bad_arguments(L):
     assert c(pairs=FAKE + 4) == pk.PA_ERR_INVALID
     assert c(dtype=9) == pk.PA_ERR_INVALID
     assert c(P=0) == pk.PA_OK
+
+
+def test_auto_partition_size(L):
+    bf = pk.PA_BF16
+    # tensor-core shapes with plenty of work take long partitions
+    assert pk.pa_decode_auto_partition_size(256, 64, 8, 128, bf, 4096) == 2048
+    assert pk.pa_decode_auto_partition_size(128, 32, 8, 128, bf, 32768) == 2048
+    # too few CTAs at long partitions: the default
+    assert pk.pa_decode_auto_partition_size(1, 64, 8, 128, bf, 32768) == 512
+    # other paths keep the default
+    assert pk.pa_decode_auto_partition_size(64, 40, 40, 128, pk.PA_F16, 2048) == 512
+    assert pk.pa_decode_auto_partition_size(256, 64, 8, 64, bf, 4096) == 512
+    assert pk.pa_decode_auto_partition_size(256, 64, 8, 128, pk.PA_F32, 4096) == 512
+    assert pk.pa_decode_auto_partition_size(4, 6, 4, 128, bf, 100) == -1
+    # the default-sized workspace covers the automatic length
+    for P in (1024, 2048):
+        assert pk.pa_decode_workspace_bytes(256, 64, 128, 4096, P) <= \
+            pk.pa_decode_workspace_bytes(256, 64, 128, 4096, 0)

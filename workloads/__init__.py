@@ -18,6 +18,7 @@ not available here; shapes follow the public model configurations):
   llama13b_ps  16 prompts x 6 samples, Hq=Hkv=40, D=128, bf16, prompt ~ U[512,1024]
                shared through forked (refcounted) blocks, 1..256 divergent tokens
   gqa70b       256 seqs, Hq=64, Hkv=8, D=128, bf16, block 16, context ~ U[256,4096]
+               (no partition length is given: the library's automatic one)
   long_prefix  128 requests forked from one 4096-token prefix (same physical
                blocks) plus a unique suffix ~ U[1,28672]; Hq=32, Hkv=8, D=128,
                bf16, block 8/16/32, split-K partitions of 512 tokens
@@ -55,7 +56,7 @@ class Spec:
     seed: int
     num_blocks: Optional[int] = None  # pool size; None = 1.25x what the script needs
     scale: Optional[float] = None     # None = 1/sqrt(D)
-    partition_size: int = 512
+    partition_size: int = 512       # 0 = the library's automatic choice
     # independent
     ctx_dist: str = "uniform"       # 'uniform' | 'lognormal' | 'explicit'
     ctx_list: Tuple[int, ...] = ()  # explicit context lengths (num_seqs of them)
@@ -102,7 +103,7 @@ LLAMA13B_PS = Spec("llama13b_ps", "bf16", 40, 40, 128, 16, "parallel_sampling", 
                    num_prompts=16, samples_per_prompt=6, prompt_lo=512, prompt_hi=1024,
                    div_lo=1, div_hi=256)
 GQA70B = Spec("gqa70b", "bf16", 64, 8, 128, 16, "independent", 256, seed=446,
-              ctx_dist="uniform", ctx_lo=256, ctx_hi=4096)
+              ctx_dist="uniform", ctx_lo=256, ctx_hi=4096, partition_size=0)
 LONG_PREFIX = Spec("long_prefix", "bf16", 32, 8, 128, 16, "shared_prefix", 128, seed=447,
                    prefix_len=4096, suffix_lo=1, suffix_hi=28672, partition_size=512)
 

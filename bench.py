@@ -23,6 +23,11 @@ scaling; the step time is the max over ranks.
 
 --impl reference times the oracle (the plain fp64 CPU implementation) on the
 host cores on the same workload and metric, one bounded sample per step.
+
+--op swap (1 GPU) measures the block swap instead: every block of the
+workload's batch to a pinned host pool (scattered ids) and back, one
+pa_swap_blocks launch per direction, against one contiguous device<->pinned
+copy of the same bytes (the link's own rate).
 """
 import argparse
 import hashlib
@@ -598,6 +603,112 @@ def run_ours(args):
     return result
 
 
+def run_swap(args):
+    """Swap-out / swap-in bandwidth of pa_swap_blocks on the workload's blocks."""
+    import torch
+    import paged_kv_cache_443_b200 as pk
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: a CUDA device is required for --op swap")
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    pk.lib()
+    spec = workload_spec(args.workload)
+    sc = W.scenario(spec)
+    dt = W.torch_dtype(spec)
+    shape = (sc.num_blocks, spec.Hkv, spec.block_size, spec.D)
+    kc = torch.randn(shape, dtype=torch.float32, device=device).to(dt)
+    vc = torch.randn(shape, dtype=torch.float32, device=device).to(dt)
+    # the batch's blocks: the live ids of the scenario's block tables, in table order
+    cache_ids = []
+    bm = pk.BlockAllocator(sc.num_blocks, spec.block_size, sc.free_order.tolist())
+    for op in sc.setup_ops + sc.step_ops:
+        if op.kind == "add":
+            bm.add(op.seq)
+        elif op.kind == "fork":
+            bm.fork(op.seq, op.arg)
+        elif op.kind == "release":
+            bm.release(op.seq)
+        else:
+            bm.append(op.seq, op.arg)
+    t, _ = bm.build_tables(sc.batch, sc.max_blocks)
+    seen = set()
+    for x in t.ravel():
+        if x >= 0 and int(x) not in seen:
+            seen.add(int(x))
+            cache_ids.append(int(x))
+    n = len(cache_ids)
+    rng = np.random.default_rng(spec.seed)
+    host_ids = rng.permutation(n)
+    hk = torch.empty((n,) + shape[1:], dtype=dt).pin_memory()
+    hv = torch.empty((n,) + shape[1:], dtype=dt).pin_memory()
+    out_pairs = torch.tensor(np.stack([cache_ids, host_ids], 1), dtype=torch.int64, device=device)
+    in_pairs = torch.tensor(np.stack([host_ids, cache_ids], 1), dtype=torch.int64, device=device)
+    block_bytes = spec.Hkv * spec.block_size * spec.D * W.DTYPE_BYTES[spec.dtype]
+    moved = 2 * n * block_bytes                      # K and V, one direction
+    stream = torch.cuda.current_stream(device)
+    flat_d = torch.empty(moved, dtype=torch.uint8, device=device)
+    flat_h = torch.empty(moved, dtype=torch.uint8).pin_memory()
+
+    def timed(fn, K):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1) / K
+
+    K = max(1, min(args.steps, 20))
+    sampler = ClockSampler(0)
+    sampler.start()
+    t0 = time.time()
+    launches0 = pk.pa_launch_count()
+    out_ms = timed(lambda: pk.pa_swap_blocks(hk, hv, kc, vc, out_pairs, stream=stream), K)
+    in_ms = timed(lambda: pk.pa_swap_blocks(kc, vc, hk, hv, in_pairs, stream=stream), K)
+    launches = pk.pa_launch_count() - launches0
+    d2h_ms = timed(lambda: flat_h.copy_(flat_d, non_blocking=True), K)
+    h2d_ms = timed(lambda: flat_d.copy_(flat_h, non_blocking=True), K)
+    t1 = time.time()
+    sampler.stop()
+    assert pk.pa_device_status() == 0, "device-side check failed"
+    # round trip restores the cache bit for bit
+    ref_k = kc.clone()
+    pk.pa_swap_blocks(hk, hv, kc, vc, out_pairs, stream=stream)
+    kc.zero_()
+    pk.pa_swap_blocks(kc, vc, hk, hv, in_pairs, stream=stream)
+    torch.cuda.synchronize(device)
+    ids = torch.tensor(cache_ids, device=device)
+    assert torch.equal(kc.index_select(0, ids).view(torch.int16),
+                       ref_k.index_select(0, ids).view(torch.int16))
+    gbs = lambda ms: moved / (ms * 1e-3) / 1e9  # noqa: E731
+    rt_ms = out_ms + in_ms
+    return {
+        "metric": "swap_blocks GB/s, device <-> pinned host (K and V blocks, each direction)",
+        "op": "swap",
+        "value": round(2 * moved / (rt_ms * 1e-3) / 1e9, 2),
+        "unit": "GB/s",
+        "n_gpus": 1, "steps": K, "warmup": max(3, args.warmup),
+        "ms_per_step": round(rt_ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": spec.dtype, "data": "synthetic N(0,1) blocks",
+        "config": {"workload": f"{args.workload}: {workload_text(args.workload)}",
+                   "blocks": n, "block_bytes_per_cache": block_bytes,
+                   "bytes_per_direction": moved, "host_ids": "random permutation"},
+        "swap_out": {"ms": round(out_ms, 4), "GB/s": round(gbs(out_ms), 2)},
+        "swap_in": {"ms": round(in_ms, 4), "GB/s": round(gbs(in_ms), 2)},
+        "contiguous_copy": {"d2h_GB/s": round(gbs(d2h_ms), 2), "h2d_GB/s": round(gbs(h2d_ms), 2)},
+        "roofline": {"bound": "link", "achieved": round(2 * moved / (rt_ms * 1e-3) / 1e9, 2),
+                     "peak": round(2 * moved / ((d2h_ms + h2d_ms) * 1e-3) / 1e9, 2),
+                     "peak_kind": "contiguous cudaMemcpyAsync of the same bytes, measured here",
+                     "unit": "GB/s", "frac": round((d2h_ms + h2d_ms) / rt_ms, 4)},
+        "gpu_launches": int(launches),
+        "clocks": sampler.summary(t0, t1),
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -613,6 +724,8 @@ def main():
     ap.add_argument("--soak-seconds", type=float, default=0.5,
                     help="untimed load before the timed steps (clock samples)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--op", default="decode", choices=["decode", "swap"],
+                    help="decode: the hot path (default); swap: block swap bandwidth")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
@@ -639,6 +752,11 @@ def main():
             "gpu_launches": 0,
         }
         print(json.dumps(line), flush=True)
+        return
+
+    if args.op == "swap":
+        if rank == 0 and args.impl == "ours":
+            print(json.dumps(run_swap(args)), flush=True)
         return
 
     result = run_ours(args)

@@ -87,6 +87,17 @@ uint64_t pa_launch_count(void);
  */
 pa_status pa_device_status(unsigned int* flags_out, int clear);
 
+/*
+ * Checks the kernels' bounded-wait mechanism (no counterpart on the pages: a
+ * robustness test).  Launches one CTA on the current device that waits, with a
+ * 20 ms limit, on a shared-memory barrier that nothing will complete; the wait
+ * gives up and sets PA_DEVERR_TIMEOUT.  On return *flags_out holds the status
+ * word that launch produced (PA_DEVERR_TIMEOUT expected) and the device is
+ * usable as before; bits already pending are kept for pa_device_status.
+ * Synchronises the current device.
+ */
+pa_status pa_selftest_wait_timeout(unsigned int* flags_out);
+
 /* ------------------------------------------------------------------------ */
 /* Decode attention ([P1] "자기회귀 생성과 KV 캐시", "PagedAttention의 설계")  */
 
@@ -258,6 +269,27 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_pair
                          int num_kv_heads, int head_size, int block_size, int num_blocks,
                          pa_dtype dtype, void* stream);
 
+/*
+ * Swap ([P1] "적용 범위와 관련 연구": when GPU memory runs short a sequence's KV
+ * blocks move to CPU memory and come back later): for each pair p, physical
+ * block block_pairs[p][1] of the destination caches becomes a byte copy of
+ * block block_pairs[p][0] of the source caches (all kv heads, all slots).
+ * One cache pair is device memory, the other may be device memory or pinned
+ * host memory the GPU can address (cudaHostAlloc / cudaHostRegister with
+ * unified addressing); the copy runs as a kernel on `stream`, so one call moves
+ * any number of scattered blocks.
+ *
+ *   dst_k_cache, dst_v_cache  [dst_num_blocks][Hkv][bs][D] dtype (16-byte aligned)
+ *   src_k_cache, src_v_cache  [src_num_blocks][Hkv][bs][D] dtype (16-byte aligned)
+ *   block_pairs  [num_pairs][2] int64 (src, dst), device or GPU-addressable host memory
+ * Pairs with an id outside their pool are skipped (PA_DEVERR_PAIR).  The
+ * destinations must be distinct and must not overlap the sources.
+ */
+pa_status pa_swap_blocks(void* dst_k_cache, void* dst_v_cache, int dst_num_blocks,
+                         const void* src_k_cache, const void* src_v_cache, int src_num_blocks,
+                         const int64_t* block_pairs, int num_pairs, int num_kv_heads,
+                         int head_size, int block_size, pa_dtype dtype, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Block manager (host memory; [P1] "PagedAttention의 설계", "블록 공유";     */
 /* [P2] section 3; [P3] "4.2 PagedAttention의 접근").  Not thread-safe: use one */
@@ -306,6 +338,25 @@ pa_status pa_seq_append(pa_allocator* a, int64_t seq_id, int n_tokens, int64_t* 
 /* Drops the sequence; its blocks lose one reference each, in logical order, and
  * blocks reaching zero are pushed on the free stack. */
 pa_status pa_seq_free(pa_allocator* a, int64_t seq_id);
+
+/*
+ * Moves sequences from manager `src` to manager `dst` (same block size), e.g.
+ * to a pinned host pool when GPU memory runs short and back again ([P1]
+ * "적용 범위와 관련 연구").  Sharing among the sequences moved together is kept:
+ * walking seq_ids in order and each one's blocks in logical order, a source
+ * block met for the first time takes a fresh destination block (popped from
+ * dst's free stack) and the pair (src block, dst block) is appended to
+ * pairs_out [pairs_capacity][2]; every later holder shares that block.  The
+ * token counts move unchanged; then each sequence is freed in `src` in caller
+ * order (as pa_seq_free).  The caller runs pa_swap_blocks on the *n_pairs pairs
+ * before any block freed in `src` is written again (stream order suffices).
+ * Errors change nothing: PA_ERR_OOM when dst has fewer free blocks than the
+ * distinct blocks; PA_ERR_INVALID for an unknown id, an id already in dst, a
+ * repeated id, differing block sizes, src == dst, or pairs_capacity below
+ * the number of distinct blocks (at most the sum of the sequences' blocks).
+ */
+pa_status pa_seq_move(pa_allocator* src, pa_allocator* dst, const int64_t* seq_ids, int num_seqs,
+                      int64_t* pairs_out, int pairs_capacity, int* n_pairs);
 
 /* Tokens held by the sequence. */
 pa_status pa_seq_num_tokens(const pa_allocator* a, int64_t seq_id, int* out);

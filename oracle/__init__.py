@@ -6,7 +6,8 @@ the tests, the smoke check of ``__graft_entry__`` and the CPU-baseline leg of
 
 Parts:
   * ``pa_oracle.c`` (loaded here through ctypes): fp64 attention over the
-    paged cache, the new-token append and the copy-on-write block copy;
+    paged cache, the new-token append, the copy-on-write block copy and the
+    block swap between two caches;
   * ``allocator.py``: the block manager (allocate on demand, share by
     reference count, copy on write, reclaim);
   * ``kv_size.py``: the KV-cache size formula of "1. KV 캐시란" (hjr-study-book
@@ -48,6 +49,8 @@ def lib():
         L.or_reshape_and_cache.restype = i32
         L.or_copy_blocks.argtypes = [p, p, p, i64, i32, i32, i32, i64, i32]
         L.or_copy_blocks.restype = i32
+        L.or_swap_blocks.argtypes = [p, p, i64, p, p, i64, p, i64, i32, i32, i32, i32]
+        L.or_swap_blocks.restype = i32
         L.or_max_threads.argtypes = []
         L.or_max_threads.restype = i32
         _lib = L
@@ -138,5 +141,25 @@ def copy_blocks(k_cache, v_cache, pairs, dtype):
     NB, Hkv, bs, D = k_cache.shape
     rc = lib().or_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(pairs), pairs.shape[0],
                               Hkv, D, bs, NB, dtype)
+    if rc != 0:
+        raise ValueError("oracle: block id out of range")
+
+
+def swap_blocks(dst_k, dst_v, src_k, src_v, pairs, dtype):
+    """Block pairs[p,1] of the destination caches := block pairs[p,0] of the
+    source caches, in order (swap out to host memory or back in).
+
+    Follows "적용 범위와 관련 연구" of the supersilo.blog vLLM summary (sequences
+    move to CPU memory when GPU memory is short).
+    """
+    pairs = _c(pairs, np.int64).reshape(-1, 2)
+    for a in (dst_k, dst_v):
+        assert a.flags.c_contiguous
+    src_k, src_v = _c(src_k), _c(src_v)
+    NBd, Hkv, bs, D = dst_k.shape
+    NBs = src_k.shape[0]
+    assert src_k.shape[1:] == dst_k.shape[1:]
+    rc = lib().or_swap_blocks(_ptr(dst_k), _ptr(dst_v), NBd, _ptr(src_k), _ptr(src_v), NBs,
+                              _ptr(pairs), pairs.shape[0], Hkv, D, bs, dtype)
     if rc != 0:
         raise ValueError("oracle: block id out of range")

@@ -33,7 +33,14 @@ implementations can agree exactly):
     copy-on-write); the copy is taken before any new blocks, which follow in
     logical order;
   * an append or fork that cannot get all its blocks changes nothing and fails
-    with OOM.
+    with OOM;
+  * moving sequences to another manager (swap to CPU memory and back, "적용
+    범위와 관련 연구" of the supersilo.blog summary, which gives no mechanism)
+    keeps the sharing among the sequences moved together: going through them in
+    the caller's order and through each one's blocks in logical order, a block
+    seen for the first time takes the destination's next free block, and later
+    holders share it; the sequences are then released in the source in the
+    caller's order.
 """
 from dataclasses import dataclass, field
 from typing import Dict, List, Optional, Sequence, Tuple
@@ -146,6 +153,39 @@ class BlockManager:
             self.refcount[blk] -= 1
             if self.refcount[blk] == 0:
                 self.free.append(blk)
+
+    def move_to(self, dst: "BlockManager", seq_ids: Sequence[int]) -> List[Tuple[int, int]]:
+        """Move the sequences into dst; returns the (source block, dst block)
+        pairs whose contents must be copied."""
+        seq_ids = [int(x) for x in seq_ids]
+        if dst is self or dst.block_size != self.block_size:
+            raise Invalid("bad destination")
+        if len(set(seq_ids)) != len(seq_ids):
+            raise Invalid("repeated sequence")
+        for sid in seq_ids:
+            if sid not in self.seqs or sid in dst.seqs:
+                raise Invalid("unknown sequence or already in the destination")
+        distinct = {blk for sid in seq_ids for blk in self.seqs[sid].blocks}
+        if len(distinct) > len(dst.free):
+            raise OOM("not enough free blocks in the destination")
+        where: Dict[int, int] = {}
+        pairs: List[Tuple[int, int]] = []
+        for sid in seq_ids:
+            s = self.seqs[sid]
+            mapped = []
+            for blk in s.blocks:
+                if blk in where:
+                    dst.refcount[where[blk]] += 1
+                else:
+                    new = dst.free.pop()
+                    dst.refcount[new] = 1
+                    where[blk] = new
+                    pairs.append((blk, new))
+                mapped.append(where[blk])
+            dst.seqs[sid] = _Seq(mapped, s.num_tokens)
+        for sid in seq_ids:
+            self.release(sid)
+        return pairs
 
     def build_tables(self, seq_ids: Sequence[int], max_blocks: int):
         """Block tables [B][max_blocks] (padding -1) and context lengths [B]."""

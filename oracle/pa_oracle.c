@@ -266,6 +266,27 @@ int or_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int64_t P
   return 0;
 }
 
+/* ---- swapping blocks between two caches ----
+ * Follows "적용 범위와 관련 연구" (supersilo.blog): when GPU memory runs short, a
+ * sequence's KV blocks move to CPU memory and come back later.  For each pair p
+ * in order, block pairs[2p+1] of the destination caches becomes a byte copy of
+ * block pairs[2p] of the source caches (all kv heads, all slots).  Returns -1 on
+ * an id outside the source or destination pool. */
+int or_swap_blocks(void* dst_k, void* dst_v, int64_t dst_num_blocks, const void* src_k,
+                   const void* src_v, int64_t src_num_blocks, const int64_t* pairs, int64_t P,
+                   int Hkv, int D, int block_size, int dtype) {
+  const size_t es = (size_t)or_elem_size(dtype);
+  if (es == 0) return -1;
+  const size_t block_bytes = (size_t)Hkv * block_size * D * es;
+  for (int64_t p = 0; p < P; ++p) {
+    const int64_t src = pairs[2 * p], dst = pairs[2 * p + 1];
+    if (src < 0 || src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks) return -1;
+    memcpy((char*)dst_k + dst * block_bytes, (const char*)src_k + src * block_bytes, block_bytes);
+    memcpy((char*)dst_v + dst * block_bytes, (const char*)src_v + src * block_bytes, block_bytes);
+  }
+  return 0;
+}
+
 int or_max_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

@@ -27,13 +27,14 @@ PA_DEVERR_TABLE, PA_DEVERR_CONTEXT, PA_DEVERR_SLOT, PA_DEVERR_PAIR, PA_DEVERR_TI
 # every symbol include/pagedkv.h declares
 EXPORTS = (
     "pa_last_error", "pa_version", "pa_launch_count", "pa_device_status",
+    "pa_selftest_wait_timeout",
     "pa_decode_default_partition_size", "pa_decode_auto_partition_size",
     "pa_decode_num_partitions", "pa_decode_workspace_bytes",
     "pa_decode", "pa_decode_partitions", "pa_decode_reduce", "pa_decode_noalloc",
     "pa_reshape_and_cache",
-    "pa_copy_blocks", "pa_alloc_create", "pa_alloc_destroy", "pa_alloc_num_free",
+    "pa_copy_blocks", "pa_swap_blocks", "pa_alloc_create", "pa_alloc_destroy", "pa_alloc_num_free",
     "pa_alloc_refcount", "pa_alloc_free_stack", "pa_seq_add", "pa_seq_fork", "pa_seq_append",
-    "pa_seq_free", "pa_seq_num_tokens", "pa_build_tables",
+    "pa_seq_free", "pa_seq_move", "pa_seq_num_tokens", "pa_build_tables",
 )
 
 
@@ -70,6 +71,7 @@ def lib():
         "pa_version": ([], ctypes.c_char_p),
         "pa_launch_count": ([], ctypes.c_uint64),
         "pa_device_status": ([ctypes.POINTER(ctypes.c_uint), i32], i32),
+        "pa_selftest_wait_timeout": ([ctypes.POINTER(ctypes.c_uint)], i32),
         "pa_decode_default_partition_size": ([], i32),
         "pa_decode_auto_partition_size": ([i32, i32, i32, i32, i32, i32], i32),
         "pa_decode_num_partitions": ([i32, i32], i32),
@@ -83,6 +85,7 @@ def lib():
                                i32, i32, i32, vp], i32),
         "pa_reshape_and_cache": ([vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp], i32),
         "pa_copy_blocks": ([vp, vp, vp, i32, i32, i32, i32, i32, i32, vp], i32),
+        "pa_swap_blocks": ([vp, vp, i32, vp, vp, i32, vp, i32, i32, i32, i32, i32, vp], i32),
         "pa_alloc_create": ([i32, i32, pi32, ctypes.POINTER(vp)], i32),
         "pa_alloc_destroy": ([vp], None),
         "pa_alloc_num_free": ([vp], i32),
@@ -92,6 +95,7 @@ def lib():
         "pa_seq_fork": ([vp, i64, i64], i32),
         "pa_seq_append": ([vp, i64, i32, pi64, pi64, ctypes.POINTER(i32)], i32),
         "pa_seq_free": ([vp, i64], i32),
+        "pa_seq_move": ([vp, vp, pi64, i32, pi64, i32, ctypes.POINTER(i32)], i32),
         "pa_seq_num_tokens": ([vp, i64, ctypes.POINTER(i32)], i32),
         "pa_build_tables": ([vp, pi64, i32, i32, pi32, pi32], i32),
     }
@@ -153,6 +157,13 @@ def pa_launch_count() -> int:
 def pa_device_status(clear: bool = True) -> int:
     v = ctypes.c_uint(0)
     _check(lib().pa_device_status(ctypes.byref(v), int(clear)))
+    return int(v.value)
+
+
+def pa_selftest_wait_timeout() -> int:
+    """Status bits of a launch whose internal wait is made to run out."""
+    v = ctypes.c_uint(0)
+    _check(lib().pa_selftest_wait_timeout(ctypes.byref(v)))
     return int(v.value)
 
 
@@ -272,6 +283,28 @@ def pa_copy_blocks(k_cache, v_cache, block_pairs, stream=None) -> None:
                                 P, Hkv, D, bs, NB, _dtype_code(k_cache), _stream(stream)))
 
 
+def pa_swap_blocks(dst_k_cache, dst_v_cache, src_k_cache, src_v_cache, block_pairs,
+                   stream=None) -> None:
+    """Block block_pairs[p,1] of the destination caches := block block_pairs[p,0]
+    of the source caches.  A cache pair may be pinned host memory (torch
+    pin_memory()); block_pairs is an int64 [P, 2] tensor on the device or pinned."""
+    _contig(dst_k_cache, dst_v_cache, src_k_cache, src_v_cache, block_pairs)
+    import torch
+    NBd, Hkv, bs, D = dst_k_cache.shape
+    NBs = src_k_cache.shape[0]
+    if (tuple(src_k_cache.shape[1:]) != (Hkv, bs, D) or src_v_cache.shape != src_k_cache.shape
+            or dst_v_cache.shape != dst_k_cache.shape):
+        raise PagedKVError(PA_ERR_INVALID, "cache shape mismatch")
+    if not (dst_k_cache.dtype == dst_v_cache.dtype == src_k_cache.dtype == src_v_cache.dtype):
+        raise PagedKVError(PA_ERR_INVALID, "dtype mismatch")
+    if block_pairs.dtype != torch.int64 or (block_pairs.numel() and block_pairs.shape[-1] != 2):
+        raise PagedKVError(PA_ERR_INVALID, "block_pairs must be int64 [P, 2]")
+    P = block_pairs.numel() // 2
+    _check(lib().pa_swap_blocks(_ptr(dst_k_cache), _ptr(dst_v_cache), NBd, _ptr(src_k_cache),
+                                _ptr(src_v_cache), NBs, _ptr(block_pairs) if P else None, P, Hkv,
+                                D, bs, _dtype_code(dst_k_cache), _stream(stream)))
+
+
 # ---------------------------------------------------------------------------
 # block manager (host)
 
@@ -327,6 +360,16 @@ def pa_seq_append(h, seq_id: int, n_tokens: int) -> Tuple[List[int], List[Tuple[
 
 def pa_seq_free(h, seq_id: int) -> None:
     _check(lib().pa_seq_free(h, seq_id))
+
+
+def pa_seq_move(src, dst, seq_ids: Sequence[int], capacity: int) -> List[Tuple[int, int]]:
+    """Move sequences from manager src to dst keeping their sharing; returns the
+    (src block, dst block) pairs to copy.  capacity >= the sequences' block count."""
+    ids = (ctypes.c_int64 * max(1, len(seq_ids)))(*[int(x) for x in seq_ids])
+    buf = (ctypes.c_int64 * max(2, 2 * capacity))()
+    n = ctypes.c_int(0)
+    _check(lib().pa_seq_move(src, dst, ids, len(seq_ids), buf, capacity, ctypes.byref(n)))
+    return [(buf[2 * i], buf[2 * i + 1]) for i in range(n.value)]
 
 
 def pa_seq_num_tokens(h, seq_id: int) -> int:
@@ -390,6 +433,11 @@ class BlockAllocator:
 
     def num_tokens(self, seq_id):
         return pa_seq_num_tokens(self.h, seq_id)
+
+    def move_to(self, dst: "BlockAllocator", seq_ids):
+        """Move sequences to another manager (sharing kept); returns copy pairs."""
+        cap = sum(-(-self.num_tokens(s) // self.block_size) for s in seq_ids)
+        return pa_seq_move(self.h, dst.h, list(seq_ids), cap)
 
     def build_tables(self, seq_ids, max_blocks_per_seq):
         return pa_build_tables(self.h, seq_ids, max_blocks_per_seq)

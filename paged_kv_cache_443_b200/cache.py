@@ -6,16 +6,19 @@ tokens, taking a fresh block only when the current one is full and copying a
 shared block before it is modified ("PagedAttention의 설계", "블록 공유" on the
 supersilo.blog summary; section 3 of the blog.aqudi.me write-up); the new
 tokens' K/V are stored at their slots ("1. KV 캐시란", hjr-study-book Day 3);
-attention then reads every sequence's K/V through its block table.  No
-arithmetic happens here: slots and copy pairs come from the C++ block manager,
-every device operation is a libpagedkv.so kernel.
+attention then reads every sequence's K/V through its block table.  When GPU
+memory runs short a sequence can be swapped out to a pinned host pool and back
+("적용 범위와 관련 연구", supersilo.blog): the host pool has its own C++ block
+manager, and both directions are one pa_swap_blocks launch.  No arithmetic
+happens here: slots and copy pairs come from the C++ block managers, every
+device operation is a libpagedkv.so kernel.
 """
 from typing import List, Optional, Sequence, Tuple
 
 import torch
 
-from . import (BlockAllocator, pa_copy_blocks, pa_decode, pa_decode_num_partitions,
-               pa_decode_workspace_bytes, pa_reshape_and_cache)
+from . import (BlockAllocator, pa_copy_blocks, pa_decode, pa_decode_workspace_bytes,
+               pa_reshape_and_cache, pa_swap_blocks)
 
 
 class PagedKVCache:
@@ -33,6 +36,8 @@ class PagedKVCache:
             self.k_cache = torch.full(shape, fill, dtype=dtype, device=self.device)
             self.v_cache = torch.full(shape, fill, dtype=dtype, device=self.device)
         self.alloc = BlockAllocator(num_blocks, block_size, initial_free_order)
+        self.host_alloc = None
+        self.host_k = self.host_v = None
 
     # ---- block manager ----
     def add(self, seq_id: int) -> None:
@@ -111,3 +116,37 @@ class PagedKVCache:
                   max_context_len, partition_size=partition_size, workspace=workspace,
                   stream=stream)
         return out
+
+    # ---- swap to / from pinned host memory ----
+    def enable_swap(self, num_host_blocks: int) -> None:
+        """Pinned host caches of num_host_blocks blocks, with their own block manager."""
+        shape = (num_host_blocks, self.num_kv_heads, self.block_size, self.head_size)
+        self.host_k = torch.empty(shape, dtype=self.dtype, pin_memory=True)
+        self.host_v = torch.empty(shape, dtype=self.dtype, pin_memory=True)
+        self.host_alloc = BlockAllocator(num_host_blocks, self.block_size)
+
+    def _move(self, src_alloc, dst_alloc, src_caches, dst_caches, seq_ids, stream):
+        pairs = src_alloc.move_to(dst_alloc, seq_ids)    # host: sharing kept, all or nothing
+        if pairs:
+            t = torch.tensor(pairs, dtype=torch.int64, device=self.device)
+            pa_swap_blocks(dst_caches[0], dst_caches[1], src_caches[0], src_caches[1], t,
+                           stream=stream)
+        return pairs
+
+    def swap_out(self, seq_ids: Sequence[int], stream=None) -> List[Tuple[int, int]]:
+        """Move the sequences' blocks to the host pool and release them here
+        (blocks shared among them stay shared).  Returns the (device block,
+        host block) pairs copied; stream order keeps any later write to a
+        released block after the copy."""
+        if self.host_alloc is None:
+            raise RuntimeError("enable_swap() first")
+        return self._move(self.alloc, self.host_alloc, (self.k_cache, self.v_cache),
+                          (self.host_k, self.host_v), seq_ids, stream)
+
+    def swap_in(self, seq_ids: Sequence[int], stream=None) -> List[Tuple[int, int]]:
+        """Bring swapped-out sequences back into fresh device blocks.  Returns the
+        (host block, device block) pairs copied; block tables change accordingly."""
+        if self.host_alloc is None:
+            raise RuntimeError("enable_swap() first")
+        return self._move(self.host_alloc, self.alloc, (self.host_k, self.host_v),
+                          (self.k_cache, self.v_cache), seq_ids, stream)

@@ -8,6 +8,12 @@
 // free stack; freeing in logical order; the copy-on-write block is taken
 // before new blocks; all-or-nothing on OOM.
 //
+// Moving sequences between two managers (swap to host memory and back,
+// "적용 범위와 관련 연구" of the supersilo.blog summary) keeps the sharing among
+// the sequences moved together: a source block gets one destination block the
+// first time it is met (sequences in caller order, blocks in logical order),
+// and every later holder shares it.
+//
 // Storage: one flat refcount array, a free stack, and a hash map from sequence
 // id to its block list.  Every operation is O(blocks touched).
 #include <cstdint>
@@ -160,6 +166,65 @@ extern "C" pa_status pa_seq_free(pa_allocator* a, int64_t seq_id) {
     if (--a->refcount[b] == 0) a->free_stack.push_back(b);
   }
   a->seqs.erase(it);
+  return PA_OK;
+}
+
+extern "C" pa_status pa_seq_move(pa_allocator* src, pa_allocator* dst, const int64_t* seq_ids,
+                                 int num_seqs, int64_t* pairs_out, int pairs_capacity,
+                                 int* n_pairs) {
+  const char* fn = "pa_seq_move";
+  if (!src || !dst || !n_pairs || num_seqs < 0 || pairs_capacity < 0 ||
+      (num_seqs > 0 && !seq_ids))
+    return pa::fail(PA_ERR_INVALID, "%s: bad argument", fn);
+  if (src == dst) return pa::fail(PA_ERR_INVALID, "%s: source and destination are the same", fn);
+  if (src->block_size != dst->block_size)
+    return pa::fail(PA_ERR_INVALID, "%s: block sizes differ (%d vs %d)", fn, src->block_size,
+                    dst->block_size);
+  *n_pairs = 0;
+  // validate and count distinct blocks first: a failure changes nothing
+  std::unordered_map<int64_t, char> ids;
+  std::unordered_map<int32_t, int32_t> map;
+  int64_t distinct = 0;
+  for (int i = 0; i < num_seqs; ++i) {
+    auto it = src->seqs.find(seq_ids[i]);
+    if (it == src->seqs.end())
+      return pa::fail(PA_ERR_INVALID, "%s: unknown sequence %lld", fn, (long long)seq_ids[i]);
+    if (dst->seqs.count(seq_ids[i]))
+      return pa::fail(PA_ERR_INVALID, "%s: sequence %lld exists in the destination", fn,
+                      (long long)seq_ids[i]);
+    if (!ids.emplace(seq_ids[i], 1).second)
+      return pa::fail(PA_ERR_INVALID, "%s: sequence %lld listed twice", fn, (long long)seq_ids[i]);
+    for (int32_t b : it->second.blocks)
+      if (map.emplace(b, -1).second) ++distinct;
+  }
+  if (distinct > static_cast<int64_t>(dst->free_stack.size()))
+    return pa::fail(PA_ERR_OOM, "%s: need %lld blocks, %zu free", fn, (long long)distinct,
+                    dst->free_stack.size());
+  if (distinct > pairs_capacity || (distinct > 0 && !pairs_out))
+    return pa::fail(PA_ERR_INVALID, "%s: pairs_out holds %d pairs, %lld needed", fn,
+                    pairs_capacity, (long long)distinct);
+  int64_t np = 0;
+  for (int i = 0; i < num_seqs; ++i) {
+    const pa_allocator::Seq& s = src->seqs.find(seq_ids[i])->second;
+    pa_allocator::Seq d;
+    d.tokens = s.tokens;
+    d.blocks.reserve(s.blocks.size());
+    for (int32_t b : s.blocks) {
+      int32_t& m = map[b];
+      if (m < 0) {
+        m = dst->pop();
+        pairs_out[2 * np] = b;
+        pairs_out[2 * np + 1] = m;
+        ++np;
+      } else {
+        dst->refcount[m] += 1;
+      }
+      d.blocks.push_back(m);
+    }
+    dst->seqs.emplace(seq_ids[i], std::move(d));
+  }
+  for (int i = 0; i < num_seqs; ++i) pa_seq_free(src, seq_ids[i]);
+  *n_pairs = static_cast<int>(np);
   return PA_OK;
 }
 

@@ -324,8 +324,40 @@ extern "C" pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t*
   unsigned int* status = pa::device_status_word();
   if (!status) return PA_ERR_CUDA;
   return launch_status(fn,
-                       pa::launch_copy_blocks(k_cache, v_cache, block_pairs, num_pairs,
-                                              num_kv_heads, head_size, block_size, num_blocks, es,
+                       pa::launch_copy_blocks(k_cache, v_cache, k_cache, v_cache, block_pairs,
+                                              num_pairs, num_kv_heads, head_size, block_size,
+                                              num_blocks, num_blocks, es, status, stream),
+                       1);
+}
+
+extern "C" pa_status pa_swap_blocks(void* dst_k_cache, void* dst_v_cache, int dst_num_blocks,
+                                    const void* src_k_cache, const void* src_v_cache,
+                                    int src_num_blocks, const int64_t* block_pairs, int num_pairs,
+                                    int num_kv_heads, int head_size, int block_size,
+                                    pa_dtype dtype, void* stream) {
+  const char* fn = "pa_swap_blocks";
+  const int es = pa::elem_size(dtype);
+  if (es == 0) return pa::fail(PA_ERR_INVALID, "%s: unknown dtype %d", fn, dtype);
+  if (num_pairs < 0) return pa::fail(PA_ERR_INVALID, "%s: num_pairs < 0", fn);
+  if (num_kv_heads <= 0 || head_size <= 0 || block_size <= 0 || dst_num_blocks <= 0 ||
+      src_num_blocks <= 0)
+    return pa::fail(PA_ERR_INVALID, "%s: sizes must be positive", fn);
+  if (!supported_head(head_size))
+    return pa::fail(PA_ERR_UNSUPPORTED, "%s: head_size must be 64 or 128", fn);
+  if (!supported_block(block_size))
+    return pa::fail(PA_ERR_UNSUPPORTED, "%s: block_size must be 8, 16 or 32", fn);
+  if (num_pairs == 0) return PA_OK;
+  if (!dst_k_cache || !dst_v_cache || !src_k_cache || !src_v_cache || !block_pairs)
+    return pa::fail(PA_ERR_INVALID, "%s: NULL pointer", fn);
+  if (!pa::aligned16(dst_k_cache) || !pa::aligned16(dst_v_cache) || !pa::aligned16(src_k_cache) ||
+      !pa::aligned16(src_v_cache) || (reinterpret_cast<uintptr_t>(block_pairs) & 7u))
+    return pa::fail(PA_ERR_INVALID, "%s: caches must be 16-byte aligned, pairs 8", fn);
+  unsigned int* status = pa::device_status_word();
+  if (!status) return PA_ERR_CUDA;
+  return launch_status(fn,
+                       pa::launch_copy_blocks(dst_k_cache, dst_v_cache, src_k_cache, src_v_cache,
+                                              block_pairs, num_pairs, num_kv_heads, head_size,
+                                              block_size, src_num_blocks, dst_num_blocks, es,
                                               status, stream),
                        1);
 }

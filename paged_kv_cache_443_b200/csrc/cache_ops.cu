@@ -6,6 +6,9 @@
 // offset) is that of the block-table example of "4.2 PagedAttention의 접근".
 // Copy-on-write: "블록 공유" (supersilo.blog) and section 3 of the blog.aqudi.me
 // write-up -- a block shared by several sequences is copied before one writes.
+// Swap: "적용 범위와 관련 연구" (supersilo.blog) -- when GPU memory is short a
+// sequence's blocks move to CPU memory and back; the same copy kernel moves
+// blocks between a device cache and a pinned host cache the GPU can address.
 //
 // Both are pure data movement in 16-byte chunks: loads are coalesced along
 // the source, stores along a D-element cache row (append) or a whole
@@ -51,23 +54,27 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// grid.y strides over pairs; grid.x * blockDim.x threads stride over one block.
+// Block pairs[p][1] of the destination caches := block pairs[p][0] of the source
+// caches.  The caches may be the same (copy-on-write) or live in different
+// memories, e.g. device and pinned host (swap).  grid.y strides over pairs;
+// grid.x * blockDim.x threads stride over one block.
 __global__ void __launch_bounds__(256)
-    copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+    copy_blocks_kernel(uint4* __restrict__ dst_k, uint4* __restrict__ dst_v,
+                       const uint4* __restrict__ src_k, const uint4* __restrict__ src_v,
                        const int64_t* __restrict__ pairs, int num_pairs, int64_t chunks_per_block,
-                       int64_t num_blocks, unsigned int* status) {
+                       int64_t src_blocks, int64_t dst_blocks, unsigned int* status) {
   allow_dependents();
   for (int pr = blockIdx.y; pr < num_pairs; pr += gridDim.y) {
     const int64_t src = __ldg(pairs + 2 * pr);
     const int64_t dst = __ldg(pairs + 2 * pr + 1);
-    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+    if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
       if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(status, PA_DEVERR_PAIR);
       continue;
     }
-    const uint4* ks = k_cache + src * chunks_per_block;
-    const uint4* vs = v_cache + src * chunks_per_block;
-    uint4* kd = k_cache + dst * chunks_per_block;
-    uint4* vd = v_cache + dst * chunks_per_block;
+    const uint4* ks = src_k + src * chunks_per_block;
+    const uint4* vs = src_v + src * chunks_per_block;
+    uint4* kd = dst_k + dst * chunks_per_block;
+    uint4* vd = dst_v + dst * chunks_per_block;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < chunks_per_block;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
       kd[i] = ks[i];
@@ -116,8 +123,9 @@ int launch_reshape_and_cache(const void* key, const void* value, void* k_cache, 
   return cudaGetLastError();
 }
 
-int launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_pairs, int Hkv,
-                       int D, int block_size, int num_blocks, int esize, unsigned int* status,
+int launch_copy_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                       const int64_t* pairs, int num_pairs, int Hkv, int D, int block_size,
+                       int src_blocks, int dst_blocks, int esize, unsigned int* status,
                        void* stream) {
   const int64_t chunks = static_cast<int64_t>(Hkv) * block_size * D * esize / 16;
   const int threads = 256;
@@ -127,8 +135,8 @@ int launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int n
   const int gy = num_pairs < 65535 ? num_pairs : 65535;
   dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
   copy_blocks_kernel<<<grid, threads, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), pairs, num_pairs, chunks,
-      num_blocks, status);
+      static_cast<uint4*>(dst_k), static_cast<uint4*>(dst_v), static_cast<const uint4*>(src_k),
+      static_cast<const uint4*>(src_v), pairs, num_pairs, chunks, src_blocks, dst_blocks, status);
   return cudaGetLastError();
 }
 

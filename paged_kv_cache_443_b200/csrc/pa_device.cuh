@@ -57,14 +57,15 @@ __device__ __forceinline__ unsigned long long global_ns() {
 }
 
 // Waits for the phase of `bar` with the given parity to complete.  Bounded:
-// after kWaitTimeoutNs (or 2^31 polls) it sets PA_DEVERR_TIMEOUT in *status and
+// after `limit_ns` (or 2^31 polls) it sets PA_DEVERR_TIMEOUT in *status and
 // returns false, so a broken pipeline ends the kernel instead of hanging it.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* status) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* status,
+                                          unsigned long long limit_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t i = 1; i < 0x80000000u; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 127u) == 0 && global_ns() - t0 > kWaitTimeoutNs) break;
+    if ((i & 127u) == 0 && global_ns() - t0 > limit_ns) break;
   }
   atomicOr(status, PA_DEVERR_TIMEOUT);
   return false;

@@ -74,8 +74,9 @@ int launch_reshape_and_cache(const void* key, const void* value, void* k_cache, 
                              const int64_t* slot_mapping, int num_tokens, int Hkv, int D,
                              int block_size, int num_blocks, int esize, unsigned int* status,
                              void* stream);
-int launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_pairs, int Hkv,
-                       int D, int block_size, int num_blocks, int esize, unsigned int* status,
+int launch_copy_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                       const int64_t* pairs, int num_pairs, int Hkv, int D, int block_size,
+                       int src_blocks, int dst_blocks, int esize, unsigned int* status,
                        void* stream);
 
 // Launches `kernel` on `stream` allowing it to overlap the tail of the previous

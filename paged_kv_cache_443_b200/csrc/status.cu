@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <mutex>
 
+#include "pa_device.cuh"
 #include "pa_internal.h"
 
 namespace pa {
@@ -16,6 +17,18 @@ namespace {
 __device__ unsigned int g_status_word;
 
 thread_local char g_last_error[512] = "";
+
+// One CTA waits on an mbarrier that expects an arrival nothing makes, with a
+// short limit: the wait must give up, record PA_DEVERR_TIMEOUT and return.
+__global__ void wait_timeout_selftest_kernel(unsigned int* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  mbar_wait(&bar, 0, status, limit_ns);
+}
 std::atomic<uint64_t> g_launches{0};
 
 constexpr int kMaxDevices = 64;
@@ -78,6 +91,27 @@ extern "C" pa_status pa_device_status(unsigned int* flags_out, int clear) {
     e = cudaMemcpyToSymbol(pa::g_status_word, &zero, sizeof(zero));
     if (e != cudaSuccess)
       return pa::fail(PA_ERR_CUDA, "pa_device_status: %s", cudaGetErrorString(e));
+  }
+  return PA_OK;
+}
+
+extern "C" pa_status pa_selftest_wait_timeout(unsigned int* flags_out) {
+  if (!flags_out) return pa::fail(PA_ERR_INVALID, "pa_selftest_wait_timeout: flags_out is NULL");
+  unsigned int* status = pa::device_status_word();
+  if (!status) return PA_ERR_CUDA;
+  unsigned int before = 0;
+  pa_status st = pa_device_status(&before, 1);
+  if (st != PA_OK) return st;
+  pa::wait_timeout_selftest_kernel<<<1, 32>>>(status, 20000000ull);  // 20 ms
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess)
+    return pa::fail(PA_ERR_CUDA, "pa_selftest_wait_timeout: %s", cudaGetErrorString(e));
+  pa::count_launch();
+  st = pa_device_status(flags_out, 1);
+  if (st != PA_OK) return st;
+  if (before) {  // keep what the caller had not read yet
+    const unsigned int merged = before;
+    cudaMemcpyToSymbol(pa::g_status_word, &merged, sizeof(merged));
   }
   return PA_OK;
 }

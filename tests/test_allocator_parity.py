@@ -122,3 +122,78 @@ def test_workload_scripts_match_oracle(name):
     ta, la = a.build_tables(sc.batch, sc.max_blocks)
     to, lo = o.build_tables(sc.batch, sc.max_blocks)
     assert np.array_equal(ta, to) and np.array_equal(la, lo)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_random_moves_between_two_managers_match_oracle(seed):
+    """A device pool and a host pool on each side; sequences grow, fork, free
+    and move back and forth in random groups.  Copy pairs, tables, refcounts,
+    free stacks and OOM outcomes equal on both sides after every operation."""
+    rng = np.random.default_rng(2000 + seed)
+    for trial in range(6):
+        bs = int(rng.choice([1, 2, 4, 16]))
+        sizes = [int(rng.integers(6, 40)), int(rng.integers(3, 30))]
+        orders = [rng.permutation(n).tolist() for n in sizes]
+        A = [pk.BlockAllocator(n, bs, o) for n, o in zip(sizes, orders)]
+        O = [BlockManager(n, bs, o) for n, o in zip(sizes, orders)]
+        next_id = 0
+        for _ in range(120):
+            side = int(rng.integers(0, 2))
+            a, o = A[side], O[side]
+            live = sorted(o.seqs)
+            r = rng.random()
+            if r < 0.15 or not live:
+                a.add(next_id); o.add(next_id)
+                next_id += 1
+            elif r < 0.3:
+                p = int(rng.choice(live))
+                a.fork(p, next_id); o.fork(p, next_id)
+                next_id += 1
+            elif r < 0.6:
+                sid = int(rng.choice(live))
+                n = int(rng.integers(0, 2 * bs + 2))
+                try:
+                    want = o.append(sid, n)
+                except OOM:
+                    with pytest.raises(pk.OutOfBlocks):
+                        a.append(sid, n)
+                else:
+                    got = a.append(sid, n)
+                    assert got[0] == want[0] and [tuple(x) for x in got[1]] == want[1]
+            elif r < 0.9:
+                k = int(rng.integers(1, len(live) + 1))
+                group = [int(x) for x in rng.choice(live, size=k, replace=False)]
+                try:
+                    want = o.move_to(O[1 - side], group)
+                except OOM:
+                    with pytest.raises(pk.OutOfBlocks):
+                        a.move_to(A[1 - side], group)
+                else:
+                    got = a.move_to(A[1 - side], group)
+                    assert [tuple(x) for x in got] == [tuple(x) for x in want]
+            else:
+                sid = int(rng.choice(live))
+                a.release(sid); o.release(sid)
+            for s_ in (0, 1):
+                same_state(A[s_], O[s_], sorted(O[s_].seqs))
+
+
+def test_move_errors_map_to_statuses():
+    a, b = pk.BlockAllocator(8, 4), pk.BlockAllocator(2, 4)
+    a.add(0)
+    a.append(0, 9)
+    snap = (a.free_stack(), b.free_stack())
+    with pytest.raises(pk.OutOfBlocks):
+        a.move_to(b, [0])
+    for bad in ([0, 0], [7]):
+        with pytest.raises(pk.PagedKVError):
+            a.move_to(b, bad)
+    with pytest.raises(pk.PagedKVError):
+        a.move_to(a, [0])
+    with pytest.raises(pk.PagedKVError):
+        a.move_to(pk.BlockAllocator(8, 2), [0])
+    c = pk.BlockAllocator(8, 4)
+    with pytest.raises(pk.PagedKVError):   # capacity below the distinct blocks
+        pk.pa_seq_move(a.h, c.h, [0], 2)
+    assert snap == (a.free_stack(), b.free_stack()) and a.num_tokens(0) == 9
+    assert a.move_to(b, []) == []

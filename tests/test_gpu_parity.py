@@ -16,7 +16,7 @@ import oracle
 import paged_kv_cache_443_b200 as pk
 import workloads as W
 from pa_harness import (TOL, as_f64, build, check_bookkeeping, check_caches, check_token_slots,
-                        oracle_attention, run_step)
+                        oracle_attention, poison_bits, run_step)
 
 pytestmark = pytest.mark.gpu
 
@@ -144,10 +144,104 @@ def test_device_checks_flag_bad_values_without_faulting():
     # copy pair outside the pool
     cache.copy_on_write(torch.tensor([[0, cache.num_blocks]], dtype=torch.int64, device="cuda"))
     assert pk.pa_device_status() & pk.PA_DEVERR_PAIR
+    # swap pair outside the (smaller) destination pool
+    hk = torch.zeros((4,) + tuple(cache.k_cache.shape[1:]), dtype=cache.dtype, device="cuda")
+    hv = torch.zeros_like(hk)
+    pk.pa_swap_blocks(hk, hv, cache.k_cache, cache.v_cache,
+                      torch.tensor([[0, 4]], dtype=torch.int64, device="cuda"))
+    assert pk.pa_device_status() & pk.PA_DEVERR_PAIR
+    assert not hk.any()
     # the context is still healthy
     run_step(p, spec)
     torch.cuda.synchronize()
     assert pk.pa_device_status() == 0
+
+
+def test_bounded_wait_gives_up_and_context_survives():
+    """A pipeline wait that nothing will satisfy returns after its limit with
+    PA_DEVERR_TIMEOUT set; the device stays usable (no trap, no hang)."""
+    flags = pk.pa_selftest_wait_timeout()
+    assert flags & pk.PA_DEVERR_TIMEOUT
+    assert pk.pa_device_status() == 0
+    spec = W.small("opt13b")
+    full_check(spec)
+
+
+@pytest.mark.parametrize("name", ["tiny", "llama13b_ps"])
+def test_swap_blocks_match_oracle(name):
+    """Device -> pinned host -> second device pool, against the oracle's swap of
+    the oracle's own caches: every byte of all three pools equal.  The pairs of
+    the first copy live in pinned host memory, those of the second on the device."""
+    spec = W.small(name)
+    p, o = build(W.scenario(spec))
+    run_step(p, spec)
+    torch.cuda.synchronize()
+    NB = p.cache.num_blocks
+    rng = np.random.default_rng(3)
+    nb_host, nb_dev2 = NB // 2 + 3, NB + 5
+    src = rng.choice(NB, size=NB // 2, replace=False)
+    out_pairs = np.stack([src, rng.permutation(nb_host)[:src.size]], 1).astype(np.int64)
+    in_pairs = np.stack([out_pairs[:, 1], rng.permutation(nb_dev2)[:src.size]], 1).astype(np.int64)
+    fill = W.poison_value(spec)
+    shape = tuple(p.cache.k_cache.shape[1:])
+    host = [torch.full((nb_host,) + shape, fill, dtype=p.cache.dtype).pin_memory() for _ in range(2)]
+    dev2 = [torch.full((nb_dev2,) + shape, fill, dtype=p.cache.dtype, device="cuda")
+            for _ in range(2)]
+    pk.pa_swap_blocks(host[0], host[1], p.cache.k_cache, p.cache.v_cache,
+                      torch.from_numpy(out_pairs).pin_memory())
+    pk.pa_swap_blocks(dev2[0], dev2[1], host[0], host[1],
+                      torch.from_numpy(in_pairs).cuda())
+    torch.cuda.synchronize()
+    assert pk.pa_device_status() == 0
+    oh = [np.full((nb_host,) + shape, poison_bits(spec)) for _ in range(2)]
+    od = [np.full((nb_dev2,) + shape, poison_bits(spec)) for _ in range(2)]
+    oracle.swap_blocks(oh[0], oh[1], o.k, o.v, out_pairs, spec.dtype_code)
+    oracle.swap_blocks(od[0], od[1], oh[0], oh[1], in_pairs, spec.dtype_code)
+    for got, want in zip(host + dev2, oh + od):
+        assert W.storage_view(got).tobytes() == want.tobytes()
+    check_caches(p, o)       # the source pool is unchanged
+
+
+def test_swap_out_and_in_keeps_attention():
+    """Swap two whole sampling families and two samples of a third to the pinned
+    host pool, poison every free device block, swap back into fresh blocks:
+    decode output bit-identical to before and within tolerance of the oracle.
+    Blocks shared among the moved samples stay shared; the two lone samples
+    come back with private copies of their prompt."""
+    spec = W.small("llama13b_ps")
+    sc = W.scenario(spec)
+    p, o = build(sc)
+    before = run_step(p, spec).clone()
+    cache = p.cache
+    cache.enable_swap(cache.num_blocks)
+    moved = [0, 1, 2, 3, 4, 5, 12, 13, 14, 15, 16, 17, 7, 9]
+    out_pairs = cache.swap_out(moved)
+    assert len({d for _, d in out_pairs}) == len(out_pairs)
+    free_ids = torch.tensor(sorted(cache.alloc.free_stack()), dtype=torch.int64, device="cuda")
+    cache.k_cache.index_fill_(0, free_ids, float("nan"))
+    cache.v_cache.index_fill_(0, free_ids, float("nan"))
+    in_pairs = cache.swap_in(moved)
+    assert len(in_pairs) == len(out_pairs) and cache.host_alloc.num_free() == cache.num_blocks
+    tables, lens, max_ctx = cache.tables(sc.batch, sc.max_blocks)
+    assert torch.equal(lens, p.lens)
+    assert not torch.equal(tables, p.tables)
+    t, t0 = tables.cpu().numpy(), p.tables.cpu().numpy()
+
+    def same_block(tab, rows):
+        x = np.where(tab[rows] >= 0, tab[rows], -1 - np.arange(tab[rows].size).reshape(len(rows), -1))
+        return x.reshape(-1)[:, None] == x.reshape(-1)[None, :]
+
+    for fam in ([0, 1, 2, 3, 4, 5], [12, 13, 14, 15, 16, 17]):
+        assert np.array_equal(same_block(t, fam), same_block(t0, fam))
+    held = {int(b) for r in (6, 8, 10, 11) for b in t[r] if b >= 0}
+    assert not held & {int(b) for r in (7, 9) for b in t[r] if b >= 0}
+    after = cache.decode(p.q, tables, lens, max_ctx, spec.softmax_scale,
+                         partition_size=spec.partition_size)
+    torch.cuda.synchronize()
+    assert pk.pa_device_status() == 0
+    assert torch.equal(before.view(torch.int16), after.view(torch.int16))
+    err = np.abs(as_f64(after, spec) - oracle_attention(o, spec)).max()
+    assert err <= TOL[spec.dtype]
 
 
 def test_launch_counter_counts_kernels():

@@ -185,3 +185,118 @@ def test_random_operation_sequences_keep_invariants():
         for sid in list(bm.seqs):
             bm.release(sid)
         assert bm.num_free() == NB
+
+
+# ---------------------------------------------------------------------------
+# moving sequences to a second manager (swap to host memory and back)
+
+
+def _sharing(bm, seqs):
+    """Which (sequence, logical block) positions hold the same physical block:
+    the equivalence classes, independent of the ids themselves."""
+    first = {}
+    out = []
+    for sid in seqs:
+        row = []
+        for blk in bm.blocks_of(sid):
+            row.append(first.setdefault(blk, len(first)))
+        out.append(row)
+    return out
+
+
+def test_move_keeps_sharing_among_moved_sequences():
+    bs = 4
+    dev = BlockManager(32, bs)
+    host = BlockManager(16, bs)
+    dev.add(0)
+    dev.append(0, 10)                      # 2 full + 1 partial block
+    for c in (1, 2, 3):
+        dev.fork(0, c)
+    dev.append(1, 1)                       # copy-on-write of the partial block
+    free_before = dev.num_free()
+    pattern = _sharing(dev, [1, 2, 3])
+    pairs = dev.move_to(host, [1, 2, 3])
+    # distinct blocks of 1, 2, 3: the two full prompt blocks, the shared partial
+    # block (held by 0, 2, 3) and 1's private copy
+    assert len(pairs) == 4 and host.num_free() == 12
+    assert _sharing(host, [1, 2, 3]) == pattern
+    assert [host.num_tokens(s) for s in (1, 2, 3)] == [11, 10, 10]
+    for blk in host.blocks_of(2):
+        assert host.refcount[blk] == (3 if blk in host.blocks_of(1) else 2)
+    # device: 1's private block freed; the prompt blocks now held by 0 alone
+    assert dev.num_free() == free_before + 1
+    assert all(dev.refcount[b] == 1 for b in dev.blocks_of(0))
+    assert sorted(dev.seqs) == [0]
+    # every pair copies a block one of the moved sequences held, into the block
+    # that takes its place in the same logical position
+    src_of = dict((d, s) for s, d in pairs)
+    assert len(src_of) == len(pairs)
+
+
+def test_move_there_and_back_restores_contents_and_sharing():
+    """Track block contents as labels: after a round trip every sequence reads
+    the same labels in logical order, and the sharing pattern is unchanged."""
+    rng = np.random.default_rng(11)
+    bs = 2
+    dev = BlockManager(40, bs, rng.permutation(40).tolist())
+    host = BlockManager(40, bs, rng.permutation(40).tolist())
+    dev.add(0)
+    dev.append(0, 7)
+    dev.fork(0, 1)
+    dev.fork(0, 2)
+    dev.append(2, 3)
+    dev.add(5)
+    dev.append(5, 4)
+    label_dev = {b: ("d", b) for b in range(40)}
+    before = {s: [label_dev[b] for b in dev.blocks_of(s)] for s in (0, 1, 2, 5)}
+    pattern = _sharing(dev, [1, 2, 5])
+    out_pairs = dev.move_to(host, [1, 2, 5])
+    label_host = {}
+    for s_blk, d_blk in out_pairs:
+        label_host[d_blk] = label_dev[s_blk]
+    for s in (1, 2, 5):
+        assert [label_host[b] for b in host.blocks_of(s)] == before[s]
+    in_pairs = host.move_to(dev, [5, 2, 1])
+    for s_blk, d_blk in in_pairs:
+        label_dev[d_blk] = label_host[s_blk]
+    for s in (0, 1, 2, 5):
+        assert [label_dev[b] for b in dev.blocks_of(s)] == before[s]
+    assert _sharing(dev, [1, 2, 5]) == pattern
+    assert host.num_free() == 40 and not host.seqs
+    _check_invariants(dev)
+    _check_invariants(host)
+
+
+def test_move_single_sample_takes_private_copies():
+    dev = BlockManager(16, 4)
+    host = BlockManager(16, 4)
+    dev.add(0)
+    dev.append(0, 8)
+    dev.fork(0, 1)
+    pairs = dev.move_to(host, [1])
+    assert [s for s, _ in pairs] == dev.blocks_of(0)
+    assert all(host.refcount[b] == 1 for b in host.blocks_of(1))
+    assert all(dev.refcount[b] == 1 for b in dev.blocks_of(0))
+
+
+def test_move_errors_change_nothing():
+    dev = BlockManager(8, 4)
+    host = BlockManager(2, 4)
+    dev.add(0)
+    dev.append(0, 9)                       # 3 blocks > 2 free in host
+    snap = (dev.free_stack(), list(dev.refcount), host.free_stack())
+    with pytest.raises(OOM):
+        dev.move_to(host, [0])
+    with pytest.raises(Invalid):
+        dev.move_to(host, [0, 0])
+    with pytest.raises(Invalid):
+        dev.move_to(host, [7])
+    with pytest.raises(Invalid):
+        dev.move_to(dev, [0])
+    with pytest.raises(Invalid):
+        dev.move_to(BlockManager(8, 2), [0])
+    host.add(0)
+    with pytest.raises(Invalid):
+        dev.move_to(host, [0])
+    assert snap == (dev.free_stack(), list(dev.refcount), host.free_stack())
+    assert dev.num_tokens(0) == 9

@@ -451,3 +451,37 @@ def test_pins_catch_planted_mistakes(mistake):
     bad = _mutant_attention(q, kc, vc, tables, lens, 0.25, mistake=mistake)
     caught = (not np.all(np.isfinite(bad))) or np.abs(bad - want).max() > 1e-6
     assert caught, mistake
+
+
+def test_swap_out_and_back_in_restores_attention():
+    """"적용 범위와 관련 연구": a sequence swapped out to host memory and back in
+    (into other physical blocks) attends exactly as before; the host copy holds
+    the blocks' bytes, and blocks not named are untouched."""
+    rng = np.random.default_rng(31)
+    q, Ks, Vs, nb = random_case(rng, 3, 4, 2, 16, 8, 60, lmin=20)
+    kc, vc, t, l = paged_from_contiguous(Ks, Vs, 8, nb + 20, rng)
+    before = oracle.paged_attention(q, kc, vc, oracle.F32, t, l, 0.25)
+    b = 1
+    blocks = [int(x) for x in t[b, : -(-int(l[b]) // 8)]]
+    host_k = np.zeros((len(blocks) + 3,) + kc.shape[1:], dtype=np.float32)
+    host_v = host_k.copy()
+    out_pairs = np.array([[blk, i + 3] for i, blk in enumerate(blocks)])
+    oracle.swap_blocks(host_k, host_v, kc, vc, out_pairs, oracle.F32)
+    for i, blk in enumerate(blocks):
+        assert host_k[i + 3].tobytes() == kc[blk].tobytes()
+    assert np.all(host_k[:3] == 0)
+    # the device blocks are recycled: poison them, then swap back into fresh ids
+    used = set(int(x) for x in t[t >= 0])
+    free = [x for x in range(kc.shape[0]) if x not in used]
+    kc[blocks] = np.nan
+    vc[blocks] = np.nan
+    new_ids = free[: len(blocks)]
+    oracle.swap_blocks(kc, vc, host_k, host_v,
+                       np.array([[i + 3, nid] for i, nid in enumerate(new_ids)]), oracle.F32)
+    t2 = t.copy()
+    t2[b, : len(blocks)] = new_ids
+    after = oracle.paged_attention(q, kc, vc, oracle.F32, t2, l, 0.25)
+    assert np.array_equal(before[b], after[b])
+    assert np.array_equal(np.delete(before, b, 0), np.delete(after, b, 0))
+    with pytest.raises(ValueError):
+        oracle.swap_blocks(host_k, host_v, kc, vc, np.array([[0, host_k.shape[0]]]), oracle.F32)

@@ -23,8 +23,8 @@ import numpy as np
 
 from . import build as _build
 
-F32, F16, BF16 = 0, 1, 2
-_NP_STORAGE = {F32: np.float32, F16: np.uint16, BF16: np.uint16}
+F32, F16, BF16, E4M3 = 0, 1, 2, 3
+_NP_STORAGE = {F32: np.float32, F16: np.uint16, BF16: np.uint16, E4M3: np.uint8}
 
 _lib = None
 
@@ -45,6 +45,16 @@ def lib():
         L.or_paged_attention.argtypes = [p, p, i64, p, p, p, i32, p, i32, p,
                                          i32, i32, i32, i32, i32, i32, dbl, i32]
         L.or_paged_attention.restype = i32
+        L.or_paged_attention_kv.argtypes = [p, p, i64, p, p, p, i32, i32, dbl, dbl, p, i32, p,
+                                            i32, i32, i32, i32, i32, i32, dbl, i32]
+        L.or_paged_attention_kv.restype = i32
+        L.or_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        L.or_e4m3_to_f64.restype = dbl
+        L.or_encode_e4m3.argtypes = [p, p, i64]
+        L.or_encode_e4m3.restype = None
+        L.or_reshape_and_cache_e4m3.argtypes = [p, p, p, p, p, i64, i32, i32, i32, i64, i32,
+                                                ctypes.c_float, ctypes.c_float]
+        L.or_reshape_and_cache_e4m3.restype = i32
         L.or_reshape_and_cache.argtypes = [p, p, p, p, p, i64, i32, i32, i32, i64, i32]
         L.or_reshape_and_cache.restype = i32
         L.or_copy_blocks.argtypes = [p, p, p, i64, i32, i32, i32, i64, i32]
@@ -78,14 +88,24 @@ def decode(storage: np.ndarray, dtype: int) -> np.ndarray:
     return out.reshape(storage.shape)
 
 
+def encode_e4m3(values) -> np.ndarray:
+    """Nearest OCP E4M3 codes (ties to even, saturating at +-448) of float64 values."""
+    v = np.ascontiguousarray(values, dtype=np.float64)
+    out = np.empty(v.shape, dtype=np.uint8)
+    lib().or_encode_e4m3(_ptr(out), _ptr(v), v.size)
+    return out
+
+
 def paged_attention(q, k_cache, v_cache, dtype, block_tables, context_lens, scale,
-                    rows=None, nthreads=None):
+                    rows=None, nthreads=None, kv_dtype=None, k_scale=1.0, v_scale=1.0):
     """Decode attention over the paged cache, fp64, for every (b, h) or for ``rows``.
 
     q: [B, Hq, D] storage array (float32, or uint16 bit patterns for fp16/bf16);
     k_cache, v_cache: [num_blocks, Hkv, block_size, D] storage arrays;
     block_tables: [B, max_blocks] int32; context_lens: [B] int32;
     rows: optional [n, 2] int64 array of (b, h).  Returns [B, Hq, D] or [n, D] float64.
+    kv_dtype: storage type of the caches when it differs from q's (E4M3 codes,
+    uint8), whose elements stand for decode(code) * k_scale / * v_scale.
 
     Follows "자기회귀 생성과 KV 캐시" (scores q.k/sqrt(d_k), softmax over valid
     past positions, weighted sum of V) and "PagedAttention의 설계" (gather
@@ -105,9 +125,11 @@ def paged_attention(q, k_cache, v_cache, dtype, block_tables, context_lens, scal
         out = np.zeros((B, Hq, D), dtype=np.float64)
         n = B * Hq
     nt = max_threads() if nthreads is None else int(nthreads)
-    rc = lib().or_paged_attention(_ptr(out), _ptr(rows), n, _ptr(q), _ptr(k_cache), _ptr(v_cache),
-                                  dtype, _ptr(block_tables), block_tables.shape[1],
-                                  _ptr(context_lens), B, Hq, Hkv, D, bs, NB, float(scale), nt)
+    kvd = dtype if kv_dtype is None else kv_dtype
+    rc = lib().or_paged_attention_kv(_ptr(out), _ptr(rows), n, _ptr(q), _ptr(k_cache),
+                                     _ptr(v_cache), dtype, kvd, float(k_scale), float(v_scale),
+                                     _ptr(block_tables), block_tables.shape[1],
+                                     _ptr(context_lens), B, Hq, Hkv, D, bs, NB, float(scale), nt)
     if rc != 0:
         raise ValueError("oracle: input out of range")
     return out
@@ -128,6 +150,25 @@ def reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, dtype):
                                     _ptr(slot_mapping), slot_mapping.size, Hkv, D, bs, NB, dtype)
     if rc != 0:
         raise ValueError("oracle: slot out of range")
+
+
+def reshape_and_cache_e4m3(key, value, k_cache, v_cache, slot_mapping, dtype, k_scale, v_scale):
+    """Store the new tokens' K and V as E4M3 codes of x / scale (quotient in fp32).
+
+    key, value: [N, Hkv, D] storage arrays of dtype (f32 / f16 / bf16); caches
+    uint8 [num_blocks, Hkv, block_size, D], modified in place.  The precision
+    reading for "quantization" of "4. 이 밖의 기법들" (blog.aqudi.me).
+    """
+    key, value = _c(key), _c(value)
+    slot_mapping = _c(slot_mapping, np.int64)
+    assert k_cache.dtype == np.uint8 and v_cache.dtype == np.uint8
+    assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
+    NB, Hkv, bs, D = k_cache.shape
+    rc = lib().or_reshape_and_cache_e4m3(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
+                                         _ptr(slot_mapping), slot_mapping.size, Hkv, D, bs, NB,
+                                         dtype, float(k_scale), float(v_scale))
+    if rc != 0:
+        raise ValueError("oracle: slot out of range or bad scale")
 
 
 def copy_blocks(k_cache, v_cache, pairs, dtype):

@@ -36,7 +36,13 @@
  *   - cache layout [num_blocks][Hkv][block_size][D]; token j of a sequence sits in
  *     physical block block_tables[b][j / block_size] at offset j % block_size;
  *   - a sequence with context length 0 produces an all-zero output row;
- *   - copy-on-write pairs are applied in the given order.
+ *   - copy-on-write pairs are applied in the given order;
+ *   - a lower-precision KV cache ("quantization" in "4. 이 밖의 기법들",
+ *     blog.aqudi.me, which names no format): 8-bit OCP E4M3 codes with one
+ *     scale per cache (k_scale, v_scale); the stored code of x is
+ *     E4M3(fp32(x) / fp32(scale)), the quotient rounded once in fp32, then to
+ *     the nearest E4M3 value (ties to an even fraction), magnitudes above 448
+ *     saturating to 448; a code stands for decode(code) * scale.
  */
 #include <math.h>
 #include <stdint.h>
@@ -47,7 +53,7 @@
 #include <omp.h>
 #endif
 
-enum { OR_F32 = 0, OR_F16 = 1, OR_BF16 = 2 };
+enum { OR_F32 = 0, OR_F16 = 1, OR_BF16 = 2, OR_E4M3 = 3 };
 
 /* ---- element decoders (IEEE 754 binary16 and bfloat16 by field arithmetic) ---- */
 
@@ -83,17 +89,69 @@ double or_bf16_to_f64(uint16_t bits) {
   return sign ? -v : v;
 }
 
+/* OCP 8-bit floating point, E4M3: 1 sign bit, 4 exponent bits (bias 7), 3
+ * fraction bits; exponent field 0 is subnormal (f * 2^-9); there are no
+ * infinities and S.1111.111 is NaN, so the largest finite value is
+ * 1.75 * 2^8 = 448. */
+double or_e4m3_to_f64(uint8_t bits) {
+  int sign = (bits >> 7) & 1;
+  int e = (bits >> 3) & 0xf;
+  int f = bits & 0x7;
+  double v;
+  if (e == 15 && f == 7) {
+    v = NAN;
+  } else if (e == 0) {
+    v = ldexp((double)f, -9); /* f/8 * 2^(1-7) */
+  } else {
+    v = ldexp((double)(f + 8), e - 10); /* (1 + f/8) * 2^(e-7) */
+  }
+  return sign ? -v : v;
+}
+
+/* Nearest E4M3 code to v (ties to an even fraction field), |v| > 448 and
+ * infinities saturating to +-448, NaN to 0x7f.  Works on the exact value: the
+ * spacing of E4M3 values around v is a power of two, so v / spacing is exact
+ * in double and only the final rounding to an integer decides. */
+uint8_t or_f64_to_e4m3(double v) {
+  if (isnan(v)) return 0x7f;
+  const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+  double a = fabs(v);
+  if (a >= 448.0) return sign | 0x7e;
+  int e; /* a = m * 2^e with m in [0.5, 1) */
+  frexp(a, &e);
+  int unbiased = e - 1; /* a in [2^unbiased, 2^(unbiased+1)) */
+  if (a == 0.0 || unbiased < -6) unbiased = -6; /* subnormal range: spacing 2^-9 */
+  const double spacing = ldexp(1.0, unbiased - 3);
+  const double q = a / spacing; /* exact */
+  double n = floor(q);
+  const double rest = q - n;
+  if (rest > 0.5 || (rest == 0.5 && fmod(n, 2.0) != 0.0)) n += 1.0;
+  /* n counts spacings: in the normal range 8..16 (16 carries into the next
+   * binade), in the subnormal range 0..8 (8 is the smallest normal) */
+  const double r = n * spacing;
+  if (r >= 448.0) return sign | 0x7e; /* cannot exceed: 448 is on the grid */
+  if (r < ldexp(1.0, -6)) return sign | (uint8_t)n; /* subnormal code = fraction */
+  int re;
+  frexp(r, &re);
+  const int be = re - 1 + 7; /* biased exponent */
+  const int frac = (int)(ldexp(r, -(re - 1)) * 8.0) - 8;
+  return sign | (uint8_t)((be << 3) | frac);
+}
+
 int or_elem_size(int dtype) {
   switch (dtype) {
     case OR_F32: return 4;
     case OR_F16: return 2;
     case OR_BF16: return 2;
+    case OR_E4M3: return 1;
     default: return 0;
   }
 }
 
-/* Value of element idx of an array of the given storage type. */
+/* Value of element idx of an array of the given storage type (an E4M3 code
+ * without its scale). */
 static double load_elem(const void* base, int dtype, size_t idx) {
+  if (dtype == OR_E4M3) return or_e4m3_to_f64(((const uint8_t*)base)[idx]);
   if (dtype == OR_F32) {
     float x;
     memcpy(&x, (const char*)base + 4 * idx, 4);
@@ -107,6 +165,11 @@ static double load_elem(const void* base, int dtype, size_t idx) {
 /* Decode n elements (test helper: lets the tests pin the decoders directly). */
 void or_decode(double* out, const void* src, int dtype, int64_t n) {
   for (int64_t i = 0; i < n; ++i) out[i] = load_elem(src, dtype, (size_t)i);
+}
+
+/* Encode n values as E4M3 codes (test helper for the encoder pins). */
+void or_encode_e4m3(uint8_t* out, const double* src, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = or_f64_to_e4m3(src[i]);
 }
 
 /* ---- attention over the paged cache ----
@@ -126,12 +189,13 @@ void or_decode(double* out, const void* src, int dtype, int64_t n) {
  * [0, num_blocks), a context length < 0 or beyond max_blocks * block_size, a
  * head count that does not divide, a row outside [0,B) x [0,Hq)).
  */
-int or_paged_attention(double* out, const int64_t* rows, int64_t nrows, const void* q,
-                       const void* k_cache, const void* v_cache, int dtype,
-                       const int32_t* block_tables, int max_blocks, const int32_t* context_lens,
-                       int B, int Hq, int Hkv, int D, int block_size, int num_blocks,
-                       double scale, int nthreads) {
-  if (Hkv <= 0 || Hq % Hkv != 0 || or_elem_size(dtype) == 0 || block_size <= 0 || D <= 0)
+int or_paged_attention_kv(double* out, const int64_t* rows, int64_t nrows, const void* q,
+                          const void* k_cache, const void* v_cache, int dtype, int kv_dtype,
+                          double k_scale, double v_scale, const int32_t* block_tables,
+                          int max_blocks, const int32_t* context_lens, int B, int Hq, int Hkv,
+                          int D, int block_size, int num_blocks, double scale, int nthreads) {
+  if (Hkv <= 0 || Hq % Hkv != 0 || or_elem_size(dtype) == 0 || or_elem_size(kv_dtype) == 0 ||
+      dtype == OR_E4M3 || block_size <= 0 || D <= 0)
     return -1;
   const int G = Hq / Hkv;
   if (rows == NULL) nrows = (int64_t)B * Hq;
@@ -170,8 +234,8 @@ int or_paged_attention(double* out, const int64_t* rows, int64_t nrows, const vo
       }
       const size_t base = (size_t)(((phys * Hkv + g) * block_size + off) * D);
       for (int d = 0; d < D; ++d) {
-        K[j * D + d] = load_elem(k_cache, dtype, base + d);
-        V[j * D + d] = load_elem(v_cache, dtype, base + d);
+        K[j * D + d] = load_elem(k_cache, kv_dtype, base + d) * k_scale;
+        V[j * D + d] = load_elem(v_cache, kv_dtype, base + d) * v_scale;
       }
     }
     if (!row_bad) {
@@ -206,6 +270,17 @@ int or_paged_attention(double* out, const int64_t* rows, int64_t nrows, const vo
   return bad ? -1 : 0;
 }
 
+/* The same with a cache of the query's own type and unit scales. */
+int or_paged_attention(double* out, const int64_t* rows, int64_t nrows, const void* q,
+                       const void* k_cache, const void* v_cache, int dtype,
+                       const int32_t* block_tables, int max_blocks, const int32_t* context_lens,
+                       int B, int Hq, int Hkv, int D, int block_size, int num_blocks,
+                       double scale, int nthreads) {
+  return or_paged_attention_kv(out, rows, nrows, q, k_cache, v_cache, dtype, dtype, 1.0, 1.0,
+                               block_tables, max_blocks, context_lens, B, Hq, Hkv, D, block_size,
+                               num_blocks, scale, nthreads);
+}
+
 /* ---- appending the new tokens' K and V ----
  * Follows "1. KV 캐시란" (hjr-study-book Day 3: each step stores the new K, V
  * pair) and the slot arithmetic of the block-table example in "4.2
@@ -235,6 +310,39 @@ int or_reshape_and_cache(const void* key, const void* value, void* k_cache, void
       const size_t src = (size_t)((t * Hkv + h) * D) * es;
       memcpy((char*)k_cache + dst, (const char*)key + src, (size_t)D * es);
       memcpy((char*)v_cache + dst, (const char*)value + src, (size_t)D * es);
+    }
+  }
+  return 0;
+}
+
+/*
+ * The append into an E4M3 cache: for every t < N with slot = slot_mapping[t] >= 0
+ * and every h, d: k_cache[...][d] = E4M3(fp32(key[t][h][d]) / k_scale), the
+ * quotient rounded once in fp32 (the cache reading in the header); value alike
+ * with v_scale.  key/value are f32 / f16 / bf16 (dtype).  Returns -1 on a slot
+ * beyond the cache or a bad dtype / scale.
+ */
+int or_reshape_and_cache_e4m3(const void* key, const void* value, uint8_t* k_cache,
+                              uint8_t* v_cache, const int64_t* slot_mapping, int64_t N, int Hkv,
+                              int D, int block_size, int64_t num_blocks, int dtype,
+                              float k_scale, float v_scale) {
+  if (or_elem_size(dtype) == 0 || dtype == OR_E4M3) return -1;
+  if (!(k_scale > 0.0f) || !(v_scale > 0.0f) || isinf(k_scale) || isinf(v_scale)) return -1;
+  for (int64_t t = 0; t < N; ++t) {
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0) continue;
+    if (slot >= num_blocks * block_size) return -1;
+    const int64_t blk = slot / block_size;
+    const int64_t off = slot % block_size;
+    for (int64_t h = 0; h < Hkv; ++h) {
+      const size_t dst = (size_t)(((blk * Hkv + h) * block_size + off) * D);
+      const size_t src = (size_t)((t * Hkv + h) * D);
+      for (int d = 0; d < D; ++d) {
+        const float kq = (float)load_elem(key, dtype, src + d) / k_scale;
+        const float vq = (float)load_elem(value, dtype, src + d) / v_scale;
+        k_cache[dst + d] = or_f64_to_e4m3((double)kq);
+        v_cache[dst + d] = or_f64_to_e4m3((double)vq);
+      }
     }
   }
   return 0;

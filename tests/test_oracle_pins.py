@@ -485,3 +485,146 @@ def test_swap_out_and_back_in_restores_attention():
     assert np.array_equal(np.delete(before, b, 0), np.delete(after, b, 0))
     with pytest.raises(ValueError):
         oracle.swap_blocks(host_k, host_v, kc, vc, np.array([[0, host_k.shape[0]]]), oracle.F32)
+
+
+# ---------------------------------------------------------------------------
+# E4M3 KV cache: the format's fixed points, torch's own float8_e4m3fn casts,
+# brute-force nearest codes, and attention identities.
+
+
+def _all_codes():
+    return np.arange(256, dtype=np.uint8)
+
+
+def test_e4m3_fixed_points_of_the_format():
+    g = read_golden("e4m3_points.txt")
+    for name, vals in g.items():
+        code = vals[0]
+        v = oracle.decode(np.array([code], dtype=np.uint8), oracle.E4M3)[0]
+        if name == "nan":
+            assert np.isnan(v)
+            continue
+        assert v == vals[1], name
+        assert oracle.encode_e4m3(np.array([vals[1]]))[0] == code, name
+
+
+def test_e4m3_decode_matches_torch_for_every_code():
+    codes = _all_codes()
+    ours = oracle.decode(codes, oracle.E4M3)
+    theirs = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(theirs)
+    assert np.array_equal(np.isnan(ours), nan) and nan.sum() == 2
+    assert np.array_equal(ours[~nan], theirs[~nan])
+    # every finite code survives decode -> encode, -0 included
+    back = oracle.encode_e4m3(ours[~nan])
+    assert np.array_equal(back, codes[~nan])
+
+
+def test_e4m3_encode_matches_torch_cast_and_rounds_ties_to_even():
+    rng = np.random.default_rng(8)
+    finite = oracle.decode(_all_codes(), oracle.E4M3)
+    grid = np.unique(finite[np.isfinite(finite) & (finite >= 0)])       # 0 .. 448
+    mids = (grid[:-1] + grid[1:]) / 2                                     # exact ties
+    x = np.concatenate([
+        rng.standard_normal(50000) * 10.0 ** rng.uniform(-3, 2.4, 50000),
+        rng.uniform(-447.9, 447.9, 20000),
+        mids, -mids, np.nextafter(mids, 0), np.nextafter(mids, 1000), grid, -grid,
+    ]).astype(np.float32)
+    x = x[np.abs(x) < 448]
+    ours = oracle.encode_e4m3(x.astype(np.float64))
+    theirs = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, theirs)
+    # a tie goes to the neighbour whose fraction field is even
+    t = oracle.encode_e4m3(mids)
+    assert np.all((t & 1) == 0)
+
+
+def test_e4m3_saturates_instead_of_overflowing():
+    big = np.array([448.0, 449.0, 464.0, 479.9, 480.0, 1e6, np.inf])
+    assert np.all(oracle.encode_e4m3(big) == 0x7e)
+    assert np.all(oracle.encode_e4m3(-big) == 0xfe)
+
+
+def _nearest_code_brute_force(q):
+    """Nearest finite E4M3 value to each q by scanning all codes; ties to the
+    even fraction field; |q| beyond 448 to +-448."""
+    codes = _all_codes()
+    vals = oracle.decode(codes, oracle.E4M3)
+    ok = np.isfinite(vals)
+    codes, vals = codes[ok], vals[ok]
+    out = np.empty(q.shape, dtype=np.uint8)
+    for i, v in enumerate(q.ravel()):
+        v = min(max(float(v), -448.0), 448.0)
+        d = np.abs(vals - v)
+        best = np.flatnonzero(d == d.min())
+        cand = codes[best]
+        if len(cand) > 1:                       # +-0, or a tie between two codes
+            same = [c for c in cand if (c & 0x80) == (0x80 if np.signbit(v) else 0)]
+            cand = np.array(same or list(cand), dtype=np.uint8)
+            even = [c for c in cand if (c & 1) == 0]
+            cand = np.array(even or list(cand), dtype=np.uint8)
+        out.ravel()[i] = cand[0]
+    return out
+
+
+@pytest.mark.parametrize("dtype", [oracle.F32, oracle.F16, oracle.BF16])
+def test_e4m3_append_stores_nearest_code_of_the_fp32_quotient(dtype):
+    rng = np.random.default_rng(40 + dtype)
+    N, Hkv, D, bs, NB = 5, 2, 64, 8, 6
+    tdt = {oracle.F32: torch.float32, oracle.F16: torch.float16, oracle.BF16: torch.bfloat16}[dtype]
+    k = torch.from_numpy(rng.standard_normal((N, Hkv, D)) * 30).to(tdt)
+    v = torch.from_numpy(rng.standard_normal((N, Hkv, D)) * 0.01).to(tdt)
+    k[0, 0, :4] = torch.tensor([1e4, -1e4, 0.0, -0.0])             # saturate, signed zeros
+    k_scale, v_scale = np.float32(0.37), np.float32(1.0 / 64)
+    kc = np.zeros((NB, Hkv, bs, D), dtype=np.uint8)
+    vc = np.zeros_like(kc)
+    slots = np.array([3, 17, -1, 40, 0], dtype=np.int64)
+    st = lambda t: t.view(torch.int16).numpy().view(np.uint16) if t.dtype != torch.float32 else t.numpy()
+    oracle.reshape_and_cache_e4m3(st(k), st(v), kc, vc, slots, dtype, k_scale, v_scale)
+    kf = k.to(torch.float32).numpy()
+    vf = v.to(torch.float32).numpy()
+    for t, s in enumerate(slots):
+        if s < 0:
+            continue
+        blk, off = divmod(int(s), bs)
+        want_k = _nearest_code_brute_force(kf[t] / k_scale)       # float32 / float32
+        want_v = _nearest_code_brute_force(vf[t] / v_scale)
+        assert np.array_equal(kc[blk, :, off], want_k)
+        assert np.array_equal(vc[blk, :, off], want_v)
+    assert kc[0, 0, 3, :4].tolist() == [0x7e, 0xfe, 0x00, 0x80]     # token 0 sits in slot 3
+    # untouched slots stay as they were
+    assert kc[1].sum() == 0
+    with pytest.raises(ValueError):
+        oracle.reshape_and_cache_e4m3(st(k), st(v), kc, vc, slots, dtype, 0.0, 1.0)
+
+
+def test_e4m3_attention_identities():
+    """With power-of-two scales the E4M3 cache equals an f32 cache of
+    decode(code) * scale exactly, so the pinned f32 path must agree; with any
+    scale, v_scale scales the output and k_scale multiplies the softmax scale."""
+    rng = np.random.default_rng(12)
+    B, Hq, Hkv, D, bs, NB = 3, 4, 2, 64, 16, 12
+    codes_k = rng.integers(0, 256, (NB, Hkv, bs, D)).astype(np.uint8)
+    codes_v = rng.integers(0, 256, (NB, Hkv, bs, D)).astype(np.uint8)
+    for c in (codes_k, codes_v):                  # no NaN codes
+        c[(c & 0x7f) == 0x7f] = 0x3c
+    q = rng.standard_normal((B, Hq, D)).astype(np.float32) * 0.05
+    tables = rng.permutation(NB)[: B * 4].reshape(B, 4).astype(np.int32)
+    lens = np.array([1, 37, 64], dtype=np.int32)
+    scale = 1 / 8
+    dec = lambda c: torch.from_numpy(c).view(torch.float8_e4m3fn).to(torch.float32).numpy()
+    got = oracle.paged_attention(q, codes_k, codes_v, oracle.F32, tables, lens, scale,
+                                 kv_dtype=oracle.E4M3, k_scale=0.25, v_scale=2.0)
+    want = oracle.paged_attention(q, dec(codes_k) * np.float32(0.25), dec(codes_v) * np.float32(2.0),
+                                  oracle.F32, tables, lens, scale)
+    assert np.abs(got - want).max() <= 1e-12
+    a = oracle.paged_attention(q, codes_k, codes_v, oracle.F32, tables, lens, scale,
+                               kv_dtype=oracle.E4M3, k_scale=0.3, v_scale=0.7)
+    b = oracle.paged_attention(q, codes_k, codes_v, oracle.F32, tables, lens, scale * 0.3,
+                               kv_dtype=oracle.E4M3, k_scale=1.0, v_scale=1.0)
+    assert np.abs(a - 0.7 * b).max() <= 1e-12 * max(1.0, np.abs(a).max())
+    # a single token: the output is that token's dequantised V
+    one = oracle.paged_attention(q, codes_k, codes_v, oracle.F32, tables, lens, scale,
+                                 kv_dtype=oracle.E4M3, k_scale=0.3, v_scale=0.7)[0]
+    v0 = oracle.decode(codes_v[tables[0, 0], :, 0], oracle.E4M3) * 0.7
+    assert np.array_equal(one[:2], v0[0:1].repeat(2, 0)) and np.array_equal(one[2:], v0[1:2].repeat(2, 0))

@@ -52,6 +52,8 @@ FALLBACK_HBM_GBS = 6650.0
 
 
 def workload_spec(name):
+    if name.endswith("_fp8"):
+        return W.fp8(workload_spec(name[: -len("_fp8")]))
     if name.endswith("_quarter"):
         # a quarter of the sequences of a workload (same kernel, same per-sequence
         # shapes): the profiling case for captures that must stay small
@@ -80,6 +82,11 @@ WORKLOAD_TEXT = {
 
 
 def workload_text(name):
+    if name.endswith("_fp8"):
+        sp = workload_spec(name)
+        return (workload_text(name[: -len("_fp8")]) +
+                f"; cache of E4M3 codes (k_scale {sp.k_scale:.6g}, v_scale {sp.v_scale:.6g}), "
+                f"queries and outputs {sp.dtype}")
     if name.endswith("_quarter"):
         return workload_text(name[: -len("_quarter")]) + " (a quarter of the sequences)"
     if name == "opt13b_compact":
@@ -100,7 +107,7 @@ def step_bytes(spec, tables, lens, num_blocks_shared_ok=True):
     holding a valid token counted once (unique) and once per reader (logical),
     plus q, out, table and length bytes."""
     bs, es = spec.block_size, spec.esize
-    row = spec.Hkv * spec.D * es * 2          # K and V bytes of one token, all kv heads
+    row = spec.Hkv * spec.D * spec.kv_esize * 2   # K and V bytes of one token, all kv heads
     logical = int(lens.astype(np.int64).sum()) * row
     # unique: valid tokens of each distinct physical block
     used = {}
@@ -251,7 +258,8 @@ def partition_kernel(spec, P):
     tensor-core one for 4 or 8 query heads per kv head in fp16/bf16, head size
     128 and a partition length that is a multiple of 128; else CUDA cores."""
     G = spec.Hq // spec.Hkv
-    if spec.dtype in ("f16", "bf16") and spec.D == 128 and G in (4, 8) and P % 128 == 0:
+    if (not spec.fp8 and spec.dtype in ("f16", "bf16") and spec.D == 128 and G in (4, 8)
+            and P % 128 == 0):
         return "decode_partition_tc_kernel"
     return "decode_partition_kernel"
 
@@ -305,7 +313,7 @@ def oracle_sample_setup(spec, max_seqs=None):
     sp = replace(sp, num_blocks=None)
     sc = W.scenario(sp)
     shape = (sc.num_blocks, sp.Hkv, sp.block_size, sp.D)
-    st = np.float32 if sp.dtype == "f32" else np.uint16
+    st = {"f32": np.float32, "f16": np.uint16, "bf16": np.uint16, "e4m3": np.uint8}[sp.kv]
     kc = np.zeros(shape, dtype=st)
     vc = np.zeros(shape, dtype=st)
     bm = BlockManager(sc.num_blocks, sp.block_size, sc.free_order.tolist())
@@ -320,9 +328,14 @@ def oracle_sample_setup(spec, max_seqs=None):
             k, v = W.kv_content(sp, op.kv_id, op.arg, "cpu")
             slots, pairs = bm.append(op.seq, op.arg)
             if pairs:
-                oracle.copy_blocks(kc, vc, np.array(pairs), sp.dtype_code)
-            oracle.reshape_and_cache(W.storage_view(k), W.storage_view(v), kc, vc,
-                                     np.array(slots), sp.dtype_code)
+                oracle.copy_blocks(kc, vc, np.array(pairs), sp.kv_code)
+            if sp.fp8:
+                oracle.reshape_and_cache_e4m3(W.storage_view(k), W.storage_view(v), kc, vc,
+                                              np.array(slots), sp.dtype_code, sp.k_scale,
+                                              sp.v_scale)
+            else:
+                oracle.reshape_and_cache(W.storage_view(k), W.storage_view(v), kc, vc,
+                                         np.array(slots), sp.dtype_code)
     tables, lens = bm.build_tables(sc.batch, sc.max_blocks)
     q = W.storage_view(W.q_content(sp, len(sc.batch), "cpu"))
     return sp, q, kc, vc, tables, lens
@@ -337,13 +350,14 @@ def time_oracle(spec, budget_s=15.0, steps=None, per_step_budget_s=None):
     sp, q, kc, vc, tables, lens = oracle_sample_setup(spec, max_seqs)
     B = len(lens)
     rows_all = np.array([(b, h) for b in range(B) for h in range(sp.Hq)], dtype=np.int64)
-    row_bytes = lambda rows: int(sum(int(lens[b]) for b, _ in rows)) * sp.D * sp.esize * 2
+    row_bytes = lambda rows: int(sum(int(lens[b]) for b, _ in rows)) * sp.D * sp.kv_esize * 2
+    kv = dict(kv_dtype=sp.kv_code, k_scale=sp.k_scale, v_scale=sp.v_scale)
     # calibration on a few rows
     rng = np.random.default_rng(0)
     cal = rows_all[rng.choice(len(rows_all), size=min(len(rows_all), 4 * nthreads), replace=False)]
     t0 = time.perf_counter()
     oracle.paged_attention(q, kc, vc, sp.dtype_code, tables, lens, sp.softmax_scale, rows=cal,
-                           nthreads=nthreads)
+                           nthreads=nthreads, **kv)
     per_byte = (time.perf_counter() - t0) / max(1, row_bytes(cal))
     target = per_step_budget_s if per_step_budget_s is not None else budget_s
     n_rows = int(max(1, min(len(rows_all), target / max(per_byte * row_bytes(rows_all) / len(rows_all), 1e-9))))
@@ -353,7 +367,7 @@ def time_oracle(spec, budget_s=15.0, steps=None, per_step_budget_s=None):
         sel = rows_all[rng.choice(len(rows_all), size=n_rows, replace=False)]
         t0 = time.perf_counter()
         oracle.paged_attention(q, kc, vc, sp.dtype_code, tables, lens, sp.softmax_scale, rows=sel,
-                               nthreads=nthreads)
+                               nthreads=nthreads, **kv)
         total_t += time.perf_counter() - t0
         total_bytes += row_bytes(sel)
     # KV bytes of the sampled (sequence, query head) rows as the kernel counts them:
@@ -384,9 +398,9 @@ def run_ours(args):
 
     spec = rank_spec(workload_spec(args.workload), rank)
     sc = W.scenario(spec)
-    dt = W.torch_dtype(spec)
-    cache = PagedKVCache(sc.num_blocks, spec.block_size, spec.Hkv, spec.D, dt, device,
-                         sc.free_order.tolist(), fill=0.0)
+    cache = PagedKVCache(sc.num_blocks, spec.block_size, spec.Hkv, spec.D, W.torch_kv_dtype(spec),
+                         device, sc.free_order.tolist(), fill=0.0, k_scale=spec.k_scale,
+                         v_scale=spec.v_scale)
     for op in sc.setup_ops:
         if op.kind == "add":
             cache.add(op.seq)
@@ -429,11 +443,20 @@ def run_ours(args):
             ev[0].record(stream)
         if pairs.numel():
             pk.pa_copy_blocks(kc, vc, pairs, stream=stream)
-        pk.pa_reshape_and_cache(key, value, kc, vc, slots, stream=stream)
+        if spec.fp8:
+            pk.pa_reshape_and_cache_fp8(key, value, kc, vc, slots, spec.k_scale, spec.v_scale,
+                                        stream=stream)
+        else:
+            pk.pa_reshape_and_cache(key, value, kc, vc, slots, stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        pk.pa_decode_partitions(out, q, kc, vc, tables, lens, scale, max_ctx, partition_size=P,
-                                workspace=ws, stream=stream)
+        if spec.fp8:
+            pk.pa_decode_partitions_fp8(out, q, kc, vc, tables, lens, scale, max_ctx, spec.k_scale,
+                                        spec.v_scale, partition_size=P, workspace=ws,
+                                        stream=stream)
+        else:
+            pk.pa_decode_partitions(out, q, kc, vc, tables, lens, scale, max_ctx,
+                                    partition_size=P, workspace=ws, stream=stream)
         if ev is not None:
             ev[2].record(stream)
         if n_part > 1:
@@ -564,7 +587,7 @@ def run_ours(args):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": spec.dtype,
+            "dtype": f"e4m3 kv, {spec.dtype} q/out (fp32 math)" if spec.fp8 else spec.dtype,
             "data": "synthetic: seeded N(0,1) K/V/q in the cache dtype, context lengths and block "
                     "placement drawn as the workload states (stand-in for the ShareGPT/Alpaca-shaped "
                     "serving workloads; no dataset or weights)",
@@ -615,7 +638,7 @@ def run_swap(args):
     pk.lib()
     spec = workload_spec(args.workload)
     sc = W.scenario(spec)
-    dt = W.torch_dtype(spec)
+    dt = W.torch_kv_dtype(spec)
     shape = (sc.num_blocks, spec.Hkv, spec.block_size, spec.D)
     kc = torch.randn(shape, dtype=torch.float32, device=device).to(dt)
     vc = torch.randn(shape, dtype=torch.float32, device=device).to(dt)
@@ -644,7 +667,7 @@ def run_swap(args):
     hv = torch.empty((n,) + shape[1:], dtype=dt).pin_memory()
     out_pairs = torch.tensor(np.stack([cache_ids, host_ids], 1), dtype=torch.int64, device=device)
     in_pairs = torch.tensor(np.stack([host_ids, cache_ids], 1), dtype=torch.int64, device=device)
-    block_bytes = spec.Hkv * spec.block_size * spec.D * W.DTYPE_BYTES[spec.dtype]
+    block_bytes = spec.Hkv * spec.block_size * spec.D * spec.kv_esize
     moved = 2 * n * block_bytes                      # K and V, one direction
     stream = torch.cuda.current_stream(device)
     flat_d = torch.empty(moved, dtype=torch.uint8, device=device)
@@ -682,8 +705,8 @@ def run_swap(args):
     pk.pa_swap_blocks(kc, vc, hk, hv, in_pairs, stream=stream)
     torch.cuda.synchronize(device)
     ids = torch.tensor(cache_ids, device=device)
-    assert torch.equal(kc.index_select(0, ids).view(torch.int16),
-                       ref_k.index_select(0, ids).view(torch.int16))
+    assert torch.equal(kc.index_select(0, ids).view(torch.uint8),
+                       ref_k.index_select(0, ids).view(torch.uint8))
     gbs = lambda ms: moved / (ms * 1e-3) / 1e9  # noqa: E731
     rt_ms = out_ms + in_ms
     return {
@@ -718,7 +741,9 @@ def main():
                     choices=["tiny", "opt13b", "opt13b_compact", "llama13b_ps", "gqa70b",
                              "long_prefix_bs8", "long_prefix_bs16", "long_prefix_bs32",
                              "gqa70b_quarter", "long_prefix_bs8_quarter",
-                             "long_prefix_bs16_quarter"])
+                             "long_prefix_bs16_quarter", "opt13b_fp8", "opt13b_compact_fp8",
+                             "gqa70b_fp8", "long_prefix_bs16_fp8", "llama13b_ps_fp8",
+                             "tiny_fp8"])
     ap.add_argument("--partition-size", type=int, default=0,
                     help="split-K partition length (0: the workload's own, 512)")
     ap.add_argument("--soak-seconds", type=float, default=0.5,

@@ -62,7 +62,17 @@ typedef enum {
   PA_ERR_UNSUPPORTED = 4  /* valid request outside the implemented shapes */
 } pa_status;
 
-typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
+/*
+ * Element types.  PA_FP8_E4M3 is a cache storage type only: one byte per
+ * element, an OCP E4M3 code (1 sign, 4 exponent bits with bias 7, 3 fraction
+ * bits, largest finite 448) standing for code * scale with one scale per cache
+ * ([P2] "4. 이 밖의 기법들": quantization lowers the KV cache's precision to save
+ * memory and bandwidth; the format and per-cache scale are this library's
+ * reading).  It is accepted by pa_copy_blocks, pa_swap_blocks and
+ * pa_reshape_and_cache (codes moved as bytes) and as the cache type of the
+ * *_fp8 calls; as a query / output type it is PA_ERR_UNSUPPORTED.
+ */
+typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2, PA_FP8_E4M3 = 3 } pa_dtype;
 
 /* Bits of the per-device status word (see pa_device_status). */
 #define PA_DEVERR_TABLE 0x1u    /* a block-table entry outside [0, NB) was met */
@@ -268,6 +278,46 @@ pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache
 pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_pairs, int num_pairs,
                          int num_kv_heads, int head_size, int block_size, int num_blocks,
                          pa_dtype dtype, void* stream);
+
+/*
+ * E4M3 KV cache ([P2] "4. 이 밖의 기법들", quantization; format and scales as
+ * described at pa_dtype).
+ *
+ * pa_reshape_and_cache_fp8: as pa_reshape_and_cache, but key/value are f32 /
+ * f16 / bf16 (`dtype`) and the caches hold E4M3 codes:
+ *   k_cache[s / bs][h][s % bs][d] = E4M3(fp32(key[t][h][d]) / k_scale)
+ * (the quotient rounded once in fp32, then to the nearest E4M3 value with ties
+ * to an even fraction, magnitudes above 448 saturating to 448); value alike
+ * with v_scale.  Scales must be finite and > 0.
+ *
+ * pa_decode_fp8 / pa_decode_partitions_fp8: as pa_decode / pa_decode_partitions
+ * with q and out of type `dtype` (f32 / f16 / bf16) and caches of E4M3 codes,
+ * each standing for code * k_scale (keys) or code * v_scale (values).  The
+ * workspace and pa_decode_reduce (with `dtype`) are the same as for pa_decode;
+ * partition_size 0 means the default length.
+ */
+pa_status pa_reshape_and_cache_fp8(const void* key, const void* value, void* k_cache,
+                                   void* v_cache, const int64_t* slot_mapping, int num_tokens,
+                                   int num_kv_heads, int head_size, int block_size,
+                                   int num_blocks, pa_dtype dtype, float k_scale, float v_scale,
+                                   void* stream);
+
+pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* block_tables, int max_blocks_per_seq,
+                        const int32_t* context_lens, int num_seqs, int num_heads,
+                        int num_kv_heads, int head_size, int block_size, int num_blocks,
+                        float scale, pa_dtype dtype, float k_scale, float v_scale,
+                        int partition_size, int max_context_len, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+pa_status pa_decode_partitions_fp8(void* out, const void* q, const void* k_cache,
+                                   const void* v_cache, const int32_t* block_tables,
+                                   int max_blocks_per_seq, const int32_t* context_lens,
+                                   int num_seqs, int num_heads, int num_kv_heads, int head_size,
+                                   int block_size, int num_blocks, float scale, pa_dtype dtype,
+                                   float k_scale, float v_scale, int partition_size,
+                                   int max_context_len, void* workspace, size_t workspace_bytes,
+                                   void* stream);
 
 /*
  * Swap ([P1] "적용 범위와 관련 연구": when GPU memory runs short a sequence's KV

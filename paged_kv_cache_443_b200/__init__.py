@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpagedkv.so")
 
 PA_OK, PA_ERR_INVALID, PA_ERR_OOM, PA_ERR_CUDA, PA_ERR_UNSUPPORTED = 0, 1, 2, 3, 4
-PA_F32, PA_F16, PA_BF16 = 0, 1, 2
+PA_F32, PA_F16, PA_BF16, PA_FP8_E4M3 = 0, 1, 2, 3
 PA_DEVERR_TABLE, PA_DEVERR_CONTEXT, PA_DEVERR_SLOT, PA_DEVERR_PAIR, PA_DEVERR_TIMEOUT = (
     0x1, 0x2, 0x4, 0x8, 0x10)
 
@@ -31,7 +31,8 @@ EXPORTS = (
     "pa_decode_default_partition_size", "pa_decode_auto_partition_size",
     "pa_decode_num_partitions", "pa_decode_workspace_bytes",
     "pa_decode", "pa_decode_partitions", "pa_decode_reduce", "pa_decode_noalloc",
-    "pa_reshape_and_cache",
+    "pa_reshape_and_cache", "pa_reshape_and_cache_fp8", "pa_decode_fp8",
+    "pa_decode_partitions_fp8",
     "pa_copy_blocks", "pa_swap_blocks", "pa_alloc_create", "pa_alloc_destroy", "pa_alloc_num_free",
     "pa_alloc_refcount", "pa_alloc_free_stack", "pa_seq_add", "pa_seq_fork", "pa_seq_append",
     "pa_seq_free", "pa_seq_move", "pa_seq_num_tokens", "pa_build_tables",
@@ -84,6 +85,12 @@ def lib():
         "pa_decode_noalloc": ([vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, f32,
                                i32, i32, i32, vp], i32),
         "pa_reshape_and_cache": ([vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp], i32),
+        "pa_reshape_and_cache_fp8": ([vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, f32,
+                                      vp], i32),
+        "pa_decode_fp8": ([vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, f32, i32,
+                           f32, f32, i32, i32, vp, sz, vp], i32),
+        "pa_decode_partitions_fp8": ([vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32,
+                                      f32, i32, f32, f32, i32, i32, vp, sz, vp], i32),
         "pa_copy_blocks": ([vp, vp, vp, i32, i32, i32, i32, i32, i32, vp], i32),
         "pa_swap_blocks": ([vp, vp, i32, vp, vp, i32, vp, i32, i32, i32, i32, i32, vp], i32),
         "pa_alloc_create": ([i32, i32, pi32, ctypes.POINTER(vp)], i32),
@@ -115,7 +122,8 @@ def _check(st: int) -> None:
 
 def _dtype_code(t) -> int:
     import torch
-    codes = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
+    codes = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16,
+             torch.float8_e4m3fn: PA_FP8_E4M3}
     if t.dtype not in codes:
         raise PagedKVError(PA_ERR_INVALID, f"unsupported dtype {t.dtype}")
     return codes[t.dtype]
@@ -193,15 +201,15 @@ def pa_decode_workspace_bytes(num_seqs: int, num_heads: int, head_size: int,
 
 
 def _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, partition_size,
-                 max_context_len, workspace, stream):
+                 max_context_len, workspace, stream, kv_dtype=None):
     _contig(out, q, k_cache, v_cache, block_tables, context_lens, workspace)
     B, Hq, D = q.shape
     NB, Hkv, bs, D2 = k_cache.shape
     if D2 != D or tuple(out.shape) != (B, Hq, D) or tuple(v_cache.shape) != tuple(k_cache.shape):
         raise PagedKVError(PA_ERR_INVALID, "shape mismatch among q, out and the caches")
-    for t in (out, k_cache, v_cache):
-        if t.dtype != q.dtype:
-            raise PagedKVError(PA_ERR_INVALID, "q, out and the caches must share a dtype")
+    for t, want in ((out, q.dtype), (k_cache, kv_dtype or q.dtype), (v_cache, kv_dtype or q.dtype)):
+        if t.dtype != want:
+            raise PagedKVError(PA_ERR_INVALID, f"dtype mismatch: {t.dtype} where {want} is expected")
     import torch
     if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
         raise PagedKVError(PA_ERR_INVALID, "block_tables and context_lens must be int32")
@@ -239,6 +247,44 @@ def pa_decode_reduce(out, context_lens, max_context_len, partition_size=0, works
     _check(lib().pa_decode_reduce(_ptr(out), _ptr(context_lens), B, Hq, D, _dtype_code(out),
                                   int(partition_size), int(max_context_len), _ptr(workspace),
                                   ws_bytes, _stream(stream)))
+
+
+def pa_decode_fp8(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
+                  k_scale, v_scale, partition_size=0, workspace=None, stream=None) -> None:
+    """pa_decode over E4M3 caches (torch.float8_e4m3fn): keys stand for
+    code * k_scale, values for code * v_scale; q and out f32 / f16 / bf16."""
+    import torch
+    a = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, partition_size,
+                     max_context_len, workspace, stream, kv_dtype=torch.float8_e4m3fn)
+    _check(lib().pa_decode_fp8(*a[:15], float(k_scale), float(v_scale), *a[15:]))
+
+
+def pa_decode_partitions_fp8(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                             max_context_len, k_scale, v_scale, partition_size=0, workspace=None,
+                             stream=None) -> None:
+    import torch
+    a = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, partition_size,
+                     max_context_len, workspace, stream, kv_dtype=torch.float8_e4m3fn)
+    _check(lib().pa_decode_partitions_fp8(*a[:15], float(k_scale), float(v_scale), *a[15:]))
+
+
+def pa_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale,
+                             stream=None) -> None:
+    """Store key/value (f32 / f16 / bf16) as E4M3 codes of x / scale in the
+    float8_e4m3fn caches at their slots."""
+    _contig(key, value, k_cache, v_cache, slot_mapping)
+    import torch
+    N, Hkv, D = key.shape
+    NB, Hkv2, bs, D2 = k_cache.shape
+    if (Hkv2, D2) != (Hkv, D) or value.shape != key.shape or v_cache.shape != k_cache.shape:
+        raise PagedKVError(PA_ERR_INVALID, "shape mismatch")
+    if slot_mapping.dtype != torch.int64 or slot_mapping.numel() != N:
+        raise PagedKVError(PA_ERR_INVALID, "slot_mapping must be int64 [N]")
+    if key.dtype != value.dtype or not (k_cache.dtype == v_cache.dtype == torch.float8_e4m3fn):
+        raise PagedKVError(PA_ERR_INVALID, "key/value share a dtype; caches are float8_e4m3fn")
+    _check(lib().pa_reshape_and_cache_fp8(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
+                                          _ptr(slot_mapping), N, Hkv, D, bs, NB, _dtype_code(key),
+                                          float(k_scale), float(v_scale), _stream(stream)))
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scale,

@@ -17,24 +17,38 @@ from typing import List, Optional, Sequence, Tuple
 
 import torch
 
-from . import (BlockAllocator, pa_copy_blocks, pa_decode, pa_decode_workspace_bytes,
-               pa_reshape_and_cache, pa_swap_blocks)
+from . import (BlockAllocator, pa_copy_blocks, pa_decode, pa_decode_fp8,
+               pa_decode_workspace_bytes, pa_reshape_and_cache, pa_reshape_and_cache_fp8,
+               pa_swap_blocks)
+
+
+def _filled(shape, fill: float, dtype: torch.dtype, device) -> torch.Tensor:
+    if dtype == torch.float8_e4m3fn:   # fill the byte code (NaN -> the E4M3 NaN code)
+        code = int(torch.tensor([float(fill)]).to(dtype).view(torch.uint8)[0])
+        return torch.full(shape, code, dtype=torch.uint8, device=device).view(dtype)
+    return torch.full(shape, fill, dtype=dtype, device=device)
 
 
 class PagedKVCache:
+    """dtype: the cache's element type, or torch.float8_e4m3fn for a cache of
+    E4M3 codes standing for code * k_scale (keys) and code * v_scale (values);
+    new K/V and queries are then f32 / f16 / bf16 and quantised on append."""
+
     def __init__(self, num_blocks: int, block_size: int, num_kv_heads: int, head_size: int,
                  dtype: torch.dtype, device="cuda", initial_free_order: Optional[Sequence[int]] = None,
-                 fill: Optional[float] = None):
+                 fill: Optional[float] = None, k_scale: float = 1.0, v_scale: float = 1.0):
         self.num_blocks, self.block_size = num_blocks, block_size
         self.num_kv_heads, self.head_size = num_kv_heads, head_size
         self.dtype, self.device = dtype, torch.device(device)
+        self.fp8 = dtype == torch.float8_e4m3fn
+        self.k_scale, self.v_scale = float(k_scale), float(v_scale)
         shape = (num_blocks, num_kv_heads, block_size, head_size)
         if fill is None:
             self.k_cache = torch.empty(shape, dtype=dtype, device=self.device)
             self.v_cache = torch.empty(shape, dtype=dtype, device=self.device)
         else:
-            self.k_cache = torch.full(shape, fill, dtype=dtype, device=self.device)
-            self.v_cache = torch.full(shape, fill, dtype=dtype, device=self.device)
+            self.k_cache = _filled(shape, fill, dtype, self.device)
+            self.v_cache = _filled(shape, fill, dtype, self.device)
         self.alloc = BlockAllocator(num_blocks, block_size, initial_free_order)
         self.host_alloc = None
         self.host_k = self.host_v = None
@@ -75,7 +89,12 @@ class PagedKVCache:
     def store(self, key: torch.Tensor, value: torch.Tensor, slot_mapping, stream=None) -> None:
         if not isinstance(slot_mapping, torch.Tensor):
             slot_mapping = torch.tensor(slot_mapping, dtype=torch.int64, device=self.device)
-        if slot_mapping.numel():
+        if not slot_mapping.numel():
+            return
+        if self.fp8:
+            pa_reshape_and_cache_fp8(key, value, self.k_cache, self.v_cache, slot_mapping,
+                                     self.k_scale, self.v_scale, stream=stream)
+        else:
             pa_reshape_and_cache(key, value, self.k_cache, self.v_cache, slot_mapping, stream=stream)
 
     def append(self, seq_ids: Sequence[int], counts: Sequence[int], key: torch.Tensor,
@@ -112,9 +131,14 @@ class PagedKVCache:
             out = torch.empty_like(q)
         if workspace is None:
             workspace = self.workspace(q.shape[0], q.shape[1], max_context_len, partition_size)
-        pa_decode(out, q, self.k_cache, self.v_cache, block_tables, context_lens, scale,
-                  max_context_len, partition_size=partition_size, workspace=workspace,
-                  stream=stream)
+        if self.fp8:
+            pa_decode_fp8(out, q, self.k_cache, self.v_cache, block_tables, context_lens, scale,
+                          max_context_len, self.k_scale, self.v_scale,
+                          partition_size=partition_size, workspace=workspace, stream=stream)
+        else:
+            pa_decode(out, q, self.k_cache, self.v_cache, block_tables, context_lens, scale,
+                      max_context_len, partition_size=partition_size, workspace=workspace,
+                      stream=stream)
         return out
 
     # ---- swap to / from pinned host memory ----

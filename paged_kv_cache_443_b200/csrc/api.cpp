@@ -66,6 +66,10 @@ pa_status check_decode(const char* fn, int num_seqs, int num_heads, int num_kv_h
                        int head_size, pa_dtype dtype, int partition_size, int max_context_len,
                        int* P_out, int64_t* NP_out) {
   if (pa::elem_size(dtype) == 0) return pa::fail(PA_ERR_INVALID, "%s: unknown dtype %d", fn, dtype);
+  if (dtype == PA_FP8_E4M3)
+    return pa::fail(PA_ERR_UNSUPPORTED,
+                    "%s: E4M3 is a cache type only; q and out must be f32, f16 or bf16 (the "
+                    "*_fp8 calls take an E4M3 cache)", fn);
   if (num_seqs < 0) return pa::fail(PA_ERR_INVALID, "%s: num_seqs < 0", fn);
   if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0)
     return pa::fail(PA_ERR_INVALID, "%s: num_heads (%d) must be a positive multiple of num_kv_heads (%d)",
@@ -146,11 +150,37 @@ pa_status check_decode_full(const char* fn, void* out, const void* q, const void
   a->num_partitions = static_cast<int>(NP);
   a->scale = scale;
   a->dtype = dtype;
+  a->kv_dtype = dtype;
+  a->k_scale = a->v_scale = 1.f;
+  return PA_OK;
+}
+
+bool valid_kv_scale(float s) { return std::isfinite(s) && s > 0.f; }
+
+// pa_decode_fp8 / pa_decode_partitions_fp8: the pa_decode checks with q's
+// dtype, then the E4M3 cache and its scales.
+pa_status check_decode_fp8(const char* fn, void* out, const void* q, const void* k_cache,
+                           const void* v_cache, const int32_t* block_tables,
+                           int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                           int num_heads, int num_kv_heads, int head_size, int block_size,
+                           int num_blocks, float scale, pa_dtype dtype, float k_scale,
+                           float v_scale, int partition_size, int max_context_len,
+                           void* workspace, size_t workspace_bytes_in, pa::DecodeArgs* a) {
+  if (!valid_kv_scale(k_scale) || !valid_kv_scale(v_scale))
+    return pa::fail(PA_ERR_INVALID, "%s: k_scale and v_scale must be finite and > 0", fn);
+  pa_status st = check_decode_full(fn, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                   context_lens, num_seqs, num_heads, num_kv_heads, head_size,
+                                   block_size, num_blocks, scale, dtype, partition_size,
+                                   max_context_len, workspace, workspace_bytes_in, a);
+  if (st != PA_OK) return st;
+  a->kv_dtype = PA_FP8_E4M3;
+  a->k_scale = k_scale;
+  a->v_scale = v_scale;
   return PA_OK;
 }
 
 int launch_partitions(const pa::DecodeArgs& a, unsigned int* status, void* stream) {
-  if (pa::decode_tc_supported(a)) return pa::launch_decode_partitions_tc(a, status, stream);
+  if (a.kv_dtype == a.dtype && pa::decode_tc_supported(a)) return pa::launch_decode_partitions_tc(a, status, stream);
   return pa::launch_decode_partitions(a, status, stream);
 }
 
@@ -359,5 +389,84 @@ extern "C" pa_status pa_swap_blocks(void* dst_k_cache, void* dst_v_cache, int ds
                                               block_pairs, num_pairs, num_kv_heads, head_size,
                                               block_size, src_num_blocks, dst_num_blocks, es,
                                               status, stream),
+                       1);
+}
+
+extern "C" pa_status pa_decode_partitions_fp8(void* out, const void* q, const void* k_cache,
+                                              const void* v_cache, const int32_t* block_tables,
+                                              int max_blocks_per_seq, const int32_t* context_lens,
+                                              int num_seqs, int num_heads, int num_kv_heads,
+                                              int head_size, int block_size, int num_blocks,
+                                              float scale, pa_dtype dtype, float k_scale,
+                                              float v_scale, int partition_size,
+                                              int max_context_len, void* workspace,
+                                              size_t workspace_bytes_in, void* stream) {
+  const char* fn = "pa_decode_partitions_fp8";
+  pa::DecodeArgs a;
+  pa_status st = check_decode_fp8(fn, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                  context_lens, num_seqs, num_heads, num_kv_heads, head_size,
+                                  block_size, num_blocks, scale, dtype, k_scale, v_scale,
+                                  partition_size, max_context_len, workspace, workspace_bytes_in,
+                                  &a);
+  if (st != PA_OK || num_seqs == 0) return st;
+  unsigned int* status = pa::device_status_word();
+  if (!status) return PA_ERR_CUDA;
+  return launch_status(fn, launch_partitions(a, status, stream), 1);
+}
+
+extern "C" pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache,
+                                   const void* v_cache, const int32_t* block_tables,
+                                   int max_blocks_per_seq, const int32_t* context_lens,
+                                   int num_seqs, int num_heads, int num_kv_heads, int head_size,
+                                   int block_size, int num_blocks, float scale, pa_dtype dtype,
+                                   float k_scale, float v_scale, int partition_size,
+                                   int max_context_len, void* workspace,
+                                   size_t workspace_bytes_in, void* stream) {
+  const char* fn = "pa_decode_fp8";
+  pa::DecodeArgs a;
+  pa_status st = check_decode_fp8(fn, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                  context_lens, num_seqs, num_heads, num_kv_heads, head_size,
+                                  block_size, num_blocks, scale, dtype, k_scale, v_scale,
+                                  partition_size, max_context_len, workspace, workspace_bytes_in,
+                                  &a);
+  if (st != PA_OK || num_seqs == 0) return st;
+  unsigned int* status = pa::device_status_word();
+  if (!status) return PA_ERR_CUDA;
+  st = launch_status(fn, launch_partitions(a, status, stream), 1);
+  if (st != PA_OK || a.num_partitions <= 1) return st;
+  return launch_status(fn, pa::launch_decode_reduce(a, status, stream), 1);
+}
+
+extern "C" pa_status pa_reshape_and_cache_fp8(const void* key, const void* value, void* k_cache,
+                                              void* v_cache, const int64_t* slot_mapping,
+                                              int num_tokens, int num_kv_heads, int head_size,
+                                              int block_size, int num_blocks, pa_dtype dtype,
+                                              float k_scale, float v_scale, void* stream) {
+  const char* fn = "pa_reshape_and_cache_fp8";
+  if (pa::elem_size(dtype) == 0) return pa::fail(PA_ERR_INVALID, "%s: unknown dtype %d", fn, dtype);
+  if (dtype == PA_FP8_E4M3)
+    return pa::fail(PA_ERR_INVALID, "%s: key/value must be f32, f16 or bf16", fn);
+  if (!valid_kv_scale(k_scale) || !valid_kv_scale(v_scale))
+    return pa::fail(PA_ERR_INVALID, "%s: k_scale and v_scale must be finite and > 0", fn);
+  if (num_tokens < 0) return pa::fail(PA_ERR_INVALID, "%s: num_tokens < 0", fn);
+  if (num_kv_heads <= 0 || head_size <= 0 || block_size <= 0 || num_blocks <= 0)
+    return pa::fail(PA_ERR_INVALID, "%s: sizes must be positive", fn);
+  if (!supported_head(head_size))
+    return pa::fail(PA_ERR_UNSUPPORTED, "%s: head_size must be 64 or 128", fn);
+  if (!supported_block(block_size))
+    return pa::fail(PA_ERR_UNSUPPORTED, "%s: block_size must be 8, 16 or 32", fn);
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !k_cache || !v_cache || !slot_mapping)
+    return pa::fail(PA_ERR_INVALID, "%s: NULL device pointer", fn);
+  if (!pa::aligned16(key) || !pa::aligned16(value) || !pa::aligned16(k_cache) ||
+      !pa::aligned16(v_cache) || (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+    return pa::fail(PA_ERR_INVALID, "%s: key/value/caches must be 16-byte aligned, slots 8", fn);
+  unsigned int* status = pa::device_status_word();
+  if (!status) return PA_ERR_CUDA;
+  return launch_status(fn,
+                       pa::launch_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping,
+                                                        num_tokens, num_kv_heads, head_size,
+                                                        block_size, num_blocks, dtype, k_scale,
+                                                        v_scale, status, stream),
                        1);
 }

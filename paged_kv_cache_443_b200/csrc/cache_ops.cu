@@ -10,7 +10,7 @@
 // sequence's blocks move to CPU memory and back; the same copy kernel moves
 // blocks between a device cache and a pinned host cache the GPU can address.
 //
-// Both are pure data movement in 16-byte chunks: loads are coalesced along
+// Append and copy are pure data movement in 16-byte chunks: loads are coalesced along
 // the source, stores along a D-element cache row (append) or a whole
 // contiguous [Hkv][bs][D] block (copy).  Out-of-range slots or block ids are
 // skipped and flagged in the status word, never dereferenced.
@@ -51,6 +51,65 @@ __global__ void __launch_bounds__(256)
     const int64_t dst = (((blk * Hkv + h) << log2_bs) + off) * chunks_per_row + chunk;
     k_cache[dst] = __ldg(key + i);
     v_cache[dst] = __ldg(value + i);
+  }
+}
+
+// Append into E4M3 caches ("quantization" in "4. 이 밖의 기법들",
+// blog.aqudi.me): one thread per 16 elements of key/value [N][Hkv][D] of type
+// T; code = E4M3(x / scale) with the quotient correctly rounded in fp32 and the
+// hardware conversion rounding to nearest-even, saturating at 448; one 16-byte
+// store per cache.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    reshape_and_cache_fp8_kernel(const T* __restrict__ key, const T* __restrict__ value,
+                                 uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                                 const int64_t* __restrict__ slot_mapping, int64_t total_chunks,
+                                 int Hkv, int chunks_per_row, int log2_bs, int64_t num_slots,
+                                 float k_scale, float v_scale, unsigned int* status) {
+  allow_dependents();
+  constexpr int PER = Elem<T>::EPL;  // elements per 16-byte load of T
+  const int64_t per_token = static_cast<int64_t>(Hkv) * chunks_per_row;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total_chunks;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = i / per_token;
+    const int64_t rem = i - t * per_token;
+    const int64_t slot = __ldg(slot_mapping + t);
+    if (slot < 0) continue;
+    if (slot >= num_slots) {
+      atomicOr(status, PA_DEVERR_SLOT);
+      continue;
+    }
+    float kf[16], vf[16];
+#pragma unroll
+    for (int j = 0; j < 16 / PER; ++j) {
+      Elem<T>::unpack(__ldg(reinterpret_cast<const uint4*>(key + i * 16 + j * PER)), kf + j * PER);
+      Elem<T>::unpack(__ldg(reinterpret_cast<const uint4*>(value + i * 16 + j * PER)), vf + j * PER);
+    }
+    uint32_t kw[4], vw[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t kk = 0, vv = 0;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float2 kp = make_float2(__fdiv_rn(kf[4 * j + 2 * e], k_scale),
+                                      __fdiv_rn(kf[4 * j + 2 * e + 1], k_scale));
+        const float2 vp = make_float2(__fdiv_rn(vf[4 * j + 2 * e], v_scale),
+                                      __fdiv_rn(vf[4 * j + 2 * e + 1], v_scale));
+        kk |= static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(kp, __NV_SATFINITE, __NV_E4M3))
+              << (16 * e);
+        vv |= static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(vp, __NV_SATFINITE, __NV_E4M3))
+              << (16 * e);
+      }
+      kw[j] = kk;
+      vw[j] = vv;
+    }
+    const int64_t blk = slot >> log2_bs;
+    const int64_t off = slot & ((1 << log2_bs) - 1);
+    const int64_t h = rem / chunks_per_row;
+    const int64_t chunk = rem - h * chunks_per_row;
+    const int64_t dst = (((blk * Hkv + h) << log2_bs) + off) * chunks_per_row + chunk;
+    k_cache[dst] = make_uint4(kw[0], kw[1], kw[2], kw[3]);
+    v_cache[dst] = make_uint4(vw[0], vw[1], vw[2], vw[3]);
   }
 }
 
@@ -120,6 +179,46 @@ int launch_reshape_and_cache(const void* key, const void* value, void* k_cache, 
       static_cast<const uint4*>(key), static_cast<const uint4*>(value),
       static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), slot_mapping, total, Hkv,
       chunks_per_row, ilog2(block_size), static_cast<int64_t>(num_blocks) * block_size, status);
+  return cudaGetLastError();
+}
+
+int launch_reshape_and_cache_fp8(const void* key, const void* value, void* k_cache,
+                                 void* v_cache, const int64_t* slot_mapping, int num_tokens,
+                                 int Hkv, int D, int block_size, int num_blocks, pa_dtype dtype,
+                                 float k_scale, float v_scale, unsigned int* status,
+                                 void* stream) {
+  const int chunks_per_row = D / 16;  // 16 codes = 16 bytes per chunk
+  const int64_t total = static_cast<int64_t>(num_tokens) * Hkv * chunks_per_row;
+  const int threads = 256;
+  int64_t blocks = (total + threads - 1) / threads;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  const dim3 grid(static_cast<unsigned>(blocks));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t slots = static_cast<int64_t>(num_blocks) * block_size;
+  const int lb = ilog2(block_size);
+  uint4* kc = static_cast<uint4*>(k_cache);
+  uint4* vc = static_cast<uint4*>(v_cache);
+  switch (dtype) {
+    case PA_F32:
+      reshape_and_cache_fp8_kernel<float><<<grid, threads, 0, st>>>(
+          static_cast<const float*>(key), static_cast<const float*>(value), kc, vc, slot_mapping,
+          total, Hkv, chunks_per_row, lb, slots, k_scale, v_scale, status);
+      break;
+    case PA_F16:
+      reshape_and_cache_fp8_kernel<__half><<<grid, threads, 0, st>>>(
+          static_cast<const __half*>(key), static_cast<const __half*>(value), kc, vc,
+          slot_mapping, total, Hkv, chunks_per_row, lb, slots, k_scale, v_scale, status);
+      break;
+    case PA_BF16:
+      reshape_and_cache_fp8_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(key), static_cast<const __nv_bfloat16*>(value), kc,
+          vc, slot_mapping, total, Hkv, chunks_per_row, lb, slots, k_scale, v_scale, status);
+      break;
+    default:
+      return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 

@@ -29,6 +29,13 @@
 //     partial (m, l, o) goes to the workspace for the reduce kernel.
 //   Every mbarrier wait is bounded (pa_device.cuh); a block id outside the pool
 //   is never dereferenced (the copy is skipped and PA_DEVERR_TABLE set).
+//
+// E4M3 caches ("quantization" in "4. 이 밖의 기법들", blog.aqudi.me): the K/V
+// type TK is separate from the query/output type TQ.  A lane loads 8 codes (8
+// bytes) and widens them exactly to fp32; k_scale is folded into the query's
+// pre-scale and v_scale into the partial output, so the inner loops are those
+// of the 16-bit caches.  Half the bytes per token means twice the tokens per
+// stage (and twice the consumer warps) for the same bytes in flight.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -49,10 +56,10 @@ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 template <typename T, int D, int G, int NCW>
 struct Cfg {
   static constexpr int ES = sizeof(T);
-  static constexpr int EPL = 16 / ES;          // elements per 16-byte chunk
+  static constexpr int EPL = Elem<T>::EPL;     // elements a lane loads at once
   static constexpr int LPR = D / EPL;          // lanes per K/V row
   static constexpr int RPW = 32 / LPR;         // rows a warp covers per iteration
-  static constexpr int TOK = kStageTokens;     // tokens per stage
+  static constexpr int TOK = NCW * 8;          // tokens per stage (8 per consumer warp)
   static constexpr int TPW = TOK / NCW;        // tokens per consumer warp per stage
   static constexpr int ITERS = TPW / RPW;
   static constexpr int ROW_BYTES = D * ES;
@@ -72,7 +79,20 @@ struct Cfg {
   static_assert(TPW <= 32 && (TPW & (TPW - 1)) == 0, "score segment must fit a warp");
   static_assert(NCW * G * CB_STRIDE * 4 <= S * STAGE_BYTES, "combine buffer must fit the stages");
   static_assert(SMEM <= 227 * 1024, "shared memory");
+  static_assert(TOK % kStageTokens == 0 && TOK <= 256, "a stage is whole table words of blocks");
 };
+
+// q row chunk of EPL elements of TQ (global memory, read-only path) to fp32.
+template <typename TQ, int EPL>
+__device__ __forceinline__ void load_q(const TQ* src, float* f) {
+  constexpr int PER = Elem<TQ>::EPL;  // elements of one 16-byte load
+  static_assert(EPL % PER == 0, "q chunk must be whole 16-byte loads");
+#pragma unroll
+  for (int i = 0; i < EPL / PER; ++i) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(src + i * PER));
+    Elem<TQ>::unpack(u, f + i * PER);
+  }
+}
 
 // Butterfly reduce-scatter of N values over the lanes of a row (lane bits
 // below LPR): each halving step keeps one half of the values and adds the
@@ -120,14 +140,17 @@ struct PartitionParams {
   unsigned int* status;
   int64_t max_blocks;
   int Hq, Hkv, num_blocks, block_size, partition_size, num_partitions;
-  float scale_log2;  // scale * log2(e)
+  float scale_log2;  // scale * log2(e) (* k_scale for E4M3 caches)
+  float v_scale;     // E4M3 caches: the value scale (1 otherwise, unused)
 };
 
-template <typename T, int D, int G, int NCW>
-__global__ void __launch_bounds__(Cfg<T, D, G, NCW>::THREADS)
+template <typename TQ, typename TK, int D, int G, int NCW>
+__global__ void __launch_bounds__(Cfg<TK, D, G, NCW>::THREADS)
     decode_partition_kernel(const PartitionParams p) {
-  using C = Cfg<T, D, G, NCW>;
-  using E = Elem<T>;
+  using C = Cfg<TK, D, G, NCW>;
+  using E = Elem<TK>;
+  using EQ = Elem<TQ>;
+  constexpr bool kCoded = sizeof(TK) == 1;  // E4M3 codes
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + C::S;
@@ -156,8 +179,8 @@ __global__ void __launch_bounds__(Cfg<T, D, G, NCW>::THREADS)
   const int start = part * P;
   if (L == 0) {
     if (part == 0) {
-      T* o = static_cast<T*>(p.out) + (static_cast<int64_t>(b) * p.Hq + g * G) * D;
-      for (int i = threadIdx.x; i < G * D; i += C::THREADS) o[i] = E::from_float(0.f);
+      TQ* o = static_cast<TQ*>(p.out) + (static_cast<int64_t>(b) * p.Hq + g * G) * D;
+      for (int i = threadIdx.x; i < G * D; i += C::THREADS) o[i] = EQ::from_float(0.f);
     }
     return;
   }
@@ -236,11 +259,10 @@ __global__ void __launch_bounds__(Cfg<T, D, G, NCW>::THREADS)
 
   float qf[G][C::EPL];
   {
-    const T* qrow = static_cast<const T*>(p.q) + (static_cast<int64_t>(b) * p.Hq + g * G) * D;
+    const TQ* qrow = static_cast<const TQ*>(p.q) + (static_cast<int64_t>(b) * p.Hq + g * G) * D;
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(qrow + h * D + c * C::EPL));
-      E::unpack(u, qf[h]);
+      load_q<TQ, C::EPL>(qrow + h * D + c * C::EPL, qf[h]);
 #pragma unroll
       for (int e = 0; e < C::EPL; ++e) qf[h][e] *= p.scale_log2;
     }
@@ -261,8 +283,8 @@ __global__ void __launch_bounds__(Cfg<T, D, G, NCW>::THREADS)
       ok = false;
       break;
     }
-    const T* Ks = reinterpret_cast<const T*>(stages + s * C::STAGE_BYTES);
-    const T* Vs = reinterpret_cast<const T*>(stages + s * C::STAGE_BYTES + C::TILE_BYTES);
+    const TK* Ks = reinterpret_cast<const TK*>(stages + s * C::STAGE_BYTES);
+    const TK* Vs = reinterpret_cast<const TK*>(stages + s * C::STAGE_BYTES + C::TILE_BYTES);
     const int n_valid = min(C::TOK, end - (start + t * C::TOK));
 
     // ---- scores: partial dots over this lane's chunk, then across the row ----
@@ -270,9 +292,8 @@ __global__ void __launch_bounds__(Cfg<T, D, G, NCW>::THREADS)
 #pragma unroll
     for (int it = 0; it < C::ITERS; ++it) {
       const int row = w * C::TPW + it * C::RPW + r;
-      const uint4 u = *reinterpret_cast<const uint4*>(Ks + row * D + c * C::EPL);
       float kf[C::EPL];
-      E::unpack(u, kf);
+      E::load(Ks + row * D + c * C::EPL, kf);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         float acc = 0.f;
@@ -348,9 +369,8 @@ __global__ void __launch_bounds__(Cfg<T, D, G, NCW>::THREADS)
       const int row_local = it * C::RPW + r;
       const int row = w * C::TPW + row_local;
       if (row < n_valid) {
-        const uint4 u = *reinterpret_cast<const uint4*>(Vs + row * D + c * C::EPL);
         float vf[C::EPL];
-        E::unpack(u, vf);
+        E::load(Vs + row * D + c * C::EPL, vf);
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           const float pr = sc[h * C::TPW + row_local];
@@ -405,8 +425,9 @@ __global__ void __launch_bounds__(Cfg<T, D, G, NCW>::THREADS)
       O = fmaf(cb[(ww * G + h) * C::CB_STRIDE + d], f, O);
     }
     const int64_t hq = static_cast<int64_t>(b) * p.Hq + g * G + h;
+    if constexpr (kCoded) O *= p.v_scale;
     if (single) {
-      static_cast<T*>(p.out)[hq * D + d] = E::from_float(O / Ls);
+      static_cast<TQ*>(p.out)[hq * D + d] = EQ::from_float(O / Ls);
     } else {
       const int64_t slot = hq * p.num_partitions + part;
       p.ws_o[slot * D + d] = O;
@@ -468,12 +489,18 @@ __global__ void __launch_bounds__(128) decode_reduce_kernel(const ReduceParams p
   for (int k = 0; k < DPL; ++k) dst[k] = E::from_float(acc[k] * inv);
 }
 
-constexpr int kConsumerWarps = 4;
+// Consumer warps: 4 (32-token stages); E4M3 caches with up to 2 query heads
+// per kv head use 8 (64-token stages, the same bytes per stage).
+template <typename TK, int G>
+constexpr int consumer_warps() {
+  return (sizeof(TK) == 1 && G <= 2) ? 8 : 4;
+}
 
-template <typename T, int D, int G>
+template <typename TQ, typename TK, int D, int G>
 cudaError_t launch_partition_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
-  using C = Cfg<T, D, G, kConsumerWarps>;
-  auto kern = decode_partition_kernel<T, D, G, kConsumerWarps>;
+  constexpr int NCW = consumer_warps<TK, G>();
+  using C = Cfg<TK, D, G, NCW>;
+  auto kern = decode_partition_kernel<TQ, TK, D, G, NCW>;
   // opt in to > 48 KB of dynamic shared memory (idempotent, cheap)
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
@@ -496,29 +523,37 @@ cudaError_t launch_partition_t(const DecodeArgs& a, unsigned int* status, cudaSt
   p.block_size = a.block_size;
   p.partition_size = a.partition_size;
   p.num_partitions = a.num_partitions;
-  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.scale_log2 = a.scale * 1.4426950408889634f * a.k_scale;
+  p.v_scale = a.v_scale;
   dim3 grid(a.num_seqs, a.Hkv, a.num_partitions);
   return launch_overlapped(kern, grid, dim3(C::THREADS), C::SMEM, stream, p);
 }
 
-template <typename T, int D>
+template <typename TQ, typename TK, int D>
 cudaError_t launch_partition_g(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
   switch (a.Hq / a.Hkv) {
-    case 1: return launch_partition_t<T, D, 1>(a, status, stream);
-    case 2: return launch_partition_t<T, D, 2>(a, status, stream);
-    case 4: return launch_partition_t<T, D, 4>(a, status, stream);
-    case 8: return launch_partition_t<T, D, 8>(a, status, stream);
+    case 1: return launch_partition_t<TQ, TK, D, 1>(a, status, stream);
+    case 2: return launch_partition_t<TQ, TK, D, 2>(a, status, stream);
+    case 4: return launch_partition_t<TQ, TK, D, 4>(a, status, stream);
+    case 8: return launch_partition_t<TQ, TK, D, 8>(a, status, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <typename T>
+template <typename TQ, typename TK>
 cudaError_t launch_partition_d(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
   switch (a.D) {
-    case 64: return launch_partition_g<T, 64>(a, status, stream);
-    case 128: return launch_partition_g<T, 128>(a, status, stream);
+    case 64: return launch_partition_g<TQ, TK, 64>(a, status, stream);
+    case 128: return launch_partition_g<TQ, TK, 128>(a, status, stream);
     default: return cudaErrorInvalidValue;
   }
+}
+
+template <typename TQ>
+cudaError_t launch_partition_kv(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
+  if (a.kv_dtype == PA_FP8_E4M3) return launch_partition_d<TQ, __nv_fp8_e4m3>(a, status, stream);
+  if (a.kv_dtype != a.dtype) return cudaErrorInvalidValue;
+  return launch_partition_d<TQ, TQ>(a, status, stream);
 }
 
 template <typename T>
@@ -545,9 +580,9 @@ cudaError_t launch_reduce_t(const DecodeArgs& a, cudaStream_t stream) {
 int launch_decode_partitions(const DecodeArgs& a, unsigned int* status, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (a.dtype) {
-    case PA_F32: return launch_partition_d<float>(a, status, st);
-    case PA_F16: return launch_partition_d<__half>(a, status, st);
-    case PA_BF16: return launch_partition_d<__nv_bfloat16>(a, status, st);
+    case PA_F32: return launch_partition_kv<float>(a, status, st);
+    case PA_F16: return launch_partition_kv<__half>(a, status, st);
+    case PA_BF16: return launch_partition_kv<__nv_bfloat16>(a, status, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -5,6 +5,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -123,13 +124,17 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
 }
 
 // ---- element types ----
-// Elem<T>: EPL elements per 16-byte chunk; unpack a chunk to fp32; round fp32 to T.
+// Elem<T>: a lane's load of EPL elements (one 16-byte chunk; 8 bytes for E4M3)
+// widened to fp32 (load), unpack of a 16-byte chunk, and rounding fp32 to T.
 template <typename T>
 struct Elem;
 
 template <>
 struct Elem<float> {
   static constexpr int EPL = 4;
+  __device__ __forceinline__ static void load(const void* p, float* f) {
+    unpack(*reinterpret_cast<const uint4*>(p), f);
+  }
   __device__ __forceinline__ static void unpack(const uint4& u, float* f) {
     f[0] = __uint_as_float(u.x);
     f[1] = __uint_as_float(u.y);
@@ -142,6 +147,9 @@ struct Elem<float> {
 template <>
 struct Elem<__half> {
   static constexpr int EPL = 8;
+  __device__ __forceinline__ static void load(const void* p, float* f) {
+    unpack(*reinterpret_cast<const uint4*>(p), f);
+  }
   __device__ __forceinline__ static void unpack(const uint4& u, float* f) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -158,6 +166,9 @@ struct Elem<__half> {
 template <>
 struct Elem<__nv_bfloat16> {
   static constexpr int EPL = 8;
+  __device__ __forceinline__ static void load(const void* p, float* f) {
+    unpack(*reinterpret_cast<const uint4*>(p), f);
+  }
   __device__ __forceinline__ static void unpack(const uint4& u, float* f) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -169,6 +180,31 @@ struct Elem<__nv_bfloat16> {
   }
   __device__ __forceinline__ static __nv_bfloat16 from_float(float x) {
     return __float2bfloat16_rn(x);
+  }
+};
+
+// OCP E4M3 codes (a cache type only; the value is code * the cache's scale,
+// applied by the caller).  Every E4M3 value is an fp16 value, so the hardware
+// conversion to f16x2 and the widening to fp32 are exact.  Byte i of the
+// loaded word becomes f[i].
+template <>
+struct Elem<__nv_fp8_e4m3> {
+  static constexpr int EPL = 8;
+  __device__ __forceinline__ static void load(const void* p, float* f) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const uint32_t w[2] = {u.x, u.y};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const __nv_fp8x2_storage_t pair =
+            static_cast<__nv_fp8x2_storage_t>((w[i] >> (16 * j)) & 0xffffu);
+        const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+        const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+        f[4 * i + 2 * j] = v.x;
+        f[4 * i + 2 * j + 1] = v.y;
+      }
+    }
   }
 };
 

@@ -32,6 +32,7 @@ inline int elem_size(pa_dtype dt) {
     case PA_F32: return 4;
     case PA_F16: return 2;
     case PA_BF16: return 2;
+    case PA_FP8_E4M3: return 1;
     default: return 0;
   }
 }
@@ -54,7 +55,9 @@ struct DecodeArgs {
   int num_seqs, Hq, Hkv, D, block_size, num_blocks;
   int partition_size, num_partitions;
   float scale;
-  pa_dtype dtype;
+  pa_dtype dtype;      // q and out (and the caches unless kv_dtype says otherwise)
+  pa_dtype kv_dtype;   // the caches: dtype, or PA_FP8_E4M3
+  float k_scale = 1.f, v_scale = 1.f;  // per-cache scales of E4M3 codes
 };
 
 // Kernel launchers (kernels.cu).  They return cudaError_t as int.
@@ -74,6 +77,11 @@ int launch_reshape_and_cache(const void* key, const void* value, void* k_cache, 
                              const int64_t* slot_mapping, int num_tokens, int Hkv, int D,
                              int block_size, int num_blocks, int esize, unsigned int* status,
                              void* stream);
+// Append into an E4M3 cache; key/value of `dtype` (f32 / f16 / bf16).
+int launch_reshape_and_cache_fp8(const void* key, const void* value, void* k_cache,
+                                 void* v_cache, const int64_t* slot_mapping, int num_tokens,
+                                 int Hkv, int D, int block_size, int num_blocks, pa_dtype dtype,
+                                 float k_scale, float v_scale, unsigned int* status, void* stream);
 int launch_copy_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
                        const int64_t* pairs, int num_pairs, int Hkv, int D, int block_size,
                        int src_blocks, int dst_blocks, int esize, unsigned int* status,

@@ -25,8 +25,23 @@ TOL = {"f32": 1e-5, "f16": 2e-2, "bf16": 2e-2}
 def poison_bits(spec: W.Spec):
     """Bit pattern torch stores for NaN in the cache dtype (the fill of every
     slot no token was written to)."""
-    t = torch.full((1,), float("nan"), dtype=W.torch_dtype(spec))
+    t = torch.tensor([float("nan")]).to(W.torch_kv_dtype(spec))
     return W.storage_view(t)[0]
+
+
+def _zero_bits(spec: W.Spec):
+    return W.storage_view(torch.zeros(1).to(W.torch_kv_dtype(spec)))[0]
+
+
+def oracle_append(spec: W.Spec, key, value, k, v, slots):
+    """The oracle's append of the same draws (E4M3 quantisation for E4M3 caches)."""
+    if spec.fp8:
+        oracle.reshape_and_cache_e4m3(W.storage_view(key), W.storage_view(value), k, v,
+                                      np.asarray(slots, dtype=np.int64), spec.dtype_code,
+                                      spec.k_scale, spec.v_scale)
+    else:
+        oracle.reshape_and_cache(W.storage_view(key), W.storage_view(value), k, v,
+                                 np.asarray(slots, dtype=np.int64), spec.dtype_code)
 
 
 @dataclass
@@ -59,14 +74,15 @@ class Oracle:
 def build(sc: W.Scenario, device="cuda", with_oracle=True, poison=True):
     spec = sc.spec
     shape = (sc.num_blocks, spec.Hkv, spec.block_size, spec.D)
-    cache = PagedKVCache(sc.num_blocks, spec.block_size, spec.Hkv, spec.D, W.torch_dtype(spec),
+    cache = PagedKVCache(sc.num_blocks, spec.block_size, spec.Hkv, spec.D, W.torch_kv_dtype(spec),
                          device, sc.free_order.tolist(),
-                         fill=float("nan") if poison else 0.0)
+                         fill=float("nan") if poison else 0.0, k_scale=spec.k_scale,
+                         v_scale=spec.v_scale)
     orc = None
     if with_oracle:
         bm = BlockManager(sc.num_blocks, spec.block_size, sc.free_order.tolist())
-        fill = poison_bits(spec) if poison else W.storage_view(torch.zeros(1, dtype=W.torch_dtype(spec)))[0]
-        st = np.float32 if spec.dtype == "f32" else np.uint16
+        fill = poison_bits(spec) if poison else _zero_bits(spec)
+        st = {"f32": np.float32, "f16": np.uint16, "bf16": np.uint16, "e4m3": np.uint8}[spec.kv]
         ok = np.full(shape, fill, dtype=st)
         ov = np.full(shape, fill, dtype=st)
     for op in sc.setup_ops:
@@ -85,9 +101,8 @@ def build(sc: W.Scenario, device="cuda", with_oracle=True, poison=True):
             if with_oracle:
                 slots, pairs = bm.append(op.seq, op.arg)
                 if pairs:
-                    oracle.copy_blocks(ok, ov, np.array(pairs), spec.dtype_code)
-                oracle.reshape_and_cache(W.storage_view(k), W.storage_view(v), ok, ov,
-                                         np.array(slots), spec.dtype_code)
+                    oracle.copy_blocks(ok, ov, np.array(pairs), spec.kv_code)
+                oracle_append(spec, k, v, ok, ov, slots)
             del k, v
     # the step's appends: reserved now, executed by run_step
     seqs = [op.seq for op in sc.step_ops]
@@ -109,9 +124,8 @@ def build(sc: W.Scenario, device="cuda", with_oracle=True, poison=True):
             oslots += s
             opairs += p
         if opairs:
-            oracle.copy_blocks(ok, ov, np.array(opairs), spec.dtype_code)
-        oracle.reshape_and_cache(W.storage_view(key), W.storage_view(value), ok, ov,
-                                 np.array(oslots, dtype=np.int64), spec.dtype_code)
+            oracle.copy_blocks(ok, ov, np.array(opairs), spec.kv_code)
+        oracle_append(spec, key, value, ok, ov, oslots)
         ot, ol = bm.build_tables(sc.batch, sc.max_blocks)
         orc = Oracle(bm, ok, ov, ot, ol, W.storage_view(q), oslots, opairs)
     return prod, orc
@@ -133,7 +147,8 @@ def as_f64(t: torch.Tensor, spec: W.Spec) -> np.ndarray:
 
 def oracle_attention(o: Oracle, spec: W.Spec, rows=None):
     return oracle.paged_attention(o.q, o.k, o.v, spec.dtype_code, o.tables, o.lens,
-                                  spec.softmax_scale, rows=rows)
+                                  spec.softmax_scale, rows=rows, kv_dtype=spec.kv_code,
+                                  k_scale=spec.k_scale, v_scale=spec.v_scale)
 
 
 def check_bookkeeping(p: Product, o: Oracle):

@@ -137,3 +137,35 @@ def test_auto_partition_size(L):
     for P in (1024, 2048):
         assert pk.pa_decode_workspace_bytes(256, 64, 128, 4096, P) <= \
             pk.pa_decode_workspace_bytes(256, 64, 128, 4096, 0)
+
+
+def test_fp8_calls_reject_bad_arguments(L):
+    assert decode_call(L, dtype=pk.PA_FP8_E4M3) == pk.PA_ERR_UNSUPPORTED
+
+    def d8(k_scale=0.5, v_scale=2.0, dtype=pk.PA_BF16, **kw):
+        a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, tables=FAKE, maxb=8, lens=FAKE, B=2, Hq=8,
+                 Hkv=2, D=128, bs=16, NB=100, scale=0.1, P=0, maxctx=100)
+        a.update(kw)
+        return L.pa_decode_fp8(a["out"], a["q"], a["k"], a["v"], a["tables"], a["maxb"],
+                               a["lens"], a["B"], a["Hq"], a["Hkv"], a["D"], a["bs"], a["NB"],
+                               a["scale"], dtype, k_scale, v_scale, a["P"], a["maxctx"], None, 0,
+                               None)
+
+    before = pk.pa_launch_count()
+    for bad in (dict(k_scale=0.0), dict(v_scale=-1.0), dict(k_scale=float("inf")),
+                dict(v_scale=float("nan")), dict(dtype=pk.PA_FP8_E4M3), dict(dtype=9),
+                dict(D=96), dict(maxctx=100, P=32)):
+        want = pk.PA_ERR_UNSUPPORTED if ("D" in bad or bad.get("dtype") == pk.PA_FP8_E4M3) \
+            else pk.PA_ERR_INVALID
+        assert d8(**bad) == want, bad
+    assert d8(B=0) == pk.PA_OK
+    r = lambda dtype=pk.PA_F16, ks=1.0, vs=1.0, **kw: L.pa_reshape_and_cache_fp8(
+        FAKE, FAKE, FAKE, FAKE, kw.get("slots", FAKE), kw.get("N", 4), 2, kw.get("D", 128), 16,
+        10, dtype, ks, vs, None)
+    assert r(dtype=pk.PA_FP8_E4M3) == pk.PA_ERR_INVALID
+    assert r(ks=0.0) == pk.PA_ERR_INVALID
+    assert r(vs=float("nan")) == pk.PA_ERR_INVALID
+    assert r(D=80) == pk.PA_ERR_UNSUPPORTED
+    assert r(slots=FAKE + 4) == pk.PA_ERR_INVALID
+    assert r(N=0) == pk.PA_OK
+    assert pk.pa_launch_count() == before

@@ -91,3 +91,17 @@ def test_partition_kernel_choice():
     assert bench.partition_kernel(W.OPT13B, 512) == "decode_partition_kernel"
     assert bench.partition_kernel(W.GQA70B, 96) == "decode_partition_kernel"
     assert bench.partition_kernel(W.TINY, 512) == "decode_partition_kernel"
+    assert bench.partition_kernel(W.fp8(W.GQA70B), 2048) == "decode_partition_kernel"
+
+
+def test_fp8_workloads_count_one_byte_per_element():
+    spec = W.fp8(W.Spec("t", "bf16", 8, 2, 128, 16, "independent", 3, seed=1))
+    tables = np.array([[5, 6], [5, 7], [9, -1]], dtype=np.int32)
+    lens = np.array([20, 18, 16], dtype=np.int32)
+    unique, logical, other = bench.step_bytes(spec, tables, lens)
+    row = 2 * 2 * 128 * 1                      # K and V, 2 kv heads, D 128, one byte each
+    assert logical == (20 + 18 + 16) * row and unique == (16 + 4 + 2 + 16) * row
+    assert other == 2 * 3 * 8 * 128 * 2 + (2 + 2 + 1) * 4 + 3 * 4   # q / out stay bf16
+    s = bench.workload_spec("opt13b_fp8")
+    assert s.fp8 and s.dtype == "f16" and s.num_seqs == W.OPT13B.num_seqs
+    assert "E4M3" in bench.workload_text("gqa70b_fp8")

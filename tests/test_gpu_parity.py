@@ -288,3 +288,88 @@ def test_full_size_workloads_sampled(name):
     got = got_all[rows[:, 0], rows[:, 1]]
     assert np.isfinite(got_all).all()
     assert np.abs(got - want).max() <= TOL[spec.dtype]
+
+
+# ---------------------------------------------------------------------------
+# E4M3 caches: the quantising append bit-exact against the oracle's, attention
+# within the output dtype's tolerance of the oracle's fp64 attention over the
+# same codes (unused slots hold the E4M3 NaN code)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("scales", [(1.0, 1.0), (0.0123, 0.0171)])
+def test_fp8_append_is_bit_exact(dtype, scales):
+    tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[dtype]
+    code = W.DTYPE_CODES[dtype]
+    g = torch.Generator().manual_seed(31)
+    N, Hkv, D, bs, NB = 40, 2, 128, 16, 8
+    k = torch.randn((N, Hkv, D), generator=g) * torch.exp(torch.randn((N, Hkv, D), generator=g) * 3)
+    v = torch.randn((N, Hkv, D), generator=g)
+    # saturation, signed zeros, subnormal codes, exact ties (for scale 1)
+    special = torch.tensor([1e4, -1e4, 448.0, 464.0, 0.0, -0.0, 0.001953125, 0.0048828125,
+                            1.0625, 17.0, -1.1875, 240.0 + 8.0])
+    k[0, 0, :special.numel()] = special
+    k, v = k.to(tdt), v.to(tdt)
+    k_scale, v_scale = (float(np.float32(x)) for x in scales)
+    kc = torch.full((NB, Hkv, bs, D), 0x7f, dtype=torch.uint8, device="cuda").view(torch.float8_e4m3fn)
+    vc = kc.clone()
+    slots = torch.randperm(NB * bs, generator=g)[:N].to(torch.int64)
+    slots[3] = -1
+    pk.pa_reshape_and_cache_fp8(k.cuda(), v.cuda(), kc, vc, slots.cuda(), k_scale, v_scale)
+    torch.cuda.synchronize()
+    assert pk.pa_device_status() == 0
+    ok = np.full((NB, Hkv, bs, D), 0x7f, dtype=np.uint8)
+    ov = ok.copy()
+    oracle.reshape_and_cache_e4m3(W.storage_view(k), W.storage_view(v), ok, ov, slots.numpy(),
+                                  code, k_scale, v_scale)
+    assert np.array_equal(W.storage_view(kc), ok)
+    assert np.array_equal(W.storage_view(vc), ov)
+
+
+@pytest.mark.parametrize("name", ["tiny", "opt13b", "llama13b_ps", "gqa70b", "long_prefix"])
+def test_fp8_small_workloads(name):
+    full_check(W.fp8(W.small(name)))
+
+
+@pytest.mark.parametrize("P", [32, 64, 96, 256, 4096])
+def test_fp8_partition_sizes(P):
+    full_check(W.fp8(W.small("opt13b")), partition_size=P)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_fp8_dtype_head_group_matrix(dtype, D, G):
+    spec = W.Spec(f"m8_{dtype}_{D}_{G}", dtype, 2 * G, 2, D, 16, "independent", 5,
+                  seed=91 + G + D, ctx_dist="explicit", ctx_list=(1, 77, 300, 513, 1100),
+                  partition_size=256)
+    full_check(W.fp8(spec))
+
+
+def test_fp8_edge_context_lengths():
+    lens = (0, 1, 15, 16, 17, 31, 32, 33, 63, 64, 65, 511, 512, 513, 1024, 1025, 2047)
+    spec = W.fp8(W.Spec("edges8", "f16", 8, 8, 128, 16, "independent", len(lens), seed=6,
+                        ctx_dist="explicit", ctx_list=lens, partition_size=512))
+    got, _ = full_check(spec)
+    assert np.all(got[0] == 0.0)
+    full_check(replace(spec, block_size=8, name="edges8_bs8", partition_size=96))
+    full_check(replace(spec, block_size=32, name="edges8_bs32", partition_size=64))
+
+
+@pytest.mark.parametrize("name", ["opt13b", "gqa70b", "long_prefix_bs16"])
+def test_fp8_full_size_workloads_sampled(name):
+    base = W.long_prefix(16) if name.startswith("long_prefix") else W.FULL[name]
+    spec = W.fp8(base)
+    sc = W.scenario(spec)
+    p, o = build(sc)
+    out = run_step(p, spec)
+    torch.cuda.synchronize()
+    assert pk.pa_device_status() == 0
+    check_bookkeeping(p, o)
+    touched = sorted({s // spec.block_size for s in o.slots} | {d for _, d in o.pairs})
+    check_caches(p, o, blocks=touched)
+    rows = sampled_rows(o, spec)
+    want = oracle_attention(o, spec, rows=rows)
+    got_all = as_f64(out, spec)
+    assert np.isfinite(got_all).all()
+    assert np.abs(got_all[rows[:, 0], rows[:, 1]] - want).max() <= TOL[spec.dtype]

@@ -23,6 +23,13 @@ not available here; shapes follow the public model configurations):
                blocks) plus a unique suffix ~ U[1,28672]; Hq=32, Hkv=8, D=128,
                bf16, block 8/16/32, split-K partitions of 512 tokens
 
+Any workload can keep its cache as E4M3 codes (``fp8(spec)``, named with an
+``_fp8`` suffix): K/V are drawn as usual in the workload's dtype (which stays
+the query / output type) and quantised on append with per-cache scales
+k_scale = 0.0123 and v_scale = 0.0171 (N(0,1) contents span about +-5.5, i.e.
+codes up to about 450 / 320 before saturation; the values are not powers of
+two, so the fp32 quotient really rounds).
+
 Choices the workload descriptions leave open (stated here and in the design
 notes): the lognormal sigma 0.5; integer-uniform prompt, divergent and suffix
 lengths; pool sizes of 1.25x the blocks needed (rounded up) where no pool is
@@ -39,8 +46,9 @@ from typing import List, Optional, Tuple
 
 import numpy as np
 
-DTYPE_CODES = {"f32": 0, "f16": 1, "bf16": 2}
-DTYPE_BYTES = {"f32": 4, "f16": 2, "bf16": 2}
+DTYPE_CODES = {"f32": 0, "f16": 1, "bf16": 2, "e4m3": 3}
+DTYPE_BYTES = {"f32": 4, "f16": 2, "bf16": 2, "e4m3": 1}
+FP8_K_SCALE, FP8_V_SCALE = 0.0123, 0.0171
 
 
 @dataclass(frozen=True)
@@ -75,6 +83,10 @@ class Spec:
     prefix_len: int = 0
     suffix_lo: int = 0
     suffix_hi: int = 0
+    # cache storage: "" = the dtype itself, "e4m3" = E4M3 codes with these scales
+    kv_dtype: str = ""
+    k_scale: float = 1.0
+    v_scale: float = 1.0
 
     @property
     def dtype_code(self) -> int:
@@ -83,6 +95,22 @@ class Spec:
     @property
     def esize(self) -> int:
         return DTYPE_BYTES[self.dtype]
+
+    @property
+    def kv(self) -> str:
+        return self.kv_dtype or self.dtype
+
+    @property
+    def kv_code(self) -> int:
+        return DTYPE_CODES[self.kv]
+
+    @property
+    def kv_esize(self) -> int:
+        return DTYPE_BYTES[self.kv]
+
+    @property
+    def fp8(self) -> bool:
+        return self.kv == "e4m3"
 
     @property
     def G(self) -> int:
@@ -108,6 +136,12 @@ LONG_PREFIX = Spec("long_prefix", "bf16", 32, 8, 128, 16, "shared_prefix", 128, 
                    prefix_len=4096, suffix_lo=1, suffix_hi=28672, partition_size=512)
 
 FULL = {s.name: s for s in (TINY, OPT13B, LLAMA13B_PS, GQA70B, LONG_PREFIX)}
+
+
+def fp8(spec: Spec) -> Spec:
+    """The workload with an E4M3 cache (queries and outputs keep spec.dtype)."""
+    return replace(spec, name=spec.name + "_fp8", kv_dtype="e4m3",
+                   k_scale=float(np.float32(FP8_K_SCALE)), v_scale=float(np.float32(FP8_V_SCALE)))
 
 
 def long_prefix(block_size: int) -> Spec:
@@ -256,8 +290,15 @@ def _gen(device, seed: int):
 
 
 def torch_dtype(spec: Spec):
+    """Query / output (and new K/V) dtype."""
     import torch
     return {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[spec.dtype]
+
+
+def torch_kv_dtype(spec: Spec):
+    """Cache storage dtype."""
+    import torch
+    return torch.float8_e4m3fn if spec.fp8 else torch_dtype(spec)
 
 
 def kv_content(spec: Spec, kv_id: int, n: int, device="cpu"):
@@ -279,16 +320,19 @@ def q_content(spec: Spec, B: int, device="cpu"):
 
 
 def poison_value(spec: Spec):
-    """Fill for every cache slot no token was written to (NaN): a kernel that
-    reads an unused tail slot into its result turns the output into NaN."""
+    """Fill for every cache slot no token was written to (NaN; the E4M3 NaN
+    code for E4M3 caches): a kernel that reads an unused tail slot into its
+    result turns the output into NaN."""
     return float("nan")
 
 
 def storage_view(t):
     """A CPU tensor as the numpy array of its stored bits (float32 stays
-    float32; fp16 / bf16 become uint16 bit patterns)."""
+    float32; fp16 / bf16 become uint16 bit patterns, E4M3 uint8 codes)."""
     import torch
     t = t.detach().contiguous().cpu()
     if t.dtype == torch.float32:
         return t.numpy()
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).numpy()
     return t.view(torch.int16).numpy().view(np.uint16)

@@ -17,7 +17,9 @@
  *   [P2] blog.aqudi.me, "3. vLLM: KV cache를 블록 단위로 관리하기" (a new block
  *        when the current one fills; copy-on-write of shared prompt blocks).
  *   [P3] hjr-study-book Day 3, "1. KV 캐시란" (each decode step stores the new
- *        token's K and V) and "4.2 PagedAttention의 접근" (block-table example).
+ *        token's K and V), "4.2 PagedAttention의 접근" (block-table example) and
+ *        "5. Prefix Caching" (the KV blocks of a repeated prompt prefix are
+ *        reused across requests).
  *
  * Conventions for every call below:
  *   - Shapes use B = num_seqs, Hq = num_heads (query heads), Hkv = num_kv_heads,
@@ -357,7 +359,8 @@ pa_status pa_alloc_create(int num_blocks, int block_size, const int32_t* initial
                           pa_allocator** out);
 void pa_alloc_destroy(pa_allocator* a);
 
-/* Free blocks left; -1 for a NULL handle. */
+/* Blocks an allocation can take: the free stack plus, with prefix caching, the
+ * evictable cached blocks; -1 for a NULL handle. */
 int pa_alloc_num_free(const pa_allocator* a);
 
 /* Reference count of a block (number of sequences using it); -1 if out of range. */
@@ -386,16 +389,47 @@ pa_status pa_seq_append(pa_allocator* a, int64_t seq_id, int n_tokens, int64_t* 
                         int64_t* cow_pair_out, int* n_cow);
 
 /* Drops the sequence; its blocks lose one reference each, in logical order, and
- * blocks reaching zero are pushed on the free stack. */
+ * blocks reaching zero are pushed on the free stack (cached blocks of a prefix
+ * cache go to the back of the evictable list instead). */
 pa_status pa_seq_free(pa_allocator* a, int64_t seq_id);
+
+/*
+ * Prefix caching ([P3] "5. Prefix Caching"; [P2] "4. 이 밖의 기법들": the KV
+ * blocks of a prompt prefix that repeats across requests are reused).  The
+ * pages give no mechanism; this library's:
+ *   - each full block of a committed sequence is keyed by its content chain,
+ *     (key of the previous block or none, the block's block_size token ids),
+ *     compared exactly (no hash aliasing);
+ *   - pa_seq_add_cached creates a sequence holding the cached blocks of the
+ *     longest run of its leading full blocks whose keys are cached, stopping at
+ *     the first miss and leaving at least one token uncached; *num_cached
+ *     receives the tokens covered (a multiple of block_size).  The caller then
+ *     appends the remaining tokens with pa_seq_append and writes their K/V;
+ *   - pa_seq_commit registers the full blocks among the sequence's first
+ *     num_tokens tokens (token_ids from the start of the sequence); a key that
+ *     already has a block keeps it, and a block keeps its first key;
+ *   - a cached block whose count reaches zero stays cached as evictable; an
+ *     allocation takes the free stack first, then the least recently released
+ *     evictable block, whose key is dropped.
+ * pa_alloc_enable_prefix_cache turns this on (before or after blocks are in
+ * use); without it pa_seq_add_cached behaves as pa_seq_add (*num_cached = 0)
+ * and pa_seq_commit does nothing.  pa_alloc_evictable copies the evictable
+ * list, first to be evicted first, into out[0..capacity); *n_out = its size.
+ */
+pa_status pa_alloc_enable_prefix_cache(pa_allocator* a);
+pa_status pa_alloc_evictable(const pa_allocator* a, int32_t* out, int capacity, int* n_out);
+pa_status pa_seq_add_cached(pa_allocator* a, int64_t seq_id, const int32_t* token_ids,
+                            int num_tokens, int* num_cached);
+pa_status pa_seq_commit(pa_allocator* a, int64_t seq_id, const int32_t* token_ids,
+                        int num_tokens);
 
 /*
  * Moves sequences from manager `src` to manager `dst` (same block size), e.g.
  * to a pinned host pool when GPU memory runs short and back again ([P1]
  * "적용 범위와 관련 연구").  Sharing among the sequences moved together is kept:
  * walking seq_ids in order and each one's blocks in logical order, a source
- * block met for the first time takes a fresh destination block (popped from
- * dst's free stack) and the pair (src block, dst block) is appended to
+ * block met for the first time takes a fresh destination block (as an
+ * allocation in dst) and the pair (src block, dst block) is appended to
  * pairs_out [pairs_capacity][2]; every later holder shares that block.  The
  * token counts move unchanged; then each sequence is freed in `src` in caller
  * order (as pa_seq_free).  The caller runs pa_swap_blocks on the *n_pairs pairs

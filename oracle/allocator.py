@@ -40,7 +40,17 @@ implementations can agree exactly):
     the caller's order and through each one's blocks in logical order, a block
     seen for the first time takes the destination's next free block, and later
     holders share it; the sequences are then released in the source in the
-    caller's order.
+    caller's order;
+  * prefix caching ("5. Prefix Caching", hjr-study-book Day 3, and "prefix
+    caching" in "4. 이 밖의 기법들", blog.aqudi.me: the KV blocks of a prompt
+    prefix repeated across requests are reused; no mechanism is given): a full
+    block's key is its content chain (previous block's key, its token ids); a
+    new request takes the cached blocks of its leading full blocks up to the
+    first key with no block, leaving at least one token to compute; committing
+    a sequence registers its full blocks (a key keeps its first block, a block
+    its first key); a cached block whose count drops to zero waits on an
+    evictable list (least recently released evicted first), and an allocation
+    takes the free stack before evicting.
 """
 from dataclasses import dataclass, field
 from typing import Dict, List, Optional, Sequence, Tuple
@@ -76,10 +86,33 @@ class BlockManager:
             self.free = order
         self.refcount = [0] * num_blocks
         self.seqs: Dict[int, _Seq] = {}
+        self.prefix = False
+        self.block_of_key: Dict[tuple, int] = {}
+        self.key_of_block: Dict[int, tuple] = {}
+        self.evictable: List[int] = []
+
+    # -- block hand-out and release (shared by every operation) --
+    def _take(self) -> int:
+        if self.free:
+            blk = self.free.pop()
+        else:                                   # evict the least recently released
+            blk = self.evictable.pop(0)
+            del self.block_of_key[self.key_of_block.pop(blk)]
+        self.refcount[blk] = 1
+        return blk
+
+    def _drop(self, blk: int) -> None:
+        self.refcount[blk] -= 1
+        if self.refcount[blk] == 0:
+            if self.prefix and blk in self.key_of_block:
+                self.evictable.append(blk)
+            else:
+                self.free.append(blk)
 
     # -- queries --
     def num_free(self) -> int:
-        return len(self.free)
+        """Blocks an allocation can take (free stack + evictable)."""
+        return len(self.free) + len(self.evictable)
 
     def free_stack(self) -> List[int]:
         """The free stack bottom to top (the last entry is handed out next)."""
@@ -127,20 +160,17 @@ class BlockManager:
         blocks_after = -(-(T + n_tokens) // bs)
         new_blocks = blocks_after - len(s.blocks)
         need = new_blocks + (1 if cow else 0)
-        if need > len(self.free):
+        if need > self.num_free():
             raise OOM("not enough free blocks")
         pairs: List[Tuple[int, int]] = []
         if cow:
             old = s.blocks[-1]
-            dst = self.free.pop()
-            self.refcount[dst] = 1
-            self.refcount[old] -= 1
+            dst = self._take()
+            self._drop(old)                     # still held by its other sharers
             s.blocks[-1] = dst
             pairs.append((old, dst))
         for _ in range(new_blocks):
-            blk = self.free.pop()
-            self.refcount[blk] = 1
-            s.blocks.append(blk)
+            s.blocks.append(self._take())
         slots = [s.blocks[t // bs] * bs + t % bs for t in range(T, T + n_tokens)]
         s.num_tokens = T + n_tokens
         return slots, pairs
@@ -150,9 +180,7 @@ class BlockManager:
         if seq_id not in self.seqs:
             raise Invalid("unknown sequence")
         for blk in self.seqs.pop(seq_id).blocks:
-            self.refcount[blk] -= 1
-            if self.refcount[blk] == 0:
-                self.free.append(blk)
+            self._drop(blk)
 
     def move_to(self, dst: "BlockManager", seq_ids: Sequence[int]) -> List[Tuple[int, int]]:
         """Move the sequences into dst; returns the (source block, dst block)
@@ -166,7 +194,7 @@ class BlockManager:
             if sid not in self.seqs or sid in dst.seqs:
                 raise Invalid("unknown sequence or already in the destination")
         distinct = {blk for sid in seq_ids for blk in self.seqs[sid].blocks}
-        if len(distinct) > len(dst.free):
+        if len(distinct) > dst.num_free():
             raise OOM("not enough free blocks in the destination")
         where: Dict[int, int] = {}
         pairs: List[Tuple[int, int]] = []
@@ -177,8 +205,7 @@ class BlockManager:
                 if blk in where:
                     dst.refcount[where[blk]] += 1
                 else:
-                    new = dst.free.pop()
-                    dst.refcount[new] = 1
+                    new = dst._take()
                     where[blk] = new
                     pairs.append((blk, new))
                 mapped.append(where[blk])
@@ -186,6 +213,51 @@ class BlockManager:
         for sid in seq_ids:
             self.release(sid)
         return pairs
+
+    # -- prefix caching --
+    def enable_prefix_cache(self) -> None:
+        self.prefix = True
+
+    def add_cached(self, seq_id: int, token_ids: Sequence[int]) -> int:
+        """New sequence holding the cached blocks of its leading full blocks;
+        returns the number of tokens they cover."""
+        if seq_id in self.seqs:
+            raise Invalid("sequence exists")
+        toks = [int(t) for t in token_ids]
+        bs = self.block_size
+        blocks: List[int] = []
+        if self.prefix and toks:
+            key = None
+            for k in range((len(toks) - 1) // bs):
+                key = (key, tuple(toks[k * bs:(k + 1) * bs]))
+                blk = self.block_of_key.get(key)
+                if blk is None:
+                    break
+                if self.refcount[blk] == 0:
+                    self.evictable.remove(blk)
+                self.refcount[blk] += 1
+                blocks.append(blk)
+        self.seqs[seq_id] = _Seq(blocks, len(blocks) * bs)
+        return len(blocks) * bs
+
+    def commit(self, seq_id: int, token_ids: Sequence[int]) -> None:
+        """Register the sequence's full blocks under their content keys."""
+        if seq_id not in self.seqs:
+            raise Invalid("unknown sequence")
+        toks = [int(t) for t in token_ids]
+        s = self.seqs[seq_id]
+        if len(toks) > s.num_tokens:
+            raise Invalid("more tokens than the sequence holds")
+        if not self.prefix:
+            return
+        bs = self.block_size
+        key = None
+        for k in range(len(toks) // bs):
+            key = (key, tuple(toks[k * bs:(k + 1) * bs]))
+            blk = s.blocks[k]
+            if key not in self.block_of_key and blk not in self.key_of_block:
+                self.block_of_key[key] = blk
+                self.key_of_block[blk] = key
 
     def build_tables(self, seq_ids: Sequence[int], max_blocks: int):
         """Block tables [B][max_blocks] (padding -1) and context lengths [B]."""

@@ -36,6 +36,7 @@ EXPORTS = (
     "pa_copy_blocks", "pa_swap_blocks", "pa_alloc_create", "pa_alloc_destroy", "pa_alloc_num_free",
     "pa_alloc_refcount", "pa_alloc_free_stack", "pa_seq_add", "pa_seq_fork", "pa_seq_append",
     "pa_seq_free", "pa_seq_move", "pa_seq_num_tokens", "pa_build_tables",
+    "pa_alloc_enable_prefix_cache", "pa_alloc_evictable", "pa_seq_add_cached", "pa_seq_commit",
 )
 
 
@@ -103,6 +104,10 @@ def lib():
         "pa_seq_append": ([vp, i64, i32, pi64, pi64, ctypes.POINTER(i32)], i32),
         "pa_seq_free": ([vp, i64], i32),
         "pa_seq_move": ([vp, vp, pi64, i32, pi64, i32, ctypes.POINTER(i32)], i32),
+        "pa_alloc_enable_prefix_cache": ([vp], i32),
+        "pa_alloc_evictable": ([vp, pi32, i32, ctypes.POINTER(i32)], i32),
+        "pa_seq_add_cached": ([vp, i64, pi32, i32, ctypes.POINTER(i32)], i32),
+        "pa_seq_commit": ([vp, i64, pi32, i32], i32),
         "pa_seq_num_tokens": ([vp, i64, ctypes.POINTER(i32)], i32),
         "pa_build_tables": ([vp, pi64, i32, i32, pi32, pi32], i32),
     }
@@ -418,6 +423,37 @@ def pa_seq_move(src, dst, seq_ids: Sequence[int], capacity: int) -> List[Tuple[i
     return [(buf[2 * i], buf[2 * i + 1]) for i in range(n.value)]
 
 
+def pa_alloc_enable_prefix_cache(h) -> None:
+    _check(lib().pa_alloc_enable_prefix_cache(h))
+
+
+def pa_alloc_evictable(h) -> List[int]:
+    n = ctypes.c_int(0)
+    _check(lib().pa_alloc_evictable(h, None, 0, ctypes.byref(n)))
+    buf = (ctypes.c_int32 * max(1, n.value))()
+    _check(lib().pa_alloc_evictable(h, buf, n.value, ctypes.byref(n)))
+    return list(buf[:n.value])
+
+
+def _tokens(token_ids):
+    t = [int(x) for x in token_ids]
+    return (ctypes.c_int32 * max(1, len(t)))(*t), len(t)
+
+
+def pa_seq_add_cached(h, seq_id: int, token_ids) -> int:
+    """New sequence holding the cached blocks of its prompt's leading full
+    blocks; returns the number of tokens they cover."""
+    buf, n = _tokens(token_ids)
+    got = ctypes.c_int(0)
+    _check(lib().pa_seq_add_cached(h, seq_id, buf, n, ctypes.byref(got)))
+    return got.value
+
+
+def pa_seq_commit(h, seq_id: int, token_ids) -> None:
+    buf, n = _tokens(token_ids)
+    _check(lib().pa_seq_commit(h, seq_id, buf, n))
+
+
 def pa_seq_num_tokens(h, seq_id: int) -> int:
     n = ctypes.c_int(0)
     _check(lib().pa_seq_num_tokens(h, seq_id, ctypes.byref(n)))
@@ -479,6 +515,18 @@ class BlockAllocator:
 
     def num_tokens(self, seq_id):
         return pa_seq_num_tokens(self.h, seq_id)
+
+    def enable_prefix_cache(self):
+        pa_alloc_enable_prefix_cache(self.h)
+
+    def evictable(self):
+        return pa_alloc_evictable(self.h)
+
+    def add_cached(self, seq_id, token_ids) -> int:
+        return pa_seq_add_cached(self.h, seq_id, token_ids)
+
+    def commit(self, seq_id, token_ids):
+        pa_seq_commit(self.h, seq_id, token_ids)
 
     def move_to(self, dst: "BlockAllocator", seq_ids):
         """Move sequences to another manager (sharing kept); returns copy pairs."""

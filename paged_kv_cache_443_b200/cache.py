@@ -36,7 +36,8 @@ class PagedKVCache:
 
     def __init__(self, num_blocks: int, block_size: int, num_kv_heads: int, head_size: int,
                  dtype: torch.dtype, device="cuda", initial_free_order: Optional[Sequence[int]] = None,
-                 fill: Optional[float] = None, k_scale: float = 1.0, v_scale: float = 1.0):
+                 fill: Optional[float] = None, k_scale: float = 1.0, v_scale: float = 1.0,
+                 prefix_cache: bool = False):
         self.num_blocks, self.block_size = num_blocks, block_size
         self.num_kv_heads, self.head_size = num_kv_heads, head_size
         self.dtype, self.device = dtype, torch.device(device)
@@ -50,6 +51,8 @@ class PagedKVCache:
             self.k_cache = _filled(shape, fill, dtype, self.device)
             self.v_cache = _filled(shape, fill, dtype, self.device)
         self.alloc = BlockAllocator(num_blocks, block_size, initial_free_order)
+        if prefix_cache:
+            self.alloc.enable_prefix_cache()
         self.host_alloc = None
         self.host_k = self.host_v = None
 
@@ -62,6 +65,17 @@ class PagedKVCache:
 
     def release(self, seq_id: int) -> None:
         self.alloc.release(seq_id)
+
+    # ---- prefix caching ("5. Prefix Caching", hjr-study-book Day 3) ----
+    def add_cached(self, seq_id: int, token_ids: Sequence[int]) -> int:
+        """New request: takes the cached blocks of its prompt's leading full
+        blocks and returns how many tokens they cover; the caller appends the
+        K/V of the rest (append) and then commits the prompt."""
+        return self.alloc.add_cached(seq_id, token_ids)
+
+    def commit(self, seq_id: int, token_ids: Sequence[int]) -> None:
+        """Make the sequence's full blocks of token_ids reusable by later requests."""
+        self.alloc.commit(seq_id, token_ids)
 
     def reserve(self, seq_ids: Sequence[int], counts: Sequence[int]
                 ) -> Tuple[List[int], List[Tuple[int, int]]]:

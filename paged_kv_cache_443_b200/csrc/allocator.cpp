@@ -14,10 +14,26 @@
 // first time it is met (sequences in caller order, blocks in logical order),
 // and every later holder shares it.
 //
+// Prefix caching ("5. Prefix Caching", hjr-study-book Day 3; "prefix caching"
+// in "4. 이 밖의 기법들", blog.aqudi.me: the KV blocks of a prompt prefix that
+// repeats across requests are reused).  The pages give no mechanism; this one
+// keys every full block by its content chain -- (key of the previous block,
+// the block's token ids) -- interned as nodes of a trie, so a lookup compares
+// token ids exactly and no hash collision can alias two prefixes.  A request
+// takes the cached blocks of its longest cached chain of full blocks, leaving
+// at least one token to compute.  A cached block whose count drops to zero is
+// not freed but becomes evictable (least recently released first); blocks are
+// taken from the free stack first and only then by evicting, which drops the
+// block's key.
+//
 // Storage: one flat refcount array, a free stack, and a hash map from sequence
-// id to its block list.  Every operation is O(blocks touched).
+// id to its block list; with prefix caching a trie of keys, the block of each
+// key, and an LRU list of evictable blocks.  Every operation is O(blocks
+// touched).
 #include <cstdint>
 #include <cstring>
+#include <functional>
+#include <list>
 #include <new>
 #include <unordered_map>
 #include <vector>
@@ -30,17 +46,79 @@ struct pa_allocator {
     std::vector<int32_t> blocks;
     int64_t tokens = 0;
   };
+  struct Key {  // a full block's content chain: parent node (-1 = none), token ids
+    int64_t parent;
+    std::vector<int32_t> tokens;
+    bool operator==(const Key& o) const { return parent == o.parent && tokens == o.tokens; }
+  };
+  struct KeyHash {
+    size_t operator()(const Key& k) const {
+      uint64_t h = 1469598103934665603ull ^ static_cast<uint64_t>(k.parent);
+      for (int32_t t : k.tokens) h = (h ^ static_cast<uint32_t>(t)) * 1099511628211ull;
+      return static_cast<size_t>(h);
+    }
+  };
   int32_t num_blocks = 0;
   int32_t block_size = 0;
   std::vector<int32_t> free_stack;  // back() is handed out next
   std::vector<int32_t> refcount;
   std::unordered_map<int64_t, Seq> seqs;
+  // prefix cache
+  bool prefix = false;
+  std::unordered_map<Key, int64_t, KeyHash> nodes;  // content chain -> node id
+  std::vector<int32_t> node_block;                  // node -> cached block or -1
+  std::vector<int64_t> block_node;                  // block -> node or -1
+  std::list<int32_t> evictable;                     // front is evicted first
+  std::vector<std::list<int32_t>::iterator> evict_pos;
+
+  size_t available() const { return free_stack.size() + evictable.size(); }
 
   int32_t pop() {
-    int32_t b = free_stack.back();
-    free_stack.pop_back();
+    int32_t b;
+    if (!free_stack.empty()) {
+      b = free_stack.back();
+      free_stack.pop_back();
+    } else {  // evict the least recently released cached block
+      b = evictable.front();
+      evictable.pop_front();
+      node_block[block_node[b]] = -1;
+      block_node[b] = -1;
+    }
     refcount[b] = 1;
     return b;
+  }
+
+  // one reference fewer; at zero the block is freed, or kept evictable if cached
+  void unref(int32_t b) {
+    if (--refcount[b] != 0) return;
+    if (prefix && block_node[b] >= 0) {
+      evictable.push_back(b);
+      evict_pos[b] = std::prev(evictable.end());
+    } else {
+      free_stack.push_back(b);
+    }
+  }
+
+  // one reference more to a cached block (taken back from the evictable list at zero)
+  void ref_cached(int32_t b) {
+    if (refcount[b] == 0) evictable.erase(evict_pos[b]);
+    refcount[b] += 1;
+  }
+
+  int64_t find_node(int64_t parent, const int32_t* tokens) const {
+    Key k{parent, std::vector<int32_t>(tokens, tokens + block_size)};
+    auto it = nodes.find(k);
+    return it == nodes.end() ? -1 : it->second;
+  }
+
+  int64_t intern(int64_t parent, const int32_t* tokens) {
+    Key k{parent, std::vector<int32_t>(tokens, tokens + block_size)};
+    auto it = nodes.find(k);
+    if (it != nodes.end()) return it->second;
+    const int64_t id = static_cast<int64_t>(node_block.size());
+    nodes.emplace(std::move(k), id);
+    node_block.push_back(-1);
+    return id;
   }
 };
 
@@ -78,7 +156,7 @@ extern "C" pa_status pa_alloc_create(int num_blocks, int block_size,
 extern "C" void pa_alloc_destroy(pa_allocator* a) { delete a; }
 
 extern "C" int pa_alloc_num_free(const pa_allocator* a) {
-  return a ? static_cast<int>(a->free_stack.size()) : -1;
+  return a ? static_cast<int>(a->available()) : -1;
 }
 
 extern "C" int pa_alloc_refcount(const pa_allocator* a, int32_t block) {
@@ -94,6 +172,81 @@ extern "C" pa_status pa_alloc_free_stack(const pa_allocator* a, int32_t* out, in
   *n_out = n;
   const int m = n < capacity ? n : capacity;
   if (m > 0) std::memcpy(out, a->free_stack.data(), sizeof(int32_t) * m);
+  return PA_OK;
+}
+
+extern "C" pa_status pa_alloc_enable_prefix_cache(pa_allocator* a) {
+  if (!a) return pa::fail(PA_ERR_INVALID, "pa_alloc_enable_prefix_cache: NULL handle");
+  if (!a->prefix) {
+    a->prefix = true;
+    a->block_node.assign(a->num_blocks, -1);
+    a->evict_pos.resize(a->num_blocks);
+  }
+  return PA_OK;
+}
+
+extern "C" pa_status pa_alloc_evictable(const pa_allocator* a, int32_t* out, int capacity,
+                                        int* n_out) {
+  if (!a || !n_out || capacity < 0 || (capacity > 0 && !out))
+    return pa::fail(PA_ERR_INVALID, "pa_alloc_evictable: bad argument");
+  const int n = static_cast<int>(a->evictable.size());
+  *n_out = n;
+  int i = 0;
+  for (auto it = a->evictable.begin(); it != a->evictable.end() && i < capacity; ++it) out[i++] = *it;
+  return PA_OK;
+}
+
+extern "C" pa_status pa_seq_add_cached(pa_allocator* a, int64_t seq_id, const int32_t* token_ids,
+                                       int num_tokens, int* num_cached) {
+  const char* fn = "pa_seq_add_cached";
+  if (!a || !num_cached || num_tokens < 0 || (num_tokens > 0 && !token_ids))
+    return pa::fail(PA_ERR_INVALID, "%s: bad argument", fn);
+  if (a->seqs.count(seq_id))
+    return pa::fail(PA_ERR_INVALID, "%s: sequence %lld exists", fn, (long long)seq_id);
+  pa_allocator::Seq s;
+  if (a->prefix && num_tokens > 0) {
+    const int bs = a->block_size;
+    const int full = (num_tokens - 1) / bs;  // leave at least one token to compute
+    int64_t parent = -1;
+    for (int k = 0; k < full; ++k) {
+      const int64_t node = a->find_node(parent, token_ids + static_cast<int64_t>(k) * bs);
+      if (node < 0 || a->node_block[node] < 0) break;
+      const int32_t b = a->node_block[node];
+      a->ref_cached(b);
+      s.blocks.push_back(b);
+      parent = node;
+    }
+    s.tokens = static_cast<int64_t>(s.blocks.size()) * bs;
+  }
+  *num_cached = static_cast<int>(s.tokens);
+  a->seqs.emplace(seq_id, std::move(s));
+  return PA_OK;
+}
+
+extern "C" pa_status pa_seq_commit(pa_allocator* a, int64_t seq_id, const int32_t* token_ids,
+                                   int num_tokens) {
+  const char* fn = "pa_seq_commit";
+  if (!a || num_tokens < 0 || (num_tokens > 0 && !token_ids))
+    return pa::fail(PA_ERR_INVALID, "%s: bad argument", fn);
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end())
+    return pa::fail(PA_ERR_INVALID, "%s: unknown sequence %lld", fn, (long long)seq_id);
+  if (num_tokens > it->second.tokens)
+    return pa::fail(PA_ERR_INVALID, "%s: %d tokens given, the sequence holds %lld", fn,
+                    num_tokens, (long long)it->second.tokens);
+  if (!a->prefix) return PA_OK;
+  const int bs = a->block_size;
+  int64_t parent = -1;
+  for (int k = 0; k < num_tokens / bs; ++k) {
+    const int64_t node = a->intern(parent, token_ids + static_cast<int64_t>(k) * bs);
+    const int32_t b = it->second.blocks[k];
+    // first writer wins: a key keeps its block, a block keeps its key
+    if (a->node_block[node] < 0 && a->block_node[b] < 0) {
+      a->node_block[node] = b;
+      a->block_node[b] = node;
+    }
+    parent = node;
+  }
   return PA_OK;
 }
 
@@ -136,9 +289,9 @@ extern "C" pa_status pa_seq_append(pa_allocator* a, int64_t seq_id, int n_tokens
   const bool tail_partial = (s.tokens % bs) != 0;
   const bool cow = tail_partial && a->refcount[s.blocks.back()] > 1;
   const int64_t need = (want - have) + (cow ? 1 : 0);
-  if (need > static_cast<int64_t>(a->free_stack.size()))
+  if (need > static_cast<int64_t>(a->available()))
     return pa::fail(PA_ERR_OOM, "pa_seq_append: need %lld blocks, %zu free", (long long)need,
-                    a->free_stack.size());
+                    a->available());
   if (cow) {
     const int32_t old = s.blocks.back();
     const int32_t fresh = a->pop();
@@ -162,9 +315,7 @@ extern "C" pa_status pa_seq_free(pa_allocator* a, int64_t seq_id) {
   auto it = a->seqs.find(seq_id);
   if (it == a->seqs.end())
     return pa::fail(PA_ERR_INVALID, "pa_seq_free: unknown sequence %lld", (long long)seq_id);
-  for (int32_t b : it->second.blocks) {
-    if (--a->refcount[b] == 0) a->free_stack.push_back(b);
-  }
+  for (int32_t b : it->second.blocks) a->unref(b);
   a->seqs.erase(it);
   return PA_OK;
 }
@@ -197,9 +348,9 @@ extern "C" pa_status pa_seq_move(pa_allocator* src, pa_allocator* dst, const int
     for (int32_t b : it->second.blocks)
       if (map.emplace(b, -1).second) ++distinct;
   }
-  if (distinct > static_cast<int64_t>(dst->free_stack.size()))
+  if (distinct > static_cast<int64_t>(dst->available()))
     return pa::fail(PA_ERR_OOM, "%s: need %lld blocks, %zu free", fn, (long long)distinct,
-                    dst->free_stack.size());
+                    dst->available());
   if (distinct > pairs_capacity || (distinct > 0 && !pairs_out))
     return pa::fail(PA_ERR_INVALID, "%s: pairs_out holds %d pairs, %lld needed", fn,
                     pairs_capacity, (long long)distinct);

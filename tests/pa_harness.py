@@ -16,7 +16,7 @@ import torch
 import oracle
 import workloads as W
 from oracle.allocator import BlockManager
-from paged_kv_cache_443_b200.cache import PagedKVCache
+from paged_kv_cache_443_b200.cache import PagedKVCache, _filled
 
 # tolerances: fp32 accumulation; max abs error on outputs (fp16 / bf16 / fp32)
 TOL = {"f32": 1e-5, "f16": 2e-2, "bf16": 2e-2}
@@ -25,12 +25,11 @@ TOL = {"f32": 1e-5, "f16": 2e-2, "bf16": 2e-2}
 def poison_bits(spec: W.Spec):
     """Bit pattern torch stores for NaN in the cache dtype (the fill of every
     slot no token was written to)."""
-    t = torch.tensor([float("nan")]).to(W.torch_kv_dtype(spec))
-    return W.storage_view(t)[0]
+    return W.storage_view(_filled((1,), float("nan"), W.torch_kv_dtype(spec), "cpu"))[0]
 
 
 def _zero_bits(spec: W.Spec):
-    return W.storage_view(torch.zeros(1).to(W.torch_kv_dtype(spec)))[0]
+    return W.storage_view(_filled((1,), 0.0, W.torch_kv_dtype(spec), "cpu"))[0]
 
 
 def oracle_append(spec: W.Spec, key, value, k, v, slots):

@@ -197,3 +197,93 @@ def test_move_errors_map_to_statuses():
         pk.pa_seq_move(a.h, c.h, [0], 2)
     assert snap == (a.free_stack(), b.free_stack()) and a.num_tokens(0) == 9
     assert a.move_to(b, []) == []
+
+
+def same_prefix_state(a: pk.BlockAllocator, o: BlockManager, live):
+    same_state(a, o, live)
+    assert a.evictable() == o.evictable
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_random_prefix_cache_scripts_match_oracle(seed):
+    """Requests drawn from a few prompts (so prefixes repeat), forks, appends,
+    commits, releases and pool pressure (evictions): cached token counts,
+    slots, copy pairs, tables, refcounts, free stack and evictable list equal
+    on both sides after every operation."""
+    rng = np.random.default_rng(3000 + seed)
+    for trial in range(8):
+        NB, bs = int(rng.integers(4, 40)), int(rng.choice([1, 2, 4, 16]))
+        order = rng.permutation(NB).tolist()
+        a, o = pk.BlockAllocator(NB, bs, order), BlockManager(NB, bs, order)
+        if rng.random() < 0.9:
+            a.enable_prefix_cache()
+            o.enable_prefix_cache()
+        prompts = [rng.integers(0, 3, size=int(rng.integers(1, 5 * bs + 2))).tolist()
+                   for _ in range(4)]
+        toks = {}
+        next_id = 0
+        for _ in range(150):
+            live = sorted(o.seqs)
+            r = rng.random()
+            if r < 0.3 or not live:
+                p = prompts[int(rng.integers(0, 4))] + \
+                    rng.integers(0, 3, size=int(rng.integers(0, 3))).tolist()
+                got_o = o.add_cached(next_id, p)
+                assert a.add_cached(next_id, p) == got_o
+                toks[next_id] = p[:got_o]
+                try:
+                    want = o.append(next_id, len(p) - got_o)
+                except OOM:
+                    with pytest.raises(pk.OutOfBlocks):
+                        a.append(next_id, len(p) - got_o)
+                else:
+                    got = a.append(next_id, len(p) - got_o)
+                    assert got[0] == want[0] and [tuple(x) for x in got[1]] == want[1]
+                    toks[next_id] = p
+                    a.commit(next_id, p)
+                    o.commit(next_id, p)
+                next_id += 1
+            elif r < 0.4:
+                q = int(rng.choice(live))
+                a.fork(q, next_id)
+                o.fork(q, next_id)
+                toks[next_id] = list(toks[q])
+                next_id += 1
+            elif r < 0.7:
+                sid = int(rng.choice(live))
+                n = int(rng.integers(1, 2 * bs + 1))
+                try:
+                    want = o.append(sid, n)
+                except OOM:
+                    with pytest.raises(pk.OutOfBlocks):
+                        a.append(sid, n)
+                else:
+                    got = a.append(sid, n)
+                    assert got[0] == want[0] and [tuple(x) for x in got[1]] == want[1]
+                    toks[sid] = toks[sid] + rng.integers(0, 3, size=n).tolist()
+                    k = int(rng.integers(0, len(toks[sid]) + 1))     # commit a prefix of it
+                    a.commit(sid, toks[sid][:k])
+                    o.commit(sid, toks[sid][:k])
+            else:
+                sid = int(rng.choice(live))
+                a.release(sid)
+                o.release(sid)
+            same_prefix_state(a, o, sorted(o.seqs))
+
+
+def test_prefix_cache_errors_map_to_statuses():
+    a = pk.BlockAllocator(8, 2)
+    a.enable_prefix_cache()
+    assert a.add_cached(0, [1, 2, 3]) == 0
+    with pytest.raises(pk.PagedKVError):
+        a.add_cached(0, [1])                      # exists
+    with pytest.raises(pk.PagedKVError):
+        a.commit(5, [1])                          # unknown
+    with pytest.raises(pk.PagedKVError):
+        a.commit(0, [1, 2, 3])                    # more tokens than it holds (0)
+    a.append(0, 3)
+    a.commit(0, [1, 2, 3])
+    assert a.add_cached(1, [1, 2, 3, 4]) == 2 and a.evictable() == []
+    a.release(0)
+    a.release(1)
+    assert len(a.evictable()) == 1 and a.num_free() == 8

@@ -373,3 +373,87 @@ def test_fp8_full_size_workloads_sampled(name):
     got_all = as_f64(out, spec)
     assert np.isfinite(got_all).all()
     assert np.abs(got_all[rows[:, 0], rows[:, 1]] - want).max() <= TOL[spec.dtype]
+
+
+
+# ---------------------------------------------------------------------------
+# prefix caching: requests sharing a system prompt reuse its blocks
+
+
+def _prefix_kv(tokens, Hkv, D, dtype):
+    """K/V of every position of a prompt, a function of the prefix up to and
+    including it (identical prefixes give identical K/V, as in a model)."""
+    ks, vs = [], []
+    h = 0
+    for t in tokens:
+        h = (h * 1_000_003 + int(t) + 1) % (1 << 61)
+        g = torch.Generator().manual_seed(h)
+        ks.append(torch.randn((Hkv, D), generator=g))
+        vs.append(torch.randn((Hkv, D), generator=g))
+    return torch.stack(ks).to(dtype), torch.stack(vs).to(dtype)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_prefix_cached_requests_match_oracle_and_uncached_run(fp8):
+    from oracle.allocator import BlockManager
+    from pa_harness import oracle_append
+    from paged_kv_cache_443_b200.cache import PagedKVCache
+    base = W.Spec("prefix", "bf16", 8, 2, 128, 16, "independent", 6, seed=3, partition_size=128)
+    spec = W.fp8(base) if fp8 else base
+    rng = np.random.default_rng(5)
+    system = rng.integers(0, 1000, 300).tolist()
+    prompts = [system + rng.integers(0, 1000, int(rng.integers(1, 200))).tolist() for _ in range(6)]
+    prompts.append(list(system))                       # the bare system prompt
+    prompts.append(system[:150] + [7] + system[151:])  # diverges inside block 9
+    NB = 200
+    outs = []
+    for cached in (True, False):
+        cache = PagedKVCache(NB, 16, spec.Hkv, spec.D, W.torch_kv_dtype(spec), "cuda",
+                             fill=float("nan"), k_scale=spec.k_scale, v_scale=spec.v_scale,
+                             prefix_cache=cached)
+        bm = BlockManager(NB, 16)
+        if cached:
+            bm.enable_prefix_cache()
+        ok = np.full((NB, spec.Hkv, 16, spec.D), poison_bits(spec))
+        ov = ok.copy()
+        computed = []
+        for r, toks in enumerate(prompts):
+            n_c = cache.add_cached(r, toks)
+            assert bm.add_cached(r, toks) == n_c
+            k, v = _prefix_kv(toks, spec.Hkv, spec.D, W.torch_dtype(spec))
+            slots, pairs = cache.append([r], [len(toks) - n_c], k[n_c:].cuda(), v[n_c:].cuda())
+            want_slots, want_pairs = bm.append(r, len(toks) - n_c)
+            assert slots == want_slots and pairs == want_pairs == []
+            oracle_append(spec, k[n_c:], v[n_c:], ok, ov, want_slots)
+            cache.commit(r, toks)
+            bm.commit(r, toks)
+            computed.append(len(toks) - n_c)
+        B = len(prompts)
+        tables, lens, max_ctx = cache.tables(list(range(B)))
+        ot, ol = bm.build_tables(list(range(B)), tables.shape[1])
+        assert np.array_equal(tables.cpu().numpy(), ot) and np.array_equal(lens.cpu().numpy(), ol)
+        q = W.q_content(spec, B, "cuda")
+        out = cache.decode(q, tables, lens, max_ctx, spec.softmax_scale, partition_size=128)
+        torch.cuda.synchronize()
+        assert pk.pa_device_status() == 0
+        for dev, host in ((cache.k_cache, ok), (cache.v_cache, ov)):
+            assert W.storage_view(dev).tobytes() == host.tobytes()
+        o = Oracle_view(bm, ok, ov, ot, ol, W.storage_view(q))
+        err = np.abs(as_f64(out, spec) - oracle_attention(o, spec)).max()
+        assert err <= TOL[spec.dtype]
+        if cached:
+            # 18 full system blocks are reused by requests 1..5 and 6; the diverging
+            # request shares the first 9
+            assert computed[0] == len(prompts[0])
+            assert all(c == len(p) - 288 for c, p in zip(computed[1:6], prompts[1:6]))
+            assert computed[6] == 300 - 288 and computed[7] == 300 - 144
+            t = tables.cpu().numpy()
+            assert all((t[r, :18] == t[0, :18]).all() for r in range(1, 7))
+            assert (t[7, :9] == t[0, :9]).all() and t[7, 9] != t[0, 9]
+        outs.append(out)
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+
+
+class Oracle_view:
+    def __init__(self, bm, k, v, tables, lens, q):
+        self.bm, self.k, self.v, self.tables, self.lens, self.q = bm, k, v, tables, lens, q

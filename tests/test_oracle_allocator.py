@@ -145,7 +145,13 @@ def _check_invariants(bm):
             refs[b] += 1
     assert refs.tolist() == bm.refcount
     used = {b for b in range(NB) if refs[b] > 0}
-    assert used.isdisjoint(free) and len(used) + len(free) == NB
+    ev = list(bm.evictable)
+    assert len(set(ev)) == len(ev) and set(ev).isdisjoint(free) and used.isdisjoint(ev)
+    assert used.isdisjoint(free) and len(used) + len(free) + len(ev) == NB
+    # every evictable block is cached; cached blocks and keys pair up one to one
+    assert all(b in bm.key_of_block for b in ev)
+    assert all(bm.block_of_key[k] == b for b, k in bm.key_of_block.items())
+    assert len(bm.block_of_key) == len(bm.key_of_block)
 
 
 def test_random_operation_sequences_keep_invariants():
@@ -300,3 +306,167 @@ def test_move_errors_change_nothing():
         dev.move_to(host, [0])
     assert snap == (dev.free_stack(), list(dev.refcount), host.free_stack())
     assert dev.num_tokens(0) == 9
+
+
+
+# ---------------------------------------------------------------------------
+# prefix caching: reuse of a repeated prompt prefix's blocks
+
+
+def _prompt(*parts):
+    return [t for p in parts for t in p]
+
+
+SYS = list(range(100, 110))        # a 10-token system prompt
+
+
+def test_repeated_prompt_prefix_reuses_full_blocks():
+    bm = BlockManager(32, 4)
+    bm.enable_prefix_cache()
+    a = _prompt(SYS, [1, 2, 3, 4, 5])
+    assert bm.add_cached(0, a) == 0
+    bm.append(0, len(a))
+    bm.commit(0, a)
+    b = _prompt(SYS, [7, 8, 9, 9, 9, 9, 9])
+    assert bm.add_cached(1, b) == 8            # blocks 0, 1 hit; block 2 mixes in user tokens
+    assert bm.blocks_of(1) == bm.blocks_of(0)[:2]
+    assert [bm.refcount[x] for x in bm.blocks_of(0)] == [2, 2, 1, 1]
+    slots, pairs = bm.append(1, len(b) - 8)
+    assert pairs == [] and bm.num_tokens(1) == len(b)
+    assert bm.blocks_of(1)[2] not in bm.blocks_of(0)
+    _check_invariants(bm)
+
+
+def test_lookup_follows_the_content_chain_and_leaves_one_token():
+    bm = BlockManager(32, 4)
+    bm.enable_prefix_cache()
+    a = list(range(12))                         # exactly three full blocks
+    bm.add_cached(0, a)
+    bm.append(0, 12)
+    bm.commit(0, a)
+    # same second block after a different first block: no hit (keys chain)
+    assert bm.add_cached(1, [99, 1, 2, 3] + a[4:]) == 0
+    # the very same prompt: two blocks, the last one is computed again
+    assert bm.add_cached(2, a) == 8
+    # a longer prompt with the same 12 tokens: all three
+    assert bm.add_cached(3, a + [50]) == 12
+    assert bm.add_cached(4, []) == 0 and bm.add_cached(5, a[:4]) == 0
+    _check_invariants(bm)
+
+
+def test_released_cached_blocks_wait_evictable_and_come_back():
+    bm = BlockManager(8, 4, list(range(7, -1, -1)))   # block 0 handed out first
+    bm.enable_prefix_cache()
+    a = _prompt(SYS, [1, 2])                    # 12 tokens: 3 full blocks
+    bm.add_cached(0, a)
+    bm.append(0, 12)
+    bm.commit(0, a)
+    bm.append(0, 1)                             # a 4th, partial block (uncommitted)
+    blocks = bm.blocks_of(0)
+    bm.release(0)
+    assert bm.evictable == blocks[:3]           # logical order, oldest first
+    assert bm.free_stack()[-1] == blocks[3]
+    assert bm.num_free() == 8
+    assert bm.add_cached(1, a + [5]) == 12      # taken back from the evictable list
+    assert bm.blocks_of(1) == blocks[:3] and bm.evictable == []
+    _check_invariants(bm)
+
+
+def test_eviction_takes_free_blocks_first_then_least_recently_released():
+    bm = BlockManager(6, 2)
+    bm.enable_prefix_cache()
+    p1, p2 = [1, 1, 2, 2, 3], [4, 4, 5, 5, 6]
+    for sid, p in ((0, p1), (1, p2)):
+        bm.add_cached(sid, p)
+        bm.append(sid, len(p))
+        bm.commit(sid, p)
+    bm.release(0)
+    bm.release(1)
+    b1, b2 = bm.evictable[:2], bm.evictable[2:]
+    assert len(b1) == 2 and len(b2) == 2 and len(bm.free) == 2
+    bm.add(7)
+    bm.append(7, 4)                             # the two free blocks, no eviction
+    assert bm.evictable == b1 + b2
+    bm.append(7, 2)                             # evicts p1's first block
+    assert bm.evictable == b1[1:] + b2 and bm.blocks_of(7)[-1] == b1[0]
+    assert bm.add_cached(8, p1 + [9]) == 0       # p1's chain starts with a miss now
+    assert bm.add_cached(9, p2 + [9]) == 4
+    _check_invariants(bm)
+
+
+def test_first_committed_block_wins_a_key():
+    bm = BlockManager(16, 2)
+    bm.enable_prefix_cache()
+    p = [3, 3, 4, 4, 5]
+    for sid in (0, 1):                          # both miss: computed twice
+        assert bm.add_cached(sid, p) == 0
+        bm.append(sid, len(p))
+    bm.commit(0, p)
+    bm.commit(1, p)
+    assert bm.add_cached(2, p) == 4 and bm.blocks_of(2) == bm.blocks_of(0)[:2]
+    bm.release(1)                               # 1's full blocks were never cached
+    assert bm.evictable == [] and len(bm.free) == 16 - 3 - 3 + 3
+    _check_invariants(bm)
+
+
+def test_prefix_cache_off_is_plain_allocation():
+    bm = BlockManager(8, 2)
+    assert bm.add_cached(0, [1, 2, 3]) == 0
+    bm.append(0, 3)
+    bm.commit(0, [1, 2, 3])
+    assert bm.add_cached(1, [1, 2, 3]) == 0 and not bm.block_of_key
+    with pytest.raises(Invalid):
+        bm.commit(0, [1, 2, 3, 4])
+    with pytest.raises(Invalid):
+        bm.add_cached(0, [1])
+
+
+def test_random_prefix_cache_sequences_keep_invariants():
+    rng = np.random.default_rng(17)
+    for trial in range(20):
+        NB, bs = int(rng.integers(4, 30)), int(rng.choice([1, 2, 4]))
+        bm = BlockManager(NB, bs, rng.permutation(NB).tolist())
+        bm.enable_prefix_cache()
+        prompts = [rng.integers(0, 3, size=int(rng.integers(1, 4 * bs + 2))).tolist() for _ in range(4)]
+        toks = {}
+        next_id = 0
+        for _ in range(150):
+            live = sorted(bm.seqs)
+            r = rng.random()
+            try:
+                if r < 0.3 or not live:
+                    p = prompts[int(rng.integers(0, 4))] + rng.integers(0, 3, size=int(rng.integers(0, 3))).tolist()
+                    got = bm.add_cached(next_id, p)
+                    assert got % bs == 0 and got < max(1, len(p))
+                    toks[next_id] = p[:got]
+                    try:
+                        bm.append(next_id, len(p) - got)
+                        toks[next_id] = p
+                        bm.commit(next_id, p)
+                    except OOM:
+                        pass
+                    next_id += 1
+                elif r < 0.4:
+                    q = int(rng.choice(live))
+                    bm.fork(q, next_id)
+                    toks[next_id] = list(toks[q])
+                    next_id += 1
+                elif r < 0.7:
+                    sid = int(rng.choice(live))
+                    n = int(rng.integers(1, 2 * bs + 1))
+                    bm.append(sid, n)
+                    toks[sid] = toks[sid] + rng.integers(0, 3, size=n).tolist()
+                    bm.commit(sid, toks[sid])
+                else:
+                    bm.release(int(rng.choice(live)))
+            except OOM:
+                pass
+            _check_invariants(bm)
+            # a cached block's key is the content chain of the tokens it holds for
+            # every live sequence that uses it in that logical position
+            for sid, s in bm.seqs.items():
+                key = None
+                for k, blk in enumerate(s.blocks[: len(toks[sid]) // bs]):
+                    key = (key, tuple(toks[sid][k * bs:(k + 1) * bs]))
+                    if blk in bm.key_of_block:
+                        assert bm.key_of_block[blk] == key

@@ -250,17 +250,19 @@ def rank_spec(spec, rank):
 KERNEL_SOURCES = {
     "decode_partition_kernel": ("decode.cu", "pa_device.cuh", "pa_internal.h"),
     "decode_partition_tc_kernel": ("decode_tc.cu", "tc_common.cuh", "pa_device.cuh", "pa_internal.h"),
+    "decode_partition_tc8_kernel": ("decode_tc8.cu", "tc_common.cuh", "pa_device.cuh",
+                                    "pa_internal.h"),
 }
 
 
 def partition_kernel(spec, P):
-    """The decode-partition kernel the library picks for this launch: the
-    tensor-core one for 4 or 8 query heads per kv head in fp16/bf16, head size
-    128 and a partition length that is a multiple of 128; else CUDA cores."""
+    """The decode-partition kernel the library picks for this launch: a
+    tensor-core one (16-bit or E4M3 cache) for 4 or 8 query heads per kv head
+    with fp16/bf16 queries, head size 128 and a partition length that is a
+    multiple of 128; else CUDA cores."""
     G = spec.Hq // spec.Hkv
-    if (not spec.fp8 and spec.dtype in ("f16", "bf16") and spec.D == 128 and G in (4, 8)
-            and P % 128 == 0):
-        return "decode_partition_tc_kernel"
+    if spec.dtype in ("f16", "bf16") and spec.D == 128 and G in (4, 8) and P % 128 == 0:
+        return "decode_partition_tc8_kernel" if spec.fp8 else "decode_partition_tc_kernel"
     return "decode_partition_kernel"
 
 
@@ -742,8 +744,9 @@ def main():
                              "long_prefix_bs8", "long_prefix_bs16", "long_prefix_bs32",
                              "gqa70b_quarter", "long_prefix_bs8_quarter",
                              "long_prefix_bs16_quarter", "opt13b_fp8", "opt13b_compact_fp8",
-                             "gqa70b_fp8", "long_prefix_bs16_fp8", "llama13b_ps_fp8",
-                             "tiny_fp8"])
+                             "gqa70b_fp8", "gqa70b_quarter_fp8", "long_prefix_bs8_fp8",
+                             "long_prefix_bs16_fp8", "long_prefix_bs32_fp8",
+                             "long_prefix_bs16_quarter_fp8", "llama13b_ps_fp8", "tiny_fp8"])
     ap.add_argument("--partition-size", type=int, default=0,
                     help="split-K partition length (0: the workload's own, 512)")
     ap.add_argument("--soak-seconds", type=float, default=0.5,

@@ -37,8 +37,9 @@ int num_sms() {
   return n;
 }
 
-// Partition length pa_decode uses for partition_size = 0.  The tensor-core
-// kernel (fp16/bf16, head size 128, 4 or 8 query heads per kv head) pays a
+// Partition length pa_decode (and pa_decode_fp8) use for partition_size = 0.
+// The tensor-core kernels (fp16/bf16 queries, head size 128, 4 or 8 query heads
+// per kv head; 16-bit or E4M3 caches) pay a
 // fixed set-up and drain per CTA, so it takes the longest of 2048 / 1024 tokens
 // that still gives at least ~4 waves of CTAs (2 per SM) at the longest context;
 // everything else keeps the default.
@@ -180,6 +181,7 @@ pa_status check_decode_fp8(const char* fn, void* out, const void* q, const void*
 }
 
 int launch_partitions(const pa::DecodeArgs& a, unsigned int* status, void* stream) {
+  if (pa::decode_tc8_supported(a)) return pa::launch_decode_partitions_tc8(a, status, stream);
   if (a.kv_dtype == a.dtype && pa::decode_tc_supported(a)) return pa::launch_decode_partitions_tc(a, status, stream);
   return pa::launch_decode_partitions(a, status, stream);
 }
@@ -423,6 +425,9 @@ extern "C" pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache
                                    int max_context_len, void* workspace,
                                    size_t workspace_bytes_in, void* stream) {
   const char* fn = "pa_decode_fp8";
+  if (partition_size == 0 && num_heads > 0 && num_kv_heads > 0)   // as pa_decode
+    partition_size =
+        auto_partition(num_seqs, num_heads, num_kv_heads, head_size, dtype, max_context_len);
   pa::DecodeArgs a;
   pa_status st = check_decode_fp8(fn, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
                                   context_lens, num_seqs, num_heads, num_kv_heads, head_size,

@@ -502,13 +502,16 @@ bool make_tmap(void* map, const void* base, int rank, const int64_t* dims,
     estr[i] = 1u;
     if (i + 1 < rank) gstride[i] = static_cast<cuuint64_t>(strides_bytes[i]);
   }
-  const CUtensorMapDataType t =
-      dt == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUtensorMapDataType t = dt == PA_BF16       ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                : dt == PA_FP8_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   return fn(static_cast<CUtensorMap*>(map), t, static_cast<cuuint32_t>(rank),
             const_cast<void*>(base), gdim, gstride, bdim, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+bool tmap_available() { return encode_fn() != nullptr; }
 
 bool decode_tc_supported(const DecodeArgs& a) {
   const int G = a.Hq / a.Hkv;

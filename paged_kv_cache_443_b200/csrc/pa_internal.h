@@ -67,11 +67,18 @@ int launch_decode_reduce(const DecodeArgs& a, unsigned int* status, void* stream
 // query heads per kv head, partition length a multiple of 128.
 bool decode_tc_supported(const DecodeArgs& a);
 int launch_decode_partitions_tc(const DecodeArgs& a, unsigned int* status, void* stream);
-// A TMA tensor map of 16-bit elements with the 128-byte swizzle: `rank` dims
+// Tensor-core partition kernel over an E4M3 cache (decode_tc8.cu): f16/bf16
+// queries, head size 128, 4 or 8 query heads per kv head, partition length a
+// multiple of 128.
+bool decode_tc8_supported(const DecodeArgs& a);  // needs tmap_available()
+int launch_decode_partitions_tc8(const DecodeArgs& a, unsigned int* status, void* stream);
+// A TMA tensor map of 16-bit elements (bytes for PA_FP8_E4M3) with the 128-byte swizzle: `rank` dims
 // (innermost first), byte strides of dims 1..rank-1, a box; `map` points at a
 // CUtensorMap.  False if encoding fails.
 bool make_tmap(void* map, const void* base, int rank, const int64_t* dims,
                const int64_t* strides_bytes, const int* box, pa_dtype dt);
+// Whether the driver entry point that encodes tensor maps could be found.
+bool tmap_available();
 
 int launch_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
                              const int64_t* slot_mapping, int num_tokens, int Hkv, int D,

@@ -91,7 +91,8 @@ def test_partition_kernel_choice():
     assert bench.partition_kernel(W.OPT13B, 512) == "decode_partition_kernel"
     assert bench.partition_kernel(W.GQA70B, 96) == "decode_partition_kernel"
     assert bench.partition_kernel(W.TINY, 512) == "decode_partition_kernel"
-    assert bench.partition_kernel(W.fp8(W.GQA70B), 2048) == "decode_partition_kernel"
+    assert bench.partition_kernel(W.fp8(W.GQA70B), 2048) == "decode_partition_tc8_kernel"
+    assert bench.partition_kernel(W.fp8(W.OPT13B), 512) == "decode_partition_kernel"
 
 
 def test_fp8_workloads_count_one_byte_per_element():

@@ -457,3 +457,45 @@ def test_prefix_cached_requests_match_oracle_and_uncached_run(fp8):
 class Oracle_view:
     def __init__(self, bm, k, v, tables, lens, q):
         self.bm, self.k, self.v, self.tables, self.lens, self.q = bm, k, v, tables, lens, q
+
+
+# ---------------------------------------------------------------------------
+# E4M3 cache on the tensor-core kernel (G = 4 / 8, D = 128, f16 / bf16 queries)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("G", [4, 8])
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_fp8_tc_edges(dtype, G, bs):
+    lens = (0, 1, 63, 64, 65, 127, 128, 129, 255, 256, 257, 700)
+    spec = W.fp8(W.Spec(f"tc8_{dtype}_{G}_{bs}", dtype, 2 * G, 2, 128, bs, "independent",
+                        len(lens), seed=300 + G + bs, ctx_dist="explicit", ctx_list=lens,
+                        partition_size=256))
+    got, _ = full_check(spec)
+    assert np.all(got[0] == 0.0)
+    full_check(spec, partition_size=128)
+    full_check(spec, partition_size=4096)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("mag", [1e-6, 1e-2, 30.0, 2e3])
+def test_fp8_tc_query_magnitudes(dtype, mag):
+    """bf16 queries are staged as f16 times a per-head power of two; f16 ones as
+    they are: tiny and large queries (near-uniform and near-one-hot softmax)."""
+    if dtype == "f16" and mag > 1e3:
+        mag = 1e3                                  # f16 q must stay finite
+    spec = W.fp8(W.Spec(f"tc8q_{dtype}", dtype, 16, 2, 128, 16, "independent", 6, seed=77,
+                        ctx_dist="explicit", ctx_list=(5, 130, 300, 513, 999, 1500),
+                        partition_size=512))
+    sc = W.scenario(spec)
+    p, o = build(sc)
+    scale = torch.tensor([mag] + [1.0] * 15, device="cuda").view(1, 16, 1)
+    p.q.mul_(scale.to(p.q.dtype))
+    o.q = W.storage_view(p.q)
+    out = run_step(p, spec)
+    torch.cuda.synchronize()
+    assert pk.pa_device_status() == 0
+    got = as_f64(out, spec)
+    want = oracle_attention(o, spec)
+    assert np.isfinite(got).all()
+    assert np.abs(got - want).max() <= TOL[spec.dtype]

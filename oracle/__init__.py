@@ -48,6 +48,9 @@ def lib():
         L.or_paged_attention_kv.argtypes = [p, p, i64, p, p, p, i32, i32, dbl, dbl, p, i32, p,
                                             i32, i32, i32, i32, i32, i32, dbl, i32]
         L.or_paged_attention_kv.restype = i32
+        L.or_paged_attention_mq.argtypes = [p, p, p, p, i32, p, i32, p, p, i32, i32, i32, i32,
+                                            i32, i32, dbl, i32]
+        L.or_paged_attention_mq.restype = i32
         L.or_e4m3_to_f64.argtypes = [ctypes.c_uint8]
         L.or_e4m3_to_f64.restype = dbl
         L.or_encode_e4m3.argtypes = [p, p, i64]
@@ -130,6 +133,34 @@ def paged_attention(q, k_cache, v_cache, dtype, block_tables, context_lens, scal
                                      _ptr(v_cache), dtype, kvd, float(k_scale), float(v_scale),
                                      _ptr(block_tables), block_tables.shape[1],
                                      _ptr(context_lens), B, Hq, Hkv, D, bs, NB, float(scale), nt)
+    if rc != 0:
+        raise ValueError("oracle: input out of range")
+    return out
+
+
+def paged_attention_mq(q, k_cache, v_cache, dtype, block_tables, context_lens, query_start,
+                       scale, nthreads=None):
+    """Several new query tokens per sequence, causal among themselves.
+
+    q: [total_q, Hq, D] storage array; query_start: [B+1] int32 offsets into q
+    (sequence b's tokens are rows query_start[b] .. query_start[b+1]-1 and are
+    its last context positions).  Returns [total_q, Hq, D] float64.  Reading
+    of chunked prefill / speculative verification in "4. 이 밖의 기법들"
+    (blog.aqudi.me): query token i of sequence b attends to positions
+    0 .. context_lens[b] - Q_b + i.
+    """
+    q, k_cache, v_cache = _c(q), _c(k_cache), _c(v_cache)
+    block_tables, context_lens = _c(block_tables, np.int32), _c(context_lens, np.int32)
+    query_start = _c(query_start, np.int32)
+    T, Hq, D = q.shape
+    NB, Hkv, bs, _ = k_cache.shape
+    B = context_lens.shape[0]
+    assert query_start.shape[0] == B + 1 and int(query_start[-1]) == T
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    nt = max_threads() if nthreads is None else int(nthreads)
+    rc = lib().or_paged_attention_mq(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), dtype,
+                                     _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+                                     _ptr(query_start), B, Hq, Hkv, D, bs, NB, float(scale), nt)
     if rc != 0:
         raise ValueError("oracle: input out of range")
     return out

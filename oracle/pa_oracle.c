@@ -281,6 +281,54 @@ int or_paged_attention(double* out, const int64_t* rows, int64_t nrows, const vo
                                num_blocks, scale, nthreads);
 }
 
+/* ---- several new query tokens per sequence ----
+ * Chunked prefill and speculative verification ("4. 이 밖의 기법들",
+ * blog.aqudi.me: a long prefill cut into chunks between decode steps; several
+ * proposed tokens checked by the large model at once).  The pages give no
+ * formula beyond the attention of "자기회귀 생성과 KV 캐시" (supersilo.blog), so
+ * the reading is: sequence b's last Q_b = query_start[b+1] - query_start[b]
+ * context tokens are its new query tokens, and query token i (0 <= i < Q_b)
+ * sits at position L_b - Q_b + i and attends to positions 0 .. L_b - Q_b + i
+ * (its own included, none after it).
+ *
+ * q / out: [total_q][Hq][D] with total_q = query_start[B]; the cache, tables
+ * and context lengths as above.  Each (query token, head) is the single-query
+ * attention of or_paged_attention over its own number of positions.  Returns
+ * -1 on an input out of range (query_start not non-decreasing from 0, Q_b >
+ * L_b, and the cases of or_paged_attention).
+ */
+int or_paged_attention_mq(double* out, const void* q, const void* k_cache, const void* v_cache,
+                          int dtype, const int32_t* block_tables, int max_blocks,
+                          const int32_t* context_lens, const int32_t* query_start, int B, int Hq,
+                          int Hkv, int D, int block_size, int num_blocks, double scale,
+                          int nthreads) {
+  if (B < 0 || Hq <= 0 || query_start[0] != 0) return -1;
+  for (int b = 0; b < B; ++b)
+    if (query_start[b + 1] < query_start[b] ||
+        query_start[b + 1] - query_start[b] > context_lens[b])
+      return -1;
+  const int64_t total = query_start[B];
+  const size_t es = (size_t)or_elem_size(dtype);
+  if (es == 0) return -1;
+  /* one row at a time through the single-query definition: a one-sequence
+   * batch whose context ends at the query token's own position */
+  int bad = 0;
+  for (int b = 0; b < B && !bad; ++b) {
+    const int Qb = query_start[b + 1] - query_start[b];
+    for (int i = 0; i < Qb && !bad; ++i) {
+      const int64_t t = query_start[b] + i;
+      const int32_t len = context_lens[b] - Qb + i + 1;
+      if (or_paged_attention(out + t * Hq * D, NULL, 0, (const char*)q + (size_t)t * Hq * D * es,
+                             k_cache, v_cache, dtype, block_tables + (int64_t)b * max_blocks,
+                             max_blocks, &len, 1, Hq, Hkv, D, block_size, num_blocks, scale,
+                             nthreads) != 0)
+        bad = 1;
+    }
+  }
+  (void)total;
+  return bad ? -1 : 0;
+}
+
 /* ---- appending the new tokens' K and V ----
  * Follows "1. KV 캐시란" (hjr-study-book Day 3: each step stores the new K, V
  * pair) and the slot arithmetic of the block-table example in "4.2

@@ -628,3 +628,76 @@ def test_e4m3_attention_identities():
                                  kv_dtype=oracle.E4M3, k_scale=0.3, v_scale=0.7)[0]
     v0 = oracle.decode(codes_v[tables[0, 0], :, 0], oracle.E4M3) * 0.7
     assert np.array_equal(one[:2], v0[0:1].repeat(2, 0)) and np.array_equal(one[2:], v0[1:2].repeat(2, 0))
+
+
+# ---------------------------------------------------------------------------
+# several new query tokens per sequence (chunked prefill, speculative verify)
+
+
+def _mq_case(seed, dtype=oracle.F32, bs=16, G=2, D=64):
+    rng = np.random.default_rng(seed)
+    B, Hkv = 3, 2
+    Hq = Hkv * G
+    lens = np.array([7, 40, 130], dtype=np.int32)
+    qlen = np.array([1, 5, 17], dtype=np.int32)
+    qs = np.concatenate([[0], np.cumsum(qlen)]).astype(np.int32)
+    NB = 20
+    order = rng.permutation(NB)
+    maxb = -(-int(lens.max()) // bs)
+    tables = np.full((B, maxb), -1, dtype=np.int32)
+    k = 0
+    for b in range(B):
+        nb = -(-int(lens[b]) // bs)
+        tables[b, :nb] = order[k:k + nb]
+        k += nb
+    kc = rng.standard_normal((NB, Hkv, bs, D)).astype(np.float32)
+    vc = rng.standard_normal((NB, Hkv, bs, D)).astype(np.float32)
+    q = rng.standard_normal((int(qs[-1]), Hq, D)).astype(np.float32)
+    return q, kc, vc, tables, lens, qs, Hq, Hkv, D, bs
+
+
+def test_multi_query_matches_causal_sdpa_on_contiguous_tokens():
+    q, kc, vc, tables, lens, qs, Hq, Hkv, D, bs = _mq_case(21)
+    scale = 1 / np.sqrt(D)
+    got = oracle.paged_attention_mq(q, kc, vc, oracle.F32, tables, lens, qs, scale)
+    for b in range(len(lens)):
+        L, Qb = int(lens[b]), int(qs[b + 1] - qs[b])
+        j = np.arange(L)
+        K = kc[tables[b, j // bs], :, j % bs].transpose(1, 0, 2)      # [Hkv, L, D]
+        V = vc[tables[b, j // bs], :, j % bs].transpose(1, 0, 2)
+        Q = q[qs[b]:qs[b + 1]].transpose(1, 0, 2)                      # [Hq, Qb, D]
+        mask = j[None, :] <= (L - Qb + np.arange(Qb))[:, None]         # bottom-right causal
+        ref = F.scaled_dot_product_attention(
+            torch.from_numpy(Q).double()[None], torch.from_numpy(K).double()[None],
+            torch.from_numpy(V).double()[None], attn_mask=torch.from_numpy(mask)[None, None],
+            scale=scale, enable_gqa=True)[0].numpy().transpose(1, 0, 2)
+        assert np.abs(got[qs[b]:qs[b + 1]] - ref).max() <= 1e-12
+
+
+def test_multi_query_row_equals_decode_at_its_own_position():
+    """A prompt processed as one chunk of queries: query i sees exactly what a
+    single-query decode with context length L - Q + i + 1 sees."""
+    q, kc, vc, tables, lens, qs, Hq, Hkv, D, bs = _mq_case(22, G=4)
+    got = oracle.paged_attention_mq(q, kc, vc, oracle.F32, tables, lens, qs, 0.2)
+    b = 2
+    Qb = int(qs[b + 1] - qs[b])
+    for i in (0, 7, Qb - 1):
+        one = oracle.paged_attention(q[qs[b] + i][None], kc, vc, oracle.F32, tables[b:b + 1],
+                                     np.array([lens[b] - Qb + i + 1], dtype=np.int32), 0.2)
+        assert np.abs(got[qs[b] + i] - one[0]).max() == 0.0
+    # one query per sequence is the plain decode
+    q1 = q[qs[1:] - 1]
+    dec = oracle.paged_attention(q1, kc, vc, oracle.F32, tables, lens, 0.2)
+    one_each = oracle.paged_attention_mq(q1, kc, vc, oracle.F32, tables, lens,
+                                         np.arange(len(lens) + 1, dtype=np.int32), 0.2)
+    assert np.array_equal(dec, one_each)
+
+
+def test_multi_query_rejects_bad_offsets():
+    q, kc, vc, tables, lens, qs, Hq, Hkv, D, bs = _mq_case(23)
+    with pytest.raises(ValueError):                 # more queries than context
+        oracle.paged_attention_mq(q[:8], kc, vc, oracle.F32, tables, np.array([7, 0, 130], np.int32),
+                                  np.array([0, 1, 3, 8], np.int32), 0.1)
+    with pytest.raises(ValueError):                 # decreasing offsets
+        oracle.paged_attention_mq(q[:8], kc, vc, oracle.F32, tables, lens,
+                                  np.array([0, 5, 3, 8], np.int32), 0.1)

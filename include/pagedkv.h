@@ -282,6 +282,40 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_pair
                          pa_dtype dtype, void* stream);
 
 /*
+ * Several new query tokens per sequence: chunked prefill and speculative
+ * verification ([P2] "4. 이 밖의 기법들": a long prefill is cut into chunks run
+ * between decode steps; several proposed tokens are checked at once).  The
+ * attention is that of pa_decode ([P1] "자기회귀 생성과 KV 캐시"), with this
+ * library's reading of the position of each query: sequence b's query tokens
+ * are rows query_start_loc[b] .. query_start_loc[b+1]-1 of q, they are the
+ * LAST Q_b = query_start_loc[b+1] - query_start_loc[b] of its context_lens[b]
+ * tokens (their K/V already appended), and query token i attends to positions
+ * 0 .. context_lens[b] - Q_b + i (causal among the new tokens):
+ *
+ *   out[t][h] = sum_{j <= pos(t)} softmax_j(scale * q[t][h] . K_b[j]) V_b[j].
+ *
+ *   q, out          [total_q][Hq][D], dtype f16 or bf16
+ *   query_start_loc [num_seqs + 1] int32 (device): 0, then non-decreasing,
+ *                   ending at total_q; max_query_len >= every Q_b
+ *   k_cache, v_cache, block_tables, context_lens, max_context_len: as pa_decode
+ * Supported: f16/bf16, head_size 128, Hq/Hkv in {1, 2, 4, 8}, bs in {8, 16,
+ * 32}, partition_size 0 (= 512) or a multiple of 128.  The workspace holds the
+ * split-K partials when max_context_len exceeds the partition length
+ * (pa_decode_multi_workspace_bytes).  Offsets that are not non-decreasing, or
+ * Q_b > context_lens[b], set PA_DEVERR_CONTEXT and the sequence is skipped.
+ * One or two launches on `stream`.
+ */
+size_t pa_decode_multi_workspace_bytes(int total_q, int num_heads, int head_size,
+                                       int max_context_len, int partition_size);
+pa_status pa_decode_multi(void* out, const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* block_tables, int max_blocks_per_seq,
+                          const int32_t* context_lens, const int32_t* query_start_loc,
+                          int num_seqs, int total_q, int max_query_len, int num_heads,
+                          int num_kv_heads, int head_size, int block_size, int num_blocks,
+                          float scale, pa_dtype dtype, int partition_size, int max_context_len,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * E4M3 KV cache ([P2] "4. 이 밖의 기법들", quantization; format and scales as
  * described at pa_dtype).
  *

@@ -32,7 +32,7 @@ EXPORTS = (
     "pa_decode_num_partitions", "pa_decode_workspace_bytes",
     "pa_decode", "pa_decode_partitions", "pa_decode_reduce", "pa_decode_noalloc",
     "pa_reshape_and_cache", "pa_reshape_and_cache_fp8", "pa_decode_fp8",
-    "pa_decode_partitions_fp8",
+    "pa_decode_partitions_fp8", "pa_decode_multi", "pa_decode_multi_workspace_bytes",
     "pa_copy_blocks", "pa_swap_blocks", "pa_alloc_create", "pa_alloc_destroy", "pa_alloc_num_free",
     "pa_alloc_refcount", "pa_alloc_free_stack", "pa_seq_add", "pa_seq_fork", "pa_seq_append",
     "pa_seq_free", "pa_seq_move", "pa_seq_num_tokens", "pa_build_tables",
@@ -88,6 +88,9 @@ def lib():
         "pa_reshape_and_cache": ([vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp], i32),
         "pa_reshape_and_cache_fp8": ([vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, f32,
                                       vp], i32),
+        "pa_decode_multi": ([vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                             i32, f32, i32, i32, i32, vp, sz, vp], i32),
+        "pa_decode_multi_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
         "pa_decode_fp8": ([vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, f32, i32,
                            f32, f32, i32, i32, vp, sz, vp], i32),
         "pa_decode_partitions_fp8": ([vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32,
@@ -290,6 +293,42 @@ def pa_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale
     _check(lib().pa_reshape_and_cache_fp8(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
                                           _ptr(slot_mapping), N, Hkv, D, bs, NB, _dtype_code(key),
                                           float(k_scale), float(v_scale), _stream(stream)))
+
+
+def pa_decode_multi_workspace_bytes(total_q: int, num_heads: int, head_size: int,
+                                    max_context_len: int, partition_size: int = 0) -> int:
+    return int(lib().pa_decode_multi_workspace_bytes(total_q, num_heads, head_size,
+                                                     max_context_len, partition_size))
+
+
+def pa_decode_multi(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc, scale,
+                    max_context_len, max_query_len, partition_size=0, workspace=None,
+                    stream=None) -> None:
+    """Several new query tokens per sequence (chunked prefill / speculative
+    verify): q, out [total_q, Hq, D]; query_start_loc int32 [B+1]; sequence b's
+    queries are its last Q_b context tokens, each attending causally."""
+    _contig(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc, workspace)
+    import torch
+    T, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_cache.shape
+    if D2 != D or tuple(out.shape) != (T, Hq, D) or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise PagedKVError(PA_ERR_INVALID, "shape mismatch among q, out and the caches")
+    for t_ in (out, k_cache, v_cache):
+        if t_.dtype != q.dtype:
+            raise PagedKVError(PA_ERR_INVALID, "q, out and the caches must share a dtype")
+    if (block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32
+            or query_start_loc.dtype != torch.int32):
+        raise PagedKVError(PA_ERR_INVALID, "block_tables, context_lens, query_start_loc: int32")
+    B = context_lens.shape[0]
+    if query_start_loc.numel() != B + 1:
+        raise PagedKVError(PA_ERR_INVALID, "query_start_loc must have num_seqs + 1 entries")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().pa_decode_multi(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                 _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+                                 _ptr(query_start_loc), B, T, int(max_query_len), Hq, Hkv, D, bs,
+                                 NB, float(scale), _dtype_code(q), int(partition_size),
+                                 int(max_context_len), _ptr(workspace), ws_bytes,
+                                 _stream(stream)))
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scale,

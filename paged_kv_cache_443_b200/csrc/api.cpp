@@ -475,3 +475,90 @@ extern "C" pa_status pa_reshape_and_cache_fp8(const void* key, const void* value
                                                         v_scale, status, stream),
                        1);
 }
+
+extern "C" size_t pa_decode_multi_workspace_bytes(int total_q, int num_heads, int head_size,
+                                                  int max_context_len, int partition_size) {
+  const int P = resolve_partition(partition_size);
+  if (P < 0 || P % 128 != 0 || total_q < 0 || num_heads < 0 || head_size < 0) return 0;
+  return workspace_bytes(total_q, num_heads, head_size, num_partitions(max_context_len, P));
+}
+
+extern "C" pa_status pa_decode_multi(void* out, const void* q, const void* k_cache,
+                                     const void* v_cache, const int32_t* block_tables,
+                                     int max_blocks_per_seq, const int32_t* context_lens,
+                                     const int32_t* query_start_loc, int num_seqs, int total_q,
+                                     int max_query_len, int num_heads, int num_kv_heads,
+                                     int head_size, int block_size, int num_blocks, float scale,
+                                     pa_dtype dtype, int partition_size, int max_context_len,
+                                     void* workspace, size_t workspace_bytes_in, void* stream) {
+  const char* fn = "pa_decode_multi";
+  if (pa::elem_size(dtype) == 0) return pa::fail(PA_ERR_INVALID, "%s: unknown dtype %d", fn, dtype);
+  if (dtype != PA_F16 && dtype != PA_BF16)
+    return pa::fail(PA_ERR_UNSUPPORTED, "%s: q, out and the caches must be f16 or bf16", fn);
+  if (num_seqs < 0 || total_q < 0) return pa::fail(PA_ERR_INVALID, "%s: negative count", fn);
+  if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0)
+    return pa::fail(PA_ERR_INVALID, "%s: num_heads must be a positive multiple of num_kv_heads", fn);
+  if (!supported_group(num_heads / num_kv_heads))
+    return pa::fail(PA_ERR_UNSUPPORTED, "%s: query heads per kv head must be 1, 2, 4 or 8", fn);
+  if (num_kv_heads > 65535) return pa::fail(PA_ERR_UNSUPPORTED, "%s: num_kv_heads > 65535", fn);
+  if (head_size != 128) return pa::fail(PA_ERR_UNSUPPORTED, "%s: head_size must be 128", fn);
+  if (block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
+    return pa::fail(PA_ERR_INVALID, "%s: sizes must be positive", fn);
+  if (!supported_block(block_size))
+    return pa::fail(PA_ERR_UNSUPPORTED, "%s: block_size must be 8, 16 or 32", fn);
+  const int P = resolve_partition(partition_size);
+  if (P < 0 || P % 128 != 0)
+    return pa::fail(PA_ERR_INVALID, "%s: partition_size must be 0 or a positive multiple of 128", fn);
+  if (max_context_len < 0 ||
+      static_cast<int64_t>(max_context_len) > static_cast<int64_t>(max_blocks_per_seq) * block_size)
+    return pa::fail(PA_ERR_INVALID, "%s: max_context_len out of range", fn);
+  if (total_q > 0 && (max_query_len < 1 || max_query_len > total_q || max_query_len > max_context_len))
+    return pa::fail(PA_ERR_INVALID, "%s: max_query_len must be in [1, min(total_q, max_context_len)]", fn);
+  if (!std::isfinite(scale)) return pa::fail(PA_ERR_INVALID, "%s: scale is not finite", fn);
+  const int64_t NP = num_partitions(max_context_len, P);
+  const int G = num_heads / num_kv_heads;
+  const int64_t qblocks = total_q > 0 ? (max_query_len + pa::kMqRows / G - 1) / (pa::kMqRows / G) : 0;
+  if (qblocks * NP > 65535) return pa::fail(PA_ERR_UNSUPPORTED, "%s: too many query blocks x partitions", fn);
+  if (num_seqs == 0 || total_q == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start_loc)
+    return pa::fail(PA_ERR_INVALID, "%s: NULL device pointer", fn);
+  if (!pa::aligned16(out) || !pa::aligned16(q) || !pa::aligned16(k_cache) || !pa::aligned16(v_cache))
+    return pa::fail(PA_ERR_INVALID, "%s: out, q and the caches must be 16-byte aligned", fn);
+  if ((reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(query_start_loc) & 3u))
+    return pa::fail(PA_ERR_INVALID, "%s: int32 arrays must be 4-byte aligned", fn);
+  if (static_cast<int64_t>(num_blocks) * num_kv_heads * block_size >= (int64_t(1) << 31))
+    return pa::fail(PA_ERR_UNSUPPORTED, "%s: cache larger than 2^31 rows", fn);
+  const size_t need = workspace_bytes(total_q, num_heads, head_size, NP);
+  if (need > 0 && (!workspace || workspace_bytes_in < need || !pa::aligned16(workspace)))
+    return pa::fail(PA_ERR_INVALID, "%s: a 16-byte aligned workspace of %zu bytes is needed", fn, need);
+  if (!pa::tmap_available())
+    return pa::fail(PA_ERR_UNSUPPORTED, "%s: the driver's tensor-map encoder is unavailable", fn);
+  pa::MqArgs a;
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.query_start = query_start_loc;
+  a.workspace = need > 0 ? static_cast<float*>(workspace) : nullptr;
+  a.max_blocks = max_blocks_per_seq;
+  a.num_seqs = num_seqs;
+  a.total_q = total_q;
+  a.max_query_len = max_query_len;
+  a.Hq = num_heads;
+  a.Hkv = num_kv_heads;
+  a.D = head_size;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.partition_size = P;
+  a.num_partitions = static_cast<int>(NP);
+  a.scale = scale;
+  a.dtype = dtype;
+  unsigned int* status = pa::device_status_word();
+  if (!status) return PA_ERR_CUDA;
+  pa_status st = launch_status(fn, pa::launch_decode_mq(a, status, stream), 1);
+  if (st != PA_OK || NP <= 1) return st;
+  return launch_status(fn, pa::launch_decode_mq_reduce(a, stream), 1);
+}

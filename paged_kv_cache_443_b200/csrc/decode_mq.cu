@@ -1,0 +1,607 @@
+// decode_mq.cu -- paged attention for several new query tokens per sequence
+// (chunked prefill, speculative verification) on the tensor cores: fp16/bf16,
+// head size 128, G = Hq/Hkv in {1, 2, 4, 8}.
+//
+// What is computed ("자기회귀 생성과 KV 캐시" and "PagedAttention의 설계",
+// supersilo.blog; chunked prefill and speculative decoding in "4. 이 밖의
+// 기법들", blog.aqudi.me): sequence b's last Q_b context tokens are its query
+// tokens (rows query_start[b] .. query_start[b+1]-1 of q); query token i sits
+// at position L_b - Q_b + i and attends, through the block table, to
+// positions 0 .. L_b - Q_b + i with one softmax over them.
+//
+// With many query rows the work is query-major, as in a prefill kernel: a CTA
+// serves one (sequence, kv head, block of 128/G query tokens, partition of
+// keys); its 128 rows are (query token, query head) pairs of that kv head, and
+// per tile of 128 keys
+//
+//   S [128 rows x 128 keys] = Q [128 x 128] . K^T          (K K-major)
+//   O [128 rows x 128 dims] += P [128 x 128 keys] . V      (V MN-major)
+//
+// run on tcgen05 (kind::f16, fp32 accumulation in TMEM).  K and V tiles are
+// the TMA boxes of decode_tc.cu (one 4-D box per physical block, 128-byte
+// swizzle).  Each softmax thread owns one row: its running max, sum and
+// causal limit are thread-local, and a warp rescales its own 32 rows of O in
+// TMEM when one of its maxima grows by more than 2^8.
+//
+// Roles (6 warps): warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
+// warps 2-5 Q staging, softmax and epilogue.  About 193 KB of shared memory
+// and all 512 TMEM columns: one CTA per SM.  Every wait is bounded; block ids
+// outside the pool are skipped and flagged; inconsistent query offsets are
+// flagged (PA_DEVERR_CONTEXT) and their sequence skipped.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <type_traits>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+#include "tc_common.cuh"
+
+namespace pa {
+
+namespace {
+
+using namespace tc;
+
+constexpr unsigned FULL = 0xffffffffu;
+constexpr int TOK = 128;                   // keys per tile
+constexpr int MR = 128;                    // query rows per CTA
+constexpr int DH = 128;
+constexpr int SLOTS = 3;
+constexpr int SLOT_BYTES = TOK * 256;      // K or V tile (as in decode_tc.cu): 32 KB
+constexpr int GROUP_BYTES = 2048;
+constexpr int HALF_OFF = 1024;
+constexpr int OPA_BYTES = MR * 256;        // a 128 x 128 16-bit row-major operand: 32 KB
+constexpr int OPA_HALF = MR * 128;         // its second 64-column half
+constexpr int OFF_RING = 0;
+constexpr int OFF_Q = OFF_RING + SLOTS * SLOT_BYTES;
+constexpr int OFF_P = OFF_Q + OPA_BYTES;   // two P buffers
+constexpr int OFF_BAR = OFF_P + 2 * OPA_BYTES;
+constexpr int NBARS = 2 * SLOTS + 9;
+constexpr int OFF_TMEM = OFF_BAR + NBARS * 8;
+constexpr int SMEM_USED = OFF_TMEM + 16;
+constexpr int SMEM_BYTES = SMEM_USED + 1024;
+constexpr int THREADS = 192;
+constexpr int TMEM_COLS = 512;             // S0 [0,128), S1 [128,256), O [256,384)
+constexpr int O_COL = 256;
+constexpr float RESCALE_THRESHOLD = 8.0f;
+
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+
+// kind::f16 instruction descriptor, fp32 accumulation, M = 128, N = 128;
+// A K-major; B K-major (S) or MN-major (O).
+template <typename T>
+__device__ __forceinline__ constexpr uint32_t idesc_mq(bool b_mn_major) {
+  constexpr uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(128 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+
+// Byte offset of the 16-byte chunk c (elements 8c..8c+7) of row r of a
+// 128 x 128 16-bit operand stored as two 64-column halves with the 128-byte
+// swizzle (the canonical K-major layout).
+__device__ __forceinline__ uint32_t opa_chunk(int r, int c) {
+  return (c >> 3) * OPA_HALF + r * 128 + ((((c & 7) ^ (r & 7)) & 7) << 4);
+}
+
+struct MqParams {
+  void* out;
+  const void* q;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  const int32_t* query_start;
+  float* ws_o;
+  float* ws_m;
+  float* ws_l;
+  unsigned int* status;
+  int64_t max_blocks;
+  int num_seqs, total_q, Hq, Hkv, num_blocks, block_size, partition_size, num_partitions;
+  float scale_log2;
+};
+
+template <typename T, int G>
+__global__ void __launch_bounds__(THREADS, 1)
+    decode_mq_kernel(const MqParams p, const __grid_constant__ CUtensorMap tmap_k,
+                     const __grid_constant__ CUtensorMap tmap_v) {
+  constexpr int QB = MR / G;                        // query tokens per CTA
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* ring = smem + OFF_RING;
+  uint8_t* qop = smem + OFF_Q;
+  uint8_t* pop = smem + OFF_P;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* ring_full = bars;
+  uint64_t* ring_empty = bars + SLOTS;
+  uint64_t* s_full = bars + 2 * SLOTS;      // [2]
+  uint64_t* s_free = s_full + 2;            // [2]
+  uint64_t* p_full = s_free + 2;            // [2]
+  uint64_t* p_free = p_full + 2;            // [2]
+  uint64_t* q_ready = p_free + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
+
+  const int b = blockIdx.x, g = blockIdx.y;
+  const int qb = blockIdx.z / p.num_partitions, part = blockIdx.z % p.num_partitions;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  grid_dependency_wait();
+  allow_dependents();
+  // ---- this CTA's query rows and key range (validated) ----
+  const int q0 = p.query_start[b];
+  const int Qb = p.query_start[b + 1] - q0;
+  int L = p.context_lens[b];
+  const int P = p.partition_size;
+  int64_t cap = p.max_blocks * p.block_size;
+  const int64_t grid_cap = static_cast<int64_t>(p.num_partitions) * P;
+  cap = cap < grid_cap ? cap : grid_cap;
+  if (L < 0 || L > cap || Qb < 0 || Qb > L || q0 < 0 || q0 + Qb > p.total_q) {
+    if (threadIdx.x == 0 && qb == 0 && part == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
+    return;
+  }
+  if (qb == 0 && part == 0 && g == 0 && threadIdx.x == 0 &&
+      Qb > static_cast<int>(gridDim.z / p.num_partitions) * QB)
+    atomicOr(p.status, PA_DEVERR_CONTEXT);          // max_query_len below this Q_b
+  if (qb * QB >= Qb) return;                        // no query tokens in this block
+  const int i_last = min(Qb, (qb + 1) * QB) - 1;    // last query token of the block
+  const int pmax = L - Qb + i_last;                 // its position: the last key needed
+  const int kstart = part * P;
+  if (kstart > pmax) return;
+  const int kend = min(kstart + P, pmax + 1);
+  const int n_tiles = (kend - kstart + TOK - 1) / TOK;
+  const bool single = (pmax < P);
+
+  const int bs = p.block_size;
+  const int bpt = TOK / bs;
+  const int first_blk = kstart / bs;
+  const int last_blk = (kend + bs - 1) / bs;
+  const int32_t* trow = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SLOTS; ++s) {
+      mbar_init(&ring_full[s], 1);
+      mbar_init(&ring_empty[s], 1);
+    }
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(&s_full[j], 1);
+      mbar_init(&s_free[j], 4);
+      mbar_init(&p_full[j], 4);
+      mbar_init(&p_free[j], 1);
+    }
+    mbar_init(q_ready, 4);
+    fence_mbar_init();
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ================= producer (as in decode_tc.cu) =================
+    const int row_stride = p.Hkv * bs;
+    bool ok = true;
+    int issued = 0;
+    for (int i = 0; i < n_tiles && ok; ++i) {
+      const int b0 = first_blk + i * bpt;
+      const int nb = min(bpt, last_blk - b0);
+      const int pb = lane < nb ? __ldg(trow + b0 + lane) : -1;
+      const bool mine = lane < nb;
+      const bool valid = mine && pb >= 0 && pb < p.num_blocks;
+      if (mine && !valid) atomicOr(p.status, PA_DEVERR_TABLE);
+      const unsigned vmask = __ballot_sync(FULL, valid);
+      const uint32_t bytes = __popc(vmask) * 2u * static_cast<uint32_t>(bs) * 128u;
+      const int grp = valid ? (pb * row_stride + g * bs) / 8 : 0;
+      for (int kv = 0; kv < 2; ++kv) {
+        const int u = 2 * i + kv;
+        const int s = u % SLOTS;
+        if (u >= SLOTS && !mbar_wait(&ring_empty[s], ((u / SLOTS) - 1) & 1, p.status)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) mbar_arrive_expect_tx(&ring_full[s], bytes);
+        __syncwarp();
+        if (valid)
+          tma_load_4d(ring + s * SLOT_BYTES + lane * bs * 256, kv == 0 ? &tmap_k : &tmap_v, 0, 0,
+                      0, grp, &ring_full[s]);
+        issued = u + 1;
+      }
+    }
+    if (!ok) {
+      for (int u = issued - SLOTS < 0 ? 0 : issued - SLOTS; u < issued; ++u)
+        mbar_wait(&ring_full[u % SLOTS], (u / SLOTS) & 1, p.status);
+    }
+    return;
+  }
+
+  // rows of this CTA: r = il * G + hl  (query token il of the block, head hl)
+  const int quad = warp & 3;
+  const int r = quad * 32 + lane;
+  const int il = r / G, hl = r % G;
+  const bool row_valid = warp >= 2 && qb * QB + il < Qb;
+  const int64_t t = static_cast<int64_t>(q0) + qb * QB + il;          // query token index
+  const int pos = L - Qb + qb * QB + il;                               // its position
+
+  if (warp >= 2) {
+    // Q operand: row r = q[t][g*G + hl][:], zero for rows past the block's tokens
+    const T* src = static_cast<const T*>(p.q) + (t * p.Hq + g * G + hl) * DH;
+#pragma unroll 4
+    for (int c = 0; c < DH / 8; ++c) {
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (row_valid) v = __ldg(reinterpret_cast<const uint4*>(src + c * 8));
+      *reinterpret_cast<uint4*>(qop + opa_chunk(r, c)) = v;
+    }
+    fence_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(q_ready);
+  }
+
+  if (warp == 1) {
+    // ================= MMA issuer =================
+    if (lane == 0) {
+      const uint32_t id_s = idesc_mq<T>(false);
+      const uint32_t id_o = idesc_mq<T>(true);
+      const uint32_t ring_a = smem_addr(ring), q_a = smem_addr(qop), p_a = smem_addr(pop);
+      bool ok = true;
+      auto issue_s = [&](int i) -> bool {
+        const int u = 2 * i, s = u % SLOTS;
+        if (!mbar_wait(&ring_full[s], (u / SLOTS) & 1, p.status)) return false;
+        if (i >= 2 && !mbar_wait(&s_free[i & 1], ((i >> 1) - 1) & 1, p.status)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + (i & 1) * 128;
+#pragma unroll
+        for (int k = 0; k < DH / 16; ++k) {
+          const uint64_t a = smem_desc(q_a + (k >> 2) * OPA_HALF + (k & 3) * 32, 16, 1024);
+          const uint64_t bk =
+              smem_desc(ring_a + s * SLOT_BYTES + (k >> 2) * HALF_OFF + (k & 3) * 32, 16, GROUP_BYTES);
+          mma_f16(d, a, bk, id_s, k > 0);
+        }
+        mma_commit(&s_full[i & 1]);
+        mma_commit(&ring_empty[s]);
+        return true;
+      };
+      auto issue_o = [&](int i) -> bool {
+        const int u = 2 * i + 1, s = u % SLOTS;
+        if (!mbar_wait(&ring_full[s], (u / SLOTS) & 1, p.status)) return false;
+        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, p.status)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + O_COL;
+#pragma unroll
+        for (int k = 0; k < TOK / 16; ++k) {
+          const uint64_t a =
+              smem_desc(p_a + (i & 1) * OPA_BYTES + (k >> 2) * OPA_HALF + (k & 3) * 32, 16, 1024);
+          const uint64_t bv =
+              smem_desc(ring_a + s * SLOT_BYTES + k * 2 * GROUP_BYTES, HALF_OFF, GROUP_BYTES);
+          mma_f16(d, a, bv, id_o, (i > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(&ring_empty[s]);
+        mma_commit(&p_free[i & 1]);
+        return true;
+      };
+      ok = mbar_wait(q_ready, 0, p.status) && issue_s(0);
+      for (int i = 0; i < n_tiles && ok; ++i) {
+        if (i + 1 < n_tiles) ok = issue_s(i + 1);
+        if (ok) ok = issue_o(i);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 2) {
+    // ================= softmax: one row per thread =================
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    float m_run = -INFINITY, l_sum = 0.f;
+    bool ok = true;
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+      if (ok) ok = mbar_wait(bar, parity, p.status);
+      ok = __all_sync(FULL, ok);
+      return ok;
+    };
+    for (int i = 0; i < n_tiles; ++i) {
+      const int tile0 = kstart + i * TOK;
+      const int n_valid = min(TOK, kend - tile0);
+      const int lim = row_valid ? min(pos - tile0, n_valid - 1) : -1;  // last key column of this row
+      float sv[TOK];
+      if (wait(&s_full[i & 1], (i >> 1) & 1)) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < TOK / 32; ++c) tmem_ld32(tmem + lane_base + (i & 1) * 128 + c * 32, sv + c * 32);
+      } else {
+#pragma unroll
+        for (int j = 0; j < TOK; ++j) sv[j] = 0.f;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[i & 1]);
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < TOK; ++j) {
+        sv[j] = j <= lim ? sv[j] * p.scale_log2 : -INFINITY;
+        tmax = fmaxf(tmax, sv[j]);
+      }
+      const bool need = tmax > m_run + RESCALE_THRESHOLD;
+      if (__any_sync(FULL, need)) {
+        const float mnew = fmaxf(m_run, tmax);
+        const float alpha = (m_run == -INFINITY) ? 0.f : exp2f(m_run - mnew);
+        m_run = mnew;
+        l_sum *= alpha;
+        // O must hold every earlier tile before it is rescaled
+        if (i > 0 && wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < DH / 32; ++c) {
+            float o[32];
+            tmem_ld32(tmem + lane_base + O_COL + c * 32, o);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] *= alpha;
+            tmem_st32(tmem + lane_base + O_COL + c * 32, o);
+          }
+        }
+      }
+      if (i >= 2) wait(&p_free[i & 1], ((i >> 1) - 1) & 1);
+      uint8_t* pb = pop + (i & 1) * OPA_BYTES;
+#pragma unroll
+      for (int c = 0; c < TOK / 8; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float p0 = sv[8 * c + 2 * e] == -INFINITY ? 0.f : exp2f(sv[8 * c + 2 * e] - m_run);
+          const float p1 =
+              sv[8 * c + 2 * e + 1] == -INFINITY ? 0.f : exp2f(sv[8 * c + 2 * e + 1] - m_run);
+          l_sum += p0 + p1;
+          w[e] = static_cast<uint32_t>(to_bits<T>(p0)) | (static_cast<uint32_t>(to_bits<T>(p1)) << 16);
+        }
+        *reinterpret_cast<uint4*>(pb + opa_chunk(r, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      if (n_valid < TOK) {
+        // the last tile: zero the V rows of keys past the range, so that
+        // whatever they hold adds 0 * 0 to O
+        const int u = 2 * i + 1, s_ = u % SLOTS;
+        if (wait(&ring_full[s_], (u / SLOTS) & 1) && r >= n_valid) {
+          uint8_t* row = ring + s_ * SLOT_BYTES + (r >> 3) * GROUP_BYTES + (r & 7) * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            *reinterpret_cast<uint4*>(row + c * 16) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(row + HALF_OFF + c * 16) = make_uint4(0, 0, 0, 0);
+          }
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[i & 1]);
+    }
+    // ---- epilogue: row r of O ----
+    wait(&p_free[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1);
+    tc_fence_after();
+    const int64_t hq = t * p.Hq + g * G + hl;
+#pragma unroll 1
+    for (int c = 0; c < DH / 32; ++c) {
+      float o[32];
+      tmem_ld32(tmem + lane_base + O_COL + c * 32, o);
+      if (ok && row_valid) {
+        if (single) {
+          const float inv = 1.f / l_sum;
+          T* dst = static_cast<T*>(p.out) + hq * DH + c * 32;
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = static_cast<uint32_t>(to_bits<T>(o[j + 2 * e] * inv)) |
+                     (static_cast<uint32_t>(to_bits<T>(o[j + 2 * e + 1] * inv)) << 16);
+            *reinterpret_cast<uint4*>(dst + j) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        } else {
+          const int64_t slot = hq * p.num_partitions + part;
+          float* dst = p.ws_o + slot * DH + c * 32;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(dst + j) = make_float4(o[j], o[j + 1], o[j + 2], o[j + 3]);
+          if (c == 0) {
+            p.ws_m[slot] = m_run;
+            p.ws_l[slot] = l_sum;
+          }
+        }
+      }
+    }
+  }
+
+  // ---- teardown: warps 1-5 meet, warp 1 frees TMEM ----
+  tc_fence_before();
+  named_sync(2, 160);
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+struct MqReduceParams {
+  void* out;
+  const int32_t* context_lens;
+  const int32_t* query_start;
+  const float* ws_o;
+  const float* ws_m;
+  const float* ws_l;
+  int num_seqs, total_q, Hq, G, partition_size, num_partitions;
+};
+
+// One warp per (query token, head) whose block spanned several partitions.
+template <typename T>
+__global__ void __launch_bounds__(128) decode_mq_reduce_kernel(const MqReduceParams p) {
+  constexpr int DPL = DH / 32;
+  grid_dependency_wait();
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= static_cast<int64_t>(p.total_q) * p.Hq) return;
+  const int t = static_cast<int>(row / p.Hq);
+  // the sequence of token t: the last b with query_start[b] <= t
+  int lo = 0, hi = p.num_seqs;                      // invariant: qs[lo] <= t < qs[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (p.query_start[mid] <= t) lo = mid; else hi = mid;
+  }
+  const int b = lo;
+  const int Qb = p.query_start[b + 1] - p.query_start[b];
+  const int L = p.context_lens[b];
+  const int i = t - p.query_start[b];
+  if (Qb <= 0 || Qb > L || i < 0 || i >= Qb) return;   // flagged by the partition kernel
+  const int QB = MR / p.G;
+  const int i_last = min(Qb, (i / QB + 1) * QB) - 1;
+  const int pmax = L - Qb + i_last;
+  if (pmax < p.partition_size) return;              // written directly
+  const int pos = L - Qb + i;
+  const int np = min(pos / p.partition_size + 1, p.num_partitions);
+  const int64_t base = row * p.num_partitions;
+  float M = -INFINITY;
+  for (int k = lane; k < np; k += 32) M = fmaxf(M, p.ws_m[base + k]);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, off));
+  float Ls = 0.f;
+  for (int k = lane; k < np; k += 32) Ls += p.ws_l[base + k] * exp2f(p.ws_m[base + k] - M);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) Ls += __shfl_xor_sync(FULL, Ls, off);
+  float acc[DPL];
+#pragma unroll
+  for (int k = 0; k < DPL; ++k) acc[k] = 0.f;
+  for (int k = 0; k < np; ++k) {
+    const float f = exp2f(p.ws_m[base + k] - M);
+    const float* src = p.ws_o + (base + k) * DH + lane * DPL;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[e] = fmaf(f, src[e], acc[e]);
+  }
+  T* dst = static_cast<T*>(p.out) + row * DH + lane * DPL;
+  const float inv = 1.f / Ls;
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) dst[e] = Elem<T>::from_float(acc[e] * inv);
+}
+
+template <typename T, int G>
+cudaError_t launch_mq_t(const MqArgs& a, unsigned int* status, cudaStream_t stream) {
+  auto kern = decode_mq_kernel<T, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  CUtensorMap mk, mv;
+  const int64_t groups = static_cast<int64_t>(a.num_blocks) * a.Hkv * a.block_size / 8;
+  const int64_t dims[4] = {64, 8, 2, groups};
+  const int64_t strides[3] = {DH * 2, 128, 8 * DH * 2};
+  const int box[4] = {64, 8, 2, a.block_size / 8};
+  if (!make_tmap(&mk, a.k_cache, 4, dims, strides, box, a.dtype) ||
+      !make_tmap(&mv, a.v_cache, 4, dims, strides, box, a.dtype))
+    return cudaErrorInvalidValue;
+  MqParams p;
+  p.out = a.out;
+  p.q = a.q;
+  p.block_tables = a.block_tables;
+  p.context_lens = a.context_lens;
+  p.query_start = a.query_start;
+  const int64_t nrows = static_cast<int64_t>(a.total_q) * a.Hq * a.num_partitions;
+  p.ws_o = a.workspace;
+  p.ws_m = a.workspace ? a.workspace + nrows * DH : nullptr;
+  p.ws_l = a.workspace ? a.workspace + nrows * (DH + 1) : nullptr;
+  p.status = status;
+  p.max_blocks = a.max_blocks;
+  p.num_seqs = a.num_seqs;
+  p.total_q = a.total_q;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.num_blocks = a.num_blocks;
+  p.block_size = a.block_size;
+  p.partition_size = a.partition_size;
+  p.num_partitions = a.num_partitions;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  const int qblocks = (a.max_query_len + MR / G - 1) / (MR / G);
+  dim3 grid(a.num_seqs, a.Hkv, qblocks * a.num_partitions);
+  return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
+}
+
+template <typename T>
+cudaError_t launch_mq_reduce_t(const MqArgs& a, cudaStream_t stream) {
+  MqReduceParams p;
+  p.out = a.out;
+  p.context_lens = a.context_lens;
+  p.query_start = a.query_start;
+  const int64_t nrows = static_cast<int64_t>(a.total_q) * a.Hq * a.num_partitions;
+  p.ws_o = a.workspace;
+  p.ws_m = a.workspace + nrows * DH;
+  p.ws_l = a.workspace + nrows * (DH + 1);
+  p.num_seqs = a.num_seqs;
+  p.total_q = a.total_q;
+  p.Hq = a.Hq;
+  p.G = a.Hq / a.Hkv;
+  p.partition_size = a.partition_size;
+  p.num_partitions = a.num_partitions;
+  const int64_t warps = static_cast<int64_t>(a.total_q) * a.Hq;
+  const unsigned grid = static_cast<unsigned>((warps + 3) / 4);
+  return launch_overlapped(decode_mq_reduce_kernel<T>, dim3(grid), dim3(128), 0, stream, p);
+}
+
+template <typename T>
+cudaError_t launch_mq_g(const MqArgs& a, unsigned int* status, cudaStream_t stream) {
+  switch (a.Hq / a.Hkv) {
+    case 1: return launch_mq_t<T, 1>(a, status, stream);
+    case 2: return launch_mq_t<T, 2>(a, status, stream);
+    case 4: return launch_mq_t<T, 4>(a, status, stream);
+    case 8: return launch_mq_t<T, 8>(a, status, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+int launch_decode_mq(const MqArgs& a, unsigned int* status, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return a.dtype == PA_BF16 ? launch_mq_g<__nv_bfloat16>(a, status, st)
+                            : launch_mq_g<__half>(a, status, st);
+}
+
+int launch_decode_mq_reduce(const MqArgs& a, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return a.dtype == PA_BF16 ? launch_mq_reduce_t<__nv_bfloat16>(a, st)
+                            : launch_mq_reduce_t<__half>(a, st);
+}
+
+}  // namespace pa

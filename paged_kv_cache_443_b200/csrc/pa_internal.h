@@ -80,6 +80,26 @@ bool make_tmap(void* map, const void* base, int rank, const int64_t* dims,
 // Whether the driver entry point that encodes tensor maps could be found.
 bool tmap_available();
 
+// ---- several query tokens per sequence (decode_mq.cu) ----
+struct MqArgs {
+  void* out;
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  const int32_t* query_start;
+  float* workspace;  // may be null when num_partitions == 1
+  int64_t max_blocks;
+  int num_seqs, total_q, max_query_len, Hq, Hkv, D, block_size, num_blocks;
+  int partition_size, num_partitions;
+  float scale;
+  pa_dtype dtype;
+};
+constexpr int kMqRows = 128;  // (query token, head) rows per CTA of the multi-query kernel
+int launch_decode_mq(const MqArgs& a, unsigned int* status, void* stream);
+int launch_decode_mq_reduce(const MqArgs& a, void* stream);
+
 int launch_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
                              const int64_t* slot_mapping, int num_tokens, int Hkv, int D,
                              int block_size, int num_blocks, int esize, unsigned int* status,

@@ -499,3 +499,80 @@ def test_fp8_tc_query_magnitudes(dtype, mag):
     want = oracle_attention(o, spec)
     assert np.isfinite(got).all()
     assert np.abs(got - want).max() <= TOL[spec.dtype]
+
+
+# ---------------------------------------------------------------------------
+# several new query tokens per sequence (chunked prefill, speculative verify)
+
+
+def mq_check(spec, qlens, partition_size=512, seed=0, bad_offsets=False):
+    sc = W.scenario(spec)
+    p, o = build(sc)
+    run_step(p, spec)
+    torch.cuda.synchronize()
+    lens = o.lens.astype(np.int64)
+    qlens = np.minimum(np.asarray(qlens, dtype=np.int64), lens)
+    qs = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    T = int(qs[-1])
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    q = torch.randn((T, spec.Hq, spec.D), generator=g, device="cuda").to(W.torch_dtype(spec))
+    out = torch.full_like(q, float("nan"))
+    maxq = max(1, int(qlens.max()))
+    n = pk.pa_decode_multi_workspace_bytes(T, spec.Hq, spec.D, p.max_ctx, partition_size)
+    ws = torch.empty(n // 4, dtype=torch.float32, device="cuda") if n else None
+    qs_dev = torch.from_numpy(qs).cuda()
+    if bad_offsets:
+        qs_dev[1] = qs_dev[2] + 1                  # not non-decreasing
+    pk.pa_decode_multi(out, q, p.cache.k_cache, p.cache.v_cache, p.tables, p.lens, qs_dev,
+                       spec.softmax_scale, p.max_ctx, maxq, partition_size=partition_size,
+                       workspace=ws)
+    torch.cuda.synchronize()
+    if bad_offsets:
+        return out, pk.pa_device_status()
+    assert pk.pa_device_status() == 0
+    got = as_f64(out, spec)
+    want = oracle.paged_attention_mq(W.storage_view(q), o.k, o.v, spec.dtype_code, o.tables,
+                                     o.lens, qs, spec.softmax_scale)
+    assert np.isfinite(got).all()
+    err = np.abs(got - want).max() if T else 0.0
+    assert err <= TOL[spec.dtype], err
+    return got, want
+
+
+def mq_spec(dtype, G, bs, lens, seed, P=512):
+    return W.Spec(f"mq_{dtype}_{G}_{bs}", dtype, 2 * G, 2, 128, bs, "independent", len(lens),
+                  seed=seed, ctx_dist="explicit", ctx_list=tuple(lens), partition_size=P)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("P", [128, 512])
+def test_mq_speculative_verify(dtype, G, P):
+    spec = mq_spec(dtype, G, 16, (5, 40, 300, 513, 1100, 2000), seed=500 + G)
+    mq_check(spec, (1, 4, 8, 3, 8, 5), partition_size=P)
+
+
+@pytest.mark.parametrize("G", [1, 4, 8])
+def test_mq_chunked_prefill(G):
+    """Whole prompts and long chunks as queries: several query blocks per
+    sequence (128/G tokens each) and several key partitions."""
+    spec = mq_spec("bf16", G, 16, (200, 700, 1500, 90), seed=600 + G)
+    mq_check(spec, (200, 300, 260, 90), partition_size=256)
+
+
+@pytest.mark.parametrize("bs", [8, 32])
+def test_mq_block_sizes(bs):
+    spec = mq_spec("f16", 4, bs, (33, 257, 1000), seed=700 + bs)
+    mq_check(spec, (33, 20, 129), partition_size=128)
+
+
+def test_mq_edges():
+    spec = mq_spec("bf16", 8, 16, (0, 1, 2, 127, 128, 129, 255), seed=801)
+    mq_check(spec, (0, 1, 2, 127, 1, 129, 16), partition_size=128)
+
+
+def test_mq_bad_offsets_are_flagged_without_faulting():
+    spec = mq_spec("bf16", 4, 16, (50, 60, 70), seed=802)
+    _, status = mq_check(spec, (3, 4, 5), bad_offsets=True)
+    assert status & pk.PA_DEVERR_CONTEXT
+    mq_check(spec, (3, 4, 5))                      # the context is still healthy

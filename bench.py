@@ -24,6 +24,11 @@ scaling; the step time is the max over ranks.
 --impl reference times the oracle (the plain fp64 CPU implementation) on the
 host cores on the same workload and metric, one bounded sample per step.
 
+--op mq (1 GPU) measures the multi-query kernel (pa_decode_multi) on
+--workload verify_gqa70b (the gqa70b batch verifying 4 proposed tokens per
+sequence) or prefill_gqa70b (16 sequences with contexts U[2048,8192] whose last
+512 tokens are a prefill chunk).
+
 --op swap (1 GPU) measures the block swap instead: every block of the
 workload's batch to a pinned host pool (scattered ids) and back, one
 pa_swap_blocks launch per direction, against one contiguous device<->pinned
@@ -286,6 +291,15 @@ def profiled_traffic(workload, kernel="decode_partition_kernel"):
     if not m or not s or s.group(1) != source_digest(KERNEL_SOURCES[kernel]):
         return None
     return float(m.group(1))
+
+
+def measured_peak_tensor():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (bf16 burst)"
+    except Exception:
+        return 1590.0, "fallback"
 
 
 def measured_peak_hbm():
@@ -628,6 +642,136 @@ def run_ours(args):
     return result
 
 
+MQ_WORKLOADS = {
+    # (spec, query tokens per sequence, description)
+    "verify_gqa70b": (W.GQA70B, 4, "speculative verify: the gqa70b batch (256 seqs, Hq=64, Hkv=8, "
+                      "D=128, bf16, context U[256,4096]) checking 4 proposed tokens per sequence"),
+    "prefill_gqa70b": (None, 512, "chunked prefill: 16 sequences, Hq=64, Hkv=8, D=128, bf16, block "
+                       "16, context U[2048,8192] whose last 512 tokens are the chunk"),
+}
+
+
+def mq_spec(name):
+    from dataclasses import replace
+    if name.endswith("_quarter"):       # the profiling case: a quarter of the sequences
+        spec, Q = mq_spec(name[: -len("_quarter")])
+        return replace(spec, name=name, num_seqs=max(1, spec.num_seqs // 4)), Q
+    spec, Q, _ = MQ_WORKLOADS[name]
+    if spec is None:
+        spec = replace(W.GQA70B, name="prefill_gqa70b", num_seqs=16, ctx_lo=2048, ctx_hi=8192,
+                       seed=449)
+    return spec, Q
+
+
+def run_mq(args):
+    """Multi-query attention throughput (TFLOP/s and KV GB/s) on one GPU."""
+    import torch
+    import paged_kv_cache_443_b200 as pk
+    from paged_kv_cache_443_b200.cache import PagedKVCache
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: a CUDA device is required for --op mq")
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    pk.lib()
+    spec, Q = mq_spec(args.workload)
+    sc = W.scenario(spec)
+    cache = PagedKVCache(sc.num_blocks, spec.block_size, spec.Hkv, spec.D, W.torch_kv_dtype(spec),
+                         device, sc.free_order.tolist(), fill=0.0)
+    for op in sc.setup_ops + sc.step_ops:
+        if op.kind == "add":
+            cache.add(op.seq)
+        elif op.kind == "fork":
+            cache.fork(op.seq, op.arg)
+        elif op.kind == "release":
+            cache.release(op.seq)
+        else:
+            k, v = W.kv_content(spec, op.kv_id, op.arg, device)
+            cache.append([op.seq], [op.arg], k, v)
+            del k, v
+    tables, lens, max_ctx = cache.tables(sc.batch, sc.max_blocks)
+    lens_h = lens.cpu().numpy().astype(np.int64)
+    qlens = np.minimum(Q, lens_h)
+    qs = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    T = int(qs[-1])
+    g = torch.Generator(device=device).manual_seed(spec.seed)
+    q = torch.randn((T, spec.Hq, spec.D), generator=g, device=device).to(W.torch_dtype(spec))
+    out = torch.empty_like(q)
+    qs_d = torch.from_numpy(qs).to(device)
+    P = args.partition_size or 512
+    n = pk.pa_decode_multi_workspace_bytes(T, spec.Hq, spec.D, max_ctx, P)
+    ws = torch.empty(n // 4, dtype=torch.float32, device=device) if n else None
+    maxq = int(qlens.max())
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        pk.pa_decode_multi(out, q, cache.k_cache, cache.v_cache, tables, lens, qs_d,
+                           spec.softmax_scale, max_ctx, maxq, partition_size=P, workspace=ws,
+                           stream=stream)
+
+    unique, logical, other = step_bytes(spec, tables.cpu().numpy(), lens_h)
+    # flops: 4 * D per (query row, attended key): q.k and p.v, 2 flops each per element
+    pos_sum = sum(int(qlens[b]) * (2 * int(lens_h[b]) - int(qlens[b]) + 1) // 2
+                  for b in range(len(lens_h)))
+    flops = 4.0 * spec.D * spec.Hq * pos_sum
+    alg_bytes = unique + 2 * T * spec.Hq * spec.D * spec.esize
+    flush = unique < 8 * L2_BYTES
+    scratch = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=device) if flush else None
+    sink = torch.empty((), dtype=torch.float32, device=device)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(device)
+    assert pk.pa_device_status() == 0
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    sampler = ClockSampler(0)
+    sampler.start()
+    t0 = time.time()
+    launches0 = pk.pa_launch_count()
+    for i in range(K):
+        if flush:
+            torch.amax(scratch, dim=0, out=sink)
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(device)
+    t1 = time.time()
+    sampler.stop()
+    launches = pk.pa_launch_count() - launches0
+    assert pk.pa_device_status() == 0
+    ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    tflops = flops / (ms * 1e-3) / 1e12
+    gbs = alg_bytes / (ms * 1e-3) / 1e9
+    hbm_peak, hbm_kind = measured_peak_hbm()
+    tc_peak, tc_kind = measured_peak_tensor()
+    tensor_bound = tflops / tc_peak > gbs / hbm_peak
+    return {
+        "metric": "multi-query paged attention: TFLOP/s (tensor-bound work) or KV GB/s (HBM-bound)",
+        "op": "mq",
+        "value": round(tflops if tensor_bound else gbs, 2),
+        "unit": "TFLOP/s" if tensor_bound else "GB/s",
+        "n_gpus": 1, "steps": K, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": spec.dtype,
+        "data": "synthetic: seeded N(0,1) K/V/q, context lengths and placement as the workload states",
+        "config": {"workload": f"{args.workload}: {MQ_WORKLOADS[args.workload.replace('_quarter', '')][2]}",
+                   "num_seqs": len(sc.batch), "query_tokens": T, "query_tokens_per_seq": Q,
+                   "max_context_len": max_ctx, "partition_size": P,
+                   "kv_bytes_unique": unique, "flops": flops,
+                   "l2": "L2 flushed between timed steps" if flush else "inputs larger than L2"},
+        "tflops": round(tflops, 2), "kv_gbs": round(gbs, 2),
+        "roofline": {"kernel": "decode_mq_kernel (+ reduce)",
+                     "bound": "tensor" if tensor_bound else "hbm",
+                     "achieved": round(tflops if tensor_bound else gbs, 2),
+                     "peak": tc_peak if tensor_bound else hbm_peak,
+                     "peak_kind": tc_kind if tensor_bound else hbm_kind,
+                     "unit": "TFLOP/s" if tensor_bound else "GB/s",
+                     "frac": round(tflops / tc_peak if tensor_bound else gbs / hbm_peak, 4),
+                     "other_frac": round(gbs / hbm_peak if tensor_bound else tflops / tc_peak, 4)},
+        "gpu_launches": int(launches),
+        "clocks": sampler.summary(t0, t1),
+    }
+
+
 def run_swap(args):
     """Swap-out / swap-in bandwidth of pa_swap_blocks on the workload's blocks."""
     import torch
@@ -746,13 +890,15 @@ def main():
                              "long_prefix_bs16_quarter", "opt13b_fp8", "opt13b_compact_fp8",
                              "gqa70b_fp8", "gqa70b_quarter_fp8", "long_prefix_bs8_fp8",
                              "long_prefix_bs16_fp8", "long_prefix_bs32_fp8",
-                             "long_prefix_bs16_quarter_fp8", "llama13b_ps_fp8", "tiny_fp8"])
+                             "long_prefix_bs16_quarter_fp8", "llama13b_ps_fp8", "tiny_fp8",
+                             "verify_gqa70b", "prefill_gqa70b", "verify_gqa70b_quarter",
+                             "prefill_gqa70b_quarter"])
     ap.add_argument("--partition-size", type=int, default=0,
                     help="split-K partition length (0: the workload's own, 512)")
     ap.add_argument("--soak-seconds", type=float, default=0.5,
                     help="untimed load before the timed steps (clock samples)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--op", default="decode", choices=["decode", "swap"],
+    ap.add_argument("--op", default="decode", choices=["decode", "swap", "mq"],
                     help="decode: the hot path (default); swap: block swap bandwidth")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -785,6 +931,10 @@ def main():
     if args.op == "swap":
         if rank == 0 and args.impl == "ours":
             print(json.dumps(run_swap(args)), flush=True)
+        return
+    if args.op == "mq":
+        if rank == 0 and args.impl == "ours":
+            print(json.dumps(run_mq(args)), flush=True)
         return
 
     result = run_ours(args)

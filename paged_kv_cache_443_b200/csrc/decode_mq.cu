@@ -24,8 +24,9 @@
 // TMEM when one of its maxima grows by more than 2^8.
 //
 // Roles (6 warps): warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
-// warps 2-5 Q staging, softmax and epilogue.  About 193 KB of shared memory
-// and all 512 TMEM columns: one CTA per SM.  Every wait is bounded; block ids
+// warps 2-5 Q staging, softmax and epilogue.  A ring of four K/V tiles (one
+// CTA per SM has to keep two tiles of loads in flight by itself), about 225 KB
+// of shared memory and all 512 TMEM columns: one CTA per SM.  Every wait is bounded; block ids
 // outside the pool are skipped and flagged; inconsistent query offsets are
 // flagged (PA_DEVERR_CONTEXT) and their sequence skipped.
 #include <cuda.h>
@@ -48,7 +49,7 @@ constexpr unsigned FULL = 0xffffffffu;
 constexpr int TOK = 128;                   // keys per tile
 constexpr int MR = 128;                    // query rows per CTA
 constexpr int DH = 128;
-constexpr int SLOTS = 3;
+constexpr int SLOTS = 4;
 constexpr int SLOT_BYTES = TOK * 256;      // K or V tile (as in decode_tc.cu): 32 KB
 constexpr int GROUP_BYTES = 2048;
 constexpr int HALF_OFF = 1024;
@@ -112,6 +113,19 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
       "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
       "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
+}
+
+// One TMEM load of 128 consecutive 32-bit columns of this thread's lane, one wait.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v) {
+  uint32_t r[128];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%128];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // Byte offset of the 16-byte chunk c (elements 8c..8c+7) of row r of a
@@ -225,10 +239,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int row_stride = p.Hkv * bs;
     bool ok = true;
     int issued = 0;
+    auto table = [&](int i) {                       // lane j: block j of tile i, read a tile ahead
+      const int b0 = first_blk + i * bpt;
+      return (i < n_tiles && lane < min(bpt, last_blk - b0)) ? __ldg(trow + b0 + lane) : -1;
+    };
+    int pb_next = table(0);
     for (int i = 0; i < n_tiles && ok; ++i) {
       const int b0 = first_blk + i * bpt;
       const int nb = min(bpt, last_blk - b0);
-      const int pb = lane < nb ? __ldg(trow + b0 + lane) : -1;
+      const int pb = pb_next;
+      pb_next = table(i + 1);
       const bool mine = lane < nb;
       const bool valid = mine && pb >= 0 && pb < p.num_blocks;
       if (mine && !valid) atomicOr(p.status, PA_DEVERR_TABLE);
@@ -268,12 +288,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp >= 2) {
     // Q operand: row r = q[t][g*G + hl][:], zero for rows past the block's tokens
     const T* src = static_cast<const T*>(p.q) + (t * p.Hq + g * G + hl) * DH;
-#pragma unroll 4
-    for (int c = 0; c < DH / 8; ++c) {
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (row_valid) v = __ldg(reinterpret_cast<const uint4*>(src + c * 8));
-      *reinterpret_cast<uint4*>(qop + opa_chunk(r, c)) = v;
-    }
+    uint4 v[DH / 8];                                 // all 16 loads in flight at once
+#pragma unroll
+    for (int c = 0; c < DH / 8; ++c)
+      v[c] = row_valid ? __ldg(reinterpret_cast<const uint4*>(src + c * 8)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int c = 0; c < DH / 8; ++c) *reinterpret_cast<uint4*>(qop + opa_chunk(r, c)) = v[c];
     fence_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(q_ready);
@@ -330,6 +350,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
   } else if (warp >= 2) {
     // ================= softmax: one row per thread =================
+    // A warp whose 32 rows hold no query token (few queries per sequence) only
+    // keeps pace with the barriers and zeroes V rows; its P rows stay zero.
+    const bool warp_active = __any_sync(FULL, row_valid);
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     float m_run = -INFINITY, l_sum = 0.f;
     bool ok = true;
@@ -338,61 +361,84 @@ __global__ void __launch_bounds__(THREADS, 1)
       ok = __all_sync(FULL, ok);
       return ok;
     };
+    if (!warp_active) {
+#pragma unroll
+      for (int buf = 0; buf < 2; ++buf)
+#pragma unroll
+        for (int c = 0; c < TOK / 8; ++c)
+          *reinterpret_cast<uint4*>(pop + buf * OPA_BYTES + opa_chunk(r, c)) = make_uint4(0, 0, 0, 0);
+    }
     for (int i = 0; i < n_tiles; ++i) {
       const int tile0 = kstart + i * TOK;
       const int n_valid = min(TOK, kend - tile0);
-      const int lim = row_valid ? min(pos - tile0, n_valid - 1) : -1;  // last key column of this row
-      float sv[TOK];
-      if (wait(&s_full[i & 1], (i >> 1) & 1)) {
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < TOK / 32; ++c) tmem_ld32(tmem + lane_base + (i & 1) * 128 + c * 32, sv + c * 32);
-      } else {
-#pragma unroll
-        for (int j = 0; j < TOK; ++j) sv[j] = 0.f;
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[i & 1]);
-      float tmax = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < TOK; ++j) {
-        sv[j] = j <= lim ? sv[j] * p.scale_log2 : -INFINITY;
-        tmax = fmaxf(tmax, sv[j]);
-      }
-      const bool need = tmax > m_run + RESCALE_THRESHOLD;
-      if (__any_sync(FULL, need)) {
-        const float mnew = fmaxf(m_run, tmax);
-        const float alpha = (m_run == -INFINITY) ? 0.f : exp2f(m_run - mnew);
-        m_run = mnew;
-        l_sum *= alpha;
-        // O must hold every earlier tile before it is rescaled
-        if (i > 0 && wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
+      wait(&s_full[i & 1], (i >> 1) & 1);
+      if (warp_active) {
+        const int lim = row_valid ? min(pos - tile0, n_valid - 1) : -1;  // last key column
+        float sv[TOK];
+        if (ok) {
           tc_fence_after();
-#pragma unroll 1
-          for (int c = 0; c < DH / 32; ++c) {
-            float o[32];
-            tmem_ld32(tmem + lane_base + O_COL + c * 32, o);
+          tmem_ld128(tmem + lane_base + (i & 1) * 128, sv);
+        } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] *= alpha;
-            tmem_st32(tmem + lane_base + O_COL + c * 32, o);
+          for (int j = 0; j < TOK; ++j) sv[j] = 0.f;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[i & 1]);
+        float pm[8];                                   // 8 independent partial maxima
+#pragma unroll
+        for (int k = 0; k < 8; ++k) pm[k] = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < TOK; ++j) {
+          sv[j] = j <= lim ? sv[j] * p.scale_log2 : -INFINITY;
+          pm[j & 7] = fmaxf(pm[j & 7], sv[j]);
+        }
+        const float tmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                 fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        const bool need = tmax > m_run + RESCALE_THRESHOLD;
+        if (__any_sync(FULL, need)) {
+          const float mnew = fmaxf(m_run, tmax);
+          const float alpha = (m_run == -INFINITY) ? 0.f : exp2f(m_run - mnew);
+          m_run = mnew;
+          l_sum *= alpha;
+          // O must hold every earlier tile before it is rescaled
+          if (i > 0 && wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < DH / 32; ++c) {
+              float o[32];
+              tmem_ld32(tmem + lane_base + O_COL + c * 32, o);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) o[j] *= alpha;
+              tmem_st32(tmem + lane_base + O_COL + c * 32, o);
+            }
           }
         }
-      }
-      if (i >= 2) wait(&p_free[i & 1], ((i >> 1) - 1) & 1);
-      uint8_t* pb = pop + (i & 1) * OPA_BYTES;
+        if (i >= 2) wait(&p_free[i & 1], ((i >> 1) - 1) & 1);
+        uint8_t* pb = pop + (i & 1) * OPA_BYTES;
+        float ps[8];                                   // 8 independent partial sums
 #pragma unroll
-      for (int c = 0; c < TOK / 8; ++c) {
-        uint32_t w[4];
+        for (int k = 0; k < 8; ++k) ps[k] = 0.f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = sv[8 * c + 2 * e] == -INFINITY ? 0.f : exp2f(sv[8 * c + 2 * e] - m_run);
-          const float p1 =
-              sv[8 * c + 2 * e + 1] == -INFINITY ? 0.f : exp2f(sv[8 * c + 2 * e + 1] - m_run);
-          l_sum += p0 + p1;
-          w[e] = static_cast<uint32_t>(to_bits<T>(p0)) | (static_cast<uint32_t>(to_bits<T>(p1)) << 16);
+        for (int c = 0; c < TOK / 8; ++c) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float p0 = sv[8 * c + 2 * e] == -INFINITY ? 0.f : exp2f(sv[8 * c + 2 * e] - m_run);
+            const float p1 =
+                sv[8 * c + 2 * e + 1] == -INFINITY ? 0.f : exp2f(sv[8 * c + 2 * e + 1] - m_run);
+            ps[2 * e] += p0;
+            ps[2 * e + 1] += p1;
+            w[e] = static_cast<uint32_t>(to_bits<T>(p0)) |
+                   (static_cast<uint32_t>(to_bits<T>(p1)) << 16);
+          }
+          *reinterpret_cast<uint4*>(pb + opa_chunk(r, c)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        *reinterpret_cast<uint4*>(pb + opa_chunk(r, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+        l_sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      } else {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[i & 1]);
       }
       if (n_valid < TOK) {
         // the last tile: zero the V rows of keys past the range, so that
@@ -417,7 +463,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after();
     const int64_t hq = t * p.Hq + g * G + hl;
 #pragma unroll 1
-    for (int c = 0; c < DH / 32; ++c) {
+    for (int c = 0; c < (warp_active ? DH / 32 : 0); ++c) {
       float o[32];
       tmem_ld32(tmem + lane_base + O_COL + c * 32, o);
       if (ok && row_valid) {

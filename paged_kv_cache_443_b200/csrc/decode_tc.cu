@@ -63,7 +63,7 @@ constexpr int OFF_RING = 0;
 constexpr int OFF_Q = OFF_RING + SLOTS * SLOT_BYTES;
 constexpr int OFF_P = OFF_Q + OPB_BYTES;     // two P buffers
 constexpr int OFF_BAR = OFF_P + 2 * OPB_BYTES;
-constexpr int NBARS = 2 * SLOTS + 9;         // ring full/empty, s/p full/free, q_ready
+constexpr int NBARS = 2 * SLOTS + 10;        // ring full/empty, s/p full/free, q_ready, o_free
 constexpr int OFF_TMEM = OFF_BAR + NBARS * 8;
 constexpr int OFF_RED = OFF_TMEM + 16;       // 4 warps x 16 floats
 constexpr int SMEM_USED = OFF_RED + 4 * NPAD * 4;
@@ -85,6 +85,7 @@ struct TcParams {
   unsigned int* status;
   int64_t max_blocks;
   int Hq, Hkv, num_blocks, block_size, partition_size, num_partitions;
+  int parts_per_cta;  // consecutive partitions one CTA streams through
   float scale_log2;
 };
 
@@ -106,10 +107,14 @@ __global__ void __launch_bounds__(THREADS, 2)
   uint64_t* p_full = s_free + 2;            // [2]
   uint64_t* p_free = p_full + 2;            // [2]
   uint64_t* q_ready = p_free + 2;           // Q^T operand staged
+  uint64_t* o_free = q_ready + 1;           // a partition's O has been read out
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
   float* red = reinterpret_cast<float*>(smem + OFF_RED);
 
-  const int b = blockIdx.x, g = blockIdx.y, part = blockIdx.z;
+  // A CTA streams parts_per_cta consecutive partitions (tiles never straddle
+  // one: P is a multiple of TOK) and writes each one's partial as it ends, so
+  // short partitions do not each pay the pipeline's fill and drain.
+  const int b = blockIdx.x, g = blockIdx.y, part = blockIdx.z * p.parts_per_cta;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   grid_dependency_wait();   // the appended tokens of the previous kernel are in the cache
@@ -132,8 +137,10 @@ __global__ void __launch_bounds__(THREADS, 2)
     return;
   }
   if (start >= L) return;
-  const int end = min(L, start + P);
+  const int end = static_cast<int>(min(static_cast<int64_t>(L),
+                                       start + static_cast<int64_t>(P) * p.parts_per_cta));
   const int n_tiles = (end - start + TOK - 1) / TOK;
+  const int tpp = P / TOK;                               // tiles per partition
   const bool single = (L <= P);
 
   // ---- set-up: the producer starts streaming right after the barrier, while
@@ -158,6 +165,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         mbar_init(&p_free[j], 1);
       }
       mbar_init(q_ready, 4);
+      mbar_init(o_free, 4);
       fence_mbar_init();
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
@@ -262,6 +270,8 @@ __global__ void __launch_bounds__(THREADS, 2)
         const int u = 2 * i + 1, s = u % SLOTS;
         if (!mbar_wait(&ring_full[s], (u / SLOTS) & 1, p.status)) return false;
         if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, p.status)) return false;
+        const bool first = (i % tpp) == 0;             // a partition starts: O restarts at 0
+        if (first && i > 0 && !mbar_wait(o_free, ((i / tpp) - 1) & 1, p.status)) return false;
         tc_fence_after();
         const uint32_t d = tmem + 2 * NPAD;
 #pragma unroll
@@ -270,7 +280,7 @@ __global__ void __launch_bounds__(THREADS, 2)
               smem_desc(ring_a + s * SLOT_BYTES + k * 2 * GROUP_BYTES, HALF_OFF, GROUP_BYTES);
           const uint64_t bp =
               smem_desc(p_a + (i & 1) * OPB_BYTES + (k >> 2) * (NPAD * 128) + (k & 3) * 32, 16, 1024);
-          mma_f16(d, a, bp, id_pv, (i > 0 || k > 0) ? 1u : 0u);
+          mma_f16(d, a, bp, id_pv, (!first || k > 0) ? 1u : 0u);
         }
         mma_commit(&ring_empty[s]);
         mma_commit(&p_free[i & 1]);
@@ -303,9 +313,58 @@ __global__ void __launch_bounds__(THREADS, 2)
       ok = __all_sync(FULL, ok);
       return ok;
     };
+    // Row r of O^T (dim r, all heads) and the sums of the partition ending at
+    // tile i: the output, or the split-K partial of partition part + i / tpp.
+    auto flush = [&](int i) {
+      wait(&p_free[i & 1], (i >> 1) & 1);
+      tc_fence_after();
+      float o[16];
+      tmem_ld16(tmem + lane_base + 2 * NPAD, o);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_free);              // the next partition may reuse O
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float x = l_part[h];
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(FULL, x, off);
+        l_part[h] = x;
+      }
+      named_sync(1, 128);
+      if (lane == 0) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) red[quad * NPAD + h] = l_part[h];
+      }
+      named_sync(1, 128);
+      if (ok) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float Ls = red[h] + red[NPAD + h] + red[2 * NPAD + h] + red[3 * NPAD + h];
+          const int64_t hq = static_cast<int64_t>(b) * p.Hq + g * G + h;
+          if (single) {
+            static_cast<T*>(p.out)[hq * DH + r] = Elem<T>::from_float(o[h] / Ls);
+          } else {
+            const int64_t slot = hq * p.num_partitions + part + i / tpp;
+            p.ws_o[slot * DH + r] = o[h];
+            if (r == 0) {
+              p.ws_m[slot] = m_run[h];
+              p.ws_l[slot] = Ls;
+            }
+          }
+        }
+      }
+    };
     for (int i = 0; i < n_tiles; ++i) {
       const int n_valid = min(TOK, end - (start + i * TOK));
       const bool valid = r < n_valid;
+      const bool first = (i % tpp) == 0;
+      if (first && i > 0) {                            // a new partition: a new softmax
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          m_run[h] = -INFINITY;
+          l_part[h] = 0.f;
+        }
+      }
       float sv[16];
       if (wait(&s_full[i & 1], (i >> 1) & 1)) {
         tc_fence_after();
@@ -345,8 +404,9 @@ __global__ void __launch_bounds__(THREADS, 2)
           l_part[h] *= alpha[h];
         }
         named_sync(1, 128);
-        // O must hold every earlier tile before it is rescaled
-        if (i > 0 && wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
+        // O must hold every earlier tile of the partition before it is rescaled
+        // (at a partition's first tile O restarts from zero instead)
+        if (!first && wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
           tc_fence_after();
           float o[16];
           tmem_ld16(tmem + lane_base + 2 * NPAD, o);
@@ -383,41 +443,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[i & 1]);
-    }
-    // ---- epilogue: row r of O^T (dim r, all heads) and the sums ----
-    wait(&p_free[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1);
-    tc_fence_after();
-    float o[16];
-    tmem_ld16(tmem + lane_base + 2 * NPAD, o);
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float x = l_part[h];
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(FULL, x, off);
-      l_part[h] = x;
-    }
-    named_sync(1, 128);
-    if (lane == 0) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) red[quad * NPAD + h] = l_part[h];
-    }
-    named_sync(1, 128);
-    if (ok) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float Ls = red[h] + red[NPAD + h] + red[2 * NPAD + h] + red[3 * NPAD + h];
-        const int64_t hq = static_cast<int64_t>(b) * p.Hq + g * G + h;
-        if (single) {
-          static_cast<T*>(p.out)[hq * DH + r] = Elem<T>::from_float(o[h] / Ls);
-        } else {
-          const int64_t slot = hq * p.num_partitions + part;
-          p.ws_o[slot * DH + r] = o[h];
-          if (r == 0) {
-            p.ws_m[slot] = m_run[h];
-            p.ws_l[slot] = Ls;
-          }
-        }
-      }
+      if ((i + 1) % tpp == 0 || i == n_tiles - 1) flush(i);
     }
   }
 
@@ -433,6 +459,26 @@ __global__ void __launch_bounds__(THREADS, 2)
 }
 
 // ---- host side ----
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+// Consecutive partitions per CTA: the most of 4 / 2 that keeps a CTA's span
+// within 2048 tokens and still leaves at least 8 CTAs per SM.
+int tc_parts_per_cta(const DecodeArgs& a) {
+  const int64_t want = 8ll * sm_count();
+  for (int c : {4, 2}) {
+    const int64_t ctas = static_cast<int64_t>(a.num_seqs) * a.Hkv * ((a.num_partitions + c - 1) / c);
+    if (static_cast<int64_t>(a.partition_size) * c <= 2048 && a.num_partitions >= c && ctas >= want)
+      return c;
+  }
+  return 1;
+}
 
 template <typename T, int G>
 cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
@@ -467,8 +513,9 @@ cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t 
   p.block_size = a.block_size;
   p.partition_size = a.partition_size;
   p.num_partitions = a.num_partitions;
+  p.parts_per_cta = tc_parts_per_cta(a);
   p.scale_log2 = a.scale * 1.4426950408889634f;
-  dim3 grid(a.num_seqs, a.Hkv, a.num_partitions);
+  dim3 grid(a.num_seqs, a.Hkv, (a.num_partitions + p.parts_per_cta - 1) / p.parts_per_cta);
   return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
 }
 

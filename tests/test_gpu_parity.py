@@ -576,3 +576,28 @@ def test_mq_bad_offsets_are_flagged_without_faulting():
     _, status = mq_check(spec, (3, 4, 5), bad_offsets=True)
     assert status & pk.PA_DEVERR_CONTEXT
     mq_check(spec, (3, 4, 5))                      # the context is still healthy
+
+
+# ---------------------------------------------------------------------------
+# the tcgen05 decode kernel streaming several partitions per CTA (chosen when the
+# grid has at least 8 CTAs per SM): every partition's partial must be right
+
+
+@pytest.mark.parametrize("P", [128, 256, 512])
+def test_tc_several_partitions_per_cta(P):
+    spec = W.Spec(f"ppc_{P}", "bf16", 32, 4, 128, 16, "independent", 320, seed=900 + P,
+                  ctx_dist="uniform", ctx_lo=1, ctx_hi=2000, partition_size=P)
+    sc = W.scenario(spec)
+    p, o = build(sc)
+    out = run_step(p, spec)
+    torch.cuda.synchronize()
+    assert pk.pa_device_status() == 0
+    rows = sampled_rows(o, spec, n=160, seed=P)
+    want = oracle_attention(o, spec, rows=rows)
+    got_all = as_f64(out, spec)
+    assert np.isfinite(got_all).all()
+    assert np.abs(got_all[rows[:, 0], rows[:, 1]] - want).max() <= TOL[spec.dtype]
+    # the same batch at one partition per CTA (long partitions) agrees
+    out2 = run_step(p, spec, partition_size=4096)
+    torch.cuda.synchronize()
+    assert np.abs(as_f64(out2, spec) - got_all).max() <= TOL[spec.dtype]

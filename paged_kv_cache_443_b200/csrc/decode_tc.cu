@@ -89,7 +89,7 @@ struct TcParams {
   float scale_log2;
 };
 
-template <typename T, int G>
+template <typename T, int G, bool MULTI>
 __global__ void __launch_bounds__(THREADS, 2)
     decode_partition_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmap_k,
                                const __grid_constant__ CUtensorMap tmap_v) {
@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(THREADS, 2)
   // A CTA streams parts_per_cta consecutive partitions (tiles never straddle
   // one: P is a multiple of TOK) and writes each one's partial as it ends, so
   // short partitions do not each pay the pipeline's fill and drain.
-  const int b = blockIdx.x, g = blockIdx.y, part = blockIdx.z * p.parts_per_cta;
+  const int b = blockIdx.x, g = blockIdx.y, part = MULTI ? blockIdx.z * p.parts_per_cta : blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   grid_dependency_wait();   // the appended tokens of the previous kernel are in the cache
@@ -137,10 +137,11 @@ __global__ void __launch_bounds__(THREADS, 2)
     return;
   }
   if (start >= L) return;
-  const int end = static_cast<int>(min(static_cast<int64_t>(L),
-                                       start + static_cast<int64_t>(P) * p.parts_per_cta));
+  const int end = MULTI ? static_cast<int>(min(static_cast<int64_t>(L),
+                                               start + static_cast<int64_t>(P) * p.parts_per_cta))
+                        : min(L, start + P);
   const int n_tiles = (end - start + TOK - 1) / TOK;
-  const int tpp = P / TOK;                               // tiles per partition
+  const int tpp = MULTI ? P / TOK : (1 << 30);                               // tiles per partition
   const bool single = (L <= P);
 
   // ---- set-up: the producer starts streaming right after the barrier, while
@@ -271,7 +272,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         if (!mbar_wait(&ring_full[s], (u / SLOTS) & 1, p.status)) return false;
         if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, p.status)) return false;
         const bool first = (i % tpp) == 0;             // a partition starts: O restarts at 0
-        if (first && i > 0 && !mbar_wait(o_free, ((i / tpp) - 1) & 1, p.status)) return false;
+        if (MULTI && first && i > 0 && !mbar_wait(o_free, ((i / tpp) - 1) & 1, p.status)) return false;
         tc_fence_after();
         const uint32_t d = tmem + 2 * NPAD;
 #pragma unroll
@@ -322,7 +323,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       tmem_ld16(tmem + lane_base + 2 * NPAD, o);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(o_free);              // the next partition may reuse O
+      if (MULTI && lane == 0) mbar_arrive(o_free);              // the next partition may reuse O
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         float x = l_part[h];
@@ -358,7 +359,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       const int n_valid = min(TOK, end - (start + i * TOK));
       const bool valid = r < n_valid;
       const bool first = (i % tpp) == 0;
-      if (first && i > 0) {                            // a new partition: a new softmax
+      if (MULTI && first && i > 0) {                            // a new partition: a new softmax
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           m_run[h] = -INFINITY;
@@ -443,8 +444,9 @@ __global__ void __launch_bounds__(THREADS, 2)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[i & 1]);
-      if ((i + 1) % tpp == 0 || i == n_tiles - 1) flush(i);
+      if (MULTI && (i + 1) % tpp == 0 && i + 1 < n_tiles) flush(i);   // a partition ends mid-CTA
     }
+    flush(n_tiles - 1);                                       // the CTA's last partition
   }
 
   // ---- teardown: warps 1-5 meet, warp 1 frees TMEM ----
@@ -460,29 +462,11 @@ __global__ void __launch_bounds__(THREADS, 2)
 
 // ---- host side ----
 
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-    return 148;
-  return n;
-}
-
-// Consecutive partitions per CTA: the most of 4 / 2 that keeps a CTA's span
-// within 2048 tokens and still leaves at least 8 CTAs per SM.
-int tc_parts_per_cta(const DecodeArgs& a) {
-  const int64_t want = 8ll * sm_count();
-  for (int c : {4, 2}) {
-    const int64_t ctas = static_cast<int64_t>(a.num_seqs) * a.Hkv * ((a.num_partitions + c - 1) / c);
-    if (static_cast<int64_t>(a.partition_size) * c <= 2048 && a.num_partitions >= c && ctas >= want)
-      return c;
-  }
-  return 1;
-}
-
 template <typename T, int G>
 cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
-  auto kern = decode_partition_tc_kernel<T, G>;
+  const int ppc = tc_parts_per_cta(a);
+  // one partition per CTA compiles without the partition-streaming logic
+  auto kern = ppc > 1 ? decode_partition_tc_kernel<T, G, true> : decode_partition_tc_kernel<T, G, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // the cache [NB][Hkv][bs][128] as a 4-D tensor: 64 columns (stride 2 B),
@@ -513,13 +497,33 @@ cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t 
   p.block_size = a.block_size;
   p.partition_size = a.partition_size;
   p.num_partitions = a.num_partitions;
-  p.parts_per_cta = tc_parts_per_cta(a);
+  p.parts_per_cta = ppc;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   dim3 grid(a.num_seqs, a.Hkv, (a.num_partitions + p.parts_per_cta - 1) / p.parts_per_cta);
   return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
 }
 
 }  // namespace
+
+static int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+// Consecutive partitions per CTA: the most of 4 / 2 that keeps a CTA's span
+// within 2048 tokens and still leaves at least 8 CTAs per SM.
+int tc_parts_per_cta(const DecodeArgs& a) {
+  const int64_t want = 8ll * sm_count();
+  for (int c : {4, 2}) {
+    const int64_t ctas = static_cast<int64_t>(a.num_seqs) * a.Hkv * ((a.num_partitions + c - 1) / c);
+    if (static_cast<int64_t>(a.partition_size) * c <= 2048 && a.num_partitions >= c && ctas >= want)
+      return c;
+  }
+  return 1;
+}
 
 namespace {
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {

@@ -72,7 +72,7 @@ constexpr int OFF_ST = OFF_VOP + VOP_BYTES;
 constexpr int OFF_Q = OFF_ST + ST_SLOTS * ST_BYTES;
 constexpr int OFF_P = OFF_Q + NTERM * QT_BYTES;   // two P buffers
 constexpr int OFF_BAR = OFF_P + 2 * OPB_BYTES;
-constexpr int NBARS = 2 * KR_SLOTS + 2 * ST_SLOTS + 2 + 8 + 1;
+constexpr int NBARS = 2 * KR_SLOTS + 2 * ST_SLOTS + 2 + 8 + 2;
 constexpr int OFF_TMEM = (OFF_BAR + NBARS * 8 + 15) / 16 * 16;
 constexpr int OFF_RED = OFF_TMEM + 16;      // 4 warps x 16 floats
 constexpr int OFF_QS = OFF_RED + 4 * NPAD * 4;
@@ -113,6 +113,7 @@ struct Tc8Params {
   unsigned int* status;
   int64_t max_blocks;
   int Hq, Hkv, num_blocks, block_size, partition_size, num_partitions;
+  int parts_per_cta;  // consecutive partitions one CTA streams through
   float scale_log2;  // scale * log2(e) * k_scale
   float v_scale;
 };
@@ -145,7 +146,7 @@ __device__ __forceinline__ float2 from_e4m3x2(uint32_t c) {
   return __half22float2(*reinterpret_cast<const __half2*>(&lo));
 }
 
-template <typename T, int G>
+template <typename T, int G, bool MULTI>
 __global__ void __launch_bounds__(THREADS, 2)
     decode_partition_tc8_kernel(const Tc8Params p, const __grid_constant__ CUtensorMap tmap_k) {
   extern __shared__ uint8_t smem_raw[];
@@ -168,11 +169,13 @@ __global__ void __launch_bounds__(THREADS, 2)
   uint64_t* p_full = s_free + 2;             // [2]
   uint64_t* p_free = p_full + 2;             // [2]
   uint64_t* q_ready = p_free + 2;
+  uint64_t* o_free = q_ready + 1;            // a partition's O has been read out
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
   float* red = reinterpret_cast<float*>(smem + OFF_RED);
   float* qs = reinterpret_cast<float*>(smem + OFF_QS);
 
-  const int b = blockIdx.x, g = blockIdx.y, part = blockIdx.z;
+  // a CTA streams parts_per_cta consecutive partitions (as in decode_tc.cu)
+  const int b = blockIdx.x, g = blockIdx.y, part = MULTI ? blockIdx.z * p.parts_per_cta : blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   grid_dependency_wait();
@@ -195,8 +198,11 @@ __global__ void __launch_bounds__(THREADS, 2)
     return;
   }
   if (start >= L) return;
-  const int end = min(L, start + P);
+  const int end = MULTI ? static_cast<int>(min(static_cast<int64_t>(L),
+                                               start + static_cast<int64_t>(P) * p.parts_per_cta))
+                        : min(L, start + P);
   const int n_tiles = (end - start + TOK - 1) / TOK;
+  const int tpp = MULTI ? P / TOK : (1 << 30);                    // tiles per partition
   const bool single = (L <= P);
 
   const int bs = p.block_size;
@@ -221,6 +227,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       mbar_init(&p_free[j], 1);
     }
     mbar_init(q_ready, 4);
+    mbar_init(o_free, 4);
     fence_mbar_init();
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
   }
@@ -437,6 +444,8 @@ __global__ void __launch_bounds__(THREADS, 2)
       auto issue_pv = [&](int i) -> bool {
         if (!mbar_wait(vop_full, i & 1, p.status)) return false;
         if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, p.status)) return false;
+        const bool first = (i % tpp) == 0;     // a partition starts: O restarts at 0
+        if (MULTI && first && i > 0 && !mbar_wait(o_free, ((i / tpp) - 1) & 1, p.status)) return false;
         tc_fence_after();
         const uint32_t d = tmem + 2 * NPAD;
 #pragma unroll
@@ -444,7 +453,7 @@ __global__ void __launch_bounds__(THREADS, 2)
           const uint64_t a = smem_desc(v_a + k * 2 * GROUP_BYTES, HALF_OFF, GROUP_BYTES);
           const uint64_t bp =
               smem_desc(p_a + (i & 1) * OPB_BYTES + (k >> 2) * (NPAD * 128) + (k & 3) * 32, 16, 1024);
-          mma_f16(d, a, bp, id_pv, (i > 0 || k > 0) ? 1u : 0u);
+          mma_f16(d, a, bp, id_pv, (!first || k > 0) ? 1u : 0u);
         }
         mma_commit(vop_empty);
         mma_commit(&p_free[i & 1]);
@@ -475,9 +484,58 @@ __global__ void __launch_bounds__(THREADS, 2)
       ok = __all_sync(FULL, ok);
       return ok;
     };
+    // row r of O^T and the sums of the partition ending at tile i
+    auto flush = [&](int i) {
+      wait(&p_free[i & 1], (i >> 1) & 1);
+      tc_fence_after();
+      float o[16];
+      tmem_ld16(tmem + lane_base + 2 * NPAD, o);
+      tc_fence_before();
+      __syncwarp();
+      if (MULTI && lane == 0) mbar_arrive(o_free);      // the next partition may reuse O
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float x = l_part[h];
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(FULL, x, off);
+        l_part[h] = x;
+      }
+      named_sync(1, 128);
+      if (lane == 0) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) red[quad * NPAD + h] = l_part[h];
+      }
+      named_sync(1, 128);
+      if (ok) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float Ls = red[h] + red[NPAD + h] + red[2 * NPAD + h] + red[3 * NPAD + h];
+          const float O = o[h] * p.v_scale;
+          const int64_t hq = static_cast<int64_t>(b) * p.Hq + g * G + h;
+          if (single) {
+            static_cast<T*>(p.out)[hq * DH + r] = Elem<T>::from_float(O / Ls);
+          } else {
+            const int64_t slot = hq * p.num_partitions + part + i / tpp;
+            p.ws_o[slot * DH + r] = O;
+            if (r == 0) {
+              p.ws_m[slot] = m_run[h];
+              p.ws_l[slot] = Ls;
+            }
+          }
+        }
+      }
+    };
     for (int i = 0; i < n_tiles; ++i) {
       const int n_valid = min(TOK, end - (start + i * TOK));
       const bool valid = r < n_valid;
+      const bool first = (i % tpp) == 0;
+      if (MULTI && first && i > 0) {                    // a new partition: a new softmax
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          m_run[h] = -INFINITY;
+          l_part[h] = 0.f;
+        }
+      }
       float sv[16];
       if (wait(&s_full[i & 1], (i >> 1) & 1)) {
         tc_fence_after();
@@ -516,7 +574,7 @@ __global__ void __launch_bounds__(THREADS, 2)
           l_part[h] *= alpha[h];
         }
         named_sync(1, 128);
-        if (i > 0 && wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
+        if (!first && wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
           tc_fence_after();
           float o[16];
           tmem_ld16(tmem + lane_base + 2 * NPAD, o);
@@ -540,43 +598,9 @@ __global__ void __launch_bounds__(THREADS, 2)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[i & 1]);
+      if (MULTI && (i + 1) % tpp == 0 && i + 1 < n_tiles) flush(i);   // a partition ends mid-CTA
     }
-    // ---- epilogue ----
-    wait(&p_free[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1);
-    tc_fence_after();
-    float o[16];
-    tmem_ld16(tmem + lane_base + 2 * NPAD, o);
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float x = l_part[h];
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(FULL, x, off);
-      l_part[h] = x;
-    }
-    named_sync(1, 128);
-    if (lane == 0) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) red[quad * NPAD + h] = l_part[h];
-    }
-    named_sync(1, 128);
-    if (ok) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float Ls = red[h] + red[NPAD + h] + red[2 * NPAD + h] + red[3 * NPAD + h];
-        const float O = o[h] * p.v_scale;
-        const int64_t hq = static_cast<int64_t>(b) * p.Hq + g * G + h;
-        if (single) {
-          static_cast<T*>(p.out)[hq * DH + r] = Elem<T>::from_float(O / Ls);
-        } else {
-          const int64_t slot = hq * p.num_partitions + part;
-          p.ws_o[slot * DH + r] = O;
-          if (r == 0) {
-            p.ws_m[slot] = m_run[h];
-            p.ws_l[slot] = Ls;
-          }
-        }
-      }
-    }
+    flush(n_tiles - 1);                                       // the CTA's last partition
   }
 
   // ---- teardown: warps 1-5 meet, warp 1 frees TMEM ----
@@ -592,7 +616,9 @@ __global__ void __launch_bounds__(THREADS, 2)
 
 template <typename T, int G>
 cudaError_t launch_tc8_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
-  auto kern = decode_partition_tc8_kernel<T, G>;
+  const int ppc = tc_parts_per_cta(a);
+  // one partition per CTA compiles without the partition-streaming logic
+  auto kern = ppc > 1 ? decode_partition_tc8_kernel<T, G, true> : decode_partition_tc8_kernel<T, G, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // the K cache [NB][Hkv][bs][128] as rows of 128 codes; a box is the bs rows of
@@ -621,9 +647,10 @@ cudaError_t launch_tc8_t(const DecodeArgs& a, unsigned int* status, cudaStream_t
   p.block_size = a.block_size;
   p.partition_size = a.partition_size;
   p.num_partitions = a.num_partitions;
+  p.parts_per_cta = ppc;
   p.scale_log2 = a.scale * 1.4426950408889634f * a.k_scale;
   p.v_scale = a.v_scale;
-  dim3 grid(a.num_seqs, a.Hkv, a.num_partitions);
+  dim3 grid(a.num_seqs, a.Hkv, (a.num_partitions + p.parts_per_cta - 1) / p.parts_per_cta);
   return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk);
 }
 

@@ -67,6 +67,8 @@ int launch_decode_reduce(const DecodeArgs& a, unsigned int* status, void* stream
 // query heads per kv head, partition length a multiple of 128.
 bool decode_tc_supported(const DecodeArgs& a);
 int launch_decode_partitions_tc(const DecodeArgs& a, unsigned int* status, void* stream);
+// Consecutive partitions one CTA of a tensor-core decode kernel streams (1, 2 or 4).
+int tc_parts_per_cta(const DecodeArgs& a);
 // Tensor-core partition kernel over an E4M3 cache (decode_tc8.cu): f16/bf16
 // queries, head size 128, 4 or 8 query heads per kv head, partition length a
 // multiple of 128.

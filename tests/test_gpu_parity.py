@@ -583,10 +583,12 @@ def test_mq_bad_offsets_are_flagged_without_faulting():
 # grid has at least 8 CTAs per SM): every partition's partial must be right
 
 
+@pytest.mark.parametrize("fp8", [False, True])
 @pytest.mark.parametrize("P", [128, 256, 512])
-def test_tc_several_partitions_per_cta(P):
+def test_tc_several_partitions_per_cta(P, fp8):
     spec = W.Spec(f"ppc_{P}", "bf16", 32, 4, 128, 16, "independent", 320, seed=900 + P,
                   ctx_dist="uniform", ctx_lo=1, ctx_hi=2000, partition_size=P)
+    spec = W.fp8(spec) if fp8 else spec
     sc = W.scenario(spec)
     p, o = build(sc)
     out = run_step(p, spec)

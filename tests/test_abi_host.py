@@ -169,3 +169,44 @@ def test_fp8_calls_reject_bad_arguments(L):
     assert r(slots=FAKE + 4) == pk.PA_ERR_INVALID
     assert r(N=0) == pk.PA_OK
     assert pk.pa_launch_count() == before
+
+
+def test_multi_query_rejects_bad_arguments(L):
+    def mq(**kw):
+        a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, tables=FAKE, maxb=8, lens=FAKE, qs=FAKE, B=2,
+                 T=6, maxq=4, Hq=16, Hkv=2, D=128, bs=16, NB=100, scale=0.1, dtype=pk.PA_BF16,
+                 P=0, maxctx=100, ws=FAKE, wsb=1 << 30)
+        a.update(kw)
+        return L.pa_decode_multi(a["out"], a["q"], a["k"], a["v"], a["tables"], a["maxb"],
+                                 a["lens"], a["qs"], a["B"], a["T"], a["maxq"], a["Hq"], a["Hkv"],
+                                 a["D"], a["bs"], a["NB"], a["scale"], a["dtype"], a["P"],
+                                 a["maxctx"], a["ws"], a["wsb"], None)
+    before = pk.pa_launch_count()
+    cases = [
+        (dict(dtype=pk.PA_F32), pk.PA_ERR_UNSUPPORTED),
+        (dict(dtype=pk.PA_FP8_E4M3), pk.PA_ERR_UNSUPPORTED),
+        (dict(dtype=9), pk.PA_ERR_INVALID),
+        (dict(D=64), pk.PA_ERR_UNSUPPORTED),
+        (dict(Hq=24), pk.PA_ERR_UNSUPPORTED),
+        (dict(Hq=15), pk.PA_ERR_INVALID),
+        (dict(bs=64), pk.PA_ERR_UNSUPPORTED),
+        (dict(P=192), pk.PA_ERR_INVALID),          # not a multiple of 128
+        (dict(maxq=0), pk.PA_ERR_INVALID),
+        (dict(maxq=7), pk.PA_ERR_INVALID),         # above total_q
+        (dict(maxctx=8 * 16 + 1), pk.PA_ERR_INVALID),
+        (dict(qs=None), pk.PA_ERR_INVALID),
+        (dict(qs=FAKE + 2), pk.PA_ERR_INVALID),
+        (dict(q=FAKE + 8), pk.PA_ERR_INVALID),
+        # 1000 tokens over 256-token partitions need split-K partials
+        (dict(maxb=64, maxctx=1000, P=256, ws=None, wsb=0), pk.PA_ERR_INVALID),
+        (dict(maxb=64, maxctx=1000, P=256, wsb=64), pk.PA_ERR_INVALID),
+        (dict(scale=float("inf")), pk.PA_ERR_INVALID),
+    ]
+    for kw, want in cases:
+        assert mq(**kw) == want, kw
+        assert pk.pa_last_error()
+    assert mq(B=0) == pk.PA_OK and mq(T=0) == pk.PA_OK
+    assert pk.pa_launch_count() == before
+    assert pk.pa_decode_multi_workspace_bytes(6, 16, 128, 100, 0) == 0
+    assert pk.pa_decode_multi_workspace_bytes(6, 16, 128, 1000, 256) >= 6 * 16 * 4 * 130 * 4
+    assert pk.pa_decode_multi_workspace_bytes(6, 16, 128, 1000, 96) == 0   # invalid length

@@ -671,6 +671,8 @@ MQ_WORKLOADS = {
     # (spec, query tokens per sequence, description)
     "verify_gqa70b": (W.GQA70B, 4, "speculative verify: the gqa70b batch (256 seqs, Hq=64, Hkv=8, "
                       "D=128, bf16, context U[256,4096]) checking 4 proposed tokens per sequence"),
+    "verify2_gqa70b": (W.GQA70B, 2, "speculative verify: the gqa70b batch checking 2 proposed tokens "
+                       "per sequence (query tokens x heads = 16: the token-major decode kernel)"),
     "prefill_gqa70b": (None, 512, "chunked prefill: 16 sequences, Hq=64, Hkv=8, D=128, bf16, block "
                        "16, context U[2048,8192] whose last 512 tokens are the chunk"),
 }
@@ -784,7 +786,9 @@ def run_mq(args):
                    "kv_bytes_unique": unique, "flops": flops,
                    "l2": "L2 flushed between timed steps" if flush else "inputs larger than L2"},
         "tflops": round(tflops, 2), "kv_gbs": round(gbs, 2),
-        "roofline": {"kernel": "decode_mq_kernel (+ reduce)",
+        "roofline": {"kernel": ("decode_partition_tc_kernel, several queries (+ reduce)"
+                               if Q * spec.G <= 16 and spec.G in (4, 8)
+                               else "decode_mq_kernel (+ reduce)"),
                      "bound": "tensor" if tensor_bound else "hbm",
                      "achieved": round(tflops if tensor_bound else gbs, 2),
                      "peak": tc_peak if tensor_bound else hbm_peak,
@@ -916,7 +920,8 @@ def main():
                              "gqa70b_fp8", "gqa70b_quarter_fp8", "long_prefix_bs8_fp8",
                              "long_prefix_bs16_fp8", "long_prefix_bs32_fp8",
                              "long_prefix_bs16_quarter_fp8", "llama13b_ps_fp8", "tiny_fp8",
-                             "verify_gqa70b", "prefill_gqa70b", "verify_gqa70b_quarter",
+                             "verify_gqa70b", "verify2_gqa70b", "prefill_gqa70b",
+                             "verify_gqa70b_quarter",
                              "prefill_gqa70b_quarter"])
     ap.add_argument("--partition-size", type=int, default=0,
                     help="split-K partition length (0: the workload's own, 512)")

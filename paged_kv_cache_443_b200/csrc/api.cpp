@@ -558,7 +558,11 @@ extern "C" pa_status pa_decode_multi(void* out, const void* q, const void* k_cac
   a.dtype = dtype;
   unsigned int* status = pa::device_status_word();
   if (!status) return PA_ERR_CUDA;
-  pa_status st = launch_status(fn, pa::launch_decode_mq(a, status, stream), 1);
+  // few queries per sequence: token-major (tokens as the MMA's M, query tokens x
+  // heads as its N); else query-major, as a prefill kernel
+  const int err = pa::decode_mq_tc_supported(a) ? pa::launch_decode_mq_tc(a, status, stream)
+                                                : pa::launch_decode_mq(a, status, stream);
+  pa_status st = launch_status(fn, err, 1);
   if (st != PA_OK || NP <= 1) return st;
   return launch_status(fn, pa::launch_decode_mq_reduce(a, stream), 1);
 }

@@ -87,9 +87,16 @@ struct TcParams {
   int Hq, Hkv, num_blocks, block_size, partition_size, num_partitions;
   int parts_per_cta;  // consecutive partitions one CTA streams through
   float scale_log2;
+  // several query tokens per sequence (NQ > 1): q / out rows are tokens
+  const int32_t* query_start;
+  int total_q;
 };
 
-template <typename T, int G, bool MULTI>
+// NQ > 1 serves several query tokens per sequence (speculative verification):
+// column c of S / O is query token c / G (one of the sequence's last Qb <= NQ
+// context tokens) with head c % G, and a key counts for it only up to that
+// token's own position.  NQ = 1 is the decode step and compiles as before.
+template <typename T, int G, bool MULTI, int NQ = 1>
 __global__ void __launch_bounds__(THREADS, 2)
     decode_partition_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmap_k,
                                const __grid_constant__ CUtensorMap tmap_v) {
@@ -116,10 +123,22 @@ __global__ void __launch_bounds__(THREADS, 2)
   // short partitions do not each pay the pipeline's fill and drain.
   const int b = blockIdx.x, g = blockIdx.y, part = MULTI ? blockIdx.z * p.parts_per_cta : blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int NC = G * NQ;                // S / O columns in use
+  static_assert(NC <= NPAD, "query tokens x heads must fit the MMA's N");
 
   grid_dependency_wait();   // the appended tokens of the previous kernel are in the cache
   allow_dependents();       // the reduce kernel may start launching
   int L = p.context_lens[b];
+  int q0 = b, Qb = 1;       // first query token and query count of this sequence
+  if constexpr (NQ > 1) {
+    q0 = p.query_start[b];
+    Qb = p.query_start[b + 1] - q0;
+    if (Qb < 0 || Qb > NQ || Qb > L || q0 < 0 || q0 + Qb > p.total_q) {
+      if (threadIdx.x == 0 && blockIdx.z == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
+      return;
+    }
+    if (Qb == 0) return;
+  }
   const int P = p.partition_size;
   int64_t cap = p.max_blocks * p.block_size;
   const int64_t grid_cap = static_cast<int64_t>(p.num_partitions) * P;
@@ -130,7 +149,7 @@ __global__ void __launch_bounds__(THREADS, 2)
   }
   const int start = part * P;
   if (L == 0) {
-    if (part == 0) {
+    if (NQ == 1 && part == 0) {
       T* o = static_cast<T*>(p.out) + (static_cast<int64_t>(b) * p.Hq + g * G) * DH;
       for (int i = threadIdx.x; i < G * DH; i += THREADS) o[i] = Elem<T>::from_float(0.f);
     }
@@ -187,12 +206,15 @@ __global__ void __launch_bounds__(THREADS, 2)
     // Q^T operand (16 rows = heads, 128 columns = dims, two swizzled 64-column
     // blocks), rows >= G zero; both P buffers zeroed (their rows >= G stay 0).
     const int t = threadIdx.x - 64;
-    const T* qrow = static_cast<const T*>(p.q) + (static_cast<int64_t>(b) * p.Hq + g * G) * DH;
     for (int i = t; i < NPAD * (DH / 8); i += 128) {   // one 16-byte chunk each
-      const int h = i / (DH / 8);
+      const int h = i / (DH / 8);                      // column: query token h / G, head h % G
       const int c = i % (DH / 8);                      // chunk of 8 dims
       uint4 v = make_uint4(0, 0, 0, 0);
-      if (h < G) v = __ldg(reinterpret_cast<const uint4*>(qrow + h * DH + c * 8));
+      if (h < NC && h / G < Qb) {
+        const T* qrow = static_cast<const T*>(p.q) +
+                        ((static_cast<int64_t>(q0) + h / G) * p.Hq + g * G + h % G) * DH;
+        v = __ldg(reinterpret_cast<const uint4*>(qrow + c * 8));
+      }
       const uint32_t off = (c / 8) * (NPAD * 128) + sw128(h, (c % 8) * 8);
       *reinterpret_cast<uint4*>(qop + off) = v;
     }
@@ -299,9 +321,9 @@ __global__ void __launch_bounds__(THREADS, 2)
     const int quad = warp & 3;                 // TMEM lane quadrant of this warp
     const int r = quad * 32 + lane;            // token row of the tile / dim row of O
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    float m_run[G], l_part[G];
+    float m_run[NC], l_part[NC];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
+    for (int h = 0; h < NC; ++h) {
       m_run[h] = -INFINITY;
       l_part[h] = 0.f;
     }
@@ -325,7 +347,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       __syncwarp();
       if (MULTI && lane == 0) mbar_arrive(o_free);              // the next partition may reuse O
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
+      for (int h = 0; h < NC; ++h) {
         float x = l_part[h];
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(FULL, x, off);
@@ -334,14 +356,15 @@ __global__ void __launch_bounds__(THREADS, 2)
       named_sync(1, 128);
       if (lane == 0) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) red[quad * NPAD + h] = l_part[h];
+        for (int h = 0; h < NC; ++h) red[quad * NPAD + h] = l_part[h];
       }
       named_sync(1, 128);
       if (ok) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
+        for (int h = 0; h < NC; ++h) {
           const float Ls = red[h] + red[NPAD + h] + red[2 * NPAD + h] + red[3 * NPAD + h];
-          const int64_t hq = static_cast<int64_t>(b) * p.Hq + g * G + h;
+          const int64_t hq = (static_cast<int64_t>(q0) + h / G) * p.Hq + g * G + h % G;
+          if (NQ > 1 && h / G >= Qb) continue;
           if (single) {
             static_cast<T*>(p.out)[hq * DH + r] = Elem<T>::from_float(o[h] / Ls);
           } else {
@@ -361,7 +384,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       const bool first = (i % tpp) == 0;
       if (MULTI && first && i > 0) {                            // a new partition: a new softmax
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
+        for (int h = 0; h < NC; ++h) {
           m_run[h] = -INFINITY;
           l_part[h] = 0.f;
         }
@@ -377,26 +400,29 @@ __global__ void __launch_bounds__(THREADS, 2)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[i & 1]);
-      float s[G];
+      float s[NC];
       bool need = false;
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        s[h] = valid ? sv[h] * p.scale_log2 : -INFINITY;
+      for (int h = 0; h < NC; ++h) {
+        bool ok_h = valid;
+        if constexpr (NQ > 1)   // causal: up to query token h / G's own position
+          ok_h = ok_h && h / G < Qb && start + i * TOK + r <= L - Qb + h / G;
+        s[h] = ok_h ? sv[h] * p.scale_log2 : -INFINITY;
         need |= s[h] > m_run[h] + RESCALE_THRESHOLD;
       }
       if (bar_or(1, 128, need)) {
         // raise the running max to this tile's max (all 128 threads agree)
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
+        for (int h = 0; h < NC; ++h) {
           float x = s[h];
 #pragma unroll
           for (int off = 16; off >= 1; off >>= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, off));
           if (lane == 0) red[quad * NPAD + h] = x;
         }
         named_sync(1, 128);
-        float alpha[G];
+        float alpha[NC];
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
+        for (int h = 0; h < NC; ++h) {
           const float tmax =
               fmaxf(fmaxf(red[h], red[NPAD + h]), fmaxf(red[2 * NPAD + h], red[3 * NPAD + h]));
           const float mnew = fmaxf(m_run[h], tmax);
@@ -412,20 +438,21 @@ __global__ void __launch_bounds__(THREADS, 2)
           float o[16];
           tmem_ld16(tmem + lane_base + 2 * NPAD, o);
 #pragma unroll
-          for (int h = 0; h < G; ++h) o[h] *= alpha[h];
+          for (int h = 0; h < NC; ++h) o[h] *= alpha[h];
           tmem_st16(tmem + lane_base + 2 * NPAD, o);
         }
       }
-      float pr[G];
+      float pr[NC];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        pr[h] = valid ? exp2f(s[h] - m_run[h]) : 0.f;
+      for (int h = 0; h < NC; ++h) {
+        const bool counted = NQ > 1 ? s[h] != -INFINITY : valid;
+        pr[h] = counted ? exp2f(s[h] - m_run[h]) : 0.f;
         l_part[h] += pr[h];
       }
       if (i >= 2) wait(&p_free[i & 1], ((i >> 1) - 1) & 1);
       uint8_t* pb = pop + (i & 1) * OPB_BYTES + (r >> 6) * (NPAD * 128);
 #pragma unroll
-      for (int h = 0; h < G; ++h)
+      for (int h = 0; h < NC; ++h)
         *reinterpret_cast<uint16_t*>(pb + sw128(h, r & 63)) = to_bits<T>(pr[h]);
       if (n_valid < TOK) {
         // the last tile: zero the V rows of tokens past the end, so that
@@ -499,6 +526,8 @@ cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t 
   p.num_partitions = a.num_partitions;
   p.parts_per_cta = ppc;
   p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.query_start = nullptr;
+  p.total_q = a.num_seqs;
   dim3 grid(a.num_seqs, a.Hkv, (a.num_partitions + p.parts_per_cta - 1) / p.parts_per_cta);
   return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
 }
@@ -563,6 +592,77 @@ bool make_tmap(void* map, const void* base, int rank, const int64_t* dims,
 }
 
 bool tmap_available() { return encode_fn() != nullptr; }
+
+namespace {
+
+template <typename T, int G, int NQ>
+cudaError_t launch_tcq_t(const MqArgs& m, unsigned int* status, cudaStream_t stream) {
+  DecodeArgs a{};
+  a.num_seqs = m.num_seqs;
+  a.Hkv = m.Hkv;
+  a.partition_size = m.partition_size;
+  a.num_partitions = m.num_partitions;
+  const int ppc = tc_parts_per_cta(a);
+  auto kern = ppc > 1 ? decode_partition_tc_kernel<T, G, true, NQ>
+                      : decode_partition_tc_kernel<T, G, false, NQ>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  CUtensorMap mk, mv;
+  const int64_t groups = static_cast<int64_t>(m.num_blocks) * m.Hkv * m.block_size / 8;
+  const int64_t dims[4] = {64, 8, 2, groups};
+  const int64_t strides[3] = {DH * 2, 128, 8 * DH * 2};
+  const int box[4] = {64, 8, 2, m.block_size / 8};
+  if (!make_tmap(&mk, m.k_cache, 4, dims, strides, box, m.dtype) ||
+      !make_tmap(&mv, m.v_cache, 4, dims, strides, box, m.dtype))
+    return cudaErrorInvalidValue;
+  TcParams p;
+  p.out = m.out;
+  p.q = m.q;
+  p.block_tables = m.block_tables;
+  p.context_lens = m.context_lens;
+  const int64_t nrows = static_cast<int64_t>(m.total_q) * m.Hq * m.num_partitions;
+  p.ws_o = m.workspace;
+  p.ws_m = m.workspace ? m.workspace + nrows * DH : nullptr;
+  p.ws_l = m.workspace ? m.workspace + nrows * (DH + 1) : nullptr;
+  p.status = status;
+  p.max_blocks = m.max_blocks;
+  p.Hq = m.Hq;
+  p.Hkv = m.Hkv;
+  p.num_blocks = m.num_blocks;
+  p.block_size = m.block_size;
+  p.partition_size = m.partition_size;
+  p.num_partitions = m.num_partitions;
+  p.parts_per_cta = ppc;
+  p.scale_log2 = m.scale * 1.4426950408889634f;
+  p.query_start = m.query_start;
+  p.total_q = m.total_q;
+  dim3 grid(m.num_seqs, m.Hkv, (m.num_partitions + ppc - 1) / ppc);
+  return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
+}
+
+template <typename T>
+cudaError_t launch_tcq_g(const MqArgs& m, unsigned int* status, cudaStream_t stream) {
+  const int G = m.Hq / m.Hkv;
+  const int nq = m.max_query_len <= 2 ? 2 : 4;
+  if (G == 8) return launch_tcq_t<T, 8, 2>(m, status, stream);
+  return nq == 2 ? launch_tcq_t<T, 4, 2>(m, status, stream) : launch_tcq_t<T, 4, 4>(m, status, stream);
+}
+
+}  // namespace
+
+bool decode_mq_tc_supported(const MqArgs& m) {
+  const int G = m.Hkv > 0 ? m.Hq / m.Hkv : 0;
+  return (m.dtype == PA_F16 || m.dtype == PA_BF16) && m.D == DH && (G == 4 || G == 8) &&
+         m.max_query_len >= 1 && m.max_query_len * G <= NPAD && m.partition_size % TOK == 0 &&
+         static_cast<int64_t>(m.num_blocks) * m.Hkv * m.block_size < (int64_t(1) << 31) &&
+         encode_fn() != nullptr;
+}
+
+int launch_decode_mq_tc(const MqArgs& m, unsigned int* status, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return m.dtype == PA_BF16 ? launch_tcq_g<__nv_bfloat16>(m, status, st)
+                            : launch_tcq_g<__half>(m, status, st);
+}
 
 bool decode_tc_supported(const DecodeArgs& a) {
   const int G = a.Hq / a.Hkv;

@@ -603,3 +603,19 @@ def test_tc_several_partitions_per_cta(P, fp8):
     out2 = run_step(p, spec, partition_size=4096)
     torch.cuda.synchronize()
     assert np.abs(as_f64(out2, spec) - got_all).max() <= TOL[spec.dtype]
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("G", [4, 8])
+@pytest.mark.parametrize("P", [128, 512])
+def test_mq_few_queries_token_major(dtype, G, P):
+    """Q * G <= 16 takes the decode kernel with per-column causal limits."""
+    spec = mq_spec(dtype, G, 16, (5, 40, 300, 513, 1100, 2000, 1, 2), seed=950 + G + P)
+    qlens = (1, 4, 2, 3, 4, 1, 1, 2) if G == 4 else (1, 2, 2, 1, 2, 2, 1, 2)
+    mq_check(spec, qlens, partition_size=P)
+
+
+def test_mq_few_queries_several_partitions_per_cta():
+    spec = W.Spec("mq_ppc", "bf16", 32, 4, 128, 16, "independent", 320, seed=977,
+                  ctx_dist="uniform", ctx_lo=2, ctx_hi=2000, partition_size=128)
+    mq_check(spec, [1 + (i % 4) for i in range(320)], partition_size=128)

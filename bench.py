@@ -787,7 +787,7 @@ def run_mq(args):
                    "l2": "L2 flushed between timed steps" if flush else "inputs larger than L2"},
         "tflops": round(tflops, 2), "kv_gbs": round(gbs, 2),
         "roofline": {"kernel": ("decode_partition_tc_kernel, several queries (+ reduce)"
-                               if Q * spec.G <= 16 and spec.G in (4, 8)
+                               if Q * spec.G <= 64 and spec.G in (4, 8)
                                else "decode_mq_kernel (+ reduce)"),
                      "bound": "tensor" if tensor_bound else "hbm",
                      "achieved": round(tflops if tensor_bound else gbs, 2),

@@ -87,9 +87,11 @@ struct TcParams {
   int Hq, Hkv, num_blocks, block_size, partition_size, num_partitions;
   int parts_per_cta;  // consecutive partitions one CTA streams through
   float scale_log2;
-  // several query tokens per sequence (NQ > 1): q / out rows are tokens
+  // several query tokens per sequence (NQ > 1): q / out rows are tokens; a
+  // sequence's queries are served in groups of NQ by q_groups adjacent CTAs
   const int32_t* query_start;
   int total_q;
+  int q_groups;
 };
 
 // NQ > 1 serves several query tokens per sequence (speculative verification):
@@ -121,7 +123,8 @@ __global__ void __launch_bounds__(THREADS, 2)
   // A CTA streams parts_per_cta consecutive partitions (tiles never straddle
   // one: P is a multiple of TOK) and writes each one's partial as it ends, so
   // short partitions do not each pay the pipeline's fill and drain.
-  const int b = blockIdx.x, g = blockIdx.y, part = MULTI ? blockIdx.z * p.parts_per_cta : blockIdx.z;
+  const int b = NQ > 1 ? blockIdx.x / p.q_groups : blockIdx.x;
+  const int g = blockIdx.y, part = MULTI ? blockIdx.z * p.parts_per_cta : blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int NC = G * NQ;                // S / O columns in use
   static_assert(NC <= NPAD, "query tokens x heads must fit the MMA's N");
@@ -129,15 +132,21 @@ __global__ void __launch_bounds__(THREADS, 2)
   grid_dependency_wait();   // the appended tokens of the previous kernel are in the cache
   allow_dependents();       // the reduce kernel may start launching
   int L = p.context_lens[b];
-  int q0 = b, Qb = 1;       // first query token and query count of this sequence
+  // this CTA's query tokens: q0 .. q0 + Qb - 1, at positions L - Qall + qoff + c / G
+  int q0 = b, Qb = 1, Qall = 1, qoff = 0;
   if constexpr (NQ > 1) {
-    q0 = p.query_start[b];
-    Qb = p.query_start[b + 1] - q0;
-    if (Qb < 0 || Qb > NQ || Qb > L || q0 < 0 || q0 + Qb > p.total_q) {
-      if (threadIdx.x == 0 && blockIdx.z == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
+    const int qg = blockIdx.x % p.q_groups;
+    const int qs = p.query_start[b];
+    Qall = p.query_start[b + 1] - qs;
+    if (Qall < 0 || Qall > L || Qall > NQ * p.q_groups || qs < 0 || qs + Qall > p.total_q) {
+      if (threadIdx.x == 0 && blockIdx.z == 0 && g == 0 && qg == 0)
+        atomicOr(p.status, PA_DEVERR_CONTEXT);
       return;
     }
-    if (Qb == 0) return;
+    qoff = qg * NQ;
+    q0 = qs + qoff;
+    Qb = min(NQ, Qall - qoff);
+    if (Qb <= 0) return;
   }
   const int P = p.partition_size;
   int64_t cap = p.max_blocks * p.block_size;
@@ -406,7 +415,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       for (int h = 0; h < NC; ++h) {
         bool ok_h = valid;
         if constexpr (NQ > 1)   // causal: up to query token h / G's own position
-          ok_h = ok_h && h / G < Qb && start + i * TOK + r <= L - Qb + h / G;
+          ok_h = ok_h && h / G < Qb && start + i * TOK + r <= L - Qall + qoff + h / G;
         s[h] = ok_h ? sv[h] * p.scale_log2 : -INFINITY;
         need |= s[h] > m_run[h] + RESCALE_THRESHOLD;
       }
@@ -528,6 +537,7 @@ cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t 
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.query_start = nullptr;
   p.total_q = a.num_seqs;
+  p.q_groups = 1;
   dim3 grid(a.num_seqs, a.Hkv, (a.num_partitions + p.parts_per_cta - 1) / p.parts_per_cta);
   return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
 }
@@ -636,24 +646,26 @@ cudaError_t launch_tcq_t(const MqArgs& m, unsigned int* status, cudaStream_t str
   p.scale_log2 = m.scale * 1.4426950408889634f;
   p.query_start = m.query_start;
   p.total_q = m.total_q;
-  dim3 grid(m.num_seqs, m.Hkv, (m.num_partitions + ppc - 1) / ppc);
+  p.q_groups = (m.max_query_len + NQ - 1) / NQ;
+  dim3 grid(m.num_seqs * p.q_groups, m.Hkv, (m.num_partitions + ppc - 1) / ppc);
   return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
 }
 
 template <typename T>
 cudaError_t launch_tcq_g(const MqArgs& m, unsigned int* status, cudaStream_t stream) {
   const int G = m.Hq / m.Hkv;
-  const int nq = m.max_query_len <= 2 ? 2 : 4;
   if (G == 8) return launch_tcq_t<T, 8, 2>(m, status, stream);
-  return nq == 2 ? launch_tcq_t<T, 4, 2>(m, status, stream) : launch_tcq_t<T, 4, 4>(m, status, stream);
+  return m.max_query_len <= 2 ? launch_tcq_t<T, 4, 2>(m, status, stream)
+                              : launch_tcq_t<T, 4, 4>(m, status, stream);
 }
 
 }  // namespace
 
 bool decode_mq_tc_supported(const MqArgs& m) {
   const int G = m.Hkv > 0 ? m.Hq / m.Hkv : 0;
+  // up to 4 groups of 16 / G query tokens; longer query runs are prefill-like
   return (m.dtype == PA_F16 || m.dtype == PA_BF16) && m.D == DH && (G == 4 || G == 8) &&
-         m.max_query_len >= 1 && m.max_query_len * G <= NPAD && m.partition_size % TOK == 0 &&
+         m.max_query_len >= 1 && m.max_query_len * G <= 4 * NPAD && m.partition_size % TOK == 0 &&
          static_cast<int64_t>(m.num_blocks) * m.Hkv * m.block_size < (int64_t(1) << 31) &&
          encode_fn() != nullptr;
 }

@@ -100,8 +100,9 @@ struct MqArgs {
 };
 constexpr int kMqRows = 128;  // (query token, head) rows per CTA of the multi-query kernel
 int launch_decode_mq(const MqArgs& a, unsigned int* status, void* stream);
-// Few query tokens per sequence (max_query_len * G <= 16, G = 4 or 8): the
-// token-major tcgen05 decode kernel with per-column causal limits (decode_tc.cu).
+// Few query tokens per sequence (max_query_len * G <= 64, G = 4 or 8): the
+// token-major tcgen05 decode kernel with per-column causal limits, 16 / G query
+// tokens per CTA (decode_tc.cu).
 bool decode_mq_tc_supported(const MqArgs& a);
 int launch_decode_mq_tc(const MqArgs& a, unsigned int* status, void* stream);
 int launch_decode_mq_reduce(const MqArgs& a, void* stream);

@@ -442,8 +442,8 @@ def run_ours(args):
     out = torch.empty_like(q)
     P = args.partition_size if args.partition_size else spec.partition_size
     if P == 0:   # the workload leaves it to the library: use pa_decode's automatic length
-        P = pk.pa_decode_auto_partition_size(len(sc.batch), spec.Hq, spec.Hkv, spec.D,
-                                             spec.dtype_code, max_ctx)
+        auto = pk.pa_decode_fp8_auto_partition_size if spec.fp8 else pk.pa_decode_auto_partition_size
+        P = auto(len(sc.batch), spec.Hq, spec.Hkv, spec.D, spec.dtype_code, max_ctx)
     ws = cache.workspace(q.shape[0], q.shape[1], max_ctx, P)
     scale = spec.softmax_scale
     n_part = pk.pa_decode_num_partitions(max_ctx, P)

@@ -132,6 +132,16 @@ int pa_decode_auto_partition_size(int num_seqs, int num_heads, int num_kv_heads,
                                   pa_dtype dtype, int max_context_len);
 
 /*
+ * The partition length pa_decode_fp8 uses when it is given partition_size = 0:
+ * as pa_decode_auto_partition_size (dtype is the queries' type, f32, f16 or
+ * bf16), with 4096 among the candidates (4096 / 2048 / 1024) when the
+ * tensor-core kernel serves the launch, since an E4M3 tile is half the bytes.
+ * Returns -1 for invalid arguments (PA_FP8_E4M3 as dtype included).
+ */
+int pa_decode_fp8_auto_partition_size(int num_seqs, int num_heads, int num_kv_heads,
+                                      int head_size, pa_dtype dtype, int max_context_len);
+
+/*
  * Number of split-K partitions per sequence for a batch whose longest context
  * is max_context_len: ceil(max_context_len / P), P = the partition size (0 =
  * default).  Returns -1 for an invalid partition size.

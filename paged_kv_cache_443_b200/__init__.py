@@ -29,6 +29,7 @@ EXPORTS = (
     "pa_last_error", "pa_version", "pa_launch_count", "pa_device_status",
     "pa_selftest_wait_timeout",
     "pa_decode_default_partition_size", "pa_decode_auto_partition_size",
+    "pa_decode_fp8_auto_partition_size",
     "pa_decode_num_partitions", "pa_decode_workspace_bytes",
     "pa_decode", "pa_decode_partitions", "pa_decode_reduce", "pa_decode_noalloc",
     "pa_reshape_and_cache", "pa_reshape_and_cache_fp8", "pa_decode_fp8",
@@ -76,6 +77,7 @@ def lib():
         "pa_selftest_wait_timeout": ([ctypes.POINTER(ctypes.c_uint)], i32),
         "pa_decode_default_partition_size": ([], i32),
         "pa_decode_auto_partition_size": ([i32, i32, i32, i32, i32, i32], i32),
+        "pa_decode_fp8_auto_partition_size": ([i32, i32, i32, i32, i32, i32], i32),
         "pa_decode_num_partitions": ([i32, i32], i32),
         "pa_decode_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
         "pa_decode": ([vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, f32, i32, i32,
@@ -192,6 +194,14 @@ def pa_decode_auto_partition_size(num_seqs: int, num_heads: int, num_kv_heads: i
     """The partition length pa_decode picks for partition_size = 0 (dtype: PA_*)."""
     return int(lib().pa_decode_auto_partition_size(num_seqs, num_heads, num_kv_heads, head_size,
                                                    dtype, max_context_len))
+
+
+def pa_decode_fp8_auto_partition_size(num_seqs: int, num_heads: int, num_kv_heads: int,
+                                      head_size: int, dtype: int, max_context_len: int) -> int:
+    """The partition length pa_decode_fp8 picks for partition_size = 0 (dtype:
+    the queries' PA_* type)."""
+    return int(lib().pa_decode_fp8_auto_partition_size(num_seqs, num_heads, num_kv_heads,
+                                                       head_size, dtype, max_context_len))
 
 
 def pa_decode_num_partitions(max_context_len: int, partition_size: int = 0) -> int:

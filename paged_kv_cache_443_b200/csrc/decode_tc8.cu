@@ -1,39 +1,43 @@
 // decode_tc8.cu -- paged decode attention on the tensor cores over an E4M3 KV
-// cache, for grouped-query heads (G = Hq/Hkv in {4, 8}), head size 128, f16 or
-// bf16 queries and outputs.
+// cache, head size 128, f16 or bf16 queries and outputs, G = Hq/Hkv query
+// heads per kv head 4 or 8 (the code holds for 1 and 2 as well, where the
+// CUDA-core kernel of decode.cu is the faster one).
 //
 // What is computed is that of decode_tc.cu ("자기회귀 생성과 KV 캐시" and
 // "PagedAttention의 설계", supersilo.blog vLLM summary), with the cache's
 // elements standing for code * k_scale and code * v_scale (E4M3 codes: the
 // reading of "quantization" in "4. 이 밖의 기법들", blog.aqudi.me).  Tokens are
-// the MMA's M dimension:
+// the MMA's M dimension for S and the reduction dimension for O; both products
+// run on kind::f8f6f4 with the cache codes as they are in shared memory:
 //
-//   S^T [128 tokens x 16] = K [128 x 128] . Q^T [128 x 16]     kind::f8f6f4
-//   O^T [128 dims   x 16] += V^T [128 x 128] . P^T [128 x 16]   kind::f16
+//   S^T [128 tokens x 16] = K [128 x 128] . Q^T [128 x 16]         K-major K
+//   O^T [128 dims   x 16] += V^T [128 x 128] . P^T [128 x 16]      MN-major V^T
 //
-// * S: the K codes feed the tensor cores as they are, K-major, straight from
-//   a TMA load per physical block (rows of 128 codes, 128-byte swizzle).  The
-//   query is split into three E4M3 terms, Q * 2^e = Q1 + Q2 + Q3 (each the
-//   nearest E4M3 value of what the previous terms left; e a per-head power of
-//   two putting the head's largest |q| in [2^7, 2^8)), and S accumulates the
-//   three products.  An f16 or bf16 query has at most 11 significant bits, and
-//   each term takes the next 4, so the split is exact for every component at
-//   least 2^-6 of the head's largest (smaller ones are off by under 2^-10 in
-//   the scaled units); 2^-e and k_scale are folded into the softmax scale.
-// * O: P keeps f16's range (the lazily raised running max can leave P far
-//   below E4M3's smallest value), so V is widened to f16 (exact: every E4M3
-//   value is an f16 value) by converter warps into the MN-major layout of V^T;
-//   v_scale is applied to the output.
+// * Q: split into three E4M3 terms, Q * 2^e = Q1 + Q2 + Q3 (each the nearest
+//   E4M3 value of what the previous terms left; e a per-head power of two
+//   putting the head's largest |q| in [2^7, 2^8)), and S accumulates the three
+//   products.  An f16 or bf16 query has at most 11 significant bits, and each
+//   term takes the next 4, so the split is exact for every component at least
+//   2^-6 of the head's largest; 2^-e and k_scale are folded into the softmax
+//   scale.
+// * P: the running max is raised as soon as a score passes it by 2 (base 2),
+//   so P <= 4; P * 2^6 (<= 256, inside E4M3's range) is split into two E4M3
+//   terms the same way, P1 + P2, which keeps P to about 2^-8 of its value for
+//   P >= 2^-12 (and to 2^-16 absolutely below that).  The partial sums l add
+//   the fp32 P; 2^-6 and v_scale are applied to O.
+// * Each physical block's K and V codes arrive in one TMA load each, rows of
+//   128 codes stored with the 128-byte swizzle: the canonical K-major layout of
+//   K and, unchanged, the MN-major layout of V^T (8-token groups 1 KB apart).
 //
-// Roles in a CTA of 10 warps, one CTA per (sequence, kv head, partition):
+// Roles in a CTA of 6 warps, one CTA per (sequence, kv head, partition):
 //   warp 0     producer: block-table lookups; per tile one TMA load per block
-//              of its K codes into a ring of three 16 KB tiles, and one 1-D bulk
-//              copy per block of its V codes into a ring of two 8 KB slots;
+//              of its K codes and one of its V codes into two rings of three
+//              16 KB tiles;
 //   warp 1     TMEM owner and MMA issuer;
-//   warps 2-5  query terms, then softmax (as in decode_tc.cu), P as f16;
-//   warps 6-9  converters: a tile's V codes into registers (the slots go back
-//              at once), then the f16 V^T tile, zeros for tokens past the end.
-// About 111 KB of shared memory: two CTAs per SM.  Every wait is bounded;
+//   warps 2-5  query terms, then softmax (as in decode_tc.cu), P as two E4M3
+//              terms; they zero the V rows of tokens past the end of a final
+//              tile.
+// About 113 KB of shared memory: two CTAs per SM.  Every wait is bounded;
 // block ids outside the pool are skipped and flagged.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -56,41 +60,39 @@ constexpr int TOK = 128;                    // tokens per tile
 constexpr int NPAD = 16;                    // MMA N (heads padded)
 constexpr int DH = 128;                     // head size
 constexpr int NTERM = 3;                    // E4M3 terms of the query
-constexpr int KR_SLOTS = 3;
-constexpr int KR_BYTES = TOK * DH;          // one tile of K codes: 16 KB
-constexpr int HALF_TOK = 64;                // tokens per V staging slot
-constexpr int ST_SLOTS = 2;
-constexpr int ST_BYTES = HALF_TOK * DH;     // 8 KB of V codes
-constexpr int VOP_BYTES = TOK * DH * 2;     // the f16 V^T tile: 32 KB
-constexpr int GROUP_BYTES = 2048;           // f16 tile: 8 token rows, both 64-column halves
-constexpr int HALF_OFF = 1024;
+constexpr int PTERM = 2;                    // E4M3 terms of P
+constexpr int SLOTS = 3;                    // tiles per ring (one ring for K, one for V)
+constexpr int TILE_BYTES = TOK * DH;        // one tile of codes: 16 KB
 constexpr int QT_BYTES = NPAD * DH;         // one query term: 16 rows x 128 codes
-constexpr int OPB_BYTES = 2 * NPAD * 128;   // f16 16-row operand (P): 4 KB
+constexpr int PT_BYTES = NPAD * TOK;        // one P term: 16 rows x 128 tokens
+constexpr int PB_BYTES = PTERM * PT_BYTES;  // one P buffer (both terms)
 constexpr int OFF_KR = 0;
-constexpr int OFF_VOP = OFF_KR + KR_SLOTS * KR_BYTES;
-constexpr int OFF_ST = OFF_VOP + VOP_BYTES;
-constexpr int OFF_Q = OFF_ST + ST_SLOTS * ST_BYTES;
+constexpr int OFF_VR = OFF_KR + SLOTS * TILE_BYTES;
+constexpr int OFF_Q = OFF_VR + SLOTS * TILE_BYTES;
 constexpr int OFF_P = OFF_Q + NTERM * QT_BYTES;   // two P buffers
-constexpr int OFF_BAR = OFF_P + 2 * OPB_BYTES;
-constexpr int NBARS = 2 * KR_SLOTS + 2 * ST_SLOTS + 2 + 8 + 2;
+constexpr int OFF_BAR = OFF_P + 2 * PB_BYTES;
+constexpr int NBARS = 4 * SLOTS + 8 + 2;
 constexpr int OFF_TMEM = (OFF_BAR + NBARS * 8 + 15) / 16 * 16;
 constexpr int OFF_RED = OFF_TMEM + 16;      // 4 warps x 16 floats
 constexpr int OFF_QS = OFF_RED + 4 * NPAD * 4;
 constexpr int SMEM_USED = OFF_QS + NPAD * 4;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;
-constexpr int THREADS = 320;
+constexpr int THREADS = 192;
 constexpr int TMEM_COLS = 64;               // S0 [0,16), S1 [16,32), O [32,48)
-constexpr float RESCALE_THRESHOLD = 8.0f;
+constexpr float RESCALE_THRESHOLD = 2.0f;   // P <= 2^2
+constexpr float P_UP = 64.0f;               // P * 2^6 <= 256 < 448
+constexpr float P_DOWN = 1.0f / 64.0f;
 
 static_assert(SMEM_BYTES * 2 + 2048 <= 228 * 1024, "two CTAs per SM");
-static_assert(OFF_VOP % 1024 == 0 && OFF_Q % 1024 == 0 && OFF_P % 1024 == 0 &&
-                  QT_BYTES % 1024 == 0,
+static_assert(OFF_VR % 1024 == 0 && OFF_Q % 1024 == 0 && OFF_P % 1024 == 0 &&
+                  QT_BYTES % 1024 == 0 && PT_BYTES % 1024 == 0,
               "swizzled operands on 1 KB boundaries");
 
 // Instruction descriptor of kind::f8f6f4: E4M3 x E4M3 (format 0 for both),
-// fp32 accumulation, both operands K-major, M = 128, N = 16.
+// fp32 accumulation, M = 128, N = 16; A K-major (S) or MN-major (O), B K-major.
 constexpr uint32_t kIdescE4M3 = (1u << 4) | (static_cast<uint32_t>(NPAD >> 3) << 17) |
                                 (static_cast<uint32_t>(128 >> 4) << 24);
+constexpr uint32_t kIdescE4M3_AMN = kIdescE4M3 | (1u << 15);
 
 __device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
                                          uint32_t accumulate) {
@@ -104,7 +106,6 @@ __device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t a, uint64_t b
 struct Tc8Params {
   void* out;
   const void* q;
-  const uint8_t* v_cache;
   const int32_t* block_tables;
   const int32_t* context_lens;
   float* ws_o;
@@ -127,13 +128,6 @@ __device__ __forceinline__ void widen4(uint32_t w, uint32_t& lo, uint32_t& hi) {
       : "r"(w));
 }
 
-__device__ __forceinline__ void widen16(const uint4& c, uint4& lo, uint4& hi) {
-  widen4(c.x, lo.x, lo.y);
-  widen4(c.y, lo.z, lo.w);
-  widen4(c.z, hi.x, hi.y);
-  widen4(c.w, hi.z, hi.w);
-}
-
 // Nearest E4M3 codes of two floats (saturating; the first in the low byte).
 __device__ __forceinline__ uint32_t to_e4m3x2(float a, float b) {
   return static_cast<uint32_t>(
@@ -148,23 +142,21 @@ __device__ __forceinline__ float2 from_e4m3x2(uint32_t c) {
 
 template <typename T, int G, bool MULTI>
 __global__ void __launch_bounds__(THREADS, 2)
-    decode_partition_tc8_kernel(const Tc8Params p, const __grid_constant__ CUtensorMap tmap_k) {
+    decode_partition_tc8_kernel(const Tc8Params p, const __grid_constant__ CUtensorMap tmap_k,
+                                const __grid_constant__ CUtensorMap tmap_v) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* kring = smem + OFF_KR;
-  uint8_t* vop = smem + OFF_VOP;
-  uint8_t* stage = smem + OFF_ST;
+  uint8_t* vring = smem + OFF_VR;
   uint8_t* qop = smem + OFF_Q;
   uint8_t* pop = smem + OFF_P;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* kr_full = bars;                  // [KR_SLOTS]
-  uint64_t* kr_empty = kr_full + KR_SLOTS;   // [KR_SLOTS]
-  uint64_t* st_full = kr_empty + KR_SLOTS;   // [ST_SLOTS]
-  uint64_t* st_empty = st_full + ST_SLOTS;   // [ST_SLOTS]
-  uint64_t* vop_full = st_empty + ST_SLOTS;
-  uint64_t* vop_empty = vop_full + 1;
-  uint64_t* s_full = vop_empty + 1;          // [2]
+  uint64_t* kr_full = bars;                  // [SLOTS]
+  uint64_t* kr_empty = kr_full + SLOTS;      // [SLOTS]
+  uint64_t* vr_full = kr_empty + SLOTS;      // [SLOTS]
+  uint64_t* vr_empty = vr_full + SLOTS;      // [SLOTS]
+  uint64_t* s_full = vr_empty + SLOTS;       // [2]
   uint64_t* s_free = s_full + 2;             // [2]
   uint64_t* p_full = s_free + 2;             // [2]
   uint64_t* p_free = p_full + 2;             // [2]
@@ -210,16 +202,12 @@ __global__ void __launch_bounds__(THREADS, 2)
   const int last_blk = (end + bs - 1) / bs;
   const int32_t* trow = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < KR_SLOTS; ++s) {
+    for (int s = 0; s < SLOTS; ++s) {
       mbar_init(&kr_full[s], 1);
       mbar_init(&kr_empty[s], 1);
+      mbar_init(&vr_full[s], 1);
+      mbar_init(&vr_empty[s], 1);
     }
-    for (int s = 0; s < ST_SLOTS; ++s) {
-      mbar_init(&st_full[s], 1);
-      mbar_init(&st_empty[s], 4);
-    }
-    mbar_init(vop_full, 4);
-    mbar_init(vop_empty, 1);
     for (int j = 0; j < 2; ++j) {
       mbar_init(&s_full[j], 1);
       mbar_init(&s_free[j], 4);
@@ -230,6 +218,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     mbar_init(o_free, 4);
     fence_mbar_init();
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -246,18 +235,15 @@ __global__ void __launch_bounds__(THREADS, 2)
   if (warp == 0) {
     // ================= producer =================
     const uint32_t blk_bytes = static_cast<uint32_t>(bs) * DH;       // one (block, head) run
-    const int64_t blk_stride = static_cast<int64_t>(p.Hkv) * blk_bytes;
-    const uint8_t* vbase = p.v_cache + static_cast<int64_t>(g) * blk_bytes;
     const int bpt = TOK / bs;                 // blocks per tile (4, 8 or 16)
-    const int bph = HALF_TOK / bs;            // blocks per V staging slot (2, 4 or 8)
     bool ok = true;
-    int k_issued = 0, v_issued = 0;
+    int issued = 0;                           // tiles whose K and V loads are out
     auto table = [&](int i) {                 // lane j: block j of tile i (read one tile ahead)
       const int b0 = first_blk + i * bpt;
       return (i < n_tiles && lane < min(bpt, last_blk - b0)) ? __ldg(trow + b0 + lane) : -1;
     };
     int pb_next = table(0);
-    for (int i = 0; i < n_tiles && ok; ++i) {
+    for (int i = 0; i < n_tiles; ++i) {
       const int b0 = first_blk + i * bpt;
       const int pb_l = pb_next;
       pb_next = table(i + 1);
@@ -265,98 +251,32 @@ __global__ void __launch_bounds__(THREADS, 2)
       const bool mine_t = lane < nbt;
       const bool valid_t = mine_t && pb_l >= 0 && pb_l < p.num_blocks;
       if (mine_t && !valid_t) atomicOr(p.status, PA_DEVERR_TABLE);
-      // K: the tile's blocks straight into the swizzled K-major operand
-      {
-        const int s = i % KR_SLOTS;
-        if (i >= KR_SLOTS && !mbar_wait(&kr_empty[s], ((i / KR_SLOTS) - 1) & 1, p.status)) {
-          ok = false;
-          break;
-        }
-        const unsigned vmask = __ballot_sync(FULL, valid_t);
-        if (lane == 0) mbar_arrive_expect_tx(&kr_full[s], __popc(vmask) * blk_bytes);
-        __syncwarp();
-        if (valid_t)
-          tma_load_2d(kring + s * KR_BYTES + lane * blk_bytes, &tmap_k, 0,
-                      (pb_l * p.Hkv + g) * bs, &kr_full[s]);
-        k_issued = i + 1;
+      const unsigned vmask = __ballot_sync(FULL, valid_t);
+      const int row = (pb_l * p.Hkv + g) * bs;
+      const int s = i % SLOTS;
+      // K, then V: the tile's blocks straight into the swizzled operands
+      if (i >= SLOTS && !mbar_wait(&kr_empty[s], ((i / SLOTS) - 1) & 1, p.status)) ok = false;
+      if (!__all_sync(FULL, ok)) break;
+      if (lane == 0) mbar_arrive_expect_tx(&kr_full[s], __popc(vmask) * blk_bytes);
+      __syncwarp();
+      if (valid_t) tma_load_2d(kring + s * TILE_BYTES + lane * blk_bytes, &tmap_k, 0, row, &kr_full[s]);
+      if (i >= SLOTS && !mbar_wait(&vr_empty[s], ((i / SLOTS) - 1) & 1, p.status)) ok = false;
+      if (!__all_sync(FULL, ok)) {
+        issued = -(i + 1);                    // K of tile i is out, V is not
+        break;
       }
-      // V: two staging slots of 64 tokens
-      for (int hh = 0; hh < 2; ++hh) {
-        const int u = 2 * i + hh;
-        const int s = u % ST_SLOTS;
-        if (u >= ST_SLOTS && !mbar_wait(&st_empty[s], ((u / ST_SLOTS) - 1) & 1, p.status)) {
-          ok = false;
-          break;
-        }
-        const int j0 = hh * bph;
-        const int nb = max(0, min(bph, last_blk - (b0 + j0)));
-        const int pb = __shfl_sync(FULL, pb_l, (j0 + (lane < bph ? lane : 0)) & 31);
-        const bool valid = lane < nb && pb >= 0 && pb < p.num_blocks;
-        const unsigned vmask = __ballot_sync(FULL, valid);
-        if (lane == 0) mbar_arrive_expect_tx(&st_full[s], __popc(vmask) * blk_bytes);
-        __syncwarp();
-        if (valid)
-          bulk_load(stage + s * ST_BYTES + lane * blk_bytes,
-                    vbase + static_cast<int64_t>(pb) * blk_stride, blk_bytes, &st_full[s]);
-        v_issued = u + 1;
-      }
+      if (lane == 0) mbar_arrive_expect_tx(&vr_full[s], __popc(vmask) * blk_bytes);
+      __syncwarp();
+      if (valid_t) tma_load_2d(vring + s * TILE_BYTES + lane * blk_bytes, &tmap_v, 0, row, &vr_full[s]);
+      issued = i + 1;
     }
     if (!ok) {  // wait (bounded) for our own copies still in flight
-      for (int i = k_issued - KR_SLOTS < 0 ? 0 : k_issued - KR_SLOTS; i < k_issued; ++i)
-        mbar_wait(&kr_full[i % KR_SLOTS], (i / KR_SLOTS) & 1, p.status);
-      for (int u = v_issued - ST_SLOTS < 0 ? 0 : v_issued - ST_SLOTS; u < v_issued; ++u)
-        mbar_wait(&st_full[u % ST_SLOTS], (u / ST_SLOTS) & 1, p.status);
-    }
-    return;
-  }
-
-  if (warp >= 6) {
-    // ================= converters: V codes -> the f16 V^T operand =================
-    const int ct = threadIdx.x - 192;         // 0..127
-    const int c = ct & 7;                     // 16-code chunk of a 128-byte row
-    const int r0 = ct >> 3;                   // 0..15
-    bool ok = true;
-    auto wait = [&](uint64_t* bar, uint32_t parity) {
-      if (ok) ok = mbar_wait(bar, parity, p.status);
-      ok = __all_sync(FULL, ok);
-      return ok;
-    };
-    for (int i = 0; i < n_tiles && ok; ++i) {
-      const int n_valid = min(TOK, end - (start + i * TOK));
-      uint4 cw[2][4];
-      for (int hh = 0; hh < 2; ++hh) {
-        const int u = 2 * i + hh;
-        const int s = u % ST_SLOTS;
-        if (!wait(&st_full[s], (u / ST_SLOTS) & 1)) break;
-        const uint8_t* src = stage + s * ST_BYTES;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int rr = r0 + 16 * j;
-          cw[hh][j] = (hh * HALF_TOK + rr < n_valid)
-                          ? *reinterpret_cast<const uint4*>(src + rr * DH + c * 16)
-                          : make_uint4(0, 0, 0, 0);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&st_empty[s]);
-      }
-      if (!ok) break;
-      if (i >= 1 && !wait(vop_empty, (i - 1) & 1)) break;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int R = hh * HALF_TOK + r0 + 16 * j;     // token row within the tile
-          uint4 lo, hi;
-          widen16(cw[hh][j], lo, hi);                    // zero codes widen to +0
-          const uint32_t rb = (R >> 3) * GROUP_BYTES + (R & 7) * 128;
-          const int c0 = 2 * c, c1 = 2 * c + 1;          // 8-dim chunks of the f16 row
-          *reinterpret_cast<uint4*>(vop + rb + (c0 >> 3) * HALF_OFF + (((c0 & 7) ^ (R & 7)) << 4)) = lo;
-          *reinterpret_cast<uint4*>(vop + rb + (c1 >> 3) * HALF_OFF + (((c1 & 7) ^ (R & 7)) << 4)) = hi;
-        }
-      }
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(vop_full);
+      const int k_out = issued < 0 ? -issued : issued;
+      const int v_out = issued < 0 ? -issued - 1 : issued;
+      for (int i = k_out - SLOTS < 0 ? 0 : k_out - SLOTS; i < k_out; ++i)
+        mbar_wait(&kr_full[i % SLOTS], (i / SLOTS) & 1, p.status);
+      for (int i = v_out - SLOTS < 0 ? 0 : v_out - SLOTS; i < v_out; ++i)
+        mbar_wait(&vr_full[i % SLOTS], (i / SLOTS) & 1, p.status);
     }
     return;
   }
@@ -407,7 +327,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       }
       *reinterpret_cast<uint4*>(qop + term * QT_BYTES + row_off) = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    for (int i = t; i < 2 * OPB_BYTES / 16; i += 128)
+    for (int i = t; i < 2 * PB_BYTES / 16; i += 128)
       reinterpret_cast<uint4*>(pop)[i] = make_uint4(0, 0, 0, 0);
     fence_async_smem();
     __syncwarp();
@@ -418,13 +338,12 @@ __global__ void __launch_bounds__(THREADS, 2)
   if (warp == 1) {
     // ================= MMA issuer =================
     if (lane == 0) {
-      const uint32_t id_pv = instr_desc<__half>(true);
-      const uint32_t k_a = smem_addr(kring), v_a = smem_addr(vop);
+      const uint32_t k_a = smem_addr(kring), v_a = smem_addr(vring);
       const uint32_t q_a = smem_addr(qop), p_a = smem_addr(pop);
       bool ok = true;
       auto issue_qk = [&](int i) -> bool {
-        const int s = i % KR_SLOTS;
-        if (!mbar_wait(&kr_full[s], (i / KR_SLOTS) & 1, p.status)) return false;
+        const int s = i % SLOTS;
+        if (!mbar_wait(&kr_full[s], (i / SLOTS) & 1, p.status)) return false;
         if (i >= 2 && !mbar_wait(&s_free[i & 1], ((i >> 1) - 1) & 1, p.status)) return false;
         tc_fence_after();
         const uint32_t d = tmem + (i & 1) * NPAD;
@@ -432,7 +351,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         for (int term = 0; term < NTERM; ++term) {
 #pragma unroll
           for (int k = 0; k < DH / 32; ++k) {   // 32 codes (32 bytes) per MMA
-            const uint64_t a = smem_desc(k_a + s * KR_BYTES + k * 32, 16, 1024);
+            const uint64_t a = smem_desc(k_a + s * TILE_BYTES + k * 32, 16, 1024);
             const uint64_t bq = smem_desc(q_a + term * QT_BYTES + k * 32, 16, 1024);
             mma_e4m3(d, a, bq, kIdescE4M3, (term > 0 || k > 0) ? 1u : 0u);
           }
@@ -442,20 +361,23 @@ __global__ void __launch_bounds__(THREADS, 2)
         return true;
       };
       auto issue_pv = [&](int i) -> bool {
-        if (!mbar_wait(vop_full, i & 1, p.status)) return false;
+        const int s = i % SLOTS;
+        if (!mbar_wait(&vr_full[s], (i / SLOTS) & 1, p.status)) return false;
         if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, p.status)) return false;
         const bool first = (i % tpp) == 0;     // a partition starts: O restarts at 0
         if (MULTI && first && i > 0 && !mbar_wait(o_free, ((i / tpp) - 1) & 1, p.status)) return false;
         tc_fence_after();
         const uint32_t d = tmem + 2 * NPAD;
 #pragma unroll
-        for (int k = 0; k < TOK / 16; ++k) {
-          const uint64_t a = smem_desc(v_a + k * 2 * GROUP_BYTES, HALF_OFF, GROUP_BYTES);
-          const uint64_t bp =
-              smem_desc(p_a + (i & 1) * OPB_BYTES + (k >> 2) * (NPAD * 128) + (k & 3) * 32, 16, 1024);
-          mma_f16(d, a, bp, id_pv, (!first || k > 0) ? 1u : 0u);
+        for (int term = 0; term < PTERM; ++term) {
+#pragma unroll
+          for (int k = 0; k < TOK / 32; ++k) {  // 32 tokens per MMA: four 8-token groups
+            const uint64_t a = smem_desc(v_a + s * TILE_BYTES + k * 4096, 1024, 1024);
+            const uint64_t bp = smem_desc(p_a + (i & 1) * PB_BYTES + term * PT_BYTES + k * 32, 16, 1024);
+            mma_e4m3(d, a, bp, kIdescE4M3_AMN, (!first || term > 0 || k > 0) ? 1u : 0u);
+          }
         }
-        mma_commit(vop_empty);
+        mma_commit(&vr_empty[s]);
         mma_commit(&p_free[i & 1]);
         return true;
       };
@@ -478,6 +400,11 @@ __global__ void __launch_bounds__(THREADS, 2)
       l_part[h] = 0.f;
       sc[h] = p.scale_log2 * qs[h];
     }
+    // byte of token r in row h of a K-major, 128-byte-swizzled P term
+    uint32_t pcol[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+      pcol[h] = h * 128 + ((((r >> 4) ^ h) & 7) << 4) + (r & 15);
     bool ok = true;
     auto wait = [&](uint64_t* bar, uint32_t parity) {
       if (ok) ok = mbar_wait(bar, parity, p.status);
@@ -507,10 +434,11 @@ __global__ void __launch_bounds__(THREADS, 2)
       }
       named_sync(1, 128);
       if (ok) {
+        const float oscale = p.v_scale * P_DOWN;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           const float Ls = red[h] + red[NPAD + h] + red[2 * NPAD + h] + red[3 * NPAD + h];
-          const float O = o[h] * p.v_scale;
+          const float O = o[h] * oscale;
           const int64_t hq = static_cast<int64_t>(b) * p.Hq + g * G + h;
           if (single) {
             static_cast<T*>(p.out)[hq * DH + r] = Elem<T>::from_float(O / Ls);
@@ -590,10 +518,32 @@ __global__ void __launch_bounds__(THREADS, 2)
         l_part[h] += pr[h];
       }
       if (i >= 2) wait(&p_free[i & 1], ((i >> 1) - 1) & 1);
-      uint8_t* pb = pop + (i & 1) * OPB_BYTES + (r >> 6) * (NPAD * 128);
+      uint8_t* pb = pop + (i & 1) * PB_BYTES;
 #pragma unroll
-      for (int h = 0; h < G; ++h)
-        *reinterpret_cast<uint16_t*>(pb + sw128(h, r & 63)) = to_bits<__half>(pr[h]);
+      for (int h = 0; h < G; h += 2) {
+        // P * 2^6 = P1 + P2, two E4M3 codes per head (heads h, h+1 in one pair)
+        const float x0 = pr[h] * P_UP;
+        const float x1 = (h + 1 < G) ? pr[h + 1] * P_UP : 0.f;
+        const uint32_t c1 = to_e4m3x2(x0, x1);
+        const float2 d1 = from_e4m3x2(c1);
+        const uint32_t c2 = to_e4m3x2(x0 - d1.x, x1 - d1.y);
+        pb[pcol[h]] = static_cast<uint8_t>(c1);
+        pb[PT_BYTES + pcol[h]] = static_cast<uint8_t>(c2);
+        if (h + 1 < G) {
+          pb[pcol[h + 1]] = static_cast<uint8_t>(c1 >> 8);
+          pb[PT_BYTES + pcol[h + 1]] = static_cast<uint8_t>(c2 >> 8);
+        }
+      }
+      if (n_valid < TOK) {
+        // the last tile: zero the V rows of tokens past the end, so that
+        // whatever they hold (unused slots, stale data) adds 0 * 0 to O
+        const int s_ = i % SLOTS;
+        if (wait(&vr_full[s_], (i / SLOTS) & 1) && !valid) {
+          uint4* row = reinterpret_cast<uint4*>(vring + s_ * TILE_BYTES + r * DH);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) row[c] = make_uint4(0, 0, 0, 0);
+        }
+      }
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -614,25 +564,57 @@ __global__ void __launch_bounds__(THREADS, 2)
   }
 }
 
+constexpr int kMaxSpan = 4096;   // tokens one CTA may stream through
+constexpr int kStreamBelow = 2048;  // only partitions shorter than this are streamed
+
+int sm_count8() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0, v = 0;
+    n = (cudaGetDevice(&dev) == cudaSuccess &&
+         cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+            ? v
+            : 148;
+  }
+  return n;
+}
+
+// Consecutive partitions per CTA: for partitions shorter than kStreamBelow
+// tokens, the most of 8 / 4 / 2 that keeps a CTA's span within kMaxSpan tokens
+// and still leaves at least 8 CTAs per SM (a tile of E4M3 codes is half the
+// bytes of a 16-bit one, so a CTA streams longer before its fixed costs are
+// paid back; two partitions of 2048 were slower than one).
+int tc8_parts_per_cta(const DecodeArgs& a) {
+  if (a.partition_size >= kStreamBelow) return 1;
+  const int64_t want = 8ll * sm_count8();
+  for (int c : {8, 4, 2}) {
+    const int64_t ctas = static_cast<int64_t>(a.num_seqs) * a.Hkv * ((a.num_partitions + c - 1) / c);
+    if (static_cast<int64_t>(a.partition_size) * c <= kMaxSpan && a.num_partitions >= c && ctas >= want)
+      return c;
+  }
+  return 1;
+}
+
 template <typename T, int G>
 cudaError_t launch_tc8_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
-  const int ppc = tc_parts_per_cta(a);
+  const int ppc = tc8_parts_per_cta(a);
   // one partition per CTA compiles without the partition-streaming logic
   auto kern = ppc > 1 ? decode_partition_tc8_kernel<T, G, true> : decode_partition_tc8_kernel<T, G, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  // the K cache [NB][Hkv][bs][128] as rows of 128 codes; a box is the bs rows of
+  // each cache [NB][Hkv][bs][128] as rows of 128 codes; a box is the bs rows of
   // one (block, head), stored with the 128-byte swizzle
-  CUtensorMap mk;
+  CUtensorMap mk, mv;
   const int64_t rows = static_cast<int64_t>(a.num_blocks) * a.Hkv * a.block_size;
   const int64_t dims[2] = {DH, rows};
   const int64_t strides[1] = {DH};
   const int box[2] = {DH, a.block_size};
-  if (!make_tmap(&mk, a.k_cache, 2, dims, strides, box, PA_FP8_E4M3)) return cudaErrorInvalidValue;
+  if (!make_tmap(&mk, a.k_cache, 2, dims, strides, box, PA_FP8_E4M3) ||
+      !make_tmap(&mv, a.v_cache, 2, dims, strides, box, PA_FP8_E4M3))
+    return cudaErrorInvalidValue;
   Tc8Params p;
   p.out = a.out;
   p.q = a.q;
-  p.v_cache = static_cast<const uint8_t*>(a.v_cache);
   p.block_tables = a.block_tables;
   p.context_lens = a.context_lens;
   const int64_t nrows = static_cast<int64_t>(a.num_seqs) * a.Hq * a.num_partitions;
@@ -651,7 +633,7 @@ cudaError_t launch_tc8_t(const DecodeArgs& a, unsigned int* status, cudaStream_t
   p.scale_log2 = a.scale * 1.4426950408889634f * a.k_scale;
   p.v_scale = a.v_scale;
   dim3 grid(a.num_seqs, a.Hkv, (a.num_partitions + p.parts_per_cta - 1) / p.parts_per_cta);
-  return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk);
+  return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
 }
 
 }  // namespace

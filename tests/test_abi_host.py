@@ -133,8 +133,17 @@ def test_auto_partition_size(L):
     assert pk.pa_decode_auto_partition_size(256, 64, 8, 64, bf, 4096) == 512
     assert pk.pa_decode_auto_partition_size(256, 64, 8, 128, pk.PA_F32, 4096) == 512
     assert pk.pa_decode_auto_partition_size(4, 6, 4, 128, bf, 100) == -1
+    # over an E4M3 cache the tensor-core kernel may take 4096
+    a8 = pk.pa_decode_fp8_auto_partition_size
+    assert a8(256, 64, 8, 128, bf, 4096) == 4096
+    assert a8(128, 32, 8, 128, bf, 32768) == 4096
+    assert a8(16, 64, 8, 128, bf, 32768) == 2048
+    assert a8(1, 64, 8, 128, bf, 32768) == 512
+    assert a8(64, 40, 40, 128, pk.PA_F16, 2048) == 512
+    assert a8(256, 64, 8, 128, pk.PA_FP8_E4M3, 4096) == -1
+    assert a8(4, 6, 4, 128, bf, 100) == -1
     # the default-sized workspace covers the automatic length
-    for P in (1024, 2048):
+    for P in (1024, 2048, 4096):
         assert pk.pa_decode_workspace_bytes(256, 64, 128, 4096, P) <= \
             pk.pa_decode_workspace_bytes(256, 64, 128, 4096, 0)
 

@@ -460,11 +460,11 @@ class Oracle_view:
 
 
 # ---------------------------------------------------------------------------
-# E4M3 cache on the tensor-core kernel (G = 4 / 8, D = 128, f16 / bf16 queries)
+# E4M3 cache on the tensor-core kernel (G = 1, 2, 4, 8, D = 128, f16 / bf16 queries)
 
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
-@pytest.mark.parametrize("G", [4, 8])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
 @pytest.mark.parametrize("bs", [8, 16, 32])
 def test_fp8_tc_edges(dtype, G, bs):
     lens = (0, 1, 63, 64, 65, 127, 128, 129, 255, 256, 257, 700)
@@ -475,6 +475,59 @@ def test_fp8_tc_edges(dtype, G, bs):
     assert np.all(got[0] == 0.0)
     full_check(spec, partition_size=128)
     full_check(spec, partition_size=4096)
+
+
+@pytest.mark.parametrize("G", [1, 8])
+@pytest.mark.parametrize("slope", [0.05, -0.05, 0.004])
+@pytest.mark.parametrize("P", [0, 512])
+def test_fp8_tc_score_ramps(G, slope, P):
+    """Scores that rise along the sequence (the running max is raised in every
+    tile, O rescaled each time), fall (every later P far below the first), or
+    drift slowly: key j is a_j times a fixed sign pattern, the query that
+    pattern, so s_j log2(e) = slope * j up to E4M3 rounding of a_j."""
+    rng = np.random.default_rng(443 + G)
+    B, Hkv, D, bs, L = 2, 2, 128, 16, (1500, 700)
+    Hq = G * Hkv
+    nb = [(n + bs - 1) // bs for n in L]
+    NB = sum(nb) + 3
+    perm = rng.permutation(NB).astype(np.int32)
+    tables = np.full((B, max(nb)), -1, np.int32)
+    tables[0, :nb[0]] = perm[:nb[0]]
+    tables[1, :nb[1]] = perm[nb[0]:nb[0] + nb[1]]
+    sign = np.where(rng.random((Hkv, D)) < 0.5, -1.0, 1.0)
+    scale = 1.0 / np.sqrt(D)
+    k_scale, v_scale = 0.0123, 0.0171
+    # s_j = scale * k_scale * a_j * D, so a_j = slope * j / (log2(e) * scale * k_scale * D)
+    j = np.arange(max(L), dtype=np.float64)
+    a = slope * (j - (max(L) if slope < 0 else 0)) / (np.log2(np.e) * scale * k_scale * D)
+    a = np.clip(a, -440.0, 440.0)
+    kf = np.zeros((NB, Hkv, bs, D))
+    for b in range(B):
+        for t in range(L[b]):
+            kf[tables[b, t // bs], :, t % bs, :] = a[t] * sign
+    kcodes = oracle.encode_e4m3(kf)
+    vcodes = oracle.encode_e4m3(rng.standard_normal((NB, Hkv, bs, D)) / v_scale)
+    q = np.repeat(sign[None, :, None, :], B, 0).repeat(G, 2).reshape(B, Hq, D)
+    tdt = torch.bfloat16
+    qt = torch.tensor(q, dtype=tdt)
+    q_bits = W.storage_view(qt)
+    lens = np.array(L, np.int32)
+    want = oracle.paged_attention(q_bits, kcodes, vcodes, W.DTYPE_CODES["bf16"], tables, lens,
+                                  scale, kv_dtype=oracle.E4M3, k_scale=k_scale, v_scale=v_scale)
+    f8 = torch.float8_e4m3fn
+    kc = torch.from_numpy(kcodes).view(f8).cuda()
+    vc = torch.from_numpy(vcodes).view(f8).cuda()
+    out = torch.empty((B, Hq, D), dtype=tdt, device="cuda")
+    ws = torch.empty(pk.pa_decode_workspace_bytes(B, Hq, D, max(L), P), dtype=torch.uint8,
+                     device="cuda")
+    pk.pa_decode_fp8(out, qt.cuda(), kc, vc, torch.from_numpy(tables).cuda(),
+                     torch.from_numpy(lens).cuda(), scale, max(L), k_scale, v_scale,
+                     partition_size=P, workspace=ws)
+    torch.cuda.synchronize()
+    assert pk.pa_device_status() == 0
+    got = out.double().cpu().numpy()
+    err = np.abs(got - want).max()
+    assert err <= TOL["bf16"], err
 
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])

@@ -12,7 +12,7 @@
 //   S^T [128 tokens x 16] = K [128 x 128] . Q^T [128 x 16]     (heads padded to 16)
 //   O^T [128 dims   x 16] += V^T [128 x 128] . P^T [128 x 16]
 //
-// Roles in a CTA of 6 warps, one CTA per (sequence, kv head, partition):
+// Roles in a CTA of 6 warps, one CTA per (sequence, kv head, run of partitions):
 //   warp 0   producer: block-table lookups, one TMA load per physical block of
 //            its K (or V) rows into a ring of three 32 KB slots holding K_0, V_0,
 //            K_1, V_1, ...  The cache is viewed as a 4-D tensor (64 columns, 8
@@ -63,7 +63,7 @@ constexpr int OFF_RING = 0;
 constexpr int OFF_Q = OFF_RING + SLOTS * SLOT_BYTES;
 constexpr int OFF_P = OFF_Q + OPB_BYTES;     // two P buffers
 constexpr int OFF_BAR = OFF_P + 2 * OPB_BYTES;
-constexpr int NBARS = 2 * SLOTS + 10;        // ring full/empty, s/p full/free, q_ready, o_free
+constexpr int NBARS = 2 * SLOTS + 9;         // ring full/empty, s/p full/free, q_ready
 constexpr int OFF_TMEM = OFF_BAR + NBARS * 8;
 constexpr int OFF_RED = OFF_TMEM + 16;       // 4 warps x 16 floats
 constexpr int SMEM_USED = OFF_RED + 4 * NPAD * 4;
@@ -98,7 +98,7 @@ struct TcParams {
 // column c of S / O is query token c / G (one of the sequence's last Qb <= NQ
 // context tokens) with head c % G, and a key counts for it only up to that
 // token's own position.  NQ = 1 is the decode step and compiles as before.
-template <typename T, int G, bool MULTI, int NQ = 1>
+template <typename T, int G, int NQ = 1>
 __global__ void __launch_bounds__(THREADS, 2)
     decode_partition_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmap_k,
                                const __grid_constant__ CUtensorMap tmap_v) {
@@ -116,15 +116,15 @@ __global__ void __launch_bounds__(THREADS, 2)
   uint64_t* p_full = s_free + 2;            // [2]
   uint64_t* p_free = p_full + 2;            // [2]
   uint64_t* q_ready = p_free + 2;           // Q^T operand staged
-  uint64_t* o_free = q_ready + 1;           // a partition's O has been read out
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
   float* red = reinterpret_cast<float*>(smem + OFF_RED);
 
-  // A CTA streams parts_per_cta consecutive partitions (tiles never straddle
-  // one: P is a multiple of TOK) and writes each one's partial as it ends, so
-  // short partitions do not each pay the pipeline's fill and drain.
+  // A CTA covers parts_per_cta consecutive partitions with one softmax, so
+  // short partitions do not each pay the pipeline's fill and drain: its partial
+  // goes to the first one's slot and the others' slots get empty partials (max
+  // -inf, sum 0, output 0), which the reduce weighs by exactly 0.
   const int b = NQ > 1 ? blockIdx.x / p.q_groups : blockIdx.x;
-  const int g = blockIdx.y, part = MULTI ? blockIdx.z * p.parts_per_cta : blockIdx.z;
+  const int g = blockIdx.y, part = blockIdx.z * p.parts_per_cta;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int NC = G * NQ;                // S / O columns in use
   static_assert(NC <= NPAD, "query tokens x heads must fit the MMA's N");
@@ -165,12 +165,11 @@ __global__ void __launch_bounds__(THREADS, 2)
     return;
   }
   if (start >= L) return;
-  const int end = MULTI ? static_cast<int>(min(static_cast<int64_t>(L),
-                                               start + static_cast<int64_t>(P) * p.parts_per_cta))
-                        : min(L, start + P);
+  const int end = static_cast<int>(
+      min(static_cast<int64_t>(L), start + static_cast<int64_t>(P) * p.parts_per_cta));
   const int n_tiles = (end - start + TOK - 1) / TOK;
-  const int tpp = MULTI ? P / TOK : (1 << 30);                               // tiles per partition
   const bool single = (L <= P);
+  const int n_slots = min(p.parts_per_cta, (L + P - 1) / P - part);   // partials this CTA writes
 
   // ---- set-up: the producer starts streaming right after the barrier, while
   // the softmax warps stage Q^T and the MMA issuer waits for it ----
@@ -194,7 +193,6 @@ __global__ void __launch_bounds__(THREADS, 2)
         mbar_init(&p_free[j], 1);
       }
       mbar_init(q_ready, 4);
-      mbar_init(o_free, 4);
       fence_mbar_init();
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
@@ -302,8 +300,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         const int u = 2 * i + 1, s = u % SLOTS;
         if (!mbar_wait(&ring_full[s], (u / SLOTS) & 1, p.status)) return false;
         if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, p.status)) return false;
-        const bool first = (i % tpp) == 0;             // a partition starts: O restarts at 0
-        if (MULTI && first && i > 0 && !mbar_wait(o_free, ((i / tpp) - 1) & 1, p.status)) return false;
+        const bool first = i == 0;                     // O starts at 0
         tc_fence_after();
         const uint32_t d = tmem + 2 * NPAD;
 #pragma unroll
@@ -345,8 +342,9 @@ __global__ void __launch_bounds__(THREADS, 2)
       ok = __all_sync(FULL, ok);
       return ok;
     };
-    // Row r of O^T (dim r, all heads) and the sums of the partition ending at
-    // tile i: the output, or the split-K partial of partition part + i / tpp.
+    // Row r of O^T (dim r, all heads) and the sums of the CTA's span, whose last
+    // tile is i: the output, or the split-K partial of partition part (and
+    // empty partials for the span's other partitions).
     auto flush = [&](int i) {
       wait(&p_free[i & 1], (i >> 1) & 1);
       tc_fence_after();
@@ -354,7 +352,6 @@ __global__ void __launch_bounds__(THREADS, 2)
       tmem_ld16(tmem + lane_base + 2 * NPAD, o);
       tc_fence_before();
       __syncwarp();
-      if (MULTI && lane == 0) mbar_arrive(o_free);              // the next partition may reuse O
 #pragma unroll
       for (int h = 0; h < NC; ++h) {
         float x = l_part[h];
@@ -377,11 +374,18 @@ __global__ void __launch_bounds__(THREADS, 2)
           if (single) {
             static_cast<T*>(p.out)[hq * DH + r] = Elem<T>::from_float(o[h] / Ls);
           } else {
-            const int64_t slot = hq * p.num_partitions + part + i / tpp;
+            const int64_t slot = hq * p.num_partitions + part;
             p.ws_o[slot * DH + r] = o[h];
             if (r == 0) {
               p.ws_m[slot] = m_run[h];
               p.ws_l[slot] = Ls;
+            }
+            for (int e = 1; e < n_slots; ++e) {
+              p.ws_o[(slot + e) * DH + r] = 0.f;
+              if (r == 0) {
+                p.ws_m[slot + e] = -INFINITY;
+                p.ws_l[slot + e] = 0.f;
+              }
             }
           }
         }
@@ -390,14 +394,6 @@ __global__ void __launch_bounds__(THREADS, 2)
     for (int i = 0; i < n_tiles; ++i) {
       const int n_valid = min(TOK, end - (start + i * TOK));
       const bool valid = r < n_valid;
-      const bool first = (i % tpp) == 0;
-      if (MULTI && first && i > 0) {                            // a new partition: a new softmax
-#pragma unroll
-        for (int h = 0; h < NC; ++h) {
-          m_run[h] = -INFINITY;
-          l_part[h] = 0.f;
-        }
-      }
       float sv[16];
       if (wait(&s_full[i & 1], (i >> 1) & 1)) {
         tc_fence_after();
@@ -440,9 +436,9 @@ __global__ void __launch_bounds__(THREADS, 2)
           l_part[h] *= alpha[h];
         }
         named_sync(1, 128);
-        // O must hold every earlier tile of the partition before it is rescaled
-        // (at a partition's first tile O restarts from zero instead)
-        if (!first && wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
+        // O must hold every earlier tile before it is rescaled (at the first
+        // tile O starts from zero instead)
+        if (i > 0 && wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
           tc_fence_after();
           float o[16];
           tmem_ld16(tmem + lane_base + 2 * NPAD, o);
@@ -480,9 +476,8 @@ __global__ void __launch_bounds__(THREADS, 2)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[i & 1]);
-      if (MULTI && (i + 1) % tpp == 0 && i + 1 < n_tiles) flush(i);   // a partition ends mid-CTA
     }
-    flush(n_tiles - 1);                                       // the CTA's last partition
+    flush(n_tiles - 1);
   }
 
   // ---- teardown: warps 1-5 meet, warp 1 frees TMEM ----
@@ -501,8 +496,7 @@ __global__ void __launch_bounds__(THREADS, 2)
 template <typename T, int G>
 cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
   const int ppc = tc_parts_per_cta(a);
-  // one partition per CTA compiles without the partition-streaming logic
-  auto kern = ppc > 1 ? decode_partition_tc_kernel<T, G, true> : decode_partition_tc_kernel<T, G, false>;
+  auto kern = decode_partition_tc_kernel<T, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // the cache [NB][Hkv][bs][128] as a 4-D tensor: 64 columns (stride 2 B),
@@ -613,8 +607,7 @@ cudaError_t launch_tcq_t(const MqArgs& m, unsigned int* status, cudaStream_t str
   a.partition_size = m.partition_size;
   a.num_partitions = m.num_partitions;
   const int ppc = tc_parts_per_cta(a);
-  auto kern = ppc > 1 ? decode_partition_tc_kernel<T, G, true, NQ>
-                      : decode_partition_tc_kernel<T, G, false, NQ>;
+  auto kern = decode_partition_tc_kernel<T, G, NQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   CUtensorMap mk, mv;

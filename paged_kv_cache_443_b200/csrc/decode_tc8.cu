@@ -29,7 +29,7 @@
 //   128 codes stored with the 128-byte swizzle: the canonical K-major layout of
 //   K and, unchanged, the MN-major layout of V^T (8-token groups 1 KB apart).
 //
-// Roles in a CTA of 6 warps, one CTA per (sequence, kv head, partition):
+// Roles in a CTA of 6 warps, one CTA per (sequence, kv head, run of partitions):
 //   warp 0     producer: block-table lookups; per tile one TMA load per block
 //              of its K codes and one of its V codes into two rings of three
 //              16 KB tiles;
@@ -71,7 +71,7 @@ constexpr int OFF_VR = OFF_KR + SLOTS * TILE_BYTES;
 constexpr int OFF_Q = OFF_VR + SLOTS * TILE_BYTES;
 constexpr int OFF_P = OFF_Q + NTERM * QT_BYTES;   // two P buffers
 constexpr int OFF_BAR = OFF_P + 2 * PB_BYTES;
-constexpr int NBARS = 4 * SLOTS + 8 + 2;
+constexpr int NBARS = 4 * SLOTS + 8 + 1;
 constexpr int OFF_TMEM = (OFF_BAR + NBARS * 8 + 15) / 16 * 16;
 constexpr int OFF_RED = OFF_TMEM + 16;      // 4 warps x 16 floats
 constexpr int OFF_QS = OFF_RED + 4 * NPAD * 4;
@@ -140,7 +140,7 @@ __device__ __forceinline__ float2 from_e4m3x2(uint32_t c) {
   return __half22float2(*reinterpret_cast<const __half2*>(&lo));
 }
 
-template <typename T, int G, bool MULTI>
+template <typename T, int G>
 __global__ void __launch_bounds__(THREADS, 2)
     decode_partition_tc8_kernel(const Tc8Params p, const __grid_constant__ CUtensorMap tmap_k,
                                 const __grid_constant__ CUtensorMap tmap_v) {
@@ -161,13 +161,14 @@ __global__ void __launch_bounds__(THREADS, 2)
   uint64_t* p_full = s_free + 2;             // [2]
   uint64_t* p_free = p_full + 2;             // [2]
   uint64_t* q_ready = p_free + 2;
-  uint64_t* o_free = q_ready + 1;            // a partition's O has been read out
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
   float* red = reinterpret_cast<float*>(smem + OFF_RED);
   float* qs = reinterpret_cast<float*>(smem + OFF_QS);
 
-  // a CTA streams parts_per_cta consecutive partitions (as in decode_tc.cu)
-  const int b = blockIdx.x, g = blockIdx.y, part = MULTI ? blockIdx.z * p.parts_per_cta : blockIdx.z;
+  // a CTA covers parts_per_cta consecutive partitions with one softmax (as in
+  // decode_tc.cu): its partial goes to the first one's slot, the others' slots
+  // get empty partials (max -inf, sum 0, output 0), which the reduce weighs by 0
+  const int b = blockIdx.x, g = blockIdx.y, part = blockIdx.z * p.parts_per_cta;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   grid_dependency_wait();
@@ -190,12 +191,11 @@ __global__ void __launch_bounds__(THREADS, 2)
     return;
   }
   if (start >= L) return;
-  const int end = MULTI ? static_cast<int>(min(static_cast<int64_t>(L),
-                                               start + static_cast<int64_t>(P) * p.parts_per_cta))
-                        : min(L, start + P);
+  const int end = static_cast<int>(
+      min(static_cast<int64_t>(L), start + static_cast<int64_t>(P) * p.parts_per_cta));
   const int n_tiles = (end - start + TOK - 1) / TOK;
-  const int tpp = MULTI ? P / TOK : (1 << 30);                    // tiles per partition
   const bool single = (L <= P);
+  const int n_slots = min(p.parts_per_cta, (L + P - 1) / P - part);   // partials this CTA writes
 
   const int bs = p.block_size;
   const int first_blk = start / bs;
@@ -215,7 +215,6 @@ __global__ void __launch_bounds__(THREADS, 2)
       mbar_init(&p_free[j], 1);
     }
     mbar_init(q_ready, 4);
-    mbar_init(o_free, 4);
     fence_mbar_init();
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
@@ -364,8 +363,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         const int s = i % SLOTS;
         if (!mbar_wait(&vr_full[s], (i / SLOTS) & 1, p.status)) return false;
         if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, p.status)) return false;
-        const bool first = (i % tpp) == 0;     // a partition starts: O restarts at 0
-        if (MULTI && first && i > 0 && !mbar_wait(o_free, ((i / tpp) - 1) & 1, p.status)) return false;
+        const bool first = i == 0;             // O starts at 0
         tc_fence_after();
         const uint32_t d = tmem + 2 * NPAD;
 #pragma unroll
@@ -411,7 +409,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       ok = __all_sync(FULL, ok);
       return ok;
     };
-    // row r of O^T and the sums of the partition ending at tile i
+    // row r of O^T and the sums of the CTA's span, whose last tile is i
     auto flush = [&](int i) {
       wait(&p_free[i & 1], (i >> 1) & 1);
       tc_fence_after();
@@ -419,7 +417,6 @@ __global__ void __launch_bounds__(THREADS, 2)
       tmem_ld16(tmem + lane_base + 2 * NPAD, o);
       tc_fence_before();
       __syncwarp();
-      if (MULTI && lane == 0) mbar_arrive(o_free);      // the next partition may reuse O
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         float x = l_part[h];
@@ -443,11 +440,18 @@ __global__ void __launch_bounds__(THREADS, 2)
           if (single) {
             static_cast<T*>(p.out)[hq * DH + r] = Elem<T>::from_float(O / Ls);
           } else {
-            const int64_t slot = hq * p.num_partitions + part + i / tpp;
+            const int64_t slot = hq * p.num_partitions + part;
             p.ws_o[slot * DH + r] = O;
             if (r == 0) {
               p.ws_m[slot] = m_run[h];
               p.ws_l[slot] = Ls;
+            }
+            for (int e = 1; e < n_slots; ++e) {
+              p.ws_o[(slot + e) * DH + r] = 0.f;
+              if (r == 0) {
+                p.ws_m[slot + e] = -INFINITY;
+                p.ws_l[slot + e] = 0.f;
+              }
             }
           }
         }
@@ -456,14 +460,6 @@ __global__ void __launch_bounds__(THREADS, 2)
     for (int i = 0; i < n_tiles; ++i) {
       const int n_valid = min(TOK, end - (start + i * TOK));
       const bool valid = r < n_valid;
-      const bool first = (i % tpp) == 0;
-      if (MULTI && first && i > 0) {                    // a new partition: a new softmax
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          m_run[h] = -INFINITY;
-          l_part[h] = 0.f;
-        }
-      }
       float sv[16];
       if (wait(&s_full[i & 1], (i >> 1) & 1)) {
         tc_fence_after();
@@ -502,7 +498,7 @@ __global__ void __launch_bounds__(THREADS, 2)
           l_part[h] *= alpha[h];
         }
         named_sync(1, 128);
-        if (!first && wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
+        if (i > 0 && wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
           tc_fence_after();
           float o[16];
           tmem_ld16(tmem + lane_base + 2 * NPAD, o);
@@ -548,9 +544,8 @@ __global__ void __launch_bounds__(THREADS, 2)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[i & 1]);
-      if (MULTI && (i + 1) % tpp == 0 && i + 1 < n_tiles) flush(i);   // a partition ends mid-CTA
     }
-    flush(n_tiles - 1);                                       // the CTA's last partition
+    flush(n_tiles - 1);
   }
 
   // ---- teardown: warps 1-5 meet, warp 1 frees TMEM ----
@@ -598,8 +593,7 @@ int tc8_parts_per_cta(const DecodeArgs& a) {
 template <typename T, int G>
 cudaError_t launch_tc8_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
   const int ppc = tc8_parts_per_cta(a);
-  // one partition per CTA compiles without the partition-streaming logic
-  auto kern = ppc > 1 ? decode_partition_tc8_kernel<T, G, true> : decode_partition_tc8_kernel<T, G, false>;
+  auto kern = decode_partition_tc8_kernel<T, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // each cache [NB][Hkv][bs][128] as rows of 128 codes; a box is the bs rows of

@@ -121,10 +121,10 @@ int pa_decode_default_partition_size(void);
 
 /*
  * The partition length pa_decode uses when it is given partition_size = 0
- * (tokens; 512, 1024 or 2048).  With 4 or 8 query heads per kv head in
+ * (tokens; 512, 1024, 2048 or 4096).  With 4 or 8 query heads per kv head in
  * fp16/bf16 and head size 128 (the tensor-core kernel) it is the longest of
- * 2048 / 1024 that still gives num_seqs * num_kv_heads * ceil(max_context_len /
- * P) >= 8 * (number of SMs) CTAs; otherwise the default.  Pass it explicitly to
+ * 4096 / 2048 / 1024 that still gives num_seqs * num_kv_heads *
+ * ceil(max_context_len / P) >= 8 * (number of SMs) CTAs; otherwise the default.  Pass it explicitly to
  * pa_decode_partitions / pa_decode_reduce to reproduce pa_decode's automatic
  * choice.  Returns -1 for invalid arguments.
  */
@@ -133,10 +133,9 @@ int pa_decode_auto_partition_size(int num_seqs, int num_heads, int num_kv_heads,
 
 /*
  * The partition length pa_decode_fp8 uses when it is given partition_size = 0:
- * as pa_decode_auto_partition_size (dtype is the queries' type, f32, f16 or
- * bf16), with 4096 among the candidates (4096 / 2048 / 1024) when the
- * tensor-core kernel serves the launch, since an E4M3 tile is half the bytes.
- * Returns -1 for invalid arguments (PA_FP8_E4M3 as dtype included).
+ * the rule of pa_decode_auto_partition_size, with dtype the queries' type (f32,
+ * f16 or bf16).  Returns -1 for invalid arguments (PA_FP8_E4M3 as dtype
+ * included).
  */
 int pa_decode_fp8_auto_partition_size(int num_seqs, int num_heads, int num_kv_heads,
                                       int head_size, pa_dtype dtype, int max_context_len);

@@ -40,17 +40,16 @@ int num_sms() {
 // Partition length pa_decode (and pa_decode_fp8) use for partition_size = 0.
 // The tensor-core kernels (fp16/bf16 queries, head size 128, 4 or 8 query heads
 // per kv head; 16-bit or E4M3 caches) pay a fixed set-up and drain per CTA, so
-// it takes the longest of 2048 / 1024 tokens (4096 / 2048 / 1024 over an E4M3
-// cache, whose tiles are half the bytes) that still gives at least ~4 waves of
-// CTAs (2 per SM) at the longest context; everything else keeps the default.
+// it takes the longest of 4096 / 2048 / 1024 tokens that still gives at least
+// ~4 waves of CTAs (2 per SM) at the longest context; everything else keeps
+// the default.
 int auto_partition(int num_seqs, int num_heads, int num_kv_heads, int head_size, pa_dtype dtype,
-                   int max_context_len, bool e4m3_cache = false) {
+                   int max_context_len) {
   const int G = num_kv_heads > 0 ? num_heads / num_kv_heads : 0;
   const bool tc = (dtype == PA_F16 || dtype == PA_BF16) && head_size == 128 && (G == 4 || G == 8);
   if (!tc) return pa::kDefaultPartition;
   const int64_t want = 8ll * num_sms();
   for (int P : {4096, 2048, 1024}) {
-    if (P == 4096 && !e4m3_cache) continue;
     const int64_t ctas = static_cast<int64_t>(num_seqs) * num_kv_heads * num_partitions(max_context_len, P);
     if (ctas >= want) return P;
   }
@@ -283,7 +282,7 @@ extern "C" int pa_decode_fp8_auto_partition_size(int num_seqs, int num_heads, in
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 ||
       head_size <= 0 || pa::elem_size(dtype) == 0 || dtype == PA_FP8_E4M3 || max_context_len < 0)
     return -1;
-  return auto_partition(num_seqs, num_heads, num_kv_heads, head_size, dtype, max_context_len, true);
+  return auto_partition(num_seqs, num_heads, num_kv_heads, head_size, dtype, max_context_len);
 }
 
 extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -437,7 +436,7 @@ extern "C" pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache
   const char* fn = "pa_decode_fp8";
   if (partition_size == 0 && num_heads > 0 && num_kv_heads > 0)   // as pa_decode
     partition_size =
-        auto_partition(num_seqs, num_heads, num_kv_heads, head_size, dtype, max_context_len, true);
+        auto_partition(num_seqs, num_heads, num_kv_heads, head_size, dtype, max_context_len);
   pa::DecodeArgs a;
   pa_status st = check_decode_fp8(fn, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
                                   context_lens, num_seqs, num_heads, num_kv_heads, head_size,

@@ -546,13 +546,15 @@ static int sm_count() {
   return n;
 }
 
-// Consecutive partitions per CTA: the most of 4 / 2 that keeps a CTA's span
-// within 2048 tokens and still leaves at least 8 CTAs per SM.
+// Consecutive partitions per CTA (one softmax over them): for partitions
+// shorter than 2048 tokens, the most of 8 / 4 / 2 that keeps a CTA's span
+// within 4096 tokens and still leaves at least 8 CTAs per SM.
 int tc_parts_per_cta(const DecodeArgs& a) {
+  if (a.partition_size >= 2048) return 1;
   const int64_t want = 8ll * sm_count();
-  for (int c : {4, 2}) {
+  for (int c : {8, 4, 2}) {
     const int64_t ctas = static_cast<int64_t>(a.num_seqs) * a.Hkv * ((a.num_partitions + c - 1) / c);
-    if (static_cast<int64_t>(a.partition_size) * c <= 2048 && a.num_partitions >= c && ctas >= want)
+    if (static_cast<int64_t>(a.partition_size) * c <= 4096 && a.num_partitions >= c && ctas >= want)
       return c;
   }
   return 1;

@@ -124,8 +124,10 @@ def test_reshape_and_copy_reject_bad_arguments(L):
 def test_auto_partition_size(L):
     bf = pk.PA_BF16
     # tensor-core shapes with plenty of work take long partitions
-    assert pk.pa_decode_auto_partition_size(256, 64, 8, 128, bf, 4096) == 2048
-    assert pk.pa_decode_auto_partition_size(128, 32, 8, 128, bf, 32768) == 2048
+    assert pk.pa_decode_auto_partition_size(256, 64, 8, 128, bf, 4096) == 4096
+    assert pk.pa_decode_auto_partition_size(128, 32, 8, 128, bf, 32768) == 4096
+    assert pk.pa_decode_auto_partition_size(16, 64, 8, 128, bf, 32768) == 2048
+    assert pk.pa_decode_auto_partition_size(8, 64, 8, 128, bf, 32768) == 1024
     # too few CTAs at long partitions: the default
     assert pk.pa_decode_auto_partition_size(1, 64, 8, 128, bf, 32768) == 512
     # other paths keep the default
@@ -133,7 +135,7 @@ def test_auto_partition_size(L):
     assert pk.pa_decode_auto_partition_size(256, 64, 8, 64, bf, 4096) == 512
     assert pk.pa_decode_auto_partition_size(256, 64, 8, 128, pk.PA_F32, 4096) == 512
     assert pk.pa_decode_auto_partition_size(4, 6, 4, 128, bf, 100) == -1
-    # over an E4M3 cache the tensor-core kernel may take 4096
+    # the same rule over an E4M3 cache
     a8 = pk.pa_decode_fp8_auto_partition_size
     assert a8(256, 64, 8, 128, bf, 4096) == 4096
     assert a8(128, 32, 8, 128, bf, 32768) == 4096

@@ -207,7 +207,11 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
  * First phase of pa_decode (same arguments; partition_size = 0 means the
  * default 512 here): one CTA per (sequence, kv head, partition).  Sequences that fit one partition get their final `out` rows;
  * the others leave per-partition (max, sum, unnormalised output) partials in
- * the workspace.
+ * the workspace.  A kernel that covers several consecutive partitions with
+ * one softmax (the tensor-core kernels do, for partitions shorter than 2048
+ * tokens) writes the merged partial to the first partition's slot and empty
+ * partials (max -inf, sum 0, output 0) to the others; pa_decode_reduce gives
+ * them weight 0, so the result is the same joint softmax.
  */
 pa_status pa_decode_partitions(void* out, const void* q, const void* k_cache, const void* v_cache,
                                const int32_t* block_tables, int max_blocks_per_seq,

@@ -6,9 +6,11 @@ One step = one pass of the whole hot path over one synthetic batch: the
 copy-on-write block copies of the step (copy_blocks, when the step has any),
 the append of the step's new tokens (reshape_and_cache), and decode attention
 (decode partitions + split-K reduce).  Block-manager bookkeeping is host work
-done while the batch is built.  The default workload is the OPT-13B-shaped
-decode layer (64 sequences, 40 heads of 128, fp16, lognormal context lengths
-around 600, 20,000-block pool).
+done while the batch is built.  The default workload is the largest one that
+fits one GPU, the long-context shared-prefix decode at block size 16: 128
+requests forked from one 4096-token prefix (the same physical blocks) plus
+unique suffixes of up to 28,672 tokens, Hq=32, Hkv=8, head size 128, bf16,
+split-K partitions of 512 tokens.
 
 Printed (rank 0, one JSON line): the KV-read bandwidth of the step (algorithmic
 KV bytes / device time, aggregated over ranks), the step time, the roofline of
@@ -38,7 +40,6 @@ import argparse
 import hashlib
 import json
 import os
-import re
 import sys
 import threading
 import time
@@ -51,7 +52,7 @@ sys.path.insert(0, ROOT)
 import workloads as W  # noqa: E402
 
 METRIC = "paged decode attention µs/step and KV-read GB/s (fraction of B200 HBM peak)"
-DEFAULT_WORKLOAD = "opt13b"
+DEFAULT_WORKLOAD = "long_prefix_bs16"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 
@@ -279,18 +280,27 @@ def source_digest(files=KERNEL_SOURCES["decode_partition_kernel"]):
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload, kernel="decode_partition_kernel"):
-    """dram bytes per launch of the decode-partition kernel from the committed
-    ncu summary, if it was taken on the current source of that kernel; else None."""
-    path = os.path.join(ROOT, "profiles", f"decode_partition_{workload}.md")
-    if not os.path.exists(path):
-        return None
-    txt = open(path).read()
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.e+]+)", txt)
-    s = re.search(r"source_digest:\s*([0-9a-f]+)", txt)
-    if not m or not s or s.group(1) != source_digest(KERNEL_SOURCES[kernel]):
-        return None
-    return float(m.group(1))
+TRAFFIC_FILE = os.path.join("profiles", "dram_traffic.json")
+
+
+def profiled_traffic(workload, kernel, partition_size):
+    """DRAM bytes per launch of the decode-partition kernel, from the ncu capture
+    recorded in profiles/dram_traffic.json for this workload, kernel and
+    partition length, and only while that kernel's sources are unchanged since
+    the capture.  Returns (bytes or None, a note saying where they come from)."""
+    path = os.path.join(ROOT, TRAFFIC_FILE)
+    try:
+        with open(path) as f:
+            entries = json.load(f)["captures"]
+    except (OSError, ValueError, KeyError):
+        return None, "no ncu capture recorded"
+    for e in entries:
+        if (e.get("workload") == workload and e.get("kernel") == kernel
+                and int(e.get("partition_size", -1)) == int(partition_size)):
+            if e.get("source_digest") != source_digest(KERNEL_SOURCES[kernel]):
+                return None, "the kernel changed since its ncu capture"
+            return float(e["dram_bytes_per_launch"]), e.get("how", "ncu capture")
+    return None, "no ncu capture of this kernel at this workload and partition length"
 
 
 def measured_peak_tensor():
@@ -324,7 +334,8 @@ def oracle_sample_setup(spec, max_seqs=None):
     from dataclasses import replace
     from oracle.allocator import BlockManager
     sp = spec
-    if max_seqs is not None and spec.kind == "independent" and max_seqs < spec.num_seqs:
+    if max_seqs is not None and spec.kind in ("independent", "shared_prefix") and \
+            max_seqs < spec.num_seqs:
         sp = replace(spec, num_seqs=max_seqs)
     sp = replace(sp, num_blocks=None)
     sc = W.scenario(sp)
@@ -362,7 +373,10 @@ def time_oracle(spec, budget_s=15.0, steps=None, per_step_budget_s=None):
     (GB/s, seconds per sampled step, threads, sample description)."""
     import oracle
     nthreads = oracle.max_threads()
-    max_seqs = min(spec.num_seqs, 16) if spec.kind == "independent" else None
+    # a bounded sample: the first 16 sequences of an independent batch, the
+    # first 4 requests (with their shared prefix) of a shared-prefix batch
+    max_seqs = {"independent": min(spec.num_seqs, 16),
+                "shared_prefix": min(spec.num_seqs, 4)}.get(spec.kind)
     sp, q, kc, vc, tables, lens = oracle_sample_setup(spec, max_seqs)
     B = len(lens)
     rows_all = np.array([(b, h) for b in range(B) for h in range(sp.Hq)], dtype=np.int64)
@@ -610,7 +624,7 @@ def run_ours(args):
     alg = unique + other
     achieved = alg / (part_avg * 1e-3) / 1e9
     kname = partition_kernel(spec, P)
-    traffic = profiled_traffic(args.workload, kname)
+    traffic, traffic_note = profiled_traffic(args.workload, kname, P)
 
     result = None
     if rank == 0:
@@ -635,6 +649,10 @@ def run_ours(args):
                 "num_seqs": len(sc.batch), "num_heads": spec.Hq, "num_kv_heads": spec.Hkv,
                 "head_size": spec.D, "block_size": spec.block_size, "num_blocks": sc.num_blocks,
                 "max_context_len": max_ctx, "partition_size": P, "num_partitions": n_part,
+                "split_k": (f"{n_part} partitions of {P} tokens at the longest context; the reduce "
+                            "kernel merges them" if n_part > 1 else
+                            f"one partition of {P} tokens covers every sequence: no split-K "
+                            "reduce launch"),
                 "kv_bytes_unique": unique, "kv_bytes_logical": logical,
                 "new_tokens_per_step": int(key.shape[0]), "cow_pairs_per_step": int(pairs.shape[0]),
                 "l2": ("L2 flushed between timed steps (252 MB streamed read, excluded from the step time)"
@@ -655,6 +673,7 @@ def run_ours(args):
                 "unit": "GB/s",
                 "frac": round(achieved / peak, 4),
                 "traffic": traffic,
+                "traffic_source": traffic_note,
                 "algorithmic_bytes_per_launch": alg,
             },
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "ms_per_step": round(e2e_ms, 6),

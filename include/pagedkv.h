@@ -247,7 +247,10 @@ pa_status pa_decode_reduce(void* out, const int32_t* context_lens, int num_seqs,
  *     with PA_ERR_UNSUPPORTED (and a message) before any launch.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is looked up again when the
+ *     device's current context is a different one (after cudaDeviceReset the
+ *     library's device code is loaded anew); make the first call after such a
+ *     reset before any capture as well.
  *   - All calls on a device share the one array, which keeps the last call's
  *     contents.  Nothing in it needs to start at zero (each call writes every
  *     partial it reads), but calls that overlap on the GPU -- on different

@@ -569,8 +569,13 @@ extern "C" pa_status pa_decode_multi(void* out, const void* q, const void* k_cac
   if (!status) return PA_ERR_CUDA;
   // few queries per sequence: token-major (tokens as the MMA's M, query tokens x
   // heads as its N); else query-major, as a prefill kernel
-  const int err = pa::decode_mq_tc_supported(a) ? pa::launch_decode_mq_tc(a, status, stream)
-                                                : pa::launch_decode_mq(a, status, stream);
+  // The token-major kernel writes a sequence's outputs directly exactly when
+  // its whole context fits one partition (all its query tokens form one run);
+  // the query-major kernel decides per block of kMqRows / G query tokens.
+  const bool token_major = pa::decode_mq_tc_supported(a);
+  a.direct_qblock = token_major ? max_query_len : pa::kMqRows / G;
+  const int err = token_major ? pa::launch_decode_mq_tc(a, status, stream)
+                              : pa::launch_decode_mq(a, status, stream);
   pa_status st = launch_status(fn, err, 1);
   if (st != PA_OK || NP <= 1) return st;
   return launch_status(fn, pa::launch_decode_mq_reduce(a, stream), 1);

@@ -445,6 +445,7 @@ struct ReduceParams {
   const float* ws_o;
   const float* ws_m;
   const float* ws_l;
+  int64_t table_cap;  // tokens a block-table row holds (max_blocks * block_size), or INT64_MAX
   int num_seqs, Hq, partition_size, num_partitions;
 };
 
@@ -461,8 +462,11 @@ __global__ void __launch_bounds__(128) decode_reduce_kernel(const ReduceParams p
   const int b = static_cast<int>(row / p.Hq);
   int L = p.context_lens[b];
   L = L < 0 ? 0 : L;
-  const int64_t grid_cap = static_cast<int64_t>(p.num_partitions) * p.partition_size;
-  if (L > grid_cap) L = static_cast<int>(grid_cap);  // flagged by the partition kernel
+  // the partition kernels serve at most min(table row, partition grid) tokens
+  // (longer contexts are flagged there); read only the partials they wrote
+  int64_t cap = static_cast<int64_t>(p.num_partitions) * p.partition_size;
+  cap = p.table_cap < cap ? p.table_cap : cap;
+  if (L > cap) L = static_cast<int>(cap);
   const int np = (L + p.partition_size - 1) / p.partition_size;
   if (np <= 1) return;  // written directly by the partition kernel
   const int64_t base = row * p.num_partitions;
@@ -565,6 +569,7 @@ cudaError_t launch_reduce_t(const DecodeArgs& a, cudaStream_t stream) {
   p.ws_o = a.workspace;
   p.ws_m = a.workspace + rows * a.D;
   p.ws_l = a.workspace + rows * (a.D + 1);
+  p.table_cap = a.max_blocks > 0 ? a.max_blocks * a.block_size : INT64_MAX;
   p.num_seqs = a.num_seqs;
   p.Hq = a.Hq;
   p.partition_size = a.partition_size;

@@ -512,7 +512,8 @@ struct MqReduceParams {
   const float* ws_o;
   const float* ws_m;
   const float* ws_l;
-  int num_seqs, total_q, Hq, G, partition_size, num_partitions;
+  int num_seqs, total_q, Hq, partition_size, num_partitions;
+  int direct_qblock;  // query-token run length of the partition launcher (MqArgs)
 };
 
 // One warp per (query token, head) whose block spanned several partitions.
@@ -535,7 +536,9 @@ __global__ void __launch_bounds__(128) decode_mq_reduce_kernel(const MqReducePar
   const int L = p.context_lens[b];
   const int i = t - p.query_start[b];
   if (Qb <= 0 || Qb > L || i < 0 || i >= Qb) return;   // flagged by the partition kernel
-  const int QB = MR / p.G;
+  // the run of query tokens token i was served in (the partition launcher's
+  // grouping), and that run's last key position
+  const int QB = p.direct_qblock;
   const int i_last = min(Qb, (i / QB + 1) * QB) - 1;
   const int pmax = L - Qb + i_last;
   if (pmax < p.partition_size) return;              // written directly
@@ -617,7 +620,7 @@ cudaError_t launch_mq_reduce_t(const MqArgs& a, cudaStream_t stream) {
   p.num_seqs = a.num_seqs;
   p.total_q = a.total_q;
   p.Hq = a.Hq;
-  p.G = a.Hq / a.Hkv;
+  p.direct_qblock = a.direct_qblock > 0 ? a.direct_qblock : MR / (a.Hq / a.Hkv);
   p.partition_size = a.partition_size;
   p.num_partitions = a.num_partitions;
   const int64_t warps = static_cast<int64_t>(a.total_q) * a.Hq;

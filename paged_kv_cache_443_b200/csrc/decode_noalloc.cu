@@ -13,7 +13,11 @@
 // The array lives in every GPU that loads the library, until the process
 // exits.  In host code its name is only a host-side stand-in, so the kernels
 // are given the device address that cudaGetSymbolAddress returns for the
-// current device; that lookup runs on the first call made on each device.
+// current device; that lookup runs on the first call made on each device, and
+// again whenever the device's current context is not the one the address was
+// looked up in (after cudaDeviceReset the module is loaded anew, possibly at
+// another address).
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -29,11 +33,41 @@ constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
 __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
 
 constexpr int kMaxDevices = 64;
-float* g_scratch_addr[kMaxDevices] = {};
+struct ScratchAddr {
+  float* ptr = nullptr;
+  unsigned long long ctx_id = 0;  // context the address belongs to (0: unknown)
+};
+ScratchAddr g_scratch[kMaxDevices];
 std::mutex g_scratch_mu;
 
-// Device address of g_noalloc_scratch on the current device (looked up once
-// per device, with that device current).  nullptr on a CUDA error.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current CUDA context; false when there is
+// none yet or the driver does not offer the query.
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(f);
+  });
+  CUcontext ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS && *id != 0;
+}
+
+// Device address of g_noalloc_scratch in the current device's current context
+// (looked up with that device current, and cached per device and context).
+// nullptr on a CUDA error.
 float* scratch_address() {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -41,15 +75,21 @@ float* scratch_address() {
     pa::fail(PA_ERR_CUDA, "pa_decode_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
     return nullptr;
   }
+  unsigned long long ctx = 0;
+  const bool known = current_context_id(&ctx);
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (g_scratch_addr[dev]) return g_scratch_addr[dev];
+  ScratchAddr& c = g_scratch[dev];
+  if (c.ptr && known && c.ctx_id == ctx) return c.ptr;
   float* ptr = nullptr;
   e = cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_noalloc_scratch);
   if (e != cudaSuccess || ptr == nullptr) {
     pa::fail(PA_ERR_CUDA, "pa_decode_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
     return nullptr;
   }
-  g_scratch_addr[dev] = ptr;
+  // the lookup made the device's primary context current if none was; without
+  // a context id every call looks the address up again
+  c.ptr = ptr;
+  c.ctx_id = current_context_id(&ctx) ? ctx : 0;
   return ptr;
 }
 

@@ -97,6 +97,11 @@ struct MqArgs {
   int partition_size, num_partitions;
   float scale;
   pa_dtype dtype;
+  // Set by the partition launcher for the reduce: the partition kernel groups a
+  // sequence's query tokens in runs of this many (from the first) and writes a
+  // run's outputs directly, with no partials, when its last query token's last
+  // key lies in the first partition.
+  int direct_qblock = 0;
 };
 constexpr int kMqRows = 128;  // (query token, head) rows per CTA of the multi-query kernel
 int launch_decode_mq(const MqArgs& a, unsigned int* status, void* stream);

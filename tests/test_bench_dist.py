@@ -72,17 +72,24 @@ def test_step_bytes_unique_and_logical():
 
 
 def test_profile_digest_gates_traffic(tmp_path, monkeypatch):
-    d = bench.source_digest()
+    import json
+    d = bench.source_digest(bench.KERNEL_SOURCES["decode_partition_tc_kernel"])
     prof = tmp_path / "profiles"
     prof.mkdir()
-    (prof / "decode_partition_x.md").write_text(f"traffic_bytes_per_launch: 123\nsource_digest: {d}\n")
-    (prof / "decode_partition_y.md").write_text("traffic_bytes_per_launch: 123\nsource_digest: 0000\n")
+    k = "decode_partition_tc_kernel"
+    caps = [dict(workload="x", kernel=k, partition_size=512, source_digest=d,
+                 dram_bytes_per_launch=123, how="full launch"),
+            dict(workload="y", kernel=k, partition_size=512, source_digest="0000",
+                 dram_bytes_per_launch=123)]
+    (prof / "dram_traffic.json").write_text(json.dumps({"captures": caps}))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     # the digest is computed from the sources under ROOT; point it back at the repo
     monkeypatch.setattr(bench, "source_digest", lambda files=None: d)
-    assert bench.profiled_traffic("x") == 123.0
-    assert bench.profiled_traffic("y") is None
-    assert bench.profiled_traffic("z") is None
+    assert bench.profiled_traffic("x", k, 512) == (123.0, "full launch")
+    assert bench.profiled_traffic("x", k, 4096)[0] is None     # another launch configuration
+    assert bench.profiled_traffic("x", "decode_partition_kernel", 512)[0] is None
+    assert bench.profiled_traffic("y", k, 512)[0] is None      # kernel changed since
+    assert bench.profiled_traffic("z", k, 512)[0] is None
 
 
 def test_partition_kernel_choice():

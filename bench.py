@@ -458,7 +458,18 @@ def run_ours(args):
     if P == 0:   # the workload leaves it to the library: use pa_decode's automatic length
         auto = pk.pa_decode_fp8_auto_partition_size if spec.fp8 else pk.pa_decode_auto_partition_size
         P = auto(len(sc.batch), spec.Hq, spec.Hkv, spec.D, spec.dtype_code, max_ctx)
-    ws = cache.workspace(q.shape[0], q.shape[1], max_ctx, P)
+    # families sharing leading blocks (parallel samples, a common prefix) are
+    # decoded with each family's shared span read once, unless --grouped off
+    groups = None
+    if args.grouped == "on" or (args.grouped == "auto" and spec.kind != "independent"
+                                and not spec.fp8):
+        groups = cache.groups(tables, lens)
+        if groups.max_shared_len == 0:
+            groups = None
+    if groups is not None:
+        ws = cache.grouped_workspace(q.shape[0], q.shape[1], max_ctx, groups, P)
+    else:
+        ws = cache.workspace(q.shape[0], q.shape[1], max_ctx, P)
     scale = spec.softmax_scale
     n_part = pk.pa_decode_num_partitions(max_ctx, P)
     stream = torch.cuda.current_stream(device)
@@ -480,6 +491,14 @@ def run_ours(args):
             pk.pa_reshape_and_cache(key, value, kc, vc, slots, stream=stream)
         if ev is not None:
             ev[1].record(stream)
+        if groups is not None:
+            # one call: the groups' spans, the rest of each sequence, the reduce
+            pk.pa_decode_grouped(out, q, kc, vc, tables, lens, groups, scale, max_ctx,
+                                 partition_size=P, workspace=ws, stream=stream)
+            if ev is not None:
+                ev[2].record(stream)
+                ev[3].record(stream)
+            return
         if spec.fp8:
             pk.pa_decode_partitions_fp8(out, q, kc, vc, tables, lens, scale, max_ctx, spec.k_scale,
                                         spec.v_scale, partition_size=P, workspace=ws,
@@ -570,7 +589,7 @@ def run_ours(args):
         cache.copy_on_write(d_pairs, stream=st)
         cache.store(d_key, d_value, d_slots, stream=st)
         cache.decode(d_q, d_tables, d_lens, max_ctx, scale, out=out, partition_size=P,
-                     workspace=ws, stream=st)
+                     workspace=ws, stream=st, groups=groups)
         h_out.copy_(out, non_blocking=True)
 
     def time_e2e(step_fn):
@@ -625,6 +644,12 @@ def run_ours(args):
     achieved = alg / (part_avg * 1e-3) / 1e9
     kname = partition_kernel(spec, P)
     traffic, traffic_note = profiled_traffic(args.workload, kname, P)
+    if groups is not None:
+        # the three launches of the grouped decode are timed together (the
+        # reduce included), against the same algorithmic bytes
+        kname = ("decode_grouped: decode_partition_tc_kernel (shared spans, 16/G members per "
+                 "CTA) + " + partition_kernel(spec, P) + " (rest) + decode_reduce_kernel")
+        traffic, traffic_note = None, "three kernels timed together; see the ncu launch list"
 
     result = None
     if rank == 0:
@@ -658,12 +683,19 @@ def run_ours(args):
                 "l2": ("L2 flushed between timed steps (252 MB streamed read, excluded from the step time)"
                        if flush else f"inputs larger than L2: {unique / 1e9:.2f} GB of KV per step"),
                 "parallelism": "replicas" if world == 1 else f"replicas x{world} (no collective)",
+                "decode": (f"grouped: {groups.num_groups} families sharing up to "
+                           f"{groups.max_shared_len} leading tokens, each shared span read once "
+                           f"for its members (pa_decode_grouped)" if groups is not None
+                           else "pa_decode_partitions + pa_decode_reduce"),
             },
-            "kernels_us": {  # from the second pass, with events between the kernels
+            "kernels_us": ({  # from the second pass, with events between the kernels
                 "append_and_copy": round(float(np.mean(app_ms)) * 1e3, 3),
                 "decode_partitions": round(part_avg * 1e3, 3),
                 "decode_reduce": round(float(np.mean(red_ms)) * 1e3, 3),
-            },
+            } if groups is None else {
+                "append_and_copy": round(float(np.mean(app_ms)) * 1e3, 3),
+                "decode_grouped": round(part_avg * 1e3, 3),
+            }),
             "roofline": {
                 "kernel": kname,
                 "bound": "hbm",
@@ -950,6 +982,9 @@ def main():
     ap.add_argument("--op", default="decode", choices=["decode", "swap", "mq"],
                     help="decode: the hot path (default); swap: block swap bandwidth")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--grouped", default="auto", choices=["auto", "on", "off"],
+                    help="decode families sharing leading blocks with pa_decode_grouped "
+                         "(auto: for parallel-sampling and shared-prefix workloads)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank, world, _ = dist_env()

@@ -264,6 +264,51 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache, const
                             float scale, pa_dtype dtype, int partition_size, int max_context_len,
                             void* stream);
 
+/*
+ * Decode of sequences that share leading blocks ([P1] "블록 공유": parallel
+ * samples of one prompt, or requests with a common prefix, point at the same
+ * physical blocks).  The result is that of pa_decode on the same arguments;
+ * what changes is the work: the shared span of a group is read once for all
+ * its members, whose queries form the columns of one tensor-core tile (each
+ * column a (member, query head) pair, 16 / G members per CTA), instead of once
+ * per member.  Each member's remaining tokens are decoded as in pa_decode, and
+ * a reduce merges both parts with one softmax over all of the sequence's
+ * tokens ([P1] "PagedAttention의 설계").
+ *
+ *   group_start   [num_groups + 1] int32 (device): group i is sequences
+ *                 group_start[i] .. group_start[i+1]-1 (consecutive in the
+ *                 batch); 0 = group_start[0] <= ... <= group_start[num_groups]
+ *                 = num_seqs
+ *   shared_lens   [num_seqs] int32 (device): for each sequence, the tokens at
+ *                 its start that all members of its group share: a multiple of
+ *                 block_size, at most every member's context length, equal for
+ *                 all members of a group, and the table entries of those
+ *                 blocks the same physical blocks for all members (0: nothing
+ *                 shared)
+ *   max_group_size, max_shared_len  upper bounds of the group sizes and of
+ *                 shared_lens (size the grid and the workspace)
+ *   workspace     pa_decode_grouped_workspace_bytes(...) bytes, 16-byte aligned
+ * Other arguments as pa_decode (partition_size 0 = its automatic length).
+ * pa_build_groups computes the groups from host block tables.  Device-side
+ * checks: inconsistent groups (offsets out of order, members whose shared_lens
+ * differ or exceed their context, a length not a multiple of block_size) set
+ * PA_DEVERR_CONTEXT.  With max_shared_len = 0 or num_groups = 0 this is
+ * pa_decode; so it is for f32 / head size 64, where no tensor-core kernel
+ * serves the shared span.  Three launches: the groups' spans, the rest of each
+ * sequence, the reduce.
+ */
+size_t pa_decode_grouped_workspace_bytes(int num_seqs, int num_heads, int head_size,
+                                         int max_context_len, int max_shared_len,
+                                         int partition_size);
+pa_status pa_decode_grouped(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, int max_blocks_per_seq,
+                            const int32_t* context_lens, const int32_t* group_start,
+                            const int32_t* shared_lens, int num_groups, int max_group_size,
+                            int max_shared_len, int num_seqs, int num_heads, int num_kv_heads,
+                            int head_size, int block_size, int num_blocks, float scale,
+                            pa_dtype dtype, int partition_size, int max_context_len,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Cache updates                                                           */
 
@@ -504,6 +549,23 @@ pa_status pa_seq_num_tokens(const pa_allocator* a, int64_t seq_id, int* out);
 pa_status pa_build_tables(const pa_allocator* a, const int64_t* seq_ids, int num_seqs,
                           int max_blocks_per_seq, int32_t* block_tables_out,
                           int32_t* context_lens_out);
+
+/*
+ * Shared-prefix groups of a decode batch for pa_decode_grouped, from its host
+ * block tables (the rows pa_build_tables writes) and context lengths.
+ * Consecutive sequences whose first block is the same physical block (and
+ * holds a whole block of each one's tokens) form a group; its shared length
+ * is the longest run of leading table entries all members have in common,
+ * within the whole blocks every member's context covers, times block_size.  A
+ * group of one shares nothing (0).  Host memory only:
+ *   group_start_out [num_seqs + 1], shared_lens_out [num_seqs];
+ *   *num_groups_out, *max_group_size_out, *max_shared_len_out.
+ * PA_ERR_INVALID for a context length outside [0, max_blocks_per_seq * bs].
+ */
+pa_status pa_build_groups(const int32_t* block_tables, int num_seqs, int max_blocks_per_seq,
+                          const int32_t* context_lens, int block_size, int32_t* group_start_out,
+                          int32_t* shared_lens_out, int* num_groups_out, int* max_group_size_out,
+                          int* max_shared_len_out);
 
 #ifdef __cplusplus
 }

@@ -38,6 +38,7 @@ EXPORTS = (
     "pa_alloc_refcount", "pa_alloc_free_stack", "pa_seq_add", "pa_seq_fork", "pa_seq_append",
     "pa_seq_free", "pa_seq_move", "pa_seq_num_tokens", "pa_build_tables",
     "pa_alloc_enable_prefix_cache", "pa_alloc_evictable", "pa_seq_add_cached", "pa_seq_commit",
+    "pa_decode_grouped", "pa_decode_grouped_workspace_bytes", "pa_build_groups",
 )
 
 
@@ -115,6 +116,11 @@ def lib():
         "pa_seq_commit": ([vp, i64, pi32, i32], i32),
         "pa_seq_num_tokens": ([vp, i64, ctypes.POINTER(i32)], i32),
         "pa_build_tables": ([vp, pi64, i32, i32, pi32, pi32], i32),
+        "pa_decode_grouped": ([vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                               i32, i32, i32, f32, i32, i32, i32, vp, sz, vp], i32),
+        "pa_decode_grouped_workspace_bytes": ([i32, i32, i32, i32, i32, i32], sz),
+        "pa_build_groups": ([pi32, i32, i32, pi32, i32, pi32, pi32, ctypes.POINTER(i32),
+                             ctypes.POINTER(i32), ctypes.POINTER(i32)], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -248,6 +254,56 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_c
     _check(lib().pa_decode(*_decode_args(out, q, k_cache, v_cache, block_tables, context_lens,
                                          scale, partition_size, max_context_len, workspace,
                                          stream)))
+
+
+class Groups:
+    """Shared-prefix groups of a decode batch (pa_build_groups): group_start
+    [num_groups + 1] and shared_lens [B] int32 tensors, and their bounds."""
+
+    def __init__(self, group_start, shared_lens, num_groups, max_group_size, max_shared_len):
+        self.group_start, self.shared_lens = group_start, shared_lens
+        self.num_groups, self.max_group_size = int(num_groups), int(max_group_size)
+        self.max_shared_len = int(max_shared_len)
+
+    def to(self, device) -> "Groups":
+        return Groups(self.group_start.to(device), self.shared_lens.to(device), self.num_groups,
+                      self.max_group_size, self.max_shared_len)
+
+
+def pa_build_groups(block_tables, context_lens, block_size: int) -> Groups:
+    """Groups of consecutive sequences sharing leading physical blocks, from
+    host (CPU) int32 block tables [B, max_blocks] and context lengths [B]."""
+    import torch
+    t = block_tables.to("cpu", torch.int32).contiguous()
+    l = context_lens.to("cpu", torch.int32).contiguous()
+    B, mb = t.shape
+    gs = torch.empty(B + 1, dtype=torch.int32)
+    sl = torch.empty(max(B, 1), dtype=torch.int32)
+    ng, mg, ms = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    p32 = lambda x: ctypes.cast(x.data_ptr(), ctypes.POINTER(ctypes.c_int32))  # noqa: E731
+    _check(lib().pa_build_groups(p32(t), B, mb, p32(l), int(block_size), p32(gs), p32(sl),
+                                 ctypes.byref(ng), ctypes.byref(mg), ctypes.byref(ms)))
+    return Groups(gs[:ng.value + 1].clone(), sl[:B].clone(), ng.value, mg.value, ms.value)
+
+
+def pa_decode_grouped_workspace_bytes(num_seqs: int, num_heads: int, head_size: int,
+                                      max_context_len: int, max_shared_len: int,
+                                      partition_size: int = 0) -> int:
+    return int(lib().pa_decode_grouped_workspace_bytes(num_seqs, num_heads, head_size,
+                                                       max_context_len, max_shared_len,
+                                                       partition_size))
+
+
+def pa_decode_grouped(out, q, k_cache, v_cache, block_tables, context_lens, groups: Groups, scale,
+                      max_context_len, partition_size=0, workspace=None, stream=None) -> None:
+    """pa_decode's result, with each group's shared span read once for all its
+    members (groups: device tensors, see pa_build_groups)."""
+    a = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, partition_size,
+                     max_context_len, workspace, stream)
+    _contig(groups.group_start, groups.shared_lens)
+    _check(lib().pa_decode_grouped(*a[:7], _ptr(groups.group_start), _ptr(groups.shared_lens),
+                                   groups.num_groups, groups.max_group_size,
+                                   groups.max_shared_len, *a[7:]))
 
 
 def pa_decode_partitions(out, q, k_cache, v_cache, block_tables, context_lens, scale,

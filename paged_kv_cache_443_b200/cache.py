@@ -17,7 +17,8 @@ from typing import List, Optional, Sequence, Tuple
 
 import torch
 
-from . import (BlockAllocator, pa_copy_blocks, pa_decode, pa_decode_fp8,
+from . import (BlockAllocator, Groups, pa_build_groups, pa_copy_blocks, pa_decode,
+               pa_decode_fp8, pa_decode_grouped, pa_decode_grouped_workspace_bytes,
                pa_decode_workspace_bytes, pa_reshape_and_cache, pa_reshape_and_cache_fp8,
                pa_swap_blocks)
 
@@ -137,12 +138,35 @@ class PagedKVCache:
             return None
         return torch.empty(n // 4, dtype=torch.float32, device=self.device)
 
+    def groups(self, block_tables: torch.Tensor, context_lens: torch.Tensor) -> Groups:
+        """Shared-prefix groups of a batch (on this cache's device), from its tables."""
+        return pa_build_groups(block_tables.cpu(), context_lens.cpu(),
+                               self.block_size).to(self.device)
+
+    def grouped_workspace(self, num_seqs: int, num_heads: int, max_context_len: int,
+                          groups: Groups, partition_size: int = 0) -> Optional[torch.Tensor]:
+        n = pa_decode_grouped_workspace_bytes(num_seqs, num_heads, self.head_size,
+                                              max_context_len, groups.max_shared_len,
+                                              partition_size)
+        return torch.empty(n // 4, dtype=torch.float32, device=self.device) if n else None
+
     def decode(self, q: torch.Tensor, block_tables: torch.Tensor, context_lens: torch.Tensor,
                max_context_len: int, scale: float, out: Optional[torch.Tensor] = None,
                partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
-               stream=None) -> torch.Tensor:
+               stream=None, groups: Optional[Groups] = None) -> torch.Tensor:
+        """Decode attention of the batch; with `groups` (self.groups(...)) each
+        group's shared leading blocks are read once for all its members (16-bit
+        caches; the result is the same)."""
         if out is None:
             out = torch.empty_like(q)
+        if groups is not None and not self.fp8:
+            if workspace is None:
+                workspace = self.grouped_workspace(q.shape[0], q.shape[1], max_context_len,
+                                                   groups, partition_size)
+            pa_decode_grouped(out, q, self.k_cache, self.v_cache, block_tables, context_lens,
+                              groups, scale, max_context_len, partition_size=partition_size,
+                              workspace=workspace, stream=stream)
+            return out
         if workspace is None:
             workspace = self.workspace(q.shape[0], q.shape[1], max_context_len, partition_size)
         if self.fp8:

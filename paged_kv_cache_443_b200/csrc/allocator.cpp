@@ -414,3 +414,50 @@ extern "C" pa_status pa_build_tables(const pa_allocator* a, const int64_t* seq_i
   }
   return PA_OK;
 }
+
+extern "C" pa_status pa_build_groups(const int32_t* block_tables, int num_seqs,
+                                     int max_blocks_per_seq, const int32_t* context_lens,
+                                     int block_size, int32_t* group_start_out,
+                                     int32_t* shared_lens_out, int* num_groups_out,
+                                     int* max_group_size_out, int* max_shared_len_out) {
+  if (num_seqs < 0 || max_blocks_per_seq <= 0 || block_size <= 0 || !group_start_out ||
+      !num_groups_out || !max_group_size_out || !max_shared_len_out ||
+      (num_seqs > 0 && (!block_tables || !context_lens || !shared_lens_out)))
+    return pa::fail(PA_ERR_INVALID, "pa_build_groups: bad argument");
+  for (int b = 0; b < num_seqs; ++b)
+    if (context_lens[b] < 0 ||
+        static_cast<int64_t>(context_lens[b]) > static_cast<int64_t>(max_blocks_per_seq) * block_size)
+      return pa::fail(PA_ERR_INVALID, "pa_build_groups: context length %d of sequence %d out of range",
+                      context_lens[b], b);
+  auto row = [&](int b) { return block_tables + static_cast<int64_t>(b) * max_blocks_per_seq; };
+  // whole blocks of sequence b that hold only its tokens' slots it uses
+  auto full_blocks = [&](int b) { return context_lens[b] / block_size; };
+  int ng = 0, max_size = 0, max_shared = 0;
+  int b0 = 0;
+  while (b0 < num_seqs) {
+    // members: the following sequences whose first block is b0's first block
+    int b1 = b0 + 1;
+    if (full_blocks(b0) > 0)
+      while (b1 < num_seqs && full_blocks(b1) > 0 && row(b1)[0] == row(b0)[0]) ++b1;
+    // the leading entries every member has in common, within every member's
+    // whole blocks
+    int k = full_blocks(b0);
+    for (int m = b0 + 1; m < b1; ++m) {
+      int c = 0;
+      const int lim = k < full_blocks(m) ? k : full_blocks(m);
+      while (c < lim && row(m)[c] == row(b0)[c]) ++c;
+      k = c;
+    }
+    const int shared = b1 - b0 > 1 ? k * block_size : 0;
+    group_start_out[ng++] = b0;
+    for (int m = b0; m < b1; ++m) shared_lens_out[m] = shared;
+    max_size = max_size > b1 - b0 ? max_size : b1 - b0;
+    max_shared = max_shared > shared ? max_shared : shared;
+    b0 = b1;
+  }
+  group_start_out[ng] = num_seqs;
+  *num_groups_out = ng;
+  *max_group_size_out = max_size;
+  *max_shared_len_out = max_shared;
+  return PA_OK;
+}

@@ -580,3 +580,99 @@ extern "C" pa_status pa_decode_multi(void* out, const void* q, const void* k_cac
   if (st != PA_OK || NP <= 1) return st;
   return launch_status(fn, pa::launch_decode_mq_reduce(a, stream), 1);
 }
+
+// ---- shared-prefix groups ----
+
+namespace {
+
+int64_t grouped_span_partitions(int max_shared_len, int P) {
+  return max_shared_len > 0 ? (static_cast<int64_t>(max_shared_len) + P - 1) / P : 0;
+}
+
+}  // namespace
+
+extern "C" size_t pa_decode_grouped_workspace_bytes(int num_seqs, int num_heads, int head_size,
+                                                    int max_context_len, int max_shared_len,
+                                                    int partition_size) {
+  const int P = resolve_partition(partition_size);
+  if (P < 0 || num_seqs < 0 || num_heads < 0 || head_size < 0 || max_shared_len < 0) return 0;
+  const int64_t NPg = grouped_span_partitions(max_shared_len, P);
+  const int64_t NPs = num_partitions(max_context_len, P);
+  if (NPg == 0) return workspace_bytes(num_seqs, num_heads, head_size, NPs);
+  // with a shared span every row is reduced, even one with a single partial
+  const size_t raw = static_cast<size_t>(static_cast<int64_t>(num_seqs) * num_heads * (NPg + NPs) *
+                                         (head_size + 2) * 4);
+  return (raw + 255) / 256 * 256;
+}
+
+extern "C" pa_status pa_decode_grouped(void* out, const void* q, const void* k_cache,
+                                       const void* v_cache, const int32_t* block_tables,
+                                       int max_blocks_per_seq, const int32_t* context_lens,
+                                       const int32_t* group_start, const int32_t* shared_lens,
+                                       int num_groups, int max_group_size, int max_shared_len,
+                                       int num_seqs, int num_heads, int num_kv_heads,
+                                       int head_size, int block_size, int num_blocks,
+                                       float scale, pa_dtype dtype, int partition_size,
+                                       int max_context_len, void* workspace,
+                                       size_t workspace_bytes_in, void* stream) {
+  const char* fn = "pa_decode_grouped";
+  if (partition_size == 0 && num_heads > 0 && num_kv_heads > 0)   // as pa_decode
+    partition_size =
+        auto_partition(num_seqs, num_heads, num_kv_heads, head_size, dtype, max_context_len);
+  const int P = resolve_partition(partition_size);
+  if (num_groups < 0 || max_shared_len < 0 || max_group_size < 0)
+    return pa::fail(PA_ERR_INVALID, "%s: negative group count or size", fn);
+  if (num_groups > num_seqs)
+    return pa::fail(PA_ERR_INVALID, "%s: more groups (%d) than sequences (%d)", fn, num_groups,
+                    num_seqs);
+  if (max_shared_len > max_context_len)
+    return pa::fail(PA_ERR_INVALID, "%s: max_shared_len exceeds max_context_len", fn);
+  if (block_size > 0 && max_shared_len % block_size != 0)
+    return pa::fail(PA_ERR_INVALID, "%s: max_shared_len must be a multiple of block_size", fn);
+  if (num_groups > 0 && max_shared_len > 0 &&
+      (!group_start || !shared_lens || max_group_size < 1 || max_group_size > num_seqs))
+    return pa::fail(PA_ERR_INVALID, "%s: group_start / shared_lens / max_group_size missing", fn);
+  const int64_t NPg = P > 0 ? grouped_span_partitions(max_shared_len, P) : 0;
+  if (num_groups == 0 || NPg == 0)   // nothing shared: the plain decode
+    return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                     num_seqs, num_heads, num_kv_heads, head_size, block_size, num_blocks, scale,
+                     dtype, partition_size, max_context_len, workspace, workspace_bytes_in, stream);
+  // the checks of pa_decode, with the workspace sized for the grouped layout
+  pa::DecodeArgs a;
+  const size_t need = pa_decode_grouped_workspace_bytes(num_seqs, num_heads, head_size,
+                                                        max_context_len, max_shared_len, P);
+  pa_status st = check_decode_full(fn, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                   context_lens, num_seqs, num_heads, num_kv_heads, head_size,
+                                   block_size, num_blocks, scale, dtype, partition_size,
+                                   max_context_len, workspace, workspace_bytes_in, &a);
+  if (st != PA_OK) return st;
+  if (!workspace || workspace_bytes_in < need || !pa::aligned16(workspace))
+    return pa::fail(PA_ERR_INVALID, "%s: a 16-byte aligned workspace of %zu bytes is needed", fn,
+                    need);
+  const int64_t NP = NPg + a.num_partitions;
+  if (NP > 65535) return pa::fail(PA_ERR_UNSUPPORTED, "%s: more than 65535 partitions", fn);
+  if ((reinterpret_cast<uintptr_t>(group_start) & 3u) || (reinterpret_cast<uintptr_t>(shared_lens) & 3u))
+    return pa::fail(PA_ERR_INVALID, "%s: group_start / shared_lens must be 4-byte aligned", fn);
+  a.workspace = static_cast<float*>(workspace);
+  if (!pa::decode_group_tc_supported(a))   // same result without the sharing
+    return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                     num_seqs, num_heads, num_kv_heads, head_size, block_size, num_blocks, scale,
+                     dtype, partition_size, max_context_len, workspace, workspace_bytes_in, stream);
+  const int G = num_heads / num_kv_heads;
+  const int64_t member_runs = (max_group_size + (16 / G) - 1) / (16 / G);
+  if (static_cast<int64_t>(num_groups) * member_runs > 0x7fffffff)
+    return pa::fail(PA_ERR_UNSUPPORTED, "%s: too many groups", fn);
+  unsigned int* status = pa::device_status_word();
+  if (!status) return PA_ERR_CUDA;
+  a.num_partitions = static_cast<int>(NP);
+  a.slot_base = static_cast<int>(NPg);
+  a.seq_shift = shared_lens;
+  a.group_start = group_start;
+  a.num_groups = num_groups;
+  a.max_group_size = max_group_size;
+  st = launch_status(fn, pa::launch_decode_group_tc(a, status, stream), 1);
+  if (st != PA_OK) return st;
+  st = launch_status(fn, launch_partitions(a, status, stream), 1);
+  if (st != PA_OK) return st;
+  return launch_status(fn, pa::launch_decode_reduce(a, status, stream), 1);
+}

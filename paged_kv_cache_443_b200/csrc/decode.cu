@@ -39,6 +39,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "pa_device.cuh"
 #include "pa_internal.h"
@@ -142,6 +143,10 @@ struct PartitionParams {
   int Hq, Hkv, num_blocks, block_size, partition_size, num_partitions;
   float scale_log2;  // scale * log2(e) (* k_scale for E4M3 caches)
   float v_scale;     // E4M3 caches: the value scale (1 otherwise, unused)
+  // shared-prefix groups: seq_shift[b] leading tokens of sequence b are served
+  // by its group (nullable = 0); this launch's partials start at slot_base
+  const int32_t* seq_shift;
+  int slot_base;
 };
 
 template <typename TQ, typename TK, int D, int G, int NCW>
@@ -169,16 +174,28 @@ __global__ void __launch_bounds__(Cfg<TK, D, G, NCW>::THREADS)
   int L = p.context_lens[b];
   const int P = p.partition_size;
   // longest context this launch can serve: the table row and the partition grid
-  int64_t cap = p.max_blocks * p.block_size;
-  const int64_t grid_cap = static_cast<int64_t>(p.num_partitions) * P;
-  cap = cap < grid_cap ? cap : grid_cap;
+  const int64_t cap = p.max_blocks * p.block_size;
   if (L < 0 || L > cap) {
     if (threadIdx.x == 0 && part == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
     L = L < 0 ? 0 : static_cast<int>(cap);
   }
+  int shift = 0;           // leading tokens its group serves
+  if (p.seq_shift != nullptr) {
+    shift = p.seq_shift[b];
+    if (shift < 0 || shift % p.block_size != 0 || shift > L) {
+      if (threadIdx.x == 0 && part == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
+      shift = 0;
+    }
+    L -= shift;
+  }
+  const int64_t grid_cap = static_cast<int64_t>(p.num_partitions - p.slot_base) * P;
+  if (L > grid_cap) {
+    if (threadIdx.x == 0 && part == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
+    L = static_cast<int>(grid_cap);
+  }
   const int start = part * P;
   if (L == 0) {
-    if (part == 0) {
+    if (part == 0 && shift == 0) {
       TQ* o = static_cast<TQ*>(p.out) + (static_cast<int64_t>(b) * p.Hq + g * G) * D;
       for (int i = threadIdx.x; i < G * D; i += C::THREADS) o[i] = EQ::from_float(0.f);
     }
@@ -187,7 +204,7 @@ __global__ void __launch_bounds__(Cfg<TK, D, G, NCW>::THREADS)
   if (start >= L) return;
   const int end = min(L, start + P);
   const int n_tiles = (end - start + C::TOK - 1) / C::TOK;
-  const bool single = (L <= P);
+  const bool single = (L <= P) && shift == 0;
 
   if (threadIdx.x == 0) {
 #pragma unroll
@@ -208,7 +225,8 @@ __global__ void __launch_bounds__(Cfg<TK, D, G, NCW>::THREADS)
     const uint32_t blk_bytes = static_cast<uint32_t>(bs) * C::ROW_BYTES;
     const int64_t head_off = static_cast<int64_t>(g) * blk_bytes;
     const int64_t blk_stride = static_cast<int64_t>(p.Hkv) * blk_bytes;
-    const int32_t* trow = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
+    const int32_t* trow =
+        p.block_tables + static_cast<int64_t>(b) * p.max_blocks + shift / p.block_size;
     const char* kbase = static_cast<const char*>(p.k_cache) + head_off;
     const char* vbase = static_cast<const char*>(p.v_cache) + head_off;
     int cached = -1;
@@ -429,7 +447,7 @@ __global__ void __launch_bounds__(Cfg<TK, D, G, NCW>::THREADS)
     if (single) {
       static_cast<TQ*>(p.out)[hq * D + d] = EQ::from_float(O / Ls);
     } else {
-      const int64_t slot = hq * p.num_partitions + part;
+      const int64_t slot = hq * p.num_partitions + p.slot_base + part;
       p.ws_o[slot * D + d] = O;
       if (d == 0) {
         p.ws_m[slot] = M;
@@ -447,6 +465,11 @@ struct ReduceParams {
   const float* ws_l;
   int64_t table_cap;  // tokens a block-table row holds (max_blocks * block_size), or INT64_MAX
   int num_seqs, Hq, partition_size, num_partitions;
+  // shared-prefix groups: sequence b's first seq_shift[b] tokens were served
+  // by its group, whose partials fill slots [0, ceil(shift / P)); the rest of
+  // the sequence's partials start at slot_rest (nullable: no groups, 0)
+  const int32_t* seq_shift;
+  int slot_rest;
 };
 
 // One warp per (sequence, query head) with more than one partition:
@@ -464,28 +487,65 @@ __global__ void __launch_bounds__(128) decode_reduce_kernel(const ReduceParams p
   L = L < 0 ? 0 : L;
   // the partition kernels serve at most min(table row, partition grid) tokens
   // (longer contexts are flagged there); read only the partials they wrote
-  int64_t cap = static_cast<int64_t>(p.num_partitions) * p.partition_size;
-  cap = p.table_cap < cap ? p.table_cap : cap;
-  if (L > cap) L = static_cast<int>(cap);
-  const int np = (L + p.partition_size - 1) / p.partition_size;
-  if (np <= 1) return;  // written directly by the partition kernel
+  if (L > p.table_cap) L = static_cast<int>(p.table_cap);
+  int S = p.seq_shift ? p.seq_shift[b] : 0;   // tokens its group served
+  if (S < 0 || S > L) S = 0;                  // flagged by the partition kernel
+  const int P = p.partition_size;
+  int64_t rest = L - S;
+  const int64_t cap = static_cast<int64_t>(p.num_partitions - p.slot_rest) * P;
+  if (rest > cap) rest = cap;
+  const int np_a = (S + P - 1) / P;           // the group's partials of the shared span
+  const int np = np_a + static_cast<int>((rest + P - 1) / P);
+  if (S == 0 && np <= 1) return;  // written directly by the partition kernel
+  // partial i of the row: the group's span first, then the rest of the sequence
+  auto slot = [&](int i) { return i < np_a ? i : p.slot_rest + (i - np_a); };
   const int64_t base = row * p.num_partitions;
   float M = -INFINITY;
-  for (int i = lane; i < np; i += 32) M = fmaxf(M, p.ws_m[base + i]);
+  for (int i = lane; i < np; i += 32) M = fmaxf(M, p.ws_m[base + slot(i)]);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, off));
   float Ls = 0.f;
-  for (int i = lane; i < np; i += 32) Ls += p.ws_l[base + i] * exp2f(p.ws_m[base + i] - M);
+  for (int i = lane; i < np; i += 32)
+    Ls += p.ws_l[base + slot(i)] * exp2f(p.ws_m[base + slot(i)] - M);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) Ls += __shfl_xor_sync(FULL_MASK, Ls, off);
+  // The weighted outputs, in partition order.  Only partials with a finite
+  // max carry weight: a CTA that streamed several partitions left empty ones
+  // (max -inf, sum 0, output 0) in the other slots of its span, whose terms
+  // would add exactly 0, so they are skipped and their outputs never read.
+  // A warp takes 32 slots at a time, finds the live ones with a ballot and
+  // loads up to four of them together.
+  using V = typename std::conditional<DPL == 4, float4, float2>::type;
+  static_assert(DPL == 4 || DPL == 2, "head size 128 or 64");
   float acc[DPL];
 #pragma unroll
   for (int k = 0; k < DPL; ++k) acc[k] = 0.f;
-  for (int i = 0; i < np; ++i) {
-    const float f = exp2f(p.ws_m[base + i] - M);
-    const float* src = p.ws_o + (base + i) * D + lane * DPL;
+  for (int i0 = 0; i0 < np; i0 += 32) {
+    const int i = i0 + lane;
+    const float mi = i < np ? p.ws_m[base + slot(i)] : -INFINITY;
+    const float fi = exp2f(mi - M);
+    unsigned live = __ballot_sync(FULL_MASK, mi != -INFINITY);
+    while (live) {                      // warp-uniform
+      int ks[4];
 #pragma unroll
-    for (int k = 0; k < DPL; ++k) acc[k] = fmaf(f, src[k], acc[k]);
+      for (int u = 0; u < 4; ++u) {
+        ks[u] = live ? __ffs(live) - 1 : -1;
+        live = live ? (live & (live - 1)) : 0u;
+      }
+      V v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (ks[u] >= 0)
+          v[u] = *reinterpret_cast<const V*>(p.ws_o + (base + slot(i0 + ks[u])) * D + lane * DPL);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (ks[u] < 0) break;
+        const float f = __shfl_sync(FULL_MASK, fi, ks[u]);
+        const float* x = reinterpret_cast<const float*>(&v[u]);
+#pragma unroll
+        for (int k = 0; k < DPL; ++k) acc[k] = fmaf(f, x[k], acc[k]);
+      }
+    }
   }
   T* dst = static_cast<T*>(p.out) + row * D + lane * DPL;
   const float inv = 1.f / Ls;
@@ -529,7 +589,9 @@ cudaError_t launch_partition_t(const DecodeArgs& a, unsigned int* status, cudaSt
   p.num_partitions = a.num_partitions;
   p.scale_log2 = a.scale * 1.4426950408889634f * a.k_scale;
   p.v_scale = a.v_scale;
-  dim3 grid(a.num_seqs, a.Hkv, a.num_partitions);
+  p.seq_shift = a.seq_shift;
+  p.slot_base = a.slot_base;
+  dim3 grid(a.num_seqs, a.Hkv, a.num_partitions - a.slot_base);
   return launch_overlapped(kern, grid, dim3(C::THREADS), C::SMEM, stream, p);
 }
 
@@ -570,6 +632,8 @@ cudaError_t launch_reduce_t(const DecodeArgs& a, cudaStream_t stream) {
   p.ws_m = a.workspace + rows * a.D;
   p.ws_l = a.workspace + rows * (a.D + 1);
   p.table_cap = a.max_blocks > 0 ? a.max_blocks * a.block_size : INT64_MAX;
+  p.seq_shift = a.seq_shift;
+  p.slot_rest = a.slot_base;
   p.num_seqs = a.num_seqs;
   p.Hq = a.Hq;
   p.partition_size = a.partition_size;

@@ -92,6 +92,15 @@ struct TcParams {
   const int32_t* query_start;
   int total_q;
   int q_groups;
+  // Shared-prefix groups (pa_decode_grouped).  seq_shift[b]: tokens at the
+  // start of sequence b that the members of its group share (a multiple of the
+  // block size; nullable = 0).  With group_start set (NQ > 1) a CTA serves the
+  // shared span of group blockIdx.x / q_groups for NQ of its members, each
+  // column a (member, head) pair; otherwise a CTA serves the tokens of its
+  // sequence past seq_shift[b].  Partials go to workspace slots from slot_base.
+  const int32_t* seq_shift;
+  const int32_t* group_start;
+  int slot_base;
 };
 
 // NQ > 1 serves several query tokens per sequence (speculative verification):
@@ -123,7 +132,8 @@ __global__ void __launch_bounds__(THREADS, 2)
   // short partitions do not each pay the pipeline's fill and drain: its partial
   // goes to the first one's slot and the others' slots get empty partials (max
   // -inf, sum 0, output 0), which the reduce weighs by exactly 0.
-  const int b = NQ > 1 ? blockIdx.x / p.q_groups : blockIdx.x;
+  const bool grouped = NQ > 1 && p.group_start != nullptr;   // a group's shared span
+  int b = NQ > 1 ? blockIdx.x / p.q_groups : blockIdx.x;
   const int g = blockIdx.y, part = blockIdx.z * p.parts_per_cta;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int NC = G * NQ;                // S / O columns in use
@@ -131,10 +141,43 @@ __global__ void __launch_bounds__(THREADS, 2)
 
   grid_dependency_wait();   // the appended tokens of the previous kernel are in the cache
   allow_dependents();       // the reduce kernel may start launching
+  const int bs = p.block_size;
+  int gs = 0, ge = 0;       // group mode: the group's members gs .. ge - 1 (gs's table row)
+  if (grouped) {
+    gs = p.group_start[blockIdx.x / p.q_groups];
+    ge = p.group_start[blockIdx.x / p.q_groups + 1];
+    if (gs < 0 || ge < gs || ge > p.total_q) {      // total_q = num_seqs here
+      if (threadIdx.x == 0 && blockIdx.z == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
+      return;
+    }
+    if (gs == ge) return;
+    if (ge - gs > p.q_groups * NQ && blockIdx.x % p.q_groups == 0 && threadIdx.x == 0 &&
+        blockIdx.z == 0 && g == 0)
+      atomicOr(p.status, PA_DEVERR_CONTEXT);    // more members than max_group_size
+    b = gs;
+  }
   int L = p.context_lens[b];
   // this CTA's query tokens: q0 .. q0 + Qb - 1, at positions L - Qall + qoff + c / G
   int q0 = b, Qb = 1, Qall = 1, qoff = 0;
-  if constexpr (NQ > 1) {
+  int shift = 0;            // tokens of the sequence skipped (served by its group)
+  if (grouped) {
+    // members m0 .. m0 + Qb - 1 of the group, all attending to the whole
+    // shared span [0, S) of the first member's table (Qall = 1, qoff = 0 put
+    // every column's causal limit at the span's last token)
+    const int m0 = gs + (blockIdx.x % p.q_groups) * NQ;
+    Qb = min(NQ, ge - m0);
+    if (Qb <= 0) return;
+    const int S = p.seq_shift[gs];
+    bool bad = S < 0 || S % bs != 0 || S > L;
+    for (int m = m0; m < m0 + Qb; ++m)
+      bad |= p.seq_shift[m] != S || p.context_lens[m] < S;
+    if (bad) {
+      if (threadIdx.x == 0 && blockIdx.z == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
+      return;
+    }
+    q0 = m0;
+    L = S;
+  } else if (NQ > 1) {
     const int qg = blockIdx.x % p.q_groups;
     const int qs = p.query_start[b];
     Qall = p.query_start[b + 1] - qs;
@@ -150,15 +193,27 @@ __global__ void __launch_bounds__(THREADS, 2)
   }
   const int P = p.partition_size;
   int64_t cap = p.max_blocks * p.block_size;
-  const int64_t grid_cap = static_cast<int64_t>(p.num_partitions) * P;
-  cap = cap < grid_cap ? cap : grid_cap;
   if (L < 0 || L > cap) {
     if (threadIdx.x == 0 && part == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
     L = L < 0 ? 0 : static_cast<int>(cap);
   }
+  if (NQ == 1 && p.seq_shift != nullptr) {
+    // the tokens past the sequence's shared span (its group serves the span)
+    shift = p.seq_shift[b];
+    if (shift < 0 || shift % bs != 0 || shift > L) {
+      if (threadIdx.x == 0 && part == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
+      shift = 0;
+    }
+    L -= shift;
+  }
+  const int64_t grid_cap = static_cast<int64_t>(p.num_partitions - p.slot_base) * P;
+  if (L > grid_cap) {
+    if (threadIdx.x == 0 && part == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
+    L = static_cast<int>(grid_cap);
+  }
   const int start = part * P;
   if (L == 0) {
-    if (NQ == 1 && part == 0) {
+    if (NQ == 1 && part == 0 && shift == 0) {
       T* o = static_cast<T*>(p.out) + (static_cast<int64_t>(b) * p.Hq + g * G) * DH;
       for (int i = threadIdx.x; i < G * DH; i += THREADS) o[i] = Elem<T>::from_float(0.f);
     }
@@ -168,16 +223,17 @@ __global__ void __launch_bounds__(THREADS, 2)
   const int end = static_cast<int>(
       min(static_cast<int64_t>(L), start + static_cast<int64_t>(P) * p.parts_per_cta));
   const int n_tiles = (end - start + TOK - 1) / TOK;
-  const bool single = (L <= P);
+  // the output directly, or partials for the reduce (always for a group's span
+  // and for a sequence whose first tokens its group served)
+  const bool single = (L <= P) && !grouped && shift == 0;
   const int n_slots = min(p.parts_per_cta, (L + P - 1) / P - part);   // partials this CTA writes
 
   // ---- set-up: the producer starts streaming right after the barrier, while
   // the softmax warps stage Q^T and the MMA issuer waits for it ----
-  const int bs = p.block_size;
   const int bpt = TOK / bs;                              // blocks per tile: 4, 8 or 16
   const int first_blk = start / bs;
   const int last_blk = (end + bs - 1) / bs;
-  const int32_t* trow = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
+  const int32_t* trow = p.block_tables + static_cast<int64_t>(b) * p.max_blocks + shift / bs;
   int pb_first = -1;                                     // tile 0's table entries, read early
   if (warp == 0) {
     if (lane < min(bpt, last_blk - first_blk)) pb_first = __ldg(trow + first_blk + lane);
@@ -374,7 +430,7 @@ __global__ void __launch_bounds__(THREADS, 2)
           if (single) {
             static_cast<T*>(p.out)[hq * DH + r] = Elem<T>::from_float(o[h] / Ls);
           } else {
-            const int64_t slot = hq * p.num_partitions + part;
+            const int64_t slot = hq * p.num_partitions + p.slot_base + part;
             p.ws_o[slot * DH + r] = o[h];
             if (r == 0) {
               p.ws_m[slot] = m_run[h];
@@ -532,7 +588,61 @@ cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t 
   p.query_start = nullptr;
   p.total_q = a.num_seqs;
   p.q_groups = 1;
-  dim3 grid(a.num_seqs, a.Hkv, (a.num_partitions + p.parts_per_cta - 1) / p.parts_per_cta);
+  p.seq_shift = a.seq_shift;
+  p.group_start = nullptr;
+  p.slot_base = a.slot_base;
+  const int np = a.num_partitions - a.slot_base;
+  dim3 grid(a.num_seqs, a.Hkv, (np + p.parts_per_cta - 1) / p.parts_per_cta);
+  return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
+}
+
+// The shared spans of shared-prefix groups: NQ = 16 / G members per CTA, each
+// column a (member, head) pair, one CTA per (group, run of NQ members, kv
+// head, run of span partitions); partials into every member's slots from 0.
+template <typename T, int G>
+cudaError_t launch_group_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
+  constexpr int NQ = NPAD / G;
+  auto kern = decode_partition_tc_kernel<T, G, NQ>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  CUtensorMap mk, mv;
+  const int64_t groups = static_cast<int64_t>(a.num_blocks) * a.Hkv * a.block_size / 8;
+  const int64_t dims[4] = {64, 8, 2, groups};
+  const int64_t strides[3] = {DH * 2, 128, 8 * DH * 2};
+  const int box[4] = {64, 8, 2, a.block_size / 8};
+  if (!make_tmap(&mk, a.k_cache, 4, dims, strides, box, a.dtype) ||
+      !make_tmap(&mv, a.v_cache, 4, dims, strides, box, a.dtype))
+    return cudaErrorInvalidValue;
+  TcParams p;
+  p.out = a.out;
+  p.q = a.q;
+  p.block_tables = a.block_tables;
+  p.context_lens = a.context_lens;
+  const int64_t nrows = static_cast<int64_t>(a.num_seqs) * a.Hq * a.num_partitions;
+  p.ws_o = a.workspace;
+  p.ws_m = a.workspace + nrows * DH;
+  p.ws_l = a.workspace + nrows * (DH + 1);
+  p.status = status;
+  p.max_blocks = a.max_blocks;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.num_blocks = a.num_blocks;
+  p.block_size = a.block_size;
+  p.partition_size = a.partition_size;
+  p.num_partitions = a.num_partitions;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.query_start = nullptr;
+  p.total_q = a.num_seqs;
+  p.q_groups = (a.max_group_size + NQ - 1) / NQ;
+  p.seq_shift = a.seq_shift;
+  p.group_start = a.group_start;
+  p.slot_base = 0;
+  const int span_parts = a.slot_base;      // the groups' span partitions
+  const int64_t ctas = static_cast<int64_t>(a.num_groups) * p.q_groups * a.Hkv;
+  p.parts_per_cta = tc_parts_per_cta(ctas * span_parts, a.partition_size, span_parts);
+  // grid cap of the kernel: the span's partitions (num_partitions - slot_base)
+  p.num_partitions = a.num_partitions;
+  dim3 grid(a.num_groups * p.q_groups, a.Hkv, (span_parts + p.parts_per_cta - 1) / p.parts_per_cta);
   return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
 }
 
@@ -549,15 +659,20 @@ static int sm_count() {
 // Consecutive partitions per CTA (one softmax over them): for partitions
 // shorter than 2048 tokens, the most of 8 / 4 / 2 that keeps a CTA's span
 // within 4096 tokens and still leaves at least 8 CTAs per SM.
-int tc_parts_per_cta(const DecodeArgs& a) {
-  if (a.partition_size >= 2048) return 1;
+int tc_parts_per_cta(int64_t ctas_one_each, int partition_size, int n_parts) {
+  if (partition_size >= 2048 || n_parts <= 0) return 1;
   const int64_t want = 8ll * sm_count();
+  const int64_t rows = ctas_one_each / n_parts;      // CTAs per partition index
   for (int c : {8, 4, 2}) {
-    const int64_t ctas = static_cast<int64_t>(a.num_seqs) * a.Hkv * ((a.num_partitions + c - 1) / c);
-    if (static_cast<int64_t>(a.partition_size) * c <= 4096 && a.num_partitions >= c && ctas >= want)
-      return c;
+    const int64_t ctas = rows * ((n_parts + c - 1) / c);
+    if (static_cast<int64_t>(partition_size) * c <= 4096 && n_parts >= c && ctas >= want) return c;
   }
   return 1;
+}
+
+int tc_parts_per_cta(const DecodeArgs& a) {
+  const int np = a.num_partitions - a.slot_base;
+  return tc_parts_per_cta(static_cast<int64_t>(a.num_seqs) * a.Hkv * np, a.partition_size, np);
 }
 
 namespace {
@@ -642,6 +757,9 @@ cudaError_t launch_tcq_t(const MqArgs& m, unsigned int* status, cudaStream_t str
   p.query_start = m.query_start;
   p.total_q = m.total_q;
   p.q_groups = (m.max_query_len + NQ - 1) / NQ;
+  p.seq_shift = nullptr;
+  p.group_start = nullptr;
+  p.slot_base = 0;
   dim3 grid(m.num_seqs * p.q_groups, m.Hkv, (m.num_partitions + ppc - 1) / ppc);
   return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
 }
@@ -677,6 +795,33 @@ bool decode_tc_supported(const DecodeArgs& a) {
          a.partition_size % TOK == 0 &&
          static_cast<int64_t>(a.num_blocks) * a.Hkv * a.block_size < (int64_t(1) << 31) &&
          encode_fn() != nullptr;
+}
+
+bool decode_group_tc_supported(const DecodeArgs& a) {
+  const int G = a.Hq / a.Hkv;
+  return (a.dtype == PA_F16 || a.dtype == PA_BF16) && a.kv_dtype == a.dtype && a.D == DH &&
+         (G == 1 || G == 2 || G == 4 || G == 8) && a.partition_size % TOK == 0 &&
+         static_cast<int64_t>(a.num_blocks) * a.Hkv * a.block_size < (int64_t(1) << 31) &&
+         encode_fn() != nullptr;
+}
+
+int launch_decode_group_tc(const DecodeArgs& a, unsigned int* status, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int G = a.Hq / a.Hkv;
+  if (a.dtype == PA_BF16) {
+    switch (G) {
+      case 1: return launch_group_tc_t<__nv_bfloat16, 1>(a, status, st);
+      case 2: return launch_group_tc_t<__nv_bfloat16, 2>(a, status, st);
+      case 4: return launch_group_tc_t<__nv_bfloat16, 4>(a, status, st);
+      default: return launch_group_tc_t<__nv_bfloat16, 8>(a, status, st);
+    }
+  }
+  switch (G) {
+    case 1: return launch_group_tc_t<__half, 1>(a, status, st);
+    case 2: return launch_group_tc_t<__half, 2>(a, status, st);
+    case 4: return launch_group_tc_t<__half, 4>(a, status, st);
+    default: return launch_group_tc_t<__half, 8>(a, status, st);
+  }
 }
 
 int launch_decode_partitions_tc(const DecodeArgs& a, unsigned int* status, void* stream) {

@@ -58,6 +58,15 @@ struct DecodeArgs {
   pa_dtype dtype;      // q and out (and the caches unless kv_dtype says otherwise)
   pa_dtype kv_dtype;   // the caches: dtype, or PA_FP8_E4M3
   float k_scale = 1.f, v_scale = 1.f;  // per-cache scales of E4M3 codes
+  // Shared-prefix groups (pa_decode_grouped).  num_partitions is then the
+  // workspace's slots per (sequence, head): the groups' span partitions first,
+  // then the rest of each sequence's from slot_base.  seq_shift[b] (device,
+  // nullable) is the number of leading tokens of sequence b its group serves.
+  const int32_t* seq_shift = nullptr;
+  int slot_base = 0;          // first slot of the partition launch (and rest of the reduce)
+  // the group launch: members group_start[i] .. group_start[i+1]-1 (device)
+  const int32_t* group_start = nullptr;
+  int num_groups = 0, max_group_size = 0;
 };
 
 // Kernel launchers (kernels.cu).  They return cudaError_t as int.
@@ -67,8 +76,15 @@ int launch_decode_reduce(const DecodeArgs& a, unsigned int* status, void* stream
 // query heads per kv head, partition length a multiple of 128.
 bool decode_tc_supported(const DecodeArgs& a);
 int launch_decode_partitions_tc(const DecodeArgs& a, unsigned int* status, void* stream);
-// Consecutive partitions one CTA of a tensor-core decode kernel streams (1, 2 or 4).
+// Consecutive partitions one CTA of a tensor-core decode kernel streams (1, 2,
+// 4 or 8) when ctas_without CTAs would each serve one partition of n_parts.
 int tc_parts_per_cta(const DecodeArgs& a);
+int tc_parts_per_cta(int64_t ctas_one_each, int partition_size, int n_parts);
+// The shared spans of pa_decode_grouped's groups on the tcgen05 kernel (f16 /
+// bf16, head size 128, any G in {1, 2, 4, 8}): partials into slots from 0 of
+// every member's row; span partitions = a.slot_base.
+bool decode_group_tc_supported(const DecodeArgs& a);
+int launch_decode_group_tc(const DecodeArgs& a, unsigned int* status, void* stream);
 // Tensor-core partition kernel over an E4M3 cache (decode_tc8.cu): f16/bf16
 // queries, head size 128, 4 or 8 query heads per kv head, partition length a
 // multiple of 128.

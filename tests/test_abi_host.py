@@ -221,3 +221,124 @@ def test_multi_query_rejects_bad_arguments(L):
     assert pk.pa_decode_multi_workspace_bytes(6, 16, 128, 100, 0) == 0
     assert pk.pa_decode_multi_workspace_bytes(6, 16, 128, 1000, 256) >= 6 * 16 * 4 * 130 * 4
     assert pk.pa_decode_multi_workspace_bytes(6, 16, 128, 1000, 96) == 0   # invalid length
+
+
+# ---------------------------------------------------------------------------
+# shared-prefix groups (host helper and argument checks)
+
+
+def _groups_brute_force(tables, lens, bs):
+    """Groups by the rule pa_build_groups documents, written out plainly."""
+    B = len(lens)
+    full = [int(x) // bs for x in lens]
+    starts, shared = [], [0] * B
+    b0 = 0
+    while b0 < B:
+        members = [b0]
+        while (full[b0] > 0 and members[-1] + 1 < B and full[members[-1] + 1] > 0
+               and tables[members[-1] + 1][0] == tables[b0][0]):
+            members.append(members[-1] + 1)
+        k = full[b0]
+        for m in members[1:]:
+            c = 0
+            while c < min(k, full[m]) and tables[m][c] == tables[b0][c]:
+                c += 1
+            k = c
+        for m in members:
+            shared[m] = k * bs if len(members) > 1 else 0
+        starts.append(b0)
+        b0 = members[-1] + 1
+    return starts + [B], shared
+
+
+def test_build_groups_matches_its_rule():
+    import numpy as np
+    import torch
+    rng = np.random.default_rng(11)
+    for trial in range(200):
+        bs = int(rng.choice([8, 16, 32]))
+        B = int(rng.integers(1, 12))
+        mb = 6
+        tables = np.full((B, mb), -1, np.int32)
+        lens = np.zeros(B, np.int32)
+        pool = iter(range(1000))
+        b = 0
+        while b < B:
+            # a family of forks sharing a random number of leading blocks
+            size = int(rng.integers(1, 4))
+            common = [next(pool) for _ in range(int(rng.integers(0, mb)))]
+            for _ in range(min(size, B - b)):
+                n_blk = int(rng.integers(len(common), mb + 1))
+                row = common[:n_blk] + [next(pool) for _ in range(n_blk - len(common))]
+                L = 0 if n_blk == 0 else int(rng.integers((n_blk - 1) * bs + 1, n_blk * bs + 1))
+                tables[b, :n_blk] = row
+                lens[b] = L
+                b += 1
+        g = pk.pa_build_groups(torch.from_numpy(tables), torch.from_numpy(lens), bs)
+        starts, shared = _groups_brute_force(tables.tolist(), lens.tolist(), bs)
+        assert g.group_start.tolist() == starts, trial
+        assert g.shared_lens.tolist() == shared, trial
+        assert g.num_groups == len(starts) - 1
+        assert g.max_group_size == max(np.diff(starts))
+        assert g.max_shared_len == max(shared)
+        # what pa_decode_grouped requires of the groups
+        for i in range(g.num_groups):
+            mem = range(starts[i], starts[i + 1])
+            S = shared[starts[i]]
+            assert S % bs == 0 and all(shared[m] == S and lens[m] >= S for m in mem)
+            assert all((tables[m, :S // bs] == tables[starts[i], :S // bs]).all() for m in mem)
+
+
+def test_build_groups_of_the_workload_scripts():
+    """Parallel samples: a group per prompt sharing its whole prompt blocks;
+    shared prefix: one group of every request sharing the 4096-token prefix."""
+    import torch
+    import workloads as W
+    for spec, want in ((W.small("llama13b_ps"), "per prompt"), (W.small("long_prefix"), "one")):
+        sc = W.scenario(spec)
+        alloc = pk.BlockAllocator(sc.num_blocks, spec.block_size, sc.free_order.tolist())
+        for op in sc.setup_ops + sc.step_ops:
+            if op.kind == "add":
+                alloc.add(op.seq)
+            elif op.kind == "fork":
+                alloc.fork(op.seq, op.arg)
+            elif op.kind == "release":
+                alloc.release(op.seq)
+            else:
+                alloc.append(op.seq, op.arg)
+        t, l = alloc.build_tables(sc.batch, sc.max_blocks)
+        g = pk.pa_build_groups(torch.from_numpy(t), torch.from_numpy(l), spec.block_size)
+        if want == "one":
+            assert g.num_groups == 1 and g.max_shared_len == spec.prefix_len
+        else:
+            assert g.num_groups == spec.num_prompts
+            assert g.max_group_size == spec.samples_per_prompt
+            assert set(g.group_start.tolist()) == set(range(0, spec.num_seqs + 1,
+                                                            spec.samples_per_prompt))
+
+
+def test_grouped_decode_rejects_bad_arguments(L):
+    import ctypes as C
+    good = dict(num_groups=1, max_group_size=2, max_shared_len=16, B=2, Hq=8, Hkv=2, D=128,
+                bs=16, max_ctx=64, P=0)
+
+    def call(**kw):
+        a = dict(good, **kw)
+        fake = C.c_void_p(256)
+        return L.pa_decode_grouped(fake, fake, fake, fake, fake, 8, fake, fake, fake,
+                                   a["num_groups"], a["max_group_size"], a["max_shared_len"],
+                                   a["B"], a["Hq"], a["Hkv"], a["D"], a["bs"], 100, 0.1,
+                                   pk.PA_BF16, a["P"], a["max_ctx"], None, 0, None)
+
+    n0 = pk.pa_launch_count()
+    assert call(max_shared_len=8) == pk.PA_ERR_INVALID        # not a multiple of bs
+    assert call(max_shared_len=80) == pk.PA_ERR_INVALID       # beyond max_context_len
+    assert call(num_groups=3) == pk.PA_ERR_INVALID            # more groups than sequences
+    assert call(max_group_size=0) == pk.PA_ERR_INVALID
+    assert call() == pk.PA_ERR_INVALID                        # no workspace
+    assert pk.pa_launch_count() == n0
+    need = L.pa_decode_grouped_workspace_bytes(2, 8, 128, 64, 16, 32)
+    # slots: ceil(16/32) = 1 for the span + ceil(64/32) = 2 for the rest
+    assert need == -(-2 * 8 * 3 * 130 * 4 // 256) * 256
+    assert L.pa_decode_grouped_workspace_bytes(2, 8, 128, 64, 0, 32) == \
+        L.pa_decode_workspace_bytes(2, 8, 128, 64, 32)

@@ -268,11 +268,29 @@ def sampled_rows(o, spec, n=96, seed=0):
     return np.array(sorted(rows), dtype=np.int64)
 
 
-@pytest.mark.parametrize("name", ["tiny", "opt13b", "llama13b_ps", "gqa70b", "long_prefix_bs8",
-                                  "long_prefix_bs16", "long_prefix_bs32"])
-def test_full_size_workloads_sampled(name):
-    spec = W.long_prefix(int(name[-2:].lstrip("s"))) if name.startswith("long_prefix") else W.FULL[name]
+def compared_sequences(sc, n_random=32, seed=0):
+    """Batch indices whose every head the full-size tests compare: the longest
+    and the shortest sequence and n_random others."""
+    lens = np.asarray(sc.context_lens)
+    rng = np.random.default_rng(seed)
+    pick = {int(np.argmax(lens)), int(np.argmin(lens))}
+    rest = [b for b in range(len(lens)) if b not in pick]
+    pick |= {int(b) for b in rng.choice(rest, size=min(n_random, len(rest)), replace=False)}
+    return sorted(pick)
+
+
+def full_size_check(spec, name):
+    """One step of a full-size workload in the benchmark's launch configuration
+    (its own partition length), with a spike (boundary-dominant key, see
+    workloads.spike_plan) in every head of the compared sequences: bookkeeping
+    and touched cache blocks bit-exact, every head of those sequences within
+    tolerance of the oracle, and, for a few spiked rows, the oracle itself
+    showing that losing the spike token would move the output far beyond it."""
+    from pa_harness import oracle_row_perturbed
     sc = W.scenario(spec)
+    seqs = compared_sequences(sc)
+    P = spec.partition_size or 4096
+    sc = W.spike_plan(sc, tuple(sorted({P, 512, 4096})), seed=2, seqs=seqs)
     p, o = build(sc)
     out = run_step(p, spec)
     torch.cuda.synchronize()
@@ -282,12 +300,27 @@ def test_full_size_workloads_sampled(name):
     rng = np.random.default_rng(1)
     extra = rng.choice(sc.num_blocks, size=min(256, sc.num_blocks), replace=False).tolist()
     check_caches(p, o, blocks=sorted(set(touched) | set(extra)))
-    rows = sampled_rows(o, spec)
+    rows = np.array([(b, h) for b in seqs for h in range(spec.Hq)], dtype=np.int64)
     want = oracle_attention(o, spec, rows=rows)
     got_all = as_f64(out, spec)
     got = got_all[rows[:, 0], rows[:, 1]]
     assert np.isfinite(got_all).all()
-    assert np.abs(got - want).max() <= TOL[spec.dtype]
+    err = np.abs(got - want).max()
+    assert err <= TOL[spec.dtype], (name, err)
+    # sensitivity on this very input: a few spiked rows, the spike token dropped
+    spiked = sorted(sc.spikes.rows)
+    for r in np.random.default_rng(3).choice(spiked, size=min(6, len(spiked)), replace=False):
+        b, h, j, kind = sc.spikes.rows[int(r)]
+        k = int(np.flatnonzero((rows[:, 0] == b) & (rows[:, 1] == h))[0])
+        d = np.abs(oracle_row_perturbed(o, spec, b, h, j, "drop") - want[k]).max()
+        assert d > 10 * TOL[spec.dtype], (name, b, h, j, kind, d)
+
+
+@pytest.mark.parametrize("name", ["tiny", "opt13b", "llama13b_ps", "gqa70b", "long_prefix_bs8",
+                                  "long_prefix_bs16", "long_prefix_bs32"])
+def test_full_size_workloads(name):
+    spec = W.long_prefix(int(name[-2:].lstrip("s"))) if name.startswith("long_prefix") else W.FULL[name]
+    full_size_check(spec, name)
 
 
 # ---------------------------------------------------------------------------
@@ -357,22 +390,9 @@ def test_fp8_edge_context_lengths():
 
 
 @pytest.mark.parametrize("name", ["opt13b", "gqa70b", "long_prefix_bs16"])
-def test_fp8_full_size_workloads_sampled(name):
+def test_fp8_full_size_workloads(name):
     base = W.long_prefix(16) if name.startswith("long_prefix") else W.FULL[name]
-    spec = W.fp8(base)
-    sc = W.scenario(spec)
-    p, o = build(sc)
-    out = run_step(p, spec)
-    torch.cuda.synchronize()
-    assert pk.pa_device_status() == 0
-    check_bookkeeping(p, o)
-    touched = sorted({s // spec.block_size for s in o.slots} | {d for _, d in o.pairs})
-    check_caches(p, o, blocks=touched)
-    rows = sampled_rows(o, spec)
-    want = oracle_attention(o, spec, rows=rows)
-    got_all = as_f64(out, spec)
-    assert np.isfinite(got_all).all()
-    assert np.abs(got_all[rows[:, 0], rows[:, 1]] - want).max() <= TOL[spec.dtype]
+    full_size_check(W.fp8(base), name + "_fp8")
 
 
 

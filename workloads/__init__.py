@@ -42,7 +42,7 @@ tokens (with their copy-on-write of the shared prompt tail) for llama13b_ps.
 Context lengths include the tokens the step appends.
 """
 from dataclasses import dataclass, field, replace
-from typing import List, Optional, Tuple
+from typing import Dict, List, Optional, Sequence, Tuple
 
 import numpy as np
 
@@ -187,6 +187,14 @@ class Scenario:
     context_lens: np.ndarray        # int32 [B], expected after the step (for sizing only)
     max_blocks: int                 # block-table row length
     max_context_len: int
+    # where each sequence's tokens come from: seq id -> [(kv_id, first position,
+    # count)] in position order (a fork inherits its parent's list)
+    segments: Dict[int, List[Tuple[int, int, int]]] = field(default_factory=dict)
+    # tokens at the start of each sequence that its family (the forks of one
+    # parent) holds in common: the prompt of parallel samples, the prefix of
+    # shared-prefix requests; 0 for independent sequences
+    shared: Dict[int, int] = field(default_factory=dict)
+    spikes: Optional["SpikePlan"] = None   # boundary-dominant contents (spike_plan)
 
     @property
     def B(self) -> int:
@@ -213,13 +221,22 @@ def scenario(spec: Spec) -> Scenario:
     setup: List[Op] = []
     step: List[Op] = []
     kv = 0
+    segs: Dict[int, List[Tuple[int, int, int]]] = {}
 
     def app(lst, sid, n):
         nonlocal kv
         if n > 0:
             lst.append(Op("append", sid, int(n), kv))
+            seg = segs.setdefault(sid, [])
+            pos = seg[-1][1] + seg[-1][2] if seg else 0
+            seg.append((kv, pos, int(n)))
             kv += 1
 
+    def fork(parent, child):
+        setup.append(Op("fork", parent, child))
+        segs[child] = list(segs.get(parent, []))
+
+    shared: Dict[int, int] = {}
     if spec.kind == "independent":
         lens = _ctx_lengths(spec, rng)
         batch = list(range(spec.num_seqs))
@@ -240,7 +257,9 @@ def scenario(spec: Spec) -> Scenario:
             setup.append(Op("add", root))
             app(setup, root, prompts[p])
             for s in range(1, S):
-                setup.append(Op("fork", root, root + s))
+                fork(root, root + s)
+            for s in range(S):
+                shared[root + s] = int(prompts[p])
         for p in range(P):
             for s in range(S):
                 sid = p * S + s
@@ -258,7 +277,8 @@ def scenario(spec: Spec) -> Scenario:
         suffix = rng.integers(spec.suffix_lo, spec.suffix_hi + 1, size=spec.num_seqs)
         batch = list(range(spec.num_seqs))
         for sid in batch:
-            setup.append(Op("fork", root, sid))
+            fork(root, sid)
+            shared[sid] = int(spec.prefix_len)
         setup.append(Op("release", root))
         for sid, sfx in zip(batch, suffix):
             app(setup, sid, sfx - 1)
@@ -274,7 +294,9 @@ def scenario(spec: Spec) -> Scenario:
     lens = np.asarray(lens, dtype=np.int32)
     max_ctx = int(lens.max()) if lens.size else 0
     max_blocks = max(1, -(-max_ctx // bs))
-    return Scenario(spec, nb, free_order, setup, step, batch, lens, max_blocks, max_ctx)
+    return Scenario(spec, nb, free_order, setup, step, batch, lens, max_blocks, max_ctx,
+                    segments={sid: segs.get(sid, []) for sid in batch},
+                    shared={sid: shared.get(sid, 0) for sid in batch})
 
 
 # ---------------------------------------------------------------------------
@@ -301,22 +323,184 @@ def torch_kv_dtype(spec: Spec):
     return torch.float8_e4m3fn if spec.fp8 else torch_dtype(spec)
 
 
-def kv_content(spec: Spec, kv_id: int, n: int, device="cpu"):
-    """K and V of n appended tokens, [n, Hkv, D] each, N(0,1) in the cache dtype."""
+def kv_content(spec: Spec, kv_id: int, n: int, device="cpu", spikes: "SpikePlan" = None):
+    """K and V of n appended tokens, [n, Hkv, D] each, N(0,1) in the cache dtype;
+    with a spike plan, the planned tokens of this draw carry their spike."""
     import torch
     g = _gen(device, spec.seed * 1_000_003 + 7919 * kv_id + 17)
     shape = (n, spec.Hkv, spec.D)
     k = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
     v = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    if spikes is not None and spikes.by_kv.get(kv_id):
+        sp = spikes.by_kv[kv_id]
+        t = torch.tensor([x.t for x in sp], dtype=torch.int64, device=device)
+        hg = torch.tensor([x.g for x in sp], dtype=torch.int64, device=device)
+        kk = np.stack([x.c / np.sqrt(spec.D) * spikes.q_sign(x.row) for x in sp])
+        vv = np.stack([SPIKE_V * spikes.v_sign(x.row) for x in sp])
+        k[t, hg] = torch.tensor(kk, dtype=torch.float32, device=device)
+        v[t, hg] = torch.tensor(vv, dtype=torch.float32, device=device)
     return k.to(torch_dtype(spec)), v.to(torch_dtype(spec))
 
 
-def q_content(spec: Spec, B: int, device="cpu"):
-    """Decode queries [B, Hq, D], N(0,1) in the cache dtype."""
+def q_content(spec: Spec, B: int, device="cpu", spikes: "SpikePlan" = None):
+    """Decode queries [B, Hq, D], N(0,1) in the cache dtype; with a spike plan,
+    row (b, h) is the plan's sign vector of row id b * Hq + h."""
     import torch
+    if spikes is not None:
+        return spike_queries(spikes, B * spec.Hq, spec, device).reshape(B, spec.Hq, spec.D)
     g = _gen(device, spec.seed * 1_000_003 + 5)
     q = torch.randn((B, spec.Hq, spec.D), generator=g, device=device, dtype=torch.float32)
     return q.to(torch_dtype(spec))
+
+
+# ---------------------------------------------------------------------------
+# Boundary-dominant contents for the parity tests.
+#
+# With N(0,1) contents every token carries about 1/L of the softmax weight, so
+# losing, repeating or misplacing one token moves the output by about 1/L,
+# far below the output tolerance at realistic lengths.  A spike plan gives each
+# query row (b, h) a query that is a vector of signs s (+-1) and places, at one
+# chosen position j of its sequence and kv head, a key c / sqrt(D) * s (so the
+# row's score there is c, against background scores of about N(0, 1)) and a
+# value SPIKE_V * s' (another sign vector).  c = ln(n) + 0.5 for a row that
+# attends to n keys puts about half of the row's weight on that one token, so
+# dropping it, counting it twice or reading a neighbour in its place changes
+# the output by a large fraction of SPIKE_V.  The positions are the ones where
+# such slips happen: the first and last token, block edges, partition and
+# span edges, tile edges, the last tile of a partition, and for several query
+# tokens the key just past a query's causal limit.  Only random draws are
+# placed here; no attention is computed.
+
+SPIKE_V = 2.0
+
+
+@dataclass
+class Spike:
+    t: int        # token offset inside its append draw
+    g: int        # kv head
+    row: int      # query row id whose sign vector the key takes
+    c: float      # that row's score at this key
+
+
+@dataclass
+class SpikePlan:
+    seed: int
+    D: int
+    by_kv: Dict[int, List[Spike]]                 # kv_id -> spikes inside that draw
+    rows: Dict[int, Tuple[int, int, int, str]]    # row id -> (seq index or query token, head, position, kind)
+
+    def q_sign(self, row: int) -> np.ndarray:
+        return np.random.default_rng([self.seed, row, 1]).choice([-1.0, 1.0], self.D)
+
+    def v_sign(self, row: int) -> np.ndarray:
+        return np.random.default_rng([self.seed, row, 2]).choice([-1.0, 1.0], self.D)
+
+
+def spike_queries(plan: SpikePlan, n_rows: int, spec: Spec, device="cpu"):
+    """[n_rows, D] queries: row r is the plan's sign vector of row id r."""
+    import torch
+    q = np.stack([plan.q_sign(r) for r in range(n_rows)]) if n_rows else np.zeros((0, spec.D))
+    return torch.tensor(q, dtype=torch.float32, device=device).to(torch_dtype(spec))
+
+
+SPIKE_KINDS = ("end", "start", "partition", "partition", "block", "tile", "last_tile",
+               "shared", "shared")
+
+
+def _spike_candidate(kind, n, bs, parts, rng, shared=0):
+    """A position in [0, n) of the given kind, or None if the sequence has none.
+    `shared`: tokens its family holds in common; a kernel that serves them once
+    for the family splits the sequence at the last whole block inside them and
+    partitions the rest from there ("shared" edges)."""
+    if kind == "end":
+        return n - 1
+    if kind == "start":
+        return 0
+    if kind == "shared":
+        S = shared // bs * bs
+        if S <= 0 or S >= n:
+            return None
+        P = int(rng.choice(parts))
+        k = int(rng.integers(0, (n - 1 - S) // P + 1))        # the split or a later edge
+        return S + k * P - int(rng.integers(0, 2))
+    if kind in ("partition", "last_tile"):
+        P = int(rng.choice(parts))
+        if n <= P:
+            return None
+        k = int(rng.integers(1, (n - 1) // P + 1))          # an edge k*P inside (0, n)
+        if kind == "last_tile":
+            return k * P - 1 - int(rng.integers(0, min(128, P)))
+        return k * P - int(rng.integers(0, 2))
+    step = bs if kind == "block" else int(rng.choice((32, 128)))
+    if n <= step:
+        return None
+    k = int(rng.integers(1, (n - 1) // step + 1))
+    return k * step - int(rng.integers(0, 2))
+
+
+def _locate(segs, j):
+    for kv_id, pos0, cnt in segs:
+        if pos0 <= j < pos0 + cnt:
+            return kv_id, j - pos0
+    raise ValueError(f"position {j} is not covered by the sequence's appends")
+
+
+def spike_plan(sc: Scenario, parts: Sequence[int], seed: int = 0,
+               seqs: Optional[Sequence[int]] = None,
+               query_lens: Optional[Sequence[int]] = None) -> Scenario:
+    """The scenario with a spike plan: one spike for every query row of the
+    chosen batch indices (all by default), at a boundary position.
+
+    Decode (query_lens None): row (b, h) attends to positions [0, L_b).
+    Several query tokens (query_lens[b] = Q_b): query token i of sequence b (a
+    global token index t, rows t * Hq + h) attends to [0, L_b - Q_b + i], and
+    a further kind puts its spike just past that limit, at L_b - Q_b + i + 1
+    (a key the row must not see).  `parts` are the partition / span lengths
+    whose edges matter."""
+    spec = sc.spec
+    rng = np.random.default_rng([sc.spec.seed, seed, 4431])
+    lens = [int(x) for x in sc.context_lens]
+    pick = range(len(sc.batch)) if seqs is None else seqs
+    by_kv: Dict[int, List[Spike]] = {}
+    rows: Dict[int, Tuple[int, int, int, str]] = {}
+    taken = set()
+    qstart = None
+    if query_lens is not None:
+        qlens = [min(int(q), L) for q, L in zip(query_lens, lens)]
+        qstart = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int64)
+    for b in pick:
+        L = lens[b]
+        segs = sc.segments[sc.batch[b]]
+        if query_lens is None:
+            units = [(b, L, None)]                    # (row base, keys seen, limit)
+        else:
+            Qb = int(qstart[b + 1] - qstart[b])
+            units = [(int(qstart[b]) + i, L - Qb + i + 1, L) for i in range(Qb)]
+        for unit, n, limit in units:
+            if n <= 0:
+                continue
+            for h in range(spec.Hq):
+                g = h // spec.G
+                row = unit * spec.Hq + h
+                for _ in range(24):                   # a few tries for a free position
+                    kinds = SPIKE_KINDS + (("past_limit",) if limit is not None else ())
+                    kind = kinds[int(rng.integers(0, len(kinds)))]
+                    if kind == "past_limit":
+                        j = n if n < limit else None
+                    else:
+                        j = _spike_candidate(kind, n, spec.block_size, parts, rng,
+                                             sc.shared.get(sc.batch[b], 0))
+                    if j is None or not 0 <= j < L:
+                        continue
+                    kv_id, t = _locate(segs, j)
+                    if (kv_id, t, g) in taken:
+                        continue
+                    taken.add((kv_id, t, g))
+                    c = float(np.log(max(n, 2)) + 0.5)
+                    by_kv.setdefault(kv_id, []).append(Spike(t, g, row, c))
+                    rows[row] = (unit, h, j, kind)
+                    break
+    return replace(sc, spikes=SpikePlan(int(rng.integers(1 << 31)), spec.D, by_kv, rows))
 
 
 def poison_value(spec: Spec):

@@ -647,9 +647,10 @@ def run_ours(args):
     if groups is not None:
         # the three launches of the grouped decode are timed together (the
         # reduce included), against the same algorithmic bytes
-        kname = ("decode_grouped: decode_partition_tc_kernel (shared spans, 16/G members per "
-                 "CTA) + " + partition_kernel(spec, P) + " (rest) + decode_reduce_kernel")
-        traffic, traffic_note = None, "three kernels timed together; see the ncu launch list"
+        kname = ("decode_grouped: decode_partition_tc_kernel (the families' shared spans, "
+                 "16/G members per CTA, and the rest of every sequence in one grid) + "
+                 "decode_reduce_kernel")
+        traffic, traffic_note = None, "two kernels timed together; see the ncu launch list"
 
     result = None
     if rank == 0:
@@ -776,7 +777,7 @@ def run_mq(args):
     q = torch.randn((T, spec.Hq, spec.D), generator=g, device=device).to(W.torch_dtype(spec))
     out = torch.empty_like(q)
     qs_d = torch.from_numpy(qs).to(device)
-    P = args.partition_size or 512
+    P = args.partition_size     # 0: pa_decode_multi's automatic length
     n = pk.pa_decode_multi_workspace_bytes(T, spec.Hq, spec.D, max_ctx, P)
     ws = torch.empty(n // 4, dtype=torch.float32, device=device) if n else None
     maxq = int(qlens.max())
@@ -833,7 +834,7 @@ def run_mq(args):
         "data": "synthetic: seeded N(0,1) K/V/q, context lengths and placement as the workload states",
         "config": {"workload": f"{args.workload}: {MQ_WORKLOADS[args.workload.replace('_quarter', '')][2]}",
                    "num_seqs": len(sc.batch), "query_tokens": T, "query_tokens_per_seq": Q,
-                   "max_context_len": max_ctx, "partition_size": P,
+                   "max_context_len": max_ctx, "partition_size": P or "automatic",
                    "kv_bytes_unique": unique, "flops": flops,
                    "l2": "L2 flushed between timed steps" if flush else "inputs larger than L2"},
         "tflops": round(tflops, 2), "kv_gbs": round(gbs, 2),

@@ -294,8 +294,9 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache, const
  * differ or exceed their context, a length not a multiple of block_size) set
  * PA_DEVERR_CONTEXT.  With max_shared_len = 0 or num_groups = 0 this is
  * pa_decode; so it is for f32 / head size 64, where no tensor-core kernel
- * serves the shared span.  Three launches: the groups' spans, the rest of each
- * sequence, the reduce.
+ * serves the shared span.  Two launches: the partition kernel (the groups'
+ * spans and the rest of every sequence in one grid, all on the tensor cores)
+ * and the reduce.
  */
 size_t pa_decode_grouped_workspace_bytes(int num_seqs, int num_heads, int head_size,
                                          int max_context_len, int max_shared_len,
@@ -360,9 +361,13 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_pair
  *                   ending at total_q; max_query_len >= every Q_b
  *   k_cache, v_cache, block_tables, context_lens, max_context_len: as pa_decode
  * Supported: f16/bf16, head_size 128, Hq/Hkv in {1, 2, 4, 8}, bs in {8, 16,
- * 32}, partition_size 0 (= 512) or a multiple of 128.  The workspace holds the
- * split-K partials when max_context_len exceeds the partition length
- * (pa_decode_multi_workspace_bytes).  Offsets that are not non-decreasing, or
+ * 32}, partition_size a multiple of 128, or 0 for an automatic length of at
+ * least 512: with many query tokens (a prefill chunk) the keys are split only
+ * as far as needed for two CTAs per SM, with few (verification) pa_decode's
+ * rule applies.  The workspace holds the split-K partials when
+ * max_context_len exceeds the partition length (pa_decode_multi_workspace_bytes;
+ * with partition_size 0 it returns the size for 512, which suffices for the
+ * automatic length).  Offsets that are not non-decreasing, or
  * Q_b > context_lens[b], set PA_DEVERR_CONTEXT and the sequence is skipped.
  * One or two launches on `stream`.
  */

@@ -485,6 +485,37 @@ extern "C" pa_status pa_reshape_and_cache_fp8(const void* key, const void* value
                        1);
 }
 
+// Partition length pa_decode_multi uses for partition_size = 0.  The
+// query-major kernel (many query tokens) holds one CTA per SM, so the keys are
+// split only as far as it takes to give at least two CTAs per SM: a prefill
+// chunk of hundreds of tokens needs no split at all, and every split costs
+// fp32 partials for all of its query rows.  Few queries per sequence (the
+// token-major decode kernel) take pa_decode's rule with q_groups CTAs per
+// sequence.  Never below the default 512, so the default's workspace size
+// always suffices.
+int auto_partition_multi(int num_seqs, int num_heads, int num_kv_heads, int max_query_len,
+                         pa_dtype dtype, int max_context_len) {
+  const int G = num_heads / num_kv_heads;
+  const int P0 = pa::kDefaultPartition;
+  if (max_context_len <= P0) return P0;
+  if (G >= 4 && max_query_len * G <= 64) {           // token-major
+    const int nq = (G == 8 || max_query_len <= 2) ? 2 : 4;   // query tokens per CTA
+    const int q_groups = (max_query_len + nq - 1) / nq;
+    const int P = auto_partition(num_seqs * q_groups, num_heads, num_kv_heads, 128, dtype,
+                                 max_context_len);
+    return P < P0 ? P0 : P;
+  }
+  const int64_t qblocks = (max_query_len + pa::kMqRows / G - 1) / (pa::kMqRows / G);
+  const int64_t base = static_cast<int64_t>(num_seqs) * num_kv_heads * qblocks;
+  const int64_t want = 2ll * num_sms();
+  int64_t np = base >= want ? 1 : (want + base - 1) / base;
+  const int64_t np_max = (max_context_len + P0 - 1) / P0;
+  if (np > np_max) np = np_max;
+  int64_t P = (max_context_len + np - 1) / np;
+  P = (P + 127) / 128 * 128;
+  return static_cast<int>(P < P0 ? P0 : P);
+}
+
 extern "C" size_t pa_decode_multi_workspace_bytes(int total_q, int num_heads, int head_size,
                                                   int max_context_len, int partition_size) {
   const int P = resolve_partition(partition_size);
@@ -501,6 +532,10 @@ extern "C" pa_status pa_decode_multi(void* out, const void* q, const void* k_cac
                                      pa_dtype dtype, int partition_size, int max_context_len,
                                      void* workspace, size_t workspace_bytes_in, void* stream) {
   const char* fn = "pa_decode_multi";
+  if (partition_size == 0 && num_heads > 0 && num_kv_heads > 0 && num_heads % num_kv_heads == 0 &&
+      max_query_len > 0 && num_seqs >= 0)
+    partition_size = auto_partition_multi(num_seqs, num_heads, num_kv_heads, max_query_len, dtype,
+                                          max_context_len);
   if (pa::elem_size(dtype) == 0) return pa::fail(PA_ERR_INVALID, "%s: unknown dtype %d", fn, dtype);
   if (dtype != PA_F16 && dtype != PA_BF16)
     return pa::fail(PA_ERR_UNSUPPORTED, "%s: q, out and the caches must be f16 or bf16", fn);
@@ -660,7 +695,7 @@ extern "C" pa_status pa_decode_grouped(void* out, const void* q, const void* k_c
                      dtype, partition_size, max_context_len, workspace, workspace_bytes_in, stream);
   const int G = num_heads / num_kv_heads;
   const int64_t member_runs = (max_group_size + (16 / G) - 1) / (16 / G);
-  if (static_cast<int64_t>(num_groups) * member_runs > 0x7fffffff)
+  if (static_cast<int64_t>(num_groups) * member_runs + num_seqs > 0x7fffffff)
     return pa::fail(PA_ERR_UNSUPPORTED, "%s: too many groups", fn);
   unsigned int* status = pa::device_status_word();
   if (!status) return PA_ERR_CUDA;
@@ -671,8 +706,6 @@ extern "C" pa_status pa_decode_grouped(void* out, const void* q, const void* k_c
   a.num_groups = num_groups;
   a.max_group_size = max_group_size;
   st = launch_status(fn, pa::launch_decode_group_tc(a, status, stream), 1);
-  if (st != PA_OK) return st;
-  st = launch_status(fn, launch_partitions(a, status, stream), 1);
   if (st != PA_OK) return st;
   return launch_status(fn, pa::launch_decode_reduce(a, status, stream), 1);
 }

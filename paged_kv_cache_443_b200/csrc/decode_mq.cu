@@ -171,8 +171,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* q_ready = p_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
 
+  // the query blocks of one (sequence, kv head, key partition) are adjacent in
+  // the grid, so they run together and read that partition's K/V from L2
+  const int n_qb = gridDim.z / p.num_partitions;
   const int b = blockIdx.x, g = blockIdx.y;
-  const int qb = blockIdx.z / p.num_partitions, part = blockIdx.z % p.num_partitions;
+  const int qb = blockIdx.z % n_qb, part = blockIdx.z / n_qb;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   grid_dependency_wait();

@@ -101,6 +101,12 @@ struct TcParams {
   const int32_t* seq_shift;
   const int32_t* group_start;
   int slot_base;
+  // One launch serves both parts of a grouped decode: blockIdx.x < span_x are
+  // the groups' span CTAs (span_ppc partitions each, partials from slot 0),
+  // the others sequence blockIdx.x - span_x past its shift (parts_per_cta
+  // partitions each, partials from slot_base).
+  int span_x;
+  int span_ppc;
 };
 
 // NQ > 1 serves several query tokens per sequence (speculative verification):
@@ -132,9 +138,13 @@ __global__ void __launch_bounds__(THREADS, 2)
   // short partitions do not each pay the pipeline's fill and drain: its partial
   // goes to the first one's slot and the others' slots get empty partials (max
   // -inf, sum 0, output 0), which the reduce weighs by exactly 0.
-  const bool grouped = NQ > 1 && p.group_start != nullptr;   // a group's shared span
-  int b = NQ > 1 ? blockIdx.x / p.q_groups : blockIdx.x;
-  const int g = blockIdx.y, part = blockIdx.z * p.parts_per_cta;
+  // this CTA's work: a group's shared span, several query tokens of one
+  // sequence, or (the decode) one sequence past its shift
+  const bool grouped = NQ > 1 && p.group_start != nullptr && blockIdx.x < p.span_x;
+  const bool multi = NQ > 1 && p.query_start != nullptr;
+  int b = multi ? blockIdx.x / p.q_groups : blockIdx.x - p.span_x;
+  const int ppc = grouped ? p.span_ppc : p.parts_per_cta;
+  const int g = blockIdx.y, part = blockIdx.z * ppc;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int NC = G * NQ;                // S / O columns in use
   static_assert(NC <= NPAD, "query tokens x heads must fit the MMA's N");
@@ -177,7 +187,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     }
     q0 = m0;
     L = S;
-  } else if (NQ > 1) {
+  } else if (multi) {
     const int qg = blockIdx.x % p.q_groups;
     const int qs = p.query_start[b];
     Qall = p.query_start[b + 1] - qs;
@@ -197,7 +207,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     if (threadIdx.x == 0 && part == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
     L = L < 0 ? 0 : static_cast<int>(cap);
   }
-  if (NQ == 1 && p.seq_shift != nullptr) {
+  if (!grouped && !multi && p.seq_shift != nullptr) {
     // the tokens past the sequence's shared span (its group serves the span)
     shift = p.seq_shift[b];
     if (shift < 0 || shift % bs != 0 || shift > L) {
@@ -206,14 +216,15 @@ __global__ void __launch_bounds__(THREADS, 2)
     }
     L -= shift;
   }
-  const int64_t grid_cap = static_cast<int64_t>(p.num_partitions - p.slot_base) * P;
+  const int slot0 = grouped ? 0 : p.slot_base;        // this CTA's first workspace slot
+  const int64_t grid_cap = static_cast<int64_t>(p.num_partitions - slot0) * P;
   if (L > grid_cap) {
     if (threadIdx.x == 0 && part == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
     L = static_cast<int>(grid_cap);
   }
   const int start = part * P;
   if (L == 0) {
-    if (NQ == 1 && part == 0 && shift == 0) {
+    if (!grouped && !multi && part == 0 && shift == 0) {
       T* o = static_cast<T*>(p.out) + (static_cast<int64_t>(b) * p.Hq + g * G) * DH;
       for (int i = threadIdx.x; i < G * DH; i += THREADS) o[i] = Elem<T>::from_float(0.f);
     }
@@ -221,12 +232,12 @@ __global__ void __launch_bounds__(THREADS, 2)
   }
   if (start >= L) return;
   const int end = static_cast<int>(
-      min(static_cast<int64_t>(L), start + static_cast<int64_t>(P) * p.parts_per_cta));
+      min(static_cast<int64_t>(L), start + static_cast<int64_t>(P) * ppc));
   const int n_tiles = (end - start + TOK - 1) / TOK;
   // the output directly, or partials for the reduce (always for a group's span
   // and for a sequence whose first tokens its group served)
   const bool single = (L <= P) && !grouped && shift == 0;
-  const int n_slots = min(p.parts_per_cta, (L + P - 1) / P - part);   // partials this CTA writes
+  const int n_slots = min(ppc, (L + P - 1) / P - part);   // partials this CTA writes
 
   // ---- set-up: the producer starts streaming right after the barrier, while
   // the softmax warps stage Q^T and the MMA issuer waits for it ----
@@ -430,7 +441,7 @@ __global__ void __launch_bounds__(THREADS, 2)
           if (single) {
             static_cast<T*>(p.out)[hq * DH + r] = Elem<T>::from_float(o[h] / Ls);
           } else {
-            const int64_t slot = hq * p.num_partitions + p.slot_base + part;
+            const int64_t slot = hq * p.num_partitions + slot0 + part;
             p.ws_o[slot * DH + r] = o[h];
             if (r == 0) {
               p.ws_m[slot] = m_run[h];
@@ -591,14 +602,20 @@ cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t 
   p.seq_shift = a.seq_shift;
   p.group_start = nullptr;
   p.slot_base = a.slot_base;
+  p.span_x = 0;
+  p.span_ppc = 1;
   const int np = a.num_partitions - a.slot_base;
   dim3 grid(a.num_seqs, a.Hkv, (np + p.parts_per_cta - 1) / p.parts_per_cta);
   return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
 }
 
-// The shared spans of shared-prefix groups: NQ = 16 / G members per CTA, each
-// column a (member, head) pair, one CTA per (group, run of NQ members, kv
-// head, run of span partitions); partials into every member's slots from 0.
+// A grouped decode in one launch, with NQ = 16 / G: first the groups' shared
+// spans, each CTA serving NQ members of a group (column = (member, head)),
+// one CTA per (group, run of NQ members, kv head, run of span partitions);
+// then the rest of every sequence past its shift, one CTA per (sequence, kv
+// head, run of partitions), on the same pipeline with one member's G columns.
+// Both kinds are in one grid, so the short span CTAs and the sequences' CTAs
+// share the SMs instead of running one kernel after the other.
 template <typename T, int G>
 cudaError_t launch_group_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
   constexpr int NQ = NPAD / G;
@@ -636,13 +653,20 @@ cudaError_t launch_group_tc_t(const DecodeArgs& a, unsigned int* status, cudaStr
   p.q_groups = (a.max_group_size + NQ - 1) / NQ;
   p.seq_shift = a.seq_shift;
   p.group_start = a.group_start;
-  p.slot_base = 0;
-  const int span_parts = a.slot_base;      // the groups' span partitions
-  const int64_t ctas = static_cast<int64_t>(a.num_groups) * p.q_groups * a.Hkv;
-  p.parts_per_cta = tc_parts_per_cta(ctas * span_parts, a.partition_size, span_parts);
-  // grid cap of the kernel: the span's partitions (num_partitions - slot_base)
-  p.num_partitions = a.num_partitions;
-  dim3 grid(a.num_groups * p.q_groups, a.Hkv, (span_parts + p.parts_per_cta - 1) / p.parts_per_cta);
+  p.slot_base = a.slot_base;                       // = the groups' span partitions
+  const int span_parts = a.slot_base;
+  const int rest_parts = a.num_partitions - a.slot_base;
+  p.span_x = a.num_groups * p.q_groups;
+  // streaming: the rest by the decode kernel's rule; the spans by the same
+  // rule counting the rest's CTAs as well (they share the grid)
+  const int64_t span_rows = static_cast<int64_t>(p.span_x) * a.Hkv;
+  const int64_t rest_rows = static_cast<int64_t>(a.num_seqs) * a.Hkv;
+  p.parts_per_cta = tc_parts_per_cta(rest_rows, a.partition_size, rest_parts, 0);
+  const int64_t rest_ctas = rest_rows * ((rest_parts + p.parts_per_cta - 1) / p.parts_per_cta);
+  p.span_ppc = tc_parts_per_cta(span_rows, a.partition_size, span_parts, rest_ctas);
+  const int z_span = (span_parts + p.span_ppc - 1) / p.span_ppc;
+  const int z_rest = (rest_parts + p.parts_per_cta - 1) / p.parts_per_cta;
+  dim3 grid(p.span_x + a.num_seqs, a.Hkv, z_span > z_rest ? z_span : z_rest);
   return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
 }
 
@@ -659,20 +683,19 @@ static int sm_count() {
 // Consecutive partitions per CTA (one softmax over them): for partitions
 // shorter than 2048 tokens, the most of 8 / 4 / 2 that keeps a CTA's span
 // within 4096 tokens and still leaves at least 8 CTAs per SM.
-int tc_parts_per_cta(int64_t ctas_one_each, int partition_size, int n_parts) {
+int tc_parts_per_cta(int64_t rows, int partition_size, int n_parts, int64_t other_ctas) {
   if (partition_size >= 2048 || n_parts <= 0) return 1;
   const int64_t want = 8ll * sm_count();
-  const int64_t rows = ctas_one_each / n_parts;      // CTAs per partition index
   for (int c : {8, 4, 2}) {
-    const int64_t ctas = rows * ((n_parts + c - 1) / c);
+    const int64_t ctas = rows * ((n_parts + c - 1) / c) + other_ctas;
     if (static_cast<int64_t>(partition_size) * c <= 4096 && n_parts >= c && ctas >= want) return c;
   }
   return 1;
 }
 
 int tc_parts_per_cta(const DecodeArgs& a) {
-  const int np = a.num_partitions - a.slot_base;
-  return tc_parts_per_cta(static_cast<int64_t>(a.num_seqs) * a.Hkv * np, a.partition_size, np);
+  return tc_parts_per_cta(static_cast<int64_t>(a.num_seqs) * a.Hkv, a.partition_size,
+                          a.num_partitions - a.slot_base, 0);
 }
 
 namespace {
@@ -760,6 +783,8 @@ cudaError_t launch_tcq_t(const MqArgs& m, unsigned int* status, cudaStream_t str
   p.seq_shift = nullptr;
   p.group_start = nullptr;
   p.slot_base = 0;
+  p.span_x = 0;
+  p.span_ppc = 1;
   dim3 grid(m.num_seqs * p.q_groups, m.Hkv, (m.num_partitions + ppc - 1) / ppc);
   return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
 }

@@ -79,10 +79,13 @@ int launch_decode_partitions_tc(const DecodeArgs& a, unsigned int* status, void*
 // Consecutive partitions one CTA of a tensor-core decode kernel streams (1, 2,
 // 4 or 8) when ctas_without CTAs would each serve one partition of n_parts.
 int tc_parts_per_cta(const DecodeArgs& a);
-int tc_parts_per_cta(int64_t ctas_one_each, int partition_size, int n_parts);
-// The shared spans of pa_decode_grouped's groups on the tcgen05 kernel (f16 /
-// bf16, head size 128, any G in {1, 2, 4, 8}): partials into slots from 0 of
-// every member's row; span partitions = a.slot_base.
+// rows: CTAs per partition index (sequences x kv heads); other_ctas: CTAs of
+// other work in the same grid.
+int tc_parts_per_cta(int64_t rows, int partition_size, int n_parts, int64_t other_ctas);
+// pa_decode_grouped's partition phase on the tcgen05 kernel in one launch (f16
+// / bf16, head size 128, G in {1, 2, 4, 8}): the groups' shared spans
+// (partials into slots [0, a.slot_base) of every member's row) and the rest of
+// every sequence (slots from a.slot_base).
 bool decode_group_tc_supported(const DecodeArgs& a);
 int launch_decode_group_tc(const DecodeArgs& a, unsigned int* status, void* stream);
 // Tensor-core partition kernel over an E4M3 cache (decode_tc8.cu): f16/bf16

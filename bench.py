@@ -648,9 +648,9 @@ def run_ours(args):
         # the three launches of the grouped decode are timed together (the
         # reduce included), against the same algorithmic bytes
         kname = ("decode_grouped: decode_partition_tc_kernel (the families' shared spans, "
-                 "16/G members per CTA, and the rest of every sequence in one grid) + "
-                 "decode_reduce_kernel")
-        traffic, traffic_note = None, "two kernels timed together; see the ncu launch list"
+                 "16/G members per CTA) next to " + partition_kernel(spec, P) +
+                 " (the rest of every sequence), then decode_reduce_kernel")
+        traffic, traffic_note = None, "three kernels timed together; see the ncu launch list"
 
     result = None
     if rank == 0:

@@ -294,9 +294,12 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache, const
  * differ or exceed their context, a length not a multiple of block_size) set
  * PA_DEVERR_CONTEXT.  With max_shared_len = 0 or num_groups = 0 this is
  * pa_decode; so it is for f32 / head size 64, where no tensor-core kernel
- * serves the shared span.  Two launches: the partition kernel (the groups'
- * spans and the rest of every sequence in one grid, all on the tensor cores)
- * and the reduce.
+ * serves the shared span.  Three launches: the groups' spans run on a stream
+ * the library creates per device on first use (with two events), forked from
+ * and joined back to `stream`, next to the rest of every sequence on `stream`;
+ * then the reduce on `stream`.  Everything stays ordered on `stream` for the
+ * caller (and inside a stream capture).  Calls from several host threads are
+ * serialised around that fork and join.
  */
 size_t pa_decode_grouped_workspace_bytes(int num_seqs, int num_heads, int head_size,
                                          int max_context_len, int max_shared_len,

@@ -4,6 +4,7 @@
 // contract of every entry point.
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include <cuda_runtime.h>
 
@@ -499,7 +500,7 @@ int auto_partition_multi(int num_seqs, int num_heads, int num_kv_heads, int max_
   const int P0 = pa::kDefaultPartition;
   if (max_context_len <= P0) return P0;
   if (G >= 4 && max_query_len * G <= 64) {           // token-major
-    const int nq = (G == 8 || max_query_len <= 2) ? 2 : 4;   // query tokens per CTA
+    const int nq = pa::tc_query_tokens_per_cta(G, max_query_len);
     const int q_groups = (max_query_len + nq - 1) / nq;
     const int P = auto_partition(num_seqs * q_groups, num_heads, num_kv_heads, 128, dtype,
                                  max_context_len);
@@ -620,6 +621,40 @@ extern "C" pa_status pa_decode_multi(void* out, const void* q, const void* k_cac
 
 namespace {
 
+// pa_decode_grouped runs the groups' spans on a library-owned stream of the
+// device next to the rest of the sequences on the caller's stream: a fork
+// event recorded on the caller's stream, then a join event the caller's stream
+// waits on before the reduce.  Created on first use; the mutex keeps the
+// record / wait / launch sequence of concurrent host threads apart (an event's
+// wait binds the record before it, so reusing the two events is safe).
+struct AuxStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxAuxDevices = 64;
+AuxStream g_aux[kMaxAuxDevices];
+std::mutex g_aux_mu;
+
+AuxStream* aux_stream(int dev) {
+  if (dev < 0 || dev >= kMaxAuxDevices) return nullptr;
+  AuxStream& x = g_aux[dev];
+  if (!x.stream) {
+    cudaStream_t st = nullptr;
+    cudaEvent_t f = nullptr, j = nullptr;
+    if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess) {
+      if (f) cudaEventDestroy(f);
+      cudaStreamDestroy(st);
+      return nullptr;
+    }
+    x.stream = st;
+    x.fork = f;
+    x.join = j;
+  }
+  return &x;
+}
+
 int64_t grouped_span_partitions(int max_shared_len, int P) {
   return max_shared_len > 0 ? (static_cast<int64_t>(max_shared_len) + P - 1) / P : 0;
 }
@@ -705,7 +740,27 @@ extern "C" pa_status pa_decode_grouped(void* out, const void* q, const void* k_c
   a.group_start = group_start;
   a.num_groups = num_groups;
   a.max_group_size = max_group_size;
-  st = launch_status(fn, pa::launch_decode_group_tc(a, status, stream), 1);
-  if (st != PA_OK) return st;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return pa::fail(PA_ERR_CUDA, "%s: cudaGetDevice", fn);
+  cudaStream_t st_main = static_cast<cudaStream_t>(stream);
+  {
+    std::lock_guard<std::mutex> lk(g_aux_mu);
+    AuxStream* aux = aux_stream(dev);
+    if (aux == nullptr)   // no second stream: the spans first, then the rest
+      return pa::fail(PA_ERR_CUDA, "%s: could not create the library's auxiliary stream", fn);
+    // fork: the spans on the auxiliary stream, the rest on the caller's
+    if (cudaEventRecord(aux->fork, st_main) != cudaSuccess ||
+        cudaStreamWaitEvent(aux->stream, aux->fork, 0) != cudaSuccess)
+      return pa::fail(PA_ERR_CUDA, "%s: fork to the auxiliary stream failed", fn);
+    st = launch_status(fn, pa::launch_decode_group_tc(a, status, aux->stream), 1);
+    const pa_status st_rest = launch_status(fn, launch_partitions(a, status, stream), 1);
+    // join, whatever happened, so that the caller's stream never runs ahead
+    // of work left on the auxiliary one
+    const bool joined = cudaEventRecord(aux->join, aux->stream) == cudaSuccess &&
+                        cudaStreamWaitEvent(st_main, aux->join, 0) == cudaSuccess;
+    if (st != PA_OK) return st;
+    if (st_rest != PA_OK) return st_rest;
+    if (!joined) return pa::fail(PA_ERR_CUDA, "%s: join with the auxiliary stream failed", fn);
+  }
   return launch_status(fn, pa::launch_decode_reduce(a, status, stream), 1);
 }

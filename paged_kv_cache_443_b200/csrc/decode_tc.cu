@@ -52,27 +52,35 @@ using namespace tc;
 
 constexpr unsigned FULL = 0xffffffffu;
 constexpr int TOK = 128;                     // tokens per tile (M of the first MMA)
-constexpr int NPAD = 16;                     // N of both MMAs (heads padded)
 constexpr int DH = 128;                      // head size
-constexpr int SLOTS = 3;                     // ring slots (K or V of one tile each)
 constexpr int SLOT_BYTES = TOK * 256;        // one tile of K (or V): 32 KB
 constexpr int GROUP_BYTES = 2048;            // 8 token rows, both 64-column halves
 constexpr int HALF_OFF = 1024;               // second 64-column half of a group
-constexpr int OPB_BYTES = 2 * NPAD * 128;    // a 16-row operand in two 64-column blocks: 4 KB
-constexpr int OFF_RING = 0;
-constexpr int OFF_Q = OFF_RING + SLOTS * SLOT_BYTES;
-constexpr int OFF_P = OFF_Q + OPB_BYTES;     // two P buffers
-constexpr int OFF_BAR = OFF_P + 2 * OPB_BYTES;
-constexpr int NBARS = 2 * SLOTS + 9;         // ring full/empty, s/p full/free, q_ready
-constexpr int OFF_TMEM = OFF_BAR + NBARS * 8;
-constexpr int OFF_RED = OFF_TMEM + 16;       // 4 warps x 16 floats
-constexpr int SMEM_USED = OFF_RED + 4 * NPAD * 4;
-constexpr int SMEM_BYTES = SMEM_USED + 1024; // slack to align the base to 1024 B
 constexpr int THREADS = 192;
-constexpr int TMEM_COLS = 64;                // S0 [0,16), S1 [16,32), O [32,48)
 constexpr float RESCALE_THRESHOLD = 8.0f;    // log2 units: raise the max past 2^8 growth
 
-static_assert(SMEM_BYTES * 2 + 2048 <= 228 * 1024, "two CTAs per SM");
+// Shared-memory and TMEM layout for N = NP columns (16, or 32 for 32 query
+// tokens x heads): a ring of SLOTS K/V tiles (three at N = 16; two at N = 32,
+// so that two CTAs still share an SM), the Q^T operand and two P buffers of NP
+// rows in two swizzled 64-column blocks, barriers, the TMEM address and a
+// 4-warp reduction buffer.  TMEM: S0 [0, NP), S1 [NP, 2NP), O [2NP, 3NP).
+template <int NP>
+struct Lay {
+  static constexpr int NPAD = NP;
+  static constexpr int SLOTS = NP <= 16 ? 3 : 2;
+  static constexpr int OPB_BYTES = 2 * NP * 128;
+  static constexpr int OFF_RING = 0;
+  static constexpr int OFF_Q = OFF_RING + SLOTS * SLOT_BYTES;
+  static constexpr int OFF_P = OFF_Q + OPB_BYTES;
+  static constexpr int OFF_BAR = OFF_P + 2 * OPB_BYTES;
+  static constexpr int NBARS = 2 * SLOTS + 9;   // ring full/empty, s/p full/free, q_ready
+  static constexpr int OFF_TMEM = OFF_BAR + NBARS * 8;
+  static constexpr int OFF_RED = OFF_TMEM + 16;
+  static constexpr int SMEM_USED = OFF_RED + 4 * NP * 4;
+  static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack to align the base to 1024 B
+  static constexpr int TMEM_COLS = 3 * NP <= 64 ? 64 : 128;
+  static_assert(SMEM_BYTES * 2 + 2048 <= 228 * 1024, "two CTAs per SM");
+};
 
 struct TcParams {
   void* out;
@@ -113,10 +121,14 @@ struct TcParams {
 // column c of S / O is query token c / G (one of the sequence's last Qb <= NQ
 // context tokens) with head c % G, and a key counts for it only up to that
 // token's own position.  NQ = 1 is the decode step and compiles as before.
-template <typename T, int G, int NQ = 1>
+template <typename T, int G, int NQ = 1, int NP = 16>
 __global__ void __launch_bounds__(THREADS, 2)
     decode_partition_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmap_k,
                                const __grid_constant__ CUtensorMap tmap_v) {
+  using Y = Lay<NP>;
+  constexpr int NPAD = NP, SLOTS = Y::SLOTS, OPB_BYTES = Y::OPB_BYTES;
+  constexpr int OFF_RING = Y::OFF_RING, OFF_Q = Y::OFF_Q, OFF_P = Y::OFF_P, OFF_BAR = Y::OFF_BAR;
+  constexpr int OFF_TMEM = Y::OFF_TMEM, OFF_RED = Y::OFF_RED, TMEM_COLS = Y::TMEM_COLS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -342,8 +354,8 @@ __global__ void __launch_bounds__(THREADS, 2)
   if (warp == 1) {
     // ================= MMA issuer =================
     if (lane == 0) {
-      const uint32_t id_qk = instr_desc<T>(false);
-      const uint32_t id_pv = instr_desc<T>(true);
+      const uint32_t id_qk = instr_desc<T, NPAD>(false);
+      const uint32_t id_pv = instr_desc<T, NPAD>(true);
       const uint32_t ring_a = smem_addr(ring), q_a = smem_addr(qop), p_a = smem_addr(pop);
       bool ok = true;
       auto issue_qk = [&](int i) -> bool {
@@ -415,8 +427,8 @@ __global__ void __launch_bounds__(THREADS, 2)
     auto flush = [&](int i) {
       wait(&p_free[i & 1], (i >> 1) & 1);
       tc_fence_after();
-      float o[16];
-      tmem_ld16(tmem + lane_base + 2 * NPAD, o);
+      float o[NPAD];
+      tmem_ld_cols<NPAD>(tmem + lane_base + 2 * NPAD, o);
       tc_fence_before();
       __syncwarp();
 #pragma unroll
@@ -461,13 +473,13 @@ __global__ void __launch_bounds__(THREADS, 2)
     for (int i = 0; i < n_tiles; ++i) {
       const int n_valid = min(TOK, end - (start + i * TOK));
       const bool valid = r < n_valid;
-      float sv[16];
+      float sv[NPAD];
       if (wait(&s_full[i & 1], (i >> 1) & 1)) {
         tc_fence_after();
-        tmem_ld16(tmem + lane_base + (i & 1) * NPAD, sv);
+        tmem_ld_cols<NPAD>(tmem + lane_base + (i & 1) * NPAD, sv);
       } else {
 #pragma unroll
-        for (int h = 0; h < 16; ++h) sv[h] = 0.f;
+        for (int h = 0; h < NPAD; ++h) sv[h] = 0.f;
       }
       tc_fence_before();
       __syncwarp();
@@ -507,11 +519,11 @@ __global__ void __launch_bounds__(THREADS, 2)
         // tile O starts from zero instead)
         if (i > 0 && wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
           tc_fence_after();
-          float o[16];
-          tmem_ld16(tmem + lane_base + 2 * NPAD, o);
+          float o[NPAD];
+          tmem_ld_cols<NPAD>(tmem + lane_base + 2 * NPAD, o);
 #pragma unroll
           for (int h = 0; h < NC; ++h) o[h] *= alpha[h];
-          tmem_st16(tmem + lane_base + 2 * NPAD, o);
+          tmem_st_cols<NPAD>(tmem + lane_base + 2 * NPAD, o);
         }
       }
       float pr[NC];
@@ -564,6 +576,7 @@ template <typename T, int G>
 cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
   const int ppc = tc_parts_per_cta(a);
   auto kern = decode_partition_tc_kernel<T, G>;
+  constexpr int SMEM_BYTES = Lay<16>::SMEM_BYTES;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // the cache [NB][Hkv][bs][128] as a 4-D tensor: 64 columns (stride 2 B),
@@ -609,17 +622,17 @@ cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t 
   return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
 }
 
-// A grouped decode in one launch, with NQ = 16 / G: first the groups' shared
-// spans, each CTA serving NQ members of a group (column = (member, head)),
-// one CTA per (group, run of NQ members, kv head, run of span partitions);
-// then the rest of every sequence past its shift, one CTA per (sequence, kv
-// head, run of partitions), on the same pipeline with one member's G columns.
-// Both kinds are in one grid, so the short span CTAs and the sequences' CTAs
-// share the SMs instead of running one kernel after the other.
+// The groups' shared spans, with NQ = 16 / G: each CTA serves NQ members of a
+// group (column = (member, head)), one CTA per (group, run of NQ members, kv
+// head, run of span partitions), partials into slots [0, a.slot_base) of every
+// member's row.  (The kernel can also take the rest of every sequence in the
+// same grid, blockIdx.x >= span_x; launched alone, the rest keeps its own
+// kernel and N, which measured faster.)
 template <typename T, int G>
 cudaError_t launch_group_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
-  constexpr int NQ = NPAD / G;
+  constexpr int NQ = 16 / G;
   auto kern = decode_partition_tc_kernel<T, G, NQ>;
+  constexpr int SMEM_BYTES = Lay<16>::SMEM_BYTES;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   CUtensorMap mk, mv;
@@ -657,16 +670,13 @@ cudaError_t launch_group_tc_t(const DecodeArgs& a, unsigned int* status, cudaStr
   const int span_parts = a.slot_base;
   const int rest_parts = a.num_partitions - a.slot_base;
   p.span_x = a.num_groups * p.q_groups;
-  // streaming: the rest by the decode kernel's rule; the spans by the same
-  // rule counting the rest's CTAs as well (they share the grid)
+  // streaming by the decode kernel's rule, counting the rest's CTAs, which run
+  // at the same time on the caller's stream
   const int64_t span_rows = static_cast<int64_t>(p.span_x) * a.Hkv;
   const int64_t rest_rows = static_cast<int64_t>(a.num_seqs) * a.Hkv;
-  p.parts_per_cta = tc_parts_per_cta(rest_rows, a.partition_size, rest_parts, 0);
-  const int64_t rest_ctas = rest_rows * ((rest_parts + p.parts_per_cta - 1) / p.parts_per_cta);
-  p.span_ppc = tc_parts_per_cta(span_rows, a.partition_size, span_parts, rest_ctas);
-  const int z_span = (span_parts + p.span_ppc - 1) / p.span_ppc;
-  const int z_rest = (rest_parts + p.parts_per_cta - 1) / p.parts_per_cta;
-  dim3 grid(p.span_x + a.num_seqs, a.Hkv, z_span > z_rest ? z_span : z_rest);
+  p.parts_per_cta = 1;
+  p.span_ppc = tc_parts_per_cta(span_rows, a.partition_size, span_parts, rest_rows * rest_parts);
+  dim3 grid(p.span_x, a.Hkv, (span_parts + p.span_ppc - 1) / p.span_ppc);
   return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
 }
 
@@ -739,15 +749,13 @@ bool tmap_available() { return encode_fn() != nullptr; }
 
 namespace {
 
-template <typename T, int G, int NQ>
+template <typename T, int G, int NQ, int NP = 16>
 cudaError_t launch_tcq_t(const MqArgs& m, unsigned int* status, cudaStream_t stream) {
-  DecodeArgs a{};
-  a.num_seqs = m.num_seqs;
-  a.Hkv = m.Hkv;
-  a.partition_size = m.partition_size;
-  a.num_partitions = m.num_partitions;
-  const int ppc = tc_parts_per_cta(a);
-  auto kern = decode_partition_tc_kernel<T, G, NQ>;
+  const int q_groups = (m.max_query_len + NQ - 1) / NQ;
+  const int ppc = tc_parts_per_cta(static_cast<int64_t>(m.num_seqs) * q_groups * m.Hkv,
+                                   m.partition_size, m.num_partitions, 0);
+  auto kern = decode_partition_tc_kernel<T, G, NQ, NP>;
+  constexpr int SMEM_BYTES = Lay<NP>::SMEM_BYTES;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   CUtensorMap mk, mv;
@@ -779,7 +787,7 @@ cudaError_t launch_tcq_t(const MqArgs& m, unsigned int* status, cudaStream_t str
   p.scale_log2 = m.scale * 1.4426950408889634f;
   p.query_start = m.query_start;
   p.total_q = m.total_q;
-  p.q_groups = (m.max_query_len + NQ - 1) / NQ;
+  p.q_groups = q_groups;
   p.seq_shift = nullptr;
   p.group_start = nullptr;
   p.slot_base = 0;
@@ -789,21 +797,30 @@ cudaError_t launch_tcq_t(const MqArgs& m, unsigned int* status, cudaStream_t str
   return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
 }
 
+// Query tokens per CTA (tc_query_tokens_per_cta): up to 16 columns on the
+// N = 16 kernel, else 32 columns on the N = 32 kernel, so 4 tokens at G = 8
+// (or 8 at G = 4) share one read of the sequence's K/V.
 template <typename T>
 cudaError_t launch_tcq_g(const MqArgs& m, unsigned int* status, cudaStream_t stream) {
   const int G = m.Hq / m.Hkv;
-  if (G == 8) return launch_tcq_t<T, 8, 2>(m, status, stream);
-  return m.max_query_len <= 2 ? launch_tcq_t<T, 4, 2>(m, status, stream)
-                              : launch_tcq_t<T, 4, 4>(m, status, stream);
+  const int nq = tc_query_tokens_per_cta(G, m.max_query_len);
+  if (G == 8) {
+    return nq == 2 ? launch_tcq_t<T, 8, 2>(m, status, stream)
+                   : launch_tcq_t<T, 8, 4, 32>(m, status, stream);
+  }
+  return nq == 2 ? launch_tcq_t<T, 4, 2>(m, status, stream)
+       : nq == 4 ? launch_tcq_t<T, 4, 4>(m, status, stream)
+                 : launch_tcq_t<T, 4, 8, 32>(m, status, stream);
 }
 
 }  // namespace
 
 bool decode_mq_tc_supported(const MqArgs& m) {
   const int G = m.Hkv > 0 ? m.Hq / m.Hkv : 0;
-  // up to 4 groups of 16 / G query tokens; longer query runs are prefill-like
+  // up to 64 (query token, head) columns, in one or two CTAs per sequence;
+  // longer query runs are prefill-like
   return (m.dtype == PA_F16 || m.dtype == PA_BF16) && m.D == DH && (G == 4 || G == 8) &&
-         m.max_query_len >= 1 && m.max_query_len * G <= 4 * NPAD && m.partition_size % TOK == 0 &&
+         m.max_query_len >= 1 && m.max_query_len * G <= 64 && m.partition_size % TOK == 0 &&
          static_cast<int64_t>(m.num_blocks) * m.Hkv * m.block_size < (int64_t(1) << 31) &&
          encode_fn() != nullptr;
 }

@@ -128,6 +128,14 @@ int launch_decode_mq(const MqArgs& a, unsigned int* status, void* stream);
 // token-major tcgen05 decode kernel with per-column causal limits, 16 / G query
 // tokens per CTA (decode_tc.cu).
 bool decode_mq_tc_supported(const MqArgs& a);
+// Query tokens one CTA of the token-major kernel serves for G query heads per kv
+// head: 2 (G * 2 <= 16 columns), 4 at G = 4 (16 columns), else 32 / G (the
+// N = 32 variant: 4 at G = 8, 8 at G = 4).
+inline int tc_query_tokens_per_cta(int G, int max_query_len) {
+  if (max_query_len <= 2) return 2;
+  if (G == 4 && max_query_len <= 4) return 4;
+  return 32 / G;
+}
 int launch_decode_mq_tc(const MqArgs& a, unsigned int* status, void* stream);
 int launch_decode_mq_reduce(const MqArgs& a, void* stream);
 

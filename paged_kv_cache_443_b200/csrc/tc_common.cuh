@@ -33,12 +33,13 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-// Instruction descriptor of kind::f16 with fp32 accumulation, M = 128, N = 16.
-template <typename T>
+// Instruction descriptor of kind::f16 with fp32 accumulation, M = 128, N (16 by default).
+template <typename T, int N = kNPad>
 __device__ __forceinline__ constexpr uint32_t instr_desc(bool a_mn_major) {
   constexpr uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
+  static_assert(N % 16 == 0 && N >= 16 && N <= 256, "N of an M = 128 MMA");
   return (1u << 4) | (fmt << 7) | (fmt << 10) | ((a_mn_major ? 1u : 0u) << 15) |
-         ((uint32_t)(kNPad >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
@@ -92,6 +93,18 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
       "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
       "r"(__float_as_uint(v[15]))
       : "memory");
+}
+
+// N consecutive TMEM columns (a multiple of 16) of this thread's lane.
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float* v) {
+#pragma unroll
+  for (int j = 0; j < N / 16; ++j) tmem_ld16(taddr + 16 * j, v + 16 * j);
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const float* v) {
+#pragma unroll
+  for (int j = 0; j < N / 16; ++j) tmem_st16(taddr + 16 * j, v + 16 * j);
 }
 
 // 2-D TMA tile load (this GPU's memory, no multicast) completing on `bar`.

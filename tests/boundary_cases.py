@@ -132,6 +132,10 @@ MULTI = [
     Case("m_verify_g4_p512", "f16", 4, 16, 512, lens=MQ_LENS, query_lens=(1, 4, 2, 3, 4, 1, 4, 3)),
     Case("m_verify_g8_q8_p512", "bf16", 8, 16, 512, lens=MQ_LENS, query_lens=(1, 8, 5, 8, 3, 8, 2, 7)),
     Case("m_verify_g1_p128", "f16", 1, 16, 128, lens=MQ_LENS, query_lens=(1, 4, 8, 3, 8, 5, 2, 6)),
+    # 32 (query token, head) columns: one CTA of the N = 32 kernel per sequence
+    Case("m_verify_g8_q4_p256", "bf16", 8, 16, 256, lens=MQ_LENS, query_lens=(4, 3, 4, 1, 4, 2, 4, 3)),
+    Case("m_verify_g4_q8_bs8_p128", "f16", 4, 8, 128, lens=MQ_LENS,
+         query_lens=(8, 5, 8, 1, 7, 8, 3, 8)),
     Case("m_prefill_g1_p256", "bf16", 1, 16, 256, lens=(200, 700, 1500, 90),
          query_lens=(200, 300, 260, 90)),
     Case("m_prefill_g4_bs8_p128", "bf16", 4, 8, 128, lens=(200, 700, 1500, 90),

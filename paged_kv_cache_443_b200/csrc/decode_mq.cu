@@ -19,14 +19,17 @@
 //
 // run on tcgen05 (kind::f16, fp32 accumulation in TMEM).  K and V tiles are
 // the TMA boxes of decode_tc.cu (one 4-D box per physical block, 128-byte
-// swizzle).  Each softmax thread owns one row: its running max, sum and
-// causal limit are thread-local, and a warp rescales its own 32 rows of O in
-// TMEM when one of its maxima grows by more than 2^8.
+// swizzle).  A row's running max, sum and causal limit belong to its two
+// softmax threads, and a warp rescales its half of its 32 rows of O in TMEM
+// when one of their maxima grows by more than 2^8.
 //
-// Roles (6 warps): warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
-// warps 2-5 Q staging, softmax and epilogue.  A ring of four K/V tiles (one
-// CTA per SM has to keep two tiles of loads in flight by itself), about 225 KB
-// of shared memory and all 512 TMEM columns: one CTA per SM.  Every wait is bounded; block ids
+// Roles (10 warps): warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
+// warps 2-9 Q staging, softmax and epilogue, two threads per row: the warps
+// w and w + 4 share a TMEM lane quadrant, one takes key columns 0-63 of each
+// tile (and dims 0-63 of O), the other 64-127, and the pair agrees on each
+// row's maximum through shared memory and a named barrier.  A ring of three
+// K/V tiles, about 196 KB of shared memory and all 512 TMEM columns: one CTA
+// per SM.  Every wait is bounded; block ids
 // outside the pool are skipped and flagged; inconsistent query offsets are
 // flagged (PA_DEVERR_CONTEXT) and their sequence skipped.
 #include <cuda.h>
@@ -49,7 +52,7 @@ constexpr unsigned FULL = 0xffffffffu;
 constexpr int TOK = 128;                   // keys per tile
 constexpr int MR = 128;                    // query rows per CTA
 constexpr int DH = 128;
-constexpr int SLOTS = 4;
+constexpr int SLOTS = 3;
 constexpr int SLOT_BYTES = TOK * 256;      // K or V tile (as in decode_tc.cu): 32 KB
 constexpr int GROUP_BYTES = 2048;
 constexpr int HALF_OFF = 1024;
@@ -61,9 +64,12 @@ constexpr int OFF_P = OFF_Q + OPA_BYTES;   // two P buffers
 constexpr int OFF_BAR = OFF_P + 2 * OPA_BYTES;
 constexpr int NBARS = 2 * SLOTS + 9;
 constexpr int OFF_TMEM = OFF_BAR + NBARS * 8;
-constexpr int SMEM_USED = OFF_TMEM + 16;
+constexpr int OFF_RMAX = (OFF_TMEM + 16 + 15) / 16 * 16;   // [2 tiles][2 halves][MR] row maxima
+constexpr int OFF_RSUM = OFF_RMAX + 2 * 2 * MR * 4;          // [2 halves][MR] row sums
+constexpr int SMEM_USED = OFF_RSUM + 2 * MR * 4;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;                 // producer, MMA, 8 softmax warps
+constexpr int NSOFT = 256;                   // softmax threads: two per row
 constexpr int TMEM_COLS = 512;             // S0 [0,128), S1 [128,256), O [256,384)
 constexpr int O_COL = 256;
 constexpr float RESCALE_THRESHOLD = 8.0f;
@@ -216,11 +222,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int j = 0; j < 2; ++j) {
       mbar_init(&s_full[j], 1);
-      mbar_init(&s_free[j], 4);
-      mbar_init(&p_full[j], 4);
+      mbar_init(&s_free[j], 8);
+      mbar_init(&p_full[j], 8);
       mbar_init(&p_free[j], 1);
     }
-    mbar_init(q_ready, 4);
+    mbar_init(q_ready, 8);
     fence_mbar_init();
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
@@ -280,23 +286,31 @@ __global__ void __launch_bounds__(THREADS, 1)
     return;
   }
 
-  // rows of this CTA: r = il * G + hl  (query token il of the block, head hl)
+  // rows of this CTA: r = il * G + hl  (query token il of the block, head hl).
+  // Each row has two softmax threads in two warps of the same TMEM lane
+  // quadrant: `half` 0 takes key columns 0-63 of a tile (and dims 0-63 of O),
+  // half 1 columns 64-127 (dims 64-127).
   const int quad = warp & 3;
+  const int half = warp >= 6 ? 1 : 0;
   const int r = quad * 32 + lane;
   const int il = r / G, hl = r % G;
   const bool row_valid = warp >= 2 && qb * QB + il < Qb;
   const int64_t t = static_cast<int64_t>(q0) + qb * QB + il;          // query token index
   const int pos = L - Qb + qb * QB + il;                               // its position
+  float* rmax = reinterpret_cast<float*>(smem + OFF_RMAX);            // [2][2][MR]
+  float* rsum = reinterpret_cast<float*>(smem + OFF_RSUM);            // [2][MR]
 
   if (warp >= 2) {
-    // Q operand: row r = q[t][g*G + hl][:], zero for rows past the block's tokens
+    // Q operand: row r = q[t][g*G + hl][:] (this thread its half of the 16
+    // chunks), zero for rows past the block's tokens
     const T* src = static_cast<const T*>(p.q) + (t * p.Hq + g * G + hl) * DH;
-    uint4 v[DH / 8];                                 // all 16 loads in flight at once
+    uint4 v[DH / 16];
 #pragma unroll
-    for (int c = 0; c < DH / 8; ++c)
-      v[c] = row_valid ? __ldg(reinterpret_cast<const uint4*>(src + c * 8)) : make_uint4(0, 0, 0, 0);
+    for (int c = 0; c < DH / 16; ++c)
+      v[c] = row_valid ? __ldg(reinterpret_cast<const uint4*>(src + (half * 8 + c) * 8))
+                       : make_uint4(0, 0, 0, 0);
 #pragma unroll
-    for (int c = 0; c < DH / 8; ++c) *reinterpret_cast<uint4*>(qop + opa_chunk(r, c)) = v[c];
+    for (int c = 0; c < DH / 16; ++c) *reinterpret_cast<uint4*>(qop + opa_chunk(r, half * 8 + c)) = v[c];
     fence_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(q_ready);
@@ -352,12 +366,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     __syncwarp();
   } else if (warp >= 2) {
-    // ================= softmax: one row per thread =================
+    // ================= softmax: two threads per row =================
     // A warp whose 32 rows hold no query token (few queries per sequence) only
     // keeps pace with the barriers and zeroes V rows; its P rows stay zero.
+    // The two threads of a row meet at a named barrier of their warp pair
+    // (id 3 + quad) to agree on the row's maximum each tile.
     const bool warp_active = __any_sync(FULL, row_valid);
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    float m_run = -INFINITY, l_sum = 0.f;
+    const int col0 = half * 64;                        // this thread's key / dim columns
+    float m_run = -INFINITY, l_half = 0.f;
     bool ok = true;
     auto wait = [&](uint64_t* bar, uint32_t parity) {
       if (ok) ok = mbar_wait(bar, parity, p.status);
@@ -368,8 +385,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int buf = 0; buf < 2; ++buf)
 #pragma unroll
-        for (int c = 0; c < TOK / 8; ++c)
-          *reinterpret_cast<uint4*>(pop + buf * OPA_BYTES + opa_chunk(r, c)) = make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(pop + buf * OPA_BYTES + opa_chunk(r, half * 8 + c)) =
+              make_uint4(0, 0, 0, 0);
     }
     for (int i = 0; i < n_tiles; ++i) {
       const int tile0 = kstart + i * TOK;
@@ -377,13 +395,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       wait(&s_full[i & 1], (i >> 1) & 1);
       if (warp_active) {
         const int lim = row_valid ? min(pos - tile0, n_valid - 1) : -1;  // last key column
-        float sv[TOK];
+        float sv[64];
         if (ok) {
           tc_fence_after();
-          tmem_ld128(tmem + lane_base + (i & 1) * 128, sv);
+          tmem_ld32(tmem + lane_base + (i & 1) * 128 + col0, sv);
+          tmem_ld32(tmem + lane_base + (i & 1) * 128 + col0 + 32, sv + 32);
         } else {
 #pragma unroll
-          for (int j = 0; j < TOK; ++j) sv[j] = 0.f;
+          for (int j = 0; j < 64; ++j) sv[j] = 0.f;
         }
         tc_fence_before();
         __syncwarp();
@@ -392,28 +411,33 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int k = 0; k < 8; ++k) pm[k] = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < TOK; ++j) {
-          sv[j] = j <= lim ? sv[j] * p.scale_log2 : -INFINITY;
+        for (int j = 0; j < 64; ++j) {
+          sv[j] = col0 + j <= lim ? sv[j] * p.scale_log2 : -INFINITY;
           pm[j & 7] = fmaxf(pm[j & 7], sv[j]);
         }
-        const float tmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                                 fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        float tmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                           fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        // the row's maximum over both halves (the buffer alternates by tile, so
+        // a partner a tile ahead never overwrites what this thread still reads)
+        rmax[((i & 1) * 2 + half) * MR + r] = tmax;
+        named_sync(3 + quad, 64);
+        tmax = fmaxf(tmax, rmax[((i & 1) * 2 + (half ^ 1)) * MR + r]);
         const bool need = tmax > m_run + RESCALE_THRESHOLD;
-        if (__any_sync(FULL, need)) {
+        if (__any_sync(FULL, need)) {                  // the same for both warps of the pair
           const float mnew = fmaxf(m_run, tmax);
           const float alpha = (m_run == -INFINITY) ? 0.f : exp2f(m_run - mnew);
           m_run = mnew;
-          l_sum *= alpha;
-          // O must hold every earlier tile before it is rescaled
+          l_half *= alpha;
+          // O must hold every earlier tile before it is rescaled (its dims col0..col0+63)
           if (i > 0 && wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < DH / 32; ++c) {
+            for (int c = 0; c < 2; ++c) {
               float o[32];
-              tmem_ld32(tmem + lane_base + O_COL + c * 32, o);
+              tmem_ld32(tmem + lane_base + O_COL + col0 + c * 32, o);
 #pragma unroll
               for (int j = 0; j < 32; ++j) o[j] *= alpha;
-              tmem_st32(tmem + lane_base + O_COL + c * 32, o);
+              tmem_st32(tmem + lane_base + O_COL + col0 + c * 32, o);
             }
           }
         }
@@ -423,7 +447,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int k = 0; k < 8; ++k) ps[k] = 0.f;
 #pragma unroll
-        for (int c = 0; c < TOK / 8; ++c) {
+        for (int c = 0; c < 8; ++c) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -435,25 +459,22 @@ __global__ void __launch_bounds__(THREADS, 1)
             w[e] = static_cast<uint32_t>(to_bits<T>(p0)) |
                    (static_cast<uint32_t>(to_bits<T>(p1)) << 16);
           }
-          *reinterpret_cast<uint4*>(pb + opa_chunk(r, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(pb + opa_chunk(r, half * 8 + c)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        l_sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        l_half += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       } else {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[i & 1]);
       }
       if (n_valid < TOK) {
-        // the last tile: zero the V rows of keys past the range, so that
-        // whatever they hold adds 0 * 0 to O
+        // the last tile: zero the V rows of keys past the range (this thread
+        // its 64-dim half of row r), so that whatever they hold adds 0 * 0 to O
         const int u = 2 * i + 1, s_ = u % SLOTS;
         if (wait(&ring_full[s_], (u / SLOTS) & 1) && r >= n_valid) {
-          uint8_t* row = ring + s_ * SLOT_BYTES + (r >> 3) * GROUP_BYTES + (r & 7) * 128;
+          uint8_t* row = ring + s_ * SLOT_BYTES + (r >> 3) * GROUP_BYTES + (r & 7) * 128 + half * HALF_OFF;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            *reinterpret_cast<uint4*>(row + c * 16) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(row + HALF_OFF + c * 16) = make_uint4(0, 0, 0, 0);
-          }
+          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(row + c * 16) = make_uint4(0, 0, 0, 0);
         }
       }
       fence_async_smem();
@@ -461,18 +482,21 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[i & 1]);
     }
-    // ---- epilogue: row r of O ----
+    // ---- epilogue: row r of O, dims col0..col0+63; the row's sum over both halves ----
+    rsum[half * MR + r] = l_half;
+    named_sync(3 + quad, 64);
+    const float l_sum = l_half + rsum[(half ^ 1) * MR + r];
     wait(&p_free[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1);
     tc_fence_after();
     const int64_t hq = t * p.Hq + g * G + hl;
 #pragma unroll 1
-    for (int c = 0; c < (warp_active ? DH / 32 : 0); ++c) {
+    for (int c = 0; c < (warp_active ? 2 : 0); ++c) {
       float o[32];
-      tmem_ld32(tmem + lane_base + O_COL + c * 32, o);
+      tmem_ld32(tmem + lane_base + O_COL + col0 + c * 32, o);
       if (ok && row_valid) {
         if (single) {
           const float inv = 1.f / l_sum;
-          T* dst = static_cast<T*>(p.out) + hq * DH + c * 32;
+          T* dst = static_cast<T*>(p.out) + hq * DH + col0 + c * 32;
 #pragma unroll
           for (int j = 0; j < 32; j += 8) {
             uint32_t w[4];
@@ -484,11 +508,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         } else {
           const int64_t slot = hq * p.num_partitions + part;
-          float* dst = p.ws_o + slot * DH + c * 32;
+          float* dst = p.ws_o + slot * DH + col0 + c * 32;
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
             *reinterpret_cast<float4*>(dst + j) = make_float4(o[j], o[j + 1], o[j + 2], o[j + 3]);
-          if (c == 0) {
+          if (c == 0 && half == 0) {
             p.ws_m[slot] = m_run;
             p.ws_l[slot] = l_sum;
           }
@@ -497,9 +521,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   }
 
-  // ---- teardown: warps 1-5 meet, warp 1 frees TMEM ----
+  // ---- teardown: warps 1-9 meet, warp 1 frees TMEM ----
   tc_fence_before();
-  named_sync(2, 160);
+  named_sync(2, THREADS - 32);
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),

@@ -258,6 +258,10 @@ KERNEL_SOURCES = {
     "decode_partition_tc_kernel": ("decode_tc.cu", "tc_common.cuh", "pa_device.cuh", "pa_internal.h"),
     "decode_partition_tc8_kernel": ("decode_tc8.cu", "tc_common.cuh", "pa_device.cuh",
                                     "pa_internal.h"),
+    # pa_decode_grouped: the span and rest kernels (decode_tc.cu, or decode.cu
+    # for G = 1, 2) and the reduce (decode.cu)
+    "decode_grouped": ("decode_tc.cu", "decode.cu", "tc_common.cuh", "pa_device.cuh",
+                       "pa_internal.h"),
 }
 
 
@@ -650,7 +654,7 @@ def run_ours(args):
         kname = ("decode_grouped: decode_partition_tc_kernel (the families' shared spans, "
                  "16/G members per CTA) next to " + partition_kernel(spec, P) +
                  " (the rest of every sequence), then decode_reduce_kernel")
-        traffic, traffic_note = None, "three kernels timed together; see the ncu launch list"
+        traffic, traffic_note = profiled_traffic(args.workload, "decode_grouped", P)
 
     result = None
     if rank == 0:

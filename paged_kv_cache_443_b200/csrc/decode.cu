@@ -83,6 +83,16 @@ struct Cfg {
   static_assert(TOK % kStageTokens == 0 && TOK <= 256, "a stage is whole table words of blocks");
 };
 
+// (d0, d1) += (a0 * b0, a1 * b1) as one paired fp32 FMA (each half rounded
+// as fmaf would round it).
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 d, {%0, %1};\n\t"
+      "fma.rn.f32x2 d, a, b, d;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // q row chunk of EPL elements of TQ (global memory, read-only path) to fp32.
 template <typename TQ, int EPL>
 __device__ __forceinline__ void load_q(const TQ* src, float* f) {
@@ -314,10 +324,11 @@ __global__ void __launch_bounds__(Cfg<TK, D, G, NCW>::THREADS)
       E::load(Ks + row * D + c * C::EPL, kf);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        float acc = 0.f;
+        // even and odd elements in the two halves of a paired FMA
+        float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-        for (int e = 0; e < C::EPL; ++e) acc = fmaf(qf[h][e], kf[e], acc);
-        part_dot[h * C::ITERS + it] = acc;
+        for (int e = 0; e < C::EPL; e += 2) fma2(a0, a1, qf[h][e], qf[h][e + 1], kf[e], kf[e + 1]);
+        part_dot[h * C::ITERS + it] = a0 + a1;
       }
     }
     reduce_scatter<C::NV, C::LPR / 2>(part_dot, lane);
@@ -393,7 +404,7 @@ __global__ void __launch_bounds__(Cfg<TK, D, G, NCW>::THREADS)
         for (int h = 0; h < G; ++h) {
           const float pr = sc[h * C::TPW + row_local];
 #pragma unroll
-          for (int e = 0; e < C::EPL; ++e) o[h][e] = fmaf(pr, vf[e], o[h][e]);
+          for (int e = 0; e < C::EPL; e += 2) fma2(o[h][e], o[h][e + 1], pr, pr, vf[e], vf[e + 1]);
         }
       }
     }

@@ -134,6 +134,25 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v) {
   for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 2^x by the SFU's approximation (relative error about 2^-22; 2^-inf = +0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Two floats rounded to T and packed (the first in the low half), one cvt.
+template <typename T>
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&v);
+  } else {
+    const __half2 v = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&v);
+  }
+}
+
 // Byte offset of the 16-byte chunk c (elements 8c..8c+7) of row r of a
 // 128 x 128 16-bit operand stored as two 64-column halves with the 128-byte
 // swizzle (the canonical K-major layout).
@@ -407,16 +426,26 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[i & 1]);
+        // Every column of this thread's half visible to every row of the warp
+        // (all but the diagonal and last tiles): no mask, and the scale (> 0)
+        // moves into the exponent's FMA below, so the scores stay raw here.
+        const bool open = __all_sync(FULL, col0 + 63 <= lim);
         float pm[8];                                   // 8 independent partial maxima
 #pragma unroll
         for (int k = 0; k < 8; ++k) pm[k] = -INFINITY;
+        if (open) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          sv[j] = col0 + j <= lim ? sv[j] * p.scale_log2 : -INFINITY;
-          pm[j & 7] = fmaxf(pm[j & 7], sv[j]);
+          for (int j = 0; j < 64; ++j) pm[j & 7] = fmaxf(pm[j & 7], sv[j]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            sv[j] = col0 + j <= lim ? sv[j] * p.scale_log2 : -INFINITY;
+            pm[j & 7] = fmaxf(pm[j & 7], sv[j]);
+          }
         }
         float tmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                            fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        if (open) tmax *= p.scale_log2;
         // the row's maximum over both halves (the buffer alternates by tile, so
         // a partner a tile ahead never overwrites what this thread still reads)
         rmax[((i & 1) * 2 + half) * MR + r] = tmax;
@@ -446,18 +475,25 @@ __global__ void __launch_bounds__(THREADS, 1)
         float ps[8];                                   // 8 independent partial sums
 #pragma unroll
         for (int k = 0; k < 8; ++k) ps[k] = 0.f;
+        // P = 2^(scale * s - m): one FMA and one ex2 per column when open
+        const float neg_m = -m_run;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float p0 = sv[8 * c + 2 * e] == -INFINITY ? 0.f : exp2f(sv[8 * c + 2 * e] - m_run);
-            const float p1 =
-                sv[8 * c + 2 * e + 1] == -INFINITY ? 0.f : exp2f(sv[8 * c + 2 * e + 1] - m_run);
+            const float s0 = sv[8 * c + 2 * e], s1 = sv[8 * c + 2 * e + 1];
+            float p0, p1;
+            if (open) {
+              p0 = ex2_approx(fmaf(s0, p.scale_log2, neg_m));
+              p1 = ex2_approx(fmaf(s1, p.scale_log2, neg_m));
+            } else {
+              p0 = s0 == -INFINITY ? 0.f : ex2_approx(s0 + neg_m);
+              p1 = s1 == -INFINITY ? 0.f : ex2_approx(s1 + neg_m);
+            }
             ps[2 * e] += p0;
             ps[2 * e + 1] += p1;
-            w[e] = static_cast<uint32_t>(to_bits<T>(p0)) |
-                   (static_cast<uint32_t>(to_bits<T>(p1)) << 16);
+            w[e] = pack2<T>(p0, p1);
           }
           *reinterpret_cast<uint4*>(pb + opa_chunk(r, half * 8 + c)) = make_uint4(w[0], w[1], w[2], w[3]);
         }

@@ -10,7 +10,7 @@
 // tensor cores with tokens as the MMA's M dimension:
 //
 //   S^T [128 tokens x 16] = K [128 x 128] . Q^T [128 x 16]     (heads padded to 16)
-//   O^T [128 dims   x 16] += V^T [128 x 128] . P^T [128 x 16]
+//   O^T [128 dims   x 16] += V^T [128 x 128] . P^T [128 x 16]     (both MN-major)
 //
 // Roles in a CTA of 6 warps, one CTA per (sequence, kv head, run of partitions):
 //   warp 0   producer: block-table lookups, one TMA load per physical block of
@@ -58,6 +58,30 @@ constexpr int GROUP_BYTES = 2048;            // 8 token rows, both 64-column hal
 constexpr int HALF_OFF = 1024;               // second 64-column half of a group
 constexpr int THREADS = 192;
 constexpr float RESCALE_THRESHOLD = 8.0f;    // log2 units: raise the max past 2^8 growth
+// P^T is stored MN-major without swizzle: a 16-byte row holds 8 columns
+// (heads) of one token, 128 tokens make a 2 KB chunk of 8 columns, and the
+// chunks of columns 8-15 (and 16-31) follow at P_CHUNK strides.
+constexpr int P_CHUNK = TOK * 16;
+
+// Shared-memory matrix descriptor without swizzle (the interleaved layout):
+// core matrices of 8 rows of 16 bytes, 128 contiguous bytes each; for an
+// MN-major operand sbo steps 8 rows along K and lbo the next 16 bytes of MN.
+__device__ __forceinline__ uint64_t smem_desc_plain(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
+}
+
+// Two floats rounded to T and packed (the first in the low half), one cvt.
+template <typename T>
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&v);
+  } else {
+    const __half2 v = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&v);
+  }
+}
 
 // Shared-memory and TMEM layout for N = NP columns (16, or 32 for 32 query
 // tokens x heads): a ring of SLOTS K/V tiles (three at N = 16; two at N = 32,
@@ -68,7 +92,7 @@ template <int NP>
 struct Lay {
   static constexpr int NPAD = NP;
   static constexpr int SLOTS = NP <= 16 ? 3 : 2;
-  static constexpr int OPB_BYTES = 2 * NP * 128;
+  static constexpr int OPB_BYTES = 2 * NP * 128;   // Q^T (K-major) or P^T (MN-major): NP x 128 16-bit
   static constexpr int OFF_RING = 0;
   static constexpr int OFF_Q = OFF_RING + SLOTS * SLOT_BYTES;
   static constexpr int OFF_P = OFF_Q + OPB_BYTES;
@@ -355,7 +379,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     // ================= MMA issuer =================
     if (lane == 0) {
       const uint32_t id_qk = instr_desc<T, NPAD>(false);
-      const uint32_t id_pv = instr_desc<T, NPAD>(true);
+      const uint32_t id_pv = instr_desc<T, NPAD>(true) | (1u << 16);   // V^T and P^T MN-major
       const uint32_t ring_a = smem_addr(ring), q_a = smem_addr(qop), p_a = smem_addr(pop);
       bool ok = true;
       auto issue_qk = [&](int i) -> bool {
@@ -386,8 +410,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         for (int k = 0; k < TOK / 16; ++k) {
           const uint64_t a =
               smem_desc(ring_a + s * SLOT_BYTES + k * 2 * GROUP_BYTES, HALF_OFF, GROUP_BYTES);
-          const uint64_t bp =
-              smem_desc(p_a + (i & 1) * OPB_BYTES + (k >> 2) * (NPAD * 128) + (k & 3) * 32, 16, 1024);
+          const uint64_t bp = smem_desc_plain(p_a + (i & 1) * OPB_BYTES + k * 16 * 16, P_CHUNK, 128);
           mma_f16(d, a, bp, id_pv, (!first || k > 0) ? 1u : 0u);
         }
         mma_commit(&ring_empty[s]);
@@ -534,10 +557,19 @@ __global__ void __launch_bounds__(THREADS, 2)
         l_part[h] += pr[h];
       }
       if (i >= 2) wait(&p_free[i & 1], ((i >> 1) - 1) & 1);
-      uint8_t* pb = pop + (i & 1) * OPB_BYTES + (r >> 6) * (NPAD * 128);
+      // token r's columns are 16-byte rows of the MN-major P^T operand: heads
+      // 8c .. 8c + 7 at chunk c (columns >= NC stay 0)
+      uint8_t* pb = pop + (i & 1) * OPB_BYTES + r * 16;
 #pragma unroll
-      for (int h = 0; h < NC; ++h)
-        *reinterpret_cast<uint16_t*>(pb + sw128(h, r & 63)) = to_bits<T>(pr[h]);
+      for (int c = 0; c < (NC + 7) / 8; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int h = 8 * c + 2 * e;
+          w[e] = pack2<T>(h < NC ? pr[h < NC ? h : 0] : 0.f, h + 1 < NC ? pr[h + 1 < NC ? h + 1 : 0] : 0.f);
+        }
+        *reinterpret_cast<uint4*>(pb + c * P_CHUNK) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
       if (n_valid < TOK) {
         // the last tile: zero the V rows of tokens past the end, so that
         // whatever they hold (unused slots, stale data) adds 0 * 0 to O

@@ -11,7 +11,7 @@
 // run on kind::f8f6f4 with the cache codes as they are in shared memory:
 //
 //   S^T [128 tokens x 16] = K [128 x 128] . Q^T [128 x 16]         K-major K
-//   O^T [128 dims   x 16] += V^T [128 x 128] . P^T [128 x 16]      MN-major V^T
+//   O^T [128 dims   x 16] += V^T [128 x 128] . P^T [128 x 16]      MN-major V^T, P^T
 //
 // * Q: split into three E4M3 terms, Q * 2^e = Q1 + Q2 + Q3 (each the nearest
 //   E4M3 value of what the previous terms left; e a per-head power of two
@@ -64,7 +64,7 @@ constexpr int PTERM = 2;                    // E4M3 terms of P
 constexpr int SLOTS = 3;                    // tiles per ring (one ring for K, one for V)
 constexpr int TILE_BYTES = TOK * DH;        // one tile of codes: 16 KB
 constexpr int QT_BYTES = NPAD * DH;         // one query term: 16 rows x 128 codes
-constexpr int PT_BYTES = NPAD * TOK;        // one P term: 16 rows x 128 tokens
+constexpr int PT_BYTES = NPAD * TOK;        // one P term: 128 tokens x 16 heads (MN-major)
 constexpr int PB_BYTES = PTERM * PT_BYTES;  // one P buffer (both terms)
 constexpr int OFF_KR = 0;
 constexpr int OFF_VR = OFF_KR + SLOTS * TILE_BYTES;
@@ -93,6 +93,18 @@ static_assert(OFF_VR % 1024 == 0 && OFF_Q % 1024 == 0 && OFF_P % 1024 == 0 &&
 constexpr uint32_t kIdescE4M3 = (1u << 4) | (static_cast<uint32_t>(NPAD >> 3) << 17) |
                                 (static_cast<uint32_t>(128 >> 4) << 24);
 constexpr uint32_t kIdescE4M3_AMN = kIdescE4M3 | (1u << 15);
+// O += V^T P^T with V^T and P^T both MN-major (bits 15 and 16).
+constexpr uint32_t kIdescE4M3_AMN_BMN = kIdescE4M3_AMN | (1u << 16);
+
+// Shared-memory matrix descriptor without swizzle (the interleaved layout):
+// 16-byte core rows, 8 rows of a core matrix 16 bytes apart.  For the MN-major
+// P^T operand: each token's 16 head codes are one 16-byte row, so a core
+// matrix is 8 consecutive tokens (128 contiguous bytes), the next 8 tokens
+// sbo = 128 bytes on, and lbo (the next 16 heads) is never used at N = 16.
+__device__ __forceinline__ uint64_t smem_desc_plain(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
+}
 
 __device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
                                          uint32_t accumulate) {
@@ -371,8 +383,9 @@ __global__ void __launch_bounds__(THREADS, 2)
 #pragma unroll
           for (int k = 0; k < TOK / 32; ++k) {  // 32 tokens per MMA: four 8-token groups
             const uint64_t a = smem_desc(v_a + s * TILE_BYTES + k * 4096, 1024, 1024);
-            const uint64_t bp = smem_desc(p_a + (i & 1) * PB_BYTES + term * PT_BYTES + k * 32, 16, 1024);
-            mma_e4m3(d, a, bp, kIdescE4M3_AMN, (!first || term > 0 || k > 0) ? 1u : 0u);
+            const uint64_t bp =
+                smem_desc_plain(p_a + (i & 1) * PB_BYTES + term * PT_BYTES + k * 32 * NPAD, 128, 128);
+            mma_e4m3(d, a, bp, kIdescE4M3_AMN_BMN, (!first || term > 0 || k > 0) ? 1u : 0u);
           }
         }
         mma_commit(&vr_empty[s]);
@@ -398,11 +411,6 @@ __global__ void __launch_bounds__(THREADS, 2)
       l_part[h] = 0.f;
       sc[h] = p.scale_log2 * qs[h];
     }
-    // byte of token r in row h of a K-major, 128-byte-swizzled P term
-    uint32_t pcol[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-      pcol[h] = h * 128 + ((((r >> 4) ^ h) & 7) << 4) + (r & 15);
     bool ok = true;
     auto wait = [&](uint64_t* bar, uint32_t parity) {
       if (ok) ok = mbar_wait(bar, parity, p.status);
@@ -514,22 +522,23 @@ __global__ void __launch_bounds__(THREADS, 2)
         l_part[h] += pr[h];
       }
       if (i >= 2) wait(&p_free[i & 1], ((i >> 1) - 1) & 1);
-      uint8_t* pb = pop + (i & 1) * PB_BYTES;
+      // P * 2^6 = P1 + P2, two E4M3 codes per head (heads h, h+1 in one pair);
+      // token r's 16 head codes of each term are one 16-byte row of the
+      // MN-major P^T operand (heads >= G are 0)
+      uint32_t w1[4] = {0u, 0u, 0u, 0u}, w2[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
       for (int h = 0; h < G; h += 2) {
-        // P * 2^6 = P1 + P2, two E4M3 codes per head (heads h, h+1 in one pair)
         const float x0 = pr[h] * P_UP;
         const float x1 = (h + 1 < G) ? pr[h + 1] * P_UP : 0.f;
         const uint32_t c1 = to_e4m3x2(x0, x1);
         const float2 d1 = from_e4m3x2(c1);
         const uint32_t c2 = to_e4m3x2(x0 - d1.x, x1 - d1.y);
-        pb[pcol[h]] = static_cast<uint8_t>(c1);
-        pb[PT_BYTES + pcol[h]] = static_cast<uint8_t>(c2);
-        if (h + 1 < G) {
-          pb[pcol[h + 1]] = static_cast<uint8_t>(c1 >> 8);
-          pb[PT_BYTES + pcol[h + 1]] = static_cast<uint8_t>(c2 >> 8);
-        }
+        w1[h >> 2] |= c1 << ((h & 2) * 8);
+        w2[h >> 2] |= c2 << ((h & 2) * 8);
       }
+      uint8_t* pb = pop + (i & 1) * PB_BYTES + r * NPAD;
+      *reinterpret_cast<uint4*>(pb) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+      *reinterpret_cast<uint4*>(pb + PT_BYTES) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
       if (n_valid < TOK) {
         // the last tile: zero the V rows of tokens past the end, so that
         // whatever they hold (unused slots, stale data) adds 0 * 0 to O

@@ -88,3 +88,16 @@ def test_multi_query_case_is_sensitive(case):
             d = np.abs(got - want_all[t, h]).max()
             assert d > tol, (case.name, t, h, j, kind, how, d)
     assert "past_limit" in kinds
+
+
+def test_cases_cover_every_kind_of_boundary():
+    """Across the cases, the spikes sit at every kind of position a slip can
+    hit: first and last token, block, partition and tile edges, the last tile
+    of a partition, the split between a family's shared span and the rest, and
+    the key just past a query's causal limit."""
+    from collections import Counter
+    kinds = Counter()
+    for case in DECODE + GROUPED + MULTI:
+        kinds.update(k for (_, _, _, k) in case.scenario().spikes.rows.values())
+    for k in ("end", "start", "partition", "block", "tile", "last_tile", "shared", "past_limit"):
+        assert kinds[k] >= 20, (k, kinds)

@@ -64,8 +64,10 @@ constexpr float RESCALE_THRESHOLD = 8.0f;    // log2 units: raise the max past 2
 constexpr int P_CHUNK = TOK * 16;
 
 // Shared-memory matrix descriptor without swizzle (the interleaved layout):
-// core matrices of 8 rows of 16 bytes, 128 contiguous bytes each; for an
-// MN-major operand sbo steps 8 rows along K and lbo the next 16 bytes of MN.
+// core matrices of 8 rows of 16 bytes, 128 contiguous bytes each.  For an
+// MN-major operand in this layout the leading offset (lbo) steps to the next
+// 8 rows along K and the stride offset (sbo) to the next 16 bytes along MN
+// (the swizzled MN-major layouts use them the other way round).
 __device__ __forceinline__ uint64_t smem_desc_plain(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
@@ -410,7 +412,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         for (int k = 0; k < TOK / 16; ++k) {
           const uint64_t a =
               smem_desc(ring_a + s * SLOT_BYTES + k * 2 * GROUP_BYTES, HALF_OFF, GROUP_BYTES);
-          const uint64_t bp = smem_desc_plain(p_a + (i & 1) * OPB_BYTES + k * 16 * 16, P_CHUNK, 128);
+          const uint64_t bp = smem_desc_plain(p_a + (i & 1) * OPB_BYTES + k * 16 * 16, 128, P_CHUNK);
           mma_f16(d, a, bp, id_pv, (!first || k > 0) ? 1u : 0u);
         }
         mma_commit(&ring_empty[s]);

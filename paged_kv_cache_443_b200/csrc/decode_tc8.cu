@@ -99,8 +99,9 @@ constexpr uint32_t kIdescE4M3_AMN_BMN = kIdescE4M3_AMN | (1u << 16);
 // Shared-memory matrix descriptor without swizzle (the interleaved layout):
 // 16-byte core rows, 8 rows of a core matrix 16 bytes apart.  For the MN-major
 // P^T operand: each token's 16 head codes are one 16-byte row, so a core
-// matrix is 8 consecutive tokens (128 contiguous bytes), the next 8 tokens
-// sbo = 128 bytes on, and lbo (the next 16 heads) is never used at N = 16.
+// matrix is 8 consecutive tokens (128 contiguous bytes); the leading offset
+// steps to the next 8 tokens (128 bytes on) and the stride offset, the step to
+// the next 16 heads, is never used at N = 16.
 __device__ __forceinline__ uint64_t smem_desc_plain(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);

@@ -487,7 +487,8 @@ extern "C" pa_status pa_reshape_and_cache_fp8(const void* key, const void* value
 }
 
 // Partition length pa_decode_multi uses for partition_size = 0.  The
-// query-major kernel (many query tokens) holds one CTA per SM, so the keys are
+// query-major kernel (many query tokens; two query tiles of kMqRows rows per
+// CTA) holds one CTA per SM, so the keys are
 // split only as far as it takes to give at least two CTAs per SM: a prefill
 // chunk of hundreds of tokens needs no split at all, and every split costs
 // fp32 partials for all of its query rows.  Few queries per sequence (the
@@ -507,7 +508,8 @@ int auto_partition_multi(int num_seqs, int num_heads, int num_kv_heads, int max_
     return P < P0 ? P0 : P;
   }
   const int64_t qblocks = (max_query_len + pa::kMqRows / G - 1) / (pa::kMqRows / G);
-  const int64_t base = static_cast<int64_t>(num_seqs) * num_kv_heads * qblocks;
+  const int64_t base = static_cast<int64_t>(num_seqs) * num_kv_heads *
+                       ((qblocks + pa::kMqTiles - 1) / pa::kMqTiles);   // CTAs per key range
   const int64_t want = 2ll * num_sms();
   int64_t np = base >= want ? 1 : (want + base - 1) / base;
   const int64_t np_max = (max_context_len + P0 - 1) / P0;
@@ -563,7 +565,8 @@ extern "C" pa_status pa_decode_multi(void* out, const void* q, const void* k_cac
   const int64_t NP = num_partitions(max_context_len, P);
   const int G = num_heads / num_kv_heads;
   const int64_t qblocks = total_q > 0 ? (max_query_len + pa::kMqRows / G - 1) / (pa::kMqRows / G) : 0;
-  if (qblocks * NP > 65535) return pa::fail(PA_ERR_UNSUPPORTED, "%s: too many query blocks x partitions", fn);
+  const int64_t qpairs = (qblocks + pa::kMqTiles - 1) / pa::kMqTiles;
+  if (qpairs * NP > 65535) return pa::fail(PA_ERR_UNSUPPORTED, "%s: too many query blocks x partitions", fn);
   if (num_seqs == 0 || total_q == 0) return PA_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start_loc)
     return pa::fail(PA_ERR_INVALID, "%s: NULL device pointer", fn);
@@ -609,7 +612,7 @@ extern "C" pa_status pa_decode_multi(void* out, const void* q, const void* k_cac
   // its whole context fits one partition (all its query tokens form one run);
   // the query-major kernel decides per block of kMqRows / G query tokens.
   const bool token_major = pa::decode_mq_tc_supported(a);
-  a.direct_qblock = token_major ? max_query_len : pa::kMqRows / G;
+  a.direct_qblock = token_major ? max_query_len : pa::kMqTiles * (pa::kMqRows / G);
   const int err = token_major ? pa::launch_decode_mq_tc(a, status, stream)
                               : pa::launch_decode_mq(a, status, stream);
   pa_status st = launch_status(fn, err, 1);

@@ -10,28 +10,30 @@
 // positions 0 .. L_b - Q_b + i with one softmax over them.
 //
 // With many query rows the work is query-major, as in a prefill kernel: a CTA
-// serves one (sequence, kv head, block of 128/G query tokens, partition of
-// keys); its 128 rows are (query token, query head) pairs of that kv head, and
-// per tile of 128 keys
+// serves one (sequence, kv head, pair of blocks of 128/G query tokens,
+// partition of keys); each block's 128 rows are (query token, query head)
+// pairs of that kv head, and per tile of 128 keys, for each of the two blocks
 //
 //   S [128 rows x 128 keys] = Q [128 x 128] . K^T          (K K-major)
-//   O [128 rows x 128 dims] += P [128 x 128 keys] . V      (V MN-major)
+//   O [128 rows x 128 dims] += P [128 x 128 keys] . V      (P from TMEM, V MN-major)
 //
 // run on tcgen05 (kind::f16, fp32 accumulation in TMEM).  K and V tiles are
 // the TMA boxes of decode_tc.cu (one 4-D box per physical block, 128-byte
-// swizzle).  A row's running max, sum and causal limit belong to its two
-// softmax threads, and a warp rescales its half of its 32 rows of O in TMEM
-// when one of their maxima grows by more than 2^8.
+// swizzle).  The MMA issuer alternates between the two blocks, so the tensor
+// core runs one block's products while the softmax threads work on the
+// other's.  A row's running max, sum and causal limit belong to its two
+// softmax threads (one per 64-column half of each tile and of O); a warp
+// rescales its half of its 32 rows of O in TMEM when one of their maxima grows
+// by more than 2^8.  P goes back into the TMEM columns of the S it came from
+// and feeds the second product from there.
 //
-// Roles (10 warps): warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
-// warps 2-9 Q staging, softmax and epilogue, two threads per row: the warps
-// w and w + 4 share a TMEM lane quadrant, one takes key columns 0-63 of each
-// tile (and dims 0-63 of O), the other 64-127, and the pair agrees on each
-// row's maximum through shared memory and a named barrier.  A ring of three
-// K/V tiles, about 196 KB of shared memory and all 512 TMEM columns: one CTA
-// per SM.  Every wait is bounded; block ids
-// outside the pool are skipped and flagged; inconsistent query offsets are
-// flagged (PA_DEVERR_CONTEXT) and their sequence skipped.
+// Roles (18 warps): warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
+// warps 2-9 the first block's Q staging, softmax and epilogue, warps 10-17 the
+// second block's.  A ring of three K/V tiles and the two Q blocks, about 167
+// KB of shared memory, and all 512 TMEM columns: one CTA per SM.  Every wait
+// is bounded; block ids outside the pool are skipped and flagged;
+// inconsistent query offsets are flagged (PA_DEVERR_CONTEXT) and their
+// sequence skipped.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -50,7 +52,7 @@ using namespace tc;
 
 constexpr unsigned FULL = 0xffffffffu;
 constexpr int TOK = 128;                   // keys per tile
-constexpr int MR = 128;                    // query rows per CTA
+constexpr int MR = 128;                    // query rows per query block
 constexpr int DH = 128;
 constexpr int SLOTS = 3;
 constexpr int SLOT_BYTES = TOK * 256;      // K or V tile (as in decode_tc.cu): 32 KB
@@ -58,23 +60,24 @@ constexpr int GROUP_BYTES = 2048;
 constexpr int HALF_OFF = 1024;
 constexpr int OPA_BYTES = MR * 256;        // a 128 x 128 16-bit row-major operand: 32 KB
 constexpr int OPA_HALF = MR * 128;         // its second 64-column half
-constexpr int OFF_RING = 0;
-constexpr int OFF_Q = OFF_RING + SLOTS * SLOT_BYTES;
-constexpr int OFF_P = OFF_Q + OPA_BYTES;   // two P buffers
-constexpr int OFF_BAR = OFF_P + 2 * OPA_BYTES;
-constexpr int NBARS = 2 * SLOTS + 9;
-constexpr int OFF_TMEM = OFF_BAR + NBARS * 8;
-constexpr int OFF_RMAX = (OFF_TMEM + 16 + 15) / 16 * 16;   // [2 tiles][2 halves][MR] row maxima
-constexpr int OFF_RSUM = OFF_RMAX + 2 * 2 * MR * 4;          // [2 halves][MR] row sums
-constexpr int SMEM_USED = OFF_RSUM + 2 * MR * 4;
-constexpr int SMEM_BYTES = SMEM_USED + 1024;
-constexpr int THREADS = 320;                 // producer, MMA, 8 softmax warps
-constexpr int NSOFT = 256;                   // softmax threads: two per row
-constexpr int TMEM_COLS = 512;             // S0 [0,128), S1 [128,256), O [256,384)
-constexpr int O_COL = 256;
+constexpr int TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;
 
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+// ---- the query-major kernel with two query tiles per CTA (decode_mq_kernel) ----
+// TMEM: S of tile X at X * 128, O of tile X at 256 + X * 128; P of tile X
+// (bf16/f16 pairs) overwrites the S columns it was computed from.
+constexpr int NT = kMqTiles;                  // query tiles per CTA
+constexpr int THREADS2 = 64 + NT * 256;       // producer, MMA, 8 softmax warps per tile
+constexpr int OFF2_Q = SLOTS * SLOT_BYTES;
+constexpr int OFF2_BAR = OFF2_Q + NT * OPA_BYTES;
+constexpr int NBARS2 = 2 * SLOTS + 3 * NT + 1;  // ring full/empty, s_full, p_full, p_free, q_ready
+constexpr int OFF2_TMEM = OFF2_BAR + NBARS2 * 8;
+constexpr int OFF2_RMAX = (OFF2_TMEM + 16 + 15) / 16 * 16;  // [2 tiles parity][NT][2 halves][MR]
+constexpr int OFF2_RSUM = OFF2_RMAX + 2 * NT * 2 * MR * 4;   // [NT][2 halves][MR]
+constexpr int SMEM2_USED = OFF2_RSUM + NT * 2 * MR * 4;
+constexpr int SMEM2_BYTES = SMEM2_USED + 1024;
+static_assert(SMEM2_BYTES <= 227 * 1024, "shared memory");
+static_assert(NT == 2, "two query tiles: TMEM holds 2 x (S, O) of 128 columns");
 
 // kind::f16 instruction descriptor, fp32 accumulation, M = 128, N = 128;
 // A K-major; B K-major (S) or MN-major (O).
@@ -121,17 +124,28 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
       : "memory");
 }
 
-// One TMEM load of 128 consecutive 32-bit columns of this thread's lane, one wait.
-__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v) {
-  uint32_t r[128];
+// MMA with the A operand in TMEM (M = 128 lanes, K along the columns: two
+// 16-bit elements per 32-bit column) and B from shared memory.
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                           uint32_t idesc, uint32_t accumulate) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%128];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
-      : "r"(taddr)
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
       : "memory");
-#pragma unroll
-  for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 16 32-bit words into 16 consecutive TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* w) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),
+      "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // 2^x by the SFU's approximation (relative error about 2^-22; 2^-inf = +0).
@@ -175,32 +189,42 @@ struct MqParams {
   float scale_log2;
 };
 
+// Query-major multi-query kernel with two query tiles per CTA: a CTA serves
+// (sequence, kv head, pair of query blocks of 128 / G tokens, key partition).
+// Per 128-key tile the MMA issuer alternates between the tiles (S_A, S_B, then
+// O_A += P_A V and O_B += P_B V as each tile's softmax finishes), so the tensor
+// core works on one tile while the softmax threads work on the other.  Each
+// row has two softmax threads (warps of the same TMEM lane quadrant, one per
+// 64-column half, as in decode_mq_kernel); tile X has its own 8 warps.  P is
+// written back into the TMEM columns of the S it came from (half h's 64 keys as
+// 32 columns of 16-bit pairs at h * 64) and is the A operand of the second MMA
+// straight from TMEM, so no shared memory holds P.  Warps 0 and 1: producer
+// and MMA issuer; warps 2 + 8X .. 9 + 8X: tile X.  Shared memory: the K/V ring
+// and the two Q tiles (~167 KB); all 512 TMEM columns.
 template <typename T, int G>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS2, 1)
     decode_mq_kernel(const MqParams p, const __grid_constant__ CUtensorMap tmap_k,
-                     const __grid_constant__ CUtensorMap tmap_v) {
-  constexpr int QB = MR / G;                        // query tokens per CTA
+                      const __grid_constant__ CUtensorMap tmap_v) {
+  constexpr int QB = MR / G;                        // query tokens per tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* ring = smem + OFF_RING;
-  uint8_t* qop = smem + OFF_Q;
-  uint8_t* pop = smem + OFF_P;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint8_t* ring = smem;
+  uint8_t* qop = smem + OFF2_Q;                     // NT tiles of OPA_BYTES
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF2_BAR);
   uint64_t* ring_full = bars;
   uint64_t* ring_empty = bars + SLOTS;
-  uint64_t* s_full = bars + 2 * SLOTS;      // [2]
-  uint64_t* s_free = s_full + 2;            // [2]
-  uint64_t* p_full = s_free + 2;            // [2]
-  uint64_t* p_free = p_full + 2;            // [2]
-  uint64_t* q_ready = p_free + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
+  uint64_t* s_full = bars + 2 * SLOTS;              // [NT]
+  uint64_t* p_full = s_full + NT;                   // [NT]
+  uint64_t* p_free = p_full + NT;                   // [NT]
+  uint64_t* q_ready = p_free + NT;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF2_TMEM);
+  float* rmax = reinterpret_cast<float*>(smem + OFF2_RMAX);
+  float* rsum = reinterpret_cast<float*>(smem + OFF2_RSUM);
 
-  // the query blocks of one (sequence, kv head, key partition) are adjacent in
-  // the grid, so they run together and read that partition's K/V from L2
-  const int n_qb = gridDim.z / p.num_partitions;
+  const int n_pairs = gridDim.z / p.num_partitions;
   const int b = blockIdx.x, g = blockIdx.y;
-  const int qb = blockIdx.z % n_qb, part = blockIdx.z / n_qb;
+  const int pair = blockIdx.z % n_pairs, part = blockIdx.z / n_pairs;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   grid_dependency_wait();
@@ -214,14 +238,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int64_t grid_cap = static_cast<int64_t>(p.num_partitions) * P;
   cap = cap < grid_cap ? cap : grid_cap;
   if (L < 0 || L > cap || Qb < 0 || Qb > L || q0 < 0 || q0 + Qb > p.total_q) {
-    if (threadIdx.x == 0 && qb == 0 && part == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
+    if (threadIdx.x == 0 && pair == 0 && part == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
     return;
   }
-  if (qb == 0 && part == 0 && g == 0 && threadIdx.x == 0 &&
-      Qb > static_cast<int>(gridDim.z / p.num_partitions) * QB)
+  if (pair == 0 && part == 0 && g == 0 && threadIdx.x == 0 && Qb > n_pairs * NT * QB)
     atomicOr(p.status, PA_DEVERR_CONTEXT);          // max_query_len below this Q_b
-  if (qb * QB >= Qb) return;                        // no query tokens in this block
-  const int i_last = min(Qb, (qb + 1) * QB) - 1;    // last query token of the block
+  const int qb0 = pair * NT;                        // the CTA's first query block
+  if (qb0 * QB >= Qb) return;                       // no query tokens here
+  const int i_last = min(Qb, (qb0 + NT) * QB) - 1;  // the CTA's last query token
   const int pmax = L - Qb + i_last;                 // its position: the last key needed
   const int kstart = part * P;
   if (kstart > pmax) return;
@@ -239,13 +263,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&ring_full[s], 1);
       mbar_init(&ring_empty[s], 1);
     }
-    for (int j = 0; j < 2; ++j) {
-      mbar_init(&s_full[j], 1);
-      mbar_init(&s_free[j], 8);
-      mbar_init(&p_full[j], 8);
-      mbar_init(&p_free[j], 1);
+    for (int x = 0; x < NT; ++x) {
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[x], 8);
+      mbar_init(&p_free[x], 1);
     }
-    mbar_init(q_ready, 8);
+    mbar_init(q_ready, 8 * NT);
     fence_mbar_init();
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
@@ -263,11 +286,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ================= producer (as in decode_tc.cu) =================
+    // ================= producer (as in decode_mq_kernel) =================
     const int row_stride = p.Hkv * bs;
     bool ok = true;
     int issued = 0;
-    auto table = [&](int i) {                       // lane j: block j of tile i, read a tile ahead
+    auto table = [&](int i) {
       const int b0 = first_blk + i * bpt;
       return (i < n_tiles && lane < min(bpt, last_blk - b0)) ? __ldg(trow + b0 + lane) : -1;
     };
@@ -305,23 +328,22 @@ __global__ void __launch_bounds__(THREADS, 1)
     return;
   }
 
-  // rows of this CTA: r = il * G + hl  (query token il of the block, head hl).
-  // Each row has two softmax threads in two warps of the same TMEM lane
-  // quadrant: `half` 0 takes key columns 0-63 of a tile (and dims 0-63 of O),
-  // half 1 columns 64-127 (dims 64-127).
+  // softmax thread: tile X, row r (TMEM lane), key / dim half `half`
+  const int lw = warp - 2;                          // 0 .. 8 NT - 1 for softmax warps
+  const int X = lw >> 3;
+  const int half = (lw >> 2) & 1;
   const int quad = warp & 3;
-  const int half = warp >= 6 ? 1 : 0;
   const int r = quad * 32 + lane;
   const int il = r / G, hl = r % G;
-  const bool row_valid = warp >= 2 && qb * QB + il < Qb;
-  const int64_t t = static_cast<int64_t>(q0) + qb * QB + il;          // query token index
-  const int pos = L - Qb + qb * QB + il;                               // its position
-  float* rmax = reinterpret_cast<float*>(smem + OFF_RMAX);            // [2][2][MR]
-  float* rsum = reinterpret_cast<float*>(smem + OFF_RSUM);            // [2][MR]
+  const int qtok = (qb0 + X) * QB + il;             // query token of the row within the sequence
+  const bool row_valid = warp >= 2 && qtok < Qb;
+  const int64_t t = static_cast<int64_t>(q0) + qtok;
+  const int pos = L - Qb + qtok;
+  const int pair_bar = 3 + X * 4 + quad;            // named barrier of this row's two threads
 
   if (warp >= 2) {
-    // Q operand: row r = q[t][g*G + hl][:] (this thread its half of the 16
-    // chunks), zero for rows past the block's tokens
+    // Q operand of tile X: row r = q[t][g*G + hl][:] (this thread its 8 of
+    // the 16 chunks), zero for rows past the sequence's query tokens
     const T* src = static_cast<const T*>(p.q) + (t * p.Hq + g * G + hl) * DH;
     uint4 v[DH / 16];
 #pragma unroll
@@ -329,7 +351,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       v[c] = row_valid ? __ldg(reinterpret_cast<const uint4*>(src + (half * 8 + c) * 8))
                        : make_uint4(0, 0, 0, 0);
 #pragma unroll
-    for (int c = 0; c < DH / 16; ++c) *reinterpret_cast<uint4*>(qop + opa_chunk(r, half * 8 + c)) = v[c];
+    for (int c = 0; c < DH / 16; ++c)
+      *reinterpret_cast<uint4*>(qop + X * OPA_BYTES + opa_chunk(r, half * 8 + c)) = v[c];
     fence_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(q_ready);
@@ -340,59 +363,73 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       const uint32_t id_s = idesc_mq<T>(false);
       const uint32_t id_o = idesc_mq<T>(true);
-      const uint32_t ring_a = smem_addr(ring), q_a = smem_addr(qop), p_a = smem_addr(pop);
+      const uint32_t ring_a = smem_addr(ring), q_a = smem_addr(qop);
       bool ok = true;
-      auto issue_s = [&](int i) -> bool {
-        const int u = 2 * i, s = u % SLOTS;
-        if (!mbar_wait(&ring_full[s], (u / SLOTS) & 1, p.status)) return false;
-        if (i >= 2 && !mbar_wait(&s_free[i & 1], ((i >> 1) - 1) & 1, p.status)) return false;
-        tc_fence_after();
-        const uint32_t d = tmem + (i & 1) * 128;
+      auto issue_s = [&](int x, int i) {           // S_x = Q_x . K_i^T
+        const int s = (2 * i) % SLOTS;
+        const uint32_t d = tmem + x * 128;
 #pragma unroll
         for (int k = 0; k < DH / 16; ++k) {
-          const uint64_t a = smem_desc(q_a + (k >> 2) * OPA_HALF + (k & 3) * 32, 16, 1024);
+          const uint64_t a =
+              smem_desc(q_a + x * OPA_BYTES + (k >> 2) * OPA_HALF + (k & 3) * 32, 16, 1024);
           const uint64_t bk =
               smem_desc(ring_a + s * SLOT_BYTES + (k >> 2) * HALF_OFF + (k & 3) * 32, 16, GROUP_BYTES);
           mma_f16(d, a, bk, id_s, k > 0);
         }
-        mma_commit(&s_full[i & 1]);
-        mma_commit(&ring_empty[s]);
-        return true;
+        mma_commit(&s_full[x]);
       };
-      auto issue_o = [&](int i) -> bool {
-        const int u = 2 * i + 1, s = u % SLOTS;
-        if (!mbar_wait(&ring_full[s], (u / SLOTS) & 1, p.status)) return false;
-        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, p.status)) return false;
-        tc_fence_after();
-        const uint32_t d = tmem + O_COL;
+      auto issue_pv = [&](int x, int i) {          // O_x += P_x . V_i, P_x in TMEM
+        const int s = (2 * i + 1) % SLOTS;
+        const uint32_t d = tmem + 256 + x * 128;
 #pragma unroll
         for (int k = 0; k < TOK / 16; ++k) {
-          const uint64_t a =
-              smem_desc(p_a + (i & 1) * OPA_BYTES + (k >> 2) * OPA_HALF + (k & 3) * 32, 16, 1024);
+          // keys 16k .. 16k + 15: half k / 4's P columns
+          const uint32_t a = tmem + x * 128 + (k >> 2) * 64 + (k & 3) * 8;
           const uint64_t bv =
               smem_desc(ring_a + s * SLOT_BYTES + k * 2 * GROUP_BYTES, HALF_OFF, GROUP_BYTES);
-          mma_f16(d, a, bv, id_o, (i > 0 || k > 0) ? 1u : 0u);
+          mma_f16_ts(d, a, bv, id_o, (i > 0 || k > 0) ? 1u : 0u);
         }
-        mma_commit(&ring_empty[s]);
-        mma_commit(&p_free[i & 1]);
-        return true;
+        mma_commit(&p_free[x]);
       };
-      ok = mbar_wait(q_ready, 0, p.status) && issue_s(0);
+      auto ring_wait = [&](int u) { return mbar_wait(&ring_full[u % SLOTS], (u / SLOTS) & 1, p.status); };
+      ok = mbar_wait(q_ready, 0, p.status) && ring_wait(0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        mma_commit(&ring_empty[0]);
+      }
       for (int i = 0; i < n_tiles && ok; ++i) {
-        if (i + 1 < n_tiles) ok = issue_s(i + 1);
-        if (ok) ok = issue_o(i);
+        ok = ring_wait(2 * i + 1) && mbar_wait(&p_full[0], i & 1, p.status);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(0, i);
+        const bool more = i + 1 < n_tiles;
+        if (more) {
+          ok = ring_wait(2 * i + 2);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(0, i + 1);                       // after O_0 += P_0 V_i read P_0's columns
+        }
+        ok = mbar_wait(&p_full[1], i & 1, p.status);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(1, i);
+        mma_commit(&ring_empty[(2 * i + 1) % SLOTS]);
+        if (more) {
+          issue_s(1, i + 1);
+          mma_commit(&ring_empty[(2 * i + 2) % SLOTS]);
+        }
       }
     }
     __syncwarp();
   } else if (warp >= 2) {
-    // ================= softmax: two threads per row =================
-    // A warp whose 32 rows hold no query token (few queries per sequence) only
-    // keeps pace with the barriers and zeroes V rows; its P rows stay zero.
-    // The two threads of a row meet at a named barrier of their warp pair
-    // (id 3 + quad) to agree on the row's maximum each tile.
+    // ================= softmax of tile X, two threads per row =================
     const bool warp_active = __any_sync(FULL, row_valid);
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const int col0 = half * 64;                        // this thread's key / dim columns
+    const uint32_t s_col = tmem + lane_base + X * 128 + half * 64;      // my 64 S columns
+    const uint32_t o_col = tmem + lane_base + 256 + X * 128 + half * 64; // my 64 dims of O
+    const int col0 = half * 64;
     float m_run = -INFINITY, l_half = 0.f;
     bool ok = true;
     auto wait = [&](uint64_t* bar, uint32_t parity) {
@@ -400,135 +437,124 @@ __global__ void __launch_bounds__(THREADS, 1)
       ok = __all_sync(FULL, ok);
       return ok;
     };
-    if (!warp_active) {
-#pragma unroll
-      for (int buf = 0; buf < 2; ++buf)
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(pop + buf * OPA_BYTES + opa_chunk(r, half * 8 + c)) =
-              make_uint4(0, 0, 0, 0);
-    }
     for (int i = 0; i < n_tiles; ++i) {
       const int tile0 = kstart + i * TOK;
       const int n_valid = min(TOK, kend - tile0);
-      wait(&s_full[i & 1], (i >> 1) & 1);
+      wait(&s_full[X], i & 1);
+      tc_fence_after();
       if (warp_active) {
         const int lim = row_valid ? min(pos - tile0, n_valid - 1) : -1;  // last key column
-        float sv[64];
-        if (ok) {
-          tc_fence_after();
-          tmem_ld32(tmem + lane_base + (i & 1) * 128 + col0, sv);
-          tmem_ld32(tmem + lane_base + (i & 1) * 128 + col0 + 32, sv + 32);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 64; ++j) sv[j] = 0.f;
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_free[i & 1]);
-        // Every column of this thread's half visible to every row of the warp
-        // (all but the diagonal and last tiles): no mask, and the scale (> 0)
-        // moves into the exponent's FMA below, so the scores stay raw here.
         const bool open = __all_sync(FULL, col0 + 63 <= lim);
-        float pm[8];                                   // 8 independent partial maxima
+        // pass 1: the row's maximum over this half (raw scores when open)
+        float pm[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) pm[k] = -INFINITY;
-        if (open) {
 #pragma unroll
-          for (int j = 0; j < 64; ++j) pm[j & 7] = fmaxf(pm[j & 7], sv[j]);
-        } else {
+        for (int c = 0; c < 2; ++c) {
+          float sv[32];
+          if (ok) tmem_ld32(s_col + c * 32, sv);
+          else
 #pragma unroll
-          for (int j = 0; j < 64; ++j) {
-            sv[j] = col0 + j <= lim ? sv[j] * p.scale_log2 : -INFINITY;
-            pm[j & 7] = fmaxf(pm[j & 7], sv[j]);
+            for (int j = 0; j < 32; ++j) sv[j] = 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float x = open ? sv[j] : (col0 + c * 32 + j <= lim ? sv[j] : -INFINITY);
+            pm[j & 7] = fmaxf(pm[j & 7], x);
           }
         }
         float tmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                            fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-        if (open) tmax *= p.scale_log2;
-        // the row's maximum over both halves (the buffer alternates by tile, so
-        // a partner a tile ahead never overwrites what this thread still reads)
-        rmax[((i & 1) * 2 + half) * MR + r] = tmax;
-        named_sync(3 + quad, 64);
-        tmax = fmaxf(tmax, rmax[((i & 1) * 2 + (half ^ 1)) * MR + r]);
+        tmax = tmax == -INFINITY ? tmax : tmax * p.scale_log2;
+        rmax[(((i & 1) * NT + X) * 2 + half) * MR + r] = tmax;
+        named_sync(pair_bar, 64);
+        tmax = fmaxf(tmax, rmax[(((i & 1) * NT + X) * 2 + (half ^ 1)) * MR + r]);
         const bool need = tmax > m_run + RESCALE_THRESHOLD;
-        if (__any_sync(FULL, need)) {                  // the same for both warps of the pair
+        if (__any_sync(FULL, need)) {              // the same for both warps of the pair
           const float mnew = fmaxf(m_run, tmax);
           const float alpha = (m_run == -INFINITY) ? 0.f : exp2f(m_run - mnew);
           m_run = mnew;
           l_half *= alpha;
-          // O must hold every earlier tile before it is rescaled (its dims col0..col0+63)
-          if (i > 0 && wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
+          // O must hold every earlier tile before it is rescaled
+          if (i > 0 && wait(&p_free[X], (i - 1) & 1)) {
             tc_fence_after();
 #pragma unroll 1
             for (int c = 0; c < 2; ++c) {
               float o[32];
-              tmem_ld32(tmem + lane_base + O_COL + col0 + c * 32, o);
+              tmem_ld32(o_col + c * 32, o);
 #pragma unroll
               for (int j = 0; j < 32; ++j) o[j] *= alpha;
-              tmem_st32(tmem + lane_base + O_COL + col0 + c * 32, o);
+              tmem_st32(o_col + c * 32, o);
             }
           }
         }
-        if (i >= 2) wait(&p_free[i & 1], ((i >> 1) - 1) & 1);
-        uint8_t* pb = pop + (i & 1) * OPA_BYTES;
-        float ps[8];                                   // 8 independent partial sums
+        // pass 2: P = 2^(scale * s - m) into the first 32 of my S columns
+        const float neg_m = -m_run;
+        float ps[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) ps[k] = 0.f;
-        // P = 2^(scale * s - m): one FMA and one ex2 per column when open
-        const float neg_m = -m_run;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t w[4];
+        for (int c = 0; c < 2; ++c) {
+          float sv[32];
+          if (ok) tmem_ld32(s_col + c * 32, sv);
+          else
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float s0 = sv[8 * c + 2 * e], s1 = sv[8 * c + 2 * e + 1];
+            for (int j = 0; j < 32; ++j) sv[j] = 0.f;
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int j0 = 2 * e, j1 = 2 * e + 1;
             float p0, p1;
             if (open) {
-              p0 = ex2_approx(fmaf(s0, p.scale_log2, neg_m));
-              p1 = ex2_approx(fmaf(s1, p.scale_log2, neg_m));
+              p0 = ex2_approx(fmaf(sv[j0], p.scale_log2, neg_m));
+              p1 = ex2_approx(fmaf(sv[j1], p.scale_log2, neg_m));
             } else {
-              p0 = s0 == -INFINITY ? 0.f : ex2_approx(s0 + neg_m);
-              p1 = s1 == -INFINITY ? 0.f : ex2_approx(s1 + neg_m);
+              const bool v0 = col0 + c * 32 + j0 <= lim && m_run != -INFINITY;
+              const bool v1 = col0 + c * 32 + j1 <= lim && m_run != -INFINITY;
+              p0 = v0 ? ex2_approx(fmaf(sv[j0], p.scale_log2, neg_m)) : 0.f;
+              p1 = v1 ? ex2_approx(fmaf(sv[j1], p.scale_log2, neg_m)) : 0.f;
             }
-            ps[2 * e] += p0;
-            ps[2 * e + 1] += p1;
+            ps[(2 * e) & 7] += p0;
+            ps[(2 * e + 1) & 7] += p1;
             w[e] = pack2<T>(p0, p1);
           }
-          *reinterpret_cast<uint4*>(pb + opa_chunk(r, half * 8 + c)) = make_uint4(w[0], w[1], w[2], w[3]);
+          tmem_st16u(s_col + c * 16, w);
         }
         l_half += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       } else {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_free[i & 1]);
+        // no query row in this warp: its P rows are 0
+        uint32_t z[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) z[e] = 0u;
+        tmem_st16u(s_col, z);
+        tmem_st16u(s_col + 16, z);
       }
-      if (n_valid < TOK) {
+      if (X == 0 && n_valid < TOK) {
         // the last tile: zero the V rows of keys past the range (this thread
-        // its 64-dim half of row r), so that whatever they hold adds 0 * 0 to O
+        // its 64-dim half of row r), so that whatever they hold adds 0 to O
         const int u = 2 * i + 1, s_ = u % SLOTS;
         if (wait(&ring_full[s_], (u / SLOTS) & 1) && r >= n_valid) {
           uint8_t* row = ring + s_ * SLOT_BYTES + (r >> 3) * GROUP_BYTES + (r & 7) * 128 + half * HALF_OFF;
 #pragma unroll
           for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(row + c * 16) = make_uint4(0, 0, 0, 0);
         }
+        fence_async_smem();
       }
-      fence_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[i & 1]);
+      if (lane == 0) mbar_arrive(&p_full[X]);
     }
-    // ---- epilogue: row r of O, dims col0..col0+63; the row's sum over both halves ----
-    rsum[half * MR + r] = l_half;
-    named_sync(3 + quad, 64);
-    const float l_sum = l_half + rsum[(half ^ 1) * MR + r];
-    wait(&p_free[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1);
+    // ---- epilogue: row r of O_X, dims col0..col0+63; the row's sum over both halves ----
+    rsum[(X * 2 + half) * MR + r] = l_half;
+    named_sync(pair_bar, 64);
+    const float l_sum = l_half + rsum[(X * 2 + (half ^ 1)) * MR + r];
+    wait(&p_free[X], (n_tiles - 1) & 1);
     tc_fence_after();
     const int64_t hq = t * p.Hq + g * G + hl;
 #pragma unroll 1
     for (int c = 0; c < (warp_active ? 2 : 0); ++c) {
       float o[32];
-      tmem_ld32(tmem + lane_base + O_COL + col0 + c * 32, o);
+      tmem_ld32(o_col + c * 32, o);
       if (ok && row_valid) {
         if (single) {
           const float inv = 1.f / l_sum;
@@ -537,9 +563,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int j = 0; j < 32; j += 8) {
             uint32_t w[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              w[e] = static_cast<uint32_t>(to_bits<T>(o[j + 2 * e] * inv)) |
-                     (static_cast<uint32_t>(to_bits<T>(o[j + 2 * e + 1] * inv)) << 16);
+            for (int e = 0; e < 4; ++e) w[e] = pack2<T>(o[j + 2 * e] * inv, o[j + 2 * e + 1] * inv);
             *reinterpret_cast<uint4*>(dst + j) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         } else {
@@ -557,9 +581,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   }
 
-  // ---- teardown: warps 1-9 meet, warp 1 frees TMEM ----
+  // ---- teardown: warps 1 .. 1 + 8 NT meet, warp 1 frees TMEM ----
   tc_fence_before();
-  named_sync(2, THREADS - 32);
+  named_sync(2, THREADS2 - 32);
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
@@ -634,7 +658,7 @@ __global__ void __launch_bounds__(128) decode_mq_reduce_kernel(const MqReducePar
 template <typename T, int G>
 cudaError_t launch_mq_t(const MqArgs& a, unsigned int* status, cudaStream_t stream) {
   auto kern = decode_mq_kernel<T, G>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
   if (e != cudaSuccess) return e;
   CUtensorMap mk, mv;
   const int64_t groups = static_cast<int64_t>(a.num_blocks) * a.Hkv * a.block_size / 8;
@@ -666,8 +690,9 @@ cudaError_t launch_mq_t(const MqArgs& a, unsigned int* status, cudaStream_t stre
   p.num_partitions = a.num_partitions;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const int qblocks = (a.max_query_len + MR / G - 1) / (MR / G);
-  dim3 grid(a.num_seqs, a.Hkv, qblocks * a.num_partitions);
-  return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
+  const int pairs = (qblocks + NT - 1) / NT;
+  dim3 grid(a.num_seqs, a.Hkv, pairs * a.num_partitions);
+  return launch_overlapped(kern, grid, dim3(THREADS2), SMEM2_BYTES, stream, p, mk, mv);
 }
 
 template <typename T>
@@ -683,7 +708,7 @@ cudaError_t launch_mq_reduce_t(const MqArgs& a, cudaStream_t stream) {
   p.num_seqs = a.num_seqs;
   p.total_q = a.total_q;
   p.Hq = a.Hq;
-  p.direct_qblock = a.direct_qblock > 0 ? a.direct_qblock : MR / (a.Hq / a.Hkv);
+  p.direct_qblock = a.direct_qblock > 0 ? a.direct_qblock : NT * (MR / (a.Hq / a.Hkv));
   p.partition_size = a.partition_size;
   p.num_partitions = a.num_partitions;
   const int64_t warps = static_cast<int64_t>(a.total_q) * a.Hq;

@@ -122,7 +122,8 @@ struct MqArgs {
   // key lies in the first partition.
   int direct_qblock = 0;
 };
-constexpr int kMqRows = 128;  // (query token, head) rows per CTA of the multi-query kernel
+constexpr int kMqRows = 128;  // (query token, head) rows per query tile of the multi-query kernel
+constexpr int kMqTiles = 2;   // query tiles per CTA of the multi-query kernel
 int launch_decode_mq(const MqArgs& a, unsigned int* status, void* stream);
 // Few query tokens per sequence (max_query_len * G <= 64, G = 4 or 8): the
 // token-major tcgen05 decode kernel with per-column causal limits, 16 / G query

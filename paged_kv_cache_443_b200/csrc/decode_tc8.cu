@@ -13,13 +13,13 @@
 //   S^T [128 tokens x 16] = K [128 x 128] . Q^T [128 x 16]         K-major K
 //   O^T [128 dims   x 16] += V^T [128 x 128] . P^T [128 x 16]      MN-major V^T, P^T
 //
-// * Q: split into three E4M3 terms, Q * 2^e = Q1 + Q2 + Q3 (each the nearest
-//   E4M3 value of what the previous terms left; e a per-head power of two
-//   putting the head's largest |q| in [2^7, 2^8)), and S accumulates the three
-//   products.  An f16 or bf16 query has at most 11 significant bits, and each
-//   term takes the next 4, so the split is exact for every component at least
-//   2^-6 of the head's largest; 2^-e and k_scale are folded into the softmax
-//   scale.
+// * Q: split into E4M3 terms, Q * 2^e = Q1 + Q2 (+ Q3) (each the nearest E4M3
+//   value of what the previous terms left; e a per-head power of two putting
+//   the head's largest |q| in [2^7, 2^8)), and S accumulates their products.
+//   Each term takes the next 4 significant bits: three terms for an f16 query
+//   (11 bits), two for a bf16 one (8 bits), so the split is exact for every
+//   component at least 2^-6 of the head's largest; 2^-e and k_scale are
+//   folded into the softmax scale.
 // * P: the running max is raised as soon as a score passes it by 2 (base 2),
 //   so P <= 4; P * 2^6 (<= 256, inside E4M3's range) is split into two E4M3
 //   terms the same way, P1 + P2, which keeps P to about 2^-8 of its value for
@@ -37,7 +37,9 @@
 //   warps 2-5  query terms, then softmax (as in decode_tc.cu), P as two E4M3
 //              terms; they zero the V rows of tokens past the end of a final
 //              tile.
-// About 113 KB of shared memory: two CTAs per SM.  Every wait is bounded;
+// About 113 KB of shared memory (two CTAs per SM) for f16 queries; for bf16
+// queries two query terms, rings of two tiles and one P buffer, about 73 KB,
+// so three CTAs share an SM.  Every wait is bounded;
 // block ids outside the pool are skipped and flagged.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -59,34 +61,48 @@ constexpr unsigned FULL = 0xffffffffu;
 constexpr int TOK = 128;                    // tokens per tile
 constexpr int NPAD = 16;                    // MMA N (heads padded)
 constexpr int DH = 128;                     // head size
-constexpr int NTERM = 3;                    // E4M3 terms of the query
 constexpr int PTERM = 2;                    // E4M3 terms of P
-constexpr int SLOTS = 3;                    // tiles per ring (one ring for K, one for V)
 constexpr int TILE_BYTES = TOK * DH;        // one tile of codes: 16 KB
 constexpr int QT_BYTES = NPAD * DH;         // one query term: 16 rows x 128 codes
 constexpr int PT_BYTES = NPAD * TOK;        // one P term: 128 tokens x 16 heads (MN-major)
 constexpr int PB_BYTES = PTERM * PT_BYTES;  // one P buffer (both terms)
-constexpr int OFF_KR = 0;
-constexpr int OFF_VR = OFF_KR + SLOTS * TILE_BYTES;
-constexpr int OFF_Q = OFF_VR + SLOTS * TILE_BYTES;
-constexpr int OFF_P = OFF_Q + NTERM * QT_BYTES;   // two P buffers
-constexpr int OFF_BAR = OFF_P + 2 * PB_BYTES;
-constexpr int NBARS = 4 * SLOTS + 8 + 1;
-constexpr int OFF_TMEM = (OFF_BAR + NBARS * 8 + 15) / 16 * 16;
-constexpr int OFF_RED = OFF_TMEM + 16;      // 4 warps x 16 floats
-constexpr int OFF_QS = OFF_RED + 4 * NPAD * 4;
-constexpr int SMEM_USED = OFF_QS + NPAD * 4;
-constexpr int SMEM_BYTES = SMEM_USED + 1024;
 constexpr int THREADS = 192;
 constexpr int TMEM_COLS = 64;               // S0 [0,16), S1 [16,32), O [32,48)
 constexpr float RESCALE_THRESHOLD = 2.0f;   // P <= 2^2
 constexpr float P_UP = 64.0f;               // P * 2^6 <= 256 < 448
 constexpr float P_DOWN = 1.0f / 64.0f;
 
-static_assert(SMEM_BYTES * 2 + 2048 <= 228 * 1024, "two CTAs per SM");
-static_assert(OFF_VR % 1024 == 0 && OFF_Q % 1024 == 0 && OFF_P % 1024 == 0 &&
-                  QT_BYTES % 1024 == 0 && PT_BYTES % 1024 == 0,
-              "swizzled operands on 1 KB boundaries");
+// Shared-memory layout for NTERM query terms, SLOTS tiles per ring (one ring
+// for K codes, one for V codes) and PBUF P buffers.  Two layouts are built:
+//   3 terms, 3 + 3 slots, 2 P buffers (~113 KB): two CTAs per SM, for f16
+//     queries (11 significant bits: three 4-bit terms);
+//   2 terms, 2 + 2 slots, 1 P buffer (~73 KB): three CTAs per SM, for bf16
+//     queries (8 significant bits: two 4-bit terms are exact).  A third CTA's
+//     pipeline hides more of each tile's serial chain than a third slot does.
+template <int NTERM_, int SLOTS_, int PBUF_>
+struct Lay8 {
+  static constexpr int NTERM = NTERM_, SLOTS = SLOTS_, PBUF = PBUF_;
+  static constexpr int OFF_KR = 0;
+  static constexpr int OFF_VR = OFF_KR + SLOTS * TILE_BYTES;
+  static constexpr int OFF_Q = OFF_VR + SLOTS * TILE_BYTES;
+  static constexpr int OFF_P = OFF_Q + NTERM * QT_BYTES;
+  static constexpr int OFF_BAR = OFF_P + PBUF * PB_BYTES;
+  static constexpr int NBARS = 4 * SLOTS + 4 + 2 * PBUF + 1;
+  static constexpr int OFF_TMEM = (OFF_BAR + NBARS * 8 + 15) / 16 * 16;
+  static constexpr int OFF_RED = OFF_TMEM + 16;      // 4 warps x 16 floats
+  static constexpr int OFF_QS = OFF_RED + 4 * NPAD * 4;
+  static constexpr int SMEM_USED = OFF_QS + NPAD * 4;
+  static constexpr int SMEM_BYTES = SMEM_USED + 1024;
+  static constexpr int CTAS_PER_SM = (228 * 1024) / (SMEM_BYTES + 1024);
+  static_assert(OFF_VR % 1024 == 0 && OFF_Q % 1024 == 0 && OFF_P % 1024 == 0 &&
+                    QT_BYTES % 1024 == 0 && PT_BYTES % 1024 == 0,
+                "swizzled operands on 1 KB boundaries");
+};
+using LayF16 = Lay8<3, 3, 2>;
+using LayBF16 = Lay8<2, 2, 1>;
+static_assert(LayF16::CTAS_PER_SM >= 2, "two CTAs per SM");
+static_assert(LayBF16::CTAS_PER_SM >= 3, "three CTAs per SM");
+static_assert(3 * TMEM_COLS <= 512, "TMEM of three CTAs");
 
 // Instruction descriptor of kind::f8f6f4: E4M3 x E4M3 (format 0 for both),
 // fp32 accumulation, M = 128, N = 16; A K-major (S) or MN-major (O), B K-major.
@@ -153,10 +169,14 @@ __device__ __forceinline__ float2 from_e4m3x2(uint32_t c) {
   return __half22float2(*reinterpret_cast<const __half2*>(&lo));
 }
 
-template <typename T, int G>
-__global__ void __launch_bounds__(THREADS, 2)
+template <typename T, int G, typename Y>
+__global__ void __launch_bounds__(THREADS, Y::CTAS_PER_SM)
     decode_partition_tc8_kernel(const Tc8Params p, const __grid_constant__ CUtensorMap tmap_k,
                                 const __grid_constant__ CUtensorMap tmap_v) {
+  constexpr int NTERM = Y::NTERM, SLOTS = Y::SLOTS, PBUF = Y::PBUF;
+  constexpr int OFF_KR = Y::OFF_KR, OFF_VR = Y::OFF_VR, OFF_Q = Y::OFF_Q, OFF_P = Y::OFF_P;
+  constexpr int OFF_BAR = Y::OFF_BAR, OFF_TMEM = Y::OFF_TMEM, OFF_RED = Y::OFF_RED;
+  constexpr int OFF_QS = Y::OFF_QS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -171,9 +191,9 @@ __global__ void __launch_bounds__(THREADS, 2)
   uint64_t* vr_empty = vr_full + SLOTS;      // [SLOTS]
   uint64_t* s_full = vr_empty + SLOTS;       // [2]
   uint64_t* s_free = s_full + 2;             // [2]
-  uint64_t* p_full = s_free + 2;             // [2]
-  uint64_t* p_free = p_full + 2;             // [2]
-  uint64_t* q_ready = p_free + 2;
+  uint64_t* p_full = s_free + 2;             // [PBUF]
+  uint64_t* p_free = p_full + PBUF;          // [PBUF]
+  uint64_t* q_ready = p_free + PBUF;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
   float* red = reinterpret_cast<float*>(smem + OFF_RED);
   float* qs = reinterpret_cast<float*>(smem + OFF_QS);
@@ -224,6 +244,8 @@ __global__ void __launch_bounds__(THREADS, 2)
     for (int j = 0; j < 2; ++j) {
       mbar_init(&s_full[j], 1);
       mbar_init(&s_free[j], 4);
+    }
+    for (int j = 0; j < PBUF; ++j) {
       mbar_init(&p_full[j], 4);
       mbar_init(&p_free[j], 1);
     }
@@ -339,7 +361,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       }
       *reinterpret_cast<uint4*>(qop + term * QT_BYTES + row_off) = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    for (int i = t; i < 2 * PB_BYTES / 16; i += 128)
+    for (int i = t; i < PBUF * PB_BYTES / 16; i += 128)
       reinterpret_cast<uint4*>(pop)[i] = make_uint4(0, 0, 0, 0);
     fence_async_smem();
     __syncwarp();
@@ -375,7 +397,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       auto issue_pv = [&](int i) -> bool {
         const int s = i % SLOTS;
         if (!mbar_wait(&vr_full[s], (i / SLOTS) & 1, p.status)) return false;
-        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, p.status)) return false;
+        if (!mbar_wait(&p_full[i % PBUF], (i / PBUF) & 1, p.status)) return false;
         const bool first = i == 0;             // O starts at 0
         tc_fence_after();
         const uint32_t d = tmem + 2 * NPAD;
@@ -385,12 +407,12 @@ __global__ void __launch_bounds__(THREADS, 2)
           for (int k = 0; k < TOK / 32; ++k) {  // 32 tokens per MMA: four 8-token groups
             const uint64_t a = smem_desc(v_a + s * TILE_BYTES + k * 4096, 1024, 1024);
             const uint64_t bp =
-                smem_desc_plain(p_a + (i & 1) * PB_BYTES + term * PT_BYTES + k * 32 * NPAD, 128, 128);
+                smem_desc_plain(p_a + (i % PBUF) * PB_BYTES + term * PT_BYTES + k * 32 * NPAD, 128, 128);
             mma_e4m3(d, a, bp, kIdescE4M3_AMN_BMN, (!first || term > 0 || k > 0) ? 1u : 0u);
           }
         }
         mma_commit(&vr_empty[s]);
-        mma_commit(&p_free[i & 1]);
+        mma_commit(&p_free[i % PBUF]);
         return true;
       };
       ok = mbar_wait(q_ready, 0, p.status) && issue_qk(0);
@@ -420,7 +442,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     };
     // row r of O^T and the sums of the CTA's span, whose last tile is i
     auto flush = [&](int i) {
-      wait(&p_free[i & 1], (i >> 1) & 1);
+      wait(&p_free[i % PBUF], (i / PBUF) & 1);
       tc_fence_after();
       float o[16];
       tmem_ld16(tmem + lane_base + 2 * NPAD, o);
@@ -507,7 +529,7 @@ __global__ void __launch_bounds__(THREADS, 2)
           l_part[h] *= alpha[h];
         }
         named_sync(1, 128);
-        if (i > 0 && wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
+        if (i > 0 && wait(&p_free[(i - 1) % PBUF], ((i - 1) / PBUF) & 1)) {
           tc_fence_after();
           float o[16];
           tmem_ld16(tmem + lane_base + 2 * NPAD, o);
@@ -522,7 +544,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         pr[h] = valid ? exp2f(s[h] - m_run[h]) : 0.f;
         l_part[h] += pr[h];
       }
-      if (i >= 2) wait(&p_free[i & 1], ((i >> 1) - 1) & 1);
+      if (i >= PBUF) wait(&p_free[i % PBUF], ((i / PBUF) - 1) & 1);
       // P * 2^6 = P1 + P2, two E4M3 codes per head (heads h, h+1 in one pair);
       // token r's 16 head codes of each term are one 16-byte row of the
       // MN-major P^T operand (heads >= G are 0)
@@ -537,7 +559,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         w1[h >> 2] |= c1 << ((h & 2) * 8);
         w2[h >> 2] |= c2 << ((h & 2) * 8);
       }
-      uint8_t* pb = pop + (i & 1) * PB_BYTES + r * NPAD;
+      uint8_t* pb = pop + (i % PBUF) * PB_BYTES + r * NPAD;
       *reinterpret_cast<uint4*>(pb) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
       *reinterpret_cast<uint4*>(pb + PT_BYTES) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
       if (n_valid < TOK) {
@@ -553,7 +575,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[i & 1]);
+      if (lane == 0) mbar_arrive(&p_full[i % PBUF]);
     }
     flush(n_tiles - 1);
   }
@@ -602,8 +624,10 @@ int tc8_parts_per_cta(const DecodeArgs& a) {
 
 template <typename T, int G>
 cudaError_t launch_tc8_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
+  using Y = typename std::conditional<std::is_same<T, __nv_bfloat16>::value, LayBF16, LayF16>::type;
+  constexpr int SMEM_BYTES = Y::SMEM_BYTES;
   const int ppc = tc8_parts_per_cta(a);
-  auto kern = decode_partition_tc8_kernel<T, G>;
+  auto kern = decode_partition_tc8_kernel<T, G, Y>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // each cache [NB][Hkv][bs][128] as rows of 128 codes; a box is the bs rows of

@@ -576,6 +576,13 @@ __global__ void __launch_bounds__(THREADS, 2)
         // the last tile: zero the V rows of tokens past the end, so that
         // whatever they hold (unused slots, stale data) adds 0 * 0 to O
         const int u = 2 * i + 1, s_ = u % SLOTS;
+        // The parity wait below is only sound once the slot's previous load
+        // has landed.  With three slots that is K of tile i - 1, which S of
+        // tile i - 1 needed; with two it is V of tile i - 1, which may still be
+        // in flight (tile i's fewer blocks can land first) — wait for the MMA
+        // that read it, or the zeroing could come before tile i's V lands and
+        // bring back whatever the cache holds past the context.
+        if (SLOTS == 2 && i > 0) wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1);
         if (wait(&ring_full[s_], (u / SLOTS) & 1) && !valid) {
           uint8_t* row = ring + s_ * SLOT_BYTES + (r >> 3) * GROUP_BYTES + (r & 7) * 128;
 #pragma unroll

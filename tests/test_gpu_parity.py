@@ -696,3 +696,85 @@ def test_mq_few_queries_several_partitions_per_cta():
     spec = W.Spec("mq_ppc", "bf16", 32, 4, 128, 16, "independent", 320, seed=977,
                   ctx_dist="uniform", ctx_lo=2, ctx_hi=2000, partition_size=128)
     mq_check(spec, [1 + (i % 4) for i in range(320)], partition_size=128)
+
+
+# Repeated launches on the same inputs: every run finite and byte-identical to
+# the first.  A missed wait between an asynchronous copy and the threads that
+# patch its shared-memory tile shows up as an occasional run that differs (the
+# cache's unused slots hold NaN, so a patch overtaken by a late copy turns the
+# output non-finite); a single launch catches it only by chance.
+
+REPEATS = 24
+
+
+def _repeat_identical(launch):
+    first = launch().clone()
+    torch.cuda.synchronize()
+    assert pk.pa_device_status() == 0
+    assert torch.isfinite(first.float()).all()
+    bad = 0
+    for _ in range(REPEATS):
+        again = launch()
+        torch.cuda.synchronize()
+        bad += int(not torch.equal(first.view(torch.int16), again.view(torch.int16)))
+    assert pk.pa_device_status() == 0
+    assert bad == 0, f"{bad} of {REPEATS} runs differ from the first"
+    return first
+
+
+@pytest.mark.parametrize("G,qmax", [(8, 4), (8, 2), (4, 4), (4, 8)])
+def test_repeated_multi_query_launches_are_identical(G, qmax):
+    """Token-major multi-query decode at N = 16 and N = 32 columns (two-slot
+    ring), short last tiles after full ones."""
+    n = 160
+    spec = W.Spec(f"rep_mq_{G}_{qmax}", "bf16", 4 * G, 4, 128, 16, "independent", n,
+                  seed=1200 + G + qmax, ctx_dist="uniform", ctx_lo=130, ctx_hi=1500,
+                  partition_size=128)
+    p, o = build(W.scenario(spec))
+    run_step(p, spec)
+    torch.cuda.synchronize()
+    qlens = np.array([1 + (i % qmax) for i in range(n)], dtype=np.int64)
+    qs = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    T = int(qs[-1])
+    g = torch.Generator(device="cuda").manual_seed(G)
+    q = torch.randn((T, spec.Hq, spec.D), generator=g, device="cuda").to(W.torch_dtype(spec))
+    qs_dev = torch.from_numpy(qs).cuda()
+    ws_n = pk.pa_decode_multi_workspace_bytes(T, spec.Hq, spec.D, p.max_ctx, 128)
+    ws = torch.empty(ws_n // 4, dtype=torch.float32, device="cuda")
+    out = torch.empty_like(q)
+
+    def launch():
+        ws.fill_(float("nan"))
+        pk.pa_decode_multi(out, q, p.cache.k_cache, p.cache.v_cache, p.tables, p.lens, qs_dev,
+                           spec.softmax_scale, p.max_ctx, qmax, partition_size=128, workspace=ws)
+        return out
+
+    got = as_f64(_repeat_identical(launch), spec)
+    want = oracle.paged_attention_mq(W.storage_view(q), o.k, o.v, spec.dtype_code, o.tables,
+                                     o.lens, qs, spec.softmax_scale)
+    assert np.abs(got - want).max() <= TOL[spec.dtype]
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_repeated_decode_launches_are_identical(dtype, fp8):
+    """The tcgen05 decode kernels (E4M3: three-slot rings for f16 queries,
+    two-slot rings for bf16 queries)."""
+    spec = W.Spec(f"rep_dec_{dtype}", dtype, 32, 4, 128, 16, "independent", 256,
+                  seed=1300 + fp8, ctx_dist="uniform", ctx_lo=130, ctx_hi=3000,
+                  partition_size=512)
+    spec = W.fp8(spec) if fp8 else spec
+    p, o = build(W.scenario(spec))
+    run_step(p, spec)
+    torch.cuda.synchronize()
+    ws = p.cache.workspace(p.q.shape[0], p.q.shape[1], p.max_ctx, 512)
+    out = torch.empty_like(p.q)
+
+    def launch():
+        return p.cache.decode(p.q, p.tables, p.lens, p.max_ctx, spec.softmax_scale, out=out,
+                              partition_size=512, workspace=ws)
+
+    got = as_f64(_repeat_identical(launch), spec)
+    rows = sampled_rows(o, spec, n=96, seed=5)
+    want = oracle_attention(o, spec, rows=rows)
+    assert np.abs(got[rows[:, 0], rows[:, 1]] - want).max() <= TOL[spec.dtype]

@@ -31,11 +31,16 @@
 //   is never dereferenced (the copy is skipped and PA_DEVERR_TABLE set).
 //
 // E4M3 caches ("quantization" in "4. 이 밖의 기법들", blog.aqudi.me): the K/V
-// type TK is separate from the query/output type TQ.  A lane loads 8 codes (8
-// bytes) and widens them exactly to fp32; k_scale is folded into the query's
-// pre-scale and v_scale into the partial output, so the inner loops are those
-// of the 16-bit caches.  Half the bytes per token means twice the tokens per
-// stage (and twice the consumer warps) for the same bytes in flight.
+// type TK is separate from the query/output type TQ.  A lane loads 16 codes (16
+// bytes; 8 at G > 2); k_scale is folded into the score scale and v_scale into the partial
+// output.  Every E4M3 value is an f16 value and the hardware converts a code
+// pair to an f16x2 pair exactly.  With f16 queries the products q_e k_e and
+// p v_e are then taken by the mixed-precision FMA (two f16 operands, an fp32
+// addend and result: the product of two f16 values is exact in fp32, so this
+// is fmaf of the widened operands without the widening); with bf16 or fp32
+// queries the codes are widened to fp32 and the loops are those of the 16-bit
+// caches.  Half the bytes per token means twice the tokens per stage (and
+// twice the consumer warps) for the same bytes in flight.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -53,11 +58,14 @@ constexpr unsigned FULL_MASK = 0xffffffffu;
 constexpr int cmax(int a, int b) { return a > b ? a : b; }
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
 constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
+constexpr float RESCALE_LOG2 = 8.0f;   // raise the running max past 2^8 growth
 
 template <typename T, int D, int G, int NCW>
 struct Cfg {
   static constexpr int ES = sizeof(T);
-  static constexpr int EPL = Elem<T>::EPL;     // elements a lane loads at once
+  // elements a lane loads at once: one 16-byte chunk (8 codes at G > 2, where
+  // the query and output registers grow with G)
+  static constexpr int EPL = ES == 1 ? (G <= 2 ? 16 : 8) : Elem<T>::EPL;
   static constexpr int LPR = D / EPL;          // lanes per K/V row
   static constexpr int RPW = 32 / LPR;         // rows a warp covers per iteration
   static constexpr int TOK = NCW * 8;          // tokens per stage (8 per consumer warp)
@@ -91,6 +99,50 @@ __device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, f
       "fma.rn.f32x2 d, a, b, d;\n\tmov.b64 {%0, %1}, d;\n\t}"
       : "+f"(d0), "+f"(d1)
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// fmaf(a, b, c) for f16 a, b (raw bits) and fp32 c: the mixed-precision FMA.
+__device__ __forceinline__ float fma_h(uint16_t a, uint16_t b, float c) {
+  float d;
+  asm("fma.rn.f32.f16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ uint16_t lo16(uint32_t x) { return static_cast<uint16_t>(x & 0xffffu); }
+__device__ __forceinline__ uint16_t hi16(uint32_t x) { return static_cast<uint16_t>(x >> 16); }
+
+// 16 E4M3 codes (one 16-byte chunk in shared memory) as 8 f16x2 pairs, code
+// 2i in the low half of h[i].
+__device__ __forceinline__ void codes_to_f16x2(const void* src, uint32_t* h) {
+  const uint4 u = *reinterpret_cast<const uint4*>(src);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(
+          static_cast<__nv_fp8x2_storage_t>((w[i] >> (16 * j)) & 0xffffu), __NV_E4M3);
+      h[2 * i + j] = static_cast<uint32_t>(r.x) | (static_cast<uint32_t>(r.y) << 16);
+    }
+  }
+}
+
+// EPL elements of a K/V row chunk in shared memory widened to fp32: 16 E4M3
+// codes, or one 16-byte chunk of a 16/32-bit type.
+template <typename TK, int EPL>
+__device__ __forceinline__ void load_row(const TK* src, float* f) {
+  if constexpr (sizeof(TK) == 1 && EPL == 16) {
+    uint32_t h[8];
+    codes_to_f16x2(src, h);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
+      f[2 * i] = v.x;
+      f[2 * i + 1] = v.y;
+    }
+  } else {
+    static_assert(EPL == Elem<TK>::EPL, "one load of the element type");
+    Elem<TK>::load(src, f);
+  }
 }
 
 // q row chunk of EPL elements of TQ (global memory, read-only path) to fp32.
@@ -285,14 +337,30 @@ __global__ void __launch_bounds__(Cfg<TK, D, G, NCW>::THREADS)
   const int c = lane % C::LPR;      // 16-byte chunk of the row this lane owns
   float* sc = scores + w * C::NSM;  // [G][TPW]
 
-  float qf[G][C::EPL];
+  // f16 queries over 16-code chunks keep q as raw f16x2 pairs (the scale is
+  // applied to the finished dot); otherwise q is fp32, pre-scaled
+  constexpr bool kMixed = kCoded && std::is_same<TQ, __half>::value && C::EPL == 16;
+  constexpr int QW = kMixed ? C::EPL / 2 : 1;
+  float qf[G][kMixed ? 1 : C::EPL];
+  uint32_t qh[G][QW];
   {
     const TQ* qrow = static_cast<const TQ*>(p.q) + (static_cast<int64_t>(b) * p.Hq + g * G) * D;
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      load_q<TQ, C::EPL>(qrow + h * D + c * C::EPL, qf[h]);
+      if constexpr (kMixed) {
 #pragma unroll
-      for (int e = 0; e < C::EPL; ++e) qf[h][e] *= p.scale_log2;
+        for (int i = 0; i < QW / 4; ++i) {
+          const uint4 u = __ldg(reinterpret_cast<const uint4*>(qrow + h * D + c * C::EPL) + i);
+          qh[h][4 * i] = u.x;
+          qh[h][4 * i + 1] = u.y;
+          qh[h][4 * i + 2] = u.z;
+          qh[h][4 * i + 3] = u.w;
+        }
+      } else {
+        load_q<TQ, C::EPL>(qrow + h * D + c * C::EPL, qf[h]);
+#pragma unroll
+        for (int e = 0; e < C::EPL; ++e) qf[h][e] *= p.scale_log2;
+      }
     }
   }
   float m[G], l[G], o[G][C::EPL];
@@ -320,15 +388,31 @@ __global__ void __launch_bounds__(Cfg<TK, D, G, NCW>::THREADS)
 #pragma unroll
     for (int it = 0; it < C::ITERS; ++it) {
       const int row = w * C::TPW + it * C::RPW + r;
-      float kf[C::EPL];
-      E::load(Ks + row * D + c * C::EPL, kf);
+      if constexpr (kMixed) {
+        uint32_t kh[C::EPL / 2];
+        codes_to_f16x2(Ks + row * D + c * C::EPL, kh);
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        // even and odd elements in the two halves of a paired FMA
-        float a0 = 0.f, a1 = 0.f;
+        for (int h = 0; h < G; ++h) {
+          // even and odd elements in two accumulators, as below
+          float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-        for (int e = 0; e < C::EPL; e += 2) fma2(a0, a1, qf[h][e], qf[h][e + 1], kf[e], kf[e + 1]);
-        part_dot[h * C::ITERS + it] = a0 + a1;
+          for (int i = 0; i < C::EPL / 2; ++i) {
+            a0 = fma_h(lo16(qh[h][i]), lo16(kh[i]), a0);
+            a1 = fma_h(hi16(qh[h][i]), hi16(kh[i]), a1);
+          }
+          part_dot[h * C::ITERS + it] = (a0 + a1) * p.scale_log2;
+        }
+      } else {
+        float kf[C::EPL];
+        load_row<TK, C::EPL>(Ks + row * D + c * C::EPL, kf);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          // even and odd elements in the two halves of a paired FMA
+          float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+          for (int e = 0; e < C::EPL; e += 2) fma2(a0, a1, qf[h][e], qf[h][e + 1], kf[e], kf[e + 1]);
+          part_dot[h * C::ITERS + it] = a0 + a1;
+        }
       }
     }
     reduce_scatter<C::NV, C::LPR / 2>(part_dot, lane);
@@ -361,12 +445,18 @@ __global__ void __launch_bounds__(Cfg<TK, D, G, NCW>::THREADS)
       for (int off = C::TPW / 2; off >= 1; off >>= 1) x = fmaxf(x, __shfl_xor_sync(FULL_MASK, x, off));
       seg[ps] = x;
     }
+    // The running max is raised only when a score passes it by 2^8 (base 2),
+    // so O is rarely rescaled; P <= 2^8 meanwhile.  tmax is the same in every
+    // lane, so `raise` is warp-uniform.
     float mnew[G], alpha[G];
+    bool raise = false;
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       const float tmax = __shfl_sync(FULL_MASK, seg[(h * C::TPW) / 32], (h * C::TPW) % 32);
-      mnew[h] = fmaxf(m[h], tmax);
-      alpha[h] = (mnew[h] == -INFINITY) ? 1.f : exp2f(m[h] - mnew[h]);
+      const bool up = tmax > m[h] + RESCALE_LOG2;
+      mnew[h] = up ? tmax : m[h];
+      alpha[h] = !up ? 1.f : (m[h] == -INFINITY) ? 0.f : exp2f(m[h] - tmax);
+      raise |= up;
     }
 #pragma unroll
     for (int ps = 0; ps < C::NPASS; ++ps) {
@@ -387,8 +477,10 @@ __global__ void __launch_bounds__(Cfg<TK, D, G, NCW>::THREADS)
       const float tsum = __shfl_sync(FULL_MASK, seg[(h * C::TPW) / 32], (h * C::TPW) % 32);
       l[h] = l[h] * alpha[h] + tsum;
       m[h] = mnew[h];
+      if (raise) {
 #pragma unroll
-      for (int e = 0; e < C::EPL; ++e) o[h][e] *= alpha[h];
+        for (int e = 0; e < C::EPL; ++e) o[h][e] *= alpha[h];
+      }
     }
     __syncwarp();
 
@@ -398,13 +490,29 @@ __global__ void __launch_bounds__(Cfg<TK, D, G, NCW>::THREADS)
       const int row_local = it * C::RPW + r;
       const int row = w * C::TPW + row_local;
       if (row < n_valid) {
-        float vf[C::EPL];
-        E::load(Vs + row * D + c * C::EPL, vf);
+        if constexpr (kMixed) {
+          // P rounded to f16 (as the tensor-core kernels round it to the
+          // operand type), V exact
+          uint32_t vh[C::EPL / 2];
+          codes_to_f16x2(Vs + row * D + c * C::EPL, vh);
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float pr = sc[h * C::TPW + row_local];
+          for (int h = 0; h < G; ++h) {
+            const uint16_t ph = __half_as_ushort(__float2half_rn(sc[h * C::TPW + row_local]));
 #pragma unroll
-          for (int e = 0; e < C::EPL; e += 2) fma2(o[h][e], o[h][e + 1], pr, pr, vf[e], vf[e + 1]);
+            for (int i = 0; i < C::EPL / 2; ++i) {
+              o[h][2 * i] = fma_h(ph, lo16(vh[i]), o[h][2 * i]);
+              o[h][2 * i + 1] = fma_h(ph, hi16(vh[i]), o[h][2 * i + 1]);
+            }
+          }
+        } else {
+          float vf[C::EPL];
+          load_row<TK, C::EPL>(Vs + row * D + c * C::EPL, vf);
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float pr = sc[h * C::TPW + row_local];
+#pragma unroll
+            for (int e = 0; e < C::EPL; e += 2) fma2(o[h][e], o[h][e + 1], pr, pr, vf[e], vf[e + 1]);
+          }
         }
       }
     }

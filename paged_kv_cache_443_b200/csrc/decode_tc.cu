@@ -29,9 +29,9 @@
 //            second MMA, zeroes the V rows of invalid tokens of a final tile, and
 //            at the end reads its row of O from TMEM and writes the output or the
 //            split-K partial.
-// About 110 KB of shared memory, so two CTAs share an SM and hide each other's
-// pipeline fill.  Every mbarrier wait is bounded; block ids outside the pool are
-// skipped and flagged.
+// About 109 KB of shared memory (113 KB with 32 columns), so two CTAs share an
+// SM and hide each other's pipeline fill.  Every mbarrier wait is bounded;
+// block ids outside the pool are skipped and flagged.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -86,27 +86,63 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 }
 
 // Shared-memory and TMEM layout for N = NP columns (16, or 32 for 32 query
-// tokens x heads): a ring of SLOTS K/V tiles (three at N = 16; two at N = 32,
-// so that two CTAs still share an SM), the Q^T operand and two P buffers of NP
-// rows in two swizzled 64-column blocks, barriers, the TMEM address and a
-// 4-warp reduction buffer.  TMEM: S0 [0, NP), S1 [NP, 2NP), O [2NP, 3NP).
+// tokens x heads).  The 1024-byte aligned part holds a ring of three K/V tiles,
+// the Q^T operand and PBUF P^T buffers of NP columns (two at N = 16; one at
+// N = 32, so that two CTAs still share an SM).  The barriers, the TMEM address
+// and the 4-warp reduction buffer live in the 1 KB the allocation adds for
+// aligning the base: in front of the aligned part where the base's offset
+// leaves room, behind it otherwise (small_layout).
+// TMEM: S0 [0, NP), S1 [NP, 2NP), O [2NP, 3NP).
 template <int NP>
 struct Lay {
   static constexpr int NPAD = NP;
-  static constexpr int SLOTS = NP <= 16 ? 3 : 2;
+  static constexpr int SLOTS = 3;
+  static constexpr int PBUF = NP <= 16 ? 2 : 1;
   static constexpr int OPB_BYTES = 2 * NP * 128;   // Q^T (K-major) or P^T (MN-major): NP x 128 16-bit
   static constexpr int OFF_RING = 0;
   static constexpr int OFF_Q = OFF_RING + SLOTS * SLOT_BYTES;
   static constexpr int OFF_P = OFF_Q + OPB_BYTES;
-  static constexpr int OFF_BAR = OFF_P + 2 * OPB_BYTES;
-  static constexpr int NBARS = 2 * SLOTS + 9;   // ring full/empty, s/p full/free, q_ready
-  static constexpr int OFF_TMEM = OFF_BAR + NBARS * 8;
-  static constexpr int OFF_RED = OFF_TMEM + 16;
-  static constexpr int SMEM_USED = OFF_RED + 4 * NP * 4;
-  static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack to align the base to 1024 B
+  static constexpr int ALIGNED_BYTES = OFF_P + PBUF * OPB_BYTES;
+  // ring full/empty, S full/free, P full/free, Q ready
+  static constexpr int NBARS = 2 * SLOTS + 4 + 2 * PBUF + 1;
+  static constexpr int RED_BYTES = 4 * NP * 4;
+  static constexpr int MISC_BYTES = (NBARS * 8 + 16 + 15) / 16 * 16;   // barriers, TMEM address
+  static constexpr int SMEM_BYTES = ALIGNED_BYTES + 1024;
   static constexpr int TMEM_COLS = 3 * NP <= 64 ? 64 : 128;
-  static_assert(SMEM_BYTES * 2 + 2048 <= 228 * 1024, "two CTAs per SM");
+  // small_layout's placement always fits when these hold
+  static_assert(RED_BYTES <= 512 && RED_BYTES + 2 * MISC_BYTES <= 1024, "small buffers");
+  static_assert(2 * (SMEM_BYTES + 1024) <= 228 * 1024, "two CTAs per SM");
 };
+
+// Where the small buffers go, given the dynamic allocation's base: f bytes
+// lie in front of the aligned part and 1024 - f behind it (f a multiple of 16).
+// The reduction buffer goes in front if it fits there, else behind (1024 - f >
+// 512 >= its size); the barriers take whichever side still has room, which
+// RED_BYTES + 2 * MISC_BYTES <= 1024 guarantees.
+template <int NP>
+struct SmemPtrs {
+  uint8_t* aligned;
+  float* red;
+  uint8_t* misc;
+};
+template <int NP>
+__device__ __forceinline__ SmemPtrs<NP> small_layout(uint8_t* raw) {
+  using Y = Lay<NP>;
+  const uintptr_t b = reinterpret_cast<uintptr_t>(raw);
+  const uint32_t f = static_cast<uint32_t>(((b + 1023) & ~static_cast<uintptr_t>(1023)) - b);
+  SmemPtrs<NP> r;
+  r.aligned = raw + f;
+  uint8_t* back = r.aligned + Y::ALIGNED_BYTES;
+  if (f >= static_cast<uint32_t>(Y::RED_BYTES)) {
+    r.red = reinterpret_cast<float*>(raw);
+    r.misc = f - Y::RED_BYTES >= static_cast<uint32_t>(Y::MISC_BYTES) ? raw + Y::RED_BYTES : back;
+  } else {
+    r.red = reinterpret_cast<float*>(back);
+    r.misc = 1024 - f - Y::RED_BYTES >= static_cast<uint32_t>(Y::MISC_BYTES) ? back + Y::RED_BYTES
+                                                                               : raw;
+  }
+  return r;
+}
 
 struct TcParams {
   void* out;
@@ -152,25 +188,25 @@ __global__ void __launch_bounds__(THREADS, 2)
     decode_partition_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmap_k,
                                const __grid_constant__ CUtensorMap tmap_v) {
   using Y = Lay<NP>;
-  constexpr int NPAD = NP, SLOTS = Y::SLOTS, OPB_BYTES = Y::OPB_BYTES;
-  constexpr int OFF_RING = Y::OFF_RING, OFF_Q = Y::OFF_Q, OFF_P = Y::OFF_P, OFF_BAR = Y::OFF_BAR;
-  constexpr int OFF_TMEM = Y::OFF_TMEM, OFF_RED = Y::OFF_RED, TMEM_COLS = Y::TMEM_COLS;
+  constexpr int NPAD = NP, SLOTS = Y::SLOTS, PBUF = Y::PBUF, OPB_BYTES = Y::OPB_BYTES;
+  constexpr int OFF_RING = Y::OFF_RING, OFF_Q = Y::OFF_Q, OFF_P = Y::OFF_P;
+  constexpr int TMEM_COLS = Y::TMEM_COLS;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const SmemPtrs<NP> sp = small_layout<NP>(smem_raw);
+  uint8_t* smem = sp.aligned;
   uint8_t* ring = smem + OFF_RING;
   uint8_t* qop = smem + OFF_Q;
   uint8_t* pop = smem + OFF_P;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sp.misc);
   uint64_t* ring_full = bars;
   uint64_t* ring_empty = bars + SLOTS;
   uint64_t* s_full = bars + 2 * SLOTS;      // [2]
   uint64_t* s_free = s_full + 2;            // [2]
-  uint64_t* p_full = s_free + 2;            // [2]
-  uint64_t* p_free = p_full + 2;            // [2]
-  uint64_t* q_ready = p_free + 2;           // Q^T operand staged
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
-  float* red = reinterpret_cast<float*>(smem + OFF_RED);
+  uint64_t* p_full = s_free + 2;            // [PBUF]
+  uint64_t* p_free = p_full + PBUF;         // [PBUF]
+  uint64_t* q_ready = p_free + PBUF;        // Q^T operand staged
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sp.misc + Y::NBARS * 8);
+  float* red = sp.red;
 
   // A CTA covers parts_per_cta consecutive partitions with one softmax, so
   // short partitions do not each pay the pipeline's fill and drain: its partial
@@ -294,6 +330,8 @@ __global__ void __launch_bounds__(THREADS, 2)
       for (int j = 0; j < 2; ++j) {
         mbar_init(&s_full[j], 1);
         mbar_init(&s_free[j], 4);
+      }
+      for (int j = 0; j < PBUF; ++j) {
         mbar_init(&p_full[j], 4);
         mbar_init(&p_free[j], 1);
       }
@@ -330,7 +368,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       const uint32_t off = (c / 8) * (NPAD * 128) + sw128(h, (c % 8) * 8);
       *reinterpret_cast<uint4*>(qop + off) = v;
     }
-    for (int i = t; i < 2 * OPB_BYTES / 16; i += 128)
+    for (int i = t; i < PBUF * OPB_BYTES / 16; i += 128)
       reinterpret_cast<uint4*>(pop)[i] = make_uint4(0, 0, 0, 0);
     fence_async_smem();
     __syncwarp();
@@ -404,7 +442,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       auto issue_pv = [&](int i) -> bool {
         const int u = 2 * i + 1, s = u % SLOTS;
         if (!mbar_wait(&ring_full[s], (u / SLOTS) & 1, p.status)) return false;
-        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, p.status)) return false;
+        if (!mbar_wait(&p_full[i % PBUF], (i / PBUF) & 1, p.status)) return false;
         const bool first = i == 0;                     // O starts at 0
         tc_fence_after();
         const uint32_t d = tmem + 2 * NPAD;
@@ -412,11 +450,11 @@ __global__ void __launch_bounds__(THREADS, 2)
         for (int k = 0; k < TOK / 16; ++k) {
           const uint64_t a =
               smem_desc(ring_a + s * SLOT_BYTES + k * 2 * GROUP_BYTES, HALF_OFF, GROUP_BYTES);
-          const uint64_t bp = smem_desc_plain(p_a + (i & 1) * OPB_BYTES + k * 16 * 16, 128, P_CHUNK);
+          const uint64_t bp = smem_desc_plain(p_a + (i % PBUF) * OPB_BYTES + k * 16 * 16, 128, P_CHUNK);
           mma_f16(d, a, bp, id_pv, (!first || k > 0) ? 1u : 0u);
         }
         mma_commit(&ring_empty[s]);
-        mma_commit(&p_free[i & 1]);
+        mma_commit(&p_free[i % PBUF]);
         return true;
       };
       ok = mbar_wait(q_ready, 0, p.status) && issue_qk(0);
@@ -450,7 +488,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     // tile is i: the output, or the split-K partial of partition part (and
     // empty partials for the span's other partitions).
     auto flush = [&](int i) {
-      wait(&p_free[i & 1], (i >> 1) & 1);
+      wait(&p_free[i % PBUF], (i / PBUF) & 1);
       tc_fence_after();
       float o[NPAD];
       tmem_ld_cols<NPAD>(tmem + lane_base + 2 * NPAD, o);
@@ -542,7 +580,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         named_sync(1, 128);
         // O must hold every earlier tile before it is rescaled (at the first
         // tile O starts from zero instead)
-        if (i > 0 && wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
+        if (i > 0 && wait(&p_free[(i - 1) % PBUF], ((i - 1) / PBUF) & 1)) {
           tc_fence_after();
           float o[NPAD];
           tmem_ld_cols<NPAD>(tmem + lane_base + 2 * NPAD, o);
@@ -558,10 +596,10 @@ __global__ void __launch_bounds__(THREADS, 2)
         pr[h] = counted ? exp2f(s[h] - m_run[h]) : 0.f;
         l_part[h] += pr[h];
       }
-      if (i >= 2) wait(&p_free[i & 1], ((i >> 1) - 1) & 1);
+      if (i >= PBUF) wait(&p_free[i % PBUF], ((i / PBUF) - 1) & 1);   // P buffer read
       // token r's columns are 16-byte rows of the MN-major P^T operand: heads
       // 8c .. 8c + 7 at chunk c (columns >= NC stay 0)
-      uint8_t* pb = pop + (i & 1) * OPB_BYTES + r * 16;
+      uint8_t* pb = pop + (i % PBUF) * OPB_BYTES + r * 16;
 #pragma unroll
       for (int c = 0; c < (NC + 7) / 8; ++c) {
         uint32_t w[4];
@@ -582,7 +620,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         // in flight (tile i's fewer blocks can land first) — wait for the MMA
         // that read it, or the zeroing could come before tile i's V lands and
         // bring back whatever the cache holds past the context.
-        if (SLOTS == 2 && i > 0) wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1);
+        if (SLOTS == 2 && i > 0) wait(&p_free[(i - 1) % PBUF], ((i - 1) / PBUF) & 1);
         if (wait(&ring_full[s_], (u / SLOTS) & 1) && !valid) {
           uint8_t* row = ring + s_ * SLOT_BYTES + (r >> 3) * GROUP_BYTES + (r & 7) * 128;
 #pragma unroll
@@ -595,7 +633,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[i & 1]);
+      if (lane == 0) mbar_arrive(&p_full[i % PBUF]);
     }
     flush(n_tiles - 1);
   }
@@ -619,6 +657,8 @@ cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t 
   auto kern = decode_partition_tc_kernel<T, G>;
   constexpr int SMEM_BYTES = Lay<16>::SMEM_BYTES;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e == cudaSuccess)   // all of the SM's 228 KB as shared memory: two CTAs of up to 113 KB
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   // the cache [NB][Hkv][bs][128] as a 4-D tensor: 64 columns (stride 2 B),
   // 8 rows (256 B), 2 column halves (128 B), NB*Hkv*bs/8 row groups (2 KB); a
@@ -675,6 +715,8 @@ cudaError_t launch_group_tc_t(const DecodeArgs& a, unsigned int* status, cudaStr
   auto kern = decode_partition_tc_kernel<T, G, NQ>;
   constexpr int SMEM_BYTES = Lay<16>::SMEM_BYTES;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e == cudaSuccess)   // all of the SM's 228 KB as shared memory: two CTAs of up to 113 KB
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   CUtensorMap mk, mv;
   const int64_t groups = static_cast<int64_t>(a.num_blocks) * a.Hkv * a.block_size / 8;
@@ -798,6 +840,8 @@ cudaError_t launch_tcq_t(const MqArgs& m, unsigned int* status, cudaStream_t str
   auto kern = decode_partition_tc_kernel<T, G, NQ, NP>;
   constexpr int SMEM_BYTES = Lay<NP>::SMEM_BYTES;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e == cudaSuccess)   // all of the SM's 228 KB as shared memory: two CTAs of up to 113 KB
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   CUtensorMap mk, mv;
   const int64_t groups = static_cast<int64_t>(m.num_blocks) * m.Hkv * m.block_size / 8;

@@ -625,7 +625,8 @@ extern "C" pa_status pa_decode_multi(void* out, const void* q, const void* k_cac
 namespace {
 
 // pa_decode_grouped runs the groups' spans on a library-owned stream of the
-// device next to the rest of the sequences on the caller's stream: a fork
+// device (at its highest priority) next to the rest of the sequences on the
+// caller's stream: a fork
 // event recorded on the caller's stream, then a join event the caller's stream
 // waits on before the reduce.  Created on first use; the mutex keeps the
 // record / wait / launch sequence of concurrent host threads apart (an event's
@@ -644,7 +645,13 @@ AuxStream* aux_stream(int dev) {
   if (!x.stream) {
     cudaStream_t st = nullptr;
     cudaEvent_t f = nullptr, j = nullptr;
-    if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    // the highest priority of the device: the spans' CTAs (few, long) are
+    // placed before the rest's (many, short), which then fill the SMs the
+    // spans' last wave leaves idle instead of pushing that wave to the end
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&st, cudaStreamNonBlocking, greatest) != cudaSuccess)
+      return nullptr;
     if (cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess) {
       if (f) cudaEventDestroy(f);

@@ -259,9 +259,11 @@ KERNEL_SOURCES = {
     "decode_partition_tc8_kernel": ("decode_tc8.cu", "tc_common.cuh", "pa_device.cuh",
                                     "pa_internal.h"),
     # pa_decode_grouped: the span and rest kernels (decode_tc.cu, or decode.cu
-    # for G = 1, 2) and the reduce (decode.cu)
+    # for G = 1, 2) and the reduce (decode.cu); E4M3 caches: decode_tc8.cu
     "decode_grouped": ("decode_tc.cu", "decode.cu", "tc_common.cuh", "pa_device.cuh",
                        "pa_internal.h"),
+    "decode_grouped_fp8": ("decode_tc8.cu", "decode.cu", "tc_common.cuh", "pa_device.cuh",
+                           "pa_internal.h"),
 }
 
 
@@ -465,8 +467,7 @@ def run_ours(args):
     # families sharing leading blocks (parallel samples, a common prefix) are
     # decoded with each family's shared span read once, unless --grouped off
     groups = None
-    if args.grouped == "on" or (args.grouped == "auto" and spec.kind != "independent"
-                                and not spec.fp8):
+    if args.grouped == "on" or (args.grouped == "auto" and spec.kind != "independent"):
         groups = cache.groups(tables, lens)
         if groups.max_shared_len == 0:
             groups = None
@@ -497,8 +498,13 @@ def run_ours(args):
             ev[1].record(stream)
         if groups is not None:
             # one call: the groups' spans, the rest of each sequence, the reduce
-            pk.pa_decode_grouped(out, q, kc, vc, tables, lens, groups, scale, max_ctx,
-                                 partition_size=P, workspace=ws, stream=stream)
+            if spec.fp8:
+                pk.pa_decode_grouped_fp8(out, q, kc, vc, tables, lens, groups, scale, max_ctx,
+                                         spec.k_scale, spec.v_scale, partition_size=P,
+                                         workspace=ws, stream=stream)
+            else:
+                pk.pa_decode_grouped(out, q, kc, vc, tables, lens, groups, scale, max_ctx,
+                                     partition_size=P, workspace=ws, stream=stream)
             if ev is not None:
                 ev[2].record(stream)
                 ev[3].record(stream)
@@ -651,10 +657,12 @@ def run_ours(args):
     if groups is not None:
         # the three launches of the grouped decode are timed together (the
         # reduce included), against the same algorithmic bytes
-        kname = ("decode_grouped: decode_partition_tc_kernel (the families' shared spans, "
+        span_kernel = "decode_partition_tc8_kernel" if spec.fp8 else "decode_partition_tc_kernel"
+        kname = ("decode_grouped: " + span_kernel + " (the families' shared spans, "
                  "16/G members per CTA) next to " + partition_kernel(spec, P) +
                  " (the rest of every sequence), then decode_reduce_kernel")
-        traffic, traffic_note = profiled_traffic(args.workload, "decode_grouped", P)
+        traffic, traffic_note = profiled_traffic(
+            args.workload, "decode_grouped_fp8" if spec.fp8 else "decode_grouped", P)
 
     result = None
     if rank == 0:
@@ -690,7 +698,8 @@ def run_ours(args):
                 "parallelism": "replicas" if world == 1 else f"replicas x{world} (no collective)",
                 "decode": (f"grouped: {groups.num_groups} families sharing up to "
                            f"{groups.max_shared_len} leading tokens, each shared span read once "
-                           f"for its members (pa_decode_grouped)" if groups is not None
+                           f"for its members (pa_decode_grouped{'_fp8' if spec.fp8 else ''})"
+                           if groups is not None
                            else "pa_decode_partitions + pa_decode_reduce"),
             },
             "kernels_us": ({  # from the second pass, with events between the kernels

@@ -313,6 +313,25 @@ pa_status pa_decode_grouped(void* out, const void* q, const void* k_cache, const
                             pa_dtype dtype, int partition_size, int max_context_len,
                             void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * pa_decode_grouped over an E4M3 cache: q and out of type `dtype` (f16 or
+ * bf16 for the shared spans' tensor-core kernel), cache elements standing for
+ * code * k_scale (keys) and code * v_scale (values), as pa_decode_fp8.  The
+ * result is that of pa_decode_fp8 on the same arguments; group arguments,
+ * workspace, launches and device-side checks are those of pa_decode_grouped.
+ * With nothing shared, f32 queries or head size 64 this is pa_decode_fp8.
+ */
+pa_status pa_decode_grouped_fp8(void* out, const void* q, const void* k_cache,
+                                const void* v_cache, const int32_t* block_tables,
+                                int max_blocks_per_seq, const int32_t* context_lens,
+                                const int32_t* group_start, const int32_t* shared_lens,
+                                int num_groups, int max_group_size, int max_shared_len,
+                                int num_seqs, int num_heads, int num_kv_heads, int head_size,
+                                int block_size, int num_blocks, float scale, pa_dtype dtype,
+                                float k_scale, float v_scale, int partition_size,
+                                int max_context_len, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Cache updates                                                           */
 

@@ -38,7 +38,8 @@ EXPORTS = (
     "pa_alloc_refcount", "pa_alloc_free_stack", "pa_seq_add", "pa_seq_fork", "pa_seq_append",
     "pa_seq_free", "pa_seq_move", "pa_seq_num_tokens", "pa_build_tables",
     "pa_alloc_enable_prefix_cache", "pa_alloc_evictable", "pa_seq_add_cached", "pa_seq_commit",
-    "pa_decode_grouped", "pa_decode_grouped_workspace_bytes", "pa_build_groups",
+    "pa_decode_grouped", "pa_decode_grouped_fp8", "pa_decode_grouped_workspace_bytes",
+    "pa_build_groups",
 )
 
 
@@ -118,6 +119,9 @@ def lib():
         "pa_build_tables": ([vp, pi64, i32, i32, pi32, pi32], i32),
         "pa_decode_grouped": ([vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                i32, i32, i32, f32, i32, i32, i32, vp, sz, vp], i32),
+        "pa_decode_grouped_fp8": ([vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32,
+                                   i32, i32, i32, i32, f32, i32, f32, f32, i32, i32, vp, sz, vp],
+                                  i32),
         "pa_decode_grouped_workspace_bytes": ([i32, i32, i32, i32, i32, i32], sz),
         "pa_build_groups": ([pi32, i32, i32, pi32, i32, pi32, pi32, ctypes.POINTER(i32),
                              ctypes.POINTER(i32), ctypes.POINTER(i32)], i32),
@@ -304,6 +308,21 @@ def pa_decode_grouped(out, q, k_cache, v_cache, block_tables, context_lens, grou
     _check(lib().pa_decode_grouped(*a[:7], _ptr(groups.group_start), _ptr(groups.shared_lens),
                                    groups.num_groups, groups.max_group_size,
                                    groups.max_shared_len, *a[7:]))
+
+
+def pa_decode_grouped_fp8(out, q, k_cache, v_cache, block_tables, context_lens, groups: Groups,
+                          scale, max_context_len, k_scale, v_scale, partition_size=0,
+                          workspace=None, stream=None) -> None:
+    """pa_decode_fp8's result over E4M3 caches, with each group's shared span
+    read once for all its members."""
+    import torch
+    a = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, partition_size,
+                     max_context_len, workspace, stream, kv_dtype=torch.float8_e4m3fn)
+    _contig(groups.group_start, groups.shared_lens)
+    _check(lib().pa_decode_grouped_fp8(*a[:7], _ptr(groups.group_start), _ptr(groups.shared_lens),
+                                       groups.num_groups, groups.max_group_size,
+                                       groups.max_shared_len, *a[7:15], float(k_scale),
+                                       float(v_scale), *a[15:]))
 
 
 def pa_decode_partitions(out, q, k_cache, v_cache, block_tables, context_lens, scale,

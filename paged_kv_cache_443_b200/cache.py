@@ -18,7 +18,8 @@ from typing import List, Optional, Sequence, Tuple
 import torch
 
 from . import (BlockAllocator, Groups, pa_build_groups, pa_copy_blocks, pa_decode,
-               pa_decode_fp8, pa_decode_grouped, pa_decode_grouped_workspace_bytes,
+               pa_decode_fp8, pa_decode_grouped, pa_decode_grouped_fp8,
+               pa_decode_grouped_workspace_bytes,
                pa_decode_workspace_bytes, pa_reshape_and_cache, pa_reshape_and_cache_fp8,
                pa_swap_blocks)
 
@@ -155,17 +156,23 @@ class PagedKVCache:
                partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
                stream=None, groups: Optional[Groups] = None) -> torch.Tensor:
         """Decode attention of the batch; with `groups` (self.groups(...)) each
-        group's shared leading blocks are read once for all its members (16-bit
-        caches; the result is the same)."""
+        group's shared leading blocks are read once for all its members (the
+        result is the same)."""
         if out is None:
             out = torch.empty_like(q)
-        if groups is not None and not self.fp8:
+        if groups is not None:
             if workspace is None:
                 workspace = self.grouped_workspace(q.shape[0], q.shape[1], max_context_len,
                                                    groups, partition_size)
-            pa_decode_grouped(out, q, self.k_cache, self.v_cache, block_tables, context_lens,
-                              groups, scale, max_context_len, partition_size=partition_size,
-                              workspace=workspace, stream=stream)
+            if self.fp8:
+                pa_decode_grouped_fp8(out, q, self.k_cache, self.v_cache, block_tables,
+                                      context_lens, groups, scale, max_context_len, self.k_scale,
+                                      self.v_scale, partition_size=partition_size,
+                                      workspace=workspace, stream=stream)
+            else:
+                pa_decode_grouped(out, q, self.k_cache, self.v_cache, block_tables, context_lens,
+                                  groups, scale, max_context_len, partition_size=partition_size,
+                                  workspace=workspace, stream=stream)
             return out
         if workspace is None:
             workspace = self.workspace(q.shape[0], q.shape[1], max_context_len, partition_size)

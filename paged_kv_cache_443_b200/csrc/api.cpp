@@ -685,20 +685,34 @@ extern "C" size_t pa_decode_grouped_workspace_bytes(int num_seqs, int num_heads,
   return (raw + 255) / 256 * 256;
 }
 
-extern "C" pa_status pa_decode_grouped(void* out, const void* q, const void* k_cache,
-                                       const void* v_cache, const int32_t* block_tables,
-                                       int max_blocks_per_seq, const int32_t* context_lens,
-                                       const int32_t* group_start, const int32_t* shared_lens,
-                                       int num_groups, int max_group_size, int max_shared_len,
-                                       int num_seqs, int num_heads, int num_kv_heads,
-                                       int head_size, int block_size, int num_blocks,
-                                       float scale, pa_dtype dtype, int partition_size,
-                                       int max_context_len, void* workspace,
-                                       size_t workspace_bytes_in, void* stream) {
-  const char* fn = "pa_decode_grouped";
+namespace {
+
+// pa_decode_grouped and pa_decode_grouped_fp8 (E4M3 caches: fp8 set, the
+// cache's scales given): the same checks, groups and launches, with the plain
+// decode of the cache type where nothing is shared or no kernel serves spans.
+pa_status decode_grouped(const char* fn, void* out, const void* q, const void* k_cache,
+                         const void* v_cache, const int32_t* block_tables, int max_blocks_per_seq,
+                         const int32_t* context_lens, const int32_t* group_start,
+                         const int32_t* shared_lens, int num_groups, int max_group_size,
+                         int max_shared_len, int num_seqs, int num_heads, int num_kv_heads,
+                         int head_size, int block_size, int num_blocks, float scale,
+                         pa_dtype dtype, bool fp8, float k_scale, float v_scale,
+                         int partition_size, int max_context_len, void* workspace,
+                         size_t workspace_bytes_in, void* stream) {
   if (partition_size == 0 && num_heads > 0 && num_kv_heads > 0)   // as pa_decode
     partition_size =
         auto_partition(num_seqs, num_heads, num_kv_heads, head_size, dtype, max_context_len);
+  auto plain = [&]() {
+    return fp8 ? pa_decode_fp8(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                               context_lens, num_seqs, num_heads, num_kv_heads, head_size,
+                               block_size, num_blocks, scale, dtype, k_scale, v_scale,
+                               partition_size, max_context_len, workspace, workspace_bytes_in,
+                               stream)
+               : pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                           context_lens, num_seqs, num_heads, num_kv_heads, head_size, block_size,
+                           num_blocks, scale, dtype, partition_size, max_context_len, workspace,
+                           workspace_bytes_in, stream);
+  };
   const int P = resolve_partition(partition_size);
   if (num_groups < 0 || max_shared_len < 0 || max_group_size < 0)
     return pa::fail(PA_ERR_INVALID, "%s: negative group count or size", fn);
@@ -713,18 +727,20 @@ extern "C" pa_status pa_decode_grouped(void* out, const void* q, const void* k_c
       (!group_start || !shared_lens || max_group_size < 1 || max_group_size > num_seqs))
     return pa::fail(PA_ERR_INVALID, "%s: group_start / shared_lens / max_group_size missing", fn);
   const int64_t NPg = P > 0 ? grouped_span_partitions(max_shared_len, P) : 0;
-  if (num_groups == 0 || NPg == 0)   // nothing shared: the plain decode
-    return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
-                     num_seqs, num_heads, num_kv_heads, head_size, block_size, num_blocks, scale,
-                     dtype, partition_size, max_context_len, workspace, workspace_bytes_in, stream);
-  // the checks of pa_decode, with the workspace sized for the grouped layout
+  if (num_groups == 0 || NPg == 0) return plain();   // nothing shared
+  // the checks of the plain decode, with the workspace sized for the grouped layout
   pa::DecodeArgs a;
   const size_t need = pa_decode_grouped_workspace_bytes(num_seqs, num_heads, head_size,
                                                         max_context_len, max_shared_len, P);
-  pa_status st = check_decode_full(fn, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
-                                   context_lens, num_seqs, num_heads, num_kv_heads, head_size,
-                                   block_size, num_blocks, scale, dtype, partition_size,
-                                   max_context_len, workspace, workspace_bytes_in, &a);
+  pa_status st =
+      fp8 ? check_decode_fp8(fn, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                             context_lens, num_seqs, num_heads, num_kv_heads, head_size,
+                             block_size, num_blocks, scale, dtype, k_scale, v_scale,
+                             partition_size, max_context_len, workspace, workspace_bytes_in, &a)
+          : check_decode_full(fn, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                              context_lens, num_seqs, num_heads, num_kv_heads, head_size,
+                              block_size, num_blocks, scale, dtype, partition_size,
+                              max_context_len, workspace, workspace_bytes_in, &a);
   if (st != PA_OK) return st;
   if (!workspace || workspace_bytes_in < need || !pa::aligned16(workspace))
     return pa::fail(PA_ERR_INVALID, "%s: a 16-byte aligned workspace of %zu bytes is needed", fn,
@@ -734,10 +750,8 @@ extern "C" pa_status pa_decode_grouped(void* out, const void* q, const void* k_c
   if ((reinterpret_cast<uintptr_t>(group_start) & 3u) || (reinterpret_cast<uintptr_t>(shared_lens) & 3u))
     return pa::fail(PA_ERR_INVALID, "%s: group_start / shared_lens must be 4-byte aligned", fn);
   a.workspace = static_cast<float*>(workspace);
-  if (!pa::decode_group_tc_supported(a))   // same result without the sharing
-    return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
-                     num_seqs, num_heads, num_kv_heads, head_size, block_size, num_blocks, scale,
-                     dtype, partition_size, max_context_len, workspace, workspace_bytes_in, stream);
+  if (!(fp8 ? pa::decode_group_tc8_supported(a) : pa::decode_group_tc_supported(a)))
+    return plain();   // same result without the sharing
   const int G = num_heads / num_kv_heads;
   const int64_t member_runs = (max_group_size + (16 / G) - 1) / (16 / G);
   if (static_cast<int64_t>(num_groups) * member_runs + num_seqs > 0x7fffffff)
@@ -762,7 +776,10 @@ extern "C" pa_status pa_decode_grouped(void* out, const void* q, const void* k_c
     if (cudaEventRecord(aux->fork, st_main) != cudaSuccess ||
         cudaStreamWaitEvent(aux->stream, aux->fork, 0) != cudaSuccess)
       return pa::fail(PA_ERR_CUDA, "%s: fork to the auxiliary stream failed", fn);
-    st = launch_status(fn, pa::launch_decode_group_tc(a, status, aux->stream), 1);
+    st = launch_status(fn,
+                       fp8 ? pa::launch_decode_group_tc8(a, status, aux->stream)
+                           : pa::launch_decode_group_tc(a, status, aux->stream),
+                       1);
     const pa_status st_rest = launch_status(fn, launch_partitions(a, status, stream), 1);
     // join, whatever happened, so that the caller's stream never runs ahead
     // of work left on the auxiliary one
@@ -773,4 +790,41 @@ extern "C" pa_status pa_decode_grouped(void* out, const void* q, const void* k_c
     if (!joined) return pa::fail(PA_ERR_CUDA, "%s: join with the auxiliary stream failed", fn);
   }
   return launch_status(fn, pa::launch_decode_reduce(a, status, stream), 1);
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode_grouped(void* out, const void* q, const void* k_cache,
+                                       const void* v_cache, const int32_t* block_tables,
+                                       int max_blocks_per_seq, const int32_t* context_lens,
+                                       const int32_t* group_start, const int32_t* shared_lens,
+                                       int num_groups, int max_group_size, int max_shared_len,
+                                       int num_seqs, int num_heads, int num_kv_heads,
+                                       int head_size, int block_size, int num_blocks,
+                                       float scale, pa_dtype dtype, int partition_size,
+                                       int max_context_len, void* workspace,
+                                       size_t workspace_bytes_in, void* stream) {
+  return decode_grouped("pa_decode_grouped", out, q, k_cache, v_cache, block_tables,
+                        max_blocks_per_seq, context_lens, group_start, shared_lens, num_groups,
+                        max_group_size, max_shared_len, num_seqs, num_heads, num_kv_heads,
+                        head_size, block_size, num_blocks, scale, dtype, false, 1.f, 1.f,
+                        partition_size, max_context_len, workspace, workspace_bytes_in, stream);
+}
+
+extern "C" pa_status pa_decode_grouped_fp8(void* out, const void* q, const void* k_cache,
+                                           const void* v_cache, const int32_t* block_tables,
+                                           int max_blocks_per_seq, const int32_t* context_lens,
+                                           const int32_t* group_start, const int32_t* shared_lens,
+                                           int num_groups, int max_group_size,
+                                           int max_shared_len, int num_seqs, int num_heads,
+                                           int num_kv_heads, int head_size, int block_size,
+                                           int num_blocks, float scale, pa_dtype dtype,
+                                           float k_scale, float v_scale, int partition_size,
+                                           int max_context_len, void* workspace,
+                                           size_t workspace_bytes_in, void* stream) {
+  return decode_grouped("pa_decode_grouped_fp8", out, q, k_cache, v_cache, block_tables,
+                        max_blocks_per_seq, context_lens, group_start, shared_lens, num_groups,
+                        max_group_size, max_shared_len, num_seqs, num_heads, num_kv_heads,
+                        head_size, block_size, num_blocks, scale, dtype, true, k_scale, v_scale,
+                        partition_size, max_context_len, workspace, workspace_bytes_in, stream);
 }

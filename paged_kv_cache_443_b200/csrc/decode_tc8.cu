@@ -146,6 +146,17 @@ struct Tc8Params {
   int parts_per_cta;  // consecutive partitions one CTA streams through
   float scale_log2;  // scale * log2(e) * k_scale
   float v_scale;
+  // Shared-prefix groups (pa_decode_grouped_fp8), as in decode_tc.cu:
+  // seq_shift[b] leading tokens of sequence b are its group's shared span
+  // (nullable = 0).  NQ = 1: a CTA serves sequence blockIdx.x past its shift,
+  // partials from workspace slot slot_base.  NQ > 1 (group_start set): a CTA
+  // serves the shared span of group blockIdx.x / q_groups for NQ of its
+  // members (column = (member, head)), partials from slot 0.
+  const int32_t* seq_shift;
+  const int32_t* group_start;
+  int slot_base;
+  int total_q;       // num_seqs
+  int q_groups;      // CTAs per group along x (members / NQ, rounded up)
 };
 
 // Four E4M3 codes (one 32-bit word, code i in byte i) -> two f16x2 words
@@ -169,7 +180,9 @@ __device__ __forceinline__ float2 from_e4m3x2(uint32_t c) {
   return __half22float2(*reinterpret_cast<const __half2*>(&lo));
 }
 
-template <typename T, int G, typename Y>
+// NQ = 1 is the decode (one sequence per CTA, its G heads the columns); NQ > 1
+// serves a group's shared span for NQ members at once (G * NQ <= 16 columns).
+template <typename T, int G, typename Y, int NQ = 1>
 __global__ void __launch_bounds__(THREADS, Y::CTAS_PER_SM)
     decode_partition_tc8_kernel(const Tc8Params p, const __grid_constant__ CUtensorMap tmap_k,
                                 const __grid_constant__ CUtensorMap tmap_v) {
@@ -201,23 +214,72 @@ __global__ void __launch_bounds__(THREADS, Y::CTAS_PER_SM)
   // a CTA covers parts_per_cta consecutive partitions with one softmax (as in
   // decode_tc.cu): its partial goes to the first one's slot, the others' slots
   // get empty partials (max -inf, sum 0, output 0), which the reduce weighs by 0
-  const int b = blockIdx.x, g = blockIdx.y, part = blockIdx.z * p.parts_per_cta;
+  constexpr bool grouped = NQ > 1;
+  constexpr int NC = G * NQ;                // S / O columns in use: (member, head)
+  static_assert(NC <= NPAD, "members x heads must fit the MMA's N");
+  int b = blockIdx.x;
+  const int g = blockIdx.y, part = blockIdx.z * p.parts_per_cta;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   grid_dependency_wait();
   allow_dependents();
-  int L = p.context_lens[b];
+  const int bs = p.block_size;
+  // this CTA's query rows: sequences q0 .. q0 + Qb - 1 (columns h / G)
+  int q0 = b, Qb = 1;
+  int L = 0, shift = 0;
+  if constexpr (grouped) {
+    const int grp = blockIdx.x / p.q_groups;
+    const int gs = p.group_start[grp], ge = p.group_start[grp + 1];
+    if (gs < 0 || ge < gs || ge > p.total_q) {
+      if (threadIdx.x == 0 && blockIdx.z == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
+      return;
+    }
+    if (gs == ge) return;
+    if (ge - gs > p.q_groups * NQ && blockIdx.x % p.q_groups == 0 && threadIdx.x == 0 &&
+        blockIdx.z == 0 && g == 0)
+      atomicOr(p.status, PA_DEVERR_CONTEXT);    // more members than max_group_size
+    const int m0 = gs + (blockIdx.x % p.q_groups) * NQ;
+    Qb = min(NQ, ge - m0);
+    if (Qb <= 0) return;
+    // every member attends to the whole shared span [0, S) of the first
+    // member's table
+    const int S = p.seq_shift[gs];
+    bool bad = S < 0 || S % bs != 0 || S > p.context_lens[gs];
+    for (int m = m0; m < m0 + Qb; ++m) bad |= p.seq_shift[m] != S || p.context_lens[m] < S;
+    if (bad) {
+      if (threadIdx.x == 0 && blockIdx.z == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
+      return;
+    }
+    b = gs;
+    q0 = m0;
+    L = S;
+  } else {
+    L = p.context_lens[b];
+  }
   const int P = p.partition_size;
-  int64_t cap = p.max_blocks * p.block_size;
-  const int64_t grid_cap = static_cast<int64_t>(p.num_partitions) * P;
-  cap = cap < grid_cap ? cap : grid_cap;
+  const int64_t cap = p.max_blocks * p.block_size;
   if (L < 0 || L > cap) {
     if (threadIdx.x == 0 && part == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
     L = L < 0 ? 0 : static_cast<int>(cap);
   }
+  if (!grouped && p.seq_shift != nullptr) {
+    // the tokens past the sequence's shared span (its group serves the span)
+    shift = p.seq_shift[b];
+    if (shift < 0 || shift % bs != 0 || shift > L) {
+      if (threadIdx.x == 0 && part == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
+      shift = 0;
+    }
+    L -= shift;
+  }
+  const int slot0 = grouped ? 0 : p.slot_base;          // this CTA's first workspace slot
+  const int64_t grid_cap = static_cast<int64_t>(p.num_partitions - slot0) * P;
+  if (L > grid_cap) {
+    if (threadIdx.x == 0 && part == 0 && g == 0) atomicOr(p.status, PA_DEVERR_CONTEXT);
+    L = static_cast<int>(grid_cap);
+  }
   const int start = part * P;
   if (L == 0) {
-    if (part == 0) {
+    if (!grouped && part == 0 && shift == 0) {
       T* o = static_cast<T*>(p.out) + (static_cast<int64_t>(b) * p.Hq + g * G) * DH;
       for (int i = threadIdx.x; i < G * DH; i += THREADS) o[i] = Elem<T>::from_float(0.f);
     }
@@ -227,13 +289,14 @@ __global__ void __launch_bounds__(THREADS, Y::CTAS_PER_SM)
   const int end = static_cast<int>(
       min(static_cast<int64_t>(L), start + static_cast<int64_t>(P) * p.parts_per_cta));
   const int n_tiles = (end - start + TOK - 1) / TOK;
-  const bool single = (L <= P);
+  // the output directly, or partials for the reduce (always for a group's span
+  // and for a sequence whose first tokens its group served)
+  const bool single = (L <= P) && !grouped && shift == 0;
   const int n_slots = min(p.parts_per_cta, (L + P - 1) / P - part);   // partials this CTA writes
 
-  const int bs = p.block_size;
   const int first_blk = start / bs;
   const int last_blk = (end + bs - 1) / bs;
-  const int32_t* trow = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
+  const int32_t* trow = p.block_tables + static_cast<int64_t>(b) * p.max_blocks + shift / bs;
   if (threadIdx.x == 0) {
     for (int s = 0; s < SLOTS; ++s) {
       mbar_init(&kr_full[s], 1);
@@ -316,16 +379,17 @@ __global__ void __launch_bounds__(THREADS, Y::CTAS_PER_SM)
   }
 
   if (warp >= 2) {
-    // Query terms: thread t covers head h = t / 8 and its codes 16c..16c+15
-    // (c = t % 8); a head's 8 threads are consecutive lanes.  P buffers zeroed.
+    // Query terms: thread t covers column h = t / 8 (query row q0 + h / G,
+    // head h % G) and its codes 16c..16c+15 (c = t % 8); a column's 8 threads
+    // are consecutive lanes.  P buffers zeroed.
     const int t = threadIdx.x - 64;
     const int h = t >> 3, c = t & 7;
     float f[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) f[e] = 0.f;
-    if (h < G) {
-      const T* src =
-          static_cast<const T*>(p.q) + (static_cast<int64_t>(b) * p.Hq + g * G + h) * DH + c * 16;
+    if (h < NC && h / G < Qb) {
+      const T* src = static_cast<const T*>(p.q) +
+                     ((static_cast<int64_t>(q0) + h / G) * p.Hq + g * G + h % G) * DH + c * 16;
       Elem<T>::unpack(__ldg(reinterpret_cast<const uint4*>(src)), f);
       Elem<T>::unpack(__ldg(reinterpret_cast<const uint4*>(src + 8)), f + 8);
     }
@@ -427,9 +491,9 @@ __global__ void __launch_bounds__(THREADS, Y::CTAS_PER_SM)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    float m_run[G], l_part[G], sc[G];
+    float m_run[NC], l_part[NC], sc[NC];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
+    for (int h = 0; h < NC; ++h) {
       m_run[h] = -INFINITY;
       l_part[h] = 0.f;
       sc[h] = p.scale_log2 * qs[h];
@@ -449,7 +513,7 @@ __global__ void __launch_bounds__(THREADS, Y::CTAS_PER_SM)
       tc_fence_before();
       __syncwarp();
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
+      for (int h = 0; h < NC; ++h) {
         float x = l_part[h];
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(FULL, x, off);
@@ -458,20 +522,21 @@ __global__ void __launch_bounds__(THREADS, Y::CTAS_PER_SM)
       named_sync(1, 128);
       if (lane == 0) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) red[quad * NPAD + h] = l_part[h];
+        for (int h = 0; h < NC; ++h) red[quad * NPAD + h] = l_part[h];
       }
       named_sync(1, 128);
       if (ok) {
         const float oscale = p.v_scale * P_DOWN;
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
+        for (int h = 0; h < NC; ++h) {
+          if (h / G >= Qb) continue;
           const float Ls = red[h] + red[NPAD + h] + red[2 * NPAD + h] + red[3 * NPAD + h];
           const float O = o[h] * oscale;
-          const int64_t hq = static_cast<int64_t>(b) * p.Hq + g * G + h;
+          const int64_t hq = (static_cast<int64_t>(q0) + h / G) * p.Hq + g * G + h % G;
           if (single) {
             static_cast<T*>(p.out)[hq * DH + r] = Elem<T>::from_float(O / Ls);
           } else {
-            const int64_t slot = hq * p.num_partitions + part;
+            const int64_t slot = hq * p.num_partitions + slot0 + part;
             p.ws_o[slot * DH + r] = O;
             if (r == 0) {
               p.ws_m[slot] = m_run[h];
@@ -502,25 +567,25 @@ __global__ void __launch_bounds__(THREADS, Y::CTAS_PER_SM)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[i & 1]);
-      float s[G];
+      float s[NC];
       bool need = false;
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        s[h] = valid ? sv[h] * sc[h] : -INFINITY;
+      for (int h = 0; h < NC; ++h) {
+        s[h] = valid && h / G < Qb ? sv[h] * sc[h] : -INFINITY;
         need |= s[h] > m_run[h] + RESCALE_THRESHOLD;
       }
       if (bar_or(1, 128, need)) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
+        for (int h = 0; h < NC; ++h) {
           float x = s[h];
 #pragma unroll
           for (int off = 16; off >= 1; off >>= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, off));
           if (lane == 0) red[quad * NPAD + h] = x;
         }
         named_sync(1, 128);
-        float alpha[G];
+        float alpha[NC];
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
+        for (int h = 0; h < NC; ++h) {
           const float tmax =
               fmaxf(fmaxf(red[h], red[NPAD + h]), fmaxf(red[2 * NPAD + h], red[3 * NPAD + h]));
           const float mnew = fmaxf(m_run[h], tmax);
@@ -534,25 +599,25 @@ __global__ void __launch_bounds__(THREADS, Y::CTAS_PER_SM)
           float o[16];
           tmem_ld16(tmem + lane_base + 2 * NPAD, o);
 #pragma unroll
-          for (int h = 0; h < G; ++h) o[h] *= alpha[h];
+          for (int h = 0; h < NC; ++h) o[h] *= alpha[h];
           tmem_st16(tmem + lane_base + 2 * NPAD, o);
         }
       }
-      float pr[G];
+      float pr[NC];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        pr[h] = valid ? exp2f(s[h] - m_run[h]) : 0.f;
+      for (int h = 0; h < NC; ++h) {
+        pr[h] = s[h] != -INFINITY ? exp2f(s[h] - m_run[h]) : 0.f;
         l_part[h] += pr[h];
       }
       if (i >= PBUF) wait(&p_free[i % PBUF], ((i / PBUF) - 1) & 1);
       // P * 2^6 = P1 + P2, two E4M3 codes per head (heads h, h+1 in one pair);
       // token r's 16 head codes of each term are one 16-byte row of the
-      // MN-major P^T operand (heads >= G are 0)
+      // MN-major P^T operand (columns >= NC are 0)
       uint32_t w1[4] = {0u, 0u, 0u, 0u}, w2[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-      for (int h = 0; h < G; h += 2) {
+      for (int h = 0; h < NC; h += 2) {
         const float x0 = pr[h] * P_UP;
-        const float x1 = (h + 1 < G) ? pr[h + 1] * P_UP : 0.f;
+        const float x1 = (h + 1 < NC) ? pr[h + 1] * P_UP : 0.f;
         const uint32_t c1 = to_e4m3x2(x0, x1);
         const float2 d1 = from_e4m3x2(c1);
         const uint32_t c2 = to_e4m3x2(x0 - d1.x, x1 - d1.y);
@@ -611,23 +676,35 @@ int sm_count8() {
 // and still leaves at least 8 CTAs per SM (a tile of E4M3 codes is half the
 // bytes of a 16-bit one, so a CTA streams longer before its fixed costs are
 // paid back; two partitions of 2048 were slower than one).
-int tc8_parts_per_cta(const DecodeArgs& a) {
-  if (a.partition_size >= kStreamBelow) return 1;
+// rows: CTAs along x and y; other_ctas: CTAs of a kernel running beside it
+// (the rest of a grouped decode, for the groups' spans).
+int tc8_parts_per_cta(int64_t rows, int partition_size, int n_parts, int64_t other_ctas) {
+  if (partition_size >= kStreamBelow || n_parts <= 0) return 1;
   const int64_t want = 8ll * sm_count8();
   for (int c : {8, 4, 2}) {
-    const int64_t ctas = static_cast<int64_t>(a.num_seqs) * a.Hkv * ((a.num_partitions + c - 1) / c);
-    if (static_cast<int64_t>(a.partition_size) * c <= kMaxSpan && a.num_partitions >= c && ctas >= want)
+    const int64_t ctas = rows * ((n_parts + c - 1) / c) + other_ctas;
+    if (static_cast<int64_t>(partition_size) * c <= kMaxSpan && n_parts >= c && ctas >= want)
       return c;
   }
   return 1;
 }
 
-template <typename T, int G>
+// NQ = 1: the decode, or the rest of every sequence past its shift (partials
+// from a.slot_base).  NQ = 16 / G: the groups' shared spans, one CTA per
+// (group, run of NQ members, kv head, run of span partitions), partials into
+// slots [0, a.slot_base) of every member's row.
+template <typename T, int G, int NQ>
 cudaError_t launch_tc8_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
   using Y = typename std::conditional<std::is_same<T, __nv_bfloat16>::value, LayBF16, LayF16>::type;
   constexpr int SMEM_BYTES = Y::SMEM_BYTES;
-  const int ppc = tc8_parts_per_cta(a);
-  auto kern = decode_partition_tc8_kernel<T, G, Y>;
+  constexpr bool grouped = NQ > 1;
+  const int q_groups = grouped ? (a.max_group_size + NQ - 1) / NQ : 1;
+  const int64_t xs = grouped ? static_cast<int64_t>(a.num_groups) * q_groups : a.num_seqs;
+  const int n_parts = grouped ? a.slot_base : a.num_partitions - a.slot_base;
+  int64_t other = 0;      // the rest's CTAs next to the spans: one per (sequence, head, partition)
+  if (grouped) other = static_cast<int64_t>(a.num_seqs) * a.Hkv * (a.num_partitions - a.slot_base);
+  const int ppc = tc8_parts_per_cta(xs * a.Hkv, a.partition_size, n_parts, other);
+  auto kern = decode_partition_tc8_kernel<T, G, Y, NQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // each cache [NB][Hkv][bs][128] as rows of 128 codes; a box is the bs rows of
@@ -660,7 +737,13 @@ cudaError_t launch_tc8_t(const DecodeArgs& a, unsigned int* status, cudaStream_t
   p.parts_per_cta = ppc;
   p.scale_log2 = a.scale * 1.4426950408889634f * a.k_scale;
   p.v_scale = a.v_scale;
-  dim3 grid(a.num_seqs, a.Hkv, (a.num_partitions + p.parts_per_cta - 1) / p.parts_per_cta);
+  p.seq_shift = a.seq_shift;
+  p.group_start = grouped ? a.group_start : nullptr;
+  p.slot_base = grouped ? 0 : a.slot_base;
+  p.total_q = a.num_seqs;
+  p.q_groups = q_groups;
+  if (xs <= 0 || xs > 0x7fffffff) return cudaErrorInvalidValue;
+  dim3 grid(static_cast<unsigned>(xs), a.Hkv, (n_parts + ppc - 1) / ppc);
   return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
 }
 
@@ -678,10 +761,38 @@ int launch_decode_partitions_tc8(const DecodeArgs& a, unsigned int* status, void
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int G = a.Hq / a.Hkv;
   if (a.dtype == PA_BF16) {
-    return G == 8 ? launch_tc8_t<__nv_bfloat16, 8>(a, status, st)
-                  : launch_tc8_t<__nv_bfloat16, 4>(a, status, st);
+    return G == 8 ? launch_tc8_t<__nv_bfloat16, 8, 1>(a, status, st)
+                  : launch_tc8_t<__nv_bfloat16, 4, 1>(a, status, st);
   }
-  return G == 8 ? launch_tc8_t<__half, 8>(a, status, st) : launch_tc8_t<__half, 4>(a, status, st);
+  return G == 8 ? launch_tc8_t<__half, 8, 1>(a, status, st)
+                : launch_tc8_t<__half, 4, 1>(a, status, st);
+}
+
+bool decode_group_tc8_supported(const DecodeArgs& a) {
+  const int G = a.Hkv > 0 ? a.Hq / a.Hkv : 0;
+  return a.kv_dtype == PA_FP8_E4M3 && (a.dtype == PA_F16 || a.dtype == PA_BF16) && a.D == DH &&
+         (G == 1 || G == 2 || G == 4 || G == 8) && a.partition_size % TOK == 0 &&
+         static_cast<int64_t>(a.num_blocks) * a.Hkv * a.block_size < (int64_t(1) << 31) &&
+         tmap_available();
+}
+
+int launch_decode_group_tc8(const DecodeArgs& a, unsigned int* status, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int G = a.Hq / a.Hkv;
+  if (a.dtype == PA_BF16) {
+    switch (G) {
+      case 1: return launch_tc8_t<__nv_bfloat16, 1, 16>(a, status, st);
+      case 2: return launch_tc8_t<__nv_bfloat16, 2, 8>(a, status, st);
+      case 4: return launch_tc8_t<__nv_bfloat16, 4, 4>(a, status, st);
+      default: return launch_tc8_t<__nv_bfloat16, 8, 2>(a, status, st);
+    }
+  }
+  switch (G) {
+    case 1: return launch_tc8_t<__half, 1, 16>(a, status, st);
+    case 2: return launch_tc8_t<__half, 2, 8>(a, status, st);
+    case 4: return launch_tc8_t<__half, 4, 4>(a, status, st);
+    default: return launch_tc8_t<__half, 8, 2>(a, status, st);
+  }
 }
 
 }  // namespace pa

@@ -93,6 +93,9 @@ int launch_decode_group_tc(const DecodeArgs& a, unsigned int* status, void* stre
 // multiple of 128.
 bool decode_tc8_supported(const DecodeArgs& a);  // needs tmap_available()
 int launch_decode_partitions_tc8(const DecodeArgs& a, unsigned int* status, void* stream);
+// The groups' shared spans over an E4M3 cache (pa_decode_grouped_fp8), G = 1, 2, 4, 8.
+bool decode_group_tc8_supported(const DecodeArgs& a);  // needs tmap_available()
+int launch_decode_group_tc8(const DecodeArgs& a, unsigned int* status, void* stream);
 // A TMA tensor map of 16-bit elements (bytes for PA_FP8_E4M3) with the 128-byte swizzle: `rank` dims
 // (innermost first), byte strides of dims 1..rank-1, a box; `map` points at a
 // CUtensorMap.  False if encoding fails.

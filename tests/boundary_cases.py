@@ -179,17 +179,20 @@ class GroupCase:
     prefix: int = 1024
     suffix_hi: int = 1800
     spike_every: int = 1
+    fp8: bool = False          # E4M3 cache (pa_decode_grouped_fp8)
 
     def spec(self) -> W.Spec:
         common = dict(name=self.name, dtype=self.dtype, Hq=self.G * self.Hkv, Hkv=self.Hkv, D=128,
                       block_size=self.bs, seed=hash_seed(self.name), partition_size=self.P)
         if self.kind == "parallel_sampling":
-            return W.Spec(kind=self.kind, num_seqs=self.prompts * self.samples,
-                          num_prompts=self.prompts, samples_per_prompt=self.samples,
-                          prompt_lo=self.prompt_lo, prompt_hi=self.prompt_hi, div_lo=1,
-                          div_hi=self.div_hi, **common)
-        return W.Spec(kind=self.kind, num_seqs=self.requests, prefix_len=self.prefix, suffix_lo=1,
-                      suffix_hi=self.suffix_hi, **common)
+            s = W.Spec(kind=self.kind, num_seqs=self.prompts * self.samples,
+                       num_prompts=self.prompts, samples_per_prompt=self.samples,
+                       prompt_lo=self.prompt_lo, prompt_hi=self.prompt_hi, div_lo=1,
+                       div_hi=self.div_hi, **common)
+        else:
+            s = W.Spec(kind=self.kind, num_seqs=self.requests, prefix_len=self.prefix,
+                       suffix_lo=1, suffix_hi=self.suffix_hi, **common)
+        return W.fp8(s) if self.fp8 else s
 
     def scenario(self) -> W.Scenario:
         sc = W.scenario(self.spec())
@@ -218,4 +221,16 @@ GROUPED = [
     # per CTA (>= 8 CTAs per SM)
     GroupCase("g_lp_g4_stream", "shared_prefix", "bf16", 4, 16, 128, Hkv=4, requests=300,
               prefix=1024, suffix_hi=1800, spike_every=10),
+    # E4M3 caches: the spans on the tcgen05 E4M3 kernel with (member, head)
+    # columns; the rest on the E4M3 tensor-core kernel (G = 4, 8) or the
+    # CUDA-core kernel (G = 1, 2), each past its shift
+    GroupCase("g_e4m3_ps_g1_p128", "parallel_sampling", "bf16", 1, 16, 128, Hkv=4, fp8=True),
+    GroupCase("g_e4m3_ps_g2_p256", "parallel_sampling", "f16", 2, 16, 256, Hkv=2, fp8=True),
+    GroupCase("g_e4m3_ps_g1_20samples", "parallel_sampling", "f16", 1, 16, 512, Hkv=2,
+              prompts=2, samples=20, fp8=True),
+    GroupCase("g_e4m3_lp_g4_p512", "shared_prefix", "bf16", 4, 16, 512, fp8=True),
+    GroupCase("g_e4m3_lp_g4_bs32_p128", "shared_prefix", "f16", 4, 32, 128, fp8=True),
+    GroupCase("g_e4m3_lp_g8_bs8_p256", "shared_prefix", "bf16", 8, 8, 256, fp8=True),
+    GroupCase("g_e4m3_lp_g4_stream", "shared_prefix", "bf16", 4, 16, 128, Hkv=4, requests=300,
+              prefix=1024, suffix_hi=1800, spike_every=10, fp8=True),
 ]

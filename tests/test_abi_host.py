@@ -337,6 +337,22 @@ def test_grouped_decode_rejects_bad_arguments(L):
     assert call(max_group_size=0) == pk.PA_ERR_INVALID
     assert call() == pk.PA_ERR_INVALID                        # no workspace
     assert pk.pa_launch_count() == n0
+    # the E4M3 variant checks the same, plus the cache scales and the query type
+    def call8(q_dtype=pk.PA_BF16, k_scale=0.5, **kw):
+        a = dict(good, **kw)
+        fake = C.c_void_p(256)
+        return L.pa_decode_grouped_fp8(fake, fake, fake, fake, fake, 8, fake, fake, fake,
+                                       a["num_groups"], a["max_group_size"],
+                                       a["max_shared_len"], a["B"], a["Hq"], a["Hkv"], a["D"],
+                                       a["bs"], 100, 0.1, q_dtype, k_scale, 0.25, a["P"],
+                                       a["max_ctx"], None, 0, None)
+
+    assert call8(max_shared_len=8) == pk.PA_ERR_INVALID
+    assert call8(num_groups=3) == pk.PA_ERR_INVALID
+    assert call8(k_scale=0.0) == pk.PA_ERR_INVALID            # scales must be positive
+    assert call8(q_dtype=pk.PA_FP8_E4M3) == pk.PA_ERR_UNSUPPORTED  # queries are not codes
+    assert call8() == pk.PA_ERR_INVALID                       # no workspace
+    assert pk.pa_launch_count() == n0
     need = L.pa_decode_grouped_workspace_bytes(2, 8, 128, 64, 16, 32)
     # slots: ceil(16/32) = 1 for the span + ceil(64/32) = 2 for the rest
     assert need == -(-2 * 8 * 3 * 130 * 4 // 256) * 256

@@ -121,10 +121,11 @@ int pa_decode_default_partition_size(void);
 
 /*
  * The partition length pa_decode uses when it is given partition_size = 0
- * (tokens; 512, 1024, 2048 or 4096).  With 4 or 8 query heads per kv head in
- * fp16/bf16 and head size 128 (the tensor-core kernel) it is the longest of
- * 4096 / 2048 / 1024 that still gives num_seqs * num_kv_heads *
- * ceil(max_context_len / P) >= 8 * (number of SMs) CTAs; otherwise the default.  Pass it explicitly to
+ * (tokens; 512, 1024, 2048 or 4096): the longest P that still gives
+ * num_seqs * num_kv_heads * ceil(max_context_len / P) >= 8 * (number of SMs)
+ * CTAs, among 4096 / 2048 / 1024 with 4 or 8 query heads per kv head in
+ * fp16/bf16 and head size 128 (the tensor-core kernel), among 1024 otherwise;
+ * the default (512) when none does.  Pass it explicitly to
  * pa_decode_partitions / pa_decode_reduce to reproduce pa_decode's automatic
  * choice.  Returns -1 for invalid arguments.
  */

@@ -39,18 +39,20 @@ int num_sms() {
 }
 
 // Partition length pa_decode (and pa_decode_fp8) use for partition_size = 0.
-// The tensor-core kernels (fp16/bf16 queries, head size 128, 4 or 8 query heads
-// per kv head; 16-bit or E4M3 caches) pay a fixed set-up and drain per CTA, so
-// it takes the longest of 4096 / 2048 / 1024 tokens that still gives at least
-// ~4 waves of CTAs (2 per SM) at the longest context; everything else keeps
-// the default.
+// Every CTA pays a fixed set-up and pipeline fill, so the partitions are as
+// long as still gives at least 8 CTAs per SM at the longest context: for the
+// tensor-core kernels (fp16/bf16 queries, head size 128, 4 or 8 query heads per
+// kv head; 16-bit or E4M3 caches, which also stream several partitions per
+// CTA) the longest of 4096 / 2048 / 1024 tokens; for the CUDA-core kernel 1024
+// (2048 measured slower at opt13b: fewer, longer CTAs leave the last wave
+// thin); else the default.
 int auto_partition(int num_seqs, int num_heads, int num_kv_heads, int head_size, pa_dtype dtype,
                    int max_context_len) {
   const int G = num_kv_heads > 0 ? num_heads / num_kv_heads : 0;
   const bool tc = (dtype == PA_F16 || dtype == PA_BF16) && head_size == 128 && (G == 4 || G == 8);
-  if (!tc) return pa::kDefaultPartition;
   const int64_t want = 8ll * num_sms();
   for (int P : {4096, 2048, 1024}) {
+    if (!tc && P > 1024) continue;
     const int64_t ctas = static_cast<int64_t>(num_seqs) * num_kv_heads * num_partitions(max_context_len, P);
     if (ctas >= want) return P;
   }

@@ -130,10 +130,12 @@ def test_auto_partition_size(L):
     assert pk.pa_decode_auto_partition_size(8, 64, 8, 128, bf, 32768) == 1024
     # too few CTAs at long partitions: the default
     assert pk.pa_decode_auto_partition_size(1, 64, 8, 128, bf, 32768) == 512
-    # other paths keep the default
-    assert pk.pa_decode_auto_partition_size(64, 40, 40, 128, pk.PA_F16, 2048) == 512
-    assert pk.pa_decode_auto_partition_size(256, 64, 8, 64, bf, 4096) == 512
-    assert pk.pa_decode_auto_partition_size(256, 64, 8, 128, pk.PA_F32, 4096) == 512
+    # the CUDA-core kernel: 1024 with enough CTAs, else the default
+    assert pk.pa_decode_auto_partition_size(64, 40, 40, 128, pk.PA_F16, 2048) == 1024
+    assert pk.pa_decode_auto_partition_size(64, 40, 40, 128, pk.PA_F16, 8192) == 1024
+    assert pk.pa_decode_auto_partition_size(256, 64, 8, 64, bf, 4096) == 1024
+    assert pk.pa_decode_auto_partition_size(256, 64, 8, 128, pk.PA_F32, 4096) == 1024
+    assert pk.pa_decode_auto_partition_size(4, 40, 40, 128, pk.PA_F16, 2048) == 512
     assert pk.pa_decode_auto_partition_size(4, 6, 4, 128, bf, 100) == -1
     # the same rule over an E4M3 cache
     a8 = pk.pa_decode_fp8_auto_partition_size
@@ -141,7 +143,8 @@ def test_auto_partition_size(L):
     assert a8(128, 32, 8, 128, bf, 32768) == 4096
     assert a8(16, 64, 8, 128, bf, 32768) == 2048
     assert a8(1, 64, 8, 128, bf, 32768) == 512
-    assert a8(64, 40, 40, 128, pk.PA_F16, 2048) == 512
+    assert a8(64, 40, 40, 128, pk.PA_F16, 2048) == 1024
+    assert a8(4, 40, 40, 128, pk.PA_F16, 2048) == 512
     assert a8(256, 64, 8, 128, pk.PA_FP8_E4M3, 4096) == -1
     assert a8(4, 6, 4, 128, bf, 100) == -1
     # the default-sized workspace covers the automatic length

@@ -289,8 +289,9 @@ def full_size_check(spec, name):
     from pa_harness import oracle_row_perturbed
     sc = W.scenario(spec)
     seqs = compared_sequences(sc)
-    P = spec.partition_size or 4096
-    sc = W.spike_plan(sc, tuple(sorted({P, 512, 4096})), seed=2, seqs=seqs)
+    # spikes at the edges of every partition length the automatic rule may take
+    P = spec.partition_size
+    sc = W.spike_plan(sc, tuple(sorted({P, 512, 1024, 2048, 4096} - {0})), seed=2, seqs=seqs)
     p, o = build(sc)
     out = run_step(p, spec)
     torch.cuda.synchronize()

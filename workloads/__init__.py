@@ -126,10 +126,10 @@ TINY = Spec("tiny", "f32", 4, 4, 64, 16, "independent", 8, seed=443, num_blocks=
             scale=1.0 / 8, ctx_dist="uniform", ctx_lo=1, ctx_hi=64)
 OPT13B = Spec("opt13b", "f16", 40, 40, 128, 16, "independent", 64, seed=444,
               num_blocks=20000, ctx_dist="lognormal", ctx_median=600.0, ctx_sigma=0.5,
-              ctx_lo=16, ctx_hi=2048)
+              ctx_lo=16, ctx_hi=2048, partition_size=0)
 LLAMA13B_PS = Spec("llama13b_ps", "bf16", 40, 40, 128, 16, "parallel_sampling", 96, seed=445,
                    num_prompts=16, samples_per_prompt=6, prompt_lo=512, prompt_hi=1024,
-                   div_lo=1, div_hi=256)
+                   div_lo=1, div_hi=256, partition_size=0)
 GQA70B = Spec("gqa70b", "bf16", 64, 8, 128, 16, "independent", 256, seed=446,
               ctx_dist="uniform", ctx_lo=256, ctx_hi=4096, partition_size=0)
 LONG_PREFIX = Spec("long_prefix", "bf16", 32, 8, 128, 16, "shared_prefix", 128, seed=447,

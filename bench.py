@@ -309,6 +309,44 @@ def profiled_traffic(workload, kernel, partition_size):
     return None, "no ncu capture of this kernel at this workload and partition length"
 
 
+def record_traffic(csv_path, workload, kernel, partition_size):
+    """Record in profiles/dram_traffic.json the DRAM bytes of one decode call:
+    dram__bytes_read.sum + dram__bytes_write.sum summed over the launches of an
+    ncu CSV (--csv --print-units base) that captured exactly that call's
+    kernels, with the current digest of the kernels' sources."""
+    import csv
+    with open(csv_path, newline="") as f:
+        lines = [ln for ln in f if ln.startswith('"')]   # ncu's own "==PROF==" lines dropped
+    rows = list(csv.DictReader(lines))
+    total, launches = 0.0, set()
+    for r in rows:
+        if r.get("Metric Name") in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            if r.get("Metric Unit") not in ("byte", "bytes"):
+                raise SystemExit(f"{csv_path}: capture with --print-units base (got {r.get('Metric Unit')})")
+            total += float(r["Metric Value"].replace(",", ""))
+            launches.add(r["ID"])
+    if not launches:
+        raise SystemExit(f"{csv_path}: no dram__bytes_* rows")
+    path = os.path.join(ROOT, TRAFFIC_FILE)
+    try:
+        with open(path) as f:
+            data = json.load(f)
+    except (OSError, ValueError):
+        data = {"captures": []}
+    entry = {"workload": workload, "kernel": kernel, "partition_size": int(partition_size),
+             "source_digest": source_digest(KERNEL_SOURCES[kernel]),
+             "dram_bytes_per_launch": int(round(total)),
+             "how": (f"ncu one-pass dram__bytes_read.sum + dram__bytes_write.sum over the "
+                     f"{len(launches)} kernel launches of one call, {os.path.basename(csv_path)}")}
+    data["captures"] = [e for e in data.get("captures", [])
+                        if (e.get("workload"), e.get("kernel"), int(e.get("partition_size", -1)))
+                        != (workload, kernel, int(partition_size))] + [entry]
+    with open(path, "w") as f:
+        json.dump(data, f, indent=1)
+        f.write("\n")
+    return entry
+
+
 def measured_peak_tensor():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -999,7 +1037,16 @@ def main():
     ap.add_argument("--grouped", default="auto", choices=["auto", "on", "off"],
                     help="decode families sharing leading blocks with pa_decode_grouped "
                          "(auto: for parallel-sampling and shared-prefix workloads)")
+    ap.add_argument("--record-traffic", metavar="CSV",
+                    help="no run: record the DRAM bytes of one call from an ncu CSV into "
+                         "profiles/dram_traffic.json for --workload, --traffic-kernel and "
+                         "--partition-size")
+    ap.add_argument("--traffic-kernel", choices=sorted(KERNEL_SOURCES), default="decode_grouped")
     args = ap.parse_args()
+    if args.record_traffic:
+        print(json.dumps(record_traffic(args.record_traffic, args.workload, args.traffic_kernel,
+                                        args.partition_size)))
+        return
     args.warmup = max(3, args.warmup)
     rank, world, _ = dist_env()
 

@@ -92,6 +92,34 @@ def test_profile_digest_gates_traffic(tmp_path, monkeypatch):
     assert bench.profiled_traffic("z", k, 512)[0] is None
 
 
+def test_record_traffic_sums_one_call_and_replaces_its_entry(tmp_path, monkeypatch):
+    import json
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "dram_traffic.json").write_text(json.dumps({"captures": [
+        dict(workload="w", kernel="decode_grouped", partition_size=512, source_digest="old",
+             dram_bytes_per_launch=1),
+        dict(workload="other", kernel="decode_grouped", partition_size=512,
+             source_digest="keep", dram_bytes_per_launch=7)]}))
+    csv_path = tmp_path / "cap.csv"
+    hdr = '"ID","Kernel Name","Metric Name","Metric Unit","Metric Value"\n'
+    rows = ['"0","span","dram__bytes_read.sum","byte","1,000"', '"0","span","dram__bytes_write.sum","byte","24"',
+            '"0","span","gpu__time_duration.sum","nsecond","5"',
+            '"1","rest","dram__bytes_read.sum","byte","2000"', '"1","rest","dram__bytes_write.sum","byte","6"']
+    csv_path.write_text("==PROF== Connected\n" + hdr + "\n".join(rows) + "\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "source_digest", lambda files=None: "new")
+    e = bench.record_traffic(str(csv_path), "w", "decode_grouped", 512)
+    assert e["dram_bytes_per_launch"] == 1000 + 24 + 2000 + 6 and e["source_digest"] == "new"
+    caps = json.loads((prof / "dram_traffic.json").read_text())["captures"]
+    assert sorted(c["workload"] for c in caps) == ["other", "w"]
+    assert bench.profiled_traffic("w", "decode_grouped", 512)[0] == 3030.0
+    # values not in bytes are refused rather than mis-scaled
+    csv_path.write_text(hdr + '"0","span","dram__bytes_read.sum","Mbyte","1.5"\n')
+    with pytest.raises(SystemExit):
+        bench.record_traffic(str(csv_path), "w", "decode_grouped", 512)
+
+
 def test_partition_kernel_choice():
     assert bench.partition_kernel(W.GQA70B, 512) == "decode_partition_tc_kernel"
     assert bench.partition_kernel(W.LONG_PREFIX, 512) == "decode_partition_tc_kernel"

@@ -312,15 +312,26 @@ def profiled_traffic(workload, kernel, partition_size):
 def record_traffic(csv_path, workload, kernel, partition_size):
     """Record in profiles/dram_traffic.json the DRAM bytes of one decode call:
     dram__bytes_read.sum + dram__bytes_write.sum summed over the launches of an
-    ncu CSV (--csv --print-units base) that captured exactly that call's
-    kernels, with the current digest of the kernels' sources."""
+    ncu CSV that captured exactly that call's kernels (a capture's --csv
+    --print-units base log, or the raw page of a report), with the current
+    digest of the kernels' sources."""
     import csv
     with open(csv_path, newline="") as f:
         lines = [ln for ln in f if ln.startswith('"')]   # ncu's own "==PROF==" lines dropped
     rows = list(csv.DictReader(lines))
+    names = ("dram__bytes_read.sum", "dram__bytes_write.sum")
     total, launches = 0.0, set()
+    if rows and "Metric Name" not in rows[0]:
+        # the raw page of a report (ncu -i REP --page raw --csv --print-units base
+        # --metrics ...): one row per launch after a row of units
+        units, rows = rows[0], rows[1:]
+        for n in names:
+            if units.get(n) not in ("byte", "bytes"):
+                raise SystemExit(f"{csv_path}: capture with --print-units base (got {units.get(n)})")
+        rows = [dict(r, **{"Metric Name": n, "Metric Unit": "byte", "Metric Value": r[n]})
+                for r in rows for n in names]
     for r in rows:
-        if r.get("Metric Name") in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+        if r.get("Metric Name") in names:
             if r.get("Metric Unit") not in ("byte", "bytes"):
                 raise SystemExit(f"{csv_path}: capture with --print-units base (got {r.get('Metric Unit')})")
             total += float(r["Metric Value"].replace(",", ""))
@@ -336,7 +347,7 @@ def record_traffic(csv_path, workload, kernel, partition_size):
     entry = {"workload": workload, "kernel": kernel, "partition_size": int(partition_size),
              "source_digest": source_digest(KERNEL_SOURCES[kernel]),
              "dram_bytes_per_launch": int(round(total)),
-             "how": (f"ncu one-pass dram__bytes_read.sum + dram__bytes_write.sum over the "
+             "how": (f"ncu dram__bytes_read.sum + dram__bytes_write.sum over the "
                      f"{len(launches)} kernel launches of one call, {os.path.basename(csv_path)}")}
     data["captures"] = [e for e in data.get("captures", [])
                         if (e.get("workload"), e.get("kernel"), int(e.get("partition_size", -1)))

@@ -114,6 +114,11 @@ def test_record_traffic_sums_one_call_and_replaces_its_entry(tmp_path, monkeypat
     caps = json.loads((prof / "dram_traffic.json").read_text())["captures"]
     assert sorted(c["workload"] for c in caps) == ["other", "w"]
     assert bench.profiled_traffic("w", "decode_grouped", 512)[0] == 3030.0
+    # the raw page of a report: one row per launch after a row of units
+    csv_path.write_text('"ID","Kernel Name","dram__bytes_read.sum","dram__bytes_write.sum"\n'
+                        '"","","byte","byte"\n"0","k","433997568","4872192"\n')
+    e = bench.record_traffic(str(csv_path), "w", "decode_grouped", 1024)
+    assert e["dram_bytes_per_launch"] == 433997568 + 4872192
     # values not in bytes are refused rather than mis-scaled
     csv_path.write_text(hdr + '"0","span","dram__bytes_read.sum","Mbyte","1.5"\n')
     with pytest.raises(SystemExit):

@@ -86,18 +86,20 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 }
 
 // Shared-memory and TMEM layout for N = NP columns (16, or 32 for 32 query
-// tokens x heads).  The 1024-byte aligned part holds a ring of three K/V tiles,
-// the Q^T operand and PBUF P^T buffers of NP columns (two at N = 16; one at
-// N = 32, so that two CTAs still share an SM).  The barriers, the TMEM address
+// tokens x heads) and CTAS CTAs per SM.  The 1024-byte aligned part holds a
+// ring of K/V tiles, the Q^T operand and PBUF P^T buffers of NP columns: for
+// two CTAs per SM three tiles and two P buffers at N = 16, one at N = 32 (so
+// that two CTAs still share an SM); for three CTAs per SM two tiles and one P
+// buffer (72 KB at N = 16).  The barriers, the TMEM address
 // and the 4-warp reduction buffer live in the 1 KB the allocation adds for
 // aligning the base: in front of the aligned part where the base's offset
 // leaves room, behind it otherwise (small_layout).
 // TMEM: S0 [0, NP), S1 [NP, 2NP), O [2NP, 3NP).
-template <int NP>
+template <int NP, int CTAS = 2>
 struct Lay {
   static constexpr int NPAD = NP;
-  static constexpr int SLOTS = 3;
-  static constexpr int PBUF = NP <= 16 ? 2 : 1;
+  static constexpr int SLOTS = CTAS >= 3 ? 2 : 3;
+  static constexpr int PBUF = (NP <= 16 && CTAS < 3) ? 2 : 1;
   static constexpr int OPB_BYTES = 2 * NP * 128;   // Q^T (K-major) or P^T (MN-major): NP x 128 16-bit
   static constexpr int OFF_RING = 0;
   static constexpr int OFF_Q = OFF_RING + SLOTS * SLOT_BYTES;
@@ -111,7 +113,8 @@ struct Lay {
   static constexpr int TMEM_COLS = 3 * NP <= 64 ? 64 : 128;
   // small_layout's placement always fits when these hold
   static_assert(RED_BYTES <= 512 && RED_BYTES + 2 * MISC_BYTES <= 1024, "small buffers");
-  static_assert(2 * (SMEM_BYTES + 1024) <= 228 * 1024, "two CTAs per SM");
+  static_assert(CTAS * (SMEM_BYTES + 1024) <= 228 * 1024, "CTAS CTAs per SM");
+  static_assert(CTAS * TMEM_COLS <= 512, "TMEM of CTAS CTAs");
 };
 
 // Where the small buffers go, given the dynamic allocation's base: f bytes
@@ -119,18 +122,18 @@ struct Lay {
 // The reduction buffer goes in front if it fits there, else behind (1024 - f >
 // 512 >= its size); the barriers take whichever side still has room, which
 // RED_BYTES + 2 * MISC_BYTES <= 1024 guarantees.
-template <int NP>
+template <int NP, int CTAS>
 struct SmemPtrs {
   uint8_t* aligned;
   float* red;
   uint8_t* misc;
 };
-template <int NP>
-__device__ __forceinline__ SmemPtrs<NP> small_layout(uint8_t* raw) {
-  using Y = Lay<NP>;
+template <int NP, int CTAS>
+__device__ __forceinline__ SmemPtrs<NP, CTAS> small_layout(uint8_t* raw) {
+  using Y = Lay<NP, CTAS>;
   const uintptr_t b = reinterpret_cast<uintptr_t>(raw);
   const uint32_t f = static_cast<uint32_t>(((b + 1023) & ~static_cast<uintptr_t>(1023)) - b);
-  SmemPtrs<NP> r;
+  SmemPtrs<NP, CTAS> r;
   r.aligned = raw + f;
   uint8_t* back = r.aligned + Y::ALIGNED_BYTES;
   if (f >= static_cast<uint32_t>(Y::RED_BYTES)) {
@@ -183,16 +186,16 @@ struct TcParams {
 // column c of S / O is query token c / G (one of the sequence's last Qb <= NQ
 // context tokens) with head c % G, and a key counts for it only up to that
 // token's own position.  NQ = 1 is the decode step and compiles as before.
-template <typename T, int G, int NQ = 1, int NP = 16>
-__global__ void __launch_bounds__(THREADS, 2)
+template <typename T, int G, int NQ = 1, int NP = 16, int CTAS = 2>
+__global__ void __launch_bounds__(THREADS, CTAS)
     decode_partition_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmap_k,
                                const __grid_constant__ CUtensorMap tmap_v) {
-  using Y = Lay<NP>;
+  using Y = Lay<NP, CTAS>;
   constexpr int NPAD = NP, SLOTS = Y::SLOTS, PBUF = Y::PBUF, OPB_BYTES = Y::OPB_BYTES;
   constexpr int OFF_RING = Y::OFF_RING, OFF_Q = Y::OFF_Q, OFF_P = Y::OFF_P;
   constexpr int TMEM_COLS = Y::TMEM_COLS;
   extern __shared__ uint8_t smem_raw[];
-  const SmemPtrs<NP> sp = small_layout<NP>(smem_raw);
+  const SmemPtrs<NP, CTAS> sp = small_layout<NP, CTAS>(smem_raw);
   uint8_t* smem = sp.aligned;
   uint8_t* ring = smem + OFF_RING;
   uint8_t* qop = smem + OFF_Q;
@@ -709,13 +712,13 @@ cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t 
 // member's row.  (The kernel can also take the rest of every sequence in the
 // same grid, blockIdx.x >= span_x; launched alone, the rest keeps its own
 // kernel and N, which measured faster.)
-template <typename T, int G>
+template <typename T, int G, int CTAS = 2>
 cudaError_t launch_group_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
   constexpr int NQ = 16 / G;
-  auto kern = decode_partition_tc_kernel<T, G, NQ>;
-  constexpr int SMEM_BYTES = Lay<16>::SMEM_BYTES;
+  auto kern = decode_partition_tc_kernel<T, G, NQ, 16, CTAS>;
+  constexpr int SMEM_BYTES = Lay<16, CTAS>::SMEM_BYTES;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  if (e == cudaSuccess)   // all of the SM's 228 KB as shared memory: two CTAs of up to 113 KB
+  if (e == cudaSuccess)   // all of the SM's 228 KB as shared memory
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   CUtensorMap mk, mv;
@@ -932,20 +935,25 @@ bool decode_group_tc_supported(const DecodeArgs& a) {
          encode_fn() != nullptr;
 }
 
+// G = 1, 2 (families of parallel samples: each span is a prompt's own blocks,
+// read from HBM by few CTAs of a few tiles each) take the layout with rings of
+// two tiles and one P buffer, three CTAs per SM: more spans in flight at once
+// (llama13b_ps decode 131 -> 127 us).  G = 4, 8 keep three tiles and two CTAs
+// per SM (a long prefix served from L2: 0.5 % faster).
 int launch_decode_group_tc(const DecodeArgs& a, unsigned int* status, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int G = a.Hq / a.Hkv;
   if (a.dtype == PA_BF16) {
     switch (G) {
-      case 1: return launch_group_tc_t<__nv_bfloat16, 1>(a, status, st);
-      case 2: return launch_group_tc_t<__nv_bfloat16, 2>(a, status, st);
+      case 1: return launch_group_tc_t<__nv_bfloat16, 1, 3>(a, status, st);
+      case 2: return launch_group_tc_t<__nv_bfloat16, 2, 3>(a, status, st);
       case 4: return launch_group_tc_t<__nv_bfloat16, 4>(a, status, st);
       default: return launch_group_tc_t<__nv_bfloat16, 8>(a, status, st);
     }
   }
   switch (G) {
-    case 1: return launch_group_tc_t<__half, 1>(a, status, st);
-    case 2: return launch_group_tc_t<__half, 2>(a, status, st);
+    case 1: return launch_group_tc_t<__half, 1, 3>(a, status, st);
+    case 2: return launch_group_tc_t<__half, 2, 3>(a, status, st);
     case 4: return launch_group_tc_t<__half, 4>(a, status, st);
     default: return launch_group_tc_t<__half, 8>(a, status, st);
   }

@@ -17,8 +17,9 @@
 //   * warp 0 is the producer: it reads the block table (32 entries per
 //     coalesced load) and moves each physical (block, kv head) K and V tile --
 //     a contiguous bs*D run -- into shared memory with 1-D bulk copies on the
-//     TMA engine, into a ring of S stages of 32 tokens (about 64 KB in flight per
-//     CTA) tracked by mbarriers with transaction counts;
+//     TMA engine, into a ring of S stages of 32 tokens (32 KB in flight per CTA
+//     for 16-bit caches, six CTAs per SM; 64 KB of E4M3 codes) tracked by
+//     mbarriers with transaction counts;
 //   * NCW consumer warps each own 8 tokens of a stage: q (pre-scaled by
 //     scale*log2 e) sits in registers, a lane owns one 16-byte chunk of a K/V row,
 //     dot products are finished with a butterfly reduce-scatter across the lanes
@@ -60,7 +61,7 @@ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 constexpr float RESCALE_LOG2 = 8.0f;   // raise the running max past 2^8 growth
 
-template <typename T, int D, int G, int NCW>
+template <typename T, int D, int G, int NCW, int BUDGET = 65536>
 struct Cfg {
   static constexpr int ES = sizeof(T);
   // elements a lane loads at once: one 16-byte chunk (8 codes at G > 2, where
@@ -74,7 +75,7 @@ struct Cfg {
   static constexpr int ROW_BYTES = D * ES;
   static constexpr int TILE_BYTES = TOK * ROW_BYTES;  // K (or V) part of a stage
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-  static constexpr int S = cmin(8, cmax(2, 65536 / STAGE_BYTES));
+  static constexpr int S = cmin(8, cmax(2, BUDGET / STAGE_BYTES));   // stages in flight
   static constexpr int NV = G * ITERS;         // partial dots per lane per stage
   static constexpr int NSM = G * TPW;          // scores per warp per stage
   static constexpr int NPASS = (NSM + 31) / 32;
@@ -211,10 +212,10 @@ struct PartitionParams {
   int slot_base;
 };
 
-template <typename TQ, typename TK, int D, int G, int NCW>
-__global__ void __launch_bounds__(Cfg<TK, D, G, NCW>::THREADS)
+template <typename TQ, typename TK, int D, int G, int NCW, int BUDGET>
+__global__ void __launch_bounds__(Cfg<TK, D, G, NCW, BUDGET>::THREADS)
     decode_partition_kernel(const PartitionParams p) {
-  using C = Cfg<TK, D, G, NCW>;
+  using C = Cfg<TK, D, G, NCW, BUDGET>;
   using E = Elem<TK>;
   using EQ = Elem<TQ>;
   constexpr bool kCoded = sizeof(TK) == 1;  // E4M3 codes
@@ -679,11 +680,22 @@ constexpr int consumer_warps() {
   return (sizeof(TK) == 1 && G <= 2) ? 8 : 4;
 }
 
-template <typename TQ, typename TK, int D, int G>
+// Shared memory for the stages in flight: 32 KB for 16-bit and fp32 caches
+// (two 16 KB stages at D = 128, so that six CTAs share an SM; against four
+// stages and three CTAs, the same bytes in flight per SM but twice the
+// independent pipelines: opt13b 0.94 -> 0.96, llama13b_ps' short per-sample
+// rests 0.62 -> 0.68), 64 KB for E4M3 codes (its 288-thread CTAs are held to
+// four per SM by registers anyway, and opt13b_fp8 measured 1.5 % slower).
+template <typename TK>
+constexpr int stage_budget() {
+  return sizeof(TK) == 1 ? 65536 : 32768;
+}
+
+template <typename TQ, typename TK, int D, int G, int BUDGET = stage_budget<TK>()>
 cudaError_t launch_partition_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
   constexpr int NCW = consumer_warps<TK, G>();
-  using C = Cfg<TK, D, G, NCW>;
-  auto kern = decode_partition_kernel<TQ, TK, D, G, NCW>;
+  using C = Cfg<TK, D, G, NCW, BUDGET>;
+  auto kern = decode_partition_kernel<TQ, TK, D, G, NCW, BUDGET>;
   // opt in to > 48 KB of dynamic shared memory (idempotent, cheap)
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;

@@ -712,9 +712,8 @@ cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t 
 // member's row.  (The kernel can also take the rest of every sequence in the
 // same grid, blockIdx.x >= span_x; launched alone, the rest keeps its own
 // kernel and N, which measured faster.)
-template <typename T, int G, int CTAS = 2>
+template <typename T, int G, int CTAS = 2, int NQ = 16 / G>
 cudaError_t launch_group_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
-  constexpr int NQ = 16 / G;
   auto kern = decode_partition_tc_kernel<T, G, NQ, 16, CTAS>;
   constexpr int SMEM_BYTES = Lay<16, CTAS>::SMEM_BYTES;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
@@ -935,6 +934,19 @@ bool decode_group_tc_supported(const DecodeArgs& a) {
          encode_fn() != nullptr;
 }
 
+// Members per span CTA: 16 / G fill the MMA's 16 columns; when every family
+// has at most 8 / G members, 8 / G of them (8 columns in use) halve the
+// softmax's per-column work on every tile at the same CTA count (the MMA still
+// computes 16 columns, which costs nothing that shows).
+template <typename T, int G, int CTAS>
+int launch_group_g(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
+  if constexpr (G <= 4) {
+    if (static_cast<int64_t>(a.max_group_size) * G <= 8)
+      return launch_group_tc_t<T, G, CTAS, 8 / G>(a, status, stream);
+  }
+  return launch_group_tc_t<T, G, CTAS>(a, status, stream);
+}
+
 // G = 1, 2 (families of parallel samples: each span is a prompt's own blocks,
 // read from HBM by few CTAs of a few tiles each) take the layout with rings of
 // two tiles and one P buffer, three CTAs per SM: more spans in flight at once
@@ -945,17 +957,17 @@ int launch_decode_group_tc(const DecodeArgs& a, unsigned int* status, void* stre
   const int G = a.Hq / a.Hkv;
   if (a.dtype == PA_BF16) {
     switch (G) {
-      case 1: return launch_group_tc_t<__nv_bfloat16, 1, 3>(a, status, st);
-      case 2: return launch_group_tc_t<__nv_bfloat16, 2, 3>(a, status, st);
-      case 4: return launch_group_tc_t<__nv_bfloat16, 4>(a, status, st);
-      default: return launch_group_tc_t<__nv_bfloat16, 8>(a, status, st);
+      case 1: return launch_group_g<__nv_bfloat16, 1, 3>(a, status, st);
+      case 2: return launch_group_g<__nv_bfloat16, 2, 3>(a, status, st);
+      case 4: return launch_group_g<__nv_bfloat16, 4, 2>(a, status, st);
+      default: return launch_group_g<__nv_bfloat16, 8, 2>(a, status, st);
     }
   }
   switch (G) {
-    case 1: return launch_group_tc_t<__half, 1, 3>(a, status, st);
-    case 2: return launch_group_tc_t<__half, 2, 3>(a, status, st);
-    case 4: return launch_group_tc_t<__half, 4>(a, status, st);
-    default: return launch_group_tc_t<__half, 8>(a, status, st);
+    case 1: return launch_group_g<__half, 1, 3>(a, status, st);
+    case 2: return launch_group_g<__half, 2, 3>(a, status, st);
+    case 4: return launch_group_g<__half, 4, 2>(a, status, st);
+    default: return launch_group_g<__half, 8, 2>(a, status, st);
   }
 }
 

@@ -210,6 +210,9 @@ GROUPED = [
               samples=20),
     GroupCase("g_ps_g2_p256", "parallel_sampling", "bf16", 2, 16, 256, Hkv=2),
     GroupCase("g_ps_g8_p128", "parallel_sampling", "bf16", 8, 16, 128, Hkv=2),
+    # families of at most 8 / G members: span CTAs with 8 of the 16 columns in use
+    GroupCase("g_ps_g2_4samples", "parallel_sampling", "f16", 2, 16, 256, Hkv=2, samples=4),
+    GroupCase("g_lp_g4_2requests", "shared_prefix", "bf16", 4, 16, 512, requests=2),
     # requests forked from one prefix (the long_prefix shape, scaled down): G = 4, 8
     GroupCase("g_lp_g4_p512", "shared_prefix", "bf16", 4, 16, 512),
     GroupCase("g_lp_g4_p128", "shared_prefix", "bf16", 4, 16, 128),

@@ -776,22 +776,35 @@ bool decode_group_tc8_supported(const DecodeArgs& a) {
          tmap_available();
 }
 
+namespace {
+// 8 / G members per span CTA when every family fits (half the softmax's
+// per-column work; as in decode_tc.cu), else 16 / G
+template <typename T, int G>
+int launch_group8_g(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
+  if constexpr (G <= 4) {
+    if (static_cast<int64_t>(a.max_group_size) * G <= 8)
+      return launch_tc8_t<T, G, 8 / G>(a, status, stream);
+  }
+  return launch_tc8_t<T, G, 16 / G>(a, status, stream);
+}
+}  // namespace
+
 int launch_decode_group_tc8(const DecodeArgs& a, unsigned int* status, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int G = a.Hq / a.Hkv;
   if (a.dtype == PA_BF16) {
     switch (G) {
-      case 1: return launch_tc8_t<__nv_bfloat16, 1, 16>(a, status, st);
-      case 2: return launch_tc8_t<__nv_bfloat16, 2, 8>(a, status, st);
-      case 4: return launch_tc8_t<__nv_bfloat16, 4, 4>(a, status, st);
-      default: return launch_tc8_t<__nv_bfloat16, 8, 2>(a, status, st);
+      case 1: return launch_group8_g<__nv_bfloat16, 1>(a, status, st);
+      case 2: return launch_group8_g<__nv_bfloat16, 2>(a, status, st);
+      case 4: return launch_group8_g<__nv_bfloat16, 4>(a, status, st);
+      default: return launch_group8_g<__nv_bfloat16, 8>(a, status, st);
     }
   }
   switch (G) {
-    case 1: return launch_tc8_t<__half, 1, 16>(a, status, st);
-    case 2: return launch_tc8_t<__half, 2, 8>(a, status, st);
-    case 4: return launch_tc8_t<__half, 4, 4>(a, status, st);
-    default: return launch_tc8_t<__half, 8, 2>(a, status, st);
+    case 1: return launch_group8_g<__half, 1>(a, status, st);
+    case 2: return launch_group8_g<__half, 2>(a, status, st);
+    case 4: return launch_group8_g<__half, 4>(a, status, st);
+    default: return launch_group8_g<__half, 8>(a, status, st);
   }
 }
 

@@ -232,6 +232,9 @@ GROUPED = [
     GroupCase("g_e4m3_ps_g1_20samples", "parallel_sampling", "f16", 1, 16, 512, Hkv=2,
               prompts=2, samples=20, fp8=True),
     GroupCase("g_e4m3_lp_g4_p512", "shared_prefix", "bf16", 4, 16, 512, fp8=True),
+    GroupCase("g_e4m3_ps_g2_4samples", "parallel_sampling", "bf16", 2, 16, 128, Hkv=2, samples=4,
+              fp8=True),
+    GroupCase("g_e4m3_lp_g4_2requests", "shared_prefix", "f16", 4, 16, 256, requests=2, fp8=True),
     GroupCase("g_e4m3_lp_g4_bs32_p128", "shared_prefix", "f16", 4, 32, 128, fp8=True),
     GroupCase("g_e4m3_lp_g8_bs8_p256", "shared_prefix", "bf16", 8, 8, 256, fp8=True),
     GroupCase("g_e4m3_lp_g4_stream", "shared_prefix", "bf16", 4, 16, 128, Hkv=4, requests=300,

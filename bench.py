@@ -708,7 +708,7 @@ def run_ours(args):
         # reduce included), against the same algorithmic bytes
         span_kernel = "decode_partition_tc8_kernel" if spec.fp8 else "decode_partition_tc_kernel"
         kname = ("decode_grouped: " + span_kernel + " (the families' shared spans, "
-                 "16/G members per CTA) next to " + partition_kernel(spec, P) +
+                 "16/G or 8/G members per CTA) next to " + partition_kernel(spec, P) +
                  " (the rest of every sequence), then decode_reduce_kernel")
         traffic, traffic_note = profiled_traffic(
             args.workload, "decode_grouped_fp8" if spec.fp8 else "decode_grouped", P)

@@ -271,7 +271,8 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache, const
  * physical blocks).  The result is that of pa_decode on the same arguments;
  * what changes is the work: the shared span of a group is read once for all
  * its members, whose queries form the columns of one tensor-core tile (each
- * column a (member, query head) pair, 16 / G members per CTA), instead of once
+ * column a (member, query head) pair: 16 / G members per CTA, or 8 / G when
+ * every group has at most that many), instead of once
  * per member.  Each member's remaining tokens are decoded as in pa_decode, and
  * a reduce merges both parts with one softmax over all of the sequence's
  * tokens ([P1] "PagedAttention의 설계").

@@ -58,6 +58,17 @@ constexpr int GROUP_BYTES = 2048;            // 8 token rows, both 64-column hal
 constexpr int HALF_OFF = 1024;               // second 64-column half of a group
 constexpr int THREADS = 192;
 constexpr float RESCALE_THRESHOLD = 8.0f;    // log2 units: raise the max past 2^8 growth
+// The running max before any score: finite, so that 2^(s - m) needs no mask
+// test (a masked score is -inf and gives exactly 0) and the first raise gives
+// 2^(M_NONE - max) = 0; a partial that saw no score is written with max -inf.
+constexpr float M_NONE = -1.0e30f;
+
+// 2^x by the hardware's approximate base-2 exponential (flushes subnormals).
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 // P^T is stored MN-major without swizzle: a 16-byte row holds 8 columns
 // (heads) of one token, 128 tokens make a 2 KB chunk of 8 columns, and the
 // chunks of columns 8-15 (and 16-31) follow at P_CHUNK strides.
@@ -475,7 +486,7 @@ __global__ void __launch_bounds__(THREADS, CTAS)
     float m_run[NC], l_part[NC];
 #pragma unroll
     for (int h = 0; h < NC; ++h) {
-      m_run[h] = -INFINITY;
+      m_run[h] = M_NONE;
       l_part[h] = 0.f;
     }
     // A failed (timed-out) wait makes `ok` false for the whole warp; later waits
@@ -522,7 +533,7 @@ __global__ void __launch_bounds__(THREADS, CTAS)
             const int64_t slot = hq * p.num_partitions + slot0 + part;
             p.ws_o[slot * DH + r] = o[h];
             if (r == 0) {
-              p.ws_m[slot] = m_run[h];
+              p.ws_m[slot] = Ls > 0.f ? m_run[h] : -INFINITY;
               p.ws_l[slot] = Ls;
             }
             for (int e = 1; e < n_slots; ++e) {
@@ -576,7 +587,7 @@ __global__ void __launch_bounds__(THREADS, CTAS)
           const float tmax =
               fmaxf(fmaxf(red[h], red[NPAD + h]), fmaxf(red[2 * NPAD + h], red[3 * NPAD + h]));
           const float mnew = fmaxf(m_run[h], tmax);
-          alpha[h] = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - mnew);
+          alpha[h] = ex2_fast(m_run[h] - mnew);   // 0 after M_NONE
           m_run[h] = mnew;
           l_part[h] *= alpha[h];
         }
@@ -595,8 +606,7 @@ __global__ void __launch_bounds__(THREADS, CTAS)
       float pr[NC];
 #pragma unroll
       for (int h = 0; h < NC; ++h) {
-        const bool counted = NQ > 1 ? s[h] != -INFINITY : valid;
-        pr[h] = counted ? exp2f(s[h] - m_run[h]) : 0.f;
+        pr[h] = ex2_fast(s[h] - m_run[h]);        // masked: 2^-inf = 0
         l_part[h] += pr[h];
       }
       if (i >= PBUF) wait(&p_free[i % PBUF], ((i / PBUF) - 1) & 1);   // P buffer read

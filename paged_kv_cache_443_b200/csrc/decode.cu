@@ -61,6 +61,13 @@ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 constexpr float RESCALE_LOG2 = 8.0f;   // raise the running max past 2^8 growth
 
+// 2^x by the hardware's approximate base-2 exponential (flushes subnormals).
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <typename T, int D, int G, int NCW, int BUDGET = 65536>
 struct Cfg {
   static constexpr int ES = sizeof(T);
@@ -456,7 +463,7 @@ __global__ void __launch_bounds__(Cfg<TK, D, G, NCW, BUDGET>::THREADS)
       const float tmax = __shfl_sync(FULL_MASK, seg[(h * C::TPW) / 32], (h * C::TPW) % 32);
       const bool up = tmax > m[h] + RESCALE_LOG2;
       mnew[h] = up ? tmax : m[h];
-      alpha[h] = !up ? 1.f : (m[h] == -INFINITY) ? 0.f : exp2f(m[h] - tmax);
+      alpha[h] = !up ? 1.f : (m[h] == -INFINITY) ? 0.f : ex2_fast(m[h] - tmax);
       raise |= up;
     }
 #pragma unroll
@@ -466,7 +473,7 @@ __global__ void __launch_bounds__(Cfg<TK, D, G, NCW, BUDGET>::THREADS)
       float mh = -INFINITY;
 #pragma unroll
       for (int h = 0; h < G; ++h) mh = (h == hh) ? mnew[h] : mh;
-      const float pr = (sv[ps] == -INFINITY) ? 0.f : exp2f(sv[ps] - mh);
+      const float pr = (sv[ps] == -INFINITY) ? 0.f : ex2_fast(sv[ps] - mh);
       if (idx < C::NSM) sc[idx] = pr;
       float x = pr;
 #pragma unroll

@@ -72,6 +72,13 @@ constexpr float RESCALE_THRESHOLD = 2.0f;   // P <= 2^2
 constexpr float P_UP = 64.0f;               // P * 2^6 <= 256 < 448
 constexpr float P_DOWN = 1.0f / 64.0f;
 
+// 2^x by the hardware's approximate base-2 exponential (flushes subnormals).
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Shared-memory layout for NTERM query terms, SLOTS tiles per ring (one ring
 // for K codes, one for V codes) and PBUF P buffers.  Two layouts are built:
 //   3 terms, 3 + 3 slots, 2 P buffers (~113 KB): two CTAs per SM, for f16
@@ -589,7 +596,7 @@ __global__ void __launch_bounds__(THREADS, Y::CTAS_PER_SM)
           const float tmax =
               fmaxf(fmaxf(red[h], red[NPAD + h]), fmaxf(red[2 * NPAD + h], red[3 * NPAD + h]));
           const float mnew = fmaxf(m_run[h], tmax);
-          alpha[h] = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - mnew);
+          alpha[h] = (m_run[h] == -INFINITY) ? 0.f : ex2_fast(m_run[h] - mnew);
           m_run[h] = mnew;
           l_part[h] *= alpha[h];
         }
@@ -606,7 +613,7 @@ __global__ void __launch_bounds__(THREADS, Y::CTAS_PER_SM)
       float pr[NC];
 #pragma unroll
       for (int h = 0; h < NC; ++h) {
-        pr[h] = s[h] != -INFINITY ? exp2f(s[h] - m_run[h]) : 0.f;
+        pr[h] = s[h] != -INFINITY ? ex2_fast(s[h] - m_run[h]) : 0.f;
         l_part[h] += pr[h];
       }
       if (i >= PBUF) wait(&p_free[i % PBUF], ((i / PBUF) - 1) & 1);

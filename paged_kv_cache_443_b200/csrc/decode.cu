@@ -17,11 +17,12 @@
 //   * warp 0 is the producer: it reads the block table (32 entries per
 //     coalesced load) and moves each physical (block, kv head) K and V tile --
 //     a contiguous bs*D run -- into shared memory with 1-D bulk copies on the
-//     TMA engine, into a ring of S stages of 32 tokens (32 KB in flight per CTA
-//     for 16-bit caches, six CTAs per SM; 64 KB of E4M3 codes) tracked by
-//     mbarriers with transaction counts;
-//   * NCW consumer warps each own 8 tokens of a stage: q (pre-scaled by
-//     scale*log2 e) sits in registers, a lane owns one 16-byte chunk of a K/V row,
+//     TMA engine, into a ring of S stages (32 KB in flight per CTA for 16-bit
+//     caches, six CTAs per SM; 64 KB of E4M3 codes) tracked by mbarriers with
+//     transaction counts;
+//   * NCW consumer warps each own 8 tokens of a stage (16 for E4M3 codes at
+//     G <= 2): q (pre-scaled by scale*log2 e, or raw f16 pairs over E4M3)
+//     sits in registers, a lane owns one 16-byte chunk of a K/V row,
 //     dot products are finished with a butterfly reduce-scatter across the lanes
 //     of a row, softmax runs in base 2 on the warp's scores in shared memory,
 //     and P.V accumulates in fp32 registers;
@@ -68,7 +69,7 @@ __device__ __forceinline__ float ex2_fast(float x) {
   return y;
 }
 
-template <typename T, int D, int G, int NCW, int BUDGET = 65536>
+template <typename T, int D, int G, int NCW, int BUDGET = 65536, int TPW_ = 8>
 struct Cfg {
   static constexpr int ES = sizeof(T);
   // elements a lane loads at once: one 16-byte chunk (8 codes at G > 2, where
@@ -76,7 +77,7 @@ struct Cfg {
   static constexpr int EPL = ES == 1 ? (G <= 2 ? 16 : 8) : Elem<T>::EPL;
   static constexpr int LPR = D / EPL;          // lanes per K/V row
   static constexpr int RPW = 32 / LPR;         // rows a warp covers per iteration
-  static constexpr int TOK = NCW * 8;          // tokens per stage (8 per consumer warp)
+  static constexpr int TOK = NCW * TPW_;       // tokens per stage (TPW_ per consumer warp)
   static constexpr int TPW = TOK / NCW;        // tokens per consumer warp per stage
   static constexpr int ITERS = TPW / RPW;
   static constexpr int ROW_BYTES = D * ES;
@@ -219,10 +220,10 @@ struct PartitionParams {
   int slot_base;
 };
 
-template <typename TQ, typename TK, int D, int G, int NCW, int BUDGET>
-__global__ void __launch_bounds__(Cfg<TK, D, G, NCW, BUDGET>::THREADS)
+template <typename TQ, typename TK, int D, int G, int NCW, int BUDGET, int TPW_>
+__global__ void __launch_bounds__(Cfg<TK, D, G, NCW, BUDGET, TPW_>::THREADS)
     decode_partition_kernel(const PartitionParams p) {
-  using C = Cfg<TK, D, G, NCW, BUDGET>;
+  using C = Cfg<TK, D, G, NCW, BUDGET, TPW_>;
   using E = Elem<TK>;
   using EQ = Elem<TQ>;
   constexpr bool kCoded = sizeof(TK) == 1;  // E4M3 codes
@@ -698,11 +699,21 @@ constexpr int stage_budget() {
   return sizeof(TK) == 1 ? 65536 : 32768;
 }
 
-template <typename TQ, typename TK, int D, int G, int BUDGET = stage_budget<TK>()>
+// Tokens per consumer warp per stage: 16 for E4M3 codes at G <= 2 (128-token
+// stages of 32 KB, two in flight: each warp's fixed per-stage work -- the
+// barrier waits, the scores' round trip through shared memory, the softmax
+// shuffles -- is spread over twice the bytes; opt13b_fp8 0.765 -> 0.800), 8
+// otherwise (16-bit caches keep two 16 KB stages and six CTAs per SM).
+template <typename TK, int G>
+constexpr int warp_tokens() {
+  return (sizeof(TK) == 1 && G <= 2) ? 16 : 8;
+}
+
+template <typename TQ, typename TK, int D, int G, int BUDGET = stage_budget<TK>(), int TPW_ = 8>
 cudaError_t launch_partition_t(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
   constexpr int NCW = consumer_warps<TK, G>();
-  using C = Cfg<TK, D, G, NCW, BUDGET>;
-  auto kern = decode_partition_kernel<TQ, TK, D, G, NCW, BUDGET>;
+  using C = Cfg<TK, D, G, NCW, BUDGET, TPW_>;
+  auto kern = decode_partition_kernel<TQ, TK, D, G, NCW, BUDGET, TPW_>;
   // opt in to > 48 KB of dynamic shared memory (idempotent, cheap)
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
@@ -736,8 +747,8 @@ cudaError_t launch_partition_t(const DecodeArgs& a, unsigned int* status, cudaSt
 template <typename TQ, typename TK, int D>
 cudaError_t launch_partition_g(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
   switch (a.Hq / a.Hkv) {
-    case 1: return launch_partition_t<TQ, TK, D, 1>(a, status, stream);
-    case 2: return launch_partition_t<TQ, TK, D, 2>(a, status, stream);
+    case 1: return launch_partition_t<TQ, TK, D, 1, stage_budget<TK>(), warp_tokens<TK, 1>()>(a, status, stream);
+    case 2: return launch_partition_t<TQ, TK, D, 2, stage_budget<TK>(), warp_tokens<TK, 2>()>(a, status, stream);
     case 4: return launch_partition_t<TQ, TK, D, 4>(a, status, stream);
     case 8: return launch_partition_t<TQ, TK, D, 8>(a, status, stream);
     default: return cudaErrorInvalidValue;

@@ -779,3 +779,30 @@ def test_repeated_decode_launches_are_identical(dtype, fp8):
     rows = sampled_rows(o, spec, n=96, seed=5)
     want = oracle_attention(o, spec, rows=rows)
     assert np.abs(got[rows[:, 0], rows[:, 1]] - want).max() <= TOL[spec.dtype]
+
+
+@pytest.mark.parametrize("dtype,G,samples", [("bf16", 1, 6), ("f16", 2, 4), ("bf16", 1, 20)])
+def test_repeated_grouped_launches_are_identical(dtype, G, samples):
+    """The grouped decode's span kernel at G = 1, 2 (rings of two tiles, three
+    CTAs per SM; 8 / G or 16 / G members per CTA) and the rest kernel, with
+    spans whose last tile is partial: every run finite and byte-identical."""
+    spec = W.Spec(f"rep_grp_{G}_{samples}", dtype, 4 * G, 4, 128, 16, "parallel_sampling",
+                  4 * samples, seed=1400 + G + samples, num_prompts=4,
+                  samples_per_prompt=samples, prompt_lo=300, prompt_hi=900, div_lo=1,
+                  div_hi=200, partition_size=0)
+    p, o = build(W.scenario(spec))
+    run_step(p, spec)
+    torch.cuda.synchronize()
+    groups = p.cache.groups(p.tables, p.lens)
+    assert groups.max_shared_len > 0 and groups.max_group_size == samples
+    ws = p.cache.grouped_workspace(p.q.shape[0], p.q.shape[1], p.max_ctx, groups, 0)
+    out = torch.empty_like(p.q)
+
+    def launch():
+        ws.fill_(float("nan"))
+        return p.cache.decode(p.q, p.tables, p.lens, p.max_ctx, spec.softmax_scale, out=out,
+                              workspace=ws, groups=groups)
+
+    got = as_f64(_repeat_identical(launch), spec)
+    want = oracle_attention(o, spec)
+    assert np.abs(got - want).max() <= TOL[spec.dtype]

@@ -1,6 +1,8 @@
 // decode_tc.cu -- paged decode attention on the 5th-generation tensor cores
 // (tcgen05 + TMEM) for grouped-query heads (G = Hq/Hkv in {4, 8}), fp16/bf16,
-// head size 128.
+// head size 128; the same kernel with (member, head) columns serves the shared
+// spans of sequence families at G = 1, 2, 4, 8, and with (query token, head)
+// columns a few query tokens per sequence.
 //
 // Same contract and split-K partials as decode.cu ("자기회귀 생성과 KV 캐시" and
 // "PagedAttention의 설계", supersilo.blog vLLM summary: scores q.k/sqrt(d_k),
@@ -14,8 +16,8 @@
 //
 // Roles in a CTA of 6 warps, one CTA per (sequence, kv head, run of partitions):
 //   warp 0   producer: block-table lookups, one TMA load per physical block of
-//            its K (or V) rows into a ring of three 32 KB slots holding K_0, V_0,
-//            K_1, V_1, ...  The cache is viewed as a 4-D tensor (64 columns, 8
+//            its K (or V) rows into a ring of 32 KB slots (three; two in the
+//            three-CTA layout) holding K_0, V_0, K_1, V_1, ...  The cache is viewed as a 4-D tensor (64 columns, 8
 //            rows, 2 column halves, 8-row groups), so a block lands as
 //            [8-row group][half][8 rows x 128 B] with the 128-byte swizzle: the
 //            canonical K-major layout of K and MN-major layout of V^T, with
@@ -30,7 +32,8 @@
 //            at the end reads its row of O from TMEM and writes the output or the
 //            split-K partial.
 // About 109 KB of shared memory (113 KB with 32 columns), so two CTAs share an
-// SM and hide each other's pipeline fill.  Every mbarrier wait is bounded;
+// SM and hide each other's pipeline fill; the group spans of families at
+// G = 1, 2 use a 72 KB layout with three CTAs per SM.  Every mbarrier wait is bounded;
 // block ids outside the pool are skipped and flagged.
 #include <cuda.h>
 #include <cuda_runtime.h>

@@ -279,10 +279,17 @@ def partition_kernel(spec, P):
 
 
 def source_digest(files=KERNEL_SOURCES["decode_partition_kernel"]):
+    """Digest of the kernels' code: the sources with comments and blank lines
+    dropped, so that editing a comment does not retire a capture."""
+    import re
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "paged_kv_cache_443_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "paged_kv_cache_443_b200", "csrc", f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"(?m)^\s*//.*$|\s+//[^\"\n]*$", "", text)
+        code = "\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip())
+        h.update(code.encode("utf-8"))
     return h.hexdigest()[:16]
 
 

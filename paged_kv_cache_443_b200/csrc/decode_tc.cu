@@ -59,7 +59,12 @@ constexpr int DH = 128;                      // head size
 constexpr int SLOT_BYTES = TOK * 256;        // one tile of K (or V): 32 KB
 constexpr int GROUP_BYTES = 2048;            // 8 token rows, both 64-column halves
 constexpr int HALF_OFF = 1024;               // second 64-column half of a group
-constexpr int THREADS = 192;
+// Threads of a CTA: producer, MMA issuer and 4 softmax warps; at N = 32
+// columns 8 softmax warps, two threads per token row with 16 columns each.
+template <int NP>
+__host__ __device__ constexpr int tc_threads() {
+  return NP == 32 ? 64 + 256 : 64 + 128;
+}
 constexpr float RESCALE_THRESHOLD = 8.0f;    // log2 units: raise the max past 2^8 growth
 // The running max before any score: finite, so that 2^(s - m) needs no mask
 // test (a masked score is -inf and gives exactly 0) and the first raise gives
@@ -201,7 +206,7 @@ struct TcParams {
 // context tokens) with head c % G, and a key counts for it only up to that
 // token's own position.  NQ = 1 is the decode step and compiles as before.
 template <typename T, int G, int NQ = 1, int NP = 16, int CTAS = 2>
-__global__ void __launch_bounds__(THREADS, CTAS)
+__global__ void __launch_bounds__(tc_threads<NP>(), CTAS)
     decode_partition_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmap_k,
                                const __grid_constant__ CUtensorMap tmap_v) {
   using Y = Lay<NP, CTAS>;
@@ -239,6 +244,13 @@ __global__ void __launch_bounds__(THREADS, CTAS)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int NC = G * NQ;                // S / O columns in use
   static_assert(NC <= NPAD, "query tokens x heads must fit the MMA's N");
+  constexpr int NSPL = NP == 32 ? 2 : 1;    // softmax threads per token row
+  constexpr int NSW = 4 * NSPL;             // softmax warps
+  constexpr int NCH = NC / NSPL;            // S / O columns per softmax thread in use
+  constexpr int NLD = NPAD / NSPL;          // ... and loaded (whole 16-column TMEM loads)
+  static_assert(NLD % 16 == 0 && NCH <= NLD, "16-column TMEM loads per softmax thread");
+  static_assert(NC % (8 * NSPL) == 0 || NSPL == 1, "whole P chunks per softmax thread");
+  constexpr int KTHREADS = tc_threads<NP>();
 
   grid_dependency_wait();   // the appended tokens of the previous kernel are in the cache
   allow_dependents();       // the reduce kernel may start launching
@@ -317,7 +329,7 @@ __global__ void __launch_bounds__(THREADS, CTAS)
   if (L == 0) {
     if (!grouped && !multi && part == 0 && shift == 0) {
       T* o = static_cast<T*>(p.out) + (static_cast<int64_t>(b) * p.Hq + g * G) * DH;
-      for (int i = threadIdx.x; i < G * DH; i += THREADS) o[i] = Elem<T>::from_float(0.f);
+      for (int i = threadIdx.x; i < G * DH; i += KTHREADS) o[i] = Elem<T>::from_float(0.f);
     }
     return;
   }
@@ -346,13 +358,13 @@ __global__ void __launch_bounds__(THREADS, CTAS)
       }
       for (int j = 0; j < 2; ++j) {
         mbar_init(&s_full[j], 1);
-        mbar_init(&s_free[j], 4);
+        mbar_init(&s_free[j], NSW);
       }
       for (int j = 0; j < PBUF; ++j) {
-        mbar_init(&p_full[j], 4);
+        mbar_init(&p_full[j], NSW);
         mbar_init(&p_free[j], 1);
       }
-      mbar_init(q_ready, 4);
+      mbar_init(q_ready, NSW);
       fence_mbar_init();
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
@@ -373,7 +385,7 @@ __global__ void __launch_bounds__(THREADS, CTAS)
     // Q^T operand (16 rows = heads, 128 columns = dims, two swizzled 64-column
     // blocks), rows >= G zero; both P buffers zeroed (their rows >= G stay 0).
     const int t = threadIdx.x - 64;
-    for (int i = t; i < NPAD * (DH / 8); i += 128) {   // one 16-byte chunk each
+    for (int i = t; i < NPAD * (DH / 8); i += 32 * NSW) {   // one 16-byte chunk each
       const int h = i / (DH / 8);                      // column: query token h / G, head h % G
       const int c = i % (DH / 8);                      // chunk of 8 dims
       uint4 v = make_uint4(0, 0, 0, 0);
@@ -385,7 +397,7 @@ __global__ void __launch_bounds__(THREADS, CTAS)
       const uint32_t off = (c / 8) * (NPAD * 128) + sw128(h, (c % 8) * 8);
       *reinterpret_cast<uint4*>(qop + off) = v;
     }
-    for (int i = t; i < PBUF * OPB_BYTES / 16; i += 128)
+    for (int i = t; i < PBUF * OPB_BYTES / 16; i += 32 * NSW)
       reinterpret_cast<uint4*>(pop)[i] = make_uint4(0, 0, 0, 0);
     fence_async_smem();
     __syncwarp();
@@ -483,17 +495,22 @@ __global__ void __launch_bounds__(THREADS, CTAS)
     __syncwarp();
   } else {
     // ================= softmax warps =================
+    // NSPL threads per token row: the warps of half hf (NCH columns from c0)
+    // meet on named barrier 1 + 2 hf.
     const int quad = warp & 3;                 // TMEM lane quadrant of this warp
+    const int hf = NSPL == 1 ? 0 : (warp - 2) >> 2;   // column half (a constant 0 when NSPL = 1)
+    const int c0 = hf * NCH;                   // first S / O column of this thread
+    const int sbar = 1 + 2 * hf;
     const int r = quad * 32 + lane;            // token row of the tile / dim row of O
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    float m_run[NC], l_part[NC];
+    float m_run[NCH], l_part[NCH];
 #pragma unroll
-    for (int h = 0; h < NC; ++h) {
+    for (int h = 0; h < NCH; ++h) {
       m_run[h] = M_NONE;
       l_part[h] = 0.f;
     }
     // A failed (timed-out) wait makes `ok` false for the whole warp; later waits
-    // are then skipped, but every named barrier is still joined so the four
+    // are then skipped, but every named barrier is still joined so the
     // softmax warps never wait on each other forever.
     bool ok = true;
     auto wait = [&](uint64_t* bar, uint32_t parity) {
@@ -501,35 +518,36 @@ __global__ void __launch_bounds__(THREADS, CTAS)
       ok = __all_sync(FULL, ok);
       return ok;
     };
-    // Row r of O^T (dim r, all heads) and the sums of the CTA's span, whose last
-    // tile is i: the output, or the split-K partial of partition part (and
-    // empty partials for the span's other partitions).
+    // Row r of O^T (dim r, this thread's columns) and the sums of the CTA's
+    // span, whose last tile is i: the output, or the split-K partial of
+    // partition part (and empty partials for the span's other partitions).
     auto flush = [&](int i) {
       wait(&p_free[i % PBUF], (i / PBUF) & 1);
       tc_fence_after();
-      float o[NPAD];
-      tmem_ld_cols<NPAD>(tmem + lane_base + 2 * NPAD, o);
+      float o[NLD];
+      tmem_ld_cols<NLD>(tmem + lane_base + 2 * NPAD + c0, o);
       tc_fence_before();
       __syncwarp();
 #pragma unroll
-      for (int h = 0; h < NC; ++h) {
+      for (int h = 0; h < NCH; ++h) {
         float x = l_part[h];
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(FULL, x, off);
         l_part[h] = x;
       }
-      named_sync(1, 128);
+      named_sync(sbar, 128);
       if (lane == 0) {
 #pragma unroll
-        for (int h = 0; h < NC; ++h) red[quad * NPAD + h] = l_part[h];
+        for (int h = 0; h < NCH; ++h) red[quad * NPAD + c0 + h] = l_part[h];
       }
-      named_sync(1, 128);
+      named_sync(sbar, 128);
       if (ok) {
 #pragma unroll
-        for (int h = 0; h < NC; ++h) {
-          const float Ls = red[h] + red[NPAD + h] + red[2 * NPAD + h] + red[3 * NPAD + h];
-          const int64_t hq = (static_cast<int64_t>(q0) + h / G) * p.Hq + g * G + h % G;
-          if (NQ > 1 && h / G >= Qb) continue;
+        for (int h = 0; h < NCH; ++h) {
+          const int hg = c0 + h;                 // column: query row hg / G, head hg % G
+          const float Ls = red[hg] + red[NPAD + hg] + red[2 * NPAD + hg] + red[3 * NPAD + hg];
+          const int64_t hq = (static_cast<int64_t>(q0) + hg / G) * p.Hq + g * G + hg % G;
+          if (NQ > 1 && hg / G >= Qb) continue;
           if (single) {
             static_cast<T*>(p.out)[hq * DH + r] = Elem<T>::from_float(o[h] / Ls);
           } else {
@@ -553,62 +571,65 @@ __global__ void __launch_bounds__(THREADS, CTAS)
     for (int i = 0; i < n_tiles; ++i) {
       const int n_valid = min(TOK, end - (start + i * TOK));
       const bool valid = r < n_valid;
-      float sv[NPAD];
+      float sv[NLD];
       if (wait(&s_full[i & 1], (i >> 1) & 1)) {
         tc_fence_after();
-        tmem_ld_cols<NPAD>(tmem + lane_base + (i & 1) * NPAD, sv);
+        tmem_ld_cols<NLD>(tmem + lane_base + (i & 1) * NPAD + c0, sv);
       } else {
 #pragma unroll
-        for (int h = 0; h < NPAD; ++h) sv[h] = 0.f;
+        for (int h = 0; h < NLD; ++h) sv[h] = 0.f;
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[i & 1]);
-      float s[NC];
+      float s[NCH];
       bool need = false;
 #pragma unroll
-      for (int h = 0; h < NC; ++h) {
+      for (int h = 0; h < NCH; ++h) {
         bool ok_h = valid;
-        if constexpr (NQ > 1)   // causal: up to query token h / G's own position
-          ok_h = ok_h && h / G < Qb && start + i * TOK + r <= L - Qall + qoff + h / G;
+        if constexpr (NQ > 1) {  // causal: up to query token hg / G's own position
+          const int hg = c0 + h;
+          ok_h = ok_h && hg / G < Qb && start + i * TOK + r <= L - Qall + qoff + hg / G;
+        }
         s[h] = ok_h ? sv[h] * p.scale_log2 : -INFINITY;
         need |= s[h] > m_run[h] + RESCALE_THRESHOLD;
       }
-      if (bar_or(1, 128, need)) {
-        // raise the running max to this tile's max (all 128 threads agree)
+      if (bar_or(sbar, 128, need)) {
+        // raise the running max to this tile's max (the half's 128 threads agree)
 #pragma unroll
-        for (int h = 0; h < NC; ++h) {
+        for (int h = 0; h < NCH; ++h) {
           float x = s[h];
 #pragma unroll
           for (int off = 16; off >= 1; off >>= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, off));
-          if (lane == 0) red[quad * NPAD + h] = x;
+          if (lane == 0) red[quad * NPAD + c0 + h] = x;
         }
-        named_sync(1, 128);
-        float alpha[NC];
+        named_sync(sbar, 128);
+        float alpha[NCH];
 #pragma unroll
-        for (int h = 0; h < NC; ++h) {
+        for (int h = 0; h < NCH; ++h) {
+          const int hg = c0 + h;
           const float tmax =
-              fmaxf(fmaxf(red[h], red[NPAD + h]), fmaxf(red[2 * NPAD + h], red[3 * NPAD + h]));
+              fmaxf(fmaxf(red[hg], red[NPAD + hg]), fmaxf(red[2 * NPAD + hg], red[3 * NPAD + hg]));
           const float mnew = fmaxf(m_run[h], tmax);
           alpha[h] = ex2_fast(m_run[h] - mnew);   // 0 after M_NONE
           m_run[h] = mnew;
           l_part[h] *= alpha[h];
         }
-        named_sync(1, 128);
+        named_sync(sbar, 128);
         // O must hold every earlier tile before it is rescaled (at the first
         // tile O starts from zero instead)
         if (i > 0 && wait(&p_free[(i - 1) % PBUF], ((i - 1) / PBUF) & 1)) {
           tc_fence_after();
-          float o[NPAD];
-          tmem_ld_cols<NPAD>(tmem + lane_base + 2 * NPAD, o);
+          float o[NLD];
+          tmem_ld_cols<NLD>(tmem + lane_base + 2 * NPAD + c0, o);
 #pragma unroll
-          for (int h = 0; h < NC; ++h) o[h] *= alpha[h];
-          tmem_st_cols<NPAD>(tmem + lane_base + 2 * NPAD, o);
+          for (int h = 0; h < NCH; ++h) o[h] *= alpha[h];
+          tmem_st_cols<NLD>(tmem + lane_base + 2 * NPAD + c0, o);
         }
       }
-      float pr[NC];
+      float pr[NCH];
 #pragma unroll
-      for (int h = 0; h < NC; ++h) {
+      for (int h = 0; h < NCH; ++h) {
         pr[h] = ex2_fast(s[h] - m_run[h]);        // masked: 2^-inf = 0
         l_part[h] += pr[h];
       }
@@ -617,18 +638,20 @@ __global__ void __launch_bounds__(THREADS, CTAS)
       // 8c .. 8c + 7 at chunk c (columns >= NC stay 0)
       uint8_t* pb = pop + (i % PBUF) * OPB_BYTES + r * 16;
 #pragma unroll
-      for (int c = 0; c < (NC + 7) / 8; ++c) {
+      for (int c = 0; c < (NCH + 7) / 8; ++c) {
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int h = 8 * c + 2 * e;
-          w[e] = pack2<T>(h < NC ? pr[h < NC ? h : 0] : 0.f, h + 1 < NC ? pr[h + 1 < NC ? h + 1 : 0] : 0.f);
+          w[e] = pack2<T>(h < NCH ? pr[h < NCH ? h : 0] : 0.f,
+                          h + 1 < NCH ? pr[h + 1 < NCH ? h + 1 : 0] : 0.f);
         }
-        *reinterpret_cast<uint4*>(pb + c * P_CHUNK) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(pb + (c0 / 8 + c) * P_CHUNK) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      if (n_valid < TOK) {
+      if (n_valid < TOK && hf == 0) {
         // the last tile: zero the V rows of tokens past the end, so that
-        // whatever they hold (unused slots, stale data) adds 0 * 0 to O
+        // whatever they hold (unused slots, stale data) adds 0 * 0 to O (one
+        // half's warps do it; the MMA waits for every softmax warp)
         const int u = 2 * i + 1, s_ = u % SLOTS;
         // The parity wait below is only sound once the slot's previous load
         // has landed.  With three slots that is K of tile i - 1, which S of
@@ -654,9 +677,9 @@ __global__ void __launch_bounds__(THREADS, CTAS)
     flush(n_tiles - 1);
   }
 
-  // ---- teardown: warps 1-5 meet, warp 1 frees TMEM ----
+  // ---- teardown: warps 1 .. (all but the producer) meet, warp 1 frees TMEM ----
   tc_fence_before();
-  named_sync(2, 160);
+  named_sync(2, KTHREADS - 32);
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
@@ -716,7 +739,7 @@ cudaError_t launch_tc_t(const DecodeArgs& a, unsigned int* status, cudaStream_t 
   p.span_ppc = 1;
   const int np = a.num_partitions - a.slot_base;
   dim3 grid(a.num_seqs, a.Hkv, (np + p.parts_per_cta - 1) / p.parts_per_cta);
-  return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
+  return launch_overlapped(kern, grid, dim3(tc_threads<16>()), SMEM_BYTES, stream, p, mk, mv);
 }
 
 // The groups' shared spans, with NQ = 16 / G: each CTA serves NQ members of a
@@ -775,7 +798,7 @@ cudaError_t launch_group_tc_t(const DecodeArgs& a, unsigned int* status, cudaStr
   p.parts_per_cta = 1;
   p.span_ppc = tc_parts_per_cta(span_rows, a.partition_size, span_parts, rest_rows * rest_parts);
   dim3 grid(p.span_x, a.Hkv, (span_parts + p.span_ppc - 1) / p.span_ppc);
-  return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
+  return launch_overlapped(kern, grid, dim3(tc_threads<16>()), SMEM_BYTES, stream, p, mk, mv);
 }
 
 }  // namespace
@@ -894,7 +917,7 @@ cudaError_t launch_tcq_t(const MqArgs& m, unsigned int* status, cudaStream_t str
   p.span_x = 0;
   p.span_ppc = 1;
   dim3 grid(m.num_seqs * p.q_groups, m.Hkv, (m.num_partitions + ppc - 1) / ppc);
-  return launch_overlapped(kern, grid, dim3(THREADS), SMEM_BYTES, stream, p, mk, mv);
+  return launch_overlapped(kern, grid, dim3(tc_threads<NP>()), SMEM_BYTES, stream, p, mk, mv);
 }
 
 // Query tokens per CTA (tc_query_tokens_per_cta): up to 16 columns on the

@@ -98,11 +98,13 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
 // N consecutive TMEM columns (a multiple of 16) of this thread's lane.
 template <int N>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float* v) {
+  static_assert(N > 0 && N % 16 == 0, "whole 16-column loads");
 #pragma unroll
   for (int j = 0; j < N / 16; ++j) tmem_ld16(taddr + 16 * j, v + 16 * j);
 }
 template <int N>
 __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const float* v) {
+  static_assert(N > 0 && N % 16 == 0, "whole 16-column stores");
 #pragma unroll
   for (int j = 0; j < N / 16; ++j) tmem_st16(taddr + 16 * j, v + 16 * j);
 }
